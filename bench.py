@@ -1,0 +1,440 @@
+"""PACK3D forward throughput on B200.
+
+One step is the whole forward hot path over one batch of synthetic input at
+the 65,536-token shape (volume 32 x 32 x 64, batch 2, 8 heads, head_dim 96,
+window 7^3, blocks 8^3, bf16, random packing): index build from the batch's
+coordinates, block summaries, and the PACK3D forward with LSE.  ``value`` is
+tokens/s (B * N per step) with inputs resident in HBM; ``e2e`` measures the
+same through the C ABI from pinned host buffers, copies included.  The
+window-only mode is timed alongside.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+With N > 1 (one process per GPU under torchrun) every rank runs its own batch
+(weak scaling; the operator has no cross-rank data path) and the time is the
+maximum over ranks.  ``--impl reference`` times the CPU oracle on the host
+cores on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "PACK3D fwd tokens/s at 65k tokens bf16; % of BF16 tensor peak and HBM roofline"
+UNIT = "tokens/s"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "forward_tc_vol_32x32x64.md")
+TC_SOURCE = os.path.join(ROOT, "local_global_attention_b200", "csrc", "attn_tc.cu")
+KERNELS_PER_STEP = 10  # index build 8, block summaries 1, forward 1
+
+
+def peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            return json.load(f), "measured"
+    except (OSError, ValueError):
+        return FALLBACK_PEAKS, "fallback"
+
+
+def workload(name):
+    from local_global_attention_b200 import configs as C
+    return C.BY_NAME[name]
+
+
+def algorithmic_work(wl):
+    """Useful FLOPs of one forward (local and summary terms, 4 d per term) and
+    the minimum HBM bytes (q, k, v read, out written, lse written, plus the
+    summary builder's read of k and v)."""
+    def axis_hist(ext, r):
+        # number of window positions per coordinate along one axis
+        c = np.arange(ext)
+        return np.minimum(c + r, ext - 1) - np.maximum(c - r, 0) + 1
+    rz, ry, rx = ((w - 1) // 2 for w in wl.window)
+    wz, wy, wx = axis_hist(wl.Z, rz), axis_hist(wl.Y, ry), axis_hist(wl.X, rx)
+    local_terms = wz.sum() * wy.sum() * wx.sum()  # sum over queries of |W(i)|
+
+    def blocks_met(ext, r, bsz):
+        c = np.arange(ext)
+        lo = np.maximum(c - r, 0) // bsz
+        hi = np.minimum(c + r, ext - 1) // bsz
+        return hi - lo + 1
+    nb = wl.n_blocks
+    met = (blocks_met(wl.Z, rz, wl.block[0])[:, None, None] *
+           blocks_met(wl.Y, ry, wl.block[1])[None, :, None] *
+           blocks_met(wl.X, rx, wl.block[2])[None, None, :])
+    sum_terms = (nb - met).sum()
+    per_bh_local = 4.0 * wl.d * local_terms
+    per_bh_sum = 4.0 * wl.d * sum_terms
+    BH = wl.B * wl.H
+    esz = 2
+    rows = wl.B * wl.N * wl.H * wl.d
+    hbm = rows * esz * 4 + wl.B * wl.H * wl.N * 4 + rows * esz * 2
+    return {"local_flop": BH * per_bh_local, "summary_flop": BH * per_bh_sum,
+            "flop": BH * (per_bh_local + per_bh_sum), "hbm_bytes": hbm,
+            "fwd_bytes": rows * esz * 4 + wl.B * wl.H * wl.N * 4}
+
+
+def profile_traffic():
+    """DRAM bytes per forward launch from the committed ncu summary, if it was
+    taken on the current kernel source; else None."""
+    try:
+        text = open(PROFILE_SUMMARY).read()
+    except OSError:
+        return None
+    m_sha = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
+    m_tr = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not (m_sha and m_tr):
+        return None
+    sha = hashlib.sha256(open(TC_SOURCE, "rb").read()).hexdigest()
+    return float(m_tr.group(1)) if sha == m_sha.group(1) else None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_ours(args):
+    import torch
+
+    from local_global_attention_b200 import inputs as I
+    from local_global_attention_b200 import pack3d as P
+
+    world, rank, local = dist_setup(args.gpus)
+    wl = workload(args.workload)
+    # weak scaling: each rank its own batch (seed offset by rank)
+    wl_r = wl.replace(seed=wl.seed + 1000 * rank)
+    inp = I.make_inputs(wl_r, args.packing)
+    dev = {k: v.cuda() for k, v in inp.items() if k != "order"}
+    params = P.make_params(wl_r)
+    idx = P.IndexBuffers(params)
+    B, N, H, d = wl.B, wl.N, wl.H, wl.d
+    nb = wl.n_blocks
+    ksum = torch.empty(B, H, nb, d, dtype=torch.float32, device="cuda")
+    vsum = torch.empty_like(ksum)
+    out = torch.empty_like(dev["q"])
+    lse = torch.empty(B, H, N, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    lib = P.load()
+    import ctypes
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    pp, ip = ctypes.byref(params), ctypes.byref(idx.struct)
+    ptr = lambda t: ctypes.c_void_p(t.data_ptr())
+
+    fwd_events = []
+
+    def step(record=False, window=False):
+        rc = lib.pack3d_build_index(pp, ptr(dev["coords"]), ip, sp)
+        if not window:
+            rc |= lib.pack3d_block_summaries(pp, ip, ptr(dev["k"]), ptr(dev["v"]), ptr(ksum),
+                                             ptr(vsum), sp)
+        if record:
+            e0 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+        if window:
+            rc |= lib.pack3d_window_forward(pp, ip, ptr(dev["q"]), ptr(dev["k"]), ptr(dev["v"]),
+                                            ptr(out), ptr(lse), sp)
+        else:
+            rc |= lib.pack3d_forward(pp, ip, ptr(dev["q"]), ptr(dev["k"]), ptr(dev["v"]),
+                                     ptr(ksum), ptr(vsum), ptr(out), ptr(lse), sp)
+        if record:
+            e1 = torch.cuda.Event(enable_timing=True)
+            e1.record(stream)
+            fwd_events.append((e0, e1))
+        if rc:
+            raise RuntimeError(f"pack3d call failed: {rc}")
+
+    def timed(window=False, record=False):
+        for _ in range(args.warmup):
+            step(window=window)
+        torch.cuda.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(args.steps):
+            step(record=record, window=window)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
+        return max_over_ranks(t0.elapsed_time(t1) / args.steps, world)
+
+    with ClockSampler(local) as clk:
+        ms = timed(record=True)
+    st = P.pack3d_index_check(idx)
+    if st != P.OK:
+        raise RuntimeError(f"index status {P.strerror(st)}")
+    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in fwd_events)
+    window_ms = timed(window=True)
+
+    # end to end through the C ABI from pinned host buffers
+    host = {k: inp[k].pin_memory() for k in ("q", "k", "v", "coords")}
+    host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    host_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+
+    def e2e_step():
+        for k_ in ("coords", "q", "k", "v"):
+            dev[k_].copy_(host[k_], non_blocking=True)
+        step()
+        host_out.copy_(out, non_blocking=True)
+        host_lse.copy_(lse, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    h2d = sum(host[k_].numel() * host[k_].element_size() for k_ in host)
+    d2h = host_out.numel() * host_out.element_size() + host_lse.numel() * host_lse.element_size()
+
+    if rank != 0:
+        barrier(world)
+        return
+    pk, pk_src = peaks()
+    work = algorithmic_work(wl)
+    tokens = B * N * world
+    achieved_tflops = work["flop"] / (fwd_ms * 1e-3) / 1e12
+    peak_tf = pk["bf16_tflops_sustained"]
+    traffic = profile_traffic()
+    line = {
+        "metric": METRIC,
+        "value": tokens / (ms * 1e-3),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1)/sqrt(96) q, k, v; random packing)",
+        "config": {
+            "workload": f"{wl.name}: {wl.N} tokens x batch {B}, {H} heads, head_dim {d}, "
+                        f"window {'x'.join(map(str, wl.window))}, blocks "
+                        f"{'x'.join(map(str, wl.block))} ({nb} summaries), {args.packing} packing",
+            "step": "index build + block summaries + forward (out, lse)",
+            "global_batch": B * world,
+            "seq_len": N,
+            "parallelism": f"replicas x{world} (independent batches, no collective)",
+            "l2": "inputs larger than L2: q, k, v = "
+                  f"{3 * B * N * H * d * 2 / 1e6:.0f} MB per step, no flush",
+        },
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "roofline": {
+            "bound": "tensor",
+            "kernel": "k_forward_tc (local window + summaries, tcgen05)",
+            "achieved": achieved_tflops,
+            "peak": peak_tf,
+            "unit": "TFLOP/s",
+            "frac": achieved_tflops / peak_tf,
+            "peak_source": f"{pk_src} bf16_tflops_sustained",
+            "traffic": traffic,
+            "algorithmic_flop_per_launch": work["flop"],
+            "forward_ms": fwd_ms,
+            "forward_hbm_frac": (work["fwd_bytes"] / (fwd_ms * 1e-3) / 1e9) / pk["hbm_gbs"],
+        },
+        "window_only": {"ms_per_step": window_ms, "value": tokens / (window_ms * 1e-3),
+                        "pack3d_over_window": ms / window_ms},
+        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": UNIT, "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "clocks": clk.summary(),
+    }
+    if not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(wl, inp, args.cpu_sample)
+    barrier(world)
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline(wl, inp, n_tokens, seed=0):
+    """The CPU oracle on a bounded sample: n_tokens query positions (all heads
+    of each), timed on the host cores; tokens/s of the same workload."""
+    import oracle
+    oracle.build()
+    rng = np.random.default_rng(seed)
+    N = wl.N
+    bs = rng.integers(0, wl.B, n_tokens)
+    iis = rng.integers(0, N, n_tokens)
+    b = np.repeat(bs, wl.H)
+    i = np.repeat(iis, wl.H)
+    h = np.tile(np.arange(wl.H), n_tokens)
+    sel = oracle.flat_index(wl, b, h, i)
+    t0 = time.perf_counter()
+    ks, vs = oracle.block_summaries(wl, inp["coords"], inp["k"], inp["v"])
+    oracle.forward(wl, inp["coords"], inp["q"], inp["k"], inp["v"], sel=sel, summaries=(ks, vs))
+    dt = time.perf_counter() - t0
+    return {"value": n_tokens / dt, "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": f"{n_tokens} random query tokens x {wl.H} heads of {wl.name} "
+                      f"(block summaries of the whole batch included), {dt:.1f} s"}
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    from local_global_attention_b200 import inputs as I
+    wl = workload(args.workload)
+    inp = I.make_inputs(wl, args.packing)
+    oracle.build()
+    ks, vs = oracle.block_summaries(wl, inp["coords"], inp["k"], inp["v"])
+    rng = np.random.default_rng(1)
+    n = args.cpu_sample // 4 or 1
+
+    def one():
+        b = rng.integers(0, wl.B, n)
+        i = rng.integers(0, wl.N, n)
+        sel = oracle.flat_index(wl, np.repeat(b, wl.H), np.tile(np.arange(wl.H), n),
+                                np.repeat(i, wl.H))
+        t0 = time.perf_counter()
+        oracle.forward(wl, inp["coords"], inp["q"], inp["k"], inp["v"], sel=sel,
+                       summaries=(ks, vs))
+        return time.perf_counter() - t0
+
+    for _ in range(args.warmup):
+        one()
+    times = [one() for _ in range(args.steps)]
+    per_token = sum(times) / (n * args.steps)
+    value = 1.0 / per_token
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(times) / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (same workload and seed as the CUDA arm)",
+        "config": {"workload": f"{wl.name}, {args.packing} packing; each step a sample of "
+                               f"{n} query tokens x {wl.H} heads (summaries precomputed)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.max_threads(),
+                         "kind": "oracle", "sample": f"{n} tokens x {wl.H} heads per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="vol_32x32x64")
+    ap.add_argument("--packing", default="random")
+    ap.add_argument("--cpu-sample", type=int, default=32768,
+                    help="query tokens the CPU oracle computes for the baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1 and args.impl == "ours":
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

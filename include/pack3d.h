@@ -1,0 +1,194 @@
+/*
+ * pack3d.h - C ABI of the PACK3D local-global attention operator on NVIDIA
+ * B200 (sm_100a).
+ *
+ * The operator is the one introduced in "Geometry Matters in Packed 3D
+ * Attention" (abstract): a 3D volume is packed into a token sequence in an
+ * arbitrary memory order; each query attends, in one softmax, exactly to the
+ * tokens of its local 3D neighbourhood and to summaries of the contiguous 3D
+ * blocks that lie outside that neighbourhood; every query-key and
+ * query-summary interaction is indexed by axial RoPE on the tokens' true grid
+ * coordinates, never on their packed position, and keys are rotated before a
+ * block is summarised.  The conventions the abstract leaves open are fixed
+ * here:
+ *
+ *   - head_dim d = 3 * da; channels [0, da) rotate with z, [da, 2da) with y,
+ *     [2da, 3da) with x; inside a segment channel j pairs with j + da/2 and
+ *     turns by the angle c * rope_base^(-2j/da) (c = the token's coordinate
+ *     on that axis); v is not rotated.
+ *   - window (wz, wy, wx), all odd: the box of half-widths (w - 1) / 2
+ *     centred on the query, clipped at the volume edge (never shifted).
+ *   - blocks (bz, by, bx) tile the volume exactly (they must divide Z, Y, X);
+ *     a block's summary is the mean of its tokens' rotated keys and the mean
+ *     of their values; a query sees the summary of every block whose box does
+ *     not intersect its window box, with logit scale * q~ . kbar and no
+ *     count bias.
+ *   - scale defaults to 1 / sqrt(head_dim); lse is the natural log of the
+ *     softmax normaliser, summaries included.
+ *   - coordinates must be a bijection onto the Z x Y x X grid per batch item
+ *     (a dense volume); each batch item may use its own packing.
+ *
+ * Memory: every buffer is allocated and owned by the caller; the library
+ * never allocates or frees device memory and keeps no global state.  All
+ * pointers except the params and index structs are DEVICE pointers.  Layouts:
+ *   q, k, v, out, dout, dq, dk, dv : [B][N][H][head_dim], packed order,
+ *                                    bf16 (dtype PACK3D_BF16) or fp32;
+ *   coords                        : int16 [B][N][3] as (z, y, x);
+ *   ksum, vsum                    : fp32 [B][H][nb][head_dim], blocks in
+ *                                    raster order (nb = Z/bz * Y/by * X/bx);
+ *   lse                           : fp32 [B][H][N].
+ * N = Z * Y * X.  Every call is asynchronous on the given stream (a
+ * cudaStream_t; 0 is the legacy default stream) and returns a status code
+ * (0 on success, a negative PACK3D_ERR_* otherwise); no call synchronises
+ * except pack3d_index_check.  Errors found on the host (bad arguments) are
+ * returned before anything is launched; launch failures return
+ * PACK3D_ERR_CUDA.
+ */
+#ifndef PACK3D_H
+#define PACK3D_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PACK3D_API __attribute__((visibility("default")))
+#else
+#define PACK3D_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* pack3d_stream_t; /* the same type as cudaStream_t */
+
+enum { PACK3D_BF16 = 0, PACK3D_FP32 = 1 };
+
+enum {
+  PACK3D_OK = 0,
+  PACK3D_ERR_ARG = -1,         /* null pointer, inconsistent sizes, even window, ... */
+  PACK3D_ERR_COORDS = -2,      /* coordinates out of range or not a bijection */
+  PACK3D_ERR_CUDA = -3,        /* a CUDA launch or runtime call failed */
+  PACK3D_ERR_TIMEOUT = -4,     /* a bounded device-side wait gave up */
+  PACK3D_ERR_UNSUPPORTED = -5  /* valid operator, shape not built into this library */
+};
+
+/* Operator shape and conventions.  head_dim must be a multiple of 12 and at
+ * most 96 (12, 24, 48, 96 are built), windows odd and positive, blocks must
+ * divide the volume, 1 <= Z, Y, X <= 32767 and B * N * H * head_dim < 2^31. */
+typedef struct {
+  int32_t B, H, head_dim;
+  int32_t Z, Y, X;
+  int32_t wz, wy, wx;
+  int32_t bz, by, bx;
+  float rope_base; /* > 0 */
+  float scale;     /* softmax scale; <= 0 selects 1 / sqrt(head_dim) */
+  int32_t dtype;   /* PACK3D_BF16 or PACK3D_FP32 (inputs, outputs, gradients) */
+} pack3d_params;
+
+/* Geometry index of one packing, built by pack3d_build_index into one
+ * caller-allocated device buffer (see pack3d_index_init).  Query tiles are
+ * tile[0] x tile[1] x tile[2] boxes (z, y, x) in raster order, cut by the
+ * volume edge where the extents do not divide.
+ *   vol      int32 [B][Z*Y*X]   packed index of the token at each voxel
+ *   perm     int32 [B][N]       tile-ordered permutation: tile by tile, raster
+ *                               order inside a tile, the packed index of each
+ *                               token (a counting sort by tile)
+ *   tile_off int32 [B][T+1]     start of tile t in perm
+ *   nbr_off  int32 [T+1]        start of tile t's halo list (same for every
+ *                               batch item)
+ *   nbr      int32 [B][n_halo]  halo lists: for each tile, the packed indices
+ *                               of the tokens in the tile box widened by the
+ *                               window radius and clipped to the volume, in
+ *                               raster order
+ *   rope     float [(Z+Y+X)][head_dim/6][2]  cos and sin of c * theta_j per
+ *                               axis (z rows, then y, then x), computed in fp64
+ *   err      int32 [2]          [0]: 0 or a bit set of 1 = coordinate out of
+ *                               range, 2 = voxel held twice, 4 = a kernel
+ *                               gave up a bounded device-side wait; [1]:
+ *                               smallest offending flat token index b * N + i
+ */
+typedef struct {
+  int32_t* vol;
+  int32_t* perm;
+  int32_t* tile_off;
+  int32_t* nbr_off;
+  int32_t* nbr;
+  float* rope;
+  int32_t* err;
+  int32_t tile[3];
+  int32_t n_tiles;
+  int64_t n_halo;
+} pack3d_index;
+
+/* Bytes of device memory an index needs for these params (0 if the params
+ * are invalid).  Host-only; no CUDA call. */
+PACK3D_API size_t pack3d_index_bytes(const pack3d_params* p);
+
+/* Carve an index out of a caller-allocated device buffer of at least
+ * pack3d_index_bytes(p) bytes, aligned to 256 bytes.  Fills *out; no CUDA
+ * call.  The buffer stays owned by the caller and must outlive every use of
+ * the index. */
+PACK3D_API int pack3d_index_init(const pack3d_params* p, void* buffer, size_t bytes, pack3d_index* out);
+
+/* Build the index of one packing from its coordinates: the coordinate volume,
+ * the tile permutation by counting sort, the halo lists and the rotation
+ * table.  This is what lets attention follow the true grid coordinates instead
+ * of the packed order ("Geometry Matters in Packed 3D Attention", abstract).  Asynchronous: coordinate errors are recorded in idx->err on
+ * the device and make every later kernel using this index return without
+ * writing; call pack3d_index_check to read them. */
+PACK3D_API int pack3d_build_index(const pack3d_params* p, const int16_t* coords, pack3d_index* idx,
+                       pack3d_stream_t stream);
+
+/* Synchronise the stream and report the index's error word: PACK3D_OK,
+ * PACK3D_ERR_COORDS (bits 1 or 2), PACK3D_ERR_TIMEOUT (bit 4: a kernel that
+ * used this index gave up a bounded wait) or PACK3D_ERR_CUDA.  The only
+ * blocking call of the library. */
+PACK3D_API int pack3d_index_check(const pack3d_index* idx, pack3d_stream_t stream);
+
+/* Block summaries ("compresses only distant context into contiguous 3D block
+ * summaries"; "the rotation is applied before a block is summarized",
+ * abstract): ksum[b][h][B] = mean over the tokens of block B of R(c_j) k_j,
+ * vsum[b][h][B] = mean of v_j, accumulated in fp32 in grid order (the result
+ * does not depend on the packing). */
+PACK3D_API int pack3d_block_summaries(const pack3d_params* p, const pack3d_index* idx, const void* k,
+                           const void* v, float* ksum, float* vsum, pack3d_stream_t stream);
+
+/* Full PACK3D forward (abstract: exact local neighbourhood attention plus
+ * the block summaries, axial RoPE on grid coordinates, one softmax): out and
+ * lse for every query, from the local window keys and the summaries (from pack3d_block_summaries; they may
+ * be reused across calls with the same k, v and index). */
+PACK3D_API int pack3d_forward(const pack3d_params* p, const pack3d_index* idx, const void* q, const void* k,
+                   const void* v, const float* ksum, const float* vsum, void* out, float* lse,
+                   pack3d_stream_t stream);
+
+/* Window-only forward: the same operator without summaries (windowed
+ * attention with axial RoPE, the latency comparator the abstract names);
+ * lse covers the local keys only. */
+PACK3D_API int pack3d_window_forward(const pack3d_params* p, const pack3d_index* idx, const void* q,
+                          const void* k, const void* v, void* out, float* lse,
+                          pack3d_stream_t stream);
+
+/* Bytes of device workspace pack3d_backward needs for these params. */
+PACK3D_API size_t pack3d_backward_workspace_bytes(const pack3d_params* p);
+
+/* Backward of the full operator (the abstract calls the operator "trainable
+ * at scale"): gradients of sum(dout * out) with
+ * respect to q, k, v, through the rotation and through the block means, from
+ * the forward's out and lse.  workspace: caller-allocated, at least
+ * pack3d_backward_workspace_bytes(p) bytes, 256-byte aligned; its contents on
+ * entry do not matter.  Reductions run in a fixed order (deterministic, no
+ * floating-point atomics). */
+PACK3D_API int pack3d_backward(const pack3d_params* p, const pack3d_index* idx, const void* q, const void* k,
+                    const void* v, const void* out, const float* lse, const void* dout, void* dq,
+                    void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                    pack3d_stream_t stream);
+
+/* Human-readable text of a status code (static storage). */
+PACK3D_API const char* pack3d_strerror(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PACK3D_H */

@@ -1,0 +1,233 @@
+// C ABI of the PACK3D operator: argument checks, buffer sizing and launches.
+// Every entry point returns a status code and never throws; nothing here
+// allocates or frees device memory.
+#include <math.h>
+#include <string.h>
+
+#include "pack3d_internal.cuh"
+
+namespace p3d {
+
+int64_t halo_axis_total(int extent, int tile, int r) {
+  int64_t s = 0;
+  for (int t0 = 0; t0 < extent; t0 += tile) {
+    int lo = t0 - r < 0 ? 0 : t0 - r;
+    int end = t0 + tile < extent ? t0 + tile : extent;
+    int hi = end + r < extent ? end + r : extent;
+    s += hi - lo;
+  }
+  return s;
+}
+
+int make_geo(const pack3d_params* p, Geo* g) {
+  if (!p || !g) return PACK3D_ERR_ARG;
+  if (p->B < 1 || p->H < 1 || p->head_dim < 6 || p->head_dim % 6) return PACK3D_ERR_ARG;
+  if (p->Z < 1 || p->Y < 1 || p->X < 1 || p->Z > 32767 || p->Y > 32767 || p->X > 32767)
+    return PACK3D_ERR_ARG;
+  if (p->wz < 1 || p->wy < 1 || p->wx < 1 || !(p->wz & 1) || !(p->wy & 1) || !(p->wx & 1))
+    return PACK3D_ERR_ARG;
+  if (p->bz < 1 || p->by < 1 || p->bx < 1 || p->Z % p->bz || p->Y % p->by || p->X % p->bx)
+    return PACK3D_ERR_ARG;
+  if (!(p->rope_base > 0.f) || !isfinite(p->rope_base) || !isfinite(p->scale))
+    return PACK3D_ERR_ARG;
+  if (p->dtype != PACK3D_BF16 && p->dtype != PACK3D_FP32) return PACK3D_ERR_ARG;
+  int64_t N = (int64_t)p->Z * p->Y * p->X;
+  if ((int64_t)p->B * N * p->H * p->head_dim >= (int64_t)1 << 31) return PACK3D_ERR_ARG;
+  if (p->head_dim != 12 && p->head_dim != 24 && p->head_dim != 48 && p->head_dim != 96)
+    return PACK3D_ERR_UNSUPPORTED;
+  g->B = p->B;
+  g->H = p->H;
+  g->d = p->head_dim;
+  g->da = p->head_dim / 3;
+  g->half = g->da / 2;
+  g->Z = p->Z;
+  g->Y = p->Y;
+  g->X = p->X;
+  g->N = (int)N;
+  g->rz = (p->wz - 1) / 2;
+  g->ry = (p->wy - 1) / 2;
+  g->rx = (p->wx - 1) / 2;
+  g->bz = p->bz;
+  g->by = p->by;
+  g->bx = p->bx;
+  g->nbz = p->Z / p->bz;
+  g->nby = p->Y / p->by;
+  g->nbx = p->X / p->bx;
+  g->nb = g->nbz * g->nby * g->nbx;
+  g->nTz = (p->Z + TZ - 1) / TZ;
+  g->nTy = (p->Y + TY - 1) / TY;
+  g->nTx = (p->X + TX - 1) / TX;
+  g->nT = g->nTz * g->nTy * g->nTx;
+  g->n_halo = halo_axis_total(p->Z, TZ, g->rz) * halo_axis_total(p->Y, TY, g->ry) *
+              halo_axis_total(p->X, TX, g->rx);
+  if (g->n_halo * p->B >= (int64_t)1 << 31) return PACK3D_ERR_ARG;
+  g->tau = p->scale > 0.f ? p->scale : 1.0f / sqrtf((float)p->head_dim);
+  g->dtype = p->dtype;
+  return PACK3D_OK;
+}
+
+namespace {
+
+inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct IndexLayout {
+  size_t vol, perm, tile_off, nbr_off, nbr, rope, err, total;
+};
+
+IndexLayout index_layout(const Geo& g) {
+  IndexLayout L;
+  size_t o = 0;
+  L.vol = o;
+  o += align256(sizeof(int32_t) * (size_t)g.B * g.N);
+  L.perm = o;
+  o += align256(sizeof(int32_t) * (size_t)g.B * g.N);
+  L.tile_off = o;
+  o += align256(sizeof(int32_t) * (size_t)g.B * (g.nT + 1));
+  L.nbr_off = o;
+  o += align256(sizeof(int32_t) * (size_t)(g.nT + 1));
+  L.nbr = o;
+  o += align256(sizeof(int32_t) * (size_t)g.B * g.n_halo);
+  L.rope = o;
+  o += align256(sizeof(float) * 2 * (size_t)(g.Z + g.Y + g.X) * g.half);
+  L.err = o;
+  o += 256;
+  L.total = o;
+  return L;
+}
+
+int check_index(const Geo& g, const pack3d_index* ix) {
+  if (!ix || !ix->vol || !ix->perm || !ix->tile_off || !ix->nbr_off || !ix->nbr || !ix->rope ||
+      !ix->err)
+    return PACK3D_ERR_ARG;
+  if (ix->tile[0] != TZ || ix->tile[1] != TY || ix->tile[2] != TX || ix->n_tiles != g.nT ||
+      ix->n_halo != g.n_halo)
+    return PACK3D_ERR_ARG;
+  return PACK3D_OK;
+}
+
+}  // namespace
+}  // namespace p3d
+
+using namespace p3d;
+
+extern "C" {
+
+size_t pack3d_index_bytes(const pack3d_params* p) {
+  Geo g;
+  if (make_geo(p, &g)) return 0;
+  return index_layout(g).total;
+}
+
+int pack3d_index_init(const pack3d_params* p, void* buffer, size_t bytes, pack3d_index* out) {
+  Geo g;
+  int rc = make_geo(p, &g);
+  if (rc) return rc;
+  if (!buffer || !out || ((uintptr_t)buffer & 255)) return PACK3D_ERR_ARG;
+  IndexLayout L = index_layout(g);
+  if (bytes < L.total) return PACK3D_ERR_ARG;
+  char* base = (char*)buffer;
+  out->vol = (int32_t*)(base + L.vol);
+  out->perm = (int32_t*)(base + L.perm);
+  out->tile_off = (int32_t*)(base + L.tile_off);
+  out->nbr_off = (int32_t*)(base + L.nbr_off);
+  out->nbr = (int32_t*)(base + L.nbr);
+  out->rope = (float*)(base + L.rope);
+  out->err = (int32_t*)(base + L.err);
+  out->tile[0] = TZ;
+  out->tile[1] = TY;
+  out->tile[2] = TX;
+  out->n_tiles = g.nT;
+  out->n_halo = g.n_halo;
+  return PACK3D_OK;
+}
+
+int pack3d_build_index(const pack3d_params* p, const int16_t* coords, pack3d_index* idx,
+                       pack3d_stream_t stream) {
+  Geo g;
+  int rc = make_geo(p, &g);
+  if (rc) return rc;
+  if (!coords || (rc = check_index(g, idx))) return rc ? rc : PACK3D_ERR_ARG;
+  return launch_build_index(g, coords, idx, p->rope_base, (cudaStream_t)stream);
+}
+
+int pack3d_index_check(const pack3d_index* idx, pack3d_stream_t stream) {
+  if (!idx || !idx->err) return PACK3D_ERR_ARG;
+  int32_t err[2] = {0, 0};
+  if (cudaMemcpyAsync(err, idx->err, sizeof(err), cudaMemcpyDeviceToHost,
+                      (cudaStream_t)stream) != cudaSuccess)
+    return PACK3D_ERR_CUDA;
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return PACK3D_ERR_CUDA;
+  if (err[0] & 3) return PACK3D_ERR_COORDS;
+  return err[0] ? PACK3D_ERR_TIMEOUT : PACK3D_OK;
+}
+
+int pack3d_block_summaries(const pack3d_params* p, const pack3d_index* idx, const void* k,
+                           const void* v, float* ksum, float* vsum, pack3d_stream_t stream) {
+  Geo g;
+  int rc = make_geo(p, &g);
+  if (rc) return rc;
+  if ((rc = check_index(g, idx))) return rc;
+  if (!k || !v || !ksum || !vsum) return PACK3D_ERR_ARG;
+  return launch_block_summaries(g, idx, k, v, ksum, vsum, (cudaStream_t)stream);
+}
+
+static int forward_common(const pack3d_params* p, const pack3d_index* idx, const void* q,
+                          const void* k, const void* v, const float* ksum, const float* vsum,
+                          void* out, float* lse, bool summaries, cudaStream_t s) {
+  Geo g;
+  int rc = make_geo(p, &g);
+  if (rc) return rc;
+  if ((rc = check_index(g, idx))) return rc;
+  if (!q || !k || !v || !out || !lse || (summaries && (!ksum || !vsum))) return PACK3D_ERR_ARG;
+  if (g.dtype == PACK3D_BF16 && forward_tc_supported(g))
+    return launch_forward_tc(g, idx, q, k, v, ksum, vsum, out, lse, summaries, s);
+  return launch_forward_simt(g, idx, q, k, v, ksum, vsum, out, lse, summaries, s);
+}
+
+int pack3d_forward(const pack3d_params* p, const pack3d_index* idx, const void* q, const void* k,
+                   const void* v, const float* ksum, const float* vsum, void* out, float* lse,
+                   pack3d_stream_t stream) {
+  return forward_common(p, idx, q, k, v, ksum, vsum, out, lse, true, (cudaStream_t)stream);
+}
+
+int pack3d_window_forward(const pack3d_params* p, const pack3d_index* idx, const void* q,
+                          const void* k, const void* v, void* out, float* lse,
+                          pack3d_stream_t stream) {
+  return forward_common(p, idx, q, k, v, nullptr, nullptr, out, lse, false, (cudaStream_t)stream);
+}
+
+size_t pack3d_backward_workspace_bytes(const pack3d_params* p) {
+  Geo g;
+  if (make_geo(p, &g)) return 0;
+  return backward_workspace_bytes(g);
+}
+
+int pack3d_backward(const pack3d_params* p, const pack3d_index* idx, const void* q, const void* k,
+                    const void* v, const void* out, const float* lse, const void* dout, void* dq,
+                    void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                    pack3d_stream_t stream) {
+  Geo g;
+  int rc = make_geo(p, &g);
+  if (rc) return rc;
+  if ((rc = check_index(g, idx))) return rc;
+  if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv || !workspace)
+    return PACK3D_ERR_ARG;
+  if (((uintptr_t)workspace & 255) || workspace_bytes < backward_workspace_bytes(g))
+    return PACK3D_ERR_ARG;
+  return launch_backward(g, idx, q, k, v, out, lse, dout, dq, dk, dv, workspace,
+                         (cudaStream_t)stream);
+}
+
+const char* pack3d_strerror(int status) {
+  switch (status) {
+    case PACK3D_OK: return "ok";
+    case PACK3D_ERR_ARG: return "invalid argument";
+    case PACK3D_ERR_COORDS: return "coordinates out of range or not a bijection onto the grid";
+    case PACK3D_ERR_CUDA: return "CUDA launch or runtime error";
+    case PACK3D_ERR_TIMEOUT: return "bounded device-side wait timed out";
+    case PACK3D_ERR_UNSUPPORTED: return "shape not built into this library";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

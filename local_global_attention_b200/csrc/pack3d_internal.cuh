@@ -1,0 +1,80 @@
+// Internal declarations shared by the PACK3D CUDA translation units.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "pack3d.h"
+
+namespace p3d {
+
+// Query tile (z, y, x): 128 queries, the M of one tcgen05 MMA.
+constexpr int TZ = 4, TY = 4, TX = 8, TILE = TZ * TY * TX;
+
+// Geometry derived once on the host from pack3d_params and passed by value.
+struct Geo {
+  int B, H, d, da, half;      // half = da / 2 rotation pairs per axis
+  int Z, Y, X, N;
+  int rz, ry, rx;             // window radii
+  int bz, by, bx;             // block extents
+  int nbz, nby, nbx, nb;      // block counts
+  int nTz, nTy, nTx, nT;      // query-tile counts
+  int64_t n_halo;             // halo list length per batch item
+  float tau;                  // softmax scale
+  int dtype;                  // PACK3D_BF16 / PACK3D_FP32
+};
+
+int make_geo(const pack3d_params* p, Geo* g);  // PACK3D_OK or PACK3D_ERR_*
+
+// Halo extent of query tiles along one axis: sum over tiles of the clipped
+// length of [t*T - r, t*T + T - 1 + r].
+int64_t halo_axis_total(int extent, int tile, int r);
+
+// ---- small device helpers ------------------------------------------------
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T x);
+template <>
+__device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
+  return __bfloat162float(x);
+}
+
+template <typename T>
+__device__ __forceinline__ T from_f32(float x);
+template <>
+__device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// Rotation table entry (cos, sin) for axis a, coordinate c, pair j.
+__device__ __forceinline__ float2 rope_cs(const float* tab, const Geo& g, int a, int c, int j) {
+  int off = a == 0 ? 0 : (a == 1 ? g.Z : g.Z + g.Y);
+  return reinterpret_cast<const float2*>(tab)[(off + c) * g.half + j];
+}
+
+// ---- launchers (defined in the .cu files) --------------------------------
+
+int launch_build_index(const Geo& g, const int16_t* coords, const pack3d_index* idx,
+                       float rope_base, cudaStream_t s);
+int launch_block_summaries(const Geo& g, const pack3d_index* idx, const void* k, const void* v,
+                           float* ksum, float* vsum, cudaStream_t s);
+int launch_forward_simt(const Geo& g, const pack3d_index* idx, const void* q, const void* k,
+                        const void* v, const float* ksum, const float* vsum, void* out,
+                        float* lse, bool summaries, cudaStream_t s);
+bool forward_tc_supported(const Geo& g);
+int launch_forward_tc(const Geo& g, const pack3d_index* idx, const void* q, const void* k,
+                      const void* v, const float* ksum, const float* vsum, void* out, float* lse,
+                      bool summaries, cudaStream_t s);
+size_t backward_workspace_bytes(const Geo& g);
+int launch_backward(const Geo& g, const pack3d_index* idx, const void* q, const void* k,
+                    const void* v, const void* out, const float* lse, const void* dout, void* dq,
+                    void* dk, void* dv, void* workspace, cudaStream_t s);
+
+inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? PACK3D_OK : PACK3D_ERR_CUDA; }
+
+}  // namespace p3d

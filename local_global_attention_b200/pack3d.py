@@ -1,0 +1,272 @@
+"""Python binding of the PACK3D C ABI (include/pack3d.h) over ctypes.
+
+Argument marshalling only: every step of the operator runs in the CUDA
+library ``_build/libpack3d.so``.  Tensors are torch CUDA tensors; the functions
+keep the C names and pass ``data_ptr()`` and the current (or given) stream.
+If the library is missing or no CUDA device is present, the calls raise; there
+is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+BF16, FP32 = 0, 1
+OK, ERR_ARG, ERR_COORDS, ERR_CUDA, ERR_TIMEOUT, ERR_UNSUPPORTED = 0, -1, -2, -3, -4, -5
+
+EXPORTS = ("pack3d_index_bytes", "pack3d_index_init", "pack3d_build_index", "pack3d_index_check",
+           "pack3d_block_summaries", "pack3d_forward", "pack3d_window_forward",
+           "pack3d_backward_workspace_bytes", "pack3d_backward", "pack3d_strerror")
+
+
+class Params(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("B", "H", "head_dim", "Z", "Y", "X", "wz", "wy", "wx", "bz", "by", "bx")] + [
+        ("rope_base", ctypes.c_float), ("scale", ctypes.c_float), ("dtype", ctypes.c_int32)]
+
+
+class Index(ctypes.Structure):
+    _fields_ = [("vol", ctypes.c_void_p), ("perm", ctypes.c_void_p),
+                ("tile_off", ctypes.c_void_p), ("nbr_off", ctypes.c_void_p),
+                ("nbr", ctypes.c_void_p), ("rope", ctypes.c_void_p), ("err", ctypes.c_void_p),
+                ("tile", ctypes.c_int32 * 3), ("n_tiles", ctypes.c_int32),
+                ("n_halo", ctypes.c_int64)]
+
+
+class Pack3dError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {strerror(status)} ({status})")
+        self.status = status
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def load(build_if_missing: bool = True):
+    """Load libpack3d.so (building it in-tree first if it is missing)."""
+    global _lib
+    if _lib is None:
+        path = _build.LIB
+        if not os.path.exists(path):
+            if not build_if_missing:
+                raise OSError(f"PACK3D CUDA library not built: {path}")
+            _build.build()
+        lib = ctypes.CDLL(path)
+        P = ctypes.POINTER
+        vp = ctypes.c_void_p
+        lib.pack3d_index_bytes.argtypes = [P(Params)]
+        lib.pack3d_index_bytes.restype = ctypes.c_size_t
+        lib.pack3d_index_init.argtypes = [P(Params), vp, ctypes.c_size_t, P(Index)]
+        lib.pack3d_build_index.argtypes = [P(Params), vp, P(Index), vp]
+        lib.pack3d_index_check.argtypes = [P(Index), vp]
+        lib.pack3d_block_summaries.argtypes = [P(Params), P(Index), vp, vp, vp, vp, vp]
+        lib.pack3d_forward.argtypes = [P(Params), P(Index), vp, vp, vp, vp, vp, vp, vp, vp]
+        lib.pack3d_window_forward.argtypes = [P(Params), P(Index), vp, vp, vp, vp, vp, vp]
+        lib.pack3d_backward_workspace_bytes.argtypes = [P(Params)]
+        lib.pack3d_backward_workspace_bytes.restype = ctypes.c_size_t
+        lib.pack3d_backward.argtypes = [P(Params), P(Index), vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                        vp, ctypes.c_size_t, vp]
+        lib.pack3d_strerror.argtypes = [ctypes.c_int]
+        lib.pack3d_strerror.restype = ctypes.c_char_p
+        for name in EXPORTS:
+            getattr(lib, name).restype = getattr(lib, name).restype or ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def strerror(status: int) -> str:
+    return load().pack3d_strerror(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != OK:
+        raise Pack3dError(status, what)
+
+
+def make_params(shape, dtype=None, scale: float = 0.0) -> Params:
+    """Params from any object with ``B, H, d, Z, Y, X, window, block, rope_base``
+    (and ``dtype`` "bf16"/"fp32" unless given)."""
+    dt = dtype if dtype is not None else getattr(shape, "dtype", "bf16")
+    code = {"bf16": BF16, "fp32": FP32, torch.bfloat16: BF16, torch.float32: FP32}[dt]
+    w, b = tuple(shape.window), tuple(shape.block)
+    return Params(shape.B, shape.H, shape.d, shape.Z, shape.Y, shape.X, w[0], w[1], w[2],
+                  b[0], b[1], b[2], float(shape.rope_base), float(scale), code)
+
+
+def _stream(stream):
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("PACK3D tensors must be CUDA tensors")
+        if t is not None and not t.is_contiguous():
+            raise ValueError("PACK3D tensors must be contiguous")
+
+
+class IndexBuffers:
+    """A built index: the caller-owned device buffer and the C struct over it."""
+
+    def __init__(self, params: Params, device=None):
+        lib = load()
+        self.params = params
+        nbytes = lib.pack3d_index_bytes(ctypes.byref(params))
+        if nbytes == 0:
+            raise Pack3dError(ERR_ARG, "pack3d_index_bytes")
+        self.buffer = torch.empty(nbytes + 256, dtype=torch.uint8, device=device or "cuda")
+        base = self.buffer.data_ptr()
+        off = (-base) % 256
+        self.struct = Index()
+        _check(lib.pack3d_index_init(ctypes.byref(params), ctypes.c_void_p(base + off),
+                                     ctypes.c_size_t(nbytes), ctypes.byref(self.struct)),
+               "pack3d_index_init")
+        self.nbytes = nbytes
+
+    # Views of the index arrays (for tests and inspection).
+    def _view(self, field, count, dtype):
+        ptr = getattr(self.struct, field)
+        off = ptr - self.buffer.data_ptr()
+        esz = torch.tensor([], dtype=dtype).element_size()
+        return self.buffer[off:off + count * esz].view(dtype)
+
+    def arrays(self):
+        p, s = self.params, self.struct
+        N = p.Z * p.Y * p.X
+        T = s.n_tiles
+        return {
+            "vol": self._view("vol", p.B * N, torch.int32).view(p.B, N),
+            "perm": self._view("perm", p.B * N, torch.int32).view(p.B, N),
+            "tile_off": self._view("tile_off", p.B * (T + 1), torch.int32).view(p.B, T + 1),
+            "nbr_off": self._view("nbr_off", T + 1, torch.int32),
+            "nbr": self._view("nbr", p.B * s.n_halo, torch.int32).view(p.B, s.n_halo),
+            "rope": self._view("rope", 2 * (p.Z + p.Y + p.X) * (p.head_dim // 6), torch.float32),
+            "err": self._view("err", 2, torch.int32),
+        }
+
+
+def pack3d_build_index(params: Params, coords: torch.Tensor, index: IndexBuffers = None,
+                       stream=None) -> IndexBuffers:
+    _need_cuda(coords)
+    if coords.dtype != torch.int16:
+        raise ValueError("coords must be int16 [B, N, 3]")
+    if index is None:
+        index = IndexBuffers(params, device=coords.device)
+    _check(load().pack3d_build_index(ctypes.byref(params), _ptr(coords),
+                                     ctypes.byref(index.struct), _stream(stream)),
+           "pack3d_build_index")
+    return index
+
+
+def pack3d_index_check(index: IndexBuffers, stream=None) -> int:
+    """Synchronise and return the index status code (0, ERR_COORDS, ERR_TIMEOUT)."""
+    return int(load().pack3d_index_check(ctypes.byref(index.struct), _stream(stream)))
+
+
+def _dims(params):
+    return params.B, params.Z * params.Y * params.X, params.H, params.head_dim
+
+
+def pack3d_block_summaries(params: Params, index: IndexBuffers, k, v, ksum=None, vsum=None,
+                           stream=None):
+    _need_cuda(k, v)
+    B, N, H, d = _dims(params)
+    nb = (params.Z // params.bz) * (params.Y // params.by) * (params.X // params.bx)
+    if ksum is None:
+        ksum = torch.empty(B, H, nb, d, dtype=torch.float32, device=k.device)
+    if vsum is None:
+        vsum = torch.empty(B, H, nb, d, dtype=torch.float32, device=k.device)
+    _need_cuda(ksum, vsum)
+    _check(load().pack3d_block_summaries(ctypes.byref(params), ctypes.byref(index.struct),
+                                         _ptr(k), _ptr(v), _ptr(ksum), _ptr(vsum),
+                                         _stream(stream)), "pack3d_block_summaries")
+    return ksum, vsum
+
+
+def pack3d_forward(params: Params, index: IndexBuffers, q, k, v, ksum, vsum, out=None, lse=None,
+                   stream=None):
+    _need_cuda(q, k, v, ksum, vsum)
+    B, N, H, d = _dims(params)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty(B, H, N, dtype=torch.float32, device=q.device) if lse is None else lse
+    _need_cuda(out, lse)
+    _check(load().pack3d_forward(ctypes.byref(params), ctypes.byref(index.struct), _ptr(q),
+                                 _ptr(k), _ptr(v), _ptr(ksum), _ptr(vsum), _ptr(out), _ptr(lse),
+                                 _stream(stream)), "pack3d_forward")
+    return out, lse
+
+
+def pack3d_window_forward(params: Params, index: IndexBuffers, q, k, v, out=None, lse=None,
+                          stream=None):
+    _need_cuda(q, k, v)
+    B, N, H, d = _dims(params)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty(B, H, N, dtype=torch.float32, device=q.device) if lse is None else lse
+    _need_cuda(out, lse)
+    _check(load().pack3d_window_forward(ctypes.byref(params), ctypes.byref(index.struct),
+                                        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                                        _stream(stream)), "pack3d_window_forward")
+    return out, lse
+
+
+def pack3d_backward_workspace_bytes(params: Params) -> int:
+    return int(load().pack3d_backward_workspace_bytes(ctypes.byref(params)))
+
+
+def pack3d_backward(params: Params, index: IndexBuffers, q, k, v, out, lse, dout, dq=None,
+                    dk=None, dv=None, workspace=None, stream=None):
+    _need_cuda(q, k, v, out, lse, dout)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    nbytes = pack3d_backward_workspace_bytes(params)
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    _need_cuda(dq, dk, dv, workspace)
+    _check(load().pack3d_backward(ctypes.byref(params), ctypes.byref(index.struct), _ptr(q),
+                                  _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq),
+                                  _ptr(dk), _ptr(dv), _ptr(workspace),
+                                  ctypes.c_size_t(workspace.numel() * workspace.element_size()),
+                                  _stream(stream)), "pack3d_backward")
+    return dq, dk, dv
+
+
+class Pack3D:
+    """Convenience wrapper: one operator shape, its index, and the calls."""
+
+    def __init__(self, shape, dtype=None, scale: float = 0.0):
+        self.params = make_params(shape, dtype, scale)
+        self.index = None
+
+    def build_index(self, coords, stream=None, check=True):
+        self.index = pack3d_build_index(self.params, coords, self.index, stream)
+        if check:
+            st = pack3d_index_check(self.index, stream)
+            _check(st, "pack3d_index_check")
+        return self.index
+
+    def forward(self, q, k, v, stream=None):
+        ksum, vsum = pack3d_block_summaries(self.params, self.index, k, v, stream=stream)
+        return pack3d_forward(self.params, self.index, q, k, v, ksum, vsum, stream=stream)
+
+    def window_forward(self, q, k, v, stream=None):
+        return pack3d_window_forward(self.params, self.index, q, k, v, stream=stream)
+
+    def backward(self, q, k, v, out, lse, dout, stream=None):
+        return pack3d_backward(self.params, self.index, q, k, v, out, lse, dout, stream=stream)

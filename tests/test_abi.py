@@ -1,0 +1,87 @@
+"""The C-ABI library builds, loads and exports every entry point the header
+declares; host-side argument checks work without a GPU (no CUDA call is made)."""
+import ctypes
+import os
+import re
+from types import SimpleNamespace
+
+import pytest
+
+from local_global_attention_b200 import build as B
+from local_global_attention_b200 import pack3d as P
+
+HEADER = os.path.join(B.ROOT, "include", "pack3d.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"PACK3D_API\s+[\w\s\*]+?\b(pack3d_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return P.load()
+
+
+def test_header_declares_the_operator_calls():
+    names = declared_symbols()
+    for n in ("pack3d_build_index", "pack3d_block_summaries", "pack3d_forward",
+              "pack3d_window_forward", "pack3d_backward"):
+        assert n in names
+    assert set(names) == set(P.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def shape(**kw):
+    base = dict(B=2, H=8, d=96, Z=32, Y=32, X=64, window=(7, 7, 7), block=(8, 8, 8),
+                rope_base=100.0, dtype="bf16")
+    base.update(kw)
+    return SimpleNamespace(**base)
+
+
+def test_index_bytes_and_argument_checks(lib):
+    p = P.make_params(shape())
+    n = lib.pack3d_index_bytes(ctypes.byref(p))
+    N = 32 * 32 * 64
+    assert n >= 4 * (2 * 2 * N)  # vol + perm at least
+    for bad in (dict(window=(6, 7, 7)), dict(block=(5, 8, 8)), dict(d=90), dict(d=0),
+                dict(rope_base=0.0), dict(Z=0)):
+        assert lib.pack3d_index_bytes(ctypes.byref(P.make_params(shape(**bad)))) == 0, bad
+    # shapes the library is not built for report ERR_UNSUPPORTED, not ERR_ARG
+    idx = P.Index()
+    st = lib.pack3d_index_init(ctypes.byref(P.make_params(shape(d=36))), ctypes.c_void_p(256),
+                               ctypes.c_size_t(1 << 30), ctypes.byref(idx))
+    assert st == P.ERR_UNSUPPORTED
+    # misaligned or short buffers are rejected before any device access
+    assert lib.pack3d_index_init(ctypes.byref(p), ctypes.c_void_p(257), ctypes.c_size_t(n),
+                                 ctypes.byref(idx)) == P.ERR_ARG
+    assert lib.pack3d_index_init(ctypes.byref(p), ctypes.c_void_p(256), ctypes.c_size_t(n - 1),
+                                 ctypes.byref(idx)) == P.ERR_ARG
+    assert lib.pack3d_index_init(ctypes.byref(p), ctypes.c_void_p(1 << 20), ctypes.c_size_t(n),
+                                 ctypes.byref(idx)) == P.OK
+    assert tuple(idx.tile) == (4, 4, 8)
+    assert idx.n_tiles == 8 * 8 * 8
+    # halo list length: product over axes of the clipped tile extents
+    assert idx.n_halo == (7 + 7 + 6 * 10) ** 2 * (11 + 11 + 6 * 14)
+
+
+def test_null_pointers_rejected_without_cuda(lib):
+    p = P.make_params(shape())
+    idx = P.Index()
+    assert lib.pack3d_build_index(ctypes.byref(p), None, ctypes.byref(idx), None) == P.ERR_ARG
+    assert lib.pack3d_forward(ctypes.byref(p), ctypes.byref(idx), None, None, None, None, None,
+                              None, None, None) == P.ERR_ARG
+    assert lib.pack3d_backward(ctypes.byref(p), None, *([None] * 10), ctypes.c_size_t(0),
+                               None) == P.ERR_ARG
+
+
+def test_strerror(lib):
+    for st in (P.OK, P.ERR_ARG, P.ERR_COORDS, P.ERR_CUDA, P.ERR_TIMEOUT, P.ERR_UNSUPPORTED):
+        assert P.strerror(st)
+    assert P.strerror(12345) == "unknown status"

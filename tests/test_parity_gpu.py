@@ -1,0 +1,118 @@
+"""Forward parity of the CUDA path against the CPU oracle on seeded inputs.
+
+Small volumes (several query tiles and ragged tails) are compared element by
+element over every output; the full-size workloads in the launch
+configuration the benchmark times are compared on sampled queries the oracle
+computes one by one (corners, faces, edges and random voxels)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from local_global_attention_b200 import configs as C
+from local_global_attention_b200 import inputs as I
+from local_global_attention_b200 import pack3d as P
+
+from gpu_common import assert_close, gpu_run, oracle_sample
+
+pytestmark = pytest.mark.gpu
+
+RAGGED96 = I.Workload(name="ragged_6x10x20_d96", B=2, H=2, d=96, Z=6, Y=10, X=20,
+                      window=(5, 3, 7), block=(3, 5, 4), dtype="bf16", value_scale=1.0,
+                      seed=31)
+SMALL = [
+    C.TINY,
+    RAGGED96,
+    RAGGED96.replace(name="ragged_fp32_d96", dtype="fp32", seed=32),
+    I.Workload(name="odd_5x9x17_d48", B=1, H=3, d=48, Z=5, Y=9, X=17, window=(3, 5, 3),
+               block=(5, 3, 17), dtype="bf16", seed=33),
+    I.Workload(name="big_window_8x8x16_d96", B=1, H=2, d=96, Z=8, Y=8, X=16, window=(15, 15, 31),
+               block=(2, 4, 4), dtype="bf16", seed=34),
+    I.Workload(name="self_window_4x4x8_d96", B=1, H=2, d=96, Z=4, Y=8, X=8, window=(1, 1, 1),
+               block=(2, 2, 2), dtype="bf16", seed=35),
+    I.Workload(name="d12_fp32_6x6x6", B=2, H=2, d=12, Z=6, Y=6, X=6, window=(3, 3, 3),
+               block=(2, 3, 6), dtype="fp32", seed=36),
+    I.Workload(name="d24_bf16_4x12x9", B=1, H=2, d=24, Z=4, Y=12, X=9, window=(3, 5, 5),
+               block=(2, 6, 3), dtype="bf16", seed=37),
+]
+
+
+def full_oracle(wl, inp, window_only):
+    return oracle.forward(wl, inp["coords"], inp["q"], inp["k"], inp["v"], window_only=window_only)
+
+
+@pytest.mark.parametrize("wl", SMALL, ids=lambda w: w.name)
+@pytest.mark.parametrize("window_only", [False, True], ids=["pack3d", "window"])
+def test_forward_small_full(oracle_lib, wl, window_only):
+    inp = I.make_inputs(wl, "random")
+    res = gpu_run(wl, inp, window_only=window_only)
+    out, lse = full_oracle(wl, inp, window_only)
+    assert_close(res["out"], out, wl.dtype, "out")
+    assert_close(res["lse"], lse, wl.dtype, "lse")
+
+
+@pytest.mark.parametrize("wl", [C.TINY, RAGGED96, C.VOL16K], ids=lambda w: w.name)
+def test_block_summaries(oracle_lib, wl):
+    inp = I.make_inputs(wl, wl.packings[0])
+    res = gpu_run(wl, inp)
+    ks, vs = oracle.block_summaries(wl, inp["coords"], inp["k"], inp["v"])
+    # fp32 accumulation of exactly represented inputs: relative error ~1e-6
+    np.testing.assert_allclose(res["ksum"].double().numpy(), ks, rtol=0, atol=2e-5)
+    np.testing.assert_allclose(res["vsum"].double().numpy(), vs, rtol=0, atol=2e-5)
+
+
+@pytest.mark.slow
+def test_forward_vol16k_full(oracle_lib):
+    wl = C.VOL16K
+    inp = I.make_inputs(wl, "morton")
+    res = gpu_run(wl, inp)
+    out, lse = full_oracle(wl, inp, False)
+    assert_close(res["out"], out, wl.dtype, "out")
+    assert_close(res["lse"], lse, wl.dtype, "lse")
+
+
+@pytest.fixture(scope="module")
+def grid65k():
+    return I.grid_tensors(C.VOL65K)
+
+
+@pytest.mark.parametrize("packing", I.PACKINGS)
+def test_forward_65k_sampled(oracle_lib, grid65k, packing):
+    wl = C.VOL65K
+    inp = I.make_inputs(wl, packing, grid=grid65k)
+    res = gpu_run(wl, inp)
+    (b, h, i), out, lse = oracle_sample(wl, inp, 48, seed=5)
+    assert_close(res["out"][b, i, h], out, wl.dtype, "out")
+    assert_close(res["lse"][b, h, i], lse, wl.dtype, "lse")
+    wres = gpu_run(wl, inp, window_only=True)
+    (b, h, i), wout, wlse = oracle_sample(wl, inp, 24, window_only=True, seed=6)
+    assert_close(wres["out"][b, i, h], wout, wl.dtype, "window out")
+    assert_close(wres["lse"][b, h, i], wlse, wl.dtype, "window lse")
+
+
+def test_forward_65k_packing_equivariance_bit_exact(grid65k):
+    """Every packing of the same field gives the same per-voxel output, bit for
+    bit: all accumulation orders follow the grid, never the memory order."""
+    wl = C.VOL65K
+    ref = None
+    for packing in I.PACKINGS:
+        inp = I.make_inputs(wl, packing, grid=grid65k)
+        res = gpu_run(wl, inp)
+        out = I.unpack_rows(res["out"], inp["order"])
+        lse = I.unpack_rows(res["lse"].permute(0, 2, 1), inp["order"])
+        if ref is None:
+            ref = (out, lse)
+        else:
+            assert torch.equal(out, ref[0]), packing
+            assert torch.equal(lse, ref[1]), packing
+
+
+@pytest.mark.slow
+def test_forward_micro1m_sampled(oracle_lib):
+    wl = C.MICRO1M
+    dev = "cuda"
+    inp = I.make_inputs(wl, "block", grid=I.grid_tensors(wl, device=dev))
+    res = gpu_run(wl, inp)
+    (b, h, i), out, lse = oracle_sample(wl, inp, 64, seed=7)
+    assert_close(res["out"][b, i, h], out, wl.dtype, "out")
+    assert_close(res["lse"][b, h, i], lse, wl.dtype, "lse")
