@@ -32,7 +32,8 @@
  * never allocates or frees device memory and keeps no global state.  All
  * pointers except the params and index structs are DEVICE pointers.  Layouts:
  *   q, k, v, out, dout, dq, dk, dv : [B][N][H][head_dim], packed order,
- *                                    bf16 (dtype PACK3D_BF16) or fp32;
+ *                                    bf16 (dtype PACK3D_BF16) or fp32
+ *                                    (out is fp32 when out_fp32 is set);
  *   coords                        : int16 [B][N][3] as (z, y, x);
  *   ksum, vsum                    : fp32 [B][H][nb][head_dim], blocks in
  *                                    raster order (nb = Z/bz * Y/by * X/bx);
@@ -84,6 +85,8 @@ typedef struct {
   float rope_base; /* > 0 */
   float scale;     /* softmax scale; <= 0 selects 1 / sqrt(head_dim) */
   int32_t dtype;   /* PACK3D_BF16 or PACK3D_FP32 (inputs, outputs, gradients) */
+  int32_t out_fp32; /* nonzero: the forward's out (and the backward's out argument) is
+                       fp32 even when dtype is PACK3D_BF16 */
 } pack3d_params;
 
 /* Geometry index of one packing, built by pack3d_build_index into one

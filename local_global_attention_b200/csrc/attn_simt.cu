@@ -106,11 +106,11 @@ struct ChunkCoords {
 // Forward
 // ---------------------------------------------------------------------------
 
-template <typename T, int D, bool SUMMARY>
+template <typename T, typename TO, int D, bool SUMMARY>
 __global__ void __launch_bounds__(TILE * Split<D>::G) k_forward_simt(
     Geo g, pack3d_index ix, const T* __restrict__ q, const T* __restrict__ k,
     const T* __restrict__ v, const float* __restrict__ ksum, const float* __restrict__ vsum,
-    T* __restrict__ out, float* __restrict__ lse) {
+    TO* __restrict__ out, float* __restrict__ lse) {
   constexpr int G = Split<D>::G, CPT = Split<D>::CPT;
   if (ix.err[0]) return;
   __shared__ float sk[KC][D];
@@ -257,9 +257,9 @@ __global__ void __launch_bounds__(TILE * Split<D>::G) k_forward_simt(
 
   if (active) {
     float inv = 1.f / l;
-    T* orow = out + (((int64_t)b * g.N + qi) * g.H + h) * D;
+    TO* orow = out + (((int64_t)b * g.N + qi) * g.H + h) * D;
 #pragma unroll
-    for (int u = 0; u < CPT; ++u) orow[lane * CPT + u] = from_f32<T>(o[u] * inv);
+    for (int u = 0; u < CPT; ++u) orow[lane * CPT + u] = from_f32<TO>(o[u] * inv);
     if (lane == 0) lse[((int64_t)b * g.H + h) * g.N + qi] = (m + log2f(l)) * LN2;
   }
 }
@@ -269,8 +269,8 @@ __global__ void __launch_bounds__(TILE * Split<D>::G) k_forward_simt(
 // ---------------------------------------------------------------------------
 
 // delta_i = sum_c dout_ic * out_ic, fp32, [B][H][N].
-template <typename T>
-__global__ void k_bwd_delta(Geo g, const int32_t* __restrict__ err, const T* __restrict__ out,
+template <typename T, typename TO>
+__global__ void k_bwd_delta(Geo g, const int32_t* __restrict__ err, const TO* __restrict__ out,
                             const T* __restrict__ dout, float* delta) {
   if (err[0]) return;
   int64_t r = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;  // (b, i, h) row
@@ -278,7 +278,7 @@ __global__ void k_bwd_delta(Geo g, const int32_t* __restrict__ err, const T* __r
   int h = (int)(r % g.H);
   int64_t bi = r / g.H;
   int i = (int)(bi % g.N), b = (int)(bi / g.N);
-  const T* o = out + r * g.d;
+  const TO* o = out + r * g.d;
   const T* d = dout + r * g.d;
   float s = 0.f;
   for (int c = 0; c < g.d; ++c) s += to_f32(o[c]) * to_f32(d[c]);
@@ -660,19 +660,28 @@ __global__ void __launch_bounds__(TILE * Split<D>::G) k_bwd_dkdv(
   }
 }
 
+template <typename T, typename TO, int D>
+int forward_launch(const Geo& g, const pack3d_index* idx, const void* q, const void* k,
+                   const void* v, const float* ksum, const float* vsum, void* out, float* lse,
+                   bool summaries, cudaStream_t s) {
+  dim3 grid(g.nT, g.H, g.B);
+  dim3 block(TILE * Split<D>::G);
+  if (summaries)
+    k_forward_simt<T, TO, D, true><<<grid, block, 0, s>>>(
+        g, *idx, (const T*)q, (const T*)k, (const T*)v, ksum, vsum, (TO*)out, lse);
+  else
+    k_forward_simt<T, TO, D, false><<<grid, block, 0, s>>>(
+        g, *idx, (const T*)q, (const T*)k, (const T*)v, ksum, vsum, (TO*)out, lse);
+  return cuda_status(cudaGetLastError());
+}
+
 template <typename T, int D>
 int forward_dispatch_sum(const Geo& g, const pack3d_index* idx, const void* q, const void* k,
                          const void* v, const float* ksum, const float* vsum, void* out,
                          float* lse, bool summaries, cudaStream_t s) {
-  dim3 grid(g.nT, g.H, g.B);
-  dim3 block(TILE * Split<D>::G);
-  if (summaries)
-    k_forward_simt<T, D, true><<<grid, block, 0, s>>>(g, *idx, (const T*)q, (const T*)k,
-                                                      (const T*)v, ksum, vsum, (T*)out, lse);
-  else
-    k_forward_simt<T, D, false><<<grid, block, 0, s>>>(g, *idx, (const T*)q, (const T*)k,
-                                                       (const T*)v, ksum, vsum, (T*)out, lse);
-  return cuda_status(cudaGetLastError());
+  if (g.out_fp32)
+    return forward_launch<T, float, D>(g, idx, q, k, v, ksum, vsum, out, lse, summaries, s);
+  return forward_launch<T, T, D>(g, idx, q, k, v, ksum, vsum, out, lse, summaries, s);
 }
 
 template <typename T>
@@ -717,8 +726,12 @@ int backward_typed(const Geo& g, const pack3d_index* idx, const void* q, const v
                    void* dk, void* dv, void* workspace, cudaStream_t s) {
   BwdWs w = carve(g, workspace);
   int64_t rows = (int64_t)g.B * g.N * g.H;
-  k_bwd_delta<T><<<(unsigned)((rows + 255) / 256), 256, 0, s>>>(g, idx->err, (const T*)out,
-                                                               (const T*)dout, w.delta);
+  if (g.out_fp32)
+    k_bwd_delta<T, float><<<(unsigned)((rows + 255) / 256), 256, 0, s>>>(
+        g, idx->err, (const float*)out, (const T*)dout, w.delta);
+  else
+    k_bwd_delta<T, T><<<(unsigned)((rows + 255) / 256), 256, 0, s>>>(
+        g, idx->err, (const T*)out, (const T*)dout, w.delta);
   int rc = launch_block_summaries(g, idx, k, v, w.ksum, w.vsum, s);
   if (rc) return rc;
   dim3 sgrid((g.nb + BC - 1) / BC, g.B, g.H);

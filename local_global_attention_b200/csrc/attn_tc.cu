@@ -150,7 +150,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     k_forward_tc(Geo g, pack3d_index ix, const __nv_bfloat16* __restrict__ q,
                  const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
                  const float* __restrict__ ksum, const float* __restrict__ vsum,
-                 __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
+                 void* __restrict__ out_raw, float* __restrict__ lse) {
   if (ix.err[0]) return;
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -380,24 +380,42 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   // ---- epilogue ----
   if (!sm.abort) {
     const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-    uint4 orow[12];
-    uint32_t* ow = reinterpret_cast<uint32_t*>(orow);
+    const int64_t orow_off = (((int64_t)b * g.N + qi) * g.H + h) * D;
+    if (!g.out_fp32) {
+      uint4 orow[12];
+      uint32_t* ow = reinterpret_cast<uint32_t*>(orow);
 #pragma unroll
-    for (int part = 0; part < 3; ++part) {
-      uint32_t r[32];
-      tmem_ld32(tO + part * 32, r);
-      tmem_wait_ld();
+      for (int part = 0; part < 3; ++part) {
+        uint32_t r[32];
+        tmem_ld32(tO + part * 32, r);
+        tmem_wait_ld();
 #pragma unroll
-      for (int i = 0; i < 16; ++i)
-        ow[part * 16 + i] =
-            pack_bf16x2(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
+        for (int i = 0; i < 16; ++i)
+          ow[part * 16 + i] =
+              pack_bf16x2(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
+      }
+      if (active) {
+        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(out_raw) + orow_off);
+#pragma unroll
+        for (int i = 0; i < 12; ++i) dst[i] = orow[i];
+      }
+    } else {
+      float* dstf = reinterpret_cast<float*>(out_raw) + orow_off;
+#pragma unroll
+      for (int part = 0; part < 3; ++part) {
+        uint32_t r[32];
+        tmem_ld32(tO + part * 32, r);
+        tmem_wait_ld();
+        if (active) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            reinterpret_cast<float4*>(dstf + part * 32)[i] = make_float4(
+                __uint_as_float(r[4 * i]) * inv, __uint_as_float(r[4 * i + 1]) * inv,
+                __uint_as_float(r[4 * i + 2]) * inv, __uint_as_float(r[4 * i + 3]) * inv);
+        }
+      }
     }
-    if (active) {
-      uint4* dst = reinterpret_cast<uint4*>(out + (((int64_t)b * g.N + qi) * g.H + h) * D);
-#pragma unroll
-      for (int i = 0; i < 12; ++i) dst[i] = orow[i];
-      lse[((int64_t)b * g.H + h) * g.N + qi] = (m_run + log2f(l_run)) * LN2;
-    }
+    if (active) lse[((int64_t)b * g.H + h) * g.N + qi] = (m_run + log2f(l_run)) * LN2;
   } else if (tid == 0) {
     atomicOr(&ix.err[0], ERR_TIMEOUT_BIT);
   }
@@ -423,7 +441,7 @@ int launch_forward_tc(const Geo& g, const pack3d_index* idx, const void* q, cons
   if (e != cudaSuccess) return PACK3D_ERR_CUDA;
   kern<<<grid, NTHREADS, SMEM_REQUEST, s>>>(g, *idx, (const __nv_bfloat16*)q,
                                              (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
-                                             ksum, vsum, (__nv_bfloat16*)out, lse);
+                                             ksum, vsum, out, lse);
   return cuda_status(cudaGetLastError());
 }
 

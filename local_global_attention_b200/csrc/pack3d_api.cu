@@ -63,6 +63,7 @@ int make_geo(const pack3d_params* p, Geo* g) {
   if (g->n_halo * p->B >= (int64_t)1 << 31) return PACK3D_ERR_ARG;
   g->tau = p->scale > 0.f ? p->scale : 1.0f / sqrtf((float)p->head_dim);
   g->dtype = p->dtype;
+  g->out_fp32 = (p->out_fp32 != 0 || p->dtype == PACK3D_FP32) ? 1 : 0;
   return PACK3D_OK;
 }
 

@@ -23,6 +23,7 @@ struct Geo {
   int64_t n_halo;             // halo list length per batch item
   float tau;                  // softmax scale
   int dtype;                  // PACK3D_BF16 / PACK3D_FP32
+  int out_fp32;               // out is fp32 (also when dtype is bf16)
 };
 
 int make_geo(const pack3d_params* p, Geo* g);  // PACK3D_OK or PACK3D_ERR_*

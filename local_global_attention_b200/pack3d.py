@@ -26,7 +26,8 @@ EXPORTS = ("pack3d_index_bytes", "pack3d_index_init", "pack3d_build_index", "pac
 class Params(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
                 ("B", "H", "head_dim", "Z", "Y", "X", "wz", "wy", "wx", "bz", "by", "bx")] + [
-        ("rope_base", ctypes.c_float), ("scale", ctypes.c_float), ("dtype", ctypes.c_int32)]
+        ("rope_base", ctypes.c_float), ("scale", ctypes.c_float), ("dtype", ctypes.c_int32),
+        ("out_fp32", ctypes.c_int32)]
 
 
 class Index(ctypes.Structure):
@@ -91,14 +92,19 @@ def _check(status: int, what: str):
         raise Pack3dError(status, what)
 
 
-def make_params(shape, dtype=None, scale: float = 0.0) -> Params:
+def make_params(shape, dtype=None, scale: float = 0.0, out_fp32: bool = False) -> Params:
     """Params from any object with ``B, H, d, Z, Y, X, window, block, rope_base``
-    (and ``dtype`` "bf16"/"fp32" unless given)."""
+    (and ``dtype`` "bf16"/"fp32" unless given).  ``out_fp32`` makes the forward
+    output fp32 for bf16 inputs."""
     dt = dtype if dtype is not None else getattr(shape, "dtype", "bf16")
     code = {"bf16": BF16, "fp32": FP32, torch.bfloat16: BF16, torch.float32: FP32}[dt]
     w, b = tuple(shape.window), tuple(shape.block)
     return Params(shape.B, shape.H, shape.d, shape.Z, shape.Y, shape.X, w[0], w[1], w[2],
-                  b[0], b[1], b[2], float(shape.rope_base), float(scale), code)
+                  b[0], b[1], b[2], float(shape.rope_base), float(scale), code, int(bool(out_fp32)))
+
+
+def out_dtype(params: Params, like: torch.Tensor) -> torch.dtype:
+    return torch.float32 if params.out_fp32 else like.dtype
 
 
 def _stream(stream):
@@ -203,7 +209,7 @@ def pack3d_forward(params: Params, index: IndexBuffers, q, k, v, ksum, vsum, out
                    stream=None):
     _need_cuda(q, k, v, ksum, vsum)
     B, N, H, d = _dims(params)
-    out = torch.empty_like(q) if out is None else out
+    out = torch.empty_like(q, dtype=out_dtype(params, q)) if out is None else out
     lse = torch.empty(B, H, N, dtype=torch.float32, device=q.device) if lse is None else lse
     _need_cuda(out, lse)
     _check(load().pack3d_forward(ctypes.byref(params), ctypes.byref(index.struct), _ptr(q),
@@ -216,7 +222,7 @@ def pack3d_window_forward(params: Params, index: IndexBuffers, q, k, v, out=None
                           stream=None):
     _need_cuda(q, k, v)
     B, N, H, d = _dims(params)
-    out = torch.empty_like(q) if out is None else out
+    out = torch.empty_like(q, dtype=out_dtype(params, q)) if out is None else out
     lse = torch.empty(B, H, N, dtype=torch.float32, device=q.device) if lse is None else lse
     _need_cuda(out, lse)
     _check(load().pack3d_window_forward(ctypes.byref(params), ctypes.byref(index.struct),
@@ -250,8 +256,8 @@ def pack3d_backward(params: Params, index: IndexBuffers, q, k, v, out, lse, dout
 class Pack3D:
     """Convenience wrapper: one operator shape, its index, and the calls."""
 
-    def __init__(self, shape, dtype=None, scale: float = 0.0):
-        self.params = make_params(shape, dtype, scale)
+    def __init__(self, shape, dtype=None, scale: float = 0.0, out_fp32: bool = False):
+        self.params = make_params(shape, dtype, scale, out_fp32)
         self.index = None
 
     def build_index(self, coords, stream=None, check=True):
