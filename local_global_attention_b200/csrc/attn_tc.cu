@@ -5,28 +5,31 @@
 // window misses, in one softmax, with axial RoPE on grid coordinates.
 //
 // One CTA computes one 4 x 4 x 8 query tile (M = 128 rows) of one
-// (batch item, head):
-//   * the tile's queries are gathered through the tile permutation, rotated
-//     in registers and stored to shared memory in the 64-byte-swizzled K-major
-//     layout (head_dim 96 = three 32-channel segments, one per axis, so each
-//     rotation segment is exactly one swizzle atom column);
-//   * the tile's halo (the union of its windows) is streamed in chunks of 128
-//     keys through the halo list; each key row is rotated on the way into
-//     shared memory and each value row is stored as the MN-major B operand of
-//     the PV product;
-//   * S = Q K^T runs as six tcgen05.mma (K = 16) into TMEM; the four softmax
-//     warps (one row per thread) read S, apply the 3D window mask, keep the
-//     online max and sum, and write P (bf16) back over S in TMEM;
-//   * O += P V runs as eight tcgen05.mma with A = P read from TMEM;
-//   * after the local chunks, the block summaries are streamed the same way,
-//     with the mask "block box does not meet the window box", into the same
-//     softmax state (no count bias);
-//   * the epilogue divides by the row sum, writes out in packed order and the
-//     natural-log LSE.
-// The running max is only moved when a row's new maximum exceeds it by more
-// than 8 (log2 units), so O is rescaled in TMEM rarely; the result is the same
-// softmax.  Two CTAs share an SM (256 TMEM columns each), so one CTA's gather
-// overlaps the other's MMAs and softmax.
+// (batch item, head).  The tile's halo (the union of its windows, raster order)
+// and then the block summaries are streamed in chunks of 64 keys.  Roles:
+//
+//   * producers (warps 5-8): gather the query rows once and each chunk's key
+//     and value rows through the index, rotate queries and keys in registers
+//     (axial RoPE, fp32 arithmetic), and store them in the 64-byte-swizzled
+//     operand layout of a 3-stage shared-memory ring.  head_dim 96 is three
+//     32-channel segments, one per axis, so a rotation segment is exactly one
+//     swizzle-atom column.  Summary chunks are converted from fp32 instead;
+//   * MMA (warp 4, one thread): S_j = Q K_j^T (six tcgen05.mma, K = 16) into
+//     one of two TMEM S buffers, and O += P_j V_j (four tcgen05.mma, A = P from
+//     TMEM, B = V MN-major in shared memory), so S_{j+1} is computed while the
+//     softmax works on S_j;
+//   * softmax (warps 0-3, one query row per thread): builds the chunk's window
+//     mask as a bit set from the halo geometry (a few operations per x-row of
+//     the halo, not per key), reads S, keeps the online max and sum, writes P
+//     (bf16) over S in TMEM.  A warp whose 32 rows have no key in a chunk only
+//     writes zeros.  For summary chunks the mask is "block box does not meet
+//     the window box"; there is no count bias.  The running max moves only when
+//     a row's maximum grows by more than 8 (log2 units), so O is rescaled in
+//     TMEM rarely; the result is the same softmax.
+//
+// The epilogue divides by the row sum and writes out (packed order) and the
+// natural-log LSE.  Two CTAs share an SM (256 TMEM columns each).  Every wait
+// is bounded; a CTA that gives up sets the timeout bit of the index error word.
 #include <math.h>
 
 #include "pack3d_internal.cuh"
@@ -38,33 +41,38 @@ namespace {
 
 using namespace tc;
 
-constexpr int D = 96;                 // head dim handled by this kernel
-constexpr int KCH = 128;              // keys per chunk (N of the S MMA)
-constexpr int SEG_BYTES = 128 * 64;   // one 32-channel segment of 128 rows
-constexpr int OPND_BYTES = 3 * SEG_BYTES;
+constexpr int D = 96;                  // head dim handled by this kernel
+constexpr int KCH = 64;                // keys per chunk (N of the S MMA)
+constexpr int NSTAGE = 3;              // K/V shared-memory ring depth
+constexpr int QSEG = 128 * 64;         // one 32-channel segment of the 128 query rows
+constexpr int KSEG = KCH * 64;         // one 32-channel segment of a chunk
 constexpr uint32_t TMEM_COLS = 256;
-constexpr uint32_t COL_O = 0;         // O accumulator: columns [0, 96)
-constexpr uint32_t COL_S = 128;       // S / P: columns [128, 256)
-constexpr int NTHREADS = 128;
-constexpr uint32_t WAIT_LIMIT = 1u << 26;
+constexpr uint32_t COL_O = 0;          // O accumulator: columns [0, 96)
+constexpr uint32_t COL_S = 128;        // S/P buffer b: columns [128 + 64 b, 192 + 64 b)
+constexpr int MMA_WARP = 4;
+constexpr int PROD0 = 160;             // first producer thread
+constexpr int NPROD = 128;
+constexpr int NTHREADS = PROD0 + NPROD;
+constexpr uint32_t WAIT_LIMIT = 1u << 24;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 constexpr float RESCALE_THRESHOLD = 8.0f;
 constexpr int ERR_TIMEOUT_BIT = 4;
 
 struct Smem {
-  uint8_t q[OPND_BYTES];     // A of S = Q K^T
-  uint8_t k[OPND_BYTES];     // B of S = Q K^T (K-major)
-  uint8_t v[OPND_BYTES];     // B of O = P V (MN-major)
-  int32_t kz[KCH], ky[KCH], kx[KCH];  // key coordinates (local chunk) or block coordinates
-  uint64_t bar_s, bar_o;
+  uint8_t q[3 * QSEG];
+  uint8_t k[NSTAGE][3 * KSEG];
+  uint8_t v[NSTAGE][3 * KSEG];
+  uint64_t q_full;
+  uint64_t kv_full[NSTAGE];
+  uint64_t kv_empty[NSTAGE];
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t o_done;
   uint32_t tmem_base;
   int32_t abort;
 };
-constexpr size_t SMEM_BYTES = sizeof(Smem) + 1024;  // + alignment slack
-// Request enough shared memory that at most two CTAs share an SM (their TMEM
-// allocations of 256 columns then always fit).
-constexpr size_t SMEM_REQUEST = SMEM_BYTES > 80 * 1024 ? SMEM_BYTES : 80 * 1024;
+constexpr size_t SMEM_REQUEST = sizeof(Smem) + 1024;  // + alignment slack
 
 struct TileBox {
   int z0, y0, x0, lz, ly, lx;
@@ -89,64 +97,99 @@ __device__ __forceinline__ TileBox tile_box(const Geo& g, int t) {
   return tb;
 }
 
-// Load a 96-channel bf16 row (192 bytes) as 12 x 16 bytes.
-__device__ __forceinline__ void load_row(const __nv_bfloat16* src, uint4 (&r)[12]) {
-  const uint4* s = reinterpret_cast<const uint4*>(src);
+// ---- producer helpers --------------------------------------------------------
+
+// Rotate four words of pair members (lo) against their partners (hi): word u of
+// lo holds channels j0 + 2u, j0 + 2u + 1 of a segment, word u of hi the same
+// pairs' second members.  t = rotation table row of the segment's axis.
+__device__ __forceinline__ void rot_chunk(uint4& lo, uint4& hi, const float2* __restrict__ t,
+                                          int j0) {
+  uint32_t* a = reinterpret_cast<uint32_t*>(&lo);
+  uint32_t* b = reinterpret_cast<uint32_t*>(&hi);
 #pragma unroll
-  for (int i = 0; i < 12; ++i) r[i] = __ldg(s + i);
+  for (int u = 0; u < 4; ++u) {
+    float2 x1 = unpack_bf16x2(a[u]), x2 = unpack_bf16x2(b[u]);
+    float2 c0 = __ldg(t + j0 + 2 * u), c1 = __ldg(t + j0 + 2 * u + 1);
+    a[u] = pack_bf16x2(x1.x * c0.x - x2.x * c0.y, x1.y * c1.x - x2.y * c1.y);
+    b[u] = pack_bf16x2(x1.x * c0.y + x2.x * c0.x, x1.y * c1.y + x2.y * c1.x);
+  }
 }
 
-// Axial rotation of a loaded row in place.  Word w of the row holds channels
-// 2w, 2w+1; segment a covers words [16a, 16a + 16); channel j of a segment
-// pairs with j + 16, i.e. word w with word w + 8.
-__device__ __forceinline__ void rotate_row(uint4 (&r)[12], const float2* __restrict__ tab,
-                                           const Geo& g, int cz, int cy, int cx) {
-  uint32_t* w = reinterpret_cast<uint32_t*>(r);
-#pragma unroll
-  for (int a = 0; a < 3; ++a) {
-    int c = a == 0 ? cz : (a == 1 ? cy : cx);
-    int off = a == 0 ? 0 : (a == 1 ? g.Z : g.Z + g.Y);
-    const float2* t = tab + (off + c) * 16;
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      float2 x1 = unpack_bf16x2(w[16 * a + u]);
-      float2 x2 = unpack_bf16x2(w[16 * a + u + 8]);
-      float2 c0 = __ldg(t + 2 * u), c1 = __ldg(t + 2 * u + 1);
-      w[16 * a + u] = pack_bf16x2(x1.x * c0.x - x2.x * c0.y, x1.y * c1.x - x2.y * c1.y);
-      w[16 * a + u + 8] = pack_bf16x2(x1.x * c0.y + x2.x * c0.x, x1.y * c1.y + x2.y * c1.x);
+__device__ __forceinline__ const float2* rope_row(const float2* tab, const Geo& g, int axis,
+                                                  int c) {
+  int off = axis == 0 ? 0 : (axis == 1 ? g.Z : g.Z + g.Y);
+  return tab + (off + c) * 16;
+}
+
+// 16-byte chunk c (0..11) of a 96-channel row -> its place in an operand
+// region (three 32-channel segments of seg_bytes each, 64-byte swizzle).
+__device__ __forceinline__ void store_chunk(uint8_t* region, int seg_bytes, int row, int c,
+                                            const uint4& v) {
+  *reinterpret_cast<uint4*>(region + (c >> 2) * seg_bytes + sw64_off(row, c & 3)) = v;
+}
+
+// ---- softmax helpers -------------------------------------------------------------
+
+// Window mask of 32 consecutive halo keys [e0, e0 + 32) for one query.  The
+// halo is an hz x hy x hx box in raster order; the query's window is
+// |z - qz| <= rz, |y - qy| <= ry, x in [xlo, xhi] (halo-local coordinates).
+// The loop walks the halo x-rows the 32 keys touch (same trip count for every
+// thread); keys at or beyond nh are masked off.
+__device__ __forceinline__ uint32_t local_bits(int e0, int nh, int hx, int hy, int qz, int qy,
+                                               int rz, int ry, int xlo, int xhi) {
+  uint32_t bits = 0;
+  int r = e0 / hx;
+  int z = r / hy, y = r - z * hy;
+  int pos = r * hx - e0;  // bit position of x = 0 of row r (<= 0)
+  while (pos < 32) {
+    if (abs(z - qz) <= rz && abs(y - qy) <= ry) {
+      int lo = max(pos + xlo, 0), hi = min(pos + xhi, 31);
+      if (lo <= hi) bits |= bit_range(lo, hi);
+    }
+    pos += hx;
+    if (++y == hy) {
+      y = 0;
+      ++z;
     }
   }
+  int valid = nh - e0;
+  if (valid < 32) bits &= valid <= 0 ? 0u : (0xffffffffu >> (32 - valid));
+  return bits;
 }
 
-// Store a 96-channel row into an operand region (three 32-channel segments of
-// 128 rows x 64 bytes, 64-byte swizzle).  The same bytes serve as a K-major
-// operand (rows = M or N) and as an MN-major operand (rows = K).
-__device__ __forceinline__ void store_row(uint8_t* region, int row, const uint4 (&r)[12]) {
-#pragma unroll
-  for (int a = 0; a < 3; ++a)
-#pragma unroll
-    for (int c = 0; c < 4; ++c)
-      *reinterpret_cast<uint4*>(region + a * SEG_BYTES + sw64_off(row, c)) = r[4 * a + c];
-}
-
-__device__ __forceinline__ void zero_row(uint4 (&r)[12]) {
-#pragma unroll
-  for (int i = 0; i < 12; ++i) r[i] = make_uint4(0, 0, 0, 0);
-}
-
-__device__ __forceinline__ void fp32_row_to_bf16(const float* __restrict__ src, uint4 (&r)[12]) {
-  const float4* s = reinterpret_cast<const float4*>(src);
-  uint32_t* w = reinterpret_cast<uint32_t*>(r);
-#pragma unroll
-  for (int i = 0; i < 24; ++i) {
-    float4 f = __ldg(s + i);
-    w[2 * i] = pack_bf16x2(f.x, f.y);
-    w[2 * i + 1] = pack_bf16x2(f.z, f.w);
+// Summary mask of 32 consecutive blocks [B0, B0 + 32) (raster order over an
+// nbz x nby x nbx grid): set for blocks that do not meet the query's window,
+// i.e. outside the box [blo, bhi] of blocks the window touches.
+__device__ __forceinline__ uint32_t summary_bits(int B0, int nb, int nbx, int nby, int bzlo,
+                                                 int bzhi, int bylo, int byhi, int bxlo,
+                                                 int bxhi) {
+  uint32_t bits = 0;
+  int r = B0 / nbx;
+  int z = r / nby, y = r - z * nby;
+  int pos = r * nbx - B0;
+  while (pos < 32) {
+    int lo = max(pos, 0), hi = min(pos + nbx - 1, 31);
+    if (lo <= hi) {
+      uint32_t row = bit_range(lo, hi);
+      if (z >= bzlo && z <= bzhi && y >= bylo && y <= byhi) {
+        int elo = max(pos + bxlo, 0), ehi = min(pos + bxhi, 31);
+        if (elo <= ehi) row &= ~bit_range(elo, ehi);
+      }
+      bits |= row;
+    }
+    pos += nbx;
+    if (++y == nby) {
+      y = 0;
+      ++z;
+    }
   }
+  int valid = nb - B0;
+  if (valid < 32) bits &= valid <= 0 ? 0u : (0xffffffffu >> (32 - valid));
+  return bits;
 }
 
 template <bool SUMMARY>
-__global__ void __launch_bounds__(NTHREADS, 2)
+__global__ void __maxnreg__(112)
     k_forward_tc(Geo g, pack3d_index ix, const __nv_bfloat16* __restrict__ q,
                  const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
                  const float* __restrict__ ksum, const float* __restrict__ vsum,
@@ -155,273 +198,378 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                       ~(uintptr_t)1023);
-  const int tid = threadIdx.x, warp = tid / 32;
+  volatile int32_t* abort_flag = &sm.abort;
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int t = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const TileBox tb = tile_box(g, t);
   const int count = tb.lz * tb.ly * tb.lx;
-  const float2* __restrict__ tab = reinterpret_cast<const float2*>(ix.rope);
+  const int nh = tb.hz * tb.hy * tb.hx;
+  const int n_local = (nh + KCH - 1) / KCH;
+  const int n_sum = SUMMARY ? (g.nb + KCH - 1) / KCH : 0;
+  const int nch = n_local + n_sum;
+  const int toff = ix.tile_off[(int64_t)b * (g.nT + 1) + t];
 
   if (tid == 0) {
-    mbar_init(&sm.bar_s, 1);
-    mbar_init(&sm.bar_o, 1);
+    mbar_init(&sm.q_full, NPROD);
+    for (int s = 0; s < NSTAGE; ++s) {
+      mbar_init(&sm.kv_full[s], NPROD);
+      mbar_init(&sm.kv_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.s_full[i], 1);
+      mbar_init(&sm.p_full[i], 128);
+    }
+    mbar_init(&sm.o_done, 1);
     sm.abort = 0;
     fence_barrier_init();
   }
-  if (warp == 0) {
+  if (warp == MMA_WARP) {
     tmem_alloc(&sm.tmem_base, TMEM_COLS);
     tmem_relinquish();
   }
-
-  // ---- query row of this thread: gather, rotate, stage ----
-  const bool active = tid < count;
-  int cz = 0, cy = 0, cx = 0, qi = 0;
-  {
-    uint4 r[12];
-    if (active) {
-      cx = tb.x0 + tid % tb.lx;
-      cy = tb.y0 + (tid / tb.lx) % tb.ly;
-      cz = tb.z0 + tid / (tb.lx * tb.ly);
-      qi = ix.perm[(int64_t)b * g.N + ix.tile_off[(int64_t)b * (g.nT + 1) + t] + tid];
-      load_row(q + (((int64_t)b * g.N + qi) * g.H + h) * D, r);
-      rotate_row(r, tab, g, cz, cy, cx);
-    } else {
-      zero_row(r);
-    }
-    store_row(sm.q, tid, r);
-  }
-  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = sm.tmem_base;
-  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-  const uint32_t tS = tbase + lane_base + COL_S;
-  const uint32_t tO = tbase + lane_base + COL_O;
 
-  // O starts at zero so every PV MMA can accumulate.
-  {
-    uint32_t z[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) z[i] = 0u;
-    tmem_st32(tO + 0, z);
-    tmem_st32(tO + 32, z);
-    tmem_st32(tO + 64, z);
-    tmem_wait_st();
-  }
-
-  const float c2 = g.tau * LOG2E;  // logits -> log2 units
-  float m_run = -INFINITY, l_run = 0.f;
-  uint32_t phase = 0;
-  bool ok = true;
-
-  const int nh = tb.hz * tb.hy * tb.hx;
-  const int n_local = (nh + KCH - 1) / KCH;
-  const int n_sum = SUMMARY ? (g.nb + KCH - 1) / KCH : 0;
-  const int32_t* __restrict__ hl = ix.nbr + (int64_t)b * ix.n_halo + ix.nbr_off[t];
-  const int64_t sbase = ((int64_t)b * g.H + h) * g.nb;
-
-  for (int ch = 0; ch < n_local + n_sum; ++ch) {
-    const bool local = ch < n_local;
-    // ---- stage chunk: thread tid loads key row tid ----
+  if (tid >= PROD0) {
+    // ================= producers =================
+    const int pt = tid - PROD0;
+    const float2* __restrict__ tab = reinterpret_cast<const float2*>(ix.rope);
     {
-      uint4 kr[12], vr[12];
-      if (local) {
-        const int e = ch * KCH + tid;
-        if (e < nh) {
-          int x = tb.hx0 + e % tb.hx, y = tb.hy0 + (e / tb.hx) % tb.hy,
-              z = tb.hz0 + e / (tb.hx * tb.hy);
-          int j = hl[e];
-          int64_t row = (((int64_t)b * g.N + j) * g.H + h) * D;
-          load_row(k + row, kr);
-          load_row(v + row, vr);
-          rotate_row(kr, tab, g, z, y, x);
-          sm.kz[tid] = z;
-          sm.ky[tid] = y;
-          sm.kx[tid] = x;
-        } else {
-          zero_row(kr);
-          zero_row(vr);
-          sm.kz[tid] = -0x40000000;  // never within a window
-          sm.ky[tid] = 0;
-          sm.kx[tid] = 0;
-        }
+      uint4 r[12];
+      if (pt < count) {
+        const int cx = tb.x0 + pt % tb.lx, cy = tb.y0 + (pt / tb.lx) % tb.ly,
+                  cz = tb.z0 + pt / (tb.lx * tb.ly);
+        const int qi = ix.perm[(int64_t)b * g.N + toff + pt];
+        const uint4* src =
+            reinterpret_cast<const uint4*>(q + (((int64_t)b * g.N + qi) * g.H + h) * D);
+#pragma unroll
+        for (int i = 0; i < 12; ++i) r[i] = __ldg(src + i);
+        const float2* tz = rope_row(tab, g, 0, cz);
+        const float2* ty = rope_row(tab, g, 1, cy);
+        const float2* tx = rope_row(tab, g, 2, cx);
+        rot_chunk(r[0], r[2], tz, 0);
+        rot_chunk(r[1], r[3], tz, 8);
+        rot_chunk(r[4], r[6], ty, 0);
+        rot_chunk(r[5], r[7], ty, 8);
+        rot_chunk(r[8], r[10], tx, 0);
+        rot_chunk(r[9], r[11], tx, 8);
       } else {
-        const int B = (ch - n_local) * KCH + tid;
-        if (B < g.nb) {
-          fp32_row_to_bf16(ksum + (sbase + B) * D, kr);
-          fp32_row_to_bf16(vsum + (sbase + B) * D, vr);
-          sm.kz[tid] = B / (g.nby * g.nbx);
-          sm.ky[tid] = (B / g.nbx) % g.nby;
-          sm.kx[tid] = B % g.nbx;
-        } else {
-          zero_row(kr);
-          zero_row(vr);
-          sm.kz[tid] = -1;  // marks padding
-          sm.ky[tid] = 0;
-          sm.kx[tid] = 0;
-        }
+#pragma unroll
+        for (int i = 0; i < 12; ++i) r[i] = make_uint4(0, 0, 0, 0);
       }
-      store_row(sm.k, tid, kr);
-      store_row(sm.v, tid, vr);
+#pragma unroll
+      for (int i = 0; i < 12; ++i) store_chunk(sm.q, QSEG, pt, i, r[i]);
     }
     fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
+    mbar_arrive(&sm.q_full);
 
-    // ---- S = Q K^T ----
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t qa = smem_u32(sm.q), ka = smem_u32(sm.k);
-      constexpr uint32_t idesc = idesc_bf16(128, KCH, false);
+    const int key = pt & (KCH - 1), half = pt / KCH;
+    const int32_t* __restrict__ hl = ix.nbr + (int64_t)b * ix.n_halo + ix.nbr_off[t];
+    const int64_t sbase = ((int64_t)b * g.H + h) * g.nb;
+    // Chunks of the row this thread moves: K chunks {0,1,2,3,4,6} and V chunks
+    // {0..5} for half 0; K chunks {5,7,8,9,10,11} and V chunks {6..11} for
+    // half 1.  The K sets keep every rotation pair (word w with word w + 8 of a
+    // segment) in one thread.
+    for (int j = 0; j < nch; ++j) {
+      const int s = j % NSTAGE, round = j / NSTAGE;
+      if (round > 0 &&
+          !mbar_wait_or_abort(&sm.kv_empty[s], (round - 1) & 1, WAIT_LIMIT, abort_flag))
+        break;
+      uint8_t* kst = sm.k[s];
+      uint8_t* vst = sm.v[s];
+      uint4 kc[6];
+      if (j < n_local) {
+        const int e = j * KCH + key;
+        if (e < nh) {
+          const int x = tb.hx0 + e % tb.hx, y = tb.hy0 + (e / tb.hx) % tb.hy,
+                    z = tb.hz0 + e / (tb.hx * tb.hy);
+          const int idx = hl[e];
+          const int64_t row = (((int64_t)b * g.N + idx) * g.H + h) * D;
+          const uint4* ks = reinterpret_cast<const uint4*>(k + row);
+          const uint4* vs = reinterpret_cast<const uint4*>(v + row);
+          // values need no rotation: copied straight to shared memory
 #pragma unroll
-      for (int s = 0; s < D / 16; ++s) {
-        uint32_t off = (s >> 1) * SEG_BYTES + (s & 1) * 32;
-        mma_ss(tbase + COL_S, sdesc_sw64(qa + off, 16, 512), sdesc_sw64(ka + off, 16, 512),
-               idesc, s > 0);
-      }
-      mma_commit(&sm.bar_s);
-    }
-    if (!mbar_wait(&sm.bar_s, phase, WAIT_LIMIT)) ok = false;
-    tc_fence_after();
-
-    // ---- softmax on this thread's row ----
-    uint32_t mask[4];
-    float cmax = -INFINITY;
-#pragma unroll
-    for (int seg = 0; seg < 4; ++seg) {
-      uint32_t r[32];
-      tmem_ld32(tS + seg * 32, r);
-      tmem_wait_ld();
-      uint32_t mbits = 0;
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int kk = seg * 32 + i;
-        bool in;
-        if (local) {
-          in = abs(sm.kz[kk] - cz) <= g.rz && abs(sm.ky[kk] - cy) <= g.ry &&
-               abs(sm.kx[kk] - cx) <= g.rx;
+          for (int i = 0; i < 6; ++i) {
+            const int c = half * 6 + i;
+            cp_async16(vst + (c >> 2) * KSEG + sw64_off(key, c & 3), vs + c);
+          }
+          if (half == 0) {
+            kc[0] = __ldg(ks + 0);
+            kc[1] = __ldg(ks + 1);
+            kc[2] = __ldg(ks + 2);
+            kc[3] = __ldg(ks + 3);
+            kc[4] = __ldg(ks + 4);
+            kc[5] = __ldg(ks + 6);
+            const float2* tz = rope_row(tab, g, 0, z);
+            const float2* ty = rope_row(tab, g, 1, y);
+            rot_chunk(kc[0], kc[2], tz, 0);
+            rot_chunk(kc[1], kc[3], tz, 8);
+            rot_chunk(kc[4], kc[5], ty, 0);
+          } else {
+            kc[0] = __ldg(ks + 5);
+            kc[1] = __ldg(ks + 7);
+            kc[2] = __ldg(ks + 8);
+            kc[3] = __ldg(ks + 9);
+            kc[4] = __ldg(ks + 10);
+            kc[5] = __ldg(ks + 11);
+            const float2* ty = rope_row(tab, g, 1, y);
+            const float2* tx = rope_row(tab, g, 2, x);
+            rot_chunk(kc[0], kc[1], ty, 8);
+            rot_chunk(kc[2], kc[4], tx, 0);
+            rot_chunk(kc[3], kc[5], tx, 8);
+          }
         } else {
-          int bz0 = sm.kz[kk] * g.bz, by0 = sm.ky[kk] * g.by, bx0 = sm.kx[kk] * g.bx;
-          bool meets = bz0 + g.bz - 1 >= cz - g.rz && bz0 <= cz + g.rz &&
-                       by0 + g.by - 1 >= cy - g.ry && by0 <= cy + g.ry &&
-                       bx0 + g.bx - 1 >= cx - g.rx && bx0 <= cx + g.rx;
-          in = sm.kz[kk] >= 0 && !meets;
+#pragma unroll
+          for (int i = 0; i < 6; ++i) {
+            kc[i] = make_uint4(0, 0, 0, 0);
+            store_chunk(vst, KSEG, key, half * 6 + i, kc[i]);
+          }
         }
-        in = in && active;
-        mbits |= (in ? 1u : 0u) << i;
-        if (in) cmax = fmaxf(cmax, __uint_as_float(r[i]));
+        if (half == 0) {
+          store_chunk(kst, KSEG, key, 0, kc[0]);
+          store_chunk(kst, KSEG, key, 1, kc[1]);
+          store_chunk(kst, KSEG, key, 2, kc[2]);
+          store_chunk(kst, KSEG, key, 3, kc[3]);
+          store_chunk(kst, KSEG, key, 4, kc[4]);
+          store_chunk(kst, KSEG, key, 6, kc[5]);
+        } else {
+          store_chunk(kst, KSEG, key, 5, kc[0]);
+          store_chunk(kst, KSEG, key, 7, kc[1]);
+          store_chunk(kst, KSEG, key, 8, kc[2]);
+          store_chunk(kst, KSEG, key, 9, kc[3]);
+          store_chunk(kst, KSEG, key, 10, kc[4]);
+          store_chunk(kst, KSEG, key, 11, kc[5]);
+        }
+        cp_async_wait_all();
+      } else {
+        const int B = (j - n_local) * KCH + key;
+        // summaries: fp32 rows converted to bf16 (keys already rotated)
+#pragma unroll
+        for (int which = 0; which < 2; ++which) {
+          const float* src = which ? vsum : ksum;
+          uint8_t* dst = which ? vst : kst;
+#pragma unroll
+          for (int i = 0; i < 6; ++i) {
+            uint4 c = make_uint4(0, 0, 0, 0);
+            if (B < g.nb) {
+              const float4* f = reinterpret_cast<const float4*>(src + (sbase + B) * D) + half * 12;
+              float4 a0 = __ldg(f + 2 * i), a1 = __ldg(f + 2 * i + 1);
+              c = make_uint4(pack_bf16x2(a0.x, a0.y), pack_bf16x2(a0.z, a0.w),
+                             pack_bf16x2(a1.x, a1.y), pack_bf16x2(a1.z, a1.w));
+            }
+            store_chunk(dst, KSEG, key, half * 6 + i, c);
+          }
+        }
       }
-      mask[seg] = mbits;
+      fence_proxy_async_smem();
+      mbar_arrive(&sm.kv_full[s]);
     }
-    // Move the running max only when the chunk max exceeds it by the threshold.
-    const float cmax2 = cmax * c2;  // -inf stays -inf
-    bool bump = cmax2 > m_run + RESCALE_THRESHOLD || (m_run == -INFINITY && cmax2 > -INFINITY);
-    float corr = 1.f;
-    if (bump) {
-      corr = m_run == -INFINITY ? 1.f : exp2f(m_run - cmax2);
-      l_run *= corr;
-      m_run = cmax2;
-    }
-    if (__any_sync(0xffffffffu, corr != 1.f)) {
-      // O is not being written: the previous PV MMA completed before this chunk.
+  } else if (warp == MMA_WARP) {
+    // ================= MMA issue =================
+    if (lane == 0) {
+      const uint32_t qa = smem_u32(sm.q);
+      constexpr uint32_t idesc_s = idesc_bf16(128, KCH, false);
+      constexpr uint32_t idesc_o = idesc_bf16(128, D, true);
+      bool ok = mbar_wait_or_abort(&sm.q_full, 0, WAIT_LIMIT, abort_flag);
+      auto issue_s = [&](int j) -> bool {
+        const int s = j % NSTAGE;
+        if (!mbar_wait_or_abort(&sm.kv_full[s], (j / NSTAGE) & 1, WAIT_LIMIT, abort_flag))
+          return false;
+        tc_fence_after();
+        const uint32_t ka = smem_u32(sm.k[s]);
+        const uint32_t dst = tbase + COL_S + 64 * (j & 1);
 #pragma unroll
-      for (int part = 0; part < 3; ++part) {
-        uint32_t r[32];
-        tmem_ld32(tO + part * 32, r);
-        tmem_wait_ld();
+        for (int st = 0; st < D / 16; ++st) {
+          const uint32_t sub = (st & 1) * 32;
+          mma_ss(dst, sdesc_sw64(qa + (st >> 1) * QSEG + sub, 16, 512),
+                 sdesc_sw64(ka + (st >> 1) * KSEG + sub, 16, 512), idesc_s, st > 0);
+        }
+        mma_commit(&sm.s_full[j & 1]);
+        return true;
+      };
+      if (ok) {
+        tc_fence_after();
+        for (int j = 0; j < nch && j < 2 && ok; ++j) ok = issue_s(j);
+      }
+      for (int j = 0; j < nch && ok; ++j) {
+        if (!mbar_wait_or_abort(&sm.p_full[j & 1], (j >> 1) & 1, WAIT_LIMIT, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t va = smem_u32(sm.v[j % NSTAGE]);
+        const uint32_t pa = tbase + COL_S + 64 * (j & 1);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * corr);
-        tmem_st32(tO + part * 32, r);
+        for (int st = 0; st < KCH / 16; ++st)
+          mma_ts(tbase + COL_O, pa + 8 * st, sdesc_sw64(va + st * 16 * 64, KSEG, 512), idesc_o,
+                 (j > 0 || st > 0) ? 1u : 0u);
+        mma_commit(&sm.o_done);
+        mma_commit(&sm.kv_empty[j % NSTAGE]);
+        if (j + 2 < nch) {
+          // S buffer j & 1 holds P_j until this PV has read it
+          if (!mbar_wait_or_abort(&sm.o_done, j & 1, WAIT_LIMIT, abort_flag)) break;
+          ok = issue_s(j + 2);
+        }
       }
     }
-    const float mneg = m_run == -INFINITY ? 0.f : -m_run;
-#pragma unroll
-    for (int seg = 0; seg < 4; ++seg) {
-      uint32_t r[32];
-      tmem_ld32(tS + seg * 32, r);
-      tmem_wait_ld();
-      uint32_t p[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        bool in0 = (mask[seg] >> (2 * i)) & 1u, in1 = (mask[seg] >> (2 * i + 1)) & 1u;
-        float p0 = in0 ? exp2f(fmaf(__uint_as_float(r[2 * i]), c2, mneg)) : 0.f;
-        float p1 = in1 ? exp2f(fmaf(__uint_as_float(r[2 * i + 1]), c2, mneg)) : 0.f;
-        l_run += p0 + p1;
-        p[i] = pack_bf16x2(p0, p1);
-      }
-      // P for keys [32 seg, 32 seg + 32) goes to columns [16 seg, 16 seg + 16)
-      // of the S region, which hold S values already read.
-      tmem_st16(tS + seg * 16, p);
+    __syncwarp();
+  } else {
+    // ================= softmax (one query row per thread) =================
+    const bool active = tid < count;
+    int cz = 0, cy = 0, cx = 0, qi = 0;
+    if (active) {
+      cx = tb.x0 + tid % tb.lx;
+      cy = tb.y0 + (tid / tb.lx) % tb.ly;
+      cz = tb.z0 + tid / (tb.lx * tb.ly);
+      qi = ix.perm[(int64_t)b * g.N + toff + tid];
     }
-    tmem_wait_st();
-    tc_fence_before();
-    __syncthreads();
-
-    // ---- O += P V ----
-    if (tid == 0) {
+    const int qz = cz - tb.hz0, qy = cy - tb.hy0, qx = cx - tb.hx0;
+    const int xlo = max(qx - g.rx, 0), xhi = min(qx + g.rx, tb.hx - 1);
+    const int bzlo = max(cz - g.rz, 0) / g.bz, bzhi = min(cz + g.rz, g.Z - 1) / g.bz;
+    const int bylo = max(cy - g.ry, 0) / g.by, byhi = min(cy + g.ry, g.Y - 1) / g.by;
+    const int bxlo = max(cx - g.rx, 0) / g.bx, bxhi = min(cx + g.rx, g.X - 1) / g.bx;
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const uint32_t tO = tbase + lane_base + COL_O;
+    const float c2 = g.tau * LOG2E;  // logits -> log2 units
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nch; ++j) {
+      const int buf = j & 1;
+      // a warp leaves together: the TMEM accesses below are warp-collective
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait_or_abort(&sm.s_full[buf], (j >> 1) & 1, WAIT_LIMIT, abort_flag));
+      if (!ok) break;
       tc_fence_after();
-      const uint32_t va = smem_u32(sm.v);
-      constexpr uint32_t idesc = idesc_bf16(128, D, true);
-#pragma unroll
-      for (int s = 0; s < KCH / 16; ++s) {
-        mma_ts(tbase + COL_O, tbase + COL_S + s * 8,
-               sdesc_sw64(va + s * 16 * 64, SEG_BYTES, 512), idesc, 1);
+      const uint32_t tS = tbase + lane_base + COL_S + 64 * buf;
+      uint32_t bits0, bits1;
+      if (j < n_local) {
+        bits0 = local_bits(j * KCH, nh, tb.hx, tb.hy, qz, qy, g.rz, g.ry, xlo, xhi);
+        bits1 = local_bits(j * KCH + 32, nh, tb.hx, tb.hy, qz, qy, g.rz, g.ry, xlo, xhi);
+      } else {
+        const int B0 = (j - n_local) * KCH;
+        bits0 = summary_bits(B0, g.nb, g.nbx, g.nby, bzlo, bzhi, bylo, byhi, bxlo, bxhi);
+        bits1 = summary_bits(B0 + 32, g.nb, g.nbx, g.nby, bzlo, bzhi, bylo, byhi, bxlo, bxhi);
       }
-      mma_commit(&sm.bar_o);
+      if (!active) bits0 = bits1 = 0u;
+      if (__ballot_sync(0xffffffffu, (bits0 | bits1) != 0u) == 0u) {
+        uint32_t z[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) z[i] = 0u;
+        tmem_st16(tS, z);
+        tmem_st16(tS + 16, z);
+      } else {
+        // pass 1: masked row maximum over the 64 keys
+        float cmax = -INFINITY;
+        {
+          uint32_t sv[32];
+          tmem_ld32(tS, sv);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if ((bits0 >> i) & 1u) cmax = fmaxf(cmax, __uint_as_float(sv[i]));
+          tmem_ld32(tS + 32, sv);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if ((bits1 >> i) & 1u) cmax = fmaxf(cmax, __uint_as_float(sv[i]));
+        }
+        const float cmax2 = cmax * c2;
+        float corr = 1.f;
+        if (cmax2 > m_run + RESCALE_THRESHOLD) {
+          if (m_run != -INFINITY) corr = ex2(m_run - cmax2);
+          l_run *= corr;
+          m_run = cmax2;
+        }
+        if (__any_sync(0xffffffffu, corr != 1.f)) {
+          // O must hold every earlier PV product before it is rescaled
+          ok = __all_sync(0xffffffffu,
+                          mbar_wait_or_abort(&sm.o_done, (j - 1) & 1, WAIT_LIMIT, abort_flag));
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll 1
+          for (int part = 0; part < 3; ++part) {
+            uint32_t o[32];
+            tmem_ld32(tO + part * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * corr);
+            tmem_st32(tO + part * 32, o);
+          }
+        }
+        const float mneg = m_run == -INFINITY ? 0.f : -m_run;
+        // pass 2: P over S; keys 0-31 -> columns 0-15, keys 32-63 -> columns
+        // 16-31 (columns whose S values have been read by then)
+#pragma unroll 1
+        for (int seg = 0; seg < 2; ++seg) {
+          const uint32_t bits = seg ? bits1 : bits0;
+          uint32_t sv[32], p[16];
+          tmem_ld32(tS + 32 * seg, sv);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float a0 = ((bits >> (2 * i)) & 1u) ? fmaf(__uint_as_float(sv[2 * i]), c2, mneg) : -INFINITY;
+            float a1 = ((bits >> (2 * i + 1)) & 1u) ? fmaf(__uint_as_float(sv[2 * i + 1]), c2, mneg) : -INFINITY;
+            float e0 = ex2(a0), e1 = ex2(a1);
+            l_run += e0 + e1;
+            p[i] = pack_bf16x2(e0, e1);
+          }
+          tmem_st16(tS + 16 * seg, p);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&sm.p_full[buf]);
     }
-    if (!mbar_wait(&sm.bar_o, phase, WAIT_LIMIT)) ok = false;
-    tc_fence_after();
-    phase ^= 1;
-    if (!ok) sm.abort = 1;
-    __syncthreads();
-    if (sm.abort) break;
-  }
-
-  // ---- epilogue ----
-  if (!sm.abort) {
-    const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-    const int64_t orow_off = (((int64_t)b * g.N + qi) * g.H + h) * D;
-    if (!g.out_fp32) {
-      uint4 orow[12];
-      uint32_t* ow = reinterpret_cast<uint32_t*>(orow);
+    // ---- epilogue ----
+    // Wait for the last two PV products in order (a wait names a phase by its
+    // parity, so it must not run ahead of the barrier by two phases).
+    if (ok && nch >= 2)
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait_or_abort(&sm.o_done, (nch - 2) & 1, WAIT_LIMIT, abort_flag));
+    if (ok)
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait_or_abort(&sm.o_done, (nch - 1) & 1, WAIT_LIMIT, abort_flag));
+    if (ok) {
+      tc_fence_after();
+      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      const int64_t orow = (((int64_t)b * g.N + qi) * g.H + h) * D;
 #pragma unroll
       for (int part = 0; part < 3; ++part) {
-        uint32_t r[32];
-        tmem_ld32(tO + part * 32, r);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          ow[part * 16 + i] =
-              pack_bf16x2(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
-      }
-      if (active) {
-        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(out_raw) + orow_off);
-#pragma unroll
-        for (int i = 0; i < 12; ++i) dst[i] = orow[i];
-      }
-    } else {
-      float* dstf = reinterpret_cast<float*>(out_raw) + orow_off;
-#pragma unroll
-      for (int part = 0; part < 3; ++part) {
-        uint32_t r[32];
-        tmem_ld32(tO + part * 32, r);
+        uint32_t o[32];
+        tmem_ld32(tO + part * 32, o);
         tmem_wait_ld();
         if (active) {
+          if (g.out_fp32) {
+            float4* dst =
+                reinterpret_cast<float4*>(reinterpret_cast<float*>(out_raw) + orow + part * 32);
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            reinterpret_cast<float4*>(dstf + part * 32)[i] = make_float4(
-                __uint_as_float(r[4 * i]) * inv, __uint_as_float(r[4 * i + 1]) * inv,
-                __uint_as_float(r[4 * i + 2]) * inv, __uint_as_float(r[4 * i + 3]) * inv);
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(
+                  __uint_as_float(o[4 * i]) * inv, __uint_as_float(o[4 * i + 1]) * inv,
+                  __uint_as_float(o[4 * i + 2]) * inv, __uint_as_float(o[4 * i + 3]) * inv);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(out_raw) +
+                                                  orow + part * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_uint4(
+                  pack_bf16x2(__uint_as_float(o[8 * i]) * inv, __uint_as_float(o[8 * i + 1]) * inv),
+                  pack_bf16x2(__uint_as_float(o[8 * i + 2]) * inv,
+                              __uint_as_float(o[8 * i + 3]) * inv),
+                  pack_bf16x2(__uint_as_float(o[8 * i + 4]) * inv,
+                              __uint_as_float(o[8 * i + 5]) * inv),
+                  pack_bf16x2(__uint_as_float(o[8 * i + 6]) * inv,
+                              __uint_as_float(o[8 * i + 7]) * inv));
+          }
         }
       }
+      if (active) lse[((int64_t)b * g.H + h) * g.N + qi] = (m_run + log2f(l_run)) * LN2;
     }
-    if (active) lse[((int64_t)b * g.H + h) * g.N + qi] = (m_run + log2f(l_run)) * LN2;
-  } else if (tid == 0) {
-    atomicOr(&ix.err[0], ERR_TIMEOUT_BIT);
   }
+
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (sm.abort && tid == 0) atomicOr(&ix.err[0], ERR_TIMEOUT_BIT);
+  if (warp == MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tbase, TMEM_COLS);
   }

@@ -19,10 +19,10 @@ def to_cuda(inp):
             for k, v in inp.items()}
 
 
-def gpu_run(wl, inp, window_only=False, with_backward=False):
+def gpu_run(wl, inp, window_only=False, with_backward=False, out_fp32=False):
     """Index, summaries, forward (and backward) on the GPU; CPU tensors back."""
     d = to_cuda(inp)
-    params = P.make_params(wl)
+    params = P.make_params(wl, out_fp32=out_fp32)
     idx = P.pack3d_build_index(params, d["coords"])
     st = P.pack3d_index_check(idx)
     assert st == P.OK, P.strerror(st)
