@@ -20,7 +20,8 @@ OK, ERR_ARG, ERR_COORDS, ERR_CUDA, ERR_TIMEOUT, ERR_UNSUPPORTED = 0, -1, -2, -3,
 
 EXPORTS = ("pack3d_index_bytes", "pack3d_index_init", "pack3d_build_index", "pack3d_index_check",
            "pack3d_block_summaries", "pack3d_forward", "pack3d_window_forward",
-           "pack3d_backward_workspace_bytes", "pack3d_backward", "pack3d_strerror")
+           "pack3d_backward_workspace_bytes", "pack3d_backward", "pack3d_backward_noalloc",
+           "pack3d_strerror")
 
 
 class Params(ctypes.Structure):
@@ -75,6 +76,8 @@ def load(build_if_missing: bool = True):
         lib.pack3d_backward_workspace_bytes.restype = ctypes.c_size_t
         lib.pack3d_backward.argtypes = [P(Params), P(Index), vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                         vp, ctypes.c_size_t, vp]
+        lib.pack3d_backward_noalloc.argtypes = [P(Params), P(Index), vp, vp, vp, vp, vp, vp, vp,
+                                                vp, vp, vp]
         lib.pack3d_strerror.argtypes = [ctypes.c_int]
         lib.pack3d_strerror.restype = ctypes.c_char_p
         for name in EXPORTS:
@@ -250,6 +253,27 @@ def pack3d_backward(params: Params, index: IndexBuffers, q, k, v, out, lse, dout
                                   _ptr(dk), _ptr(dv), _ptr(workspace),
                                   ctypes.c_size_t(workspace.numel() * workspace.element_size()),
                                   _stream(stream)), "pack3d_backward")
+    return dq, dk, dv
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def pack3d_backward_noalloc(params: Params, index: IndexBuffers, q, k, v, out, lse, dout,
+                            dq=None, dk=None, dv=None, stream=None):
+    """pack3d_backward without a workspace argument: the library's static
+    device scratch array (NOALLOC_SCRATCH_BYTES) stands in for it.  Calls that
+    overlap on the GPU share that array and race; the first call on a device
+    looks the array up and should precede any stream capture."""
+    _need_cuda(q, k, v, out, lse, dout)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _need_cuda(dq, dk, dv)
+    _check(load().pack3d_backward_noalloc(ctypes.byref(params), ctypes.byref(index.struct),
+                                          _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                                          _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+                                          _stream(stream)), "pack3d_backward_noalloc")
     return dq, dk, dv
 
 
