@@ -8,12 +8,13 @@
 // (batch item, head).  The tile's halo (the union of its windows, raster order)
 // and then the block summaries are streamed in chunks of 64 keys.  Roles:
 //
-//   * producers (warps 5-8): gather the query rows once and each chunk's key
-//     and value rows through the index, rotate queries and keys in registers
-//     (axial RoPE, fp32 arithmetic), and store them in the 64-byte-swizzled
-//     operand layout of a 3-stage shared-memory ring.  head_dim 96 is three
-//     32-channel segments, one per axis, so a rotation segment is exactly one
-//     swizzle-atom column.  Summary chunks are converted from fp32 instead;
+//   * producers (warps 5-6, one key per thread): gather the query rows once
+//     (rotated in registers) and each chunk's key and value rows through the
+//     index with cp.async, one chunk ahead, into the 64-byte-swizzled operand
+//     layout of a 3-stage shared-memory ring; once a chunk has landed its key
+//     rows are rotated in place (axial RoPE, fp32 arithmetic).  head_dim 96 is
+//     three 32-channel segments, one per axis, so a rotation segment is exactly
+//     one swizzle-atom column.  Summary chunks are converted from fp32 instead;
 //   * MMA (warp 4, one thread): S_j = Q K_j^T (six tcgen05.mma, K = 16) into
 //     one of two TMEM S buffers, and O += P_j V_j (four tcgen05.mma, A = P from
 //     TMEM, B = V MN-major in shared memory), so S_{j+1} is computed while the
@@ -51,9 +52,9 @@ constexpr uint32_t COL_O = 0;          // O accumulator: columns [0, 96)
 constexpr uint32_t COL_S = 128;        // S/P buffer b: columns [128 + 64 b, 192 + 64 b)
 constexpr int MMA_WARP = 4;
 constexpr int PROD0 = 160;             // first producer thread
-constexpr int NPROD = 128;
+constexpr int NPROD = KCH;             // one producer thread per key of a chunk
 constexpr int NTHREADS = PROD0 + NPROD;
-constexpr uint32_t WAIT_LIMIT = 1u << 24;
+constexpr uint32_t WAIT_LIMIT = 1u << 20;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 constexpr float RESCALE_THRESHOLD = 8.0f;
@@ -68,7 +69,8 @@ struct Smem {
   uint64_t kv_empty[NSTAGE];
   uint64_t s_full[2];
   uint64_t p_full[2];
-  uint64_t o_done;
+  uint64_t o_done;   // one phase per PV product
+  uint64_t o_final;  // one phase: every PV product of the tile is done
   uint32_t tmem_base;
   int32_t abort;
 };
@@ -121,11 +123,29 @@ __device__ __forceinline__ const float2* rope_row(const float2* tab, const Geo& 
   return tab + (off + c) * 16;
 }
 
-// 16-byte chunk c (0..11) of a 96-channel row -> its place in an operand
+// Axial rotation of a whole 96-channel row held as 12 chunks: segment a is
+// chunks 4a..4a+3, and word w of a segment pairs with word w + 8.
+__device__ __forceinline__ void rotate_row(uint4 (&r)[12], const float2* __restrict__ tab,
+                                           const Geo& g, int cz, int cy, int cx) {
+  const float2* tz = rope_row(tab, g, 0, cz);
+  const float2* ty = rope_row(tab, g, 1, cy);
+  const float2* tx = rope_row(tab, g, 2, cx);
+  rot_chunk(r[0], r[2], tz, 0);
+  rot_chunk(r[1], r[3], tz, 8);
+  rot_chunk(r[4], r[6], ty, 0);
+  rot_chunk(r[5], r[7], ty, 8);
+  rot_chunk(r[8], r[10], tx, 0);
+  rot_chunk(r[9], r[11], tx, 8);
+}
+
+// 16-byte chunk c (0..11) of a 96-channel row <-> its place in an operand
 // region (three 32-channel segments of seg_bytes each, 64-byte swizzle).
 __device__ __forceinline__ void store_chunk(uint8_t* region, int seg_bytes, int row, int c,
                                             const uint4& v) {
   *reinterpret_cast<uint4*>(region + (c >> 2) * seg_bytes + sw64_off(row, c & 3)) = v;
+}
+__device__ __forceinline__ uint4 load_chunk(const uint8_t* region, int seg_bytes, int row, int c) {
+  return *reinterpret_cast<const uint4*>(region + (c >> 2) * seg_bytes + sw64_off(row, c & 3));
 }
 
 // ---- softmax helpers -------------------------------------------------------------
@@ -189,7 +209,7 @@ __device__ __forceinline__ uint32_t summary_bits(int B0, int nb, int nbx, int nb
 }
 
 template <bool SUMMARY>
-__global__ void __maxnreg__(112)
+__global__ void __launch_bounds__(NTHREADS, 2)
     k_forward_tc(Geo g, pack3d_index ix, const __nv_bfloat16* __restrict__ q,
                  const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
                  const float* __restrict__ ksum, const float* __restrict__ vsum,
@@ -220,6 +240,7 @@ __global__ void __maxnreg__(112)
       mbar_init(&sm.p_full[i], 128);
     }
     mbar_init(&sm.o_done, 1);
+    mbar_init(&sm.o_final, 1);
     sm.abort = 0;
     fence_barrier_init();
   }
@@ -233,139 +254,110 @@ __global__ void __maxnreg__(112)
   const uint32_t tbase = sm.tmem_base;
 
   if (tid >= PROD0) {
-    // ================= producers =================
+    // ================= producers (one key row of each chunk per thread) =================
     const int pt = tid - PROD0;
     const float2* __restrict__ tab = reinterpret_cast<const float2*>(ix.rope);
-    {
+    // queries: rows pt and pt + 64, gathered, rotated, stored once
+    for (int qr = pt; qr < 128; qr += NPROD) {
       uint4 r[12];
-      if (pt < count) {
-        const int cx = tb.x0 + pt % tb.lx, cy = tb.y0 + (pt / tb.lx) % tb.ly,
-                  cz = tb.z0 + pt / (tb.lx * tb.ly);
-        const int qi = ix.perm[(int64_t)b * g.N + toff + pt];
+      if (qr < count) {
+        const int cx = tb.x0 + qr % tb.lx, cy = tb.y0 + (qr / tb.lx) % tb.ly,
+                  cz = tb.z0 + qr / (tb.lx * tb.ly);
+        const int qi = ix.perm[(int64_t)b * g.N + toff + qr];
         const uint4* src =
             reinterpret_cast<const uint4*>(q + (((int64_t)b * g.N + qi) * g.H + h) * D);
 #pragma unroll
         for (int i = 0; i < 12; ++i) r[i] = __ldg(src + i);
-        const float2* tz = rope_row(tab, g, 0, cz);
-        const float2* ty = rope_row(tab, g, 1, cy);
-        const float2* tx = rope_row(tab, g, 2, cx);
-        rot_chunk(r[0], r[2], tz, 0);
-        rot_chunk(r[1], r[3], tz, 8);
-        rot_chunk(r[4], r[6], ty, 0);
-        rot_chunk(r[5], r[7], ty, 8);
-        rot_chunk(r[8], r[10], tx, 0);
-        rot_chunk(r[9], r[11], tx, 8);
+        rotate_row(r, tab, g, cz, cy, cx);
       } else {
 #pragma unroll
         for (int i = 0; i < 12; ++i) r[i] = make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
-      for (int i = 0; i < 12; ++i) store_chunk(sm.q, QSEG, pt, i, r[i]);
+      for (int i = 0; i < 12; ++i) store_chunk(sm.q, QSEG, qr, i, r[i]);
     }
     fence_proxy_async_smem();
     mbar_arrive(&sm.q_full);
 
-    const int key = pt & (KCH - 1), half = pt / KCH;
+    const int key = pt;
     const int32_t* __restrict__ hl = ix.nbr + (int64_t)b * ix.n_halo + ix.nbr_off[t];
     const int64_t sbase = ((int64_t)b * g.H + h) * g.nb;
-    // Chunks of the row this thread moves: K chunks {0,1,2,3,4,6} and V chunks
-    // {0..5} for half 0; K chunks {5,7,8,9,10,11} and V chunks {6..11} for
-    // half 1.  The K sets keep every rotation pair (word w with word w + 8 of a
-    // segment) in one thread.
-    for (int j = 0; j < nch; ++j) {
+    // Local chunks: the raw key and value rows are copied asynchronously into
+    // the chunk's stage one chunk ahead; once they have landed the key row is
+    // rotated in place.  Returns false if a wait gave up.
+    auto issue = [&](int j) -> bool {
       const int s = j % NSTAGE, round = j / NSTAGE;
       if (round > 0 &&
           !mbar_wait_or_abort(&sm.kv_empty[s], (round - 1) & 1, WAIT_LIMIT, abort_flag))
-        break;
-      uint8_t* kst = sm.k[s];
-      uint8_t* vst = sm.v[s];
-      uint4 kc[6];
+        return false;
+      if (j < n_local) {
+        const int e = j * KCH + key;
+        if (e < nh) {
+          const int64_t row = (((int64_t)b * g.N + hl[e]) * g.H + h) * D;
+          const uint4* ks = reinterpret_cast<const uint4*>(k + row);
+          const uint4* vs = reinterpret_cast<const uint4*>(v + row);
+#pragma unroll
+          for (int c = 0; c < 12; ++c) {
+            cp_async16(sm.k[s] + (c >> 2) * KSEG + sw64_off(key, c & 3), ks + c);
+            cp_async16(sm.v[s] + (c >> 2) * KSEG + sw64_off(key, c & 3), vs + c);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 12; ++c) {
+            store_chunk(sm.k[s], KSEG, key, c, make_uint4(0, 0, 0, 0));
+            store_chunk(sm.v[s], KSEG, key, c, make_uint4(0, 0, 0, 0));
+          }
+        }
+      }
+      cp_async_commit();
+      return true;
+    };
+    bool ok = issue(0);
+    for (int j = 0; j < nch && ok; ++j) {
+      const int s = j % NSTAGE;
+      if (j + 1 < nch) {
+        ok = issue(j + 1);
+        if (!ok) break;
+        cp_async_wait_group<1>();
+      } else {
+        cp_async_wait_group<0>();
+      }
       if (j < n_local) {
         const int e = j * KCH + key;
         if (e < nh) {
           const int x = tb.hx0 + e % tb.hx, y = tb.hy0 + (e / tb.hx) % tb.hy,
                     z = tb.hz0 + e / (tb.hx * tb.hy);
-          const int idx = hl[e];
-          const int64_t row = (((int64_t)b * g.N + idx) * g.H + h) * D;
-          const uint4* ks = reinterpret_cast<const uint4*>(k + row);
-          const uint4* vs = reinterpret_cast<const uint4*>(v + row);
-          // values need no rotation: copied straight to shared memory
+          uint4 r[12];
 #pragma unroll
-          for (int i = 0; i < 6; ++i) {
-            const int c = half * 6 + i;
-            cp_async16(vst + (c >> 2) * KSEG + sw64_off(key, c & 3), vs + c);
-          }
-          if (half == 0) {
-            kc[0] = __ldg(ks + 0);
-            kc[1] = __ldg(ks + 1);
-            kc[2] = __ldg(ks + 2);
-            kc[3] = __ldg(ks + 3);
-            kc[4] = __ldg(ks + 4);
-            kc[5] = __ldg(ks + 6);
-            const float2* tz = rope_row(tab, g, 0, z);
-            const float2* ty = rope_row(tab, g, 1, y);
-            rot_chunk(kc[0], kc[2], tz, 0);
-            rot_chunk(kc[1], kc[3], tz, 8);
-            rot_chunk(kc[4], kc[5], ty, 0);
-          } else {
-            kc[0] = __ldg(ks + 5);
-            kc[1] = __ldg(ks + 7);
-            kc[2] = __ldg(ks + 8);
-            kc[3] = __ldg(ks + 9);
-            kc[4] = __ldg(ks + 10);
-            kc[5] = __ldg(ks + 11);
-            const float2* ty = rope_row(tab, g, 1, y);
-            const float2* tx = rope_row(tab, g, 2, x);
-            rot_chunk(kc[0], kc[1], ty, 8);
-            rot_chunk(kc[2], kc[4], tx, 0);
-            rot_chunk(kc[3], kc[5], tx, 8);
-          }
-        } else {
+          for (int c = 0; c < 12; ++c) r[c] = load_chunk(sm.k[s], KSEG, key, c);
+          rotate_row(r, tab, g, z, y, x);
 #pragma unroll
-          for (int i = 0; i < 6; ++i) {
-            kc[i] = make_uint4(0, 0, 0, 0);
-            store_chunk(vst, KSEG, key, half * 6 + i, kc[i]);
-          }
+          for (int c = 0; c < 12; ++c) store_chunk(sm.k[s], KSEG, key, c, r[c]);
         }
-        if (half == 0) {
-          store_chunk(kst, KSEG, key, 0, kc[0]);
-          store_chunk(kst, KSEG, key, 1, kc[1]);
-          store_chunk(kst, KSEG, key, 2, kc[2]);
-          store_chunk(kst, KSEG, key, 3, kc[3]);
-          store_chunk(kst, KSEG, key, 4, kc[4]);
-          store_chunk(kst, KSEG, key, 6, kc[5]);
-        } else {
-          store_chunk(kst, KSEG, key, 5, kc[0]);
-          store_chunk(kst, KSEG, key, 7, kc[1]);
-          store_chunk(kst, KSEG, key, 8, kc[2]);
-          store_chunk(kst, KSEG, key, 9, kc[3]);
-          store_chunk(kst, KSEG, key, 10, kc[4]);
-          store_chunk(kst, KSEG, key, 11, kc[5]);
-        }
-        cp_async_wait_all();
       } else {
-        const int B = (j - n_local) * KCH + key;
         // summaries: fp32 rows converted to bf16 (keys already rotated)
+        const int B = (j - n_local) * KCH + key;
 #pragma unroll
         for (int which = 0; which < 2; ++which) {
           const float* src = which ? vsum : ksum;
-          uint8_t* dst = which ? vst : kst;
-#pragma unroll
-          for (int i = 0; i < 6; ++i) {
-            uint4 c = make_uint4(0, 0, 0, 0);
+          uint8_t* dst = which ? sm.v[s] : sm.k[s];
+#pragma unroll 4
+          for (int c = 0; c < 12; ++c) {
+            uint4 w = make_uint4(0, 0, 0, 0);
             if (B < g.nb) {
-              const float4* f = reinterpret_cast<const float4*>(src + (sbase + B) * D) + half * 12;
-              float4 a0 = __ldg(f + 2 * i), a1 = __ldg(f + 2 * i + 1);
-              c = make_uint4(pack_bf16x2(a0.x, a0.y), pack_bf16x2(a0.z, a0.w),
+              const float4* f = reinterpret_cast<const float4*>(src + (sbase + B) * D);
+              float4 a0 = __ldg(f + 2 * c), a1 = __ldg(f + 2 * c + 1);
+              w = make_uint4(pack_bf16x2(a0.x, a0.y), pack_bf16x2(a0.z, a0.w),
                              pack_bf16x2(a1.x, a1.y), pack_bf16x2(a1.z, a1.w));
             }
-            store_chunk(dst, KSEG, key, half * 6 + i, c);
+            store_chunk(dst, KSEG, key, c, w);
           }
         }
       }
       fence_proxy_async_smem();
       mbar_arrive(&sm.kv_full[s]);
     }
+    cp_async_wait_group<0>();
   } else if (warp == MMA_WARP) {
     // ================= MMA issue =================
     if (lane == 0) {
@@ -404,6 +396,7 @@ __global__ void __maxnreg__(112)
                  (j > 0 || st > 0) ? 1u : 0u);
         mma_commit(&sm.o_done);
         mma_commit(&sm.kv_empty[j % NSTAGE]);
+        if (j == nch - 1) mma_commit(&sm.o_final);
         if (j + 2 < nch) {
           // S buffer j & 1 holds P_j until this PV has read it
           if (!mbar_wait_or_abort(&sm.o_done, j & 1, WAIT_LIMIT, abort_flag)) break;
@@ -520,14 +513,11 @@ __global__ void __maxnreg__(112)
       mbar_arrive(&sm.p_full[buf]);
     }
     // ---- epilogue ----
-    // Wait for the last two PV products in order (a wait names a phase by its
-    // parity, so it must not run ahead of the barrier by two phases).
-    if (ok && nch >= 2)
-      ok = __all_sync(0xffffffffu,
-                      mbar_wait_or_abort(&sm.o_done, (nch - 2) & 1, WAIT_LIMIT, abort_flag));
+    // o_final completes once, after the last PV product.  (Waiting on o_done
+    // here could name a phase by a parity the barrier has already passed twice:
+    // a wait must never trail the barrier by two phases.)
     if (ok)
-      ok = __all_sync(0xffffffffu,
-                      mbar_wait_or_abort(&sm.o_done, (nch - 1) & 1, WAIT_LIMIT, abort_flag));
+      ok = __all_sync(0xffffffffu, mbar_wait_or_abort(&sm.o_final, 0, WAIT_LIMIT, abort_flag));
     if (ok) {
       tc_fence_after();
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
@@ -584,9 +574,12 @@ int launch_forward_tc(const Geo& g, const pack3d_index* idx, const void* q, cons
                       bool summaries, cudaStream_t s) {
   dim3 grid(g.nT, g.H, g.B);
   auto kern = summaries ? k_forward_tc<true> : k_forward_tc<false>;
-  cudaError_t e =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_REQUEST);
-  if (e != cudaSuccess) return PACK3D_ERR_CUDA;
+  // Two CTAs per SM: enough shared memory for both, and the largest carveout.
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)SMEM_REQUEST) != cudaSuccess ||
+      cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+    return PACK3D_ERR_CUDA;
   kern<<<grid, NTHREADS, SMEM_REQUEST, s>>>(g, *idx, (const __nv_bfloat16*)q,
                                              (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
                                              ksum, vsum, out, lse);

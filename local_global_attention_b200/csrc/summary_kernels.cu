@@ -7,12 +7,13 @@
 // R(c_j) k_j, not R(.) of a mean.
 //
 // HBM-bound: every k and v row is read once.  One CTA per (block, batch item,
-// head); its threads form TG token groups of d/4 lanes, each lane owning two
-// adjacent rotation pairs (four output channels).  A lane reads 2 x 4 bytes of
-// k (the pair members sit da/2 channels apart) and 2 x 4 bytes of v per token;
-// the d/4 lanes of a token group read one 2d-byte row contiguously.  Tokens
-// are visited through the coordinate volume in block raster order, so the
-// accumulation order, and the result, do not depend on the packing.
+// head).  In the general kernel the threads form TG token groups of d/4 lanes,
+// each lane owning two adjacent rotation pairs (four output channels): a lane
+// reads 2 x 4 bytes of k (the pair members sit da/2 channels apart) and 2 x 4
+// bytes of v per token, and the d/4 lanes of a token group read one 2d-byte
+// row contiguously.  The bf16 head_dim-96 kernel reads 16-byte chunks instead.
+// Tokens are visited through the coordinate volume in block raster order, so
+// the accumulation order, and the result, do not depend on the packing.
 #include "pack3d_internal.cuh"
 
 namespace p3d {
@@ -100,11 +101,86 @@ __global__ void __launch_bounds__(256) k_block_summaries(Geo g, const int32_t* _
   }
 }
 
+// bf16, head_dim 96: 16-byte loads.  Six lanes cover a 192-byte row; lane u
+// owns chunk c1 = 4 (u / 2) + u % 2 and its rotation partner c2 = c1 + 2
+// (segment u / 2, pairs 8 (u % 2) .. 8 (u % 2) + 7), for both k and v.
+// 32 token groups per CTA; the partial sums are combined in a fixed order.
+constexpr int TG96 = 32;
+
+__global__ void __launch_bounds__(TG96 * 6) k_block_summaries_bf16_d96(
+    Geo g, const int32_t* __restrict__ vol, const float* __restrict__ rope,
+    const int32_t* __restrict__ err, const __nv_bfloat16* __restrict__ k,
+    const __nv_bfloat16* __restrict__ v, float* ksum, float* vsum) {
+  if (err[0]) return;
+  __shared__ float red[TG96][2][96];
+  const int u = threadIdx.x % 6, grp = threadIdx.x / 6;
+  const int blk = blockIdx.x, b = blockIdx.y, h = blockIdx.z;
+  const int Bz = blk / (g.nby * g.nbx), By = (blk / g.nbx) % g.nby, Bx = blk % g.nbx;
+  const int a = u / 2, c1 = 4 * a + (u & 1), c2 = c1 + 2, j0 = 8 * (u & 1);
+  const int axis_off = a == 0 ? 0 : (a == 1 ? g.Z : g.Z + g.Y);
+  const float2* __restrict__ tab = reinterpret_cast<const float2*>(rope);
+  float kx1[8], kx2[8], vx1[8], vx2[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) kx1[i] = kx2[i] = vx1[i] = vx2[i] = 0.f;
+  const int cnt = g.bz * g.by * g.bx;
+  const int32_t* vb = vol + (int64_t)b * g.N;
+#pragma unroll 2
+  for (int e = grp; e < cnt; e += TG96) {
+    const int x = e % g.bx, y = (e / g.bx) % g.by, z = e / (g.bx * g.by);
+    const int cz = Bz * g.bz + z, cy = By * g.by + y, cx = Bx * g.bx + x;
+    const int tok = vb[(cz * g.Y + cy) * g.X + cx];
+    const uint4* kr = reinterpret_cast<const uint4*>(k + (((int64_t)b * g.N + tok) * g.H + h) * 96);
+    const uint4* vr = reinterpret_cast<const uint4*>(v + (((int64_t)b * g.N + tok) * g.H + h) * 96);
+    const uint4 ka = __ldg(kr + c1), kb = __ldg(kr + c2), va = __ldg(vr + c1), vb2 = __ldg(vr + c2);
+    const int ca = a == 0 ? cz : (a == 1 ? cy : cx);
+    const float2* t = tab + (axis_off + ca) * 16 + j0;
+    const uint32_t* kaw = reinterpret_cast<const uint32_t*>(&ka);
+    const uint32_t* kbw = reinterpret_cast<const uint32_t*>(&kb);
+    const uint32_t* vaw = reinterpret_cast<const uint32_t*>(&va);
+    const uint32_t* vbw = reinterpret_cast<const uint32_t*>(&vb2);
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      float2 x1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(kaw + w));
+      float2 x2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(kbw + w));
+      float2 cs0 = __ldg(t + 2 * w), cs1 = __ldg(t + 2 * w + 1);
+      kx1[2 * w] += x1.x * cs0.x - x2.x * cs0.y;
+      kx2[2 * w] += x1.x * cs0.y + x2.x * cs0.x;
+      kx1[2 * w + 1] += x1.y * cs1.x - x2.y * cs1.y;
+      kx2[2 * w + 1] += x1.y * cs1.y + x2.y * cs1.x;
+      float2 y1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(vaw + w));
+      float2 y2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(vbw + w));
+      vx1[2 * w] += y1.x;
+      vx1[2 * w + 1] += y1.y;
+      vx2[2 * w] += y2.x;
+      vx2[2 * w + 1] += y2.y;
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    red[grp][0][8 * c1 + i] = kx1[i];
+    red[grp][0][8 * c2 + i] = kx2[i];
+    red[grp][1][8 * c1 + i] = vx1[i];
+    red[grp][1][8 * c2 + i] = vx2[i];
+  }
+  __syncthreads();
+  const int which = threadIdx.x / 96, ch = threadIdx.x % 96;
+  float acc = 0.f;
+  for (int q = 0; q < TG96; ++q) acc += red[q][which][ch];
+  const int64_t o = (((int64_t)b * g.H + h) * g.nb + blk) * 96 + ch;
+  (which ? vsum : ksum)[o] = acc / (float)cnt;
+}
+
 }  // namespace
 
 int launch_block_summaries(const Geo& g, const pack3d_index* idx, const void* k, const void* v,
                            float* ksum, float* vsum, cudaStream_t s) {
   dim3 grid(g.nb, g.B, g.H);
+  if (g.dtype == PACK3D_BF16 && g.d == 96) {
+    k_block_summaries_bf16_d96<<<grid, TG96 * 6, 0, s>>>(g, idx->vol, idx->rope, idx->err,
+                                                          (const __nv_bfloat16*)k,
+                                                          (const __nv_bfloat16*)v, ksum, vsum);
+    return cuda_status(cudaGetLastError());
+  }
   int threads = TG * (g.d / 4);
   size_t smem = sizeof(float) * TG * 2 * g.d;
   if (g.dtype == PACK3D_BF16)
