@@ -8,25 +8,27 @@
 // (batch item, head).  The tile's halo (the union of its windows, raster order)
 // and then the block summaries are streamed in chunks of 64 keys.  Roles:
 //
-//   * producers (warps 5-6, one key per thread): gather the query rows once
-//     (rotated in registers) and each chunk's key and value rows through the
-//     index with cp.async, one chunk ahead, into the 64-byte-swizzled operand
-//     layout of a 3-stage shared-memory ring; once a chunk has landed its key
-//     rows are rotated in place (axial RoPE, fp32 arithmetic).  head_dim 96 is
-//     three 32-channel segments, one per axis, so a rotation segment is exactly
-//     one swizzle-atom column.  Summary chunks are converted from fp32 instead;
+//   * producers (warps 5-6, one key per thread): copy each chunk's key and
+//     value rows through the index with cp.async, two chunks ahead, into the
+//     64-byte-swizzled operand layout of a 3-stage shared-memory ring, and
+//     rotate a chunk's key rows in place once they have landed (axial RoPE, fp32 arithmetic, the
+//     rotation-table rows of the tile's halo staged in shared memory), or
+//     convert summary rows from fp32.  head_dim 96 is three 32-channel
+//     segments, one per axis, so a rotation segment is exactly one swizzle-atom
+//     column;
 //   * MMA (warp 4, one thread): S_j = Q K_j^T (six tcgen05.mma, K = 16) into
 //     one of two TMEM S buffers, and O += P_j V_j (four tcgen05.mma, A = P from
 //     TMEM, B = V MN-major in shared memory), so S_{j+1} is computed while the
 //     softmax works on S_j;
-//   * softmax (warps 0-3, one query row per thread): builds the chunk's window
-//     mask as a bit set from the halo geometry (a few operations per x-row of
-//     the halo, not per key), reads S, keeps the online max and sum, writes P
-//     (bf16) over S in TMEM.  A warp whose 32 rows have no key in a chunk only
-//     writes zeros.  For summary chunks the mask is "block box does not meet
-//     the window box"; there is no count bias.  The running max moves only when
-//     a row's maximum grows by more than 8 (log2 units), so O is rescaled in
-//     TMEM rarely; the result is the same softmax.
+//   * softmax warps (0-3, one query row per thread): gather and rotate the
+//     query rows once; per chunk build the window mask as a bit set from the
+//     halo geometry (a few operations per halo x-row, walked with a cursor, not
+//     per key), read S, keep the online max and sum, write P (bf16) over S in
+//     TMEM.  A warp whose 32 rows have no key in a chunk only writes zeros.
+//     For summary chunks the mask is "block box does not meet the window box";
+//     there is no count bias.  The running max moves only when a row's maximum
+//     grows by more than 8 (log2 units), so O is rescaled in TMEM rarely; the
+//     result is the same softmax.
 //
 // The epilogue divides by the row sum and writes out (packed order) and the
 // natural-log LSE.  Two CTAs share an SM (256 TMEM columns each).  Every wait
@@ -59,11 +61,15 @@ constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 constexpr float RESCALE_THRESHOLD = 8.0f;
 constexpr int ERR_TIMEOUT_BIT = 4;
+constexpr int TAB_ROWS = 64;           // rotation-table rows staged in shared memory
+constexpr int TAB_STRIDE = 18;         // float2 per staged row: 16 + 2 of padding, so rows
+                                       // of consecutive coordinates start on different banks
 
 struct Smem {
   uint8_t q[3 * QSEG];
   uint8_t k[NSTAGE][3 * KSEG];
   uint8_t v[NSTAGE][3 * KSEG];
+  float2 tab[TAB_ROWS * TAB_STRIDE];  // rotation-table rows of the halo box
   uint64_t q_full;
   uint64_t kv_full[NSTAGE];
   uint64_t kv_empty[NSTAGE];
@@ -99,37 +105,44 @@ __device__ __forceinline__ TileBox tile_box(const Geo& g, int t) {
   return tb;
 }
 
-// ---- producer helpers --------------------------------------------------------
+// ---- rotation ------------------------------------------------------------------
 
 // Rotate four words of pair members (lo) against their partners (hi): word u of
 // lo holds channels j0 + 2u, j0 + 2u + 1 of a segment, word u of hi the same
-// pairs' second members.  t = rotation table row of the segment's axis.
-__device__ __forceinline__ void rot_chunk(uint4& lo, uint4& hi, const float2* __restrict__ t,
-                                          int j0) {
+// pairs' second members.  t = rotation-table row of the segment's axis.
+__device__ __forceinline__ void rot_chunk(uint4& lo, uint4& hi, const float2* t, int j0) {
   uint32_t* a = reinterpret_cast<uint32_t*>(&lo);
   uint32_t* b = reinterpret_cast<uint32_t*>(&hi);
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
     float2 x1 = unpack_bf16x2(a[u]), x2 = unpack_bf16x2(b[u]);
-    float2 c0 = __ldg(t + j0 + 2 * u), c1 = __ldg(t + j0 + 2 * u + 1);
-    a[u] = pack_bf16x2(x1.x * c0.x - x2.x * c0.y, x1.y * c1.x - x2.y * c1.y);
-    b[u] = pack_bf16x2(x1.x * c0.y + x2.x * c0.x, x1.y * c1.y + x2.y * c1.x);
+    const float4 cs = *reinterpret_cast<const float4*>(t + j0 + 2 * u);  // pairs j, j + 1
+    a[u] = pack_bf16x2(x1.x * cs.x - x2.x * cs.y, x1.y * cs.z - x2.y * cs.w);
+    b[u] = pack_bf16x2(x1.x * cs.y + x2.x * cs.x, x1.y * cs.w + x2.y * cs.z);
   }
 }
 
-__device__ __forceinline__ const float2* rope_row(const float2* tab, const Geo& g, int axis,
-                                                  int c) {
-  int off = axis == 0 ? 0 : (axis == 1 ? g.Z : g.Z + g.Y);
-  return tab + (off + c) * 16;
-}
+// Rows of the rotation table (16 (cos, sin) pairs per coordinate value) for the
+// coordinates a tile can touch: its halo box, staged in shared memory when they
+// fit (z rows, then y rows, then x rows), else read from the global table.
+struct RopeRows {
+  const float2* z;  // row of coordinate c is z + (c - bz) * stride
+  const float2* y;
+  const float2* x;
+  int bz, by, bx, stride;
+  __device__ __forceinline__ const float2* row(int axis, int c) const {
+    return axis == 0 ? z + (c - bz) * stride
+                     : (axis == 1 ? y + (c - by) * stride : x + (c - bx) * stride);
+  }
+};
 
 // Axial rotation of a whole 96-channel row held as 12 chunks: segment a is
 // chunks 4a..4a+3, and word w of a segment pairs with word w + 8.
-__device__ __forceinline__ void rotate_row(uint4 (&r)[12], const float2* __restrict__ tab,
-                                           const Geo& g, int cz, int cy, int cx) {
-  const float2* tz = rope_row(tab, g, 0, cz);
-  const float2* ty = rope_row(tab, g, 1, cy);
-  const float2* tx = rope_row(tab, g, 2, cx);
+__device__ __forceinline__ void rotate_row(uint4 (&r)[12], const RopeRows& rr, int cz, int cy,
+                                           int cx) {
+  const float2* tz = rr.row(0, cz);
+  const float2* ty = rr.row(1, cy);
+  const float2* tx = rr.row(2, cx);
   rot_chunk(r[0], r[2], tz, 0);
   rot_chunk(r[1], r[3], tz, 8);
   rot_chunk(r[4], r[6], ty, 0);
@@ -148,22 +161,37 @@ __device__ __forceinline__ uint4 load_chunk(const uint8_t* region, int seg_bytes
   return *reinterpret_cast<const uint4*>(region + (c >> 2) * seg_bytes + sw64_off(row, c & 3));
 }
 
-// ---- softmax helpers -------------------------------------------------------------
+// ---- masks ---------------------------------------------------------------------
 
-// Window mask of 32 consecutive halo keys [e0, e0 + 32) for one query.  The
-// halo is an hz x hy x hx box in raster order; the query's window is
-// |z - qz| <= rz, |y - qy| <= ry, x in [xlo, xhi] (halo-local coordinates).
-// The loop walks the halo x-rows the 32 keys touch (same trip count for every
-// thread); keys at or beyond nh are masked off.
-__device__ __forceinline__ uint32_t local_bits(int e0, int nh, int hx, int hy, int qz, int qy,
-                                               int rz, int ry, int xlo, int xhi) {
+// Walks the rows of a raster-ordered box (rows of `len` items, `ny` rows per
+// plane) in step with 32-item segments, so no division is needed per segment.
+struct RowCursor {
+  int start;  // index of the first item of the current row
+  int z, y;   // the current row's plane and row within the plane
+  int row;    // the current row's raster index (z * ny + y)
+  __device__ __forceinline__ void advance_to(int e, int len, int ny) {
+    while (start + len <= e) {
+      start += len;
+      ++row;
+      if (++y == ny) {
+        y = 0;
+        ++z;
+      }
+    }
+  }
+};
+
+// Window mask of the 32 halo keys [e0, e0 + 32) for one query: the halo is an
+// hz x hy x hx box in raster order and the window is |z - qz| <= rz,
+// |y - qy| <= ry, x in [xlo, xhi] (halo-local).  `c` is at the row holding e0.
+__device__ __forceinline__ uint32_t local_bits(RowCursor c, int e0, int nh, int hx, int hy, int qz,
+                                               int qy, int rz, int ry, int xlo, int xhi) {
   uint32_t bits = 0;
-  int r = e0 / hx;
-  int z = r / hy, y = r - z * hy;
-  int pos = r * hx - e0;  // bit position of x = 0 of row r (<= 0)
+  int pos = c.start - e0;  // bit of x = 0 of the current row (<= 0)
+  int z = c.z, y = c.y;
   while (pos < 32) {
     if (abs(z - qz) <= rz && abs(y - qy) <= ry) {
-      int lo = max(pos + xlo, 0), hi = min(pos + xhi, 31);
+      const int lo = max(pos + xlo, 0), hi = min(pos + xhi, 31);
       if (lo <= hi) bits |= bit_range(lo, hi);
     }
     pos += hx;
@@ -172,27 +200,26 @@ __device__ __forceinline__ uint32_t local_bits(int e0, int nh, int hx, int hy, i
       ++z;
     }
   }
-  int valid = nh - e0;
+  const int valid = nh - e0;
   if (valid < 32) bits &= valid <= 0 ? 0u : (0xffffffffu >> (32 - valid));
   return bits;
 }
 
-// Summary mask of 32 consecutive blocks [B0, B0 + 32) (raster order over an
-// nbz x nby x nbx grid): set for blocks that do not meet the query's window,
-// i.e. outside the box [blo, bhi] of blocks the window touches.
-__device__ __forceinline__ uint32_t summary_bits(int B0, int nb, int nbx, int nby, int bzlo,
-                                                 int bzhi, int bylo, int byhi, int bxlo,
+// Summary mask of the 32 blocks [B0, B0 + 32) (raster order over an
+// nbz x nby x nbx grid): set for blocks outside the box [blo, bhi] of blocks
+// the query's window touches.  `c` is at the block row holding B0.
+__device__ __forceinline__ uint32_t summary_bits(RowCursor c, int B0, int nb, int nbx, int nby,
+                                                 int bzlo, int bzhi, int bylo, int byhi, int bxlo,
                                                  int bxhi) {
   uint32_t bits = 0;
-  int r = B0 / nbx;
-  int z = r / nby, y = r - z * nby;
-  int pos = r * nbx - B0;
+  int pos = c.start - B0;
+  int z = c.z, y = c.y;
   while (pos < 32) {
-    int lo = max(pos, 0), hi = min(pos + nbx - 1, 31);
+    const int lo = max(pos, 0), hi = min(pos + nbx - 1, 31);
     if (lo <= hi) {
       uint32_t row = bit_range(lo, hi);
       if (z >= bzlo && z <= bzhi && y >= bylo && y <= byhi) {
-        int elo = max(pos + bxlo, 0), ehi = min(pos + bxhi, 31);
+        const int elo = max(pos + bxlo, 0), ehi = min(pos + bxhi, 31);
         if (elo <= ehi) row &= ~bit_range(elo, ehi);
       }
       bits |= row;
@@ -203,9 +230,72 @@ __device__ __forceinline__ uint32_t summary_bits(int B0, int nb, int nbx, int nb
       ++z;
     }
   }
-  int valid = nb - B0;
+  const int valid = nb - B0;
   if (valid < 32) bits &= valid <= 0 ? 0u : (0xffffffffu >> (32 - valid));
   return bits;
+}
+
+// Precomputed form of the masks above for boxes whose rows fit 128 bits and
+// whose rows are at most 32 items long: `rows` has bit r set for the rows r
+// (raster over z, y) the mask keeps or drops as a whole, and `pattern` is the
+// per-row item mask repeated with period `len` over 64 bits.  For the 32 items
+// [e0, e0 + 32), with the cursor at the row holding e0, the result is
+// (row bit AND pattern bit) per item - a handful of bit operations, no
+// data-dependent branches.
+struct RowMask {
+  uint32_t rows[4];
+  uint64_t pattern;
+  __device__ __forceinline__ uint32_t row_bit(int r) const {
+    const int w = r >> 5;
+    const uint32_t word = w == 0 ? rows[0] : (w == 1 ? rows[1] : (w == 2 ? rows[2] : rows[3]));
+    return (word >> (r & 31)) & 1u;
+  }
+  // items of [e0, e0 + 32) whose row bit and pattern bit are both set
+  __device__ __forceinline__ uint32_t segment(const RowCursor& c, int e0, int len) const {
+    const int off = e0 - c.start;          // position of e0 inside its row
+    const int r0 = c.row;                  // index of the row holding e0
+    const uint32_t xb = (uint32_t)(pattern >> off);
+    uint32_t rb = 0;
+    for (int k = 0, lo = -off; lo < 32; ++k, lo += len) {
+      const uint32_t m = bit_range(max(lo, 0), min(lo + len - 1, 31));
+      rb |= row_bit(r0 + k) ? m : 0u;
+    }
+    return rb & xb;
+  }
+};
+
+__device__ __forceinline__ uint64_t periodic(uint32_t m, int len) {
+  uint64_t p = m;
+  for (int s = len; s < 64; s += len) p |= (uint64_t)m << s;
+  return p;
+}
+
+// P = 2^(S c2 + mneg) for the keys in `bits`, 0 elsewhere; returns the sum.
+__device__ __forceinline__ float exp_pack(const uint32_t (&sv)[32], uint32_t bits, float c2,
+                                          float mneg, uint32_t (&p)[16]) {
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float a0 = ((bits >> (2 * i)) & 1u) ? fmaf(__uint_as_float(sv[2 * i]), c2, mneg)
+                                              : -INFINITY;
+    const float a1 = ((bits >> (2 * i + 1)) & 1u) ? fmaf(__uint_as_float(sv[2 * i + 1]), c2, mneg)
+                                                  : -INFINITY;
+    const float e0 = ex2(a0), e1 = ex2(a1);
+    acc[i & 3] += e0 + e1;
+    p[i] = pack_bf16x2(e0, e1);
+  }
+  return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
+
+// Maximum of S over the keys in `bits` (-inf if none), with independent chains.
+__device__ __forceinline__ float masked_max(const uint32_t (&sv)[32], uint32_t bits) {
+  float m[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) m[i] = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < 32; ++i)
+    if ((bits >> i) & 1u) m[i & 3] = fmaxf(m[i & 3], __uint_as_float(sv[i]));
+  return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
 }
 
 template <bool SUMMARY>
@@ -230,7 +320,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   const int toff = ix.tile_off[(int64_t)b * (g.nT + 1) + t];
 
   if (tid == 0) {
-    mbar_init(&sm.q_full, NPROD);
+    mbar_init(&sm.q_full, 128);
     for (int s = 0; s < NSTAGE; ++s) {
       mbar_init(&sm.kv_full[s], NPROD);
       mbar_init(&sm.kv_empty[s], 1);
@@ -248,6 +338,35 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     tmem_alloc(&sm.tmem_base, TMEM_COLS);
     tmem_relinquish();
   }
+  // rotation-table rows of the halo box (all threads stage; producers and
+  // softmax warps read)
+  RopeRows rr;
+  {
+    const float2* gt = reinterpret_cast<const float2*>(ix.rope);
+    const int rows = tb.hz + tb.hy + tb.hx;
+    if (rows <= TAB_ROWS) {
+      for (int e = tid; e < rows * 16; e += NTHREADS) {
+        const int r = e / 16, jj = e % 16;
+        const int grow = r < tb.hz ? tb.hz0 + r
+                                   : (r < tb.hz + tb.hy ? g.Z + tb.hy0 + r - tb.hz
+                                                        : g.Z + g.Y + tb.hx0 + r - tb.hz - tb.hy);
+        sm.tab[r * TAB_STRIDE + jj] = gt[grow * 16 + jj];
+      }
+      rr.z = sm.tab;
+      rr.y = sm.tab + tb.hz * TAB_STRIDE;
+      rr.x = sm.tab + (tb.hz + tb.hy) * TAB_STRIDE;
+      rr.bz = tb.hz0;
+      rr.by = tb.hy0;
+      rr.bx = tb.hx0;
+      rr.stride = TAB_STRIDE;
+    } else {
+      rr.z = gt;
+      rr.y = gt + g.Z * 16;
+      rr.x = gt + (g.Z + g.Y) * 16;
+      rr.bz = rr.by = rr.bx = 0;
+      rr.stride = 16;
+    }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -255,45 +374,26 @@ __global__ void __launch_bounds__(NTHREADS, 2)
 
   if (tid >= PROD0) {
     // ================= producers (one key row of each chunk per thread) =================
-    const int pt = tid - PROD0;
-    const float2* __restrict__ tab = reinterpret_cast<const float2*>(ix.rope);
-    // queries: rows pt and pt + 64, gathered, rotated, stored once
-    for (int qr = pt; qr < 128; qr += NPROD) {
-      uint4 r[12];
-      if (qr < count) {
-        const int cx = tb.x0 + qr % tb.lx, cy = tb.y0 + (qr / tb.lx) % tb.ly,
-                  cz = tb.z0 + qr / (tb.lx * tb.ly);
-        const int qi = ix.perm[(int64_t)b * g.N + toff + qr];
-        const uint4* src =
-            reinterpret_cast<const uint4*>(q + (((int64_t)b * g.N + qi) * g.H + h) * D);
-#pragma unroll
-        for (int i = 0; i < 12; ++i) r[i] = __ldg(src + i);
-        rotate_row(r, tab, g, cz, cy, cx);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 12; ++i) r[i] = make_uint4(0, 0, 0, 0);
-      }
-#pragma unroll
-      for (int i = 0; i < 12; ++i) store_chunk(sm.q, QSEG, qr, i, r[i]);
-    }
-    fence_proxy_async_smem();
-    mbar_arrive(&sm.q_full);
-
-    const int key = pt;
+    const int key = tid - PROD0;
     const int32_t* __restrict__ hl = ix.nbr + (int64_t)b * ix.n_halo + ix.nbr_off[t];
     const int64_t sbase = ((int64_t)b * g.H + h) * g.nb;
-    // Local chunks: the raw key and value rows are copied asynchronously into
-    // the chunk's stage one chunk ahead; once they have landed the key row is
-    // rotated in place.  Returns false if a wait gave up.
+    int next_row = (key < nh) ? hl[key] : 0;  // neighbour index of the next chunk to issue
+    // Copy chunk j's raw key and value rows into its stage (zero rows past the
+    // halo); one cp.async group per chunk.  False if a wait gave up.
     auto issue = [&](int j) -> bool {
       const int s = j % NSTAGE, round = j / NSTAGE;
+      const int row_idx = next_row;
+      if (j + 1 < n_local) {
+        const int en = (j + 1) * KCH + key;
+        next_row = en < nh ? hl[en] : 0;
+      }
       if (round > 0 &&
           !mbar_wait_or_abort(&sm.kv_empty[s], (round - 1) & 1, WAIT_LIMIT, abort_flag))
         return false;
       if (j < n_local) {
         const int e = j * KCH + key;
         if (e < nh) {
-          const int64_t row = (((int64_t)b * g.N + hl[e]) * g.H + h) * D;
+          const int64_t row = (((int64_t)b * g.N + row_idx) * g.H + h) * D;
           const uint4* ks = reinterpret_cast<const uint4*>(k + row);
           const uint4* vs = reinterpret_cast<const uint4*>(v + row);
 #pragma unroll
@@ -304,35 +404,44 @@ __global__ void __launch_bounds__(NTHREADS, 2)
         } else {
 #pragma unroll
           for (int c = 0; c < 12; ++c) {
-            store_chunk(sm.k[s], KSEG, key, c, make_uint4(0, 0, 0, 0));
-            store_chunk(sm.v[s], KSEG, key, c, make_uint4(0, 0, 0, 0));
+            cp_async16_zero(sm.k[s] + (c >> 2) * KSEG + sw64_off(key, c & 3), k);
+            cp_async16_zero(sm.v[s] + (c >> 2) * KSEG + sw64_off(key, c & 3), v);
           }
         }
       }
       cp_async_commit();
       return true;
     };
+    // Two chunks in flight: chunk j + 2 is issued after chunk j has been
+    // rotated (issuing it first would wait on chunk j - 1's PV product, which
+    // the MMA thread issues only after S_j, i.e. after this rotation).
     bool ok = issue(0);
+    if (ok && nch > 1) ok = issue(1);
+    // the halo-local coordinate of this thread's key in chunk j, advanced
+    // without division
+    int kx = key % tb.hx, ky = (key / tb.hx) % tb.hy, kz = key / (tb.hx * tb.hy);
     for (int j = 0; j < nch && ok; ++j) {
       const int s = j % NSTAGE;
-      if (j + 1 < nch) {
-        ok = issue(j + 1);
-        if (!ok) break;
-        cp_async_wait_group<1>();
-      } else {
+      if (j + 1 < nch)
+        cp_async_wait_group<1>();  // chunk j + 1 may still be in flight
+      else
         cp_async_wait_group<0>();
-      }
       if (j < n_local) {
-        const int e = j * KCH + key;
-        if (e < nh) {
-          const int x = tb.hx0 + e % tb.hx, y = tb.hy0 + (e / tb.hx) % tb.hy,
-                    z = tb.hz0 + e / (tb.hx * tb.hy);
+        if (j * KCH + key < nh) {
           uint4 r[12];
 #pragma unroll
           for (int c = 0; c < 12; ++c) r[c] = load_chunk(sm.k[s], KSEG, key, c);
-          rotate_row(r, tab, g, z, y, x);
+          rotate_row(r, rr, tb.hz0 + kz, tb.hy0 + ky, tb.hx0 + kx);
 #pragma unroll
           for (int c = 0; c < 12; ++c) store_chunk(sm.k[s], KSEG, key, c, r[c]);
+        }
+        kx += KCH;
+        while (kx >= tb.hx) {
+          kx -= tb.hx;
+          if (++ky == tb.hy) {
+            ky = 0;
+            ++kz;
+          }
         }
       } else {
         // summaries: fp32 rows converted to bf16 (keys already rotated)
@@ -346,7 +455,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
             uint4 w = make_uint4(0, 0, 0, 0);
             if (B < g.nb) {
               const float4* f = reinterpret_cast<const float4*>(src + (sbase + B) * D);
-              float4 a0 = __ldg(f + 2 * c), a1 = __ldg(f + 2 * c + 1);
+              const float4 a0 = __ldg(f + 2 * c), a1 = __ldg(f + 2 * c + 1);
               w = make_uint4(pack_bf16x2(a0.x, a0.y), pack_bf16x2(a0.z, a0.w),
                              pack_bf16x2(a1.x, a1.y), pack_bf16x2(a1.z, a1.w));
             }
@@ -356,6 +465,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       }
       fence_proxy_async_smem();
       mbar_arrive(&sm.kv_full[s]);
+      if (j + 2 < nch) ok = issue(j + 2);
     }
     cp_async_wait_group<0>();
   } else if (warp == MMA_WARP) {
@@ -406,7 +516,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     }
     __syncwarp();
   } else {
-    // ================= softmax (one query row per thread) =================
+    // ================= softmax warps (one query row per thread) =================
     const bool active = tid < count;
     int cz = 0, cy = 0, cx = 0, qi = 0;
     if (active) {
@@ -415,15 +525,50 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       cz = tb.z0 + tid / (tb.lx * tb.ly);
       qi = ix.perm[(int64_t)b * g.N + toff + tid];
     }
+    {
+      // this thread's query row: gathered, rotated, stored once
+      uint4 r[12];
+      if (active) {
+        const uint4* src =
+            reinterpret_cast<const uint4*>(q + (((int64_t)b * g.N + qi) * g.H + h) * D);
+#pragma unroll
+        for (int i = 0; i < 12; ++i) r[i] = __ldg(src + i);
+        rotate_row(r, rr, cz, cy, cx);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 12; ++i) r[i] = make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int i = 0; i < 12; ++i) store_chunk(sm.q, QSEG, tid, i, r[i]);
+      fence_proxy_async_smem();
+      mbar_arrive(&sm.q_full);
+    }
     const int qz = cz - tb.hz0, qy = cy - tb.hy0, qx = cx - tb.hx0;
     const int xlo = max(qx - g.rx, 0), xhi = min(qx + g.rx, tb.hx - 1);
-    const int bzlo = max(cz - g.rz, 0) / g.bz, bzhi = min(cz + g.rz, g.Z - 1) / g.bz;
-    const int bylo = max(cy - g.ry, 0) / g.by, byhi = min(cy + g.ry, g.Y - 1) / g.by;
-    const int bxlo = max(cx - g.rx, 0) / g.bx, bxhi = min(cx + g.rx, g.X - 1) / g.bx;
+    // Precomputed window mask (halo rows in the window; x range as a periodic
+    // pattern) when the halo's rows fit, else the per-row walk.
+    const bool fast_local = tb.hz * tb.hy <= 128 && tb.hx <= 32;
+    RowMask lm;
+    if (fast_local) {
+      lm.rows[0] = lm.rows[1] = lm.rows[2] = lm.rows[3] = 0u;
+      const int ylo = max(qy - g.ry, 0), yhi = min(qy + g.ry, tb.hy - 1);
+      for (int z = max(qz - g.rz, 0); z <= min(qz + g.rz, tb.hz - 1); ++z) {
+        // rows z * hy + [ylo, yhi] of plane z, spread over the four words
+        const int a = z * tb.hy + ylo, e = z * tb.hy + yhi;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const int lo = max(a - 32 * w, 0), hi = min(e - 32 * w, 31);
+          if (lo <= hi) lm.rows[w] |= bit_range(lo, hi);
+        }
+      }
+      lm.pattern = periodic(bit_range(xlo, xhi), tb.hx);
+    }
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     const uint32_t tO = tbase + lane_base + COL_O;
     const float c2 = g.tau * LOG2E;  // logits -> log2 units
     float m_run = -INFINITY, l_run = 0.f;
+    RowCursor hc = {0, 0, 0, 0};  // halo rows (hx keys each, hy rows per plane)
+    RowCursor bc = {0, 0, 0, 0};  // block rows (nbx blocks each, nby rows per plane)
     bool ok = true;
     for (int j = 0; j < nch; ++j) {
       const int buf = j & 1;
@@ -435,12 +580,32 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       const uint32_t tS = tbase + lane_base + COL_S + 64 * buf;
       uint32_t bits0, bits1;
       if (j < n_local) {
-        bits0 = local_bits(j * KCH, nh, tb.hx, tb.hy, qz, qy, g.rz, g.ry, xlo, xhi);
-        bits1 = local_bits(j * KCH + 32, nh, tb.hx, tb.hy, qz, qy, g.rz, g.ry, xlo, xhi);
+        const int e0 = j * KCH;
+        hc.advance_to(e0, tb.hx, tb.hy);
+        if (fast_local) {
+          bits0 = lm.segment(hc, e0, tb.hx);
+          hc.advance_to(e0 + 32, tb.hx, tb.hy);
+          bits1 = lm.segment(hc, e0 + 32, tb.hx);
+          const int valid = nh - e0;  // keys past the halo
+          if (valid < 64) {
+            bits0 &= valid <= 0 ? 0u : (valid >= 32 ? 0xffffffffu : (0xffffffffu >> (32 - valid)));
+            bits1 &= valid <= 32 ? 0u : (0xffffffffu >> (64 - valid));
+          }
+        } else {
+          bits0 = local_bits(hc, e0, nh, tb.hx, tb.hy, qz, qy, g.rz, g.ry, xlo, xhi);
+          hc.advance_to(e0 + 32, tb.hx, tb.hy);
+          bits1 = local_bits(hc, e0 + 32, nh, tb.hx, tb.hy, qz, qy, g.rz, g.ry, xlo, xhi);
+        }
       } else {
         const int B0 = (j - n_local) * KCH;
-        bits0 = summary_bits(B0, g.nb, g.nbx, g.nby, bzlo, bzhi, bylo, byhi, bxlo, bxhi);
-        bits1 = summary_bits(B0 + 32, g.nb, g.nbx, g.nby, bzlo, bzhi, bylo, byhi, bxlo, bxhi);
+        // the box of blocks this query's window touches
+        const int bzlo = max(cz - g.rz, 0) / g.bz, bzhi = min(cz + g.rz, g.Z - 1) / g.bz;
+        const int bylo = max(cy - g.ry, 0) / g.by, byhi = min(cy + g.ry, g.Y - 1) / g.by;
+        const int bxlo = max(cx - g.rx, 0) / g.bx, bxhi = min(cx + g.rx, g.X - 1) / g.bx;
+        bc.advance_to(B0, g.nbx, g.nby);
+        bits0 = summary_bits(bc, B0, g.nb, g.nbx, g.nby, bzlo, bzhi, bylo, byhi, bxlo, bxhi);
+        bc.advance_to(B0 + 32, g.nbx, g.nby);
+        bits1 = summary_bits(bc, B0 + 32, g.nb, g.nbx, g.nby, bzlo, bzhi, bylo, byhi, bxlo, bxhi);
       }
       if (!active) bits0 = bits1 = 0u;
       if (__ballot_sync(0xffffffffu, (bits0 | bits1) != 0u) == 0u) {
@@ -450,20 +615,16 @@ __global__ void __launch_bounds__(NTHREADS, 2)
         tmem_st16(tS, z);
         tmem_st16(tS + 16, z);
       } else {
-        // pass 1: masked row maximum over the 64 keys
-        float cmax = -INFINITY;
+        // pass 1: masked row maximum (one 32-column segment in registers at a time)
+        float cmax;
         {
           uint32_t sv[32];
           tmem_ld32(tS, sv);
           tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if ((bits0 >> i) & 1u) cmax = fmaxf(cmax, __uint_as_float(sv[i]));
+          cmax = masked_max(sv, bits0);
           tmem_ld32(tS + 32, sv);
           tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if ((bits1 >> i) & 1u) cmax = fmaxf(cmax, __uint_as_float(sv[i]));
+          cmax = fmaxf(cmax, masked_max(sv, bits1));
         }
         const float cmax2 = cmax * c2;
         float corr = 1.f;
@@ -472,6 +633,22 @@ __global__ void __launch_bounds__(NTHREADS, 2)
           l_run *= corr;
           m_run = cmax2;
         }
+        const float mneg = m_run == -INFINITY ? 0.f : -m_run;
+        // pass 2: P over S; keys 0-31 -> columns 0-15, keys 32-63 -> columns
+        // 16-31 (columns whose S values have been read by then)
+        {
+          uint32_t sv[32], p[16];
+          tmem_ld32(tS, sv);
+          tmem_wait_ld();
+          l_run += exp_pack(sv, bits0, c2, mneg, p);
+          tmem_st16(tS, p);
+          tmem_ld32(tS + 32, sv);
+          tmem_wait_ld();
+          l_run += exp_pack(sv, bits1, c2, mneg, p);
+          tmem_st16(tS + 16, p);
+        }
+        // rescale O after P and before this chunk's PV product, which is issued
+        // only after p_full below
         if (__any_sync(0xffffffffu, corr != 1.f)) {
           // O must hold every earlier PV product before it is rescaled
           ok = __all_sync(0xffffffffu,
@@ -487,25 +664,6 @@ __global__ void __launch_bounds__(NTHREADS, 2)
             for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * corr);
             tmem_st32(tO + part * 32, o);
           }
-        }
-        const float mneg = m_run == -INFINITY ? 0.f : -m_run;
-        // pass 2: P over S; keys 0-31 -> columns 0-15, keys 32-63 -> columns
-        // 16-31 (columns whose S values have been read by then)
-#pragma unroll 1
-        for (int seg = 0; seg < 2; ++seg) {
-          const uint32_t bits = seg ? bits1 : bits0;
-          uint32_t sv[32], p[16];
-          tmem_ld32(tS + 32 * seg, sv);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float a0 = ((bits >> (2 * i)) & 1u) ? fmaf(__uint_as_float(sv[2 * i]), c2, mneg) : -INFINITY;
-            float a1 = ((bits >> (2 * i + 1)) & 1u) ? fmaf(__uint_as_float(sv[2 * i + 1]), c2, mneg) : -INFINITY;
-            float e0 = ex2(a0), e1 = ex2(a1);
-            l_run += e0 + e1;
-            p[i] = pack_bf16x2(e0, e1);
-          }
-          tmem_st16(tS + 16 * seg, p);
         }
       }
       tmem_wait_st();

@@ -101,73 +101,125 @@ __global__ void __launch_bounds__(256) k_block_summaries(Geo g, const int32_t* _
   }
 }
 
-// bf16, head_dim 96: 16-byte loads.  Six lanes cover a 192-byte row; lane u
-// owns chunk c1 = 4 (u / 2) + u % 2 and its rotation partner c2 = c1 + 2
-// (segment u / 2, pairs 8 (u % 2) .. 8 (u % 2) + 7), for both k and v.
-// 32 token groups per CTA; the partial sums are combined in a fixed order.
-constexpr int TG96 = 32;
+// bf16, head_dim 96: 16-byte loads, two heads per CTA so that a token group
+// reads 384 contiguous bytes of k and of v.  Lane u (12 per token) serves head
+// u / 6 and owns chunk c1 = 4 (w / 2) + w % 2 (w = u % 6) and its rotation
+// partner c2 = c1 + 2 (segment w / 2, pairs 8 (w % 2) .. 8 (w % 2) + 7).  The
+// voxel -> token lookups of the next tokens are issued before the current
+// tokens' arithmetic.  Partial sums of the 16 token groups are combined in a
+// fixed order.
+constexpr int HG96 = 2, LANES96 = 6 * HG96, TG96 = 16, TAB96 = 48;
+constexpr int TABS96 = 18;  // staged row stride in float2 (16 + padding against bank conflicts)
 
-__global__ void __launch_bounds__(TG96 * 6) k_block_summaries_bf16_d96(
+__global__ void __launch_bounds__(TG96 * LANES96) k_block_summaries_bf16_d96(
     Geo g, const int32_t* __restrict__ vol, const float* __restrict__ rope,
     const int32_t* __restrict__ err, const __nv_bfloat16* __restrict__ k,
     const __nv_bfloat16* __restrict__ v, float* ksum, float* vsum) {
   if (err[0]) return;
-  __shared__ float red[TG96][2][96];
-  const int u = threadIdx.x % 6, grp = threadIdx.x / 6;
-  const int blk = blockIdx.x, b = blockIdx.y, h = blockIdx.z;
+  __shared__ float red[TG96][HG96][2][96];
+  __shared__ float2 tab_s[TAB96 * TABS96];
+  const int u = threadIdx.x % LANES96, grp = threadIdx.x / LANES96;
+  const int hh = u / 6, w = u % 6;
+  const int blk = blockIdx.x, b = blockIdx.y, h = blockIdx.z * HG96 + hh;
+  const bool live = h < g.H;
   const int Bz = blk / (g.nby * g.nbx), By = (blk / g.nbx) % g.nby, Bx = blk % g.nbx;
-  const int a = u / 2, c1 = 4 * a + (u & 1), c2 = c1 + 2, j0 = 8 * (u & 1);
-  const int axis_off = a == 0 ? 0 : (a == 1 ? g.Z : g.Z + g.Y);
-  const float2* __restrict__ tab = reinterpret_cast<const float2*>(rope);
+  const int a = w / 2, c1 = 4 * a + (w & 1), c2 = c1 + 2, j0 = 8 * (w & 1);
+  // rotation-table rows of this block's coordinates (z, then y, then x rows),
+  // staged in shared memory when they fit
+  const float2* gtab = reinterpret_cast<const float2*>(rope);
+  const float2* tab;  // row of coordinate c on this lane's axis: tab + (c - base) * stride
+  int base, stride;
+  const bool staged = g.bz + g.by + g.bx <= TAB96;
+  if (staged) {
+    const int rows = g.bz + g.by + g.bx;
+    for (int e = threadIdx.x; e < rows * 16; e += blockDim.x) {
+      const int r = e / 16, jj = e % 16;
+      const int grow = r < g.bz ? Bz * g.bz + r
+                                : (r < g.bz + g.by ? g.Z + By * g.by + r - g.bz
+                                                   : g.Z + g.Y + Bx * g.bx + r - g.bz - g.by);
+      tab_s[r * TABS96 + jj] = gtab[grow * 16 + jj];
+    }
+    __syncthreads();
+    tab = a == 0 ? tab_s : (a == 1 ? tab_s + g.bz * TABS96 : tab_s + (g.bz + g.by) * TABS96);
+    base = a == 0 ? Bz * g.bz : (a == 1 ? By * g.by : Bx * g.bx);
+    stride = TABS96;
+  } else {
+    tab = a == 0 ? gtab : (a == 1 ? gtab + g.Z * 16 : gtab + (g.Z + g.Y) * 16);
+    base = 0;
+    stride = 16;
+  }
   float kx1[8], kx2[8], vx1[8], vx2[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) kx1[i] = kx2[i] = vx1[i] = vx2[i] = 0.f;
   const int cnt = g.bz * g.by * g.bx;
   const int32_t* vb = vol + (int64_t)b * g.N;
-#pragma unroll 2
-  for (int e = grp; e < cnt; e += TG96) {
-    const int x = e % g.bx, y = (e / g.bx) % g.by, z = e / (g.bx * g.by);
-    const int cz = Bz * g.bz + z, cy = By * g.by + y, cx = Bx * g.bx + x;
-    const int tok = vb[(cz * g.Y + cy) * g.X + cx];
-    const uint4* kr = reinterpret_cast<const uint4*>(k + (((int64_t)b * g.N + tok) * g.H + h) * 96);
-    const uint4* vr = reinterpret_cast<const uint4*>(v + (((int64_t)b * g.N + tok) * g.H + h) * 96);
-    const uint4 ka = __ldg(kr + c1), kb = __ldg(kr + c2), va = __ldg(vr + c1), vb2 = __ldg(vr + c2);
-    const int ca = a == 0 ? cz : (a == 1 ? cy : cx);
-    const float2* t = tab + (axis_off + ca) * 16 + j0;
-    const uint32_t* kaw = reinterpret_cast<const uint32_t*>(&ka);
-    const uint32_t* kbw = reinterpret_cast<const uint32_t*>(&kb);
-    const uint32_t* vaw = reinterpret_cast<const uint32_t*>(&va);
-    const uint32_t* vbw = reinterpret_cast<const uint32_t*>(&vb2);
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      float2 x1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(kaw + w));
-      float2 x2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(kbw + w));
-      float2 cs0 = __ldg(t + 2 * w), cs1 = __ldg(t + 2 * w + 1);
-      kx1[2 * w] += x1.x * cs0.x - x2.x * cs0.y;
-      kx2[2 * w] += x1.x * cs0.y + x2.x * cs0.x;
-      kx1[2 * w + 1] += x1.y * cs1.x - x2.y * cs1.y;
-      kx2[2 * w + 1] += x1.y * cs1.y + x2.y * cs1.x;
-      float2 y1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(vaw + w));
-      float2 y2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(vbw + w));
-      vx1[2 * w] += y1.x;
-      vx1[2 * w + 1] += y1.y;
-      vx2[2 * w] += y2.x;
-      vx2[2 * w + 1] += y2.y;
+  auto voxel = [&](int e, int& cz, int& cy, int& cx) {
+    cx = Bx * g.bx + e % g.bx;
+    cy = By * g.by + (e / g.bx) % g.by;
+    cz = Bz * g.bz + e / (g.bx * g.by);
+  };
+  int e = grp, cz, cy, cx;
+  voxel(e, cz, cy, cx);
+  int tok = (live && e < cnt) ? vb[(cz * g.Y + cy) * g.X + cx] : 0;
+  for (; e < cnt; e += TG96) {
+    // next token's lookup first
+    const int en = e + TG96;
+    int nz = 0, ny = 0, nx = 0, ntok = 0;
+    if (en < cnt) {
+      voxel(en, nz, ny, nx);
+      if (live) ntok = vb[(nz * g.Y + ny) * g.X + nx];
     }
+    if (live) {
+      const int64_t row = (((int64_t)b * g.N + tok) * g.H + h) * 96;
+      const uint4* kr = reinterpret_cast<const uint4*>(k + row);
+      const uint4* vr = reinterpret_cast<const uint4*>(v + row);
+      const uint4 ka = __ldg(kr + c1), kb = __ldg(kr + c2), va = __ldg(vr + c1),
+                  vb2 = __ldg(vr + c2);
+      const int ca = a == 0 ? cz : (a == 1 ? cy : cx);
+      const float2* t = tab + (ca - base) * stride + j0;
+      const uint32_t* kaw = reinterpret_cast<const uint32_t*>(&ka);
+      const uint32_t* kbw = reinterpret_cast<const uint32_t*>(&kb);
+      const uint32_t* vaw = reinterpret_cast<const uint32_t*>(&va);
+      const uint32_t* vbw = reinterpret_cast<const uint32_t*>(&vb2);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float2 x1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(kaw + q));
+        float2 x2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(kbw + q));
+        const float4 cs = *reinterpret_cast<const float4*>(t + 2 * q);  // pairs j, j + 1
+        kx1[2 * q] += x1.x * cs.x - x2.x * cs.y;
+        kx2[2 * q] += x1.x * cs.y + x2.x * cs.x;
+        kx1[2 * q + 1] += x1.y * cs.z - x2.y * cs.w;
+        kx2[2 * q + 1] += x1.y * cs.w + x2.y * cs.z;
+        float2 y1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(vaw + q));
+        float2 y2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(vbw + q));
+        vx1[2 * q] += y1.x;
+        vx1[2 * q + 1] += y1.y;
+        vx2[2 * q] += y2.x;
+        vx2[2 * q + 1] += y2.y;
+      }
+    }
+    tok = ntok;
+    cz = nz;
+    cy = ny;
+    cx = nx;
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    red[grp][0][8 * c1 + i] = kx1[i];
-    red[grp][0][8 * c2 + i] = kx2[i];
-    red[grp][1][8 * c1 + i] = vx1[i];
-    red[grp][1][8 * c2 + i] = vx2[i];
+    red[grp][hh][0][8 * c1 + i] = kx1[i];
+    red[grp][hh][0][8 * c2 + i] = kx2[i];
+    red[grp][hh][1][8 * c1 + i] = vx1[i];
+    red[grp][hh][1][8 * c2 + i] = vx2[i];
   }
   __syncthreads();
-  const int which = threadIdx.x / 96, ch = threadIdx.x % 96;
-  float acc = 0.f;
-  for (int q = 0; q < TG96; ++q) acc += red[q][which][ch];
-  const int64_t o = (((int64_t)b * g.H + h) * g.nb + blk) * 96 + ch;
-  (which ? vsum : ksum)[o] = acc / (float)cnt;
+  for (int o = threadIdx.x; o < HG96 * 2 * 96; o += TG96 * LANES96) {
+    const int oh = o / 192, which = (o / 96) % 2, ch = o % 96;
+    const int hout = blockIdx.z * HG96 + oh;
+    if (hout >= g.H) continue;
+    float acc = 0.f;
+    for (int q = 0; q < TG96; ++q) acc += red[q][oh][which][ch];
+    const int64_t idx = (((int64_t)b * g.H + hout) * g.nb + blk) * 96 + ch;
+    (which ? vsum : ksum)[idx] = acc / (float)cnt;
+  }
 }
 
 }  // namespace
@@ -176,9 +228,10 @@ int launch_block_summaries(const Geo& g, const pack3d_index* idx, const void* k,
                            float* ksum, float* vsum, cudaStream_t s) {
   dim3 grid(g.nb, g.B, g.H);
   if (g.dtype == PACK3D_BF16 && g.d == 96) {
-    k_block_summaries_bf16_d96<<<grid, TG96 * 6, 0, s>>>(g, idx->vol, idx->rope, idx->err,
-                                                          (const __nv_bfloat16*)k,
-                                                          (const __nv_bfloat16*)v, ksum, vsum);
+    dim3 grid96(g.nb, g.B, (g.H + HG96 - 1) / HG96);
+    k_block_summaries_bf16_d96<<<grid96, TG96 * LANES96, 0, s>>>(
+        g, idx->vol, idx->rope, idx->err, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, ksum,
+        vsum);
     return cuda_status(cudaGetLastError());
   }
   int threads = TG * (g.d / 4);

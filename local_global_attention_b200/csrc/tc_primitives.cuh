@@ -73,6 +73,18 @@ __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src)
                "l"(gmem_src)
                : "memory");
 }
+// 16 zero bytes written through the same asynchronous path (nothing is read).
+__device__ __forceinline__ void cp_async16_zero(void* smem_dst, const void* any_gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, 0;" ::"r"(smem_u32(smem_dst)),
+               "l"(any_gmem)
+               : "memory");
+}
+// Arrive on the mbarrier once every earlier cp.async of this thread has landed
+// (the arrival counts against the barrier's expected count).
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;" ::: "memory");
 }
