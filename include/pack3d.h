@@ -157,20 +157,51 @@ PACK3D_API int pack3d_index_check(const pack3d_index* idx, pack3d_stream_t strea
 PACK3D_API int pack3d_block_summaries(const pack3d_params* p, const pack3d_index* idx, const void* k,
                            const void* v, float* ksum, float* vsum, pack3d_stream_t stream);
 
+/* Bytes of device workspace pack3d_forward and pack3d_window_forward need for
+ * these params; 0 when the call needs none (fp32, or a head_dim other than 96,
+ * which run on the CUDA cores).  At the 65,536-token, batch 2, 8-head, d = 96
+ * shape: 403 MB (grid-order copies of the rotated keys and of the values, and
+ * bf16 copies of the summaries). */
+PACK3D_API size_t pack3d_forward_workspace_bytes(const pack3d_params* p);
+
 /* Full PACK3D forward (abstract: exact local neighbourhood attention plus
  * the block summaries, axial RoPE on grid coordinates, one softmax): out and
- * lse for every query, from the local window keys and the summaries (from pack3d_block_summaries; they may
- * be reused across calls with the same k, v and index). */
-PACK3D_API int pack3d_forward(const pack3d_params* p, const pack3d_index* idx, const void* q, const void* k,
-                   const void* v, const float* ksum, const float* vsum, void* out, float* lse,
-                   pack3d_stream_t stream);
+ * lse for every query, from the local window keys and the summaries (from
+ * pack3d_block_summaries; they may be reused across calls with the same k, v
+ * and index).  workspace: caller-allocated device memory of at least
+ * pack3d_forward_workspace_bytes(p) bytes, 256-byte aligned (may be NULL when
+ * that size is 0); its contents on entry do not matter and it holds no result
+ * afterwards.  PACK3D_ERR_ARG if it is missing, short or misaligned. */
+PACK3D_API int pack3d_forward(const pack3d_params* p, const pack3d_index* idx, const void* q,
+                              const void* k, const void* v, const float* ksum, const float* vsum,
+                              void* workspace, size_t workspace_bytes, void* out, float* lse,
+                              pack3d_stream_t stream);
 
 /* Window-only forward: the same operator without summaries (windowed
  * attention with axial RoPE, the latency comparator the abstract names);
- * lse covers the local keys only. */
-PACK3D_API int pack3d_window_forward(const pack3d_params* p, const pack3d_index* idx, const void* q,
-                          const void* k, const void* v, void* out, float* lse,
-                          pack3d_stream_t stream);
+ * lse covers the local keys only.  workspace as for pack3d_forward. */
+PACK3D_API int pack3d_window_forward(const pack3d_params* p, const pack3d_index* idx,
+                                     const void* q, const void* k, const void* v, void* workspace,
+                                     size_t workspace_bytes, void* out, float* lse,
+                                     pack3d_stream_t stream);
+
+/* The two halves of the tensor-core forward, for callers that run several
+ * forwards against the same keys and values (or time the halves apart).
+ * pack3d_stage_kv writes into the workspace the rotated keys and the values in
+ * grid order and, when ksum and vsum are given (both or neither), bf16 copies
+ * of the summaries.  pack3d_forward_staged then computes out and lse from q and
+ * a workspace staged with the same params, k, v and index (with_summaries != 0:
+ * the full operator, staged with summaries; 0: window only).
+ * pack3d_forward = pack3d_stage_kv + pack3d_forward_staged.  Both return
+ * PACK3D_ERR_UNSUPPORTED where pack3d_forward_workspace_bytes is 0, and
+ * PACK3D_ERR_ARG for a missing, short or misaligned workspace. */
+PACK3D_API int pack3d_stage_kv(const pack3d_params* p, const pack3d_index* idx, const void* k,
+                               const void* v, const float* ksum, const float* vsum,
+                               void* workspace, size_t workspace_bytes, pack3d_stream_t stream);
+PACK3D_API int pack3d_forward_staged(const pack3d_params* p, const pack3d_index* idx,
+                                     const void* q, const void* workspace, size_t workspace_bytes,
+                                     int with_summaries, void* out, float* lse,
+                                     pack3d_stream_t stream);
 
 /* Bytes of device workspace pack3d_backward needs for these params. */
 PACK3D_API size_t pack3d_backward_workspace_bytes(const pack3d_params* p);

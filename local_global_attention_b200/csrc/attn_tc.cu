@@ -4,36 +4,47 @@
 // exactly to its clipped 3D window and to the summaries of the blocks its
 // window misses, in one softmax, with axial RoPE on grid coordinates.
 //
-// One CTA computes one 4 x 4 x 8 query tile (M = 128 rows) of one
-// (batch item, head).  The tile's halo (the union of its windows, raster order)
-// and then the block summaries are streamed in chunks of 64 keys.  Roles:
+// Two kernels per call:
 //
-//   * producers (warps 5-6, one key per thread): copy each chunk's key and
-//     value rows through the index with cp.async, two chunks ahead, into the
-//     64-byte-swizzled operand layout of a 3-stage shared-memory ring, and
-//     rotate a chunk's key rows in place once they have landed (axial RoPE, fp32 arithmetic, the
-//     rotation-table rows of the tile's halo staged in shared memory), or
-//     convert summary rows from fp32.  head_dim 96 is three 32-channel
-//     segments, one per axis, so a rotation segment is exactly one swizzle-atom
-//     column;
-//   * MMA (warp 4, one thread): S_j = Q K_j^T (six tcgen05.mma, K = 16) into
-//     one of two TMEM S buffers, and O += P_j V_j (four tcgen05.mma, A = P from
-//     TMEM, B = V MN-major in shared memory), so S_{j+1} is computed while the
-//     softmax works on S_j;
-//   * softmax warps (0-3, one query row per thread): gather and rotate the
-//     query rows once; per chunk build the window mask as a bit set from the
-//     halo geometry (a few operations per halo x-row, walked with a cursor, not
-//     per key), read S, keep the online max and sum, write P (bf16) over S in
-//     TMEM.  A warp whose 32 rows have no key in a chunk only writes zeros.
-//     For summary chunks the mask is "block box does not meet the window box";
-//     there is no count bias.  The running max moves only when a row's maximum
-//     grows by more than 8 (log2 units), so O is rescaled in TMEM rarely; the
-//     result is the same softmax.
+//   k_grid_kv: reads every key and value row once through the coordinate
+//     volume, applies the axial rotation to the key (fp32 arithmetic, the
+//     table built in fp64 by the index build) and writes both in grid order,
+//     one [Z][Y][X][96] bf16 volume per (batch item, head).  With the packing
+//     undone here, the halo of a query tile is a 3-D box of the grid, which the
+//     tensor-memory accelerator (TMA) copies as tiled loads; no key is gathered
+//     or rotated twice.
+//
+//   k_forward_tc: one CTA per 4 x 4 x 8 query tile (M = 128 rows) of one
+//     (batch item, head).  The tile's clipped halo box is covered by chunks of
+//     16 (x) x 2 (y) x 2 (z) = 64 keys, then the block summaries (bf16 copies,
+//     64 per chunk), all streamed through one online softmax.  Roles:
+//
+//     * TMA (warp 5, one thread): per chunk six box loads (three 32-channel
+//       segments of K and of V, 64-byte swizzle: exactly the K-major operand
+//       layout of the MMAs) into a 3-stage shared-memory ring; positions
+//       outside the volume are filled with zeros by the copy and masked;
+//     * MMA (warp 4, one thread): S_j = Q K_j^T (six tcgen05.mma, K = 16) into
+//       one of two TMEM S buffers, and O += P_j V_j (four tcgen05.mma, A = P
+//       from TMEM, B = V MN-major in shared memory), so S_{j+1} is computed
+//       while the softmax works on S_j;
+//     * softmax (warps 0-3, one query row per thread, warp w = tile plane w):
+//       gather and rotate the query rows once; per chunk form the window mask
+//       from three per-query bit sets over the halo (z planes, y rows, x
+//       columns), read the chunk's 64 S values in one go, keep the online max
+//       and sum, write P (bf16) over S in TMEM.  A warp whose 32 queries see
+//       none of a chunk's keys (a z-plane pair outside their window) only
+//       writes zeros.  Summary chunks use the mask "block box does not meet the
+//       window box"; there is no count bias.  The running max moves only when
+//       a row's maximum grows by more than 8 (log2 units), so O is rescaled in
+//       TMEM rarely; the result is the same softmax.
 //
 // The epilogue divides by the row sum and writes out (packed order) and the
 // natural-log LSE.  Two CTAs share an SM (256 TMEM columns each).  Every wait
 // is bounded; a CTA that gives up sets the timeout bit of the index error word.
+#include <cuda.h>
 #include <math.h>
+
+#include <algorithm>
 
 #include "pack3d_internal.cuh"
 #include "tc_primitives.cuh"
@@ -44,32 +55,30 @@ namespace {
 
 using namespace tc;
 
-constexpr int D = 96;                  // head dim handled by this kernel
-constexpr int KCH = 64;                // keys per chunk (N of the S MMA)
-constexpr int NSTAGE = 3;              // K/V shared-memory ring depth
-constexpr int QSEG = 128 * 64;         // one 32-channel segment of the 128 query rows
-constexpr int KSEG = KCH * 64;         // one 32-channel segment of a chunk
+constexpr int D = 96;                      // head dim handled by this path
+constexpr int KCH = 64;                    // keys per chunk (N of the S MMA)
+constexpr int BXK = 16, BYK = 2, BZK = 2;  // chunk box (x, y, z) of the halo
+constexpr int NSTAGE = 3;                  // K/V shared-memory ring depth
+constexpr int QSEG = 128 * 64;             // one 32-channel segment of the 128 query rows
+constexpr int KSEG = KCH * 64;             // one 32-channel segment of a chunk
+constexpr uint32_t CHUNK_BYTES = 6 * KSEG; // K and V of one chunk
 constexpr uint32_t TMEM_COLS = 256;
-constexpr uint32_t COL_O = 0;          // O accumulator: columns [0, 96)
-constexpr uint32_t COL_S = 128;        // S/P buffer b: columns [128 + 64 b, 192 + 64 b)
+constexpr uint32_t COL_O = 0;              // O accumulator: columns [0, 96)
+constexpr uint32_t COL_S = 128;            // S/P buffer b: columns [128 + 64 b, 192 + 64 b)
 constexpr int MMA_WARP = 4;
-constexpr int PROD0 = 160;             // first producer thread
-constexpr int NPROD = KCH;             // one producer thread per key of a chunk
-constexpr int NTHREADS = PROD0 + NPROD;
+constexpr int TMA_WARP = 5;
+constexpr int NTHREADS = 192;
 constexpr uint32_t WAIT_LIMIT = 1u << 20;
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
 constexpr float RESCALE_THRESHOLD = 8.0f;
 constexpr int ERR_TIMEOUT_BIT = 4;
-constexpr int TAB_ROWS = 64;           // rotation-table rows staged in shared memory
-constexpr int TAB_STRIDE = 18;         // float2 per staged row: 16 + 2 of padding, so rows
-                                       // of consecutive coordinates start on different banks
+constexpr int MAX_HALO = 64;               // halo extent per axis the 64-bit masks cover
 
 struct Smem {
   uint8_t q[3 * QSEG];
   uint8_t k[NSTAGE][3 * KSEG];
   uint8_t v[NSTAGE][3 * KSEG];
-  float2 tab[TAB_ROWS * TAB_STRIDE];  // rotation-table rows of the halo box
   uint64_t q_full;
   uint64_t kv_full[NSTAGE];
   uint64_t kv_empty[NSTAGE];
@@ -109,7 +118,8 @@ __device__ __forceinline__ TileBox tile_box(const Geo& g, int t) {
 
 // Rotate four words of pair members (lo) against their partners (hi): word u of
 // lo holds channels j0 + 2u, j0 + 2u + 1 of a segment, word u of hi the same
-// pairs' second members.  t = rotation-table row of the segment's axis.
+// pairs' second members.  t = rotation-table row (16 (cos, sin) pairs) of the
+// segment's axis at the row's coordinate.
 __device__ __forceinline__ void rot_chunk(uint4& lo, uint4& hi, const float2* t, int j0) {
   uint32_t* a = reinterpret_cast<uint32_t*>(&lo);
   uint32_t* b = reinterpret_cast<uint32_t*>(&hi);
@@ -122,43 +132,67 @@ __device__ __forceinline__ void rot_chunk(uint4& lo, uint4& hi, const float2* t,
   }
 }
 
-// Rows of the rotation table (16 (cos, sin) pairs per coordinate value) for the
-// coordinates a tile can touch: its halo box, staged in shared memory when they
-// fit (z rows, then y rows, then x rows), else read from the global table.
-struct RopeRows {
-  const float2* z;  // row of coordinate c is z + (c - bz) * stride
-  const float2* y;
-  const float2* x;
-  int bz, by, bx, stride;
-  __device__ __forceinline__ const float2* row(int axis, int c) const {
-    return axis == 0 ? z + (c - bz) * stride
-                     : (axis == 1 ? y + (c - by) * stride : x + (c - bx) * stride);
+// ---- grid-order rotated keys and values ------------------------------------------
+
+// One CTA per (64-voxel piece of an x row, row z * Y + y, batch item).  Key
+// items are (head, voxel, segment, half): 8 channels and their 8 partners,
+// rotated; value items (head, voxel, 16-byte chunk) are copied.  Consecutive
+// threads cover one 192-byte row, so reads (through the volume) and writes
+// (grid order) are whole rows.
+constexpr int GRID_XS = 64;
+
+__global__ void __launch_bounds__(256)
+    k_grid_kv(Geo g, pack3d_index ix, const __nv_bfloat16* __restrict__ k,
+              const __nv_bfloat16* __restrict__ v, __nv_bfloat16* __restrict__ kg,
+              __nv_bfloat16* __restrict__ vg) {
+  if (ix.err[0]) return;
+  __shared__ int32_t tok[GRID_XS];
+  const int xb = blockIdx.x * GRID_XS, zy = blockIdx.y, b = blockIdx.z;
+  const int z = zy / g.Y, y = zy % g.Y;
+  const int nx = min(GRID_XS, g.X - xb);
+  const int64_t vox0 = ((int64_t)b * g.Z * g.Y + zy) * g.X + xb;
+  for (int i = threadIdx.x; i < nx; i += blockDim.x) tok[i] = ix.vol[vox0 + i];
+  __syncthreads();
+  const float2* tab = reinterpret_cast<const float2*>(ix.rope);
+  const int H = g.H;
+  // first element of (b, h, z, y, x = xb) in the grid-order volumes
+  auto grid_row = [&](int h) {
+    return ((((int64_t)b * H + h) * g.Z + z) * g.Y + y) * g.X + xb;
+  };
+  for (int it = threadIdx.x; it < H * nx * 6; it += blockDim.x) {
+    const int u = it & 1, s = (it >> 1) % 3, rem = it / 6;
+    const int x = rem % nx, h = rem / nx;
+    const uint4* src = reinterpret_cast<const uint4*>(
+        k + (((int64_t)b * g.N + tok[x]) * H + h) * D + s * 32 + u * 8);
+    uint4 lo = __ldg(src), hi = __ldg(src + 2);
+    const int c = s == 0 ? z : (s == 1 ? y : xb + x);
+    const int row = (s == 0 ? 0 : (s == 1 ? g.Z : g.Z + g.Y)) + c;
+    rot_chunk(lo, hi, tab + row * 16, u * 8);
+    uint4* dst = reinterpret_cast<uint4*>(kg + (grid_row(h) + x) * D + s * 32 + u * 8);
+    dst[0] = lo;
+    dst[2] = hi;
   }
-};
-
-// Axial rotation of a whole 96-channel row held as 12 chunks: segment a is
-// chunks 4a..4a+3, and word w of a segment pairs with word w + 8.
-__device__ __forceinline__ void rotate_row(uint4 (&r)[12], const RopeRows& rr, int cz, int cy,
-                                           int cx) {
-  const float2* tz = rr.row(0, cz);
-  const float2* ty = rr.row(1, cy);
-  const float2* tx = rr.row(2, cx);
-  rot_chunk(r[0], r[2], tz, 0);
-  rot_chunk(r[1], r[3], tz, 8);
-  rot_chunk(r[4], r[6], ty, 0);
-  rot_chunk(r[5], r[7], ty, 8);
-  rot_chunk(r[8], r[10], tx, 0);
-  rot_chunk(r[9], r[11], tx, 8);
+  for (int it = threadIdx.x; it < H * nx * 12; it += blockDim.x) {
+    const int c = it % 12, rem = it / 12;
+    const int x = rem % nx, h = rem / nx;
+    const uint4* src =
+        reinterpret_cast<const uint4*>(v + (((int64_t)b * g.N + tok[x]) * H + h) * D) + c;
+    uint4* dst = reinterpret_cast<uint4*>(vg + (grid_row(h) + x) * D) + c;
+    *dst = __ldg(src);
+  }
 }
 
-// 16-byte chunk c (0..11) of a 96-channel row <-> its place in an operand
-// region (three 32-channel segments of seg_bytes each, 64-byte swizzle).
-__device__ __forceinline__ void store_chunk(uint8_t* region, int seg_bytes, int row, int c,
-                                            const uint4& v) {
-  *reinterpret_cast<uint4*>(region + (c >> 2) * seg_bytes + sw64_off(row, c & 3)) = v;
-}
-__device__ __forceinline__ uint4 load_chunk(const uint8_t* region, int seg_bytes, int row, int c) {
-  return *reinterpret_cast<const uint4*>(region + (c >> 2) * seg_bytes + sw64_off(row, c & 3));
+// fp32 summaries -> bf16 copies (the tensor-core operand type), same layout.
+__global__ void k_summaries_bf16(const float4* __restrict__ ks, const float4* __restrict__ vs,
+                                 uint2* __restrict__ kb, uint2* __restrict__ vb, int64_t n4,
+                                 const int32_t* __restrict__ err) {
+  if (err[0]) return;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const float4 a = ks[i], c = vs[i];
+    kb[i] = make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w));
+    vb[i] = make_uint2(pack_bf16x2(c.x, c.y), pack_bf16x2(c.z, c.w));
+  }
 }
 
 // ---- masks ---------------------------------------------------------------------
@@ -168,11 +202,9 @@ __device__ __forceinline__ uint4 load_chunk(const uint8_t* region, int seg_bytes
 struct RowCursor {
   int start;  // index of the first item of the current row
   int z, y;   // the current row's plane and row within the plane
-  int row;    // the current row's raster index (z * ny + y)
   __device__ __forceinline__ void advance_to(int e, int len, int ny) {
     while (start + len <= e) {
       start += len;
-      ++row;
       if (++y == ny) {
         y = 0;
         ++z;
@@ -180,30 +212,6 @@ struct RowCursor {
     }
   }
 };
-
-// Window mask of the 32 halo keys [e0, e0 + 32) for one query: the halo is an
-// hz x hy x hx box in raster order and the window is |z - qz| <= rz,
-// |y - qy| <= ry, x in [xlo, xhi] (halo-local).  `c` is at the row holding e0.
-__device__ __forceinline__ uint32_t local_bits(RowCursor c, int e0, int nh, int hx, int hy, int qz,
-                                               int qy, int rz, int ry, int xlo, int xhi) {
-  uint32_t bits = 0;
-  int pos = c.start - e0;  // bit of x = 0 of the current row (<= 0)
-  int z = c.z, y = c.y;
-  while (pos < 32) {
-    if (abs(z - qz) <= rz && abs(y - qy) <= ry) {
-      const int lo = max(pos + xlo, 0), hi = min(pos + xhi, 31);
-      if (lo <= hi) bits |= bit_range(lo, hi);
-    }
-    pos += hx;
-    if (++y == hy) {
-      y = 0;
-      ++z;
-    }
-  }
-  const int valid = nh - e0;
-  if (valid < 32) bits &= valid <= 0 ? 0u : (0xffffffffu >> (32 - valid));
-  return bits;
-}
 
 // Summary mask of the 32 blocks [B0, B0 + 32) (raster order over an
 // nbz x nby x nbx grid): set for blocks outside the box [blo, bhi] of blocks
@@ -235,44 +243,10 @@ __device__ __forceinline__ uint32_t summary_bits(RowCursor c, int B0, int nb, in
   return bits;
 }
 
-// Precomputed form of the masks above for boxes whose rows fit 128 bits and
-// whose rows are at most 32 items long: `rows` has bit r set for the rows r
-// (raster over z, y) the mask keeps or drops as a whole, and `pattern` is the
-// per-row item mask repeated with period `len` over 64 bits.  For the 32 items
-// [e0, e0 + 32), with the cursor at the row holding e0, the result is
-// (row bit AND pattern bit) per item - a handful of bit operations, no
-// data-dependent branches.
-struct RowMask {
-  uint32_t rows[4];
-  uint64_t pattern;
-  __device__ __forceinline__ uint32_t row_bit(int r) const {
-    const int w = r >> 5;
-    const uint32_t word = w == 0 ? rows[0] : (w == 1 ? rows[1] : (w == 2 ? rows[2] : rows[3]));
-    return (word >> (r & 31)) & 1u;
-  }
-  // items of [e0, e0 + 32) whose row bit and pattern bit are both set
-  __device__ __forceinline__ uint32_t segment(const RowCursor& c, int e0, int len) const {
-    const int off = e0 - c.start;          // position of e0 inside its row
-    const int r0 = c.row;                  // index of the row holding e0
-    const uint32_t xb = (uint32_t)(pattern >> off);
-    uint32_t rb = 0;
-    for (int k = 0, lo = -off; lo < 32; ++k, lo += len) {
-      const uint32_t m = bit_range(max(lo, 0), min(lo + len - 1, 31));
-      rb |= row_bit(r0 + k) ? m : 0u;
-    }
-    return rb & xb;
-  }
-};
-
-__device__ __forceinline__ uint64_t periodic(uint32_t m, int len) {
-  uint64_t p = m;
-  for (int s = len; s < 64; s += len) p |= (uint64_t)m << s;
-  return p;
-}
-
-// P = 2^(S c2 + mneg) for the keys in `bits`, 0 elsewhere; returns the sum.
+// P = 2^(S c2 + mneg) for the keys in `bits`, 0 elsewhere, packed in pairs into
+// p[0..15]; returns the sum.
 __device__ __forceinline__ float exp_pack(const uint32_t (&sv)[32], uint32_t bits, float c2,
-                                          float mneg, uint32_t (&p)[16]) {
+                                          float mneg, uint32_t* p) {
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
@@ -298,12 +272,23 @@ __device__ __forceinline__ float masked_max(const uint32_t (&sv)[32], uint32_t b
   return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
 }
 
+// 16-byte chunk c (0..11) of a 96-channel row -> its place in an operand region
+// (three 32-channel segments of seg_bytes each, 64-byte swizzle).
+__device__ __forceinline__ void store_chunk(uint8_t* region, int seg_bytes, int row, int c,
+                                            const uint4& v) {
+  *reinterpret_cast<uint4*>(region + (c >> 2) * seg_bytes + sw64_off(row, c & 3)) = v;
+}
+
+struct Maps {
+  CUtensorMap kg, vg;  // [B*H][Z][Y][X][96] bf16, box {32, 16, 2, 2, 1}
+  CUtensorMap ks, vs;  // [B*H][nb][96] bf16, box {32, 64, 1}
+};
+
 template <bool SUMMARY>
 __global__ void __launch_bounds__(NTHREADS, 2)
     k_forward_tc(Geo g, pack3d_index ix, const __nv_bfloat16* __restrict__ q,
-                 const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
-                 const float* __restrict__ ksum, const float* __restrict__ vsum,
-                 void* __restrict__ out_raw, float* __restrict__ lse) {
+                 const __grid_constant__ Maps maps, void* __restrict__ out_raw,
+                 float* __restrict__ lse) {
   if (ix.err[0]) return;
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -312,17 +297,16 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int t = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const TileBox tb = tile_box(g, t);
-  const int count = tb.lz * tb.ly * tb.lx;
-  const int nh = tb.hz * tb.hy * tb.hx;
-  const int n_local = (nh + KCH - 1) / KCH;
+  const int nzc = (tb.hz + BZK - 1) / BZK, nyc = (tb.hy + BYK - 1) / BYK,
+            nxc = (tb.hx + BXK - 1) / BXK;
+  const int n_local = nzc * nyc * nxc;
   const int n_sum = SUMMARY ? (g.nb + KCH - 1) / KCH : 0;
   const int nch = n_local + n_sum;
-  const int toff = ix.tile_off[(int64_t)b * (g.nT + 1) + t];
 
   if (tid == 0) {
     mbar_init(&sm.q_full, 128);
     for (int s = 0; s < NSTAGE; ++s) {
-      mbar_init(&sm.kv_full[s], NPROD);
+      mbar_init(&sm.kv_full[s], 1);
       mbar_init(&sm.kv_empty[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -338,136 +322,55 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     tmem_alloc(&sm.tmem_base, TMEM_COLS);
     tmem_relinquish();
   }
-  // rotation-table rows of the halo box (all threads stage; producers and
-  // softmax warps read)
-  RopeRows rr;
-  {
-    const float2* gt = reinterpret_cast<const float2*>(ix.rope);
-    const int rows = tb.hz + tb.hy + tb.hx;
-    if (rows <= TAB_ROWS) {
-      for (int e = tid; e < rows * 16; e += NTHREADS) {
-        const int r = e / 16, jj = e % 16;
-        const int grow = r < tb.hz ? tb.hz0 + r
-                                   : (r < tb.hz + tb.hy ? g.Z + tb.hy0 + r - tb.hz
-                                                        : g.Z + g.Y + tb.hx0 + r - tb.hz - tb.hy);
-        sm.tab[r * TAB_STRIDE + jj] = gt[grow * 16 + jj];
-      }
-      rr.z = sm.tab;
-      rr.y = sm.tab + tb.hz * TAB_STRIDE;
-      rr.x = sm.tab + (tb.hz + tb.hy) * TAB_STRIDE;
-      rr.bz = tb.hz0;
-      rr.by = tb.hy0;
-      rr.bx = tb.hx0;
-      rr.stride = TAB_STRIDE;
-    } else {
-      rr.z = gt;
-      rr.y = gt + g.Z * 16;
-      rr.x = gt + (g.Z + g.Y) * 16;
-      rr.bz = rr.by = rr.bx = 0;
-      rr.stride = 16;
-    }
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = sm.tmem_base;
 
-  if (tid >= PROD0) {
-    // ================= producers (one key row of each chunk per thread) =================
-    const int key = tid - PROD0;
-    const int32_t* __restrict__ hl = ix.nbr + (int64_t)b * ix.n_halo + ix.nbr_off[t];
-    const int64_t sbase = ((int64_t)b * g.H + h) * g.nb;
-    int next_row = (key < nh) ? hl[key] : 0;  // neighbour index of the next chunk to issue
-    // Copy chunk j's raw key and value rows into its stage (zero rows past the
-    // halo); one cp.async group per chunk.  False if a wait gave up.
-    auto issue = [&](int j) -> bool {
-      const int s = j % NSTAGE, round = j / NSTAGE;
-      const int row_idx = next_row;
-      if (j + 1 < n_local) {
-        const int en = (j + 1) * KCH + key;
-        next_row = en < nh ? hl[en] : 0;
-      }
-      if (round > 0 &&
-          !mbar_wait_or_abort(&sm.kv_empty[s], (round - 1) & 1, WAIT_LIMIT, abort_flag))
-        return false;
-      if (j < n_local) {
-        const int e = j * KCH + key;
-        if (e < nh) {
-          const int64_t row = (((int64_t)b * g.N + row_idx) * g.H + h) * D;
-          const uint4* ks = reinterpret_cast<const uint4*>(k + row);
-          const uint4* vs = reinterpret_cast<const uint4*>(v + row);
+  if (warp == TMA_WARP) {
+    // ================= TMA producer =================
+    if (lane == 0) {
+      tma_prefetch_map(&maps.kg);
+      tma_prefetch_map(&maps.vg);
+      const int bh = b * g.H + h;
+      int xc = 0, yc = 0, zc = 0;
+      int issued = 0;
+      for (int j = 0; j < nch; ++j) {
+        const int s = j % NSTAGE, round = j / NSTAGE;
+        if (round > 0 &&
+            !mbar_wait_or_abort(&sm.kv_empty[s], (round - 1) & 1, WAIT_LIMIT, abort_flag))
+          break;
+        mbar_arrive_expect_tx(&sm.kv_full[s], CHUNK_BYTES);
+        if (j < n_local) {
+          const int x = tb.hx0 + BXK * xc, y = tb.hy0 + BYK * yc, z = tb.hz0 + BZK * zc;
 #pragma unroll
-          for (int c = 0; c < 12; ++c) {
-            cp_async16(sm.k[s] + (c >> 2) * KSEG + sw64_off(key, c & 3), ks + c);
-            cp_async16(sm.v[s] + (c >> 2) * KSEG + sw64_off(key, c & 3), vs + c);
+          for (int seg = 0; seg < 3; ++seg) {
+            tma_load_5d(sm.k[s] + seg * KSEG, &maps.kg, seg * 32, x, y, z, bh, &sm.kv_full[s]);
+            tma_load_5d(sm.v[s] + seg * KSEG, &maps.vg, seg * 32, x, y, z, bh, &sm.kv_full[s]);
+          }
+          if (++xc == nxc) {
+            xc = 0;
+            if (++yc == nyc) {
+              yc = 0;
+              ++zc;
+            }
           }
         } else {
+          const int B0 = (j - n_local) * KCH;
 #pragma unroll
-          for (int c = 0; c < 12; ++c) {
-            cp_async16_zero(sm.k[s] + (c >> 2) * KSEG + sw64_off(key, c & 3), k);
-            cp_async16_zero(sm.v[s] + (c >> 2) * KSEG + sw64_off(key, c & 3), v);
+          for (int seg = 0; seg < 3; ++seg) {
+            tma_load_3d(sm.k[s] + seg * KSEG, &maps.ks, seg * 32, B0, bh, &sm.kv_full[s]);
+            tma_load_3d(sm.v[s] + seg * KSEG, &maps.vs, seg * 32, B0, bh, &sm.kv_full[s]);
           }
         }
+        issued = j + 1;
       }
-      cp_async_commit();
-      return true;
-    };
-    // Two chunks in flight: chunk j + 2 is issued after chunk j has been
-    // rotated (issuing it first would wait on chunk j - 1's PV product, which
-    // the MMA thread issues only after S_j, i.e. after this rotation).
-    bool ok = issue(0);
-    if (ok && nch > 1) ok = issue(1);
-    // the halo-local coordinate of this thread's key in chunk j, advanced
-    // without division
-    int kx = key % tb.hx, ky = (key / tb.hx) % tb.hy, kz = key / (tb.hx * tb.hy);
-    for (int j = 0; j < nch && ok; ++j) {
-      const int s = j % NSTAGE;
-      if (j + 1 < nch)
-        cp_async_wait_group<1>();  // chunk j + 1 may still be in flight
-      else
-        cp_async_wait_group<0>();
-      if (j < n_local) {
-        if (j * KCH + key < nh) {
-          uint4 r[12];
-#pragma unroll
-          for (int c = 0; c < 12; ++c) r[c] = load_chunk(sm.k[s], KSEG, key, c);
-          rotate_row(r, rr, tb.hz0 + kz, tb.hy0 + ky, tb.hx0 + kx);
-#pragma unroll
-          for (int c = 0; c < 12; ++c) store_chunk(sm.k[s], KSEG, key, c, r[c]);
-        }
-        kx += KCH;
-        while (kx >= tb.hx) {
-          kx -= tb.hx;
-          if (++ky == tb.hy) {
-            ky = 0;
-            ++kz;
-          }
-        }
-      } else {
-        // summaries: fp32 rows converted to bf16 (keys already rotated)
-        const int B = (j - n_local) * KCH + key;
-#pragma unroll
-        for (int which = 0; which < 2; ++which) {
-          const float* src = which ? vsum : ksum;
-          uint8_t* dst = which ? sm.v[s] : sm.k[s];
-#pragma unroll 4
-          for (int c = 0; c < 12; ++c) {
-            uint4 w = make_uint4(0, 0, 0, 0);
-            if (B < g.nb) {
-              const float4* f = reinterpret_cast<const float4*>(src + (sbase + B) * D);
-              const float4 a0 = __ldg(f + 2 * c), a1 = __ldg(f + 2 * c + 1);
-              w = make_uint4(pack_bf16x2(a0.x, a0.y), pack_bf16x2(a0.z, a0.w),
-                             pack_bf16x2(a1.x, a1.y), pack_bf16x2(a1.z, a1.w));
-            }
-            store_chunk(dst, KSEG, key, c, w);
-          }
-        }
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(&sm.kv_full[s]);
-      if (j + 2 < nch) ok = issue(j + 2);
+      // Copies still in flight must land before the CTA ends (bounded: they
+      // complete unless the memory system has failed).
+      for (int j = max(0, issued - NSTAGE); j < issued; ++j)
+        mbar_wait(&sm.kv_full[j % NSTAGE], (j / NSTAGE) & 1, WAIT_LIMIT);
     }
-    cp_async_wait_group<0>();
+    __syncwarp();
   } else if (warp == MMA_WARP) {
     // ================= MMA issue =================
     if (lane == 0) {
@@ -517,14 +420,12 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     __syncwarp();
   } else {
     // ================= softmax warps (one query row per thread) =================
-    const bool active = tid < count;
-    int cz = 0, cy = 0, cx = 0, qi = 0;
-    if (active) {
-      cx = tb.x0 + tid % tb.lx;
-      cy = tb.y0 + (tid / tb.lx) % tb.ly;
-      cz = tb.z0 + tid / (tb.lx * tb.ly);
-      qi = ix.perm[(int64_t)b * g.N + toff + tid];
-    }
+    // row tid = (plane tid / 32, row (tid / 8) % 4, column tid % 8) of the tile
+    const int lzi = tid >> 5, lyi = (tid >> 3) & 3, lxi = tid & 7;
+    const bool active = lzi < tb.lz && lyi < tb.ly && lxi < tb.lx;
+    const int cz = tb.z0 + lzi, cy = tb.y0 + lyi, cx = tb.x0 + lxi;
+    int qi = 0;
+    if (active) qi = ix.vol[(((int64_t)b * g.Z + cz) * g.Y + cy) * g.X + cx];
     {
       // this thread's query row: gathered, rotated, stored once
       uint4 r[12];
@@ -533,7 +434,16 @@ __global__ void __launch_bounds__(NTHREADS, 2)
             reinterpret_cast<const uint4*>(q + (((int64_t)b * g.N + qi) * g.H + h) * D);
 #pragma unroll
         for (int i = 0; i < 12; ++i) r[i] = __ldg(src + i);
-        rotate_row(r, rr, cz, cy, cx);
+        const float2* tab = reinterpret_cast<const float2*>(ix.rope);
+        const float2* tz = tab + cz * 16;
+        const float2* ty = tab + (g.Z + cy) * 16;
+        const float2* tx = tab + (g.Z + g.Y + cx) * 16;
+        rot_chunk(r[0], r[2], tz, 0);
+        rot_chunk(r[1], r[3], tz, 8);
+        rot_chunk(r[4], r[6], ty, 0);
+        rot_chunk(r[5], r[7], ty, 8);
+        rot_chunk(r[8], r[10], tx, 0);
+        rot_chunk(r[9], r[11], tx, 8);
       } else {
 #pragma unroll
         for (int i = 0; i < 12; ++i) r[i] = make_uint4(0, 0, 0, 0);
@@ -543,32 +453,20 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       fence_proxy_async_smem();
       mbar_arrive(&sm.q_full);
     }
-    const int qz = cz - tb.hz0, qy = cy - tb.hy0, qx = cx - tb.hx0;
-    const int xlo = max(qx - g.rx, 0), xhi = min(qx + g.rx, tb.hx - 1);
-    // Precomputed window mask (halo rows in the window; x range as a periodic
-    // pattern) when the halo's rows fit, else the per-row walk.
-    const bool fast_local = tb.hz * tb.hy <= 128 && tb.hx <= 32;
-    RowMask lm;
-    if (fast_local) {
-      lm.rows[0] = lm.rows[1] = lm.rows[2] = lm.rows[3] = 0u;
-      const int ylo = max(qy - g.ry, 0), yhi = min(qy + g.ry, tb.hy - 1);
-      for (int z = max(qz - g.rz, 0); z <= min(qz + g.rz, tb.hz - 1); ++z) {
-        // rows z * hy + [ylo, yhi] of plane z, spread over the four words
-        const int a = z * tb.hy + ylo, e = z * tb.hy + yhi;
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          const int lo = max(a - 32 * w, 0), hi = min(e - 32 * w, 31);
-          if (lo <= hi) lm.rows[w] |= bit_range(lo, hi);
-        }
-      }
-      lm.pattern = periodic(bit_range(xlo, xhi), tb.hx);
+    // The window as bit sets over halo-local positions (in-volume positions
+    // only, so zero-filled keys outside the volume are never selected).
+    uint64_t zwin = 0, ywin = 0, xwin = 0;
+    if (active) {
+      zwin = bit_range64(max(cz - g.rz, 0) - tb.hz0, min(cz + g.rz, g.Z - 1) - tb.hz0);
+      ywin = bit_range64(max(cy - g.ry, 0) - tb.hy0, min(cy + g.ry, g.Y - 1) - tb.hy0);
+      xwin = bit_range64(max(cx - g.rx, 0) - tb.hx0, min(cx + g.rx, g.X - 1) - tb.hx0);
     }
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     const uint32_t tO = tbase + lane_base + COL_O;
     const float c2 = g.tau * LOG2E;  // logits -> log2 units
     float m_run = -INFINITY, l_run = 0.f;
-    RowCursor hc = {0, 0, 0, 0};  // halo rows (hx keys each, hy rows per plane)
-    RowCursor bc = {0, 0, 0, 0};  // block rows (nbx blocks each, nby rows per plane)
+    RowCursor bc = {0, 0, 0};  // block rows (nbx blocks each, nby rows per plane)
+    int xc = 0, yc = 0, zc = 0;
     bool ok = true;
     for (int j = 0; j < nch; ++j) {
       const int buf = j & 1;
@@ -580,21 +478,19 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       const uint32_t tS = tbase + lane_base + COL_S + 64 * buf;
       uint32_t bits0, bits1;
       if (j < n_local) {
-        const int e0 = j * KCH;
-        hc.advance_to(e0, tb.hx, tb.hy);
-        if (fast_local) {
-          bits0 = lm.segment(hc, e0, tb.hx);
-          hc.advance_to(e0 + 32, tb.hx, tb.hy);
-          bits1 = lm.segment(hc, e0 + 32, tb.hx);
-          const int valid = nh - e0;  // keys past the halo
-          if (valid < 64) {
-            bits0 &= valid <= 0 ? 0u : (valid >= 32 ? 0xffffffffu : (0xffffffffu >> (32 - valid)));
-            bits1 &= valid <= 32 ? 0u : (0xffffffffu >> (64 - valid));
+        // key (dz, dy, dx) of the chunk box is bit (dz * 2 + dy) * 16 + dx
+        const uint32_t xp = (uint32_t)(xwin >> (BXK * xc)) & 0xffffu;
+        const uint32_t yb = (uint32_t)(ywin >> (BYK * yc)) & 3u;
+        const uint32_t zb = (uint32_t)(zwin >> (BZK * zc)) & 3u;
+        const uint32_t row16 = ((yb & 1u) ? xp : 0u) | ((yb & 2u) ? (xp << 16) : 0u);
+        bits0 = (zb & 1u) ? row16 : 0u;
+        bits1 = (zb & 2u) ? row16 : 0u;
+        if (++xc == nxc) {
+          xc = 0;
+          if (++yc == nyc) {
+            yc = 0;
+            ++zc;
           }
-        } else {
-          bits0 = local_bits(hc, e0, nh, tb.hx, tb.hy, qz, qy, g.rz, g.ry, xlo, xhi);
-          hc.advance_to(e0 + 32, tb.hx, tb.hy);
-          bits1 = local_bits(hc, e0 + 32, nh, tb.hx, tb.hy, qz, qy, g.rz, g.ry, xlo, xhi);
         }
       } else {
         const int B0 = (j - n_local) * KCH;
@@ -606,26 +502,19 @@ __global__ void __launch_bounds__(NTHREADS, 2)
         bits0 = summary_bits(bc, B0, g.nb, g.nbx, g.nby, bzlo, bzhi, bylo, byhi, bxlo, bxhi);
         bc.advance_to(B0 + 32, g.nbx, g.nby);
         bits1 = summary_bits(bc, B0 + 32, g.nb, g.nbx, g.nby, bzlo, bzhi, bylo, byhi, bxlo, bxhi);
+        if (!active) bits0 = bits1 = 0u;
       }
-      if (!active) bits0 = bits1 = 0u;
       if (__ballot_sync(0xffffffffu, (bits0 | bits1) != 0u) == 0u) {
-        uint32_t z[16];
+        uint32_t zero[32];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) z[i] = 0u;
-        tmem_st16(tS, z);
-        tmem_st16(tS + 16, z);
+        for (int i = 0; i < 32; ++i) zero[i] = 0u;
+        tmem_st32(tS, zero);
       } else {
-        // pass 1: masked row maximum (one 32-column segment in registers at a time)
-        float cmax;
-        {
-          uint32_t sv[32];
-          tmem_ld32(tS, sv);
-          tmem_wait_ld();
-          cmax = masked_max(sv, bits0);
-          tmem_ld32(tS + 32, sv);
-          tmem_wait_ld();
-          cmax = fmaxf(cmax, masked_max(sv, bits1));
-        }
+        uint32_t sa[32], sb[32];
+        tmem_ld32(tS, sa);
+        tmem_ld32(tS + 32, sb);
+        tmem_wait_ld();
+        const float cmax = fmaxf(masked_max(sa, bits0), masked_max(sb, bits1));
         const float cmax2 = cmax * c2;
         float corr = 1.f;
         if (cmax2 > m_run + RESCALE_THRESHOLD) {
@@ -634,21 +523,13 @@ __global__ void __launch_bounds__(NTHREADS, 2)
           m_run = cmax2;
         }
         const float mneg = m_run == -INFINITY ? 0.f : -m_run;
-        // pass 2: P over S; keys 0-31 -> columns 0-15, keys 32-63 -> columns
-        // 16-31 (columns whose S values have been read by then)
-        {
-          uint32_t sv[32], p[16];
-          tmem_ld32(tS, sv);
-          tmem_wait_ld();
-          l_run += exp_pack(sv, bits0, c2, mneg, p);
-          tmem_st16(tS, p);
-          tmem_ld32(tS + 32, sv);
-          tmem_wait_ld();
-          l_run += exp_pack(sv, bits1, c2, mneg, p);
-          tmem_st16(tS + 16, p);
-        }
-        // rescale O after P and before this chunk's PV product, which is issued
-        // only after p_full below
+        // P over S: keys 0-63 -> columns 0-31 (S is already in registers)
+        uint32_t p[32];
+        l_run += exp_pack(sa, bits0, c2, mneg, p);
+        l_run += exp_pack(sb, bits1, c2, mneg, p + 16);
+        tmem_st32(tS, p);
+        // rescale O before this chunk's PV product, which is issued only
+        // after p_full below
         if (__any_sync(0xffffffffu, corr != 1.f)) {
           // O must hold every earlier PV product before it is rescaled
           ok = __all_sync(0xffffffffu,
@@ -723,13 +604,110 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   }
 }
 
+// ---- host side --------------------------------------------------------------------
+
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                 const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                 const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// The driver's tensor-map encoder, looked up once through the runtime (no
+// link-time dependency on the driver library).
+EncodeTiled encode_fn() {
+  static EncodeTiled fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) !=
+            cudaSuccess ||
+        qr != cudaDriverEntryPointSuccess)
+      return (EncodeTiled) nullptr;
+    return reinterpret_cast<EncodeTiled>(p);
+  }();
+  return fn;
+}
+
+// bf16 tensor of `rank` dims (innermost first, dims[0] = 96 channels, dense);
+// box {32, box[1..]}, 64-byte swizzle, zero fill outside the tensor.
+bool encode_bf16(CUtensorMap* m, void* base, int rank, const uint64_t* dims,
+                 const uint32_t* box) {
+  EncodeTiled fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gdim[5], gstride[4];
+  cuuint32_t bdim[5], estride[5];
+  uint64_t stride = 2;
+  for (int i = 0; i < rank; ++i) {
+    gdim[i] = dims[i];
+    bdim[i] = box[i];
+    estride[i] = 1;
+    stride *= dims[i];
+    if (i + 1 < rank) gstride[i] = stride;
+  }
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, base, gdim, gstride, bdim, estride,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct WsLayout {
+  size_t kg, vg, ks, vs, total;
+};
+
+WsLayout ws_layout(const Geo& g) {
+  auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  const size_t vol = (size_t)g.B * g.H * g.Z * g.Y * g.X * D * 2;
+  const size_t sum = (size_t)g.B * g.H * g.nb * D * 2;
+  WsLayout w;
+  w.kg = 0;
+  w.vg = al(vol);
+  w.ks = w.vg + al(vol);
+  w.vs = w.ks + al(sum);
+  w.total = w.vs + al(sum);
+  return w;
+}
+
 }  // namespace
 
-bool forward_tc_supported(const Geo& g) { return g.d == D && g.dtype == PACK3D_BF16; }
+bool forward_tc_supported(const Geo& g) {
+  return g.d == D && g.dtype == PACK3D_BF16 && TZ + 2 * g.rz <= MAX_HALO &&
+         TY + 2 * g.ry <= MAX_HALO && TX + 2 * g.rx <= MAX_HALO;
+}
 
-int launch_forward_tc(const Geo& g, const pack3d_index* idx, const void* q, const void* k,
-                      const void* v, const float* ksum, const float* vsum, void* out, float* lse,
-                      bool summaries, cudaStream_t s) {
+size_t forward_tc_workspace_bytes(const Geo& g) {
+  return forward_tc_supported(g) ? ws_layout(g).total : 0;
+}
+
+int launch_stage_kv(const Geo& g, const pack3d_index* idx, const void* k, const void* v,
+                    const float* ksum, const float* vsum, void* ws, cudaStream_t s) {
+  const WsLayout w = ws_layout(g);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  dim3 ggrid((g.X + GRID_XS - 1) / GRID_XS, g.Z * g.Y, g.B);
+  k_grid_kv<<<ggrid, 256, 0, s>>>(g, *idx, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
+                                  reinterpret_cast<__nv_bfloat16*>(base + w.kg),
+                                  reinterpret_cast<__nv_bfloat16*>(base + w.vg));
+  if (ksum && vsum) {
+    const int64_t n4 = (int64_t)g.B * g.H * g.nb * D / 4;
+    const int blocks = (int)std::min<int64_t>((n4 + 255) / 256, 148 * 8);
+    k_summaries_bf16<<<blocks, 256, 0, s>>>((const float4*)ksum, (const float4*)vsum,
+                                            reinterpret_cast<uint2*>(base + w.ks),
+                                            reinterpret_cast<uint2*>(base + w.vs), n4, idx->err);
+  }
+  return cuda_status(cudaGetLastError());
+}
+
+int launch_attention_tc(const Geo& g, const pack3d_index* idx, const void* q, void* ws,
+                        void* out, float* lse, bool summaries, cudaStream_t s) {
+  const WsLayout w = ws_layout(g);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  Maps maps;
+  const uint64_t vdims[5] = {(uint64_t)D, (uint64_t)g.X, (uint64_t)g.Y, (uint64_t)g.Z,
+                             (uint64_t)g.B * g.H};
+  const uint32_t vbox[5] = {32, BXK, BYK, BZK, 1};
+  const uint64_t sdims[3] = {(uint64_t)D, (uint64_t)g.nb, (uint64_t)g.B * g.H};
+  const uint32_t sbox[3] = {32, KCH, 1};
+  if (!encode_bf16(&maps.kg, base + w.kg, 5, vdims, vbox) ||
+      !encode_bf16(&maps.vg, base + w.vg, 5, vdims, vbox) ||
+      !encode_bf16(&maps.ks, base + w.ks, 3, sdims, sbox) ||
+      !encode_bf16(&maps.vs, base + w.vs, 3, sdims, sbox))
+    return PACK3D_ERR_CUDA;
   dim3 grid(g.nT, g.H, g.B);
   auto kern = summaries ? k_forward_tc<true> : k_forward_tc<false>;
   // Two CTAs per SM: enough shared memory for both, and the largest carveout.
@@ -738,9 +716,7 @@ int launch_forward_tc(const Geo& g, const pack3d_index* idx, const void* q, cons
       cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
                            (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess)
     return PACK3D_ERR_CUDA;
-  kern<<<grid, NTHREADS, SMEM_REQUEST, s>>>(g, *idx, (const __nv_bfloat16*)q,
-                                             (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
-                                             ksum, vsum, out, lse);
+  kern<<<grid, NTHREADS, SMEM_REQUEST, s>>>(g, *idx, (const __nv_bfloat16*)q, maps, out, lse);
   return cuda_status(cudaGetLastError());
 }
 

@@ -172,29 +172,72 @@ int pack3d_block_summaries(const pack3d_params* p, const pack3d_index* idx, cons
   return launch_block_summaries(g, idx, k, v, ksum, vsum, (cudaStream_t)stream);
 }
 
+size_t pack3d_forward_workspace_bytes(const pack3d_params* p) {
+  Geo g;
+  if (make_geo(p, &g)) return 0;
+  return forward_tc_workspace_bytes(g);
+}
+
 static int forward_common(const pack3d_params* p, const pack3d_index* idx, const void* q,
                           const void* k, const void* v, const float* ksum, const float* vsum,
-                          void* out, float* lse, bool summaries, cudaStream_t s) {
+                          void* ws, size_t ws_bytes, void* out, float* lse, bool summaries,
+                          cudaStream_t s) {
   Geo g;
   int rc = make_geo(p, &g);
   if (rc) return rc;
   if ((rc = check_index(g, idx))) return rc;
   if (!q || !k || !v || !out || !lse || (summaries && (!ksum || !vsum))) return PACK3D_ERR_ARG;
-  if (g.dtype == PACK3D_BF16 && forward_tc_supported(g))
-    return launch_forward_tc(g, idx, q, k, v, ksum, vsum, out, lse, summaries, s);
+  const size_t need = forward_tc_workspace_bytes(g);
+  if (need) {
+    if (!ws || ((uintptr_t)ws & 255) || ws_bytes < need) return PACK3D_ERR_ARG;
+    if ((rc = launch_stage_kv(g, idx, k, v, ksum, vsum, ws, s))) return rc;
+    return launch_attention_tc(g, idx, q, ws, out, lse, summaries, s);
+  }
   return launch_forward_simt(g, idx, q, k, v, ksum, vsum, out, lse, summaries, s);
 }
 
+int pack3d_stage_kv(const pack3d_params* p, const pack3d_index* idx, const void* k, const void* v,
+                    const float* ksum, const float* vsum, void* workspace, size_t workspace_bytes,
+                    pack3d_stream_t stream) {
+  Geo g;
+  int rc = make_geo(p, &g);
+  if (rc) return rc;
+  if ((rc = check_index(g, idx))) return rc;
+  const size_t need = forward_tc_workspace_bytes(g);
+  if (!need) return PACK3D_ERR_UNSUPPORTED;
+  if (!k || !v || (!ksum != !vsum) || !workspace || ((uintptr_t)workspace & 255) ||
+      workspace_bytes < need)
+    return PACK3D_ERR_ARG;
+  return launch_stage_kv(g, idx, k, v, ksum, vsum, workspace, (cudaStream_t)stream);
+}
+
+int pack3d_forward_staged(const pack3d_params* p, const pack3d_index* idx, const void* q,
+                          const void* workspace, size_t workspace_bytes, int with_summaries,
+                          void* out, float* lse, pack3d_stream_t stream) {
+  Geo g;
+  int rc = make_geo(p, &g);
+  if (rc) return rc;
+  if ((rc = check_index(g, idx))) return rc;
+  const size_t need = forward_tc_workspace_bytes(g);
+  if (!need) return PACK3D_ERR_UNSUPPORTED;
+  if (!q || !out || !lse || !workspace || ((uintptr_t)workspace & 255) || workspace_bytes < need)
+    return PACK3D_ERR_ARG;
+  return launch_attention_tc(g, idx, q, const_cast<void*>(workspace), out, lse,
+                             with_summaries != 0, (cudaStream_t)stream);
+}
+
 int pack3d_forward(const pack3d_params* p, const pack3d_index* idx, const void* q, const void* k,
-                   const void* v, const float* ksum, const float* vsum, void* out, float* lse,
-                   pack3d_stream_t stream) {
-  return forward_common(p, idx, q, k, v, ksum, vsum, out, lse, true, (cudaStream_t)stream);
+                   const void* v, const float* ksum, const float* vsum, void* workspace,
+                   size_t workspace_bytes, void* out, float* lse, pack3d_stream_t stream) {
+  return forward_common(p, idx, q, k, v, ksum, vsum, workspace, workspace_bytes, out, lse, true,
+                        (cudaStream_t)stream);
 }
 
 int pack3d_window_forward(const pack3d_params* p, const pack3d_index* idx, const void* q,
-                          const void* k, const void* v, void* out, float* lse,
-                          pack3d_stream_t stream) {
-  return forward_common(p, idx, q, k, v, nullptr, nullptr, out, lse, false, (cudaStream_t)stream);
+                          const void* k, const void* v, void* workspace, size_t workspace_bytes,
+                          void* out, float* lse, pack3d_stream_t stream) {
+  return forward_common(p, idx, q, k, v, nullptr, nullptr, workspace, workspace_bytes, out, lse,
+                        false, (cudaStream_t)stream);
 }
 
 size_t pack3d_backward_workspace_bytes(const pack3d_params* p) {

@@ -68,9 +68,13 @@ int launch_forward_simt(const Geo& g, const pack3d_index* idx, const void* q, co
                         const void* v, const float* ksum, const float* vsum, void* out,
                         float* lse, bool summaries, cudaStream_t s);
 bool forward_tc_supported(const Geo& g);
-int launch_forward_tc(const Geo& g, const pack3d_index* idx, const void* q, const void* k,
-                      const void* v, const float* ksum, const float* vsum, void* out, float* lse,
-                      bool summaries, cudaStream_t s);
+size_t forward_tc_workspace_bytes(const Geo& g);  // 0 when the path does not apply
+// grid-order rotated keys and values (and bf16 summaries when ksum, vsum are
+// given) into the workspace; then the attention kernel reading them
+int launch_stage_kv(const Geo& g, const pack3d_index* idx, const void* k, const void* v,
+                    const float* ksum, const float* vsum, void* ws, cudaStream_t s);
+int launch_attention_tc(const Geo& g, const pack3d_index* idx, const void* q, void* ws,
+                        void* out, float* lse, bool summaries, cudaStream_t s);
 size_t backward_workspace_bytes(const Geo& g);
 int launch_backward(const Geo& g, const pack3d_index* idx, const void* q, const void* k,
                     const void* v, const void* out, const float* lse, const void* dout, void* dq,

@@ -94,6 +94,40 @@ __device__ __forceinline__ void cp_async_wait_group() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// ---- TMA (tiled bulk tensor copies) --------------------------------------------
+
+// Arrive once and add `bytes` to the transaction count the current phase waits
+// for (the TMA copies signalled on this barrier complete them).
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+// One box of a 5-D / 3-D tensor map (coordinates innermost first) into shared
+// memory; completion is signalled on `bar` as transaction bytes.  Plain loads
+// from this GPU's memory, no multicast.
+__device__ __forceinline__ void tma_load_5d(void* dst, const void* map, int c0, int c1, int c2,
+                                            int c3, int c4, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4),
+      "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(void* dst, const void* map, int c0, int c1, int c2,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_map(const void* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
 // ---- tensor memory ------------------------------------------------------------
 
 // Allocate `ncols` TMEM columns (power of two >= 32); the base address is
@@ -253,6 +287,12 @@ __device__ __forceinline__ float ex2(float x) {
 // Bits lo..hi (inclusive, 0 <= lo <= hi <= 31) set.
 __device__ __forceinline__ uint32_t bit_range(int lo, int hi) {
   return (0xffffffffu >> (31 - hi)) & (0xffffffffu << lo);
+}
+
+// Bits lo..hi (inclusive, 0 <= lo <= hi <= 63) of a 64-bit word; 0 if lo > hi.
+__device__ __forceinline__ uint64_t bit_range64(int lo, int hi) {
+  if (lo > hi) return 0;
+  return (~0ull >> (63 - hi)) & (~0ull << lo);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

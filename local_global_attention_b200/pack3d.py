@@ -19,7 +19,8 @@ BF16, FP32 = 0, 1
 OK, ERR_ARG, ERR_COORDS, ERR_CUDA, ERR_TIMEOUT, ERR_UNSUPPORTED = 0, -1, -2, -3, -4, -5
 
 EXPORTS = ("pack3d_index_bytes", "pack3d_index_init", "pack3d_build_index", "pack3d_index_check",
-           "pack3d_block_summaries", "pack3d_forward", "pack3d_window_forward",
+           "pack3d_block_summaries", "pack3d_forward_workspace_bytes", "pack3d_forward",
+           "pack3d_window_forward", "pack3d_stage_kv", "pack3d_forward_staged",
            "pack3d_backward_workspace_bytes", "pack3d_backward", "pack3d_backward_noalloc",
            "pack3d_strerror")
 
@@ -70,8 +71,16 @@ def load(build_if_missing: bool = True):
         lib.pack3d_build_index.argtypes = [P(Params), vp, P(Index), vp]
         lib.pack3d_index_check.argtypes = [P(Index), vp]
         lib.pack3d_block_summaries.argtypes = [P(Params), P(Index), vp, vp, vp, vp, vp]
-        lib.pack3d_forward.argtypes = [P(Params), P(Index), vp, vp, vp, vp, vp, vp, vp, vp]
-        lib.pack3d_window_forward.argtypes = [P(Params), P(Index), vp, vp, vp, vp, vp, vp]
+        lib.pack3d_forward_workspace_bytes.argtypes = [P(Params)]
+        lib.pack3d_forward_workspace_bytes.restype = ctypes.c_size_t
+        lib.pack3d_forward.argtypes = [P(Params), P(Index), vp, vp, vp, vp, vp, vp,
+                                       ctypes.c_size_t, vp, vp, vp]
+        lib.pack3d_window_forward.argtypes = [P(Params), P(Index), vp, vp, vp, vp,
+                                              ctypes.c_size_t, vp, vp, vp]
+        lib.pack3d_stage_kv.argtypes = [P(Params), P(Index), vp, vp, vp, vp, vp, ctypes.c_size_t,
+                                        vp]
+        lib.pack3d_forward_staged.argtypes = [P(Params), P(Index), vp, vp, ctypes.c_size_t,
+                                              ctypes.c_int, vp, vp, vp]
         lib.pack3d_backward_workspace_bytes.argtypes = [P(Params)]
         lib.pack3d_backward_workspace_bytes.restype = ctypes.c_size_t
         lib.pack3d_backward.argtypes = [P(Params), P(Index), vp, vp, vp, vp, vp, vp, vp, vp, vp,
@@ -208,29 +217,78 @@ def pack3d_block_summaries(params: Params, index: IndexBuffers, k, v, ksum=None,
     return ksum, vsum
 
 
+def pack3d_forward_workspace_bytes(params: Params) -> int:
+    return int(load().pack3d_forward_workspace_bytes(ctypes.byref(params)))
+
+
+def _forward_workspace(params, workspace, device):
+    nbytes = pack3d_forward_workspace_bytes(params)
+    if workspace is None and nbytes:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    if workspace is None:
+        return None, 0
+    _need_cuda(workspace)
+    return workspace, workspace.numel() * workspace.element_size()
+
+
 def pack3d_forward(params: Params, index: IndexBuffers, q, k, v, ksum, vsum, out=None, lse=None,
-                   stream=None):
+                   workspace=None, stream=None):
     _need_cuda(q, k, v, ksum, vsum)
     B, N, H, d = _dims(params)
     out = torch.empty_like(q, dtype=out_dtype(params, q)) if out is None else out
     lse = torch.empty(B, H, N, dtype=torch.float32, device=q.device) if lse is None else lse
     _need_cuda(out, lse)
+    ws, nbytes = _forward_workspace(params, workspace, q.device)
     _check(load().pack3d_forward(ctypes.byref(params), ctypes.byref(index.struct), _ptr(q),
-                                 _ptr(k), _ptr(v), _ptr(ksum), _ptr(vsum), _ptr(out), _ptr(lse),
-                                 _stream(stream)), "pack3d_forward")
+                                 _ptr(k), _ptr(v), _ptr(ksum), _ptr(vsum),
+                                 None if ws is None else _ptr(ws), ctypes.c_size_t(nbytes),
+                                 _ptr(out), _ptr(lse), _stream(stream)), "pack3d_forward")
     return out, lse
 
 
 def pack3d_window_forward(params: Params, index: IndexBuffers, q, k, v, out=None, lse=None,
-                          stream=None):
+                          workspace=None, stream=None):
     _need_cuda(q, k, v)
     B, N, H, d = _dims(params)
     out = torch.empty_like(q, dtype=out_dtype(params, q)) if out is None else out
     lse = torch.empty(B, H, N, dtype=torch.float32, device=q.device) if lse is None else lse
     _need_cuda(out, lse)
+    ws, nbytes = _forward_workspace(params, workspace, q.device)
     _check(load().pack3d_window_forward(ctypes.byref(params), ctypes.byref(index.struct),
-                                        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                                        _ptr(q), _ptr(k), _ptr(v),
+                                        None if ws is None else _ptr(ws),
+                                        ctypes.c_size_t(nbytes), _ptr(out), _ptr(lse),
                                         _stream(stream)), "pack3d_window_forward")
+    return out, lse
+
+
+def pack3d_stage_kv(params: Params, index: IndexBuffers, k, v, ksum=None, vsum=None,
+                    workspace=None, stream=None):
+    """Stage rotated keys and values in grid order (and bf16 summaries) for
+    pack3d_forward_staged; returns the workspace."""
+    _need_cuda(k, v)
+    ws, nbytes = _forward_workspace(params, workspace, k.device)
+    _check(load().pack3d_stage_kv(ctypes.byref(params), ctypes.byref(index.struct), _ptr(k),
+                                  _ptr(v), None if ksum is None else _ptr(ksum),
+                                  None if vsum is None else _ptr(vsum),
+                                  None if ws is None else _ptr(ws), ctypes.c_size_t(nbytes),
+                                  _stream(stream)), "pack3d_stage_kv")
+    return ws
+
+
+def pack3d_forward_staged(params: Params, index: IndexBuffers, q, workspace, with_summaries=True,
+                          out=None, lse=None, stream=None):
+    _need_cuda(q, workspace)
+    B, N, H, d = _dims(params)
+    out = torch.empty_like(q, dtype=out_dtype(params, q)) if out is None else out
+    lse = torch.empty(B, H, N, dtype=torch.float32, device=q.device) if lse is None else lse
+    _need_cuda(out, lse)
+    _check(load().pack3d_forward_staged(ctypes.byref(params), ctypes.byref(index.struct), _ptr(q),
+                                        _ptr(workspace),
+                                        ctypes.c_size_t(workspace.numel() *
+                                                        workspace.element_size()),
+                                        int(bool(with_summaries)), _ptr(out), _ptr(lse),
+                                        _stream(stream)), "pack3d_forward_staged")
     return out, lse
 
 

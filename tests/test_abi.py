@@ -76,7 +76,7 @@ def test_null_pointers_rejected_without_cuda(lib):
     idx = P.Index()
     assert lib.pack3d_build_index(ctypes.byref(p), None, ctypes.byref(idx), None) == P.ERR_ARG
     assert lib.pack3d_forward(ctypes.byref(p), ctypes.byref(idx), None, None, None, None, None,
-                              None, None, None) == P.ERR_ARG
+                              None, ctypes.c_size_t(0), None, None, None) == P.ERR_ARG
     assert lib.pack3d_backward(ctypes.byref(p), None, *([None] * 10), ctypes.c_size_t(0),
                                None) == P.ERR_ARG
 
@@ -85,3 +85,28 @@ def test_strerror(lib):
     for st in (P.OK, P.ERR_ARG, P.ERR_COORDS, P.ERR_CUDA, P.ERR_TIMEOUT, P.ERR_UNSUPPORTED):
         assert P.strerror(st)
     assert P.strerror(12345) == "unknown status"
+
+
+def test_forward_workspace_size_and_checks(lib):
+    """The tensor-core forward's workspace: grid-order copies of the rotated
+    keys and of the values plus bf16 summary copies (256-byte aligned
+    sections); none for the CUDA-core paths.  A missing, short or misaligned
+    workspace is rejected before anything is launched."""
+    al = lambda x: (x + 255) // 256 * 256
+    p = P.make_params(shape())
+    vol = 2 * 8 * 32 * 32 * 64 * 96 * 2
+    summ = 2 * 8 * (4 * 4 * 8) * 96 * 2
+    need = lib.pack3d_forward_workspace_bytes(ctypes.byref(p))
+    assert need == 2 * al(vol) + 2 * al(summ)
+    assert lib.pack3d_forward_workspace_bytes(ctypes.byref(P.make_params(shape(dtype="fp32")))) == 0
+    assert lib.pack3d_forward_workspace_bytes(ctypes.byref(P.make_params(shape(d=48)))) == 0
+    idx = P.Index()
+    assert lib.pack3d_index_init(ctypes.byref(p), ctypes.c_void_p(1 << 20), ctypes.c_size_t(1 << 40),
+                                 ctypes.byref(idx)) == P.OK
+    fake = ctypes.c_void_p(1 << 30)
+    for ws, nbytes in ((None, need), (ctypes.c_void_p((1 << 32) + 16), need),
+                       (ctypes.c_void_p(1 << 32), need - 1)):
+        assert lib.pack3d_forward(ctypes.byref(p), ctypes.byref(idx), fake, fake, fake, fake, fake,
+                                  ws, ctypes.c_size_t(nbytes), fake, fake, None) == P.ERR_ARG
+        assert lib.pack3d_window_forward(ctypes.byref(p), ctypes.byref(idx), fake, fake, fake, ws,
+                                         ctypes.c_size_t(nbytes), fake, fake, None) == P.ERR_ARG
