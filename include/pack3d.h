@@ -186,18 +186,22 @@ PACK3D_API int pack3d_window_forward(const pack3d_params* p, const pack3d_index*
                                      pack3d_stream_t stream);
 
 /* The two halves of the tensor-core forward, for callers that run several
- * forwards against the same keys and values (or time the halves apart).
+ * forwards against the same keys and values, or that want the block
+ * summaries and the staging in one pass over k and v.
  * pack3d_stage_kv writes into the workspace the rotated keys and the values in
- * grid order and, when ksum and vsum are given (both or neither), bf16 copies
- * of the summaries.  pack3d_forward_staged then computes out and lse from q and
- * a workspace staged with the same params, k, v and index (with_summaries != 0:
- * the full operator, staged with summaries; 0: window only).
- * pack3d_forward = pack3d_stage_kv + pack3d_forward_staged.  Both return
- * PACK3D_ERR_UNSUPPORTED where pack3d_forward_workspace_bytes is 0, and
- * PACK3D_ERR_ARG for a missing, short or misaligned workspace. */
+ * grid order.  When ksum and vsum are given (both or neither) it also computes
+ * the block summaries in the same pass - OUTPUTS, the same values
+ * pack3d_block_summaries writes - and stages their bf16 copies.
+ * pack3d_forward_staged then computes out and lse from q and a workspace
+ * staged with the same params, k, v and index (with_summaries != 0: the full
+ * operator, which needs a staging with summaries; 0: window only).
+ * pack3d_forward = pack3d_stage_kv without summaries + staging of the given
+ * summaries + pack3d_forward_staged.  Both return PACK3D_ERR_UNSUPPORTED where
+ * pack3d_forward_workspace_bytes is 0, and PACK3D_ERR_ARG for a missing,
+ * short or misaligned workspace. */
 PACK3D_API int pack3d_stage_kv(const pack3d_params* p, const pack3d_index* idx, const void* k,
-                               const void* v, const float* ksum, const float* vsum,
-                               void* workspace, size_t workspace_bytes, pack3d_stream_t stream);
+                               const void* v, float* ksum, float* vsum, void* workspace,
+                               size_t workspace_bytes, pack3d_stream_t stream);
 PACK3D_API int pack3d_forward_staged(const pack3d_params* p, const pack3d_index* idx,
                                      const void* q, const void* workspace, size_t workspace_bytes,
                                      int with_summaries, void* out, float* lse,

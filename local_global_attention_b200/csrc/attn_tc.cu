@@ -27,13 +27,13 @@
 //       one of two TMEM S buffers, and O += P_j V_j (four tcgen05.mma, A = P
 //       from TMEM, B = V MN-major in shared memory), so S_{j+1} is computed
 //       while the softmax works on S_j;
-//     * softmax (warps 0-3, one query row per thread, warp w = tile plane w):
+//     * softmax (warps 0-3, one query row per thread, warp w = a 2 x 2 x 8 box):
 //       gather and rotate the query rows once; per chunk form the window mask
 //       from three per-query bit sets over the halo (z planes, y rows, x
 //       columns), read the chunk's 64 S values in one go, keep the online max
 //       and sum, write P (bf16) over S in TMEM.  A warp whose 32 queries see
-//       none of a chunk's keys (a z-plane pair outside their window) only
-//       writes zeros.  Summary chunks use the mask "block box does not meet the
+//       none of a chunk's keys (its plane or row pair outside their windows)
+//       only writes zeros.  Summary chunks use the mask "block box does not meet the
 //       window box"; there is no count bias.  The running max moves only when
 //       a row's maximum grows by more than 8 (log2 units), so O is rescaled in
 //       TMEM rarely; the result is the same softmax.
@@ -74,11 +74,23 @@ constexpr float LN2 = 0.6931471805599453f;
 constexpr float RESCALE_THRESHOLD = 8.0f;
 constexpr int ERR_TIMEOUT_BIT = 4;
 constexpr int MAX_HALO = 64;               // halo extent per axis the 64-bit masks cover
+// Window mask as 16 extra contraction channels of S = Q K^T ("penalty"
+// channels): a query row carries a one-hot of its tile-local z (4), y (4) and
+// x (8) position, a key row -2^14 in every channel whose tile position's window
+// misses it (all of them outside the volume), so a masked logit is at most
+// -2^14 (below -2400 in log2 units at tau = 96^-1/2) and its exponential is 0.
+constexpr uint16_t BF16_ONE = 0x3F80, BF16_PEN = 0xC680;  // 1.0, -16384.0
+// Floor of the running max (log2 units): a chunk whose keys are all masked
+// never raises it, so their exponentials stay 0.  Logits below this floor
+// (-693 in natural units) are outside the supported range.
+constexpr float M_FLOOR = -1000.0f;
 
 struct Smem {
   uint8_t q[3 * QSEG];
   uint8_t k[NSTAGE][3 * KSEG];
   uint8_t v[NSTAGE][3 * KSEG];
+  uint8_t qp[128 * 32];         // penalty channels of the query rows (32-byte swizzle)
+  uint8_t kp[NSTAGE][KCH * 32];  // penalty channels of each stage's key rows
   uint64_t q_full;
   uint64_t kv_full[NSTAGE];
   uint64_t kv_empty[NSTAGE];
@@ -261,6 +273,30 @@ __device__ __forceinline__ float exp_pack(const uint32_t (&sv)[32], uint32_t bit
   return (acc[0] + acc[1]) + (acc[2] + acc[3]);
 }
 
+// P = 2^(S c2 + mneg) for all 32 keys (masked ones carry the penalty), packed
+// in pairs into p[0..15]; returns the sum.
+__device__ __forceinline__ float exp_pack_all(const uint32_t (&sv)[32], float c2, float mneg,
+                                              uint32_t* p) {
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float e0 = ex2(fmaf(__uint_as_float(sv[2 * i]), c2, mneg));
+    const float e1 = ex2(fmaf(__uint_as_float(sv[2 * i + 1]), c2, mneg));
+    acc[i & 3] += e0 + e1;
+    p[i] = pack_bf16x2(e0, e1);
+  }
+  return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
+
+__device__ __forceinline__ float plain_max(const uint32_t (&sv)[32]) {
+  float m[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) m[i] = __uint_as_float(sv[i]);
+#pragma unroll
+  for (int i = 4; i < 32; ++i) m[i & 3] = fmaxf(m[i & 3], __uint_as_float(sv[i]));
+  return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+}
+
 // Maximum of S over the keys in `bits` (-inf if none), with independent chains.
 __device__ __forceinline__ float masked_max(const uint32_t (&sv)[32], uint32_t bits) {
   float m[4];
@@ -306,7 +342,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   if (tid == 0) {
     mbar_init(&sm.q_full, 128);
     for (int s = 0; s < NSTAGE; ++s) {
-      mbar_init(&sm.kv_full[s], 1);
+      mbar_init(&sm.kv_full[s], 2);  // TMA bytes + the penalty rows
       mbar_init(&sm.kv_empty[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -328,18 +364,21 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   const uint32_t tbase = sm.tmem_base;
 
   if (warp == TMA_WARP) {
-    // ================= TMA producer =================
+    // ================= TMA producer (lane 0) and penalty rows (all lanes) =================
     if (lane == 0) {
       tma_prefetch_map(&maps.kg);
       tma_prefetch_map(&maps.vg);
-      const int bh = b * g.H + h;
-      int xc = 0, yc = 0, zc = 0;
-      int issued = 0;
-      for (int j = 0; j < nch; ++j) {
-        const int s = j % NSTAGE, round = j / NSTAGE;
-        if (round > 0 &&
-            !mbar_wait_or_abort(&sm.kv_empty[s], (round - 1) & 1, WAIT_LIMIT, abort_flag))
-          break;
+    }
+    const int bh = b * g.H + h;
+    int xc = 0, yc = 0, zc = 0;
+    int issued = 0;
+    for (int j = 0; j < nch; ++j) {
+      const int s = j % NSTAGE, round = j / NSTAGE;
+      bool ok = true;
+      if (lane == 0 && round > 0)
+        ok = mbar_wait_or_abort(&sm.kv_empty[s], (round - 1) & 1, WAIT_LIMIT, abort_flag);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      if (lane == 0) {
         mbar_arrive_expect_tx(&sm.kv_full[s], CHUNK_BYTES);
         if (j < n_local) {
           const int x = tb.hx0 + BXK * xc, y = tb.hy0 + BYK * yc, z = tb.hz0 + BZK * zc;
@@ -347,13 +386,6 @@ __global__ void __launch_bounds__(NTHREADS, 2)
           for (int seg = 0; seg < 3; ++seg) {
             tma_load_5d(sm.k[s] + seg * KSEG, &maps.kg, seg * 32, x, y, z, bh, &sm.kv_full[s]);
             tma_load_5d(sm.v[s] + seg * KSEG, &maps.vg, seg * 32, x, y, z, bh, &sm.kv_full[s]);
-          }
-          if (++xc == nxc) {
-            xc = 0;
-            if (++yc == nyc) {
-              yc = 0;
-              ++zc;
-            }
           }
         } else {
           const int B0 = (j - n_local) * KCH;
@@ -363,13 +395,52 @@ __global__ void __launch_bounds__(NTHREADS, 2)
             tma_load_3d(sm.v[s] + seg * KSEG, &maps.vs, seg * 32, B0, bh, &sm.kv_full[s]);
           }
         }
-        issued = j + 1;
       }
-      // Copies still in flight must land before the CTA ends (bounded: they
-      // complete unless the memory system has failed).
+      if (j < n_local) {
+        // penalty rows of the chunk's keys (dz, dy, dx): key r = (dz * 2 + dy) * 16 + dx
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int r = lane + 32 * half;
+          const int kz = tb.hz0 + BZK * zc + (r >> 5), ky = tb.hy0 + BYK * yc + ((r >> 4) & 1),
+                    kx = tb.hx0 + BXK * xc + (r & 15);
+          const bool inside = kz < g.Z && ky < g.Y && kx < g.X;
+          uint32_t w[8];
+#pragma unroll
+          for (int a = 0; a < 4; a += 2) {
+            const uint32_t p0 = (!inside || abs(kz - (tb.z0 + a)) > g.rz) ? BF16_PEN : 0u;
+            const uint32_t p1 = (!inside || abs(kz - (tb.z0 + a + 1)) > g.rz) ? BF16_PEN : 0u;
+            w[a / 2] = p0 | (p1 << 16);
+            const uint32_t q0 = (!inside || abs(ky - (tb.y0 + a)) > g.ry) ? BF16_PEN : 0u;
+            const uint32_t q1 = (!inside || abs(ky - (tb.y0 + a + 1)) > g.ry) ? BF16_PEN : 0u;
+            w[2 + a / 2] = q0 | (q1 << 16);
+          }
+#pragma unroll
+          for (int a = 0; a < 8; a += 2) {
+            const uint32_t p0 = (!inside || abs(kx - (tb.x0 + a)) > g.rx) ? BF16_PEN : 0u;
+            const uint32_t p1 = (!inside || abs(kx - (tb.x0 + a + 1)) > g.rx) ? BF16_PEN : 0u;
+            w[4 + a / 2] = p0 | (p1 << 16);
+          }
+          *reinterpret_cast<uint4*>(sm.kp[s] + sw32_off(r, 0)) = make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(sm.kp[s] + sw32_off(r, 1)) = make_uint4(w[4], w[5], w[6], w[7]);
+        }
+        fence_proxy_async_smem();
+        if (++xc == nxc) {
+          xc = 0;
+          if (++yc == nyc) {
+            yc = 0;
+            ++zc;
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.kv_full[s]);
+      issued = j + 1;
+    }
+    // Copies still in flight must land before the CTA ends (bounded: they
+    // complete unless the memory system has failed).
+    if (lane == 0)
       for (int j = max(0, issued - NSTAGE); j < issued; ++j)
         mbar_wait(&sm.kv_full[j % NSTAGE], (j / NSTAGE) & 1, WAIT_LIMIT);
-    }
     __syncwarp();
   } else if (warp == MMA_WARP) {
     // ================= MMA issue =================
@@ -391,6 +462,9 @@ __global__ void __launch_bounds__(NTHREADS, 2)
           mma_ss(dst, sdesc_sw64(qa + (st >> 1) * QSEG + sub, 16, 512),
                  sdesc_sw64(ka + (st >> 1) * KSEG + sub, 16, 512), idesc_s, st > 0);
         }
+        if (j < n_local)  // + the window penalty (summary chunks are masked by the softmax)
+          mma_ss(dst, sdesc_sw32(smem_u32(sm.qp), 16, 256), sdesc_sw32(smem_u32(sm.kp[s]), 16, 256),
+                 idesc_s, 1u);
         mma_commit(&sm.s_full[j & 1]);
         return true;
       };
@@ -420,8 +494,12 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     __syncwarp();
   } else {
     // ================= softmax warps (one query row per thread) =================
-    // row tid = (plane tid / 32, row (tid / 8) % 4, column tid % 8) of the tile
-    const int lzi = tid >> 5, lyi = (tid >> 3) & 3, lxi = tid & 7;
+    // Row tid of the tile: warp w holds planes 2 (w / 2) + {0, 1}, rows
+    // 2 (w % 2) + {0, 1}, all 8 columns - a 2 x 2 x 8 box, whose windows meet
+    // only 4 of the 5 plane pairs and 4 of the 5 row pairs of an interior halo,
+    // so the warp skips about a third of the chunks.
+    const int lzi = (warp >> 1) * 2 + (lane >> 4), lyi = (warp & 1) * 2 + ((lane >> 3) & 1),
+              lxi = lane & 7;
     const bool active = lzi < tb.lz && lyi < tb.ly && lxi < tb.lx;
     const int cz = tb.z0 + lzi, cy = tb.y0 + lyi, cx = tb.x0 + lxi;
     int qi = 0;
@@ -450,6 +528,18 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       }
 #pragma unroll
       for (int i = 0; i < 12; ++i) store_chunk(sm.q, QSEG, tid, i, r[i]);
+      // penalty channels: one-hot of (z, y, x) within the tile
+      uint32_t w[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int c0 = 2 * i, c1 = 2 * i + 1;
+        auto hot = [&](int c) -> uint32_t {
+          return (c < 4 ? c == lzi : (c < 8 ? c - 4 == lyi : c - 8 == lxi)) ? BF16_ONE : 0u;
+        };
+        w[i] = hot(c0) | (hot(c1) << 16);
+      }
+      *reinterpret_cast<uint4*>(sm.qp + sw32_off(tid, 0)) = make_uint4(w[0], w[1], w[2], w[3]);
+      *reinterpret_cast<uint4*>(sm.qp + sw32_off(tid, 1)) = make_uint4(w[4], w[5], w[6], w[7]);
       fence_proxy_async_smem();
       mbar_arrive(&sm.q_full);
     }
@@ -464,7 +554,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     const uint32_t tO = tbase + lane_base + COL_O;
     const float c2 = g.tau * LOG2E;  // logits -> log2 units
-    float m_run = -INFINITY, l_run = 0.f;
+    float m_run = M_FLOOR, l_run = 0.f;
     RowCursor bc = {0, 0, 0};  // block rows (nbx blocks each, nby rows per plane)
     int xc = 0, yc = 0, zc = 0;
     bool ok = true;
@@ -514,23 +604,34 @@ __global__ void __launch_bounds__(NTHREADS, 2)
         tmem_ld32(tS, sa);
         tmem_ld32(tS + 32, sb);
         tmem_wait_ld();
-        const float cmax = fmaxf(masked_max(sa, bits0), masked_max(sb, bits1));
+        const bool local = j < n_local;  // masked by the penalty channels
+        const float cmax = local ? fmaxf(plain_max(sa), plain_max(sb))
+                                 : fmaxf(masked_max(sa, bits0), masked_max(sb, bits1));
         const float cmax2 = cmax * c2;
         float corr = 1.f;
+        bool rescale_o = false;
         if (cmax2 > m_run + RESCALE_THRESHOLD) {
-          if (m_run != -INFINITY) corr = ex2(m_run - cmax2);
+          corr = ex2(m_run - cmax2);
+          // O is exactly zero while l is (every P so far was 0)
+          rescale_o = l_run != 0.f;
           l_run *= corr;
           m_run = cmax2;
         }
-        const float mneg = m_run == -INFINITY ? 0.f : -m_run;
+        const float mneg = -m_run;
         // P over S: keys 0-63 -> columns 0-31 (S is already in registers)
         uint32_t p[32];
-        l_run += exp_pack(sa, bits0, c2, mneg, p);
-        l_run += exp_pack(sb, bits1, c2, mneg, p + 16);
+        if (local) {
+          l_run += exp_pack_all(sa, c2, mneg, p);
+          l_run += exp_pack_all(sb, c2, mneg, p + 16);
+        } else {
+          l_run += exp_pack(sa, bits0, c2, mneg, p);
+          l_run += exp_pack(sb, bits1, c2, mneg, p + 16);
+        }
         tmem_st32(tS, p);
         // rescale O before this chunk's PV product, which is issued only
         // after p_full below
-        if (__any_sync(0xffffffffu, corr != 1.f)) {
+        if (__any_sync(0xffffffffu, rescale_o)) {
+          const float co = rescale_o ? corr : 1.f;
           // O must hold every earlier PV product before it is rescaled
           ok = __all_sync(0xffffffffu,
                           mbar_wait_or_abort(&sm.o_done, (j - 1) & 1, WAIT_LIMIT, abort_flag));
@@ -542,7 +643,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
             tmem_ld32(tO + part * 32, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * corr);
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * co);
             tmem_st32(tO + part * 32, o);
           }
         }
@@ -676,14 +777,19 @@ size_t forward_tc_workspace_bytes(const Geo& g) {
 }
 
 int launch_stage_kv(const Geo& g, const pack3d_index* idx, const void* k, const void* v,
-                    const float* ksum, const float* vsum, void* ws, cudaStream_t s) {
+                    const float* ksum, const float* vsum, void* ws, StageMode mode,
+                    cudaStream_t s) {
   const WsLayout w = ws_layout(g);
   uint8_t* base = static_cast<uint8_t*>(ws);
+  if (mode == STAGE_COMPUTE)
+    return launch_block_summaries_staged(g, idx, k, v, const_cast<float*>(ksum),
+                                         const_cast<float*>(vsum), base + w.kg, base + w.vg,
+                                         base + w.ks, base + w.vs, s);
   dim3 ggrid((g.X + GRID_XS - 1) / GRID_XS, g.Z * g.Y, g.B);
   k_grid_kv<<<ggrid, 256, 0, s>>>(g, *idx, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
                                   reinterpret_cast<__nv_bfloat16*>(base + w.kg),
                                   reinterpret_cast<__nv_bfloat16*>(base + w.vg));
-  if (ksum && vsum) {
+  if (mode == STAGE_CONVERT) {
     const int64_t n4 = (int64_t)g.B * g.H * g.nb * D / 4;
     const int blocks = (int)std::min<int64_t>((n4 + 255) / 256, 148 * 8);
     k_summaries_bf16<<<blocks, 256, 0, s>>>((const float4*)ksum, (const float4*)vsum,

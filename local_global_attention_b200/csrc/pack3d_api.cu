@@ -190,14 +190,16 @@ static int forward_common(const pack3d_params* p, const pack3d_index* idx, const
   const size_t need = forward_tc_workspace_bytes(g);
   if (need) {
     if (!ws || ((uintptr_t)ws & 255) || ws_bytes < need) return PACK3D_ERR_ARG;
-    if ((rc = launch_stage_kv(g, idx, k, v, ksum, vsum, ws, s))) return rc;
+    if ((rc = launch_stage_kv(g, idx, k, v, ksum, vsum, ws,
+                              summaries ? STAGE_CONVERT : STAGE_NO_SUMMARIES, s)))
+      return rc;
     return launch_attention_tc(g, idx, q, ws, out, lse, summaries, s);
   }
   return launch_forward_simt(g, idx, q, k, v, ksum, vsum, out, lse, summaries, s);
 }
 
 int pack3d_stage_kv(const pack3d_params* p, const pack3d_index* idx, const void* k, const void* v,
-                    const float* ksum, const float* vsum, void* workspace, size_t workspace_bytes,
+                    float* ksum, float* vsum, void* workspace, size_t workspace_bytes,
                     pack3d_stream_t stream) {
   Geo g;
   int rc = make_geo(p, &g);
@@ -208,7 +210,8 @@ int pack3d_stage_kv(const pack3d_params* p, const pack3d_index* idx, const void*
   if (!k || !v || (!ksum != !vsum) || !workspace || ((uintptr_t)workspace & 255) ||
       workspace_bytes < need)
     return PACK3D_ERR_ARG;
-  return launch_stage_kv(g, idx, k, v, ksum, vsum, workspace, (cudaStream_t)stream);
+  return launch_stage_kv(g, idx, k, v, ksum, vsum, workspace,
+                         ksum ? STAGE_COMPUTE : STAGE_NO_SUMMARIES, (cudaStream_t)stream);
 }
 
 int pack3d_forward_staged(const pack3d_params* p, const pack3d_index* idx, const void* q,

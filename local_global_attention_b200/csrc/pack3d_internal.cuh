@@ -69,10 +69,19 @@ int launch_forward_simt(const Geo& g, const pack3d_index* idx, const void* q, co
                         float* lse, bool summaries, cudaStream_t s);
 bool forward_tc_supported(const Geo& g);
 size_t forward_tc_workspace_bytes(const Geo& g);  // 0 when the path does not apply
-// grid-order rotated keys and values (and bf16 summaries when ksum, vsum are
-// given) into the workspace; then the attention kernel reading them
+// Block summaries (bf16, head_dim 96) computed in the pass that also writes
+// the grid-order rotated keys and values and bf16 summary copies.
+int launch_block_summaries_staged(const Geo& g, const pack3d_index* idx, const void* k,
+                                  const void* v, float* ksum, float* vsum, void* kg, void* vg,
+                                  void* ksb, void* vsb, cudaStream_t s);
+// Staging of the tensor-core forward's workspace: grid-order rotated keys and
+// values, and the summaries' bf16 copies - converted from given summaries
+// (STAGE_CONVERT), computed in the same pass (STAGE_COMPUTE: ksum, vsum are
+// outputs), or left out (STAGE_NO_SUMMARIES).  Then the attention kernel.
+enum StageMode { STAGE_NO_SUMMARIES = 0, STAGE_CONVERT = 1, STAGE_COMPUTE = 2 };
 int launch_stage_kv(const Geo& g, const pack3d_index* idx, const void* k, const void* v,
-                    const float* ksum, const float* vsum, void* ws, cudaStream_t s);
+                    const float* ksum, const float* vsum, void* ws, StageMode mode,
+                    cudaStream_t s);
 int launch_attention_tc(const Geo& g, const pack3d_index* idx, const void* q, void* ws,
                         void* out, float* lse, bool summaries, cudaStream_t s);
 size_t backward_workspace_bytes(const Geo& g);

@@ -108,13 +108,25 @@ __global__ void __launch_bounds__(256) k_block_summaries(Geo g, const int32_t* _
 // voxel -> token lookups of the next tokens are issued before the current
 // tokens' arithmetic.  Partial sums of the 16 token groups are combined in a
 // fixed order.
+//
+// STAGE: the same pass also writes what the tensor-core forward reads - the
+// rotated key rows and the value rows in grid order ([b][h][z][y][x][96] bf16,
+// kg and vg) and bf16 copies of the summaries (ksb, vsb) - so k and v are read
+// from HBM once per step.  The rotated values written are the ones summed
+// (rounded to bf16 once), and the fp32 summaries are the same bits as without
+// STAGE.
+struct StageOut {
+  __nv_bfloat16 *kg, *vg, *ksb, *vsb;
+};
+
 constexpr int HG96 = 2, LANES96 = 6 * HG96, TG96 = 16, TAB96 = 48;
 constexpr int TABS96 = 18;  // staged row stride in float2 (16 + padding against bank conflicts)
 
+template <bool STAGE>
 __global__ void __launch_bounds__(TG96 * LANES96) k_block_summaries_bf16_d96(
     Geo g, const int32_t* __restrict__ vol, const float* __restrict__ rope,
     const int32_t* __restrict__ err, const __nv_bfloat16* __restrict__ k,
-    const __nv_bfloat16* __restrict__ v, float* ksum, float* vsum) {
+    const __nv_bfloat16* __restrict__ v, float* ksum, float* vsum, StageOut so) {
   if (err[0]) return;
   __shared__ float red[TG96][HG96][2][96];
   __shared__ float2 tab_s[TAB96 * TABS96];
@@ -181,21 +193,40 @@ __global__ void __launch_bounds__(TG96 * LANES96) k_block_summaries_bf16_d96(
       const uint32_t* kbw = reinterpret_cast<const uint32_t*>(&kb);
       const uint32_t* vaw = reinterpret_cast<const uint32_t*>(&va);
       const uint32_t* vbw = reinterpret_cast<const uint32_t*>(&vb2);
+      uint4 ra, rb;  // rotated chunks c1, c2 (bf16), for the grid-order copy
+      uint32_t* raw = reinterpret_cast<uint32_t*>(&ra);
+      uint32_t* rbw = reinterpret_cast<uint32_t*>(&rb);
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         float2 x1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(kaw + q));
         float2 x2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(kbw + q));
         const float4 cs = *reinterpret_cast<const float4*>(t + 2 * q);  // pairs j, j + 1
-        kx1[2 * q] += x1.x * cs.x - x2.x * cs.y;
-        kx2[2 * q] += x1.x * cs.y + x2.x * cs.x;
-        kx1[2 * q + 1] += x1.y * cs.z - x2.y * cs.w;
-        kx2[2 * q + 1] += x1.y * cs.w + x2.y * cs.z;
+        const float r1a = x1.x * cs.x - x2.x * cs.y, r2a = x1.x * cs.y + x2.x * cs.x;
+        const float r1b = x1.y * cs.z - x2.y * cs.w, r2b = x1.y * cs.w + x2.y * cs.z;
+        kx1[2 * q] += r1a;
+        kx2[2 * q] += r2a;
+        kx1[2 * q + 1] += r1b;
+        kx2[2 * q + 1] += r2b;
+        if (STAGE) {
+          __nv_bfloat162 pa = __floats2bfloat162_rn(r1a, r1b), pb = __floats2bfloat162_rn(r2a, r2b);
+          raw[q] = *reinterpret_cast<uint32_t*>(&pa);
+          rbw[q] = *reinterpret_cast<uint32_t*>(&pb);
+        }
         float2 y1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(vaw + q));
         float2 y2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(vbw + q));
         vx1[2 * q] += y1.x;
         vx1[2 * q + 1] += y1.y;
         vx2[2 * q] += y2.x;
         vx2[2 * q + 1] += y2.y;
+      }
+      if (STAGE) {
+        const int64_t grow = ((((int64_t)b * g.H + h) * g.Z + cz) * g.Y + cy) * g.X + cx;
+        uint4* kd = reinterpret_cast<uint4*>(so.kg + grow * 96);
+        uint4* vd = reinterpret_cast<uint4*>(so.vg + grow * 96);
+        kd[c1] = ra;
+        kd[c2] = rb;
+        vd[c1] = va;
+        vd[c2] = vb2;
       }
     }
     tok = ntok;
@@ -218,7 +249,9 @@ __global__ void __launch_bounds__(TG96 * LANES96) k_block_summaries_bf16_d96(
     float acc = 0.f;
     for (int q = 0; q < TG96; ++q) acc += red[q][oh][which][ch];
     const int64_t idx = (((int64_t)b * g.H + hout) * g.nb + blk) * 96 + ch;
-    (which ? vsum : ksum)[idx] = acc / (float)cnt;
+    const float mean = acc / (float)cnt;
+    (which ? vsum : ksum)[idx] = mean;
+    if (STAGE) (which ? so.vsb : so.ksb)[idx] = __float2bfloat16_rn(mean);
   }
 }
 
@@ -229,9 +262,9 @@ int launch_block_summaries(const Geo& g, const pack3d_index* idx, const void* k,
   dim3 grid(g.nb, g.B, g.H);
   if (g.dtype == PACK3D_BF16 && g.d == 96) {
     dim3 grid96(g.nb, g.B, (g.H + HG96 - 1) / HG96);
-    k_block_summaries_bf16_d96<<<grid96, TG96 * LANES96, 0, s>>>(
+    k_block_summaries_bf16_d96<false><<<grid96, TG96 * LANES96, 0, s>>>(
         g, idx->vol, idx->rope, idx->err, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, ksum,
-        vsum);
+        vsum, StageOut{});
     return cuda_status(cudaGetLastError());
   }
   int threads = TG * (g.d / 4);
@@ -244,6 +277,18 @@ int launch_block_summaries(const Geo& g, const pack3d_index* idx, const void* k,
     k_block_summaries<float><<<grid, threads, smem, s>>>(g, idx->vol, idx->rope, idx->err,
                                                          (const float*)k, (const float*)v, ksum,
                                                          vsum);
+  return cuda_status(cudaGetLastError());
+}
+
+int launch_block_summaries_staged(const Geo& g, const pack3d_index* idx, const void* k,
+                                  const void* v, float* ksum, float* vsum, void* kg, void* vg,
+                                  void* ksb, void* vsb, cudaStream_t s) {
+  if (g.dtype != PACK3D_BF16 || g.d != 96) return PACK3D_ERR_UNSUPPORTED;
+  dim3 grid96(g.nb, g.B, (g.H + HG96 - 1) / HG96);
+  StageOut so{(__nv_bfloat16*)kg, (__nv_bfloat16*)vg, (__nv_bfloat16*)ksb, (__nv_bfloat16*)vsb};
+  k_block_summaries_bf16_d96<true><<<grid96, TG96 * LANES96, 0, s>>>(
+      g, idx->vol, idx->rope, idx->err, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, ksum,
+      vsum, so);
   return cuda_status(cudaGetLastError());
 }
 

@@ -227,6 +227,19 @@ __device__ __forceinline__ uint64_t sdesc_sw64(uint32_t saddr, uint32_t lbo_byte
   return d;
 }
 
+// As sdesc_sw64 for rows of 32 bytes with the 32-byte swizzle (layout type 6;
+// stride byte offset = 8 rows x 32 bytes).
+__device__ __forceinline__ uint64_t sdesc_sw32(uint32_t saddr, uint32_t lbo_bytes,
+                                               uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)6 << 61;
+  return d;
+}
+
 // Instruction descriptor for kind::f16 with bf16 A and B, fp32 accumulate.
 // b_mn_major: B stored with N contiguous (MN-major).
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major) {
@@ -275,6 +288,13 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
 // The region must start on a 512-byte boundary.
 __device__ __forceinline__ uint32_t sw64_off(uint32_t r, uint32_t c) {
   return r * 64u + ((c ^ ((r >> 1) & 3u)) << 4);
+}
+
+// Byte offset of 16-byte chunk `c` (0..1) of row `r` in a region of 32-byte
+// rows with the 32-byte swizzle (chunk index XOR bit 2 of the row); the region
+// starts on a 256-byte boundary.
+__device__ __forceinline__ uint32_t sw32_off(uint32_t r, uint32_t c) {
+  return r * 32u + ((c ^ ((r >> 2) & 1u)) << 4);
 }
 
 // 2^x on the special-function unit (PTX ex2.approx.ftz.f32); 2^-inf = 0.

@@ -130,3 +130,34 @@ def test_forward_micro1m_sampled(oracle_lib):
     (b, h, i), out, lse = oracle_sample(wl, inp, 64, seed=7)
     assert_close(res["out"][b, i, h], out, wl.dtype, "out")
     assert_close(res["lse"][b, h, i], lse, wl.dtype, "lse")
+
+
+@pytest.mark.parametrize("wl", [RAGGED96, C.VOL16K], ids=lambda w: w.name)
+def test_staged_halves(oracle_lib, wl):
+    """pack3d_stage_kv with summaries computes the same summaries as
+    pack3d_block_summaries (bit for bit) and stages the same grid-order keys
+    and values as pack3d_forward does; pack3d_forward_staged then gives
+    pack3d_forward's result, and the window-only halves pack3d_window_forward's."""
+    inp = I.make_inputs(wl, "random")
+    d = {k: v.cuda() for k, v in inp.items() if k != "order"}
+    params = P.make_params(wl)
+    idx = P.pack3d_build_index(params, d["coords"])
+    ks_ref, vs_ref = P.pack3d_block_summaries(params, idx, d["k"], d["v"])
+    out_ref, lse_ref = P.pack3d_forward(params, idx, d["q"], d["k"], d["v"], ks_ref, vs_ref)
+    wout_ref, wlse_ref = P.pack3d_window_forward(params, idx, d["q"], d["k"], d["v"])
+    # staging alone (what pack3d_forward stages) vs staging fused with the summaries
+    ws_plain = P.pack3d_stage_kv(params, idx, d["k"], d["v"])
+    ks = torch.full_like(ks_ref, float("nan"))
+    vs = torch.full_like(vs_ref, float("nan"))
+    ws = P.pack3d_stage_kv(params, idx, d["k"], d["v"], ks, vs)
+    torch.cuda.synchronize()
+    assert torch.equal(ks, ks_ref) and torch.equal(vs, vs_ref)
+    kv_bytes = 2 * wl.B * wl.H * wl.N * wl.d * 2  # grid-order k and v (256-aligned here)
+    assert torch.equal(ws[:kv_bytes], ws_plain[:kv_bytes])
+    out, lse = P.pack3d_forward_staged(params, idx, d["q"], ws, with_summaries=True)
+    assert torch.equal(out, out_ref) and torch.equal(lse, lse_ref)
+    wout, wlse = P.pack3d_forward_staged(params, idx, d["q"], ws_plain, with_summaries=False)
+    assert torch.equal(wout, wout_ref) and torch.equal(wlse, wlse_ref)
+    assert P.pack3d_index_check(idx) == P.OK
+    ref = oracle.forward(wl, inp["coords"], inp["q"], inp["k"], inp["v"])
+    assert_close(out.cpu(), ref[0], wl.dtype, "out")
