@@ -58,13 +58,15 @@ using namespace tc;
 constexpr int D = 96;                      // head dim handled by this path
 constexpr int KCH = 64;                    // keys per chunk (N of the S MMA)
 constexpr int BXK = 16, BYK = 2, BZK = 2;  // chunk box (x, y, z) of the halo
-constexpr int NSTAGE = 3;                  // K/V shared-memory ring depth
-constexpr int QSEG = 128 * 64;             // one 32-channel segment of the 128 query rows
+constexpr int NSTAGE = 4;                  // K/V shared-memory ring depth
 constexpr int KSEG = KCH * 64;             // one 32-channel segment of a chunk
 constexpr uint32_t CHUNK_BYTES = 6 * KSEG; // K and V of one chunk
 constexpr uint32_t TMEM_COLS = 256;
-constexpr uint32_t COL_O = 0;              // O accumulator: columns [0, 96)
-constexpr uint32_t COL_S = 128;            // S/P buffer b: columns [128 + 64 b, 192 + 64 b)
+// Tensor memory (128 lanes = query rows, 256 columns of 32 bits):
+constexpr uint32_t COL_O = 0;              // O accumulator, fp32: columns [0, 96)
+constexpr uint32_t COL_P = 96;             // P, bf16 pairs: columns [96, 128)
+constexpr uint32_t COL_S = 128;            // S, fp32: columns [128, 192)
+constexpr uint32_t COL_Q = 192;            // rotated Q + penalty one-hot, bf16 pairs: [192, 248)
 constexpr int MMA_WARP = 4;
 constexpr int TMA_WARP = 5;
 constexpr int NTHREADS = 192;
@@ -86,17 +88,16 @@ constexpr uint16_t BF16_ONE = 0x3F80, BF16_PEN = 0xC680;  // 1.0, -16384.0
 constexpr float M_FLOOR = -1000.0f;
 
 struct Smem {
-  uint8_t q[3 * QSEG];
   uint8_t k[NSTAGE][3 * KSEG];
   uint8_t v[NSTAGE][3 * KSEG];
-  uint8_t qp[128 * 32];         // penalty channels of the query rows (32-byte swizzle)
-  uint8_t kp[NSTAGE][KCH * 32];  // penalty channels of each stage's key rows
-  uint64_t q_full;
+  uint8_t kp[NSTAGE][KCH * 32];  // penalty channels of each stage's key rows (32-byte swizzle)
+  uint64_t q_full;               // Q is in tensor memory
   uint64_t kv_full[NSTAGE];
   uint64_t kv_empty[NSTAGE];
-  uint64_t s_full[2];
-  uint64_t p_full[2];
-  uint64_t o_done;   // one phase per PV product
+  uint64_t s_full;   // one phase per chunk: S_j computed
+  uint64_t s_free;   // one phase per chunk: S_j read by the softmax
+  uint64_t p_full;   // one phase per chunk: P_j written
+  uint64_t o_done;   // one phase per PV product (P and O may be touched)
   uint64_t o_final;  // one phase: every PV product of the tile is done
   uint32_t tmem_base;
   int32_t abort;
@@ -275,17 +276,32 @@ __device__ __forceinline__ float exp_pack(const uint32_t (&sv)[32], uint32_t bit
 
 // P = 2^(S c2 + mneg) for all 32 keys (masked ones carry the penalty), packed
 // in pairs into p[0..15]; returns the sum.
+// The scaling and the running sums use the paired fp32 instructions
+// (fma/add.rn.f32x2: two values per instruction).
 __device__ __forceinline__ float exp_pack_all(const uint32_t (&sv)[32], float c2, float mneg,
                                               uint32_t* p) {
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  uint64_t acc[2] = {0ull, 0ull};
+  uint64_t cc, mm;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(cc) : "f"(c2));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(mm) : "f"(mneg));
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    const float e0 = ex2(fmaf(__uint_as_float(sv[2 * i]), c2, mneg));
-    const float e1 = ex2(fmaf(__uint_as_float(sv[2 * i + 1]), c2, mneg));
-    acc[i & 3] += e0 + e1;
+    uint64_t sp, a;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(sp) : "r"(sv[2 * i]), "r"(sv[2 * i + 1]));
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(a) : "l"(sp), "l"(cc), "l"(mm));
+    float a0, a1;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(a));
+    const float e0 = ex2(a0), e1 = ex2(a1);
+    uint64_t ep;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(ep) : "f"(e0), "f"(e1));
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(acc[i & 1]) : "l"(acc[i & 1]), "l"(ep));
     p[i] = pack_bf16x2(e0, e1);
   }
-  return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+  uint64_t t;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(t) : "l"(acc[0]), "l"(acc[1]));
+  float t0, t1;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(t0), "=f"(t1) : "l"(t));
+  return t0 + t1;
 }
 
 __device__ __forceinline__ float plain_max(const uint32_t (&sv)[32]) {
@@ -306,13 +322,6 @@ __device__ __forceinline__ float masked_max(const uint32_t (&sv)[32], uint32_t b
   for (int i = 0; i < 32; ++i)
     if ((bits >> i) & 1u) m[i & 3] = fmaxf(m[i & 3], __uint_as_float(sv[i]));
   return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
-}
-
-// 16-byte chunk c (0..11) of a 96-channel row -> its place in an operand region
-// (three 32-channel segments of seg_bytes each, 64-byte swizzle).
-__device__ __forceinline__ void store_chunk(uint8_t* region, int seg_bytes, int row, int c,
-                                            const uint4& v) {
-  *reinterpret_cast<uint4*>(region + (c >> 2) * seg_bytes + sw64_off(row, c & 3)) = v;
 }
 
 struct Maps {
@@ -345,10 +354,9 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       mbar_init(&sm.kv_full[s], 2);  // TMA bytes + the penalty rows
       mbar_init(&sm.kv_empty[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&sm.s_full[i], 1);
-      mbar_init(&sm.p_full[i], 128);
-    }
+    mbar_init(&sm.s_full, 1);
+    mbar_init(&sm.s_free, 128);
+    mbar_init(&sm.p_full, 128);
     mbar_init(&sm.o_done, 1);
     mbar_init(&sm.o_final, 1);
     sm.abort = 0;
@@ -445,50 +453,53 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   } else if (warp == MMA_WARP) {
     // ================= MMA issue =================
     if (lane == 0) {
-      const uint32_t qa = smem_u32(sm.q);
       constexpr uint32_t idesc_s = idesc_bf16(128, KCH, false);
       constexpr uint32_t idesc_o = idesc_bf16(128, D, true);
+      // Descriptors are formed once: a descriptor's low field is the address
+      // in 16-byte units, so an operand at a byte offset is the base
+      // descriptor plus offset / 16 (all shared-memory addresses < 256 KB).
+      const uint64_t kd0 = sdesc_sw64(smem_u32(sm.k[0]), 16, 512);
+      const uint64_t vd0 = sdesc_sw64(smem_u32(sm.v[0]), KSEG, 512);
+      const uint64_t kpd0 = sdesc_sw32(smem_u32(sm.kp[0]), 16, 256);
       bool ok = mbar_wait_or_abort(&sm.q_full, 0, WAIT_LIMIT, abort_flag);
+      // S_j = Q K_j^T: A = Q from tensor memory (8 columns per K = 16 step),
+      // B = the chunk's key rows (K-major, 64-byte swizzle)
       auto issue_s = [&](int j) -> bool {
         const int s = j % NSTAGE;
         if (!mbar_wait_or_abort(&sm.kv_full[s], (j / NSTAGE) & 1, WAIT_LIMIT, abort_flag))
           return false;
         tc_fence_after();
-        const uint32_t ka = smem_u32(sm.k[s]);
-        const uint32_t dst = tbase + COL_S + 64 * (j & 1);
+        const uint64_t kd = kd0 + (uint64_t)((s * 3 * KSEG) >> 4);
 #pragma unroll
-        for (int st = 0; st < D / 16; ++st) {
-          const uint32_t sub = (st & 1) * 32;
-          mma_ss(dst, sdesc_sw64(qa + (st >> 1) * QSEG + sub, 16, 512),
-                 sdesc_sw64(ka + (st >> 1) * KSEG + sub, 16, 512), idesc_s, st > 0);
-        }
+        for (int st = 0; st < D / 16; ++st)
+          mma_ts(tbase + COL_S, tbase + COL_Q + 8 * st,
+                 kd + (uint64_t)(((st >> 1) * KSEG + (st & 1) * 32) >> 4), idesc_s, st > 0);
         if (j < n_local)  // + the window penalty (summary chunks are masked by the softmax)
-          mma_ss(dst, sdesc_sw32(smem_u32(sm.qp), 16, 256), sdesc_sw32(smem_u32(sm.kp[s]), 16, 256),
+          mma_ts(tbase + COL_S, tbase + COL_Q + 48, kpd0 + (uint64_t)((s * KCH * 32) >> 4),
                  idesc_s, 1u);
-        mma_commit(&sm.s_full[j & 1]);
+        mma_commit(&sm.s_full);
         return true;
       };
-      if (ok) {
+      if (ok && nch > 0) {
         tc_fence_after();
-        for (int j = 0; j < nch && j < 2 && ok; ++j) ok = issue_s(j);
+        ok = issue_s(0);
       }
       for (int j = 0; j < nch && ok; ++j) {
-        if (!mbar_wait_or_abort(&sm.p_full[j & 1], (j >> 1) & 1, WAIT_LIMIT, abort_flag)) break;
+        // S_{j+1} once the softmax has read S_j: it runs while P_j is formed
+        if (j + 1 < nch) {
+          if (!mbar_wait_or_abort(&sm.s_free, j & 1, WAIT_LIMIT, abort_flag)) break;
+          if (!(ok = issue_s(j + 1))) break;
+        }
+        if (!mbar_wait_or_abort(&sm.p_full, j & 1, WAIT_LIMIT, abort_flag)) break;
         tc_fence_after();
-        const uint32_t va = smem_u32(sm.v[j % NSTAGE]);
-        const uint32_t pa = tbase + COL_S + 64 * (j & 1);
+        const uint64_t vd = vd0 + (uint64_t)(((j % NSTAGE) * 3 * KSEG) >> 4);
 #pragma unroll
         for (int st = 0; st < KCH / 16; ++st)
-          mma_ts(tbase + COL_O, pa + 8 * st, sdesc_sw64(va + st * 16 * 64, KSEG, 512), idesc_o,
-                 (j > 0 || st > 0) ? 1u : 0u);
+          mma_ts(tbase + COL_O, tbase + COL_P + 8 * st, vd + (uint64_t)((st * 16 * 64) >> 4),
+                 idesc_o, (j > 0 || st > 0) ? 1u : 0u);
         mma_commit(&sm.o_done);
         mma_commit(&sm.kv_empty[j % NSTAGE]);
         if (j == nch - 1) mma_commit(&sm.o_final);
-        if (j + 2 < nch) {
-          // S buffer j & 1 holds P_j until this PV has read it
-          if (!mbar_wait_or_abort(&sm.o_done, j & 1, WAIT_LIMIT, abort_flag)) break;
-          ok = issue_s(j + 2);
-        }
       }
     }
     __syncwarp();
@@ -526,8 +537,28 @@ __global__ void __launch_bounds__(NTHREADS, 2)
 #pragma unroll
         for (int i = 0; i < 12; ++i) r[i] = make_uint4(0, 0, 0, 0);
       }
+      // into this thread's tensor-memory lane: channel pairs in columns
+      // [COL_Q, COL_Q + 48), then the penalty channels
+      const uint32_t tq = tbase + ((uint32_t)(warp * 32) << 16) + COL_Q;
+      {
+        uint32_t w32[32], w16[16];
 #pragma unroll
-      for (int i = 0; i < 12; ++i) store_chunk(sm.q, QSEG, tid, i, r[i]);
+        for (int i = 0; i < 8; ++i) {
+          w32[4 * i] = r[i].x;
+          w32[4 * i + 1] = r[i].y;
+          w32[4 * i + 2] = r[i].z;
+          w32[4 * i + 3] = r[i].w;
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          w16[4 * i] = r[8 + i].x;
+          w16[4 * i + 1] = r[8 + i].y;
+          w16[4 * i + 2] = r[8 + i].z;
+          w16[4 * i + 3] = r[8 + i].w;
+        }
+        tmem_st32(tq, w32);
+        tmem_st16(tq + 32, w16);
+      }
       // penalty channels: one-hot of (z, y, x) within the tile
       uint32_t w[8];
 #pragma unroll
@@ -538,9 +569,9 @@ __global__ void __launch_bounds__(NTHREADS, 2)
         };
         w[i] = hot(c0) | (hot(c1) << 16);
       }
-      *reinterpret_cast<uint4*>(sm.qp + sw32_off(tid, 0)) = make_uint4(w[0], w[1], w[2], w[3]);
-      *reinterpret_cast<uint4*>(sm.qp + sw32_off(tid, 1)) = make_uint4(w[4], w[5], w[6], w[7]);
-      fence_proxy_async_smem();
+      tmem_st8(tq + 48, w);
+      tmem_wait_st();
+      tc_fence_before();
       mbar_arrive(&sm.q_full);
     }
     // The window as bit sets over halo-local positions (in-volume positions
@@ -553,21 +584,21 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     }
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     const uint32_t tO = tbase + lane_base + COL_O;
+    const uint32_t tP = tbase + lane_base + COL_P;
+    const uint32_t tS = tbase + lane_base + COL_S;
     const float c2 = g.tau * LOG2E;  // logits -> log2 units
     float m_run = M_FLOOR, l_run = 0.f;
     RowCursor bc = {0, 0, 0};  // block rows (nbx blocks each, nby rows per plane)
     int xc = 0, yc = 0, zc = 0;
     bool ok = true;
     for (int j = 0; j < nch; ++j) {
-      const int buf = j & 1;
       // a warp leaves together: the TMEM accesses below are warp-collective
       ok = __all_sync(0xffffffffu,
-                      mbar_wait_or_abort(&sm.s_full[buf], (j >> 1) & 1, WAIT_LIMIT, abort_flag));
+                      mbar_wait_or_abort(&sm.s_full, j & 1, WAIT_LIMIT, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      const uint32_t tS = tbase + lane_base + COL_S + 64 * buf;
       uint32_t bits0, bits1;
-      if (j < n_local) {
+      if (!SUMMARY || j < n_local) {
         // key (dz, dy, dx) of the chunk box is bit (dz * 2 + dy) * 16 + dx
         const uint32_t xp = (uint32_t)(xwin >> (BXK * xc)) & 0xffffu;
         const uint32_t yb = (uint32_t)(ywin >> (BYK * yc)) & 3u;
@@ -594,22 +625,27 @@ __global__ void __launch_bounds__(NTHREADS, 2)
         bits1 = summary_bits(bc, B0 + 32, g.nb, g.nbx, g.nby, bzlo, bzhi, bylo, byhi, bxlo, bxhi);
         if (!active) bits0 = bits1 = 0u;
       }
-      if (__ballot_sync(0xffffffffu, (bits0 | bits1) != 0u) == 0u) {
-        uint32_t zero[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) zero[i] = 0u;
-        tmem_st32(tS, zero);
-      } else {
-        uint32_t sa[32], sb[32];
+      const bool skip = __ballot_sync(0xffffffffu, (bits0 | bits1) != 0u) == 0u;
+      uint32_t sa[32], sb[32];
+      if (!skip) {
         tmem_ld32(tS, sa);
         tmem_ld32(tS + 32, sb);
         tmem_wait_ld();
-        const bool local = j < n_local;  // masked by the penalty channels
+      }
+      // S_j is in registers: the MMA may overwrite it with S_{j+1}
+      tc_fence_before();
+      mbar_arrive(&sm.s_free);
+      uint32_t p[32];
+      float corr = 1.f;
+      bool rescale_o = false;
+      if (skip) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) p[i] = 0u;
+      } else {
+        const bool local = !SUMMARY || j < n_local;  // masked by the penalty channels
         const float cmax = local ? fmaxf(plain_max(sa), plain_max(sb))
                                  : fmaxf(masked_max(sa, bits0), masked_max(sb, bits1));
         const float cmax2 = cmax * c2;
-        float corr = 1.f;
-        bool rescale_o = false;
         if (cmax2 > m_run + RESCALE_THRESHOLD) {
           corr = ex2(m_run - cmax2);
           // O is exactly zero while l is (every P so far was 0)
@@ -618,8 +654,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
           m_run = cmax2;
         }
         const float mneg = -m_run;
-        // P over S: keys 0-63 -> columns 0-31 (S is already in registers)
-        uint32_t p[32];
+        // keys 0-63 -> P columns 0-31
         if (local) {
           l_run += exp_pack_all(sa, c2, mneg, p);
           l_run += exp_pack_all(sb, c2, mneg, p + 16);
@@ -627,30 +662,31 @@ __global__ void __launch_bounds__(NTHREADS, 2)
           l_run += exp_pack(sa, bits0, c2, mneg, p);
           l_run += exp_pack(sb, bits1, c2, mneg, p + 16);
         }
-        tmem_st32(tS, p);
-        // rescale O before this chunk's PV product, which is issued only
-        // after p_full below
-        if (__any_sync(0xffffffffu, rescale_o)) {
-          const float co = rescale_o ? corr : 1.f;
-          // O must hold every earlier PV product before it is rescaled
-          ok = __all_sync(0xffffffffu,
-                          mbar_wait_or_abort(&sm.o_done, (j - 1) & 1, WAIT_LIMIT, abort_flag));
-          if (!ok) break;
-          tc_fence_after();
+      }
+      // P and O are free once PV_{j-1} is done (the MMA issues PV_j only after
+      // p_full below, so this phase is never two behind)
+      if (j > 0) {
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait_or_abort(&sm.o_done, (j - 1) & 1, WAIT_LIMIT, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+      }
+      tmem_st32(tP, p);
+      if (__any_sync(0xffffffffu, rescale_o)) {
+        const float co = rescale_o ? corr : 1.f;
 #pragma unroll 1
-          for (int part = 0; part < 3; ++part) {
-            uint32_t o[32];
-            tmem_ld32(tO + part * 32, o);
-            tmem_wait_ld();
+        for (int part = 0; part < 6; ++part) {
+          uint32_t o[16];
+          tmem_ld16(tO + part * 16, o);
+          tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * co);
-            tmem_st32(tO + part * 32, o);
-          }
+          for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * co);
+          tmem_st16(tO + part * 16, o);
         }
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&sm.p_full[buf]);
+      mbar_arrive(&sm.p_full);
     }
     // ---- epilogue ----
     // o_final completes once, after the last PV product.  (Waiting on o_done
