@@ -349,14 +349,14 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   const int nch = n_local + n_sum;
 
   if (tid == 0) {
-    mbar_init(&sm.q_full, 128);
+    mbar_init(&sm.q_full, 4);  // softmax barriers: one arrival per softmax warp
     for (int s = 0; s < NSTAGE; ++s) {
       mbar_init(&sm.kv_full[s], 2);  // TMA bytes + the penalty rows
       mbar_init(&sm.kv_empty[s], 1);
     }
     mbar_init(&sm.s_full, 1);
-    mbar_init(&sm.s_free, 128);
-    mbar_init(&sm.p_full, 128);
+    mbar_init(&sm.s_free, 4);
+    mbar_init(&sm.p_full, 4);
     mbar_init(&sm.o_done, 1);
     mbar_init(&sm.o_final, 1);
     sm.abort = 0;
@@ -451,8 +451,8 @@ __global__ void __launch_bounds__(NTHREADS, 2)
         mbar_wait(&sm.kv_full[j % NSTAGE], (j / NSTAGE) & 1, WAIT_LIMIT);
     __syncwarp();
   } else if (warp == MMA_WARP) {
-    // ================= MMA issue =================
-    if (lane == 0) {
+    // ================= MMA issue (the whole warp, converged; one lane issues) =================
+    {
       constexpr uint32_t idesc_s = idesc_bf16(128, KCH, false);
       constexpr uint32_t idesc_o = idesc_bf16(128, D, true);
       // Descriptors are formed once: a descriptor's low field is the address
@@ -461,23 +461,25 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       const uint64_t kd0 = sdesc_sw64(smem_u32(sm.k[0]), 16, 512);
       const uint64_t vd0 = sdesc_sw64(smem_u32(sm.v[0]), KSEG, 512);
       const uint64_t kpd0 = sdesc_sw32(smem_u32(sm.kp[0]), 16, 256);
-      bool ok = mbar_wait_or_abort(&sm.q_full, 0, WAIT_LIMIT, abort_flag);
+      auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, mbar_wait_or_abort(bar, parity, WAIT_LIMIT, abort_flag));
+      };
+      bool ok = wait_all(&sm.q_full, 0);
       // S_j = Q K_j^T: A = Q from tensor memory (8 columns per K = 16 step),
       // B = the chunk's key rows (K-major, 64-byte swizzle)
       auto issue_s = [&](int j) -> bool {
         const int s = j % NSTAGE;
-        if (!mbar_wait_or_abort(&sm.kv_full[s], (j / NSTAGE) & 1, WAIT_LIMIT, abort_flag))
-          return false;
+        if (!wait_all(&sm.kv_full[s], (j / NSTAGE) & 1)) return false;
         tc_fence_after();
         const uint64_t kd = kd0 + (uint64_t)((s * 3 * KSEG) >> 4);
 #pragma unroll
         for (int st = 0; st < D / 16; ++st)
-          mma_ts(tbase + COL_S, tbase + COL_Q + 8 * st,
-                 kd + (uint64_t)(((st >> 1) * KSEG + (st & 1) * 32) >> 4), idesc_s, st > 0);
+          mma_ts_warp(tbase + COL_S, tbase + COL_Q + 8 * st,
+                      kd + (uint64_t)(((st >> 1) * KSEG + (st & 1) * 32) >> 4), idesc_s, st > 0);
         if (j < n_local)  // + the window penalty (summary chunks are masked by the softmax)
-          mma_ts(tbase + COL_S, tbase + COL_Q + 48, kpd0 + (uint64_t)((s * KCH * 32) >> 4),
-                 idesc_s, 1u);
-        mma_commit(&sm.s_full);
+          mma_ts_warp(tbase + COL_S, tbase + COL_Q + 48, kpd0 + (uint64_t)((s * KCH * 32) >> 4),
+                      idesc_s, 1u);
+        mma_commit_warp(&sm.s_full);
         return true;
       };
       if (ok && nch > 0) {
@@ -487,19 +489,19 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       for (int j = 0; j < nch && ok; ++j) {
         // S_{j+1} once the softmax has read S_j: it runs while P_j is formed
         if (j + 1 < nch) {
-          if (!mbar_wait_or_abort(&sm.s_free, j & 1, WAIT_LIMIT, abort_flag)) break;
+          if (!wait_all(&sm.s_free, j & 1)) break;
           if (!(ok = issue_s(j + 1))) break;
         }
-        if (!mbar_wait_or_abort(&sm.p_full, j & 1, WAIT_LIMIT, abort_flag)) break;
+        if (!wait_all(&sm.p_full, j & 1)) break;
         tc_fence_after();
         const uint64_t vd = vd0 + (uint64_t)(((j % NSTAGE) * 3 * KSEG) >> 4);
 #pragma unroll
         for (int st = 0; st < KCH / 16; ++st)
-          mma_ts(tbase + COL_O, tbase + COL_P + 8 * st, vd + (uint64_t)((st * 16 * 64) >> 4),
-                 idesc_o, (j > 0 || st > 0) ? 1u : 0u);
-        mma_commit(&sm.o_done);
-        mma_commit(&sm.kv_empty[j % NSTAGE]);
-        if (j == nch - 1) mma_commit(&sm.o_final);
+          mma_ts_warp(tbase + COL_O, tbase + COL_P + 8 * st, vd + (uint64_t)((st * 16 * 64) >> 4),
+                      idesc_o, (j > 0 || st > 0) ? 1u : 0u);
+        mma_commit_warp(&sm.o_done);
+        mma_commit_warp(&sm.kv_empty[j % NSTAGE]);
+        if (j == nch - 1) mma_commit_warp(&sm.o_final);
       }
     }
     __syncwarp();
@@ -572,7 +574,8 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       tmem_st8(tq + 48, w);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&sm.q_full);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.q_full);
     }
     // The window as bit sets over halo-local positions (in-volume positions
     // only, so zero-filled keys outside the volume are never selected).
@@ -634,7 +637,8 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       }
       // S_j is in registers: the MMA may overwrite it with S_{j+1}
       tc_fence_before();
-      mbar_arrive(&sm.s_free);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.s_free);
       uint32_t p[32];
       float corr = 1.f;
       bool rescale_o = false;
@@ -686,7 +690,8 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&sm.p_full);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.p_full);
     }
     // ---- epilogue ----
     // o_final completes once, after the last PV product.  (Waiting on o_done

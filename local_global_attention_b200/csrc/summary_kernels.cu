@@ -170,69 +170,90 @@ __global__ void __launch_bounds__(TG96 * LANES96) k_block_summaries_bf16_d96(
     cy = By * g.by + (e / g.bx) % g.by;
     cz = Bz * g.bz + e / (g.bx * g.by);
   };
-  int e = grp, cz, cy, cx;
-  voxel(e, cz, cy, cx);
-  int tok = (live && e < cnt) ? vb[(cz * g.Y + cy) * g.X + cx] : 0;
-  for (; e < cnt; e += TG96) {
-    // next token's lookup first
-    const int en = e + TG96;
-    int nz = 0, ny = 0, nx = 0, ntok = 0;
-    if (en < cnt) {
-      voxel(en, nz, ny, nx);
-      if (live) ntok = vb[(nz * g.Y + ny) * g.X + nx];
-    }
-    if (live) {
-      const int64_t row = (((int64_t)b * g.N + tok) * g.H + h) * 96;
-      const uint4* kr = reinterpret_cast<const uint4*>(k + row);
-      const uint4* vr = reinterpret_cast<const uint4*>(v + row);
-      const uint4 ka = __ldg(kr + c1), kb = __ldg(kr + c2), va = __ldg(vr + c1),
-                  vb2 = __ldg(vr + c2);
-      const int ca = a == 0 ? cz : (a == 1 ? cy : cx);
-      const float2* t = tab + (ca - base) * stride + j0;
-      const uint32_t* kaw = reinterpret_cast<const uint32_t*>(&ka);
-      const uint32_t* kbw = reinterpret_cast<const uint32_t*>(&kb);
-      const uint32_t* vaw = reinterpret_cast<const uint32_t*>(&va);
-      const uint32_t* vbw = reinterpret_cast<const uint32_t*>(&vb2);
-      uint4 ra, rb;  // rotated chunks c1, c2 (bf16), for the grid-order copy
-      uint32_t* raw = reinterpret_cast<uint32_t*>(&ra);
-      uint32_t* rbw = reinterpret_cast<uint32_t*>(&rb);
+  // One token's rows (already loaded): rotate, accumulate, and with STAGE
+  // write the grid-order copies.
+  auto consume = [&](const uint4& ka, const uint4& kb, const uint4& va, const uint4& vb2, int cz,
+                     int cy, int cx) {
+    const int ca = a == 0 ? cz : (a == 1 ? cy : cx);
+    const float2* t = tab + (ca - base) * stride + j0;
+    const uint32_t* kaw = reinterpret_cast<const uint32_t*>(&ka);
+    const uint32_t* kbw = reinterpret_cast<const uint32_t*>(&kb);
+    const uint32_t* vaw = reinterpret_cast<const uint32_t*>(&va);
+    const uint32_t* vbw = reinterpret_cast<const uint32_t*>(&vb2);
+    uint4 ra, rb;  // rotated chunks c1, c2 (bf16), for the grid-order copy
+    uint32_t* raw = reinterpret_cast<uint32_t*>(&ra);
+    uint32_t* rbw = reinterpret_cast<uint32_t*>(&rb);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float2 x1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(kaw + q));
-        float2 x2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(kbw + q));
-        const float4 cs = *reinterpret_cast<const float4*>(t + 2 * q);  // pairs j, j + 1
-        const float r1a = x1.x * cs.x - x2.x * cs.y, r2a = x1.x * cs.y + x2.x * cs.x;
-        const float r1b = x1.y * cs.z - x2.y * cs.w, r2b = x1.y * cs.w + x2.y * cs.z;
-        kx1[2 * q] += r1a;
-        kx2[2 * q] += r2a;
-        kx1[2 * q + 1] += r1b;
-        kx2[2 * q + 1] += r2b;
-        if (STAGE) {
-          __nv_bfloat162 pa = __floats2bfloat162_rn(r1a, r1b), pb = __floats2bfloat162_rn(r2a, r2b);
-          raw[q] = *reinterpret_cast<uint32_t*>(&pa);
-          rbw[q] = *reinterpret_cast<uint32_t*>(&pb);
-        }
-        float2 y1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(vaw + q));
-        float2 y2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(vbw + q));
-        vx1[2 * q] += y1.x;
-        vx1[2 * q + 1] += y1.y;
-        vx2[2 * q] += y2.x;
-        vx2[2 * q + 1] += y2.y;
-      }
+    for (int q = 0; q < 4; ++q) {
+      float2 x1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(kaw + q));
+      float2 x2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(kbw + q));
+      const float4 cs = *reinterpret_cast<const float4*>(t + 2 * q);  // pairs j, j + 1
+      const float r1a = x1.x * cs.x - x2.x * cs.y, r2a = x1.x * cs.y + x2.x * cs.x;
+      const float r1b = x1.y * cs.z - x2.y * cs.w, r2b = x1.y * cs.w + x2.y * cs.z;
+      kx1[2 * q] += r1a;
+      kx2[2 * q] += r2a;
+      kx1[2 * q + 1] += r1b;
+      kx2[2 * q + 1] += r2b;
       if (STAGE) {
-        const int64_t grow = ((((int64_t)b * g.H + h) * g.Z + cz) * g.Y + cy) * g.X + cx;
-        uint4* kd = reinterpret_cast<uint4*>(so.kg + grow * 96);
-        uint4* vd = reinterpret_cast<uint4*>(so.vg + grow * 96);
-        kd[c1] = ra;
-        kd[c2] = rb;
-        vd[c1] = va;
-        vd[c2] = vb2;
+        __nv_bfloat162 pa = __floats2bfloat162_rn(r1a, r1b), pb = __floats2bfloat162_rn(r2a, r2b);
+        raw[q] = *reinterpret_cast<uint32_t*>(&pa);
+        rbw[q] = *reinterpret_cast<uint32_t*>(&pb);
       }
+      float2 y1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(vaw + q));
+      float2 y2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(vbw + q));
+      vx1[2 * q] += y1.x;
+      vx1[2 * q + 1] += y1.y;
+      vx2[2 * q] += y2.x;
+      vx2[2 * q + 1] += y2.y;
     }
-    tok = ntok;
-    cz = nz;
-    cy = ny;
-    cx = nx;
+    if (STAGE) {
+      const int64_t grow = ((((int64_t)b * g.H + h) * g.Z + cz) * g.Y + cy) * g.X + cx;
+      uint4* kd = reinterpret_cast<uint4*>(so.kg + grow * 96);
+      uint4* vd = reinterpret_cast<uint4*>(so.vg + grow * 96);
+      kd[c1] = ra;
+      kd[c2] = rb;
+      vd[c1] = va;
+      vd[c2] = vb2;
+    }
+  };
+  auto lookup = [&](int e, int& cz, int& cy, int& cx) -> int {
+    if (e >= cnt) return 0;
+    voxel(e, cz, cy, cx);
+    return live ? vb[(cz * g.Y + cy) * g.X + cx] : 0;
+  };
+  // Tokens e and e + TG96 per iteration (their loads in flight together), the
+  // next pair's lookups issued first; each thread still adds its tokens in
+  // the order e, e + TG96, e + 2 TG96, ...
+  int az = 0, ay = 0, ax = 0, bz2 = 0, by2 = 0, bx2 = 0;
+  int ta = lookup(grp, az, ay, ax), tb2 = lookup(grp + TG96, bz2, by2, bx2);
+  for (int e = grp; e < cnt; e += 2 * TG96) {
+    const bool has_b = e + TG96 < cnt;
+    int naz = 0, nay = 0, nax = 0, nbz = 0, nby = 0, nbx = 0;
+    const int nta = lookup(e + 2 * TG96, naz, nay, nax);
+    const int ntb = lookup(e + 3 * TG96, nbz, nby, nbx);
+    if (live) {
+      const uint4* kra = reinterpret_cast<const uint4*>(k + (((int64_t)b * g.N + ta) * g.H + h) * 96);
+      const uint4* vra = reinterpret_cast<const uint4*>(v + (((int64_t)b * g.N + ta) * g.H + h) * 96);
+      const uint4 ka = __ldg(kra + c1), kb = __ldg(kra + c2), va = __ldg(vra + c1),
+                  vb2 = __ldg(vra + c2);
+      uint4 kbA = make_uint4(0, 0, 0, 0), kbB = kbA, vbA = kbA, vbB = kbA;
+      if (has_b) {
+        const uint4* krb =
+            reinterpret_cast<const uint4*>(k + (((int64_t)b * g.N + tb2) * g.H + h) * 96);
+        const uint4* vrb =
+            reinterpret_cast<const uint4*>(v + (((int64_t)b * g.N + tb2) * g.H + h) * 96);
+        kbA = __ldg(krb + c1);
+        kbB = __ldg(krb + c2);
+        vbA = __ldg(vrb + c1);
+        vbB = __ldg(vrb + c2);
+      }
+      consume(ka, kb, va, vb2, az, ay, ax);
+      if (has_b) consume(kbA, kbB, vbA, vbB, bz2, by2, bx2);
+    }
+    ta = nta;
+    tb2 = ntb;
+    az = naz; ay = nay; ax = nax;
+    bz2 = nbz; by2 = nby; bx2 = nbx;
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
