@@ -156,6 +156,8 @@ class ClockSampler:
 
 
 def dist_setup(n_gpus):
+    """One process per GPU (torchrun env).  NCCL on GPUs; gloo where there is
+    none (the CPU tests of this host logic)."""
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -163,9 +165,13 @@ def dist_setup(n_gpus):
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        timeout = datetime.timedelta(seconds=120)
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=timeout,
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=timeout)
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return world, rank, local
@@ -178,13 +184,26 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """Maximum of a per-rank time over all ranks (every rank gets it)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_workload(wl, rank):
+    """Weak scaling: every rank runs its own batch of the same shape (seed
+    offset by the rank), so there is no data-path collective."""
+    return wl.replace(seed=wl.seed + 1000 * rank)
+
+
+def whole_job_rate(tokens_per_rank, world, ms):
+    """Tokens/s of the whole job: all ranks' tokens over the slowest rank's time."""
+    return tokens_per_rank * world / (ms * 1e-3)
 
 
 def run_ours(args):
@@ -195,8 +214,7 @@ def run_ours(args):
 
     world, rank, local = dist_setup(args.gpus)
     wl = workload(args.workload)
-    # weak scaling: each rank its own batch (seed offset by rank)
-    wl_r = wl.replace(seed=wl.seed + 1000 * rank)
+    wl_r = rank_workload(wl, rank)
     inp = I.make_inputs(wl_r, args.packing)
     dev = {k: v.cuda() for k, v in inp.items() if k != "order"}
     params = P.make_params(wl_r)
@@ -301,7 +319,7 @@ def run_ours(args):
     traffic = profile_traffic()
     line = {
         "metric": METRIC,
-        "value": tokens / (ms * 1e-3),
+        "value": whole_job_rate(B * N, world, ms),
         "unit": UNIT,
         "n_gpus": world,
         "steps": args.steps,
@@ -383,7 +401,8 @@ def run_reference(args):
     oracle.build()
     ks, vs = oracle.block_summaries(wl, inp["coords"], inp["k"], inp["v"])
     rng = np.random.default_rng(1)
-    n = args.cpu_sample // 4 or 1
+    # sample per step sized so that the whole run takes about a minute of CPU
+    n = 256
 
     def one():
         b = rng.integers(0, wl.B, n)
@@ -395,6 +414,9 @@ def run_reference(args):
                        summaries=(ks, vs))
         return time.perf_counter() - t0
 
+    per_tok = one() / n  # calibration
+    n = int(max(16, min(args.cpu_sample // 4, 60.0 / max(per_tok, 1e-9) /
+                        (args.steps + args.warmup))))
     for _ in range(args.warmup):
         one()
     times = [one() for _ in range(args.steps)]

@@ -1,0 +1,74 @@
+"""Multi-rank host logic of bench.py on CPU (gloo, world size 2).
+
+The benchmark runs one process per GPU with independent batches (weak scaling,
+no data-path collective); its only collectives are barriers and the maximum of
+the per-rank times.  These tests run that logic as two gloo ranks."""
+import io
+import json
+import os
+import socket
+import sys
+from contextlib import redirect_stdout
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+
+def free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def worker(rank, world, port, out_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      LOCAL_RANK=str(rank), WORLD_SIZE=str(world))
+    import torch.distributed as dist
+
+    import bench
+    from local_global_attention_b200 import configs as C
+    w, r, local = bench.dist_setup(world)
+    assert (w, r, local) == (world, rank, rank)
+    assert dist.get_backend() == "gloo"
+    # every rank gets the maximum of the per-rank times
+    t = bench.max_over_ranks(10.0 + rank, w)
+    bench.barrier(w)
+    wl = bench.rank_workload(C.VOL65K, rank)
+    with open(os.path.join(out_dir, f"rank{rank}.json"), "w") as f:
+        json.dump({"max": t, "seed": wl.seed, "shape": [wl.B, wl.H, wl.Z, wl.Y, wl.X]}, f)
+    bench.barrier(w)
+    dist.destroy_process_group()
+
+
+def test_two_gloo_ranks(tmp_path):
+    world = 2
+    mp.spawn(worker, args=(world, free_port(), str(tmp_path)), nprocs=world, join=True)
+    res = [json.load(open(tmp_path / f"rank{r}.json")) for r in range(world)]
+    # max over ranks, seen by every rank
+    assert all(r["max"] == 11.0 for r in res)
+    # weak scaling: same shape, different batches
+    assert res[0]["shape"] == res[1]["shape"]
+    assert res[0]["seed"] != res[1]["seed"]
+
+
+def test_whole_job_rate_counts_all_ranks():
+    import bench
+    # 131,072 tokens per rank, 4 ranks, slowest rank 2 ms
+    assert bench.whole_job_rate(131072, 4, 2.0) == pytest.approx(131072 * 4 / 2e-3)
+
+
+def test_reference_arm_only_on_rank_zero(monkeypatch):
+    """Under torchrun the oracle arm runs on rank 0 alone; other ranks exit
+    without work or output."""
+    import bench
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setenv("RANK", "1")
+    args = type("A", (), dict(workload="vol_32x32x64", packing="random", steps=1, warmup=3,
+                              cpu_sample=64))()
+    buf = io.StringIO()
+    with redirect_stdout(buf):
+        bench.run_reference(args)
+    assert buf.getvalue() == ""
