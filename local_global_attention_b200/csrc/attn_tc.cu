@@ -826,10 +826,16 @@ int launch_stage_kv(const Geo& g, const pack3d_index* idx, const void* k, const 
     return launch_block_summaries_staged(g, idx, k, v, const_cast<float*>(ksum),
                                          const_cast<float*>(vsum), base + w.kg, base + w.vg,
                                          base + w.ks, base + w.vs, s);
-  dim3 ggrid((g.X + GRID_XS - 1) / GRID_XS, g.Z * g.Y, g.B);
-  k_grid_kv<<<ggrid, 256, 0, s>>>(g, *idx, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
-                                  reinterpret_cast<__nv_bfloat16*>(base + w.kg),
-                                  reinterpret_cast<__nv_bfloat16*>(base + w.vg));
+  // staging alone: the summary kernel's bulk gather where it applies
+  int rc = launch_stage_bulk(g, idx, k, v, base + w.kg, base + w.vg, s);
+  if (rc == PACK3D_ERR_UNSUPPORTED) {
+    dim3 ggrid((g.X + GRID_XS - 1) / GRID_XS, g.Z * g.Y, g.B);
+    k_grid_kv<<<ggrid, 256, 0, s>>>(g, *idx, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
+                                    reinterpret_cast<__nv_bfloat16*>(base + w.kg),
+                                    reinterpret_cast<__nv_bfloat16*>(base + w.vg));
+  } else if (rc) {
+    return rc;
+  }
   if (mode == STAGE_CONVERT) {
     const int64_t n4 = (int64_t)g.B * g.H * g.nb * D / 4;
     const int blocks = (int)std::min<int64_t>((n4 + 255) / 256, 148 * 8);

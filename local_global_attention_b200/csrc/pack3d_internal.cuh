@@ -74,6 +74,10 @@ size_t forward_tc_workspace_bytes(const Geo& g);  // 0 when the path does not ap
 int launch_block_summaries_staged(const Geo& g, const pack3d_index* idx, const void* k,
                                   const void* v, float* ksum, float* vsum, void* kg, void* vg,
                                   void* ksb, void* vsb, cudaStream_t s);
+// Grid-order rotated keys and values alone (bf16, head_dim 96, up to 8
+// heads: PACK3D_ERR_UNSUPPORTED otherwise), by the summary kernel's gather.
+int launch_stage_bulk(const Geo& g, const pack3d_index* idx, const void* k, const void* v,
+                      void* kg, void* vg, cudaStream_t s);
 // Staging of the tensor-core forward's workspace: grid-order rotated keys and
 // values, and the summaries' bf16 copies - converted from given summaries
 // (STAGE_CONVERT), computed in the same pass (STAGE_COMPUTE: ksum, vsum are

@@ -15,6 +15,7 @@
 // Tokens are visited through the coordinate volume in block raster order, so
 // the accumulation order, and the result, do not depend on the packing.
 #include "pack3d_internal.cuh"
+#include "tc_primitives.cuh"
 
 namespace p3d {
 
@@ -278,10 +279,230 @@ __global__ void __launch_bounds__(TG96 * LANES96) k_block_summaries_bf16_d96(
 
 }  // namespace
 
+// bf16, head_dim 96, up to 8 heads: the block's token rows (all heads, k and
+// v: 2 x H x 192 bytes per token) are gathered through the volume with bulk
+// asynchronous copies into a shared-memory ring (BS_STAGES stages of BS_TPS
+// tokens) by one producer warp, so 32 tokens per CTA are in flight; twelve
+// consumer warps take thread (group g, item c): token g of each stage, item
+// c = (head, segment, half) - 8 channels of k and their 8 rotation partners,
+// and the same channels of v.  A thread adds its tokens in block-raster order
+// (g, g + 8, ...), the 8 groups are then summed in order, so the result does
+// not depend on the packing.  With STAGE the rotated key rows and the value
+// rows are also written in grid order with bf16 copies of the summaries.  Null
+// summary pointers skip those outputs (staging alone).
+constexpr int BS_TPS = 8, BS_STAGES = 4, BS_MAXH = 8;
+constexpr int BS_ITEMS = BS_MAXH * 6;                       // (head, segment, half)
+constexpr int BS_CONSUMERS = BS_ITEMS * BS_TPS;             // 384 threads
+constexpr int BS_THREADS = BS_CONSUMERS + 32;               // + the producer warp
+constexpr int BS_ROW = BS_MAXH * 96 * 2;                    // bytes of one token's k (or v)
+constexpr uint32_t BS_WAIT = 1u << 22;
+struct BulkSmem {
+  uint8_t ring[BS_STAGES][BS_TPS][2][BS_ROW];  // reused for the final reduction
+  float2 tab[TAB96 * TABS96];
+  uint64_t full[BS_STAGES], empty[BS_STAGES];
+  int32_t abort;
+};
+static_assert(sizeof(float) * BS_TPS * BS_ITEMS * 32 <= sizeof(uint8_t) * BS_STAGES * BS_TPS * 2 * BS_ROW,
+              "reduction buffer must fit the ring");
+
+template <bool STAGE>
+__global__ void __launch_bounds__(BS_THREADS, 2) k_summaries_bulk(
+    Geo g, const int32_t* __restrict__ vol, const float* __restrict__ rope,
+    int32_t* __restrict__ err, const __nv_bfloat16* __restrict__ k,
+    const __nv_bfloat16* __restrict__ v, float* ksum, float* vsum, StageOut so) {
+  using namespace tc;
+  if (err[0]) return;
+  extern __shared__ uint8_t bs_raw[];
+  BulkSmem& sm = *reinterpret_cast<BulkSmem*>((reinterpret_cast<uintptr_t>(bs_raw) + 127) &
+                                              ~(uintptr_t)127);
+  const int tid = threadIdx.x;
+  const int blk = blockIdx.x, b = blockIdx.y;
+  const int Bz = blk / (g.nby * g.nbx), By = (blk / g.nbx) % g.nby, Bx = blk % g.nbx;
+  const int cnt = g.bz * g.by * g.bx;
+  const int n_stage_rounds = (cnt + BS_TPS - 1) / BS_TPS;
+  const uint32_t row_bytes = (uint32_t)g.H * 96 * 2;
+  volatile int32_t* abort_flag = &sm.abort;
+  if (tid == 0) {
+    for (int s = 0; s < BS_STAGES; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], BS_CONSUMERS / 32);
+    }
+    sm.abort = 0;
+    fence_barrier_init();
+  }
+  // rotation-table rows of this block's coordinates (z rows, y rows, x rows)
+  const float2* gtab = reinterpret_cast<const float2*>(rope);
+  for (int e = tid; e < (g.bz + g.by + g.bx) * 16; e += BS_THREADS) {
+    const int r = e / 16, jj = e % 16;
+    const int grow = r < g.bz ? Bz * g.bz + r
+                              : (r < g.bz + g.by ? g.Z + By * g.by + r - g.bz
+                                                 : g.Z + g.Y + Bx * g.bx + r - g.bz - g.by);
+    sm.tab[r * TABS96 + jj] = gtab[grow * 16 + jj];
+  }
+  __syncthreads();
+  auto voxel = [&](int e, int& cz, int& cy, int& cx) {
+    cx = Bx * g.bx + e % g.bx;
+    cy = By * g.by + (e / g.bx) % g.by;
+    cz = Bz * g.bz + e / (g.bx * g.by);
+  };
+  // consumer item and partial sums (8 channels of k and their partners, same of v)
+  const int grp = tid / BS_ITEMS, c = tid % BS_ITEMS;
+  float kx1[8], kx2[8], vx1[8], vx2[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) kx1[i] = kx2[i] = vx1[i] = vx2[i] = 0.f;
+  if (tid >= BS_CONSUMERS) {
+    // ---- producer warp: lane i copies token i of each stage ----
+    const int lane = tid - BS_CONSUMERS;
+    const int32_t* vb = vol + (int64_t)b * g.N;
+    for (int r = 0; r < n_stage_rounds; ++r) {
+      const int s = r % BS_STAGES;
+      bool ok = true;
+      if (lane == 0 && r >= BS_STAGES)
+        ok = mbar_wait_or_abort(&sm.empty[s], ((r / BS_STAGES) - 1) & 1, BS_WAIT, abort_flag);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      const int ntok = min(BS_TPS, cnt - r * BS_TPS);
+      if (lane == 0) mbar_arrive_expect_tx(&sm.full[s], (uint32_t)ntok * 2 * row_bytes);
+      __syncwarp();
+      if (lane < ntok) {
+        int cz, cy, cx;
+        voxel(r * BS_TPS + lane, cz, cy, cx);
+        const int64_t tok = vb[(cz * g.Y + cy) * g.X + cx];
+        bulk_load(sm.ring[s][lane][0], k + (((int64_t)b * g.N + tok) * g.H) * 96, row_bytes,
+                  &sm.full[s]);
+        bulk_load(sm.ring[s][lane][1], v + (((int64_t)b * g.N + tok) * g.H) * 96, row_bytes,
+                  &sm.full[s]);
+      }
+    }
+    // every copy issued has been waited for by the consumers unless they gave up
+    if (lane == 0)
+      for (int r = max(0, n_stage_rounds - BS_STAGES); r < n_stage_rounds; ++r)
+        mbar_wait(&sm.full[r % BS_STAGES], (r / BS_STAGES) & 1, BS_WAIT);
+    __syncwarp();
+  } else {
+    // ---- consumers ----
+    const int h = c / 6, w = c % 6;
+    const bool live = h < g.H;
+    const int a = w / 2, c1 = 4 * a + (w & 1), c2 = c1 + 2, j0 = 8 * (w & 1);
+    const float2* tab = a == 0 ? sm.tab : (a == 1 ? sm.tab + g.bz * TABS96 : sm.tab + (g.bz + g.by) * TABS96);
+    const int base = a == 0 ? Bz * g.bz : (a == 1 ? By * g.by : Bx * g.bx);
+    for (int r = 0; r < n_stage_rounds; ++r) {
+      const int s = r % BS_STAGES;
+      if (!__all_sync(0xffffffffu, mbar_wait_or_abort(&sm.full[s], (r / BS_STAGES) & 1, BS_WAIT,
+                                                       abort_flag)))
+        break;
+      const int e = r * BS_TPS + grp;
+      if (live && e < cnt) {
+        int cz, cy, cx;
+        voxel(e, cz, cy, cx);
+        const uint4* kr = reinterpret_cast<const uint4*>(sm.ring[s][grp][0] + h * 192);
+        const uint4* vr = reinterpret_cast<const uint4*>(sm.ring[s][grp][1] + h * 192);
+        const uint4 ka = kr[c1], kb = kr[c2], va = vr[c1], vb2 = vr[c2];
+        const int ca = a == 0 ? cz : (a == 1 ? cy : cx);
+        const float2* t = tab + (ca - base) * TABS96 + j0;
+        const uint32_t* kaw = reinterpret_cast<const uint32_t*>(&ka);
+        const uint32_t* kbw = reinterpret_cast<const uint32_t*>(&kb);
+        const uint32_t* vaw = reinterpret_cast<const uint32_t*>(&va);
+        const uint32_t* vbw = reinterpret_cast<const uint32_t*>(&vb2);
+        uint4 ra, rb;
+        uint32_t* raw = reinterpret_cast<uint32_t*>(&ra);
+        uint32_t* rbw = reinterpret_cast<uint32_t*>(&rb);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float2 x1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(kaw + q));
+          float2 x2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(kbw + q));
+          const float4 cs = *reinterpret_cast<const float4*>(t + 2 * q);  // pairs j, j + 1
+          const float r1a = x1.x * cs.x - x2.x * cs.y, r2a = x1.x * cs.y + x2.x * cs.x;
+          const float r1b = x1.y * cs.z - x2.y * cs.w, r2b = x1.y * cs.w + x2.y * cs.z;
+          kx1[2 * q] += r1a;
+          kx2[2 * q] += r2a;
+          kx1[2 * q + 1] += r1b;
+          kx2[2 * q + 1] += r2b;
+          if (STAGE) {
+            __nv_bfloat162 pa = __floats2bfloat162_rn(r1a, r1b), pb = __floats2bfloat162_rn(r2a, r2b);
+            raw[q] = *reinterpret_cast<uint32_t*>(&pa);
+            rbw[q] = *reinterpret_cast<uint32_t*>(&pb);
+          }
+          float2 y1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(vaw + q));
+          float2 y2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(vbw + q));
+          vx1[2 * q] += y1.x;
+          vx1[2 * q + 1] += y1.y;
+          vx2[2 * q] += y2.x;
+          vx2[2 * q + 1] += y2.y;
+        }
+        if (STAGE) {
+          const int64_t grow = ((((int64_t)b * g.H + h) * g.Z + cz) * g.Y + cy) * g.X + cx;
+          uint4* kd = reinterpret_cast<uint4*>(so.kg + grow * 96);
+          uint4* vd = reinterpret_cast<uint4*>(so.vg + grow * 96);
+          kd[c1] = ra;
+          kd[c2] = rb;
+          vd[c1] = va;
+          vd[c2] = vb2;
+        }
+      }
+      __syncwarp();
+      if ((tid & 31) == 0) mbar_arrive(&sm.empty[s]);
+    }
+  }
+  // every stage is consumed (or abandoned): the ring takes the partial sums
+  // [group][item][32]
+  __syncthreads();
+  if (sm.abort) {
+    if (tid == 0) atomicOr(&err[0], 4);
+    return;
+  }
+  if (tid < BS_CONSUMERS) {
+    float* red = reinterpret_cast<float*>(&sm.ring[0][0][0][0]);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      red[(grp * BS_ITEMS + c) * 32 + i] = kx1[i];
+      red[(grp * BS_ITEMS + c) * 32 + 8 + i] = kx2[i];
+      red[(grp * BS_ITEMS + c) * 32 + 16 + i] = vx1[i];
+      red[(grp * BS_ITEMS + c) * 32 + 24 + i] = vx2[i];
+    }
+  }
+  __syncthreads();
+  // sums over the groups in order, means, outputs
+  const float* red = reinterpret_cast<const float*>(&sm.ring[0][0][0][0]);
+  const float inv_cnt = 1.f / (float)cnt;
+  for (int o = tid; o < g.H * 2 * 96; o += BS_THREADS) {
+    const int h = o / 192, which = (o / 96) % 2, ch = o % 96;
+    // channel ch of head h lives in item (h, w) at slot 8 * (half) + i
+    const int seg = ch / 32, within = ch % 32, hi = within >= 16, jj = within % 16;
+    const int w = seg * 2 + (jj >= 8), i = jj % 8;
+    const int slot = (which ? 16 : 0) + (hi ? 8 : 0) + i;
+    float acc = 0.f;
+    for (int q = 0; q < BS_TPS; ++q) acc += red[(q * BS_ITEMS + h * 6 + w) * 32 + slot];
+    const int64_t idx = (((int64_t)b * g.H + h) * g.nb + blk) * 96 + ch;
+    const float mean = acc * inv_cnt;
+    if (ksum) (which ? vsum : ksum)[idx] = mean;
+    if (STAGE && so.ksb) (which ? so.vsb : so.ksb)[idx] = __float2bfloat16_rn(mean);
+  }
+}
+
+// The bulk-copy kernel: up to 8 heads; the block's rotation-table rows staged.
+bool bulk_supported(const Geo& g) {
+  return g.H <= BS_MAXH && g.bz + g.by + g.bx <= TAB96;
+}
+
+template <bool STAGE>
+int launch_bulk(const Geo& g, const pack3d_index* idx, const void* k, const void* v, float* ksum,
+                float* vsum, StageOut so, cudaStream_t s) {
+  const size_t smem = sizeof(BulkSmem) + 128;
+  auto kern = k_summaries_bulk<STAGE>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return PACK3D_ERR_CUDA;
+  kern<<<dim3(g.nb, g.B), BS_THREADS, smem, s>>>(g, idx->vol, idx->rope, idx->err,
+                                                  (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
+                                                  ksum, vsum, so);
+  return cuda_status(cudaGetLastError());
+}
+
 int launch_block_summaries(const Geo& g, const pack3d_index* idx, const void* k, const void* v,
                            float* ksum, float* vsum, cudaStream_t s) {
   dim3 grid(g.nb, g.B, g.H);
   if (g.dtype == PACK3D_BF16 && g.d == 96) {
+    if (bulk_supported(g)) return launch_bulk<false>(g, idx, k, v, ksum, vsum, StageOut{}, s);
     dim3 grid96(g.nb, g.B, (g.H + HG96 - 1) / HG96);
     k_block_summaries_bf16_d96<false><<<grid96, TG96 * LANES96, 0, s>>>(
         g, idx->vol, idx->rope, idx->err, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, ksum,
@@ -301,12 +522,20 @@ int launch_block_summaries(const Geo& g, const pack3d_index* idx, const void* k,
   return cuda_status(cudaGetLastError());
 }
 
+int launch_stage_bulk(const Geo& g, const pack3d_index* idx, const void* k, const void* v,
+                      void* kg, void* vg, cudaStream_t s) {
+  if (g.dtype != PACK3D_BF16 || g.d != 96 || !bulk_supported(g)) return PACK3D_ERR_UNSUPPORTED;
+  StageOut so{(__nv_bfloat16*)kg, (__nv_bfloat16*)vg, nullptr, nullptr};
+  return launch_bulk<true>(g, idx, k, v, nullptr, nullptr, so, s);
+}
+
 int launch_block_summaries_staged(const Geo& g, const pack3d_index* idx, const void* k,
                                   const void* v, float* ksum, float* vsum, void* kg, void* vg,
                                   void* ksb, void* vsb, cudaStream_t s) {
   if (g.dtype != PACK3D_BF16 || g.d != 96) return PACK3D_ERR_UNSUPPORTED;
   dim3 grid96(g.nb, g.B, (g.H + HG96 - 1) / HG96);
   StageOut so{(__nv_bfloat16*)kg, (__nv_bfloat16*)vg, (__nv_bfloat16*)ksb, (__nv_bfloat16*)vsb};
+  if (bulk_supported(g)) return launch_bulk<true>(g, idx, k, v, ksum, vsum, so, s);
   k_block_summaries_bf16_d96<true><<<grid96, TG96 * LANES96, 0, s>>>(
       g, idx->vol, idx->rope, idx->err, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, ksum,
       vsum, so);

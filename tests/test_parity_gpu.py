@@ -20,6 +20,9 @@ pytestmark = pytest.mark.gpu
 RAGGED96 = I.Workload(name="ragged_6x10x20_d96", B=2, H=2, d=96, Z=6, Y=10, X=20,
                       window=(5, 3, 7), block=(3, 5, 4), dtype="bf16", value_scale=1.0,
                       seed=31)
+# more heads than the bulk gather of the staging pass takes (its fallback path)
+HEADS10 = I.Workload(name="heads10_4x8x16_d96", B=1, H=10, d=96, Z=4, Y=8, X=16,
+                     window=(3, 3, 5), block=(2, 4, 4), dtype="bf16", seed=38)
 SMALL = [
     C.TINY,
     RAGGED96,
@@ -34,6 +37,7 @@ SMALL = [
                block=(2, 3, 6), dtype="fp32", seed=36),
     I.Workload(name="d24_bf16_4x12x9", B=1, H=2, d=24, Z=4, Y=12, X=9, window=(3, 5, 5),
                block=(2, 6, 3), dtype="bf16", seed=37),
+    HEADS10,
 ]
 
 
@@ -132,7 +136,7 @@ def test_forward_micro1m_sampled(oracle_lib):
     assert_close(res["lse"][b, h, i], lse, wl.dtype, "lse")
 
 
-@pytest.mark.parametrize("wl", [RAGGED96, C.VOL16K], ids=lambda w: w.name)
+@pytest.mark.parametrize("wl", [RAGGED96, HEADS10, C.VOL16K], ids=lambda w: w.name)
 def test_staged_halves(oracle_lib, wl):
     """pack3d_stage_kv with summaries computes the same summaries as
     pack3d_block_summaries (bit for bit) and stages the same grid-order keys
