@@ -125,6 +125,7 @@ class Workload:
     values: str = "normal"       # "normal" or "smooth"
     value_scale: float = 1.0     # multiplies the N(0,1) draws ("normal" only)
     rope_base: float = 100.0
+    rope_mode: int = 0           # 0: axial RoPE on grid coordinates; 1: 1-D RoPE on the packed position
     packings: tuple = ("raster",)
     seed: int = 0
     backward: bool = False

@@ -30,7 +30,11 @@ ERR = {0: "ok", -1: "bad argument", -2: "bad coordinates", -3: "out of memory"}
 class Params(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
                 ("B", "H", "d", "Z", "Y", "X", "wz", "wy", "wx", "bz", "by", "bx")] + [
-        ("base", ctypes.c_double), ("scale", ctypes.c_double)]
+        ("base", ctypes.c_double), ("scale", ctypes.c_double), ("rope_mode", ctypes.c_int32)]
+
+# rope_mode: 0 = axial RoPE on grid coordinates (PACK3D); 1 = one-dimensional
+# RoPE on the packed position (the packed-sequence comparison mode)
+ROPE_AXIAL, ROPE_PACKED = 0, 1
 
 
 def build(force: bool = False) -> str:
@@ -73,7 +77,8 @@ def max_threads() -> int:
 def params(shape) -> Params:
     w, b = tuple(shape.window), tuple(shape.block)
     return Params(shape.B, shape.H, shape.d, shape.Z, shape.Y, shape.X, w[0], w[1], w[2],
-                  b[0], b[1], b[2], float(shape.rope_base), float(getattr(shape, "scale", 0.0) or 0.0))
+                  b[0], b[1], b[2], float(shape.rope_base), float(getattr(shape, "scale", 0.0) or 0.0),
+                  int(getattr(shape, "rope_mode", 0) or 0))
 
 
 def _as_input(x):

@@ -28,6 +28,14 @@
  *      S(i)), with no count bias; one softmax over both sets.
  *   6. o_i = softmax-weighted sum of v_j and vbar_B; lse_i = m + ln(l).
  *
+ * Packed-sequence comparison mode (rope_mode = 1): the same operator with the
+ * rotation of step 1 replaced by the standard one-dimensional RoPE on the
+ * token's position p in the packed sequence (its index in memory order): the
+ * whole head is one segment, channel j pairs with j + d/2, theta_j =
+ * base^(-2j/d), angle p * theta_j.  Windows, blocks and summaries stay
+ * geometric.  This is the positional encoding the abstract contrasts with
+ * axial RoPE on grid coordinates; with it the result depends on the packing.
+ *
  * Every loop runs in grid order (never in packed order), so results do not
  * depend on the memory order of the tokens.  Inputs are read as fp64, fp32 or
  * bf16 bit patterns and widened exactly to fp64; all arithmetic is fp64 with
@@ -50,7 +58,8 @@ typedef struct {
   int32_t wz, wy, wx;
   int32_t bz, by, bx;
   double base;
-  double scale; /* tau; <= 0 means 1/sqrt(d) */
+  double scale;      /* tau; <= 0 means 1/sqrt(d) */
+  int32_t rope_mode; /* 0: axial on grid coordinates; 1: 1-D on the packed position */
 } orc_params;
 
 enum { ORC_OK = 0, ORC_ERR_ARG = -1, ORC_ERR_COORDS = -2, ORC_ERR_MEM = -3 };
@@ -75,6 +84,7 @@ static int check_params(const orc_params* p) {
   if (p->bz < 1 || p->by < 1 || p->bx < 1) return ORC_ERR_ARG;
   if (p->Z % p->bz || p->Y % p->by || p->X % p->bx) return ORC_ERR_ARG;
   if (!(p->base > 0.0)) return ORC_ERR_ARG;
+  if (p->rope_mode != 0 && p->rope_mode != 1) return ORC_ERR_ARG;
   return ORC_OK;
 }
 
@@ -92,9 +102,24 @@ static int nblocks(const orc_params* p) {
   return (p->Z / p->bz) * (p->Y / p->by) * (p->X / p->bx);
 }
 
-/* cos and sin of c * theta_j for every axis, coordinate value and pair j:
- * tab[((axis_offset + c) * (da/2) + j) * 2 + {0,1}], axis offsets 0, Z, Z+Y. */
+/* Axial mode: cos and sin of c * theta_j for every axis, coordinate value and
+ * pair j: tab[((axis_offset + c) * (da/2) + j) * 2 + {0,1}], axis offsets 0, Z,
+ * Z+Y.  Packed mode: cos and sin of p * theta_j for every packed position p < N
+ * and pair j < d/2: tab[(p * (d/2) + j) * 2 + {0,1}]. */
 static double* rope_table(const orc_params* p) {
+  if (p->rope_mode == 1) {
+    size_t N = nvox(p);
+    int half = p->d / 2;
+    double* tab = (double*)malloc(N * half * 2 * sizeof(double));
+    if (!tab) return NULL;
+    for (size_t pos = 0; pos < N; ++pos)
+      for (int j = 0; j < half; ++j) {
+        double theta = pow(p->base, -2.0 * j / (double)p->d);
+        tab[(pos * half + j) * 2 + 0] = cos((double)pos * theta);
+        tab[(pos * half + j) * 2 + 1] = sin((double)pos * theta);
+      }
+    return tab;
+  }
   int da = p->d / 3, half = da / 2;
   int ext[3] = {p->Z, p->Y, p->X};
   size_t rows = (size_t)p->Z + p->Y + p->X;
@@ -111,9 +136,21 @@ static double* rope_table(const orc_params* p) {
   return tab;
 }
 
-/* out = R(c) in (transpose = 0) or R(c)^T in (transpose = 1). */
+/* out = R in (transpose = 0) or R^T in (transpose = 1), R the rotation of the
+ * token with grid coordinate c and packed position pos. */
 static void rope_apply(const orc_params* p, const double* tab, const double* in,
-                       const int c[3], int transpose, double* out) {
+                       const int c[3], size_t pos, int transpose, double* out) {
+  if (p->rope_mode == 1) {
+    int half = p->d / 2;
+    const double* t = tab + pos * half * 2;
+    for (int j = 0; j < half; ++j) {
+      double x1 = in[j], x2 = in[j + half];
+      double cs = t[2 * j], sn = transpose ? -t[2 * j + 1] : t[2 * j + 1];
+      out[j] = x1 * cs - x2 * sn;
+      out[j + half] = x1 * sn + x2 * cs;
+    }
+    return;
+  }
   int da = p->d / 3, half = da / 2;
   int off[3] = {0, p->Z, p->Z + p->Y};
   for (int a = 0; a < 3; ++a) {
@@ -237,7 +274,7 @@ int oracle_rope(const orc_params* p, const int16_t* coords, const void* x, int d
       coord_of(coords, p, b, i, c);
       for (int h = 0; h < p->H; ++h) {
         load_row(x, dtype, p, b, i, h, row);
-        rope_apply(p, tab, row, c, transpose, out + (((size_t)b * N + i) * p->H + h) * p->d);
+        rope_apply(p, tab, row, c, i, transpose, out + (((size_t)b * N + i) * p->H + h) * p->d);
       }
     }
   free(row);
@@ -267,7 +304,7 @@ static void summaries_bh(const orc_params* p, const double* tab, const int32_t* 
           int cj[3];
           coord_of(coords, p, b, j, cj);
           load_row(k, dtype, p, b, j, h, row);
-          rope_apply(p, tab, row, cj, 0, rot);
+          rope_apply(p, tab, row, cj, j, 0, rot);
           for (int c = 0; c < d; ++c) kd[c] += rot[c];
           load_row(v, dtype, p, b, j, h, row);
           for (int c = 0; c < d; ++c) vd[c] += row[c];
@@ -340,7 +377,7 @@ static int query_logits(const orc_params* p, const double* tab, const int32_t* v
   int c[3];
   coord_of(coords, p, b, i, c);
   load_row(q, dtype, p, b, i, h, s->row);
-  rope_apply(p, tab, s->row, c, 0, s->qrot);
+  rope_apply(p, tab, s->row, c, i, 0, s->qrot);
   int rz = (p->wz - 1) / 2, ry = (p->wy - 1) / 2, rx = (p->wx - 1) / 2;
   int n = 0;
   for (int z = c[0] - rz; z <= c[0] + rz; ++z) {
@@ -352,7 +389,7 @@ static int query_logits(const orc_params* p, const double* tab, const int32_t* v
         size_t j = (size_t)vb[vox_id(p, z, y, x)];
         int cj[3] = {z, y, x};
         load_row(k, dtype, p, b, j, h, s->row);
-        rope_apply(p, tab, s->row, cj, 0, s->krot);
+        rope_apply(p, tab, s->row, cj, j, 0, s->krot);
         double acc = 0.0;
         for (int e = 0; e < d; ++e) acc += s->qrot[e] * s->krot[e];
         s->logit[n] = tau * acc;
@@ -540,7 +577,7 @@ int oracle_backward(const orc_params* p, const int16_t* coords, const void* q, c
               int cj[3];
               coord_of(coords, p, b, j, cj);
               load_row(k, dtype, p, b, j, h, s.row);
-              rope_apply(p, tab, s.row, cj, 0, s.krot);
+              rope_apply(p, tab, s.row, cj, j, 0, s.krot);
               for (int e = 0; e < d; ++e) {
                 dqr[e] += tau * dS * s.krot[e];
                 dkrot[j * d + e] += tau * dS * s.qrot[e];
@@ -556,7 +593,7 @@ int oracle_backward(const orc_params* p, const int16_t* coords, const void* q, c
             }
           }
           int ci[3] = {z, y, x};
-          rope_apply(p, tab, dqr, ci, 1, dq + (((size_t)b * N + i) * p->H + h) * d);
+          rope_apply(p, tab, dqr, ci, i, 1, dq + (((size_t)b * N + i) * p->H + h) * d);
         }
     /* Spread the summary gradients over the block members, rotate back. */
     for (int z = 0; z < p->Z; ++z)
@@ -572,7 +609,7 @@ int oracle_backward(const orc_params* p, const int16_t* coords, const void* q, c
           }
           int cj[3] = {z, y, x};
           for (int e = 0; e < d; ++e) tmp[e] = dkrot[j * d + e];
-          rope_apply(p, tab, tmp, cj, 1, dk + (((size_t)b * N + j) * p->H + h) * d);
+          rope_apply(p, tab, tmp, cj, j, 1, dk + (((size_t)b * N + j) * p->H + h) * d);
           for (int e = 0; e < d; ++e) dv[(((size_t)b * N + j) * p->H + h) * d + e] = dvacc[j * d + e];
         }
     free(P);

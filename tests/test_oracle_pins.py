@@ -395,3 +395,92 @@ def test_bad_coordinates_rejected(oracle_lib):
     out[0, 3, 2] = 2
     with pytest.raises(ValueError):
         oracle.volume(s, out)
+
+
+# ---- packed-sequence comparison mode (1-D RoPE on the packed position) -------
+
+def packed_shape(**kw):
+    s = shape(**kw)
+    s.rope_mode = oracle.ROPE_PACKED
+    return s
+
+
+def rotate_complex_1d(x, base):
+    """One-dimensional RoPE as complex multiplication: pair (j, j + d/2) is the
+    complex number x_j + i x_{j+d/2}, multiplied by exp(i p base^(-2j/d)) with p
+    the row's position along axis -3 (the packed index)."""
+    x = np.asarray(x, np.float64)
+    d = x.shape[-1]
+    h = d // 2
+    theta = base ** (-2.0 * np.arange(h) / d)
+    pos = np.arange(x.shape[-3], dtype=np.float64)[:, None, None]
+    z = (x[..., :h] + 1j * x[..., h:]) * np.exp(1j * pos * theta)
+    return np.concatenate([z.real, z.imag], axis=-1)
+
+
+def test_packed_rope_matches_complex_rotation(oracle_lib):
+    s = packed_shape(B=2, H=3, d=18, Z=5, Y=3, X=7, block=(1, 1, 1))
+    packed, coords, _ = rand_inputs(s, seed=21)
+    got = oracle.rope(s, coords, packed["q"])
+    want = rotate_complex_1d(packed["q"].numpy(), s.rope_base)
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+    back = oracle.rope(s, coords, torch.from_numpy(got), transpose=True)
+    np.testing.assert_allclose(back, packed["q"].numpy(), rtol=0, atol=1e-12)
+
+
+def test_packed_rope_logit_depends_only_on_packed_displacement(oracle_lib):
+    """With the same q and k in every row, q~_i . k~_j is a function of j - i."""
+    s = packed_shape(B=1, H=1, d=24, Z=4, Y=4, X=4, block=(1, 1, 1))
+    rng = np.random.default_rng(4)
+    N = s.Z * s.Y * s.X
+    q, k = rng.standard_normal(s.d), rng.standard_normal(s.d)
+    coords = I.coords_of_order(rng.permutation(N), s.Z, s.Y, s.X)[None]
+    rq = oracle.rope(s, coords, np.broadcast_to(q, (1, N, 1, s.d)).copy())[0, :, 0]
+    rk = oracle.rope(s, coords, np.broadcast_to(k, (1, N, 1, s.d)).copy())[0, :, 0]
+    L = rq @ rk.T
+    for dlt in (-7, -1, 0, 3, 11):
+        diag = np.array([L[i, i + dlt] for i in range(max(0, -dlt), min(N, N - dlt))])
+        np.testing.assert_allclose(diag, diag[0], rtol=0, atol=1e-11)
+
+
+def test_packed_mode_full_window_is_dense_1d_rope_attention(oracle_lib):
+    """Full windows and 1x1x1 blocks: dense softmax attention over the packed
+    sequence with one-dimensional RoPE (torch SDPA on independently rotated
+    rows)."""
+    s = packed_shape(B=2, H=2, d=12, Z=3, Y=4, X=5, window=(5, 7, 9), block=(1, 1, 1))
+    packed, coords, _ = rand_inputs(s, seed=22)
+    out, lse = oracle.forward(s, coords, packed["q"], packed["k"], packed["v"])
+    tau = 1.0 / math.sqrt(s.d)
+    for b in range(s.B):
+        qr = torch.from_numpy(rotate_complex_1d(packed["q"][b].numpy(), s.rope_base))
+        kr = torch.from_numpy(rotate_complex_1d(packed["k"][b].numpy(), s.rope_base))
+        q, k, v = (t.permute(1, 0, 2) for t in (qr, kr, packed["v"][b]))
+        ro = torch.nn.functional.scaled_dot_product_attention(q, k, v, scale=tau)
+        rl = torch.logsumexp(tau * q @ k.transpose(1, 2), dim=-1)
+        np.testing.assert_allclose(out[b], ro.permute(1, 0, 2).numpy(), rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse[b], rl.numpy(), rtol=0, atol=1e-12)
+
+
+def test_packed_mode_depends_on_the_packing(oracle_lib):
+    """The failure mode the pages contrast axial RoPE with: the same field under
+    two packings gives the same per-voxel output with axial RoPE and different
+    outputs with RoPE on the packed position."""
+    res = {}
+    for mode in (oracle.ROPE_AXIAL, oracle.ROPE_PACKED):
+        s = shape(B=1, H=2, d=12, Z=4, Y=4, X=8, window=(3, 3, 3), block=(2, 2, 4))
+        s.rope_mode = mode
+        g = torch.Generator().manual_seed(23)
+        N = s.Z * s.Y * s.X
+        grid = {n: torch.randn(1, N, s.H, s.d, generator=g, dtype=torch.float64) for n in "qkv"}
+        outs = []
+        for packing in ("raster", "random"):
+            order = I.packing_order(packing, s.Z, s.Y, s.X, s.block, 5, 0)
+            coords = I.coords_of_order(order, s.Z, s.Y, s.X)[None]
+            pk = {n: t[:, torch.from_numpy(order)] for n, t in grid.items()}
+            out, _ = oracle.forward(s, coords, pk["q"], pk["k"], pk["v"])
+            o = np.empty_like(out)
+            o[0, order] = out[0]
+            outs.append(o)
+        res[mode] = np.abs(outs[0] - outs[1]).max()
+    assert res[oracle.ROPE_AXIAL] == 0.0
+    assert res[oracle.ROPE_PACKED] > 1e-3
