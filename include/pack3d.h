@@ -64,6 +64,7 @@ extern "C" {
 typedef struct CUstream_st* pack3d_stream_t; /* the same type as cudaStream_t */
 
 enum { PACK3D_BF16 = 0, PACK3D_FP32 = 1 };
+enum { PACK3D_ROPE_AXIAL = 0, PACK3D_ROPE_PACKED = 1 };
 
 enum {
   PACK3D_OK = 0,
@@ -87,6 +88,11 @@ typedef struct {
   int32_t dtype;   /* PACK3D_BF16 or PACK3D_FP32 (inputs, outputs, gradients) */
   int32_t out_fp32; /* nonzero: the forward's out (and the backward's out argument) is
                        fp32 even when dtype is PACK3D_BF16 */
+  int32_t rope_mode; /* PACK3D_ROPE_AXIAL (0, the operator): axial RoPE on grid
+                        coordinates; PACK3D_ROPE_PACKED (1, the comparison mode):
+                        one-dimensional RoPE on the token's packed index (pairs
+                        j, j + head_dim/2, theta_j = rope_base^(-2j/head_dim));
+                        windows, blocks and summaries stay geometric */
 } pack3d_params;
 
 /* Geometry index of one packing, built by pack3d_build_index into one

@@ -73,29 +73,42 @@ __device__ __forceinline__ float group_sum(float v) {
   return v;
 }
 
-// Rotated channel c of row x (global memory), by the coordinate (z, y, x) -
-// transpose = true applies R^T.
+// Rotated channel c of a row, for the token with coordinate (z, y, x) and
+// packed index pos - transpose = true applies R^T.  Axial mode: segment
+// a = c / da, pair (j, j + da/2) of it; packed mode: pair (j, j + d/2).
+template <typename T>
+__device__ __forceinline__ float rot_row_channel(const T* row, const float* rope, const Geo& g,
+                                                 int c, int cz, int cy, int cx, int pos,
+                                                 bool transpose) {
+  int base, len, p, a = 0, ca = 0;
+  if (g.rope_mode == PACK3D_ROPE_PACKED) {
+    base = 0;
+    len = g.d / 2;
+    p = c;
+  } else {
+    a = c / g.da;
+    base = a * g.da;
+    len = g.half;
+    p = c % g.da;
+    ca = a == 0 ? cz : (a == 1 ? cy : cx);
+  }
+  int j = p < len ? p : p - len;
+  float2 cs = rope_cs(rope, g, a, ca, pos, j);
+  float sn = transpose ? -cs.y : cs.y;
+  float x1 = to_f32(row[base + j]), x2 = to_f32(row[base + j + len]);
+  return p < len ? x1 * cs.x - x2 * sn : x1 * sn + x2 * cs.x;
+}
+
 template <typename T>
 __device__ __forceinline__ float rot_channel(const T* row, const float* rope, const Geo& g, int c,
-                                             int cz, int cy, int cx, bool transpose) {
-  int a = c / g.da, p = c % g.da;
-  int ca = a == 0 ? cz : (a == 1 ? cy : cx);
-  int j = p < g.half ? p : p - g.half;
-  float2 cs = rope_cs(rope, g, a, ca, j);
-  float sn = transpose ? -cs.y : cs.y;
-  float x1 = to_f32(row[a * g.da + j]), x2 = to_f32(row[a * g.da + j + g.half]);
-  return p < g.half ? x1 * cs.x - x2 * sn : x1 * sn + x2 * cs.x;
+                                             int cz, int cy, int cx, int pos, bool transpose) {
+  return rot_row_channel(row, rope, g, c, cz, cy, cx, pos, transpose);
 }
 
 __device__ __forceinline__ float rot_channel_smem(const float* row, const float* rope, const Geo& g,
-                                                  int c, int cz, int cy, int cx, bool transpose) {
-  int a = c / g.da, p = c % g.da;
-  int ca = a == 0 ? cz : (a == 1 ? cy : cx);
-  int j = p < g.half ? p : p - g.half;
-  float2 cs = rope_cs(rope, g, a, ca, j);
-  float sn = transpose ? -cs.y : cs.y;
-  float x1 = row[a * g.da + j], x2 = row[a * g.da + j + g.half];
-  return p < g.half ? x1 * cs.x - x2 * sn : x1 * sn + x2 * cs.x;
+                                                  int c, int cz, int cy, int cx, int pos,
+                                                  bool transpose) {
+  return rot_row_channel(row, rope, g, c, cz, cy, cx, pos, transpose);
 }
 
 struct ChunkCoords {
@@ -133,7 +146,7 @@ __global__ void __launch_bounds__(TILE * Split<D>::G) k_forward_simt(
 #pragma unroll
     for (int u = 0; u < CPT; ++u) {
       int c = lane * CPT + u;
-      qr[u] = active ? qscale * rot_channel(qrow, ix.rope, g, c, cz, cy, cx, false) : 0.f;
+      qr[u] = active ? qscale * rot_channel(qrow, ix.rope, g, c, cz, cy, cx, qi, false) : 0.f;
       o[u] = 0.f;
     }
   }
@@ -153,7 +166,7 @@ __global__ void __launch_bounds__(TILE * Split<D>::G) k_forward_simt(
         halo_coord(tg, base + kk, z, y, x);
         int j = hl[base + kk];
         int64_t row = (((int64_t)b * g.N + j) * g.H + h) * D;
-        kv = rot_channel(k + row, ix.rope, g, c, z, y, x, false);
+        kv = rot_channel(k + row, ix.rope, g, c, z, y, x, j, false);
         vv = to_f32(v[row + c]);
         if (c == 0) {
           cc.z[kk] = z;
@@ -338,7 +351,7 @@ __global__ void __launch_bounds__(256) k_bwd_summary(Geo g, pack3d_index ix,
           tile_coord(tg, qb + qq, z, y, x);
           int i = ix.perm[(int64_t)b * g.N + toff + qb + qq];
           int64_t row = (((int64_t)b * g.N + i) * g.H + h) * D;
-          qv = rot_channel(q + row, ix.rope, g, c, z, y, x, false);
+          qv = rot_channel(q + row, ix.rope, g, c, z, y, x, i, false);
           dv = to_f32(dout[row + c]);
           if (c == 0) {
             sqc[qq][0] = z;
@@ -435,7 +448,7 @@ __global__ void __launch_bounds__(TILE * Split<D>::G) k_bwd_dq(
 #pragma unroll
   for (int u = 0; u < CPT; ++u) {
     int c = lane * CPT + u;
-    qr[u] = active ? rot_channel(q + qrow, ix.rope, g, c, cz, cy, cx, false) : 0.f;
+    qr[u] = active ? rot_channel(q + qrow, ix.rope, g, c, cz, cy, cx, qi, false) : 0.f;
     dO[u] = active ? to_f32(dout[qrow + c]) : 0.f;
     dqr[u] = 0.f;
   }
@@ -456,7 +469,7 @@ __global__ void __launch_bounds__(TILE * Split<D>::G) k_bwd_dq(
         halo_coord(tg, base + kk, z, y, x);
         int j = hl[base + kk];
         int64_t row = (((int64_t)b * g.N + j) * g.H + h) * D;
-        kv = rot_channel(k + row, ix.rope, g, c, z, y, x, false);
+        kv = rot_channel(k + row, ix.rope, g, c, z, y, x, j, false);
         vv = to_f32(v[row + c]);
         if (c == 0) {
           cc.z[kk] = z;
@@ -541,7 +554,7 @@ __global__ void __launch_bounds__(TILE * Split<D>::G) k_bwd_dq(
 #pragma unroll
       for (int u = 0; u < CPT; ++u) {
         int c = lane * CPT + u;
-        dq[qrow + c] = from_f32<T>(rot_channel_smem(sbuf + r * D, ix.rope, g, c, cz, cy, cx, true));
+        dq[qrow + c] = from_f32<T>(rot_channel_smem(sbuf + r * D, ix.rope, g, c, cz, cy, cx, qi, true));
       }
     }
   }
@@ -577,7 +590,7 @@ __global__ void __launch_bounds__(TILE * Split<D>::G) k_bwd_dkdv(
 #pragma unroll
   for (int u = 0; u < CPT; ++u) {
     int c = lane * CPT + u;
-    kr[u] = active ? rot_channel(k + krow, ix.rope, g, c, cz, cy, cx, false) : 0.f;
+    kr[u] = active ? rot_channel(k + krow, ix.rope, g, c, cz, cy, cx, kj, false) : 0.f;
     vr[u] = active ? to_f32(v[krow + c]) : 0.f;
     dkr[u] = 0.f;
     dvr[u] = 0.f;
@@ -596,7 +609,7 @@ __global__ void __launch_bounds__(TILE * Split<D>::G) k_bwd_dkdv(
         halo_coord(tg, base + qq, z, y, x);
         int i = hl[base + qq];
         int64_t row = (((int64_t)b * g.N + i) * g.H + h) * D;
-        qv = rot_channel(q + row, ix.rope, g, c, z, y, x, false);
+        qv = rot_channel(q + row, ix.rope, g, c, z, y, x, i, false);
         dov = to_f32(dout[row + c]);
         if (c == 0) {
           cc.z[qq] = z;
@@ -653,7 +666,7 @@ __global__ void __launch_bounds__(TILE * Split<D>::G) k_bwd_dkdv(
 #pragma unroll
       for (int u = 0; u < CPT; ++u) {
         int c = lane * CPT + u;
-        dk[krow + c] = from_f32<T>(rot_channel_smem(sbuf + r * D, ix.rope, g, c, cz, cy, cx, true));
+        dk[krow + c] = from_f32<T>(rot_channel_smem(sbuf + r * D, ix.rope, g, c, cz, cy, cx, kj, true));
         dv[krow + c] = from_f32<T>(dvr[u]);
       }
     }

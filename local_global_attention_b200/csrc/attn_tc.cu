@@ -148,8 +148,8 @@ __device__ __forceinline__ void rot_chunk(uint4& lo, uint4& hi, const float2* t,
 // ---- grid-order rotated keys and values ------------------------------------------
 
 // One CTA per (64-voxel piece of an x row, row z * Y + y, batch item).  Key
-// items are (head, voxel, segment, half): 8 channels and their 8 partners,
-// rotated; value items (head, voxel, 16-byte chunk) are copied.  Consecutive
+// items are (head, voxel, item w of item96): 8 channels and their 8 rotation
+// partners, rotated; value items (head, voxel, 16-byte chunk) are copied.  Consecutive
 // threads cover one 192-byte row, so reads (through the volume) and writes
 // (grid order) are whole rows.
 constexpr int GRID_XS = 64;
@@ -166,24 +166,23 @@ __global__ void __launch_bounds__(256)
   const int64_t vox0 = ((int64_t)b * g.Z * g.Y + zy) * g.X + xb;
   for (int i = threadIdx.x; i < nx; i += blockDim.x) tok[i] = ix.vol[vox0 + i];
   __syncthreads();
-  const float2* tab = reinterpret_cast<const float2*>(ix.rope);
   const int H = g.H;
   // first element of (b, h, z, y, x = xb) in the grid-order volumes
   auto grid_row = [&](int h) {
     return ((((int64_t)b * H + h) * g.Z + z) * g.Y + y) * g.X + xb;
   };
   for (int it = threadIdx.x; it < H * nx * 6; it += blockDim.x) {
-    const int u = it & 1, s = (it >> 1) % 3, rem = it / 6;
+    const int w = it % 6, rem = it / 6;
     const int x = rem % nx, h = rem / nx;
-    const uint4* src = reinterpret_cast<const uint4*>(
-        k + (((int64_t)b * g.N + tok[x]) * H + h) * D + s * 32 + u * 8);
-    uint4 lo = __ldg(src), hi = __ldg(src + 2);
-    const int c = s == 0 ? z : (s == 1 ? y : xb + x);
-    const int row = (s == 0 ? 0 : (s == 1 ? g.Z : g.Z + g.Y)) + c;
-    rot_chunk(lo, hi, tab + row * 16, u * 8);
-    uint4* dst = reinterpret_cast<uint4*>(kg + (grid_row(h) + x) * D + s * 32 + u * 8);
-    dst[0] = lo;
-    dst[2] = hi;
+    const Item96 item = item96(g, w);
+    const uint4* src =
+        reinterpret_cast<const uint4*>(k + (((int64_t)b * g.N + tok[x]) * H + h) * D);
+    uint4 lo = __ldg(src + item.c1), hi = __ldg(src + item.c2);
+    const int c = item.a == 0 ? z : (item.a == 1 ? y : xb + x);
+    rot_chunk(lo, hi, rope_row96(ix.rope, g, item.a, c, tok[x]), item.j0);
+    uint4* dst = reinterpret_cast<uint4*>(kg + (grid_row(h) + x) * D);
+    dst[item.c1] = lo;
+    dst[item.c2] = hi;
   }
   for (int it = threadIdx.x; it < H * nx * 12; it += blockDim.x) {
     const int c = it % 12, rem = it / 12;
@@ -525,16 +524,22 @@ __global__ void __launch_bounds__(NTHREADS, 2)
             reinterpret_cast<const uint4*>(q + (((int64_t)b * g.N + qi) * g.H + h) * D);
 #pragma unroll
         for (int i = 0; i < 12; ++i) r[i] = __ldg(src + i);
-        const float2* tab = reinterpret_cast<const float2*>(ix.rope);
-        const float2* tz = tab + cz * 16;
-        const float2* ty = tab + (g.Z + cy) * 16;
-        const float2* tx = tab + (g.Z + g.Y + cx) * 16;
-        rot_chunk(r[0], r[2], tz, 0);
-        rot_chunk(r[1], r[3], tz, 8);
-        rot_chunk(r[4], r[6], ty, 0);
-        rot_chunk(r[5], r[7], ty, 8);
-        rot_chunk(r[8], r[10], tx, 0);
-        rot_chunk(r[9], r[11], tx, 8);
+        if (g.rope_mode == PACK3D_ROPE_PACKED) {
+          // one-dimensional rotation by the packed index: chunk w pairs with w + 6
+          const float2* tp = rope_row96(ix.rope, g, 0, 0, qi);
+#pragma unroll
+          for (int w = 0; w < 6; ++w) rot_chunk(r[w], r[w + 6], tp, 8 * w);
+        } else {
+          const float2* tz = rope_row96(ix.rope, g, 0, cz, qi);
+          const float2* ty = rope_row96(ix.rope, g, 1, cy, qi);
+          const float2* tx = rope_row96(ix.rope, g, 2, cx, qi);
+          rot_chunk(r[0], r[2], tz, 0);
+          rot_chunk(r[1], r[3], tz, 8);
+          rot_chunk(r[4], r[6], ty, 0);
+          rot_chunk(r[5], r[7], ty, 8);
+          rot_chunk(r[8], r[10], tx, 0);
+          rot_chunk(r[9], r[11], tx, 8);
+        }
       } else {
 #pragma unroll
         for (int i = 0; i < 12; ++i) r[i] = make_uint4(0, 0, 0, 0);

@@ -135,14 +135,17 @@ __global__ void k_halo_lists(Geo g, const int32_t* __restrict__ vol,
   }
 }
 
-// cos and sin of c * base^(-2j/da), evaluated in double precision.
+// cos and sin of c * base^(-2j/da) (axial: c a coordinate value of an axis)
+// or of p * base^(-2j/d) (packed mode: p a packed position), evaluated in
+// double precision.
 __global__ void k_rope_table(Geo g, float base, float* tab) {
-  int e = blockIdx.x * blockDim.x + threadIdx.x;
-  int rows = g.Z + g.Y + g.X;
-  if (e >= rows * g.half) return;
-  int row = e / g.half, j = e % g.half;
-  int c = row < g.Z ? row : (row < g.Z + g.Y ? row - g.Z : row - g.Z - g.Y);
-  double theta = pow((double)base, -2.0 * (double)j / (double)g.da);
+  int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  const bool packed = g.rope_mode == PACK3D_ROPE_PACKED;
+  int64_t rows = packed ? g.N : g.Z + g.Y + g.X;
+  if (e >= rows * g.rope_len) return;
+  int row = (int)(e / g.rope_len), j = (int)(e % g.rope_len);
+  int c = packed ? row : (row < g.Z ? row : (row < g.Z + g.Y ? row - g.Z : row - g.Z - g.Y));
+  double theta = pow((double)base, -2.0 * (double)j / (double)(packed ? g.d : g.da));
   double sn, cs;
   sincos((double)c * theta, &sn, &cs);
   tab[2 * e + 0] = (float)cs;
@@ -174,8 +177,10 @@ int launch_build_index(const Geo& g, const int16_t* coords, const pack3d_index* 
   k_halo_sizes<<<(g.nT + 255) / 256, 256, 0, s>>>(g, cnt);
   k_exclusive_scan<1024><<<1, 1024, 0, s>>>(cnt, idx->nbr_off, g.nT, 0, 0);
   k_halo_lists<<<dim3(g.nT, g.B), 256, 0, s>>>(g, idx->vol, idx->nbr_off, idx->nbr, idx->err);
-  int rows = (g.Z + g.Y + g.X) * g.half;
-  k_rope_table<<<(rows + 255) / 256, 256, 0, s>>>(g, rope_base, idx->rope);
+  const int64_t entries =
+      (g.rope_mode == PACK3D_ROPE_PACKED ? (int64_t)g.N : (int64_t)(g.Z + g.Y + g.X)) *
+      g.rope_len;
+  k_rope_table<<<(unsigned)((entries + 255) / 256), 256, 0, s>>>(g, rope_base, idx->rope);
   return cuda_status(cudaGetLastError());
 }
 

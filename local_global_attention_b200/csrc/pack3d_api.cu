@@ -31,6 +31,8 @@ int make_geo(const pack3d_params* p, Geo* g) {
   if (!(p->rope_base > 0.f) || !isfinite(p->rope_base) || !isfinite(p->scale))
     return PACK3D_ERR_ARG;
   if (p->dtype != PACK3D_BF16 && p->dtype != PACK3D_FP32) return PACK3D_ERR_ARG;
+  if (p->rope_mode != PACK3D_ROPE_AXIAL && p->rope_mode != PACK3D_ROPE_PACKED)
+    return PACK3D_ERR_ARG;
   int64_t N = (int64_t)p->Z * p->Y * p->X;
   if ((int64_t)p->B * N * p->H * p->head_dim >= (int64_t)1 << 31) return PACK3D_ERR_ARG;
   if (p->head_dim != 12 && p->head_dim != 24 && p->head_dim != 48 && p->head_dim != 96)
@@ -64,6 +66,8 @@ int make_geo(const pack3d_params* p, Geo* g) {
   g->tau = p->scale > 0.f ? p->scale : 1.0f / sqrtf((float)p->head_dim);
   g->dtype = p->dtype;
   g->out_fp32 = (p->out_fp32 != 0 || p->dtype == PACK3D_FP32) ? 1 : 0;
+  g->rope_mode = p->rope_mode;
+  g->rope_len = p->rope_mode == PACK3D_ROPE_PACKED ? p->head_dim / 2 : g->half;
   return PACK3D_OK;
 }
 
@@ -89,7 +93,11 @@ IndexLayout index_layout(const Geo& g) {
   L.nbr = o;
   o += align256(sizeof(int32_t) * (size_t)g.B * g.n_halo);
   L.rope = o;
-  o += align256(sizeof(float) * 2 * (size_t)(g.Z + g.Y + g.X) * g.half);
+  // rotation table: a row per coordinate value of each axis (axial) or per
+  // packed position (packed mode)
+  const size_t rope_rows = g.rope_mode == PACK3D_ROPE_PACKED ? (size_t)g.N
+                                                             : (size_t)(g.Z + g.Y + g.X);
+  o += align256(sizeof(float) * 2 * rope_rows * g.rope_len);
   L.err = o;
   o += 256;
   L.total = o;

@@ -24,6 +24,8 @@ struct Geo {
   float tau;                  // softmax scale
   int dtype;                  // PACK3D_BF16 / PACK3D_FP32
   int out_fp32;               // out is fp32 (also when dtype is bf16)
+  int rope_mode;              // PACK3D_ROPE_AXIAL / PACK3D_ROPE_PACKED
+  int rope_len;               // (cos, sin) pairs per rotation-table row
 };
 
 int make_geo(const pack3d_params* p, Geo* g);  // PACK3D_OK or PACK3D_ERR_*
@@ -52,10 +54,49 @@ __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
   return __float2bfloat16_rn(x);
 }
 
-// Rotation table entry (cos, sin) for axis a, coordinate c, pair j.
-__device__ __forceinline__ float2 rope_cs(const float* tab, const Geo& g, int a, int c, int j) {
+// Rotation table entry (cos, sin) of pair j for a token: axial mode, the row of
+// coordinate c on axis a (rows: Z values, then Y, then X); packed mode, the row
+// of the token's packed index pos.
+__device__ __forceinline__ float2 rope_cs(const float* tab, const Geo& g, int a, int c, int pos,
+                                          int j) {
+  const float2* t = reinterpret_cast<const float2*>(tab);
+  if (g.rope_mode == PACK3D_ROPE_PACKED) return t[(int64_t)pos * g.rope_len + j];
   int off = a == 0 ? 0 : (a == 1 ? g.Z : g.Z + g.Y);
-  return reinterpret_cast<const float2*>(tab)[(off + c) * g.half + j];
+  return t[(off + c) * g.rope_len + j];
+}
+
+// First (cos, sin) of a row of the rotation table used by the 16-byte-chunk
+// kernels (head_dim 96): axial mode, axis a's row of coordinate c; packed mode,
+// the row of position pos.
+__device__ __forceinline__ const float2* rope_row96(const float* tab, const Geo& g, int a, int c,
+                                                    int pos) {
+  const float2* t = reinterpret_cast<const float2*>(tab);
+  if (g.rope_mode == PACK3D_ROPE_PACKED) return t + (int64_t)pos * 48;
+  return t + ((a == 0 ? 0 : (a == 1 ? g.Z : g.Z + g.Y)) + c) * 16;
+}
+
+// Item w (0..5) of a head-dim-96 row for the chunk kernels: 16-byte chunk c1
+// (8 channels, the first members of 8 rotation pairs), its partner chunk c2,
+// the first pair index j0 in the table row, and the axis whose coordinate
+// selects the row.  Axial: segment a = w / 2 (32 channels), pairs (j, j + 16);
+// packed: pairs (j, j + 48) over the whole row.
+struct Item96 {
+  int c1, c2, j0, a;
+};
+__device__ __forceinline__ Item96 item96(const Geo& g, int w) {
+  Item96 it;
+  if (g.rope_mode == PACK3D_ROPE_PACKED) {
+    it.c1 = w;
+    it.c2 = w + 6;
+    it.j0 = 8 * w;
+    it.a = 0;
+  } else {
+    it.a = w / 2;
+    it.c1 = 4 * it.a + (w & 1);
+    it.c2 = it.c1 + 2;
+    it.j0 = 8 * (w & 1);
+  }
+  return it;
 }
 
 // ---- launchers (defined in the .cu files) --------------------------------

@@ -50,10 +50,14 @@ __global__ void __launch_bounds__(256) k_block_summaries(Geo g, const int32_t* _
   const int lane = threadIdx.x % lanes, grp = threadIdx.x / lanes;
   const int blk = blockIdx.x, b = blockIdx.y, h = blockIdx.z;
   const int Bz = blk / (g.nby * g.nbx), By = (blk / g.nbx) % g.nby, Bx = blk % g.nbx;
-  // Lane -> axis a and first pair j (pairs j, j+1 of that axis).
+  // Lane -> axis a and first pair j (pairs j, j+1 of that axis); packed mode:
+  // pairs j, j + 1 of the whole row, partners d/2 channels on.
+  const bool packed = g.rope_mode == PACK3D_ROPE_PACKED;
   const int pairs_per_axis = g.half / 2;  // lanes per axis
-  const int a = lane / pairs_per_axis, j = (lane % pairs_per_axis) * 2;
-  const int c1 = a * g.da + j, c2 = c1 + g.half;  // channels of x1 (and +1), x2 (and +1)
+  const int a = packed ? 0 : lane / pairs_per_axis;
+  const int j = packed ? lane * 2 : (lane % pairs_per_axis) * 2;
+  const int c1 = packed ? j : a * g.da + j;  // channels of x1 (and +1)
+  const int c2 = c1 + g.rope_len;            // channels of x2 (and +1)
   float kx1a = 0.f, kx1b = 0.f, kx2a = 0.f, kx2b = 0.f;
   float vx1a = 0.f, vx1b = 0.f, vx2a = 0.f, vx2b = 0.f;
   const int cnt = g.bz * g.by * g.bx;
@@ -70,7 +74,7 @@ __global__ void __launch_bounds__(256) k_block_summaries(Geo g, const int32_t* _
       float2 v1 = Pair2<T>::f(*reinterpret_cast<const P2*>(v + row + c1));
       float2 v2 = Pair2<T>::f(*reinterpret_cast<const P2*>(v + row + c2));
       int ca = a == 0 ? cz : (a == 1 ? cy : cx);
-      float2 csa = rope_cs(rope, g, a, ca, j), csb = rope_cs(rope, g, a, ca, j + 1);
+      float2 csa = rope_cs(rope, g, a, ca, tok, j), csb = rope_cs(rope, g, a, ca, tok, j + 1);
       kx1a += k1.x * csa.x - k2.x * csa.y;
       kx2a += k1.x * csa.y + k2.x * csa.x;
       kx1b += k1.y * csb.x - k2.y * csb.y;
@@ -136,13 +140,16 @@ __global__ void __launch_bounds__(TG96 * LANES96) k_block_summaries_bf16_d96(
   const int blk = blockIdx.x, b = blockIdx.y, h = blockIdx.z * HG96 + hh;
   const bool live = h < g.H;
   const int Bz = blk / (g.nby * g.nbx), By = (blk / g.nbx) % g.nby, Bx = blk % g.nbx;
-  const int a = w / 2, c1 = 4 * a + (w & 1), c2 = c1 + 2, j0 = 8 * (w & 1);
+  const Item96 item = item96(g, w);
+  const int a = item.a, c1 = item.c1, c2 = item.c2, j0 = item.j0;
+  const bool packed = g.rope_mode == PACK3D_ROPE_PACKED;
   // rotation-table rows of this block's coordinates (z, then y, then x rows),
-  // staged in shared memory when they fit
+  // staged in shared memory when they fit (packed mode: the rows of the tokens'
+  // positions, read from the table)
   const float2* gtab = reinterpret_cast<const float2*>(rope);
   const float2* tab;  // row of coordinate c on this lane's axis: tab + (c - base) * stride
   int base, stride;
-  const bool staged = g.bz + g.by + g.bx <= TAB96;
+  const bool staged = !packed && g.bz + g.by + g.bx <= TAB96;
   if (staged) {
     const int rows = g.bz + g.by + g.bx;
     for (int e = threadIdx.x; e < rows * 16; e += blockDim.x) {
@@ -174,9 +181,10 @@ __global__ void __launch_bounds__(TG96 * LANES96) k_block_summaries_bf16_d96(
   // One token's rows (already loaded): rotate, accumulate, and with STAGE
   // write the grid-order copies.
   auto consume = [&](const uint4& ka, const uint4& kb, const uint4& va, const uint4& vb2, int cz,
-                     int cy, int cx) {
+                     int cy, int cx, int tok_of_consume) {
     const int ca = a == 0 ? cz : (a == 1 ? cy : cx);
-    const float2* t = tab + (ca - base) * stride + j0;
+    const float2* t = packed ? rope_row96(rope, g, 0, 0, tok_of_consume) + j0
+                             : tab + (ca - base) * stride + j0;
     const uint32_t* kaw = reinterpret_cast<const uint32_t*>(&ka);
     const uint32_t* kbw = reinterpret_cast<const uint32_t*>(&kb);
     const uint32_t* vaw = reinterpret_cast<const uint32_t*>(&va);
@@ -248,8 +256,8 @@ __global__ void __launch_bounds__(TG96 * LANES96) k_block_summaries_bf16_d96(
         vbA = __ldg(vrb + c1);
         vbB = __ldg(vrb + c2);
       }
-      consume(ka, kb, va, vb2, az, ay, ax);
-      if (has_b) consume(kbA, kbB, vbA, vbB, bz2, by2, bx2);
+      consume(ka, kb, va, vb2, az, ay, ax, ta);
+      if (has_b) consume(kbA, kbB, vbA, vbB, bz2, by2, bx2, tb2);
     }
     ta = nta;
     tb2 = ntb;
@@ -299,6 +307,7 @@ constexpr uint32_t BS_WAIT = 1u << 22;
 struct BulkSmem {
   uint8_t ring[BS_STAGES][BS_TPS][2][BS_ROW];  // reused for the final reduction
   float2 tab[TAB96 * TABS96];
+  int32_t tok[BS_STAGES][BS_TPS];  // packed index of each slot's token
   uint64_t full[BS_STAGES], empty[BS_STAGES];
   int32_t abort;
 };
@@ -332,7 +341,8 @@ __global__ void __launch_bounds__(BS_THREADS, 2) k_summaries_bulk(
   }
   // rotation-table rows of this block's coordinates (z rows, y rows, x rows)
   const float2* gtab = reinterpret_cast<const float2*>(rope);
-  for (int e = tid; e < (g.bz + g.by + g.bx) * 16; e += BS_THREADS) {
+  const int tab_rows = g.rope_mode == PACK3D_ROPE_PACKED ? 0 : g.bz + g.by + g.bx;
+  for (int e = tid; e < tab_rows * 16; e += BS_THREADS) {
     const int r = e / 16, jj = e % 16;
     const int grow = r < g.bz ? Bz * g.bz + r
                               : (r < g.bz + g.by ? g.Z + By * g.by + r - g.bz
@@ -361,12 +371,17 @@ __global__ void __launch_bounds__(BS_THREADS, 2) k_summaries_bulk(
         ok = mbar_wait_or_abort(&sm.empty[s], ((r / BS_STAGES) - 1) & 1, BS_WAIT, abort_flag);
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       const int ntok = min(BS_TPS, cnt - r * BS_TPS);
-      if (lane == 0) mbar_arrive_expect_tx(&sm.full[s], (uint32_t)ntok * 2 * row_bytes);
-      __syncwarp();
+      int64_t tok = 0;
       if (lane < ntok) {
         int cz, cy, cx;
         voxel(r * BS_TPS + lane, cz, cy, cx);
-        const int64_t tok = vb[(cz * g.Y + cy) * g.X + cx];
+        tok = vb[(cz * g.Y + cy) * g.X + cx];
+        sm.tok[s][lane] = (int32_t)tok;  // published by the arrive below
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive_expect_tx(&sm.full[s], (uint32_t)ntok * 2 * row_bytes);
+      __syncwarp();
+      if (lane < ntok) {
         bulk_load(sm.ring[s][lane][0], k + (((int64_t)b * g.N + tok) * g.H) * 96, row_bytes,
                   &sm.full[s]);
         bulk_load(sm.ring[s][lane][1], v + (((int64_t)b * g.N + tok) * g.H) * 96, row_bytes,
@@ -382,7 +397,9 @@ __global__ void __launch_bounds__(BS_THREADS, 2) k_summaries_bulk(
     // ---- consumers ----
     const int h = c / 6, w = c % 6;
     const bool live = h < g.H;
-    const int a = w / 2, c1 = 4 * a + (w & 1), c2 = c1 + 2, j0 = 8 * (w & 1);
+    const Item96 item = item96(g, w);
+    const int a = item.a, c1 = item.c1, c2 = item.c2, j0 = item.j0;
+    const bool packed = g.rope_mode == PACK3D_ROPE_PACKED;
     const float2* tab = a == 0 ? sm.tab : (a == 1 ? sm.tab + g.bz * TABS96 : sm.tab + (g.bz + g.by) * TABS96);
     const int base = a == 0 ? Bz * g.bz : (a == 1 ? By * g.by : Bx * g.bx);
     for (int r = 0; r < n_stage_rounds; ++r) {
@@ -398,7 +415,8 @@ __global__ void __launch_bounds__(BS_THREADS, 2) k_summaries_bulk(
         const uint4* vr = reinterpret_cast<const uint4*>(sm.ring[s][grp][1] + h * 192);
         const uint4 ka = kr[c1], kb = kr[c2], va = vr[c1], vb2 = vr[c2];
         const int ca = a == 0 ? cz : (a == 1 ? cy : cx);
-        const float2* t = tab + (ca - base) * TABS96 + j0;
+        const float2* t = packed ? rope_row96(rope, g, 0, 0, sm.tok[s][grp]) + j0
+                                 : tab + (ca - base) * TABS96 + j0;
         const uint32_t* kaw = reinterpret_cast<const uint32_t*>(&ka);
         const uint32_t* kbw = reinterpret_cast<const uint32_t*>(&kb);
         const uint32_t* vaw = reinterpret_cast<const uint32_t*>(&va);
@@ -466,9 +484,17 @@ __global__ void __launch_bounds__(BS_THREADS, 2) k_summaries_bulk(
   const float inv_cnt = 1.f / (float)cnt;
   for (int o = tid; o < g.H * 2 * 96; o += BS_THREADS) {
     const int h = o / 192, which = (o / 96) % 2, ch = o % 96;
-    // channel ch of head h lives in item (h, w) at slot 8 * (half) + i
-    const int seg = ch / 32, within = ch % 32, hi = within >= 16, jj = within % 16;
-    const int w = seg * 2 + (jj >= 8), i = jj % 8;
+    // channel ch of head h: 16-byte chunk ch / 8 is chunk c1 (slots 0-7) or c2
+    // (slots 8-15) of one item w of item96; values at slots 16-31
+    const int chunk = ch / 8, i = ch % 8;
+    int w, hi;
+    if (g.rope_mode == PACK3D_ROPE_PACKED) {
+      hi = chunk >= 6;
+      w = chunk % 6;
+    } else {
+      hi = (chunk & 3) >= 2;
+      w = 2 * (chunk >> 2) + (chunk & 1);
+    }
     const int slot = (which ? 16 : 0) + (hi ? 8 : 0) + i;
     float acc = 0.f;
     for (int q = 0; q < BS_TPS; ++q) acc += red[(q * BS_ITEMS + h * 6 + w) * 32 + slot];

@@ -16,6 +16,7 @@ import torch
 from . import build as _build
 
 BF16, FP32 = 0, 1
+ROPE_AXIAL, ROPE_PACKED = 0, 1  # axial RoPE on grid coordinates / 1-D RoPE on the packed index
 OK, ERR_ARG, ERR_COORDS, ERR_CUDA, ERR_TIMEOUT, ERR_UNSUPPORTED = 0, -1, -2, -3, -4, -5
 
 EXPORTS = ("pack3d_index_bytes", "pack3d_index_init", "pack3d_build_index", "pack3d_index_check",
@@ -29,7 +30,7 @@ class Params(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
                 ("B", "H", "head_dim", "Z", "Y", "X", "wz", "wy", "wx", "bz", "by", "bx")] + [
         ("rope_base", ctypes.c_float), ("scale", ctypes.c_float), ("dtype", ctypes.c_int32),
-        ("out_fp32", ctypes.c_int32)]
+        ("out_fp32", ctypes.c_int32), ("rope_mode", ctypes.c_int32)]
 
 
 class Index(ctypes.Structure):
@@ -106,13 +107,14 @@ def _check(status: int, what: str):
 
 def make_params(shape, dtype=None, scale: float = 0.0, out_fp32: bool = False) -> Params:
     """Params from any object with ``B, H, d, Z, Y, X, window, block, rope_base``
-    (and ``dtype`` "bf16"/"fp32" unless given).  ``out_fp32`` makes the forward
-    output fp32 for bf16 inputs."""
+    (and ``dtype`` "bf16"/"fp32" unless given, ``rope_mode`` 0 unless set).
+    ``out_fp32`` makes the forward output fp32 for bf16 inputs."""
     dt = dtype if dtype is not None else getattr(shape, "dtype", "bf16")
     code = {"bf16": BF16, "fp32": FP32, torch.bfloat16: BF16, torch.float32: FP32}[dt]
     w, b = tuple(shape.window), tuple(shape.block)
     return Params(shape.B, shape.H, shape.d, shape.Z, shape.Y, shape.X, w[0], w[1], w[2],
-                  b[0], b[1], b[2], float(shape.rope_base), float(scale), code, int(bool(out_fp32)))
+                  b[0], b[1], b[2], float(shape.rope_base), float(scale), code, int(bool(out_fp32)),
+                  int(getattr(shape, "rope_mode", 0) or 0))
 
 
 def out_dtype(params: Params, like: torch.Tensor) -> torch.dtype:

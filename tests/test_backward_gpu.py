@@ -50,3 +50,15 @@ def test_backward_train65k_properties():
     sdo = inp["dout"].double().sum(dim=1)
     rel = ((sdv - sdo).abs().max() / sdo.abs().max()).item()
     assert rel < 2e-2, rel
+
+
+PACKED_CASES = [
+    CASES[1].replace(name="packed_rope_fp32_6x10x20", rope_mode=1, seed=45),
+    CASES[2].replace(name="packed_rope_bf16_6x10x20", rope_mode=1, seed=46),
+]
+
+
+@pytest.mark.parametrize("wl", PACKED_CASES, ids=lambda w: w.name)
+def test_backward_packed_rope_mode(oracle_lib, wl):
+    """The comparison mode (1-D RoPE on the packed index) through the backward."""
+    test_backward_full(oracle_lib, wl)
