@@ -231,17 +231,25 @@ def run_ours(args):
     lib = P.load()
     import ctypes
     sp = ctypes.c_void_p(stream.cuda_stream)
-    pp, ip = ctypes.byref(params), ctypes.byref(idx.struct)
+    pp_ax, ip_ax = ctypes.byref(params), ctypes.byref(idx.struct)
     ptr = lambda t: ctypes.c_void_p(t.data_ptr())
 
     fwd_events = []
 
-    def step(record=False, window=False, bufs=None, res=None):
+    # the packed-sequence comparison mode (1-D RoPE on the packed index): its own
+    # params and index (the rotation table differs), the same step
+    params_pk = P.make_params(wl_r)
+    params_pk.rope_mode = P.ROPE_PACKED
+    idx_pk = P.IndexBuffers(params_pk)
+    pp_pk, ip_pk = ctypes.byref(params_pk), ctypes.byref(idx_pk.struct)
+
+    def step(record=False, window=False, bufs=None, res=None, packed_rope=False):
         # index build; block summaries computed in the pass that stages the
         # rotated keys and the values in grid order (pack3d_stage_kv); the
         # attention (pack3d_forward_staged), timed on its own
         d_ = dev if bufs is None else bufs
         o_, l_ = (out, lse) if res is None else res
+        pp, ip = (pp_pk, ip_pk) if packed_rope else (pp_ax, ip_ax)
         rc = lib.pack3d_build_index(pp, ptr(d_["coords"]), ip, sp)
         rc |= lib.pack3d_stage_kv(pp, ip, ptr(d_["k"]), ptr(d_["v"]),
                                   None if window else ptr(ksum), None if window else ptr(vsum),
@@ -258,9 +266,9 @@ def run_ours(args):
         if rc:
             raise RuntimeError(f"pack3d call failed: {rc}")
 
-    def timed(window=False, record=False):
+    def timed(window=False, record=False, packed_rope=False):
         for _ in range(args.warmup):
-            step(window=window)
+            step(window=window, packed_rope=packed_rope)
         torch.cuda.synchronize()
         barrier(world)
         torch.cuda.synchronize()
@@ -268,7 +276,7 @@ def run_ours(args):
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record(stream)
         for _ in range(args.steps):
-            step(record=record, window=window)
+            step(record=record, window=window, packed_rope=packed_rope)
         t1.record(stream)
         torch.cuda.synchronize()
         barrier(world)
@@ -282,6 +290,9 @@ def run_ours(args):
         raise RuntimeError(f"index status {P.strerror(st)}")
     fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in fwd_events)
     window_ms = timed(window=True)
+    packed_ms = timed(packed_rope=True)
+    if P.pack3d_index_check(idx_pk) != P.OK:
+        raise RuntimeError("index status of the packed-RoPE run")
 
     # End to end through the C ABI: every step copies its inputs from pinned
     # host memory and reads its outputs back.  Two device buffer sets and two
@@ -389,6 +400,8 @@ def run_ours(args):
         },
         "window_only": {"ms_per_step": window_ms, "value": tokens / (window_ms * 1e-3),
                         "pack3d_over_window": ms / window_ms},
+        "packed_rope_mode": {"ms_per_step": packed_ms, "value": tokens / (packed_ms * 1e-3),
+                             "note": "comparison mode: 1-D RoPE on the packed index, same step"},
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": UNIT, "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "clocks": clk.summary(),
