@@ -39,6 +39,7 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "forward_tc_vol_32x32x64.md")
 TC_SOURCE = os.path.join(ROOT, "local_global_attention_b200", "csrc", "attn_tc.cu")
+FP32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # CUDA-core fp32 FMA peak, nominal
 KERNELS_PER_STEP = 11  # index build 9, summaries + staging 1, attention 1
 
 
@@ -83,7 +84,11 @@ def algorithmic_work(wl):
     esz = 2
     rows = wl.B * wl.N * wl.H * wl.d
     hbm = rows * esz * 4 + wl.B * wl.H * wl.N * 4 + rows * esz * 2
+    # backward: S recomputed (2d), dP = dO.v (2d), dq, dk and dv updates (2d
+    # each): 10 d FLOPs per local and per summary term
+    per_bh_bwd = 10.0 * wl.d * (local_terms + sum_terms)
     return {"local_flop": BH * per_bh_local, "summary_flop": BH * per_bh_sum,
+            "bwd_flop": BH * per_bh_bwd,
             "flop": BH * (per_bh_local + per_bh_sum), "hbm_bytes": hbm,
             "fwd_bytes": rows * esz * 4 + wl.B * wl.H * wl.N * 4}
 
@@ -291,6 +296,37 @@ def run_ours(args):
     fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in fwd_events)
     window_ms = timed(window=True)
     packed_ms = timed(packed_rope=True)
+
+    # the backward (dq, dk, dv from the forward's out and lse) at the same shape,
+    # with dO ~ N(0, 1): CUDA cores, fp32 arithmetic
+    g_do = torch.Generator().manual_seed(wl_r.seed + 7)
+    dout = torch.randn(B, N, H, d, generator=g_do).to(dev["q"].dtype).cuda()
+    dq, dk, dv = (torch.empty_like(dev["q"]) for _ in range(3))
+    bws_bytes = P.pack3d_backward_workspace_bytes(params)
+    bws = torch.empty(max(bws_bytes, 1), dtype=torch.uint8, device="cuda")
+    step()  # the forward the backward reads
+
+    def backward():
+        rc = lib.pack3d_backward(pp_ax, ip_ax, ptr(dev["q"]), ptr(dev["k"]), ptr(dev["v"]),
+                                 ptr(out), ptr(lse), ptr(dout), ptr(dq), ptr(dk), ptr(dv),
+                                 ptr(bws), ctypes.c_size_t(bws_bytes), sp)
+        if rc:
+            raise RuntimeError(f"pack3d_backward failed: {rc}")
+
+    bw_steps = max(3, min(args.steps, 20))
+    for _ in range(3):
+        backward()
+    torch.cuda.synchronize()
+    b0 = torch.cuda.Event(enable_timing=True)
+    b1 = torch.cuda.Event(enable_timing=True)
+    b0.record(stream)
+    for _ in range(bw_steps):
+        backward()
+    b1.record(stream)
+    torch.cuda.synchronize()
+    bwd_ms = max_over_ranks(b0.elapsed_time(b1) / bw_steps, world)
+    if P.pack3d_index_check(idx) != P.OK:
+        raise RuntimeError("index status after the backward")
     if P.pack3d_index_check(idx_pk) != P.OK:
         raise RuntimeError("index status of the packed-RoPE run")
 
@@ -397,6 +433,18 @@ def run_ours(args):
             "algorithmic_flop_per_launch": work["flop"],
             "forward_ms": fwd_ms,
             "forward_hbm_frac": (work["fwd_bytes"] / (fwd_ms * 1e-3) / 1e9) / pk["hbm_gbs"],
+        },
+        "backward": {
+            "ms_per_call": bwd_ms,
+            "calls": bw_steps,
+            "kernels": "attn_simt.cu (CUDA cores, fp32 arithmetic)",
+            "roofline": {"bound": "alu", "unit": "TFLOP/s",
+                         "achieved": work["bwd_flop"] / (bwd_ms * 1e-3) / 1e12,
+                         "peak": FP32_TFLOPS,
+                         "frac": work["bwd_flop"] / (bwd_ms * 1e-3) / 1e12 / FP32_TFLOPS,
+                         "peak_source": "148 SMs x 128 fp32 FMA lanes x 2 FLOP x 1.965 GHz "
+                                        "(nominal unit count and clock)",
+                         "algorithmic_flop_per_call": work["bwd_flop"]},
         },
         "window_only": {"ms_per_step": window_ms, "value": tokens / (window_ms * 1e-3),
                         "pack3d_over_window": ms / window_ms},
