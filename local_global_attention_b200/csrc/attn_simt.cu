@@ -14,6 +14,8 @@
 // coordinate array is read.
 #include <math.h>
 
+#include <algorithm>
+
 #include "pack3d_internal.cuh"
 
 namespace p3d {
@@ -112,8 +114,86 @@ __device__ __forceinline__ float rot_channel_smem(const float* row, const float*
 }
 
 struct ChunkCoords {
-  int z[KC], y[KC], x[KC];
+  int z[KC], y[KC], x[KC], tok[KC];
 };
+
+// Dot product of a thread's CPT channels with a staged fp32 row (16-byte
+// aligned), summed in channel order, read 16 bytes at a time.
+template <int CPT>
+__device__ __forceinline__ float dot_row(const float (&r)[CPT], const float* row) {
+  static_assert(CPT % 4 == 0, "channels per thread must be a multiple of 4");
+  const float4* p = reinterpret_cast<const float4*>(row);
+  float acc = 0.f;
+#pragma unroll
+  for (int v = 0; v < CPT / 4; ++v) {
+    const float4 x = p[v];
+    acc += r[4 * v] * x.x;
+    acc += r[4 * v + 1] * x.y;
+    acc += r[4 * v + 2] * x.z;
+    acc += r[4 * v + 3] * x.w;
+  }
+  return acc;
+}
+
+// Stage a chunk of token rows into shared memory as fp32: xo = R(c) x (the
+// rotated row) and yo = y (plain), for the tokens whose packed index and
+// coordinate the caller has put into tok / cz / cy / cx.  NT threads share
+// the chunk, NT / ROWS per row, each rotation pair (both channels of it) read
+// once; every thread's loads are independent, so their latencies overlap.
+// Rows nrows .. ROWS-1 are zero-filled.
+template <typename T, int D, int ROWS, int NT>
+__device__ __forceinline__ void stage_rows(const Geo& g, const float* __restrict__ rope,
+                                           const T* __restrict__ x, const T* __restrict__ y,
+                                           int b, int h, const int* tok, const int* cz,
+                                           const int* cy, const int* cx, int nrows, float* xo,
+                                           float* yo, int ld) {
+  static_assert(NT % ROWS == 0, "threads must divide evenly over the rows");
+  constexpr int TPR = NT / ROWS, PAIRS = D / 2, HALF = D / 6, DA = D / 3;
+  const int r = threadIdx.x / TPR, sub = threadIdx.x % TPR;
+  float* xr = xo + r * ld;
+  float* yr = yo + r * ld;
+  if (r >= nrows) {
+    for (int c = sub; c < D; c += TPR) xr[c] = yr[c] = 0.f;
+    return;
+  }
+  const int i = tok[r];
+  const int64_t row = (((int64_t)b * g.N + i) * g.H + h) * D;
+  const bool packed = g.rope_mode == PACK3D_ROPE_PACKED;
+#pragma unroll
+  for (int m = 0; m < (PAIRS + TPR - 1) / TPR; ++m) {
+    const int pr = sub + m * TPR;
+    if (pr < PAIRS) {
+      int a = 0, ca = 0, j = pr, c1 = pr, c2 = pr + PAIRS;
+      if (!packed) {
+        a = pr / HALF;
+        j = pr - a * HALF;
+        c1 = a * DA + j;
+        c2 = c1 + HALF;
+        ca = a == 0 ? cz[r] : (a == 1 ? cy[r] : cx[r]);
+      }
+      const float2 cs = rope_cs(rope, g, a, ca, i, j);
+      const float x1 = to_f32(x[row + c1]), x2 = to_f32(x[row + c2]);
+      xr[c1] = x1 * cs.x - x2 * cs.y;
+      xr[c2] = x1 * cs.y + x2 * cs.x;
+      yr[c1] = to_f32(y[row + c1]);
+      yr[c2] = to_f32(y[row + c2]);
+    }
+  }
+}
+
+// acc[u] += a * row[u] over a thread's CPT channels of a staged fp32 row.
+template <int CPT>
+__device__ __forceinline__ void axpy_row(float (&acc)[CPT], float a, const float* row) {
+  const float4* p = reinterpret_cast<const float4*>(row);
+#pragma unroll
+  for (int v = 0; v < CPT / 4; ++v) {
+    const float4 x = p[v];
+    acc[4 * v] += a * x.x;
+    acc[4 * v + 1] += a * x.y;
+    acc[4 * v + 2] += a * x.z;
+    acc[4 * v + 3] += a * x.w;
+  }
+}
 
 // ---------------------------------------------------------------------------
 // Forward
@@ -313,10 +393,12 @@ __global__ void __launch_bounds__(256) k_bwd_summary(Geo g, pack3d_index ix,
                                                     const float* __restrict__ vsum, float* dks,
                                                     float* dvs) {
   if (ix.err[0]) return;
-  __shared__ float sq[QC][D];
-  __shared__ float sdo[QC][D];
-  __shared__ float skb[BC][D];
-  __shared__ float svb[BC][D];
+  // rows padded to D + 1 floats: the dot products read rows kk of skb / svb at
+  // the same channel from 8 threads, which would otherwise share a bank
+  __shared__ float sq[QC][D + 1];
+  __shared__ float sdo[QC][D + 1];
+  __shared__ float skb[BC][D + 1];
+  __shared__ float svb[BC][D + 1];
   __shared__ float sP[QC][BC];
   __shared__ float sdS[QC][BC];
   __shared__ int sqc[QC][3];
@@ -420,6 +502,203 @@ __global__ void __launch_bounds__(256) k_bwd_summary(Geo g, pack3d_index ix,
   }
 }
 
+// Summary gradients for d = 96, register-tiled.  One CTA owns a chunk of
+// S96_NB summaries of one (batch item, head) and a contiguous range of query
+// tiles (a split); it keeps k̄, v̄ of its summaries in shared memory and walks
+// its queries in chunks of S96_QC:
+//   phase 1: S = q~ k̄^T and dP = dO v̄^T for the chunk (each warp a 16 x 16
+//            piece, each thread 2 x 4 of both, float4 operand reads);
+//            P = exp(tau S - lse) where the query's window misses the block
+//            (0 where it meets it), dS = P (dP - delta), both to shared memory;
+//   phase 2: dk̄ += dS^T q~ and dv̄ += P^T dO, each thread 4 summaries x 6
+//            channels of both in registers.
+// Partial sums per split go to a workspace and are added in split order by
+// k_bwd_summary_reduce, so the result does not depend on scheduling.
+constexpr int S96_NB = 64, S96_QC = 32, S96_LD = 100, S96_LDP = 68, S96_THREADS = 256;
+
+struct Sum96Smem {
+  float ks[S96_NB][S96_LD];
+  float vs[S96_NB][S96_LD];
+  float q[S96_QC][S96_LD];
+  float dout[S96_QC][S96_LD];
+  float p[S96_QC][S96_LDP];
+  float ds[S96_QC][S96_LDP];
+  float lse[S96_QC], del[S96_QC];
+  int qz[S96_QC], qy[S96_QC], qx[S96_QC], tok[S96_QC];
+  int bz0[S96_NB], by0[S96_NB], bx0[S96_NB];
+};
+
+template <typename T>
+__global__ void __launch_bounds__(S96_THREADS, 2) k_bwd_summary96(
+    Geo g, pack3d_index ix, const T* __restrict__ q, const T* __restrict__ dout,
+    const float* __restrict__ lse, const float* __restrict__ delta,
+    const float* __restrict__ ksum, const float* __restrict__ vsum, int nsplit,
+    float* __restrict__ part) {
+  constexpr int D = 96;
+  if (ix.err[0]) return;
+  extern __shared__ __align__(16) unsigned char s96_raw[];
+  Sum96Smem& sm = *reinterpret_cast<Sum96Smem*>(s96_raw);
+  const int nbc = (g.nb + S96_NB - 1) / S96_NB;
+  const int bc = blockIdx.x % nbc, split = blockIdx.x / nbc;
+  const int b = blockIdx.y, h = blockIdx.z, B0 = bc * S96_NB;
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int64_t sbase = ((int64_t)b * g.H + h) * g.nb;
+  for (int e = tid; e < S96_NB * D; e += S96_THREADS) {
+    int r = e / D, c = e % D;
+    bool ok = B0 + r < g.nb;
+    sm.ks[r][c] = ok ? ksum[(sbase + B0 + r) * D + c] : 0.f;
+    sm.vs[r][c] = ok ? vsum[(sbase + B0 + r) * D + c] : 0.f;
+    if (c == 0) {
+      int Bk = B0 + r;
+      sm.bz0[r] = (Bk / (g.nby * g.nbx)) * g.bz;
+      sm.by0[r] = ((Bk / g.nbx) % g.nby) * g.by;
+      sm.bx0[r] = (Bk % g.nbx) * g.bx;
+    }
+  }
+  // phase-1 roles: warp piece (wq, wb) of 16 queries x 16 summaries; lane
+  // (lq, lb) takes queries wq*16 + lq + 8i and summaries wb*16 + lb + 4j
+  const int wq = warp / 4, wb = warp % 4, lq = lane / 4, lb = lane % 4;
+  // phase-2 roles: summaries 4*tb .. 4*tb+3, channels 6*tc .. 6*tc+5
+  const int tb = tid / 16, tc = tid % 16;
+  float dk[4][6], dv[4][6];
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+#pragma unroll
+    for (int u = 0; u < 6; ++u) dk[j][u] = dv[j][u] = 0.f;
+
+  const int t0 = (int)((int64_t)split * g.nT / nsplit);
+  const int t1 = (int)((int64_t)(split + 1) * g.nT / nsplit);
+  const int64_t lbase = ((int64_t)b * g.H + h) * g.N;
+  for (int t = t0; t < t1; ++t) {
+    const TileGeo tg = tile_geo(g, t);
+    const int count = tg.lz * tg.ly * tg.lx;
+    const int toff = ix.tile_off[(int64_t)b * (g.nT + 1) + t];
+    for (int qb = 0; qb < count; qb += S96_QC) {
+      const int nq = min(S96_QC, count - qb);
+      __syncthreads();
+      if (tid < nq) {
+        tile_coord(tg, qb + tid, sm.qz[tid], sm.qy[tid], sm.qx[tid]);
+        const int i = ix.perm[(int64_t)b * g.N + toff + qb + tid];
+        sm.tok[tid] = i;
+        sm.lse[tid] = lse[lbase + i];
+        sm.del[tid] = delta[lbase + i];
+      }
+      __syncthreads();
+      stage_rows<T, D, S96_QC, S96_THREADS>(g, ix.rope, q, dout, b, h, sm.tok, sm.qz, sm.qy,
+                                            sm.qx, nq, &sm.q[0][0], &sm.dout[0][0], S96_LD);
+      __syncthreads();
+      // ---- phase 1 ----
+      {
+        float s[2][4], dp[2][4];
+#pragma unroll
+        for (int i = 0; i < 2; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) s[i][j] = dp[i][j] = 0.f;
+        const int qr0 = wq * 16 + lq, br0 = wb * 16 + lb;
+#pragma unroll 1
+        for (int k = 0; k < D; k += 4) {
+          float4 a[2], w[4];
+#pragma unroll
+          for (int i = 0; i < 2; ++i) a[i] = *reinterpret_cast<const float4*>(&sm.q[qr0 + 8 * i][k]);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) w[j] = *reinterpret_cast<const float4*>(&sm.ks[br0 + 4 * j][k]);
+#pragma unroll
+          for (int i = 0; i < 2; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              s[i][j] += a[i].x * w[j].x + a[i].y * w[j].y + a[i].z * w[j].z + a[i].w * w[j].w;
+#pragma unroll
+          for (int i = 0; i < 2; ++i)
+            a[i] = *reinterpret_cast<const float4*>(&sm.dout[qr0 + 8 * i][k]);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) w[j] = *reinterpret_cast<const float4*>(&sm.vs[br0 + 4 * j][k]);
+#pragma unroll
+          for (int i = 0; i < 2; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              dp[i][j] += a[i].x * w[j].x + a[i].y * w[j].y + a[i].z * w[j].z + a[i].w * w[j].w;
+        }
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int qq = qr0 + 8 * i;
+          const int cz = sm.qz[qq], cy = sm.qy[qq], cx = sm.qx[qq];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int bb = br0 + 4 * j;
+            const int bz0 = sm.bz0[bb], by0 = sm.by0[bb], bx0 = sm.bx0[bb];
+            const bool meets = bz0 + g.bz - 1 >= cz - g.rz && bz0 <= cz + g.rz &&
+                               by0 + g.by - 1 >= cy - g.ry && by0 <= cy + g.ry &&
+                               bx0 + g.bx - 1 >= cx - g.rx && bx0 <= cx + g.rx;
+            const bool in = qq < nq && B0 + bb < g.nb && !meets;
+            const float P = in ? expf(g.tau * s[i][j] - sm.lse[qq]) : 0.f;
+            sm.p[qq][bb] = P;
+            sm.ds[qq][bb] = P * (dp[i][j] - sm.del[qq]);
+          }
+        }
+      }
+      __syncthreads();
+      // ---- phase 2 ----
+      for (int qq = 0; qq < nq; ++qq) {
+        const float4 pv = *reinterpret_cast<const float4*>(&sm.p[qq][4 * tb]);
+        const float4 dsv = *reinterpret_cast<const float4*>(&sm.ds[qq][4 * tb]);
+        float xq[6], xo[6];
+#pragma unroll
+        for (int m = 0; m < 3; ++m) {
+          float2 a = *reinterpret_cast<const float2*>(&sm.q[qq][6 * tc + 2 * m]);
+          float2 o = *reinterpret_cast<const float2*>(&sm.dout[qq][6 * tc + 2 * m]);
+          xq[2 * m] = a.x;
+          xq[2 * m + 1] = a.y;
+          xo[2 * m] = o.x;
+          xo[2 * m + 1] = o.y;
+        }
+        const float pj[4] = {pv.x, pv.y, pv.z, pv.w};
+        const float dj[4] = {dsv.x, dsv.y, dsv.z, dsv.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+          for (int u = 0; u < 6; ++u) {
+            dk[j][u] += dj[j] * xq[u];
+            dv[j][u] += pj[j] * xo[u];
+          }
+      }
+    }
+  }
+  // partials: part[split][b][h][summary][2][D]
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int Bk = B0 + 4 * tb + j;
+    if (Bk < g.nb) {
+      float* dst = part + ((((int64_t)split * g.B + b) * g.H + h) * g.nb + Bk) * 2 * D;
+#pragma unroll
+      for (int u = 0; u < 6; ++u) {
+        dst[6 * tc + u] = dk[j][u];
+        dst[D + 6 * tc + u] = dv[j][u];
+      }
+    }
+  }
+}
+
+// dks = tau * sum over splits of the dk̄ partials, dvs = the same for dv̄
+// (fixed split order).
+__global__ void k_bwd_summary_reduce(Geo g, const int32_t* __restrict__ err, int nsplit,
+                                     const float* __restrict__ part, float* __restrict__ dks,
+                                     float* __restrict__ dvs) {
+  if (err[0]) return;
+  const int64_t per = (int64_t)g.B * g.H * g.nb * g.d;
+  const int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (e >= per) return;
+  const int64_t row = e / g.d;
+  const int c = (int)(e % g.d);
+  float sk = 0.f, sv = 0.f;
+  for (int s = 0; s < nsplit; ++s) {
+    const float* src = part + ((int64_t)s * per / g.d + row) * 2 * g.d;
+    sk += src[c];
+    sv += src[g.d + c];
+  }
+  dks[e] = g.tau * sk;
+  dvs[e] = sv;
+}
+
 // dq: query-major, the forward's structure.
 template <typename T, int D, bool SUMMARY>
 __global__ void __launch_bounds__(TILE * Split<D>::G) k_bwd_dq(
@@ -429,7 +708,7 @@ __global__ void __launch_bounds__(TILE * Split<D>::G) k_bwd_dq(
     const float* __restrict__ vsum, T* __restrict__ dq) {
   constexpr int G = Split<D>::G, CPT = Split<D>::CPT;
   if (ix.err[0]) return;
-  __shared__ float sbuf[2 * KC * D];
+  __shared__ __align__(16) float sbuf[2 * KC * D];
   float(*sk)[D] = reinterpret_cast<float(*)[D]>(sbuf);
   float(*sv)[D] = reinterpret_cast<float(*)[D]>(sbuf + KC * D);
   __shared__ ChunkCoords cc;
@@ -461,40 +740,36 @@ __global__ void __launch_bounds__(TILE * Split<D>::G) k_bwd_dq(
   for (int base = 0; base < nh; base += KC) {
     const int nk = min(KC, nh - base);
     __syncthreads();
-    for (int e = threadIdx.x; e < KC * D; e += blockDim.x) {
-      int kk = e / D, c = e % D;
-      float kv = 0.f, vv = 0.f;
-      if (kk < nk) {
-        int z, y, x;
-        halo_coord(tg, base + kk, z, y, x);
-        int j = hl[base + kk];
-        int64_t row = (((int64_t)b * g.N + j) * g.H + h) * D;
-        kv = rot_channel(k + row, ix.rope, g, c, z, y, x, j, false);
-        vv = to_f32(v[row + c]);
-        if (c == 0) {
-          cc.z[kk] = z;
-          cc.y[kk] = y;
-          cc.x[kk] = x;
-        }
-      }
-      sk[kk][c] = kv;
-      sv[kk][c] = vv;
+    if (threadIdx.x < nk) {
+      const int kk = threadIdx.x;
+      halo_coord(tg, base + kk, cc.z[kk], cc.y[kk], cc.x[kk]);
+      cc.tok[kk] = hl[base + kk];
     }
     __syncthreads();
-    for (int kk = 0; kk < KC; ++kk) {
-      float ps = 0.f, pd = 0.f;
-#pragma unroll
-      for (int u = 0; u < CPT; ++u) {
-        ps += qr[u] * sk[kk][lane * CPT + u];
-        pd += dO[u] * sv[kk][lane * CPT + u];
-      }
-      float s = group_sum<G>(ps), dp = group_sum<G>(pd);
-      bool in = active && kk < nk && abs(cc.z[kk] - cz) <= g.rz && abs(cc.y[kk] - cy) <= g.ry &&
-                abs(cc.x[kk] - cx) <= g.rx;
-      float P = in ? expf(g.tau * s - lse_i) : 0.f;
-      float dS = P * (dp - del_i);
-#pragma unroll
-      for (int u = 0; u < CPT; ++u) dqr[u] += g.tau * dS * sk[kk][lane * CPT + u];
+    stage_rows<T, D, KC, TILE * G>(g, ix.rope, k, v, b, h, cc.tok, cc.z, cc.y, cc.x, nk,
+                                   &sk[0][0], &sv[0][0], D);
+    __syncthreads();
+    // keys in pairs (two independent dot-product chains per thread); a pair
+    // outside every window of the warp's queries adds nothing and is skipped
+    for (int kk = 0; kk < KC; kk += 2) {
+      const bool in0 = active && kk < nk && abs(cc.z[kk] - cz) <= g.rz &&
+                       abs(cc.y[kk] - cy) <= g.ry && abs(cc.x[kk] - cx) <= g.rx;
+      const bool in1 = active && kk + 1 < nk && abs(cc.z[kk + 1] - cz) <= g.rz &&
+                       abs(cc.y[kk + 1] - cy) <= g.ry && abs(cc.x[kk + 1] - cx) <= g.rx;
+      if (!__any_sync(0xffffffffu, in0 || in1)) continue;
+      const float ps0 = dot_row(qr, &sk[kk][lane * CPT]);
+      const float ps1 = dot_row(qr, &sk[kk + 1][lane * CPT]);
+      const float pd0 = dot_row(dO, &sv[kk][lane * CPT]);
+      const float pd1 = dot_row(dO, &sv[kk + 1][lane * CPT]);
+      const float s0 = group_sum<G>(ps0), s1 = group_sum<G>(ps1);
+      const float dp0 = group_sum<G>(pd0), dp1 = group_sum<G>(pd1);
+      // re-read the staged rows below instead of holding them in registers
+      __syncwarp();
+      const float P0 = in0 ? expf(g.tau * s0 - lse_i) : 0.f;
+      const float P1 = in1 ? expf(g.tau * s1 - lse_i) : 0.f;
+      const float dS0 = P0 * (dp0 - del_i), dS1 = P1 * (dp1 - del_i);
+      axpy_row(dqr, g.tau * dS0, &sk[kk][lane * CPT]);
+      axpy_row(dqr, g.tau * dS1, &sk[kk + 1][lane * CPT]);
     }
   }
   if (SUMMARY) {
@@ -520,12 +795,8 @@ __global__ void __launch_bounds__(TILE * Split<D>::G) k_bwd_dq(
       }
       __syncthreads();
       for (int kk = 0; kk < KC; ++kk) {
-        float ps = 0.f, pd = 0.f;
-#pragma unroll
-        for (int u = 0; u < CPT; ++u) {
-          ps += qr[u] * sk[kk][lane * CPT + u];
-          pd += dO[u] * sv[kk][lane * CPT + u];
-        }
+        const float ps = dot_row(qr, &sk[kk][lane * CPT]);
+        const float pd = dot_row(dO, &sv[kk][lane * CPT]);
         float s = group_sum<G>(ps), dp = group_sum<G>(pd);
         int bz0 = cc.z[kk] * g.bz, by0 = cc.y[kk] * g.by, bx0 = cc.x[kk] * g.bx;
         bool meets = bz0 + g.bz - 1 >= cz - g.rz && bz0 <= cz + g.rz &&
@@ -534,8 +805,7 @@ __global__ void __launch_bounds__(TILE * Split<D>::G) k_bwd_dq(
         bool in = active && kk < nk && !meets;
         float P = in ? expf(g.tau * s - lse_i) : 0.f;
         float dS = P * (dp - del_i);
-#pragma unroll
-        for (int u = 0; u < CPT; ++u) dqr[u] += g.tau * dS * sk[kk][lane * CPT + u];
+        axpy_row(dqr, g.tau * dS, &sk[kk][lane * CPT]);
       }
     }
   }
@@ -570,7 +840,7 @@ __global__ void __launch_bounds__(TILE * Split<D>::G) k_bwd_dkdv(
     const float* __restrict__ dvs, T* __restrict__ dk, T* __restrict__ dv) {
   constexpr int G = Split<D>::G, CPT = Split<D>::CPT;
   if (ix.err[0]) return;
-  __shared__ float sbuf[2 * KC * D];
+  __shared__ __align__(16) float sbuf[2 * KC * D];
   float(*sq)[D] = reinterpret_cast<float(*)[D]>(sbuf);
   float(*sdo)[D] = reinterpret_cast<float(*)[D]>(sbuf + KC * D);
   __shared__ float slse[KC], sdel[KC];
@@ -601,45 +871,41 @@ __global__ void __launch_bounds__(TILE * Split<D>::G) k_bwd_dkdv(
   for (int base = 0; base < nh; base += KC) {
     const int nq = min(KC, nh - base);
     __syncthreads();
-    for (int e = threadIdx.x; e < KC * D; e += blockDim.x) {
-      int qq = e / D, c = e % D;
-      float qv = 0.f, dov = 0.f;
-      if (qq < nq) {
-        int z, y, x;
-        halo_coord(tg, base + qq, z, y, x);
-        int i = hl[base + qq];
-        int64_t row = (((int64_t)b * g.N + i) * g.H + h) * D;
-        qv = rot_channel(q + row, ix.rope, g, c, z, y, x, i, false);
-        dov = to_f32(dout[row + c]);
-        if (c == 0) {
-          cc.z[qq] = z;
-          cc.y[qq] = y;
-          cc.x[qq] = x;
-          slse[qq] = lse[lbase + i];
-          sdel[qq] = delta[lbase + i];
-        }
-      }
-      sq[qq][c] = qv;
-      sdo[qq][c] = dov;
+    if (threadIdx.x < nq) {
+      const int qq = threadIdx.x;
+      halo_coord(tg, base + qq, cc.z[qq], cc.y[qq], cc.x[qq]);
+      const int i = hl[base + qq];
+      cc.tok[qq] = i;
+      slse[qq] = lse[lbase + i];
+      sdel[qq] = delta[lbase + i];
     }
     __syncthreads();
-    for (int qq = 0; qq < KC; ++qq) {
-      float ps = 0.f, pd = 0.f;
-#pragma unroll
-      for (int u = 0; u < CPT; ++u) {
-        ps += kr[u] * sq[qq][lane * CPT + u];
-        pd += vr[u] * sdo[qq][lane * CPT + u];
-      }
-      float s = group_sum<G>(ps), dp = group_sum<G>(pd);
-      bool in = active && qq < nq && abs(cc.z[qq] - cz) <= g.rz && abs(cc.y[qq] - cy) <= g.ry &&
-                abs(cc.x[qq] - cx) <= g.rx;
-      float P = in ? expf(g.tau * s - slse[qq]) : 0.f;
-      float dS = P * (dp - sdel[qq]);
-#pragma unroll
-      for (int u = 0; u < CPT; ++u) {
-        dkr[u] += g.tau * dS * sq[qq][lane * CPT + u];
-        dvr[u] += P * sdo[qq][lane * CPT + u];
-      }
+    stage_rows<T, D, KC, TILE * G>(g, ix.rope, q, dout, b, h, cc.tok, cc.z, cc.y, cc.x, nq,
+                                   &sq[0][0], &sdo[0][0], D);
+    __syncthreads();
+    // queries in pairs (two independent dot-product chains per thread); a
+    // pair whose windows miss every key of the warp adds nothing and is skipped
+    for (int qq = 0; qq < KC; qq += 2) {
+      const bool in0 = active && qq < nq && abs(cc.z[qq] - cz) <= g.rz &&
+                       abs(cc.y[qq] - cy) <= g.ry && abs(cc.x[qq] - cx) <= g.rx;
+      const bool in1 = active && qq + 1 < nq && abs(cc.z[qq + 1] - cz) <= g.rz &&
+                       abs(cc.y[qq + 1] - cy) <= g.ry && abs(cc.x[qq + 1] - cx) <= g.rx;
+      if (!__any_sync(0xffffffffu, in0 || in1)) continue;
+      const float ps0 = dot_row(kr, &sq[qq][lane * CPT]);
+      const float ps1 = dot_row(kr, &sq[qq + 1][lane * CPT]);
+      const float pd0 = dot_row(vr, &sdo[qq][lane * CPT]);
+      const float pd1 = dot_row(vr, &sdo[qq + 1][lane * CPT]);
+      const float s0 = group_sum<G>(ps0), s1 = group_sum<G>(ps1);
+      const float dp0 = group_sum<G>(pd0), dp1 = group_sum<G>(pd1);
+      // re-read the staged rows below instead of holding them in registers
+      __syncwarp();
+      const float P0 = in0 ? expf(g.tau * s0 - slse[qq]) : 0.f;
+      const float P1 = in1 ? expf(g.tau * s1 - slse[qq + 1]) : 0.f;
+      const float dS0 = P0 * (dp0 - sdel[qq]), dS1 = P1 * (dp1 - sdel[qq + 1]);
+      axpy_row(dkr, g.tau * dS0, &sq[qq][lane * CPT]);
+      axpy_row(dkr, g.tau * dS1, &sq[qq + 1][lane * CPT]);
+      axpy_row(dvr, P0, &sdo[qq][lane * CPT]);
+      axpy_row(dvr, P1, &sdo[qq + 1][lane * CPT]);
     }
   }
   if (SUMMARY && active) {
@@ -711,10 +977,21 @@ int forward_dispatch(const Geo& g, const pack3d_index* idx, const void* q, const
 }
 
 struct BwdWs {
-  float *delta, *ksum, *vsum, *dks, *dvs;
+  float *delta, *ksum, *vsum, *dks, *dvs, *part;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Query splits of the d = 96 summary-gradient kernel: as many CTAs as fit in
+// one wave of two CTAs per SM, at most one split per query tile, at most 32.
+inline int summary96_splits(const Geo& g) {
+  if (g.d != 96) return 0;
+  const int nbc = (g.nb + S96_NB - 1) / S96_NB;
+  const int64_t groups = (int64_t)g.B * g.H * nbc;
+  int64_t s = (2 * 148) / groups;
+  s = std::min<int64_t>(s, std::min(g.nT, 32));
+  return (int)std::max<int64_t>(s, 1);
+}
 
 BwdWs carve(const Geo& g, void* ws) {
   char* p = (char*)ws;
@@ -730,6 +1007,8 @@ BwdWs carve(const Geo& g, void* ws) {
   w.dks = (float*)p;
   p += align256(ns);
   w.dvs = (float*)p;
+  p += align256(ns);
+  w.part = (float*)p;
   return w;
 }
 
@@ -747,9 +1026,31 @@ int backward_typed(const Geo& g, const pack3d_index* idx, const void* q, const v
         g, idx->err, (const T*)out, (const T*)dout, w.delta);
   int rc = launch_block_summaries(g, idx, k, v, w.ksum, w.vsum, s);
   if (rc) return rc;
-  dim3 sgrid((g.nb + BC - 1) / BC, g.B, g.H);
-  k_bwd_summary<T, D><<<sgrid, 256, 0, s>>>(g, *idx, (const T*)q, (const T*)dout, lse, w.delta,
-                                            w.ksum, w.vsum, w.dks, w.dvs);
+  if constexpr (D == 96) {
+    const int nsplit = summary96_splits(g);
+    const int nbc = (g.nb + S96_NB - 1) / S96_NB;
+    static bool attr_set = false;
+    if (!attr_set) {
+      cudaError_t e = cudaFuncSetAttribute(k_bwd_summary96<T>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)sizeof(Sum96Smem));
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_bwd_summary96<T>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared);
+      if (e != cudaSuccess) return cuda_status(e);
+      attr_set = true;
+    }
+    dim3 sgrid(nbc * nsplit, g.B, g.H);
+    k_bwd_summary96<T><<<sgrid, S96_THREADS, sizeof(Sum96Smem), s>>>(
+        g, *idx, (const T*)q, (const T*)dout, lse, w.delta, w.ksum, w.vsum, nsplit, w.part);
+    const int64_t per = (int64_t)g.B * g.H * g.nb * g.d;
+    k_bwd_summary_reduce<<<(unsigned)((per + 255) / 256), 256, 0, s>>>(g, idx->err, nsplit,
+                                                                       w.part, w.dks, w.dvs);
+  } else {
+    dim3 sgrid((g.nb + BC - 1) / BC, g.B, g.H);
+    k_bwd_summary<T, D><<<sgrid, 256, 0, s>>>(g, *idx, (const T*)q, (const T*)dout, lse,
+                                              w.delta, w.ksum, w.vsum, w.dks, w.dvs);
+  }
   dim3 grid(g.nT, g.H, g.B);
   dim3 block(TILE * Split<D>::G);
   k_bwd_dq<T, D, true><<<grid, block, 0, s>>>(g, *idx, (const T*)q, (const T*)k, (const T*)v,
@@ -787,7 +1088,7 @@ int launch_forward_simt(const Geo& g, const pack3d_index* idx, const void* q, co
 size_t backward_workspace_bytes(const Geo& g) {
   size_t nd = sizeof(float) * (size_t)g.B * g.H * g.N;
   size_t ns = sizeof(float) * (size_t)g.B * g.H * g.nb * g.d;
-  return align256(nd) + 4 * align256(ns);
+  return align256(nd) + 4 * align256(ns) + 2 * (size_t)summary96_splits(g) * ns;
 }
 
 int launch_backward(const Geo& g, const pack3d_index* idx, const void* q, const void* k,
