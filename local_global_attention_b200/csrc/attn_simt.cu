@@ -117,6 +117,30 @@ struct ChunkCoords {
   int z[KC], y[KC], x[KC], tok[KC];
 };
 
+// The backward's local loops stage the halo box plane by plane: a whole
+// z-plane of it per chunk, or as many of the plane's rows as fit in CAPK
+// tokens.  Inside a chunk every warp visits only the rows its tokens' windows
+// reach, so warps do not wait on rows that only other warps need.
+constexpr int CAPK = 160;
+struct PlaneMeta {
+  int z[CAPK], y[CAPK], x[CAPK], tok[CAPK];
+};
+
+// z and y extent of a warp's active tokens (a ragged tile's warp may span rows).
+struct WarpBox {
+  int zlo, zhi, ylo, yhi;
+};
+
+__device__ __forceinline__ WarpBox warp_box(bool active, int cz, int cy) {
+  constexpr int BIG = 1 << 29;
+  WarpBox w;
+  w.zlo = __reduce_min_sync(0xffffffffu, active ? cz : BIG);
+  w.zhi = __reduce_max_sync(0xffffffffu, active ? cz : -BIG);
+  w.ylo = __reduce_min_sync(0xffffffffu, active ? cy : BIG);
+  w.yhi = __reduce_max_sync(0xffffffffu, active ? cy : -BIG);
+  return w;
+}
+
 // Dot product of a thread's CPT channels with a staged fp32 row (16-byte
 // aligned), summed in channel order, read 16 bytes at a time.
 template <int CPT>
@@ -135,28 +159,17 @@ __device__ __forceinline__ float dot_row(const float (&r)[CPT], const float* row
   return acc;
 }
 
-// Stage a chunk of token rows into shared memory as fp32: xo = R(c) x (the
-// rotated row) and yo = y (plain), for the tokens whose packed index and
-// coordinate the caller has put into tok / cz / cy / cx.  NT threads share
-// the chunk, NT / ROWS per row, each rotation pair (both channels of it) read
-// once; every thread's loads are independent, so their latencies overlap.
-// Rows nrows .. ROWS-1 are zero-filled.
-template <typename T, int D, int ROWS, int NT>
-__device__ __forceinline__ void stage_rows(const Geo& g, const float* __restrict__ rope,
-                                           const T* __restrict__ x, const T* __restrict__ y,
-                                           int b, int h, const int* tok, const int* cz,
-                                           const int* cy, const int* cx, int nrows, float* xo,
-                                           float* yo, int ld) {
-  static_assert(NT % ROWS == 0, "threads must divide evenly over the rows");
-  constexpr int TPR = NT / ROWS, PAIRS = D / 2, HALF = D / 6, DA = D / 3;
-  const int r = threadIdx.x / TPR, sub = threadIdx.x % TPR;
-  float* xr = xo + r * ld;
-  float* yr = yo + r * ld;
-  if (r >= nrows) {
-    for (int c = sub; c < D; c += TPR) xr[c] = yr[c] = 0.f;
-    return;
-  }
-  const int i = tok[r];
+// One staged token row as fp32: xr = R(c) x (the rotated row) and yr = y
+// (plain), for the token with packed index i and coordinate (cz, cy, cx).
+// TPR threads share the row (sub = 0 .. TPR-1), each rotation pair (both
+// channels of it) read once; a thread's loads are independent of each other,
+// so their latencies overlap.
+template <typename T, int D, int TPR>
+__device__ __forceinline__ void stage_one_row(const Geo& g, const float* __restrict__ rope,
+                                              const T* __restrict__ x, const T* __restrict__ y,
+                                              int b, int h, int i, int cz, int cy, int cx, int sub,
+                                              float* xr, float* yr) {
+  constexpr int PAIRS = D / 2, HALF = D / 6, DA = D / 3;
   const int64_t row = (((int64_t)b * g.N + i) * g.H + h) * D;
   const bool packed = g.rope_mode == PACK3D_ROPE_PACKED;
 #pragma unroll
@@ -169,7 +182,7 @@ __device__ __forceinline__ void stage_rows(const Geo& g, const float* __restrict
         j = pr - a * HALF;
         c1 = a * DA + j;
         c2 = c1 + HALF;
-        ca = a == 0 ? cz[r] : (a == 1 ? cy[r] : cx[r]);
+        ca = a == 0 ? cz : (a == 1 ? cy : cx);
       }
       const float2 cs = rope_cs(rope, g, a, ca, i, j);
       const float x1 = to_f32(x[row + c1]), x2 = to_f32(x[row + c2]);
@@ -179,6 +192,42 @@ __device__ __forceinline__ void stage_rows(const Geo& g, const float* __restrict
       yr[c2] = to_f32(y[row + c2]);
     }
   }
+}
+
+// Stage ROWS token rows (row stride ld floats) with NT threads, NT / ROWS per
+// row; rows nrows .. ROWS-1 are zero-filled.
+template <typename T, int D, int ROWS, int NT>
+__device__ __forceinline__ void stage_rows(const Geo& g, const float* __restrict__ rope,
+                                           const T* __restrict__ x, const T* __restrict__ y,
+                                           int b, int h, const int* tok, const int* cz,
+                                           const int* cy, const int* cx, int nrows, float* xo,
+                                           float* yo, int ld) {
+  static_assert(NT % ROWS == 0, "threads must divide evenly over the rows");
+  constexpr int TPR = NT / ROWS;
+  const int r = threadIdx.x / TPR, sub = threadIdx.x % TPR;
+  float* xr = xo + r * ld;
+  float* yr = yo + r * ld;
+  if (r >= nrows) {
+    for (int c = sub; c < D; c += TPR) xr[c] = yr[c] = 0.f;
+    return;
+  }
+  stage_one_row<T, D, TPR>(g, rope, x, y, b, h, tok[r], cz[r], cy[r], cx[r], sub, xr, yr);
+}
+
+// Stage nrows token rows (row stride D) with NT threads, 16 per row, as many
+// passes as needed; nothing beyond nrows is written.
+template <typename T, int D, int NT>
+__device__ __forceinline__ void stage_rows_n(const Geo& g, const float* __restrict__ rope,
+                                             const T* __restrict__ x, const T* __restrict__ y,
+                                             int b, int h, const int* tok, const int* cz,
+                                             const int* cy, const int* cx, int nrows, float* xo,
+                                             float* yo) {
+  constexpr int TPR = 16;
+  static_assert(NT % TPR == 0, "threads must divide evenly over the rows");
+  const int sub = threadIdx.x % TPR;
+  for (int r = threadIdx.x / TPR; r < nrows; r += NT / TPR)
+    stage_one_row<T, D, TPR>(g, rope, x, y, b, h, tok[r], cz[r], cy[r], cx[r], sub, xo + r * D,
+                             yo + r * D);
 }
 
 // acc[u] += a * row[u] over a thread's CPT channels of a staged fp32 row.
@@ -708,10 +757,13 @@ __global__ void __launch_bounds__(TILE * Split<D>::G) k_bwd_dq(
     const float* __restrict__ vsum, T* __restrict__ dq) {
   constexpr int G = Split<D>::G, CPT = Split<D>::CPT;
   if (ix.err[0]) return;
-  __shared__ __align__(16) float sbuf[2 * KC * D];
-  float(*sk)[D] = reinterpret_cast<float(*)[D]>(sbuf);
-  float(*sv)[D] = reinterpret_cast<float(*)[D]>(sbuf + KC * D);
+  // dynamic: staged keys and values, 2 * CAPK rows of D floats
+  extern __shared__ __align__(16) float bwd_dyn[];
+  float* const sbuf = bwd_dyn;
+  float(*sk)[D] = reinterpret_cast<float(*)[D]>(bwd_dyn);
+  float(*sv)[D] = reinterpret_cast<float(*)[D]>(bwd_dyn + CAPK * D);
   __shared__ ChunkCoords cc;
+  __shared__ PlaneMeta pm;
   const int t = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int qs = threadIdx.x / G, lane = threadIdx.x % G;
   const TileGeo tg = tile_geo(g, t);
@@ -735,41 +787,53 @@ __global__ void __launch_bounds__(TILE * Split<D>::G) k_bwd_dq(
   const float lse_i = active ? lse[lrow] : 0.f;
   const float del_i = active ? delta[lrow] : 0.f;
 
-  const int nh = tg.hz * tg.hy * tg.hx;
   const int32_t* hl = ix.nbr + (int64_t)b * ix.n_halo + ix.nbr_off[t];
-  for (int base = 0; base < nh; base += KC) {
-    const int nk = min(KC, nh - base);
-    __syncthreads();
-    if (threadIdx.x < nk) {
-      const int kk = threadIdx.x;
-      halo_coord(tg, base + kk, cc.z[kk], cc.y[kk], cc.x[kk]);
-      cc.tok[kk] = hl[base + kk];
-    }
-    __syncthreads();
-    stage_rows<T, D, KC, TILE * G>(g, ix.rope, k, v, b, h, cc.tok, cc.z, cc.y, cc.x, nk,
-                                   &sk[0][0], &sv[0][0], D);
-    __syncthreads();
-    // keys in pairs (two independent dot-product chains per thread); a pair
-    // outside every window of the warp's queries adds nothing and is skipped
-    for (int kk = 0; kk < KC; kk += 2) {
-      const bool in0 = active && kk < nk && abs(cc.z[kk] - cz) <= g.rz &&
-                       abs(cc.y[kk] - cy) <= g.ry && abs(cc.x[kk] - cx) <= g.rx;
-      const bool in1 = active && kk + 1 < nk && abs(cc.z[kk + 1] - cz) <= g.rz &&
-                       abs(cc.y[kk + 1] - cy) <= g.ry && abs(cc.x[kk + 1] - cx) <= g.rx;
-      if (!__any_sync(0xffffffffu, in0 || in1)) continue;
-      const float ps0 = dot_row(qr, &sk[kk][lane * CPT]);
-      const float ps1 = dot_row(qr, &sk[kk + 1][lane * CPT]);
-      const float pd0 = dot_row(dO, &sv[kk][lane * CPT]);
-      const float pd1 = dot_row(dO, &sv[kk + 1][lane * CPT]);
-      const float s0 = group_sum<G>(ps0), s1 = group_sum<G>(ps1);
-      const float dp0 = group_sum<G>(pd0), dp1 = group_sum<G>(pd1);
-      // re-read the staged rows below instead of holding them in registers
-      __syncwarp();
-      const float P0 = in0 ? expf(g.tau * s0 - lse_i) : 0.f;
-      const float P1 = in1 ? expf(g.tau * s1 - lse_i) : 0.f;
-      const float dS0 = P0 * (dp0 - del_i), dS1 = P1 * (dp1 - del_i);
-      axpy_row(dqr, g.tau * dS0, &sk[kk][lane * CPT]);
-      axpy_row(dqr, g.tau * dS1, &sk[kk + 1][lane * CPT]);
+  const WarpBox wb = warp_box(active, cz, cy);
+  const int rpc = min(tg.hy, CAPK / tg.hx);  // halo rows per chunk
+  for (int pz = 0; pz < tg.hz; ++pz) {
+    const int zk = tg.hz0 + pz;
+    const bool zneed = zk >= wb.zlo - g.rz && zk <= wb.zhi + g.rz;  // warp-uniform
+    for (int ry0 = 0; ry0 < tg.hy; ry0 += rpc) {
+      const int nr = min(rpc, tg.hy - ry0), nk = nr * tg.hx;
+      const int base = (pz * tg.hy + ry0) * tg.hx;
+      __syncthreads();
+      for (int e = threadIdx.x; e < nk; e += blockDim.x) {
+        halo_coord(tg, base + e, pm.z[e], pm.y[e], pm.x[e]);
+        pm.tok[e] = hl[base + e];
+      }
+      __syncthreads();
+      stage_rows_n<T, D, TILE * G>(g, ix.rope, k, v, b, h, pm.tok, pm.z, pm.y, pm.x, nk,
+                                   &sk[0][0], &sv[0][0]);
+      __syncthreads();
+      if (!zneed) continue;
+      for (int r = 0; r < nr; ++r) {
+        const int yk = tg.hy0 + ry0 + r;
+        if (yk < wb.ylo - g.ry || yk > wb.yhi + g.ry) continue;  // warp-uniform
+        const bool rowin = active && abs(zk - cz) <= g.rz && abs(yk - cy) <= g.ry;
+        const int k0 = r * tg.hx, k1 = k0 + tg.hx;
+        // keys in pairs (two independent dot-product chains per thread); at an
+        // odd row end the second key repeats the first with weight 0.  A pair
+        // outside every window of the warp's queries is skipped.
+        for (int ka = k0; ka < k1; ka += 2) {
+          const int kb = min(ka + 1, k1 - 1);
+          const bool in0 = rowin && abs(pm.x[ka] - cx) <= g.rx;
+          const bool in1 = rowin && ka + 1 < k1 && abs(pm.x[kb] - cx) <= g.rx;
+          if (!__any_sync(0xffffffffu, in0 || in1)) continue;
+          const float ps0 = dot_row(qr, &sk[ka][lane * CPT]);
+          const float ps1 = dot_row(qr, &sk[kb][lane * CPT]);
+          const float pd0 = dot_row(dO, &sv[ka][lane * CPT]);
+          const float pd1 = dot_row(dO, &sv[kb][lane * CPT]);
+          const float s0 = group_sum<G>(ps0), s1 = group_sum<G>(ps1);
+          const float dp0 = group_sum<G>(pd0), dp1 = group_sum<G>(pd1);
+          // re-read the staged rows below instead of holding them in registers
+          __syncwarp();
+          const float P0 = in0 ? expf(g.tau * s0 - lse_i) : 0.f;
+          const float P1 = in1 ? expf(g.tau * s1 - lse_i) : 0.f;
+          const float dS0 = P0 * (dp0 - del_i), dS1 = P1 * (dp1 - del_i);
+          axpy_row(dqr, g.tau * dS0, &sk[ka][lane * CPT]);
+          axpy_row(dqr, g.tau * dS1, &sk[kb][lane * CPT]);
+        }
+      }
     }
   }
   if (SUMMARY) {
@@ -840,11 +904,13 @@ __global__ void __launch_bounds__(TILE * Split<D>::G) k_bwd_dkdv(
     const float* __restrict__ dvs, T* __restrict__ dk, T* __restrict__ dv) {
   constexpr int G = Split<D>::G, CPT = Split<D>::CPT;
   if (ix.err[0]) return;
-  __shared__ __align__(16) float sbuf[2 * KC * D];
-  float(*sq)[D] = reinterpret_cast<float(*)[D]>(sbuf);
-  float(*sdo)[D] = reinterpret_cast<float(*)[D]>(sbuf + KC * D);
-  __shared__ float slse[KC], sdel[KC];
-  __shared__ ChunkCoords cc;
+  // dynamic: staged queries and dO rows, 2 * CAPK rows of D floats
+  extern __shared__ __align__(16) float bwd_dyn[];
+  float* const sbuf = bwd_dyn;
+  float(*sq)[D] = reinterpret_cast<float(*)[D]>(bwd_dyn);
+  float(*sdo)[D] = reinterpret_cast<float(*)[D]>(bwd_dyn + CAPK * D);
+  __shared__ float slse[CAPK], sdel[CAPK];
+  __shared__ PlaneMeta pm;
   const int t = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int ks = threadIdx.x / G, lane = threadIdx.x % G;
   const TileGeo tg = tile_geo(g, t);
@@ -866,46 +932,58 @@ __global__ void __launch_bounds__(TILE * Split<D>::G) k_bwd_dkdv(
     dvr[u] = 0.f;
   }
   const int64_t lbase = ((int64_t)b * g.H + h) * g.N;
-  const int nh = tg.hz * tg.hy * tg.hx;
   const int32_t* hl = ix.nbr + (int64_t)b * ix.n_halo + ix.nbr_off[t];
-  for (int base = 0; base < nh; base += KC) {
-    const int nq = min(KC, nh - base);
-    __syncthreads();
-    if (threadIdx.x < nq) {
-      const int qq = threadIdx.x;
-      halo_coord(tg, base + qq, cc.z[qq], cc.y[qq], cc.x[qq]);
-      const int i = hl[base + qq];
-      cc.tok[qq] = i;
-      slse[qq] = lse[lbase + i];
-      sdel[qq] = delta[lbase + i];
-    }
-    __syncthreads();
-    stage_rows<T, D, KC, TILE * G>(g, ix.rope, q, dout, b, h, cc.tok, cc.z, cc.y, cc.x, nq,
-                                   &sq[0][0], &sdo[0][0], D);
-    __syncthreads();
-    // queries in pairs (two independent dot-product chains per thread); a
-    // pair whose windows miss every key of the warp adds nothing and is skipped
-    for (int qq = 0; qq < KC; qq += 2) {
-      const bool in0 = active && qq < nq && abs(cc.z[qq] - cz) <= g.rz &&
-                       abs(cc.y[qq] - cy) <= g.ry && abs(cc.x[qq] - cx) <= g.rx;
-      const bool in1 = active && qq + 1 < nq && abs(cc.z[qq + 1] - cz) <= g.rz &&
-                       abs(cc.y[qq + 1] - cy) <= g.ry && abs(cc.x[qq + 1] - cx) <= g.rx;
-      if (!__any_sync(0xffffffffu, in0 || in1)) continue;
-      const float ps0 = dot_row(kr, &sq[qq][lane * CPT]);
-      const float ps1 = dot_row(kr, &sq[qq + 1][lane * CPT]);
-      const float pd0 = dot_row(vr, &sdo[qq][lane * CPT]);
-      const float pd1 = dot_row(vr, &sdo[qq + 1][lane * CPT]);
-      const float s0 = group_sum<G>(ps0), s1 = group_sum<G>(ps1);
-      const float dp0 = group_sum<G>(pd0), dp1 = group_sum<G>(pd1);
-      // re-read the staged rows below instead of holding them in registers
-      __syncwarp();
-      const float P0 = in0 ? expf(g.tau * s0 - slse[qq]) : 0.f;
-      const float P1 = in1 ? expf(g.tau * s1 - slse[qq + 1]) : 0.f;
-      const float dS0 = P0 * (dp0 - sdel[qq]), dS1 = P1 * (dp1 - sdel[qq + 1]);
-      axpy_row(dkr, g.tau * dS0, &sq[qq][lane * CPT]);
-      axpy_row(dkr, g.tau * dS1, &sq[qq + 1][lane * CPT]);
-      axpy_row(dvr, P0, &sdo[qq][lane * CPT]);
-      axpy_row(dvr, P1, &sdo[qq + 1][lane * CPT]);
+  const WarpBox wb = warp_box(active, cz, cy);
+  const int rpc = min(tg.hy, CAPK / tg.hx);  // halo rows per chunk
+  for (int pz = 0; pz < tg.hz; ++pz) {
+    const int zq = tg.hz0 + pz;
+    const bool zneed = zq >= wb.zlo - g.rz && zq <= wb.zhi + g.rz;  // warp-uniform
+    for (int ry0 = 0; ry0 < tg.hy; ry0 += rpc) {
+      const int nr = min(rpc, tg.hy - ry0), nq = nr * tg.hx;
+      const int base = (pz * tg.hy + ry0) * tg.hx;
+      __syncthreads();
+      for (int e = threadIdx.x; e < nq; e += blockDim.x) {
+        halo_coord(tg, base + e, pm.z[e], pm.y[e], pm.x[e]);
+        const int i = hl[base + e];
+        pm.tok[e] = i;
+        slse[e] = lse[lbase + i];
+        sdel[e] = delta[lbase + i];
+      }
+      __syncthreads();
+      stage_rows_n<T, D, TILE * G>(g, ix.rope, q, dout, b, h, pm.tok, pm.z, pm.y, pm.x, nq,
+                                   &sq[0][0], &sdo[0][0]);
+      __syncthreads();
+      if (!zneed) continue;
+      for (int r = 0; r < nr; ++r) {
+        const int yq = tg.hy0 + ry0 + r;
+        if (yq < wb.ylo - g.ry || yq > wb.yhi + g.ry) continue;  // warp-uniform
+        const bool rowin = active && abs(zq - cz) <= g.rz && abs(yq - cy) <= g.ry;
+        const int q0 = r * tg.hx, q1 = q0 + tg.hx;
+        // queries in pairs (two independent dot-product chains per thread); at
+        // an odd row end the second query repeats the first with weight 0.  A
+        // pair whose windows miss every key of the warp is skipped.
+        for (int qa = q0; qa < q1; qa += 2) {
+          const int qb = min(qa + 1, q1 - 1);
+          const bool in0 = rowin && abs(pm.x[qa] - cx) <= g.rx;
+          const bool in1 = rowin && qa + 1 < q1 && abs(pm.x[qb] - cx) <= g.rx;
+          if (!__any_sync(0xffffffffu, in0 || in1)) continue;
+          const float ps0 = dot_row(kr, &sq[qa][lane * CPT]);
+          const float ps1 = dot_row(kr, &sq[qb][lane * CPT]);
+          const float pd0 = dot_row(vr, &sdo[qa][lane * CPT]);
+          const float pd1 = dot_row(vr, &sdo[qb][lane * CPT]);
+          const float s0 = group_sum<G>(ps0), s1 = group_sum<G>(ps1);
+          const float dp0 = group_sum<G>(pd0), dp1 = group_sum<G>(pd1);
+          // re-read the staged rows below instead of holding them in registers
+          __syncwarp();
+          const float P0 = in0 ? expf(g.tau * s0 - slse[qa]) : 0.f;
+          const float P1 = in1 ? expf(g.tau * s1 - slse[qb]) : 0.f;
+          const float dS0 = P0 * (dp0 - sdel[qa]), dS1 = P1 * (dp1 - sdel[qb]);
+          axpy_row(dkr, g.tau * dS0, &sq[qa][lane * CPT]);
+          axpy_row(dkr, g.tau * dS1, &sq[qb][lane * CPT]);
+          axpy_row(dvr, P0, &sdo[qa][lane * CPT]);
+          axpy_row(dvr, P1, &sdo[qb][lane * CPT]);
+        }
+      }
     }
   }
   if (SUMMARY && active) {
@@ -1051,14 +1129,27 @@ int backward_typed(const Geo& g, const pack3d_index* idx, const void* q, const v
     k_bwd_summary<T, D><<<sgrid, 256, 0, s>>>(g, *idx, (const T*)q, (const T*)dout, lse,
                                               w.delta, w.ksum, w.vsum, w.dks, w.dvs);
   }
+  // one halo row must fit in a staged chunk
+  if (TX + 2 * g.rx > CAPK) return PACK3D_ERR_UNSUPPORTED;
+  const size_t dyn = 2 * (size_t)CAPK * D * sizeof(float);
+  static bool local_attr_set = false;
+  if (!local_attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(k_bwd_dq<T, D, true>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k_bwd_dkdv<T, D, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
+    if (e != cudaSuccess) return cuda_status(e);
+    local_attr_set = true;
+  }
   dim3 grid(g.nT, g.H, g.B);
   dim3 block(TILE * Split<D>::G);
-  k_bwd_dq<T, D, true><<<grid, block, 0, s>>>(g, *idx, (const T*)q, (const T*)k, (const T*)v,
-                                              (const T*)dout, lse, w.delta, w.ksum, w.vsum,
-                                              (T*)dq);
-  k_bwd_dkdv<T, D, true><<<grid, block, 0, s>>>(g, *idx, (const T*)q, (const T*)k, (const T*)v,
-                                                (const T*)dout, lse, w.delta, w.dks, w.dvs,
-                                                (T*)dk, (T*)dv);
+  k_bwd_dq<T, D, true><<<grid, block, dyn, s>>>(g, *idx, (const T*)q, (const T*)k, (const T*)v,
+                                                (const T*)dout, lse, w.delta, w.ksum, w.vsum,
+                                                (T*)dq);
+  k_bwd_dkdv<T, D, true><<<grid, block, dyn, s>>>(g, *idx, (const T*)q, (const T*)k,
+                                                  (const T*)v, (const T*)dout, lse, w.delta,
+                                                  w.dks, w.dvs, (T*)dk, (T*)dv);
   return cuda_status(cudaGetLastError());
 }
 
