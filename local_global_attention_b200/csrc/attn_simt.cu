@@ -131,6 +131,22 @@ struct WarpBox {
   int zlo, zhi, ylo, yhi;
 };
 
+// Token slot s (0 .. TILE-1) of a tile for the backward's token-major
+// kernels: each group of 8 slots (one warp at head_dim 96) takes a 2x2x2 box
+// of the 4x4x8 tile, so the union of its windows is 8 wide along every axis
+// (a row of 8 along x would need 7 x 7 x 14).  Returns whether the box cell
+// lies inside the clipped tile; e is its raster index there.
+__device__ __forceinline__ bool box_slot(const TileGeo& tg, int s, int& z, int& y, int& x,
+                                         int& e) {
+  static_assert(TZ == 4 && TY == 4 && TX == 8, "slot boxes assume a 4x4x8 tile");
+  const int w = s >> 3, l = s & 7;
+  z = tg.z0 + 2 * (w >> 3) + ((l >> 2) & 1);
+  y = tg.y0 + 2 * ((w >> 2) & 1) + ((l >> 1) & 1);
+  x = tg.x0 + 2 * (w & 3) + (l & 1);
+  e = ((z - tg.z0) * tg.ly + (y - tg.y0)) * tg.lx + (x - tg.x0);
+  return z < tg.z0 + tg.lz && y < tg.y0 + tg.ly && x < tg.x0 + tg.lx;
+}
+
 __device__ __forceinline__ WarpBox warp_box(bool active, int cz, int cy) {
   constexpr int BIG = 1 << 29;
   WarpBox w;
@@ -767,13 +783,9 @@ __global__ void __launch_bounds__(TILE * Split<D>::G) k_bwd_dq(
   const int t = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int qs = threadIdx.x / G, lane = threadIdx.x % G;
   const TileGeo tg = tile_geo(g, t);
-  const int count = tg.lz * tg.ly * tg.lx;
-  const bool active = qs < count;
-  int cz = 0, cy = 0, cx = 0, qi = 0;
-  if (active) {
-    tile_coord(tg, qs, cz, cy, cx);
-    qi = ix.perm[(int64_t)b * g.N + ix.tile_off[(int64_t)b * (g.nT + 1) + t] + qs];
-  }
+  int cz = 0, cy = 0, cx = 0, qe = 0, qi = 0;
+  const bool active = box_slot(tg, qs, cz, cy, cx, qe);
+  if (active) qi = ix.perm[(int64_t)b * g.N + ix.tile_off[(int64_t)b * (g.nT + 1) + t] + qe];
   const int64_t qrow = (((int64_t)b * g.N + qi) * g.H + h) * D;
   float qr[CPT], dO[CPT], dqr[CPT];
 #pragma unroll
@@ -914,13 +926,9 @@ __global__ void __launch_bounds__(TILE * Split<D>::G) k_bwd_dkdv(
   const int t = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int ks = threadIdx.x / G, lane = threadIdx.x % G;
   const TileGeo tg = tile_geo(g, t);
-  const int count = tg.lz * tg.ly * tg.lx;
-  const bool active = ks < count;
-  int cz = 0, cy = 0, cx = 0, kj = 0;
-  if (active) {
-    tile_coord(tg, ks, cz, cy, cx);
-    kj = ix.perm[(int64_t)b * g.N + ix.tile_off[(int64_t)b * (g.nT + 1) + t] + ks];
-  }
+  int cz = 0, cy = 0, cx = 0, ke = 0, kj = 0;
+  const bool active = box_slot(tg, ks, cz, cy, cx, ke);
+  if (active) kj = ix.perm[(int64_t)b * g.N + ix.tile_off[(int64_t)b * (g.nT + 1) + t] + ke];
   const int64_t krow = (((int64_t)b * g.N + kj) * g.H + h) * D;
   float kr[CPT], vr[CPT], dkr[CPT], dvr[CPT];
 #pragma unroll
