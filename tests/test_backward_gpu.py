@@ -22,6 +22,10 @@ CASES = [
                block=(8, 8, 8), dtype="bf16", value_scale=1.0 / np.sqrt(96), seed=43),
     I.Workload(name="d12_fp32_4x6x8", B=1, H=2, d=12, Z=4, Y=6, X=8, window=(3, 3, 3),
                block=(2, 3, 4), dtype="fp32", seed=44),
+    # a wide y/x window: a halo plane (18 rows of 22) is staged in three row
+    # chunks, and halo rows clipped at the volume edge have odd lengths
+    I.Workload(name="wide_window_fp32_5x20x26", B=1, H=2, d=96, Z=5, Y=20, X=26,
+               window=(3, 15, 15), block=(5, 4, 13), dtype="fp32", seed=47),
 ]
 
 
