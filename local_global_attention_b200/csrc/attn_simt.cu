@@ -5,13 +5,16 @@
 // Operator ("Geometry Matters in Packed 3D Attention", abstract): exact
 // attention over each query's clipped 3D window plus the summaries of the
 // blocks that do not meet the window, one softmax, axial RoPE on grid
-// coordinates.  One CTA serves one query tile of one (batch item, head);
-// G = d / 24 threads (at least 1) share a query, each owning CPT = d / G
+// coordinates.  One CTA serves one 4 x 4 x 8 tile of one (batch item, head).
+// G = d / 24 threads (at least 1) share a token, each owning CPT = d / G
 // channels, and dot products are finished with warp shuffles inside the
-// group.  Keys are staged per chunk of KC tokens in shared memory, already
-// rotated, as fp32.  Every reduction runs in a fixed order; key coordinates are
-// derived from the halo box, query coordinates from the tile box, so no
-// coordinate array is read.
+// group.  The forward stages keys per chunk of KC tokens in shared memory,
+// already rotated, as fp32.  The backward's dq and dk/dv kernels give each
+// warp a 2 x 2 x 2 box of the tile.  They stage the halo one z-plane at a time
+// and let each warp walk only the halo rows its box's windows reach.  The
+// summary gradients at d = 96 have their own register-tiled kernel.  Every
+// reduction runs in a fixed order.  Key coordinates come from the halo box
+// and query coordinates from the tile box, so no coordinate array is read.
 #include <math.h>
 
 #include <algorithm>
