@@ -106,7 +106,7 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
 
 // One box of a 5-D / 3-D tensor map (coordinates innermost first) into shared
 // memory; completion is signalled on `bar` as transaction bytes.  Plain loads
-// from this GPU's memory, no multicast.
+// from this GPU's memory into this CTA's shared memory only.
 __device__ __forceinline__ void tma_load_5d(void* dst, const void* map, int c0, int c1, int c2,
                                             int c3, int c4, uint64_t* bar) {
   asm volatile(
@@ -126,7 +126,7 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const void* map, int c0, 
 }
 // Contiguous global -> shared copy of `bytes` (a multiple of 16; both
 // addresses 16-byte aligned), completion signalled on `bar` as transaction
-// bytes.  No multicast.
+// bytes.  The destination is this CTA's shared memory only.
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
                                           uint64_t* bar) {
   asm volatile(
