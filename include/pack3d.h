@@ -18,8 +18,11 @@
  *     on that axis); v is not rotated.
  *   - window (wz, wy, wx), all odd: the box of half-widths (w - 1) / 2
  *     centred on the query, clipped at the volume edge (never shifted).
- *   - blocks (bz, by, bx) tile the volume exactly (they must divide Z, Y, X);
- *     a block's summary is the mean of its tokens' rotated keys and the mean
+ *   - blocks (bz, by, bx) tile the volume; this library is built for extents
+ *     that divide Z, Y, X (others report PACK3D_ERR_UNSUPPORTED: the operator
+ *     then cuts the last block along an axis at the volume's edge and averages
+ *     over the tokens it holds); a block's summary is the mean of its tokens'
+ *     rotated keys and the mean
  *     of their values; a query sees the summary of every block whose box does
  *     not intersect its window box, with logit scale * q~ . kbar and no
  *     count bias.
@@ -76,8 +79,10 @@ enum {
 };
 
 /* Operator shape and conventions.  head_dim must be a multiple of 12 and at
- * most 96 (12, 24, 48, 96 are built), windows odd and positive, blocks must
- * divide the volume, 1 <= Z, Y, X <= 32767 and B * N * H * head_dim < 2^31. */
+ * most 96 (12, 24, 48, 96 are built), windows odd and positive, block extents
+ * positive (extents that do not divide the volume report
+ * PACK3D_ERR_UNSUPPORTED), 1 <= Z, Y, X <= 32767 and
+ * B * N * H * head_dim < 2^31. */
 typedef struct {
   int32_t B, H, head_dim;
   int32_t Z, Y, X;

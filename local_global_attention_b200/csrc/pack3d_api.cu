@@ -26,8 +26,7 @@ int make_geo(const pack3d_params* p, Geo* g) {
     return PACK3D_ERR_ARG;
   if (p->wz < 1 || p->wy < 1 || p->wx < 1 || !(p->wz & 1) || !(p->wy & 1) || !(p->wx & 1))
     return PACK3D_ERR_ARG;
-  if (p->bz < 1 || p->by < 1 || p->bx < 1 || p->Z % p->bz || p->Y % p->by || p->X % p->bx)
-    return PACK3D_ERR_ARG;
+  if (p->bz < 1 || p->by < 1 || p->bx < 1) return PACK3D_ERR_ARG;
   if (!(p->rope_base > 0.f) || !isfinite(p->rope_base) || !isfinite(p->scale))
     return PACK3D_ERR_ARG;
   if (p->dtype != PACK3D_BF16 && p->dtype != PACK3D_FP32) return PACK3D_ERR_ARG;
@@ -37,6 +36,8 @@ int make_geo(const pack3d_params* p, Geo* g) {
   if ((int64_t)p->B * N * p->H * p->head_dim >= (int64_t)1 << 31) return PACK3D_ERR_ARG;
   if (p->head_dim != 12 && p->head_dim != 24 && p->head_dim != 48 && p->head_dim != 96)
     return PACK3D_ERR_UNSUPPORTED;
+  // blocks cut at the volume's edge are a valid operator the kernels do not build
+  if (p->Z % p->bz || p->Y % p->by || p->X % p->bx) return PACK3D_ERR_UNSUPPORTED;
   g->B = p->B;
   g->H = p->H;
   g->d = p->head_dim;

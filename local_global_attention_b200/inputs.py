@@ -58,7 +58,7 @@ def packing_order(name: str, Z: int, Y: int, X: int, block=(1, 1, 1), seed: int 
         return np.argsort(_morton_codes(c, nbits), kind="stable").astype(np.int64)
     if name == "block":
         bz, by, bx = block
-        nby, nbx = Y // by, X // bx
+        nby, nbx = -(-Y // by), -(-X // bx)
         bid = ((c[:, 0] // bz) * nby + (c[:, 1] // by)) * nbx + (c[:, 2] // bx)
         inner = ((c[:, 0] % bz) * by + (c[:, 1] % by)) * bx + (c[:, 2] % bx)
         return np.lexsort((inner, bid)).astype(np.int64)
@@ -138,7 +138,9 @@ class Workload:
 
     @property
     def n_blocks(self) -> int:
-        return (self.Z // self.block[0]) * (self.Y // self.block[1]) * (self.X // self.block[2])
+        # the last block along an axis is cut at the volume's edge when the
+        # extent does not divide the volume
+        return (-(-self.Z // self.block[0])) * (-(-self.Y // self.block[1])) * (-(-self.X // self.block[2]))
 
     def replace(self, **kw) -> "Workload":
         d = dict(self.__dict__)

@@ -166,7 +166,7 @@ def block_summaries(shape, coords, k, v):
     ka, dt = _as_input(k)
     va, dt2 = _as_input(v)
     assert dt == dt2
-    nb = (shape.Z // shape.block[0]) * (shape.Y // shape.block[1]) * (shape.X // shape.block[2])
+    nb = (-(-shape.Z // shape.block[0])) * (-(-shape.Y // shape.block[1])) * (-(-shape.X // shape.block[2]))
     ks = np.empty((shape.B, shape.H, nb, shape.d), np.float64)
     vs = np.empty_like(ks)
     _check(lib().oracle_block_summaries(ctypes.byref(params(shape)), _ptr(c), _ptr(ka),

@@ -21,8 +21,10 @@
  *   2. W(i): the tokens j whose coordinate lies in the box
  *      [c_i - r, c_i + r] (r = (w - 1) / 2 per axis) clipped to the volume.
  *   3. Blocks: the volume cut into contiguous bz x by x bx boxes, in raster
- *      order.  kbar_B = mean over the block's tokens of k~_j, vbar_B = mean of
- *      v_j, summed in raster order inside the block.
+ *      order; where an extent does not divide the volume, the last box along
+ *      that axis is cut at the volume's edge.  kbar_B = mean over the block's
+ *      tokens of k~_j, vbar_B = mean of v_j (over the tokens the block actually
+ *      holds), summed in raster order inside the block.
  *   4. S(i): the blocks whose box does not intersect the window box of i.
  *   5. Logits tau * q~_i . k~_j (j in W(i)) and tau * q~_i . kbar_B (B in
  *      S(i)), with no count bias; one softmax over both sets.
@@ -82,7 +84,6 @@ static int check_params(const orc_params* p) {
   if (p->wz < 1 || p->wy < 1 || p->wx < 1) return ORC_ERR_ARG;
   if (p->wz % 2 == 0 || p->wy % 2 == 0 || p->wx % 2 == 0) return ORC_ERR_ARG;
   if (p->bz < 1 || p->by < 1 || p->bx < 1) return ORC_ERR_ARG;
-  if (p->Z % p->bz || p->Y % p->by || p->X % p->bx) return ORC_ERR_ARG;
   if (!(p->base > 0.0)) return ORC_ERR_ARG;
   if (p->rope_mode != 0 && p->rope_mode != 1) return ORC_ERR_ARG;
   return ORC_OK;
@@ -98,8 +99,20 @@ static size_t vox_id(const orc_params* p, int z, int y, int x) {
   return ((size_t)z * p->Y + y) * p->X + x;
 }
 
+/* Blocks along each axis (the last one cut at the volume's edge when the
+ * extent does not divide the volume). */
+static int nb_axis(int dim, int ext) { return (dim + ext - 1) / ext; }
+
 static int nblocks(const orc_params* p) {
-  return (p->Z / p->bz) * (p->Y / p->by) * (p->X / p->bx);
+  return nb_axis(p->Z, p->bz) * nb_axis(p->Y, p->by) * nb_axis(p->X, p->bx);
+}
+
+/* Number of tokens block (Bz, By, Bx) holds: its box clipped to the volume. */
+static double block_count(const orc_params* p, int Bz, int By, int Bx) {
+  int lz = (Bz + 1) * p->bz < p->Z ? p->bz : p->Z - Bz * p->bz;
+  int ly = (By + 1) * p->by < p->Y ? p->by : p->Y - By * p->by;
+  int lx = (Bx + 1) * p->bx < p->X ? p->bx : p->X - Bx * p->bx;
+  return (double)lz * ly * lx;
 }
 
 /* Axial mode: cos and sin of c * theta_j for every axis, coordinate value and
@@ -287,19 +300,19 @@ int oracle_rope(const orc_params* p, const int16_t* coords, const void* x, int d
 static void summaries_bh(const orc_params* p, const double* tab, const int32_t* vb,
                          const int16_t* coords, const void* k, const void* v, int dtype, int b,
                          int h, double* ks, double* vs) {
-  int nby = p->Y / p->by, nbx = p->X / p->bx;
+  int nby = nb_axis(p->Y, p->by), nbx = nb_axis(p->X, p->bx);
   int nb = nblocks(p), d = p->d;
-  double cnt = (double)p->bz * p->by * p->bx;
   double* row = (double*)malloc(sizeof(double) * d);
   double* rot = (double*)malloc(sizeof(double) * d);
   for (int B = 0; B < nb; ++B) {
     int Bz = B / (nby * nbx), By = (B / nbx) % nby, Bx = B % nbx;
     double* kd = ks + (size_t)B * d;
     double* vd = vs + (size_t)B * d;
+    double cnt = block_count(p, Bz, By, Bx);
     for (int c = 0; c < d; ++c) kd[c] = vd[c] = 0.0;
-    for (int z = Bz * p->bz; z < (Bz + 1) * p->bz; ++z)
-      for (int y = By * p->by; y < (By + 1) * p->by; ++y)
-        for (int x = Bx * p->bx; x < (Bx + 1) * p->bx; ++x) {
+    for (int z = Bz * p->bz; z < (Bz + 1) * p->bz && z < p->Z; ++z)
+      for (int y = By * p->by; y < (By + 1) * p->by && y < p->Y; ++y)
+        for (int x = Bx * p->bx; x < (Bx + 1) * p->bx && x < p->X; ++x) {
           size_t j = (size_t)vb[vox_id(p, z, y, x)];
           int cj[3];
           coord_of(coords, p, b, j, cj);
@@ -399,7 +412,7 @@ static int query_logits(const orc_params* p, const double* tab, const int32_t* v
     }
   }
   if (!window_only) {
-    int nby = p->Y / p->by, nbx = p->X / p->bx, nb = nblocks(p);
+    int nby = nb_axis(p->Y, p->by), nbx = nb_axis(p->X, p->bx), nb = nblocks(p);
     for (int B = 0; B < nb; ++B) {
       int Bc[3] = {B / (nby * nbx), (B / nbx) % nby, B % nbx};
       if (block_meets_window(p, Bc, c)) continue;
@@ -520,8 +533,7 @@ int oracle_backward(const orc_params* p, const int16_t* coords, const void* q, c
     return rc;
   }
   double tau = tau_of(p);
-  double cnt = (double)p->bz * p->by * p->bx;
-  int nby = p->Y / p->by, nbx = p->X / p->bx;
+  int nby = nb_axis(p->Y, p->by), nbx = nb_axis(p->X, p->bx);
   int BH = p->B * p->H;
 #pragma omp parallel for schedule(dynamic, 1)
   for (int bh = 0; bh < BH; ++bh) {
@@ -602,6 +614,7 @@ int oracle_backward(const orc_params* p, const int16_t* coords, const void* q, c
           size_t j = (size_t)vb[vox_id(p, z, y, x)];
           if (!window_only) {
             size_t B = ((size_t)(z / p->bz) * nby + (size_t)(y / p->by)) * nbx + (x / p->bx);
+            double cnt = block_count(p, z / p->bz, y / p->by, x / p->bx);
             for (int e = 0; e < d; ++e) {
               dkrot[j * d + e] += dks[B * d + e] / cnt;
               dvacc[j * d + e] += dvs[B * d + e] / cnt;

@@ -174,21 +174,28 @@ def test_one_token_blocks_are_dense_attention(oracle_lib, window):
 
 # ---- summaries --------------------------------------------------------------
 
-def test_summary_logit_is_mean_of_member_logits(oracle_lib):
+@pytest.mark.parametrize("dims,block", [((4, 6, 6), (2, 3, 2)), ((5, 6, 7), (2, 4, 3))],
+                         ids=["dividing", "cut_at_edge"])
+def test_summary_logit_is_mean_of_member_logits(oracle_lib, dims, block):
     """Property (iii): tau q~ . kbar_B = mean over j in B of tau q~ . k~_j, and
-    vbar is the mean of the members' values; blocks found from the coordinates."""
-    s = shape(B=2, H=2, d=12, Z=4, Y=6, X=6, block=(2, 3, 2))
+    vbar is the mean of the members' values; blocks found from the coordinates.
+    Where an extent does not divide the volume, the last blocks hold fewer
+    tokens and the means run over those."""
+    Z, Y, X = dims
+    s = shape(B=2, H=2, d=12, Z=Z, Y=Y, X=X, block=block)
     packed, coords, _ = rand_inputs(s, seed=8)
     ks, vs = oracle.block_summaries(s, coords, packed["k"], packed["v"])
     kr = oracle.rope(s, coords, packed["k"])
     qr = oracle.rope(s, coords, packed["q"])
-    nby, nbx = s.Y // s.block[1], s.X // s.block[2]
+    nby, nbx = -(-s.Y // s.block[1]), -(-s.X // s.block[2])
     for b in range(s.B):
         c = coords[b].astype(np.int64)
         bid = ((c[:, 0] // s.block[0]) * nby + c[:, 1] // s.block[1]) * nbx + c[:, 2] // s.block[2]
         for B in range(ks.shape[2]):
             members = np.nonzero(bid == B)[0]
-            assert members.size == np.prod(s.block)
+            Bc = (B // (nby * nbx), (B // nbx) % nby, B % nbx)
+            held = np.prod([min(e, n - i * e) for i, e, n in zip(Bc, s.block, (Z, Y, X))])
+            assert members.size == held
             for h in range(s.H):
                 ql = qr[b, :, h] @ ks[b, h, B]
                 want = (qr[b, :, h] @ kr[b, members, h].T).mean(axis=1)
@@ -242,6 +249,9 @@ def brute_force(s, packed, coords, b, window_only=False):
     dict(Z=6, Y=4, X=4, window=(3, 1, 5), block=(3, 2, 2)),
     dict(Z=4, Y=4, X=8, window=(1, 3, 3), block=(4, 2, 4)),
     dict(Z=5, Y=5, X=5, window=(5, 5, 3), block=(5, 1, 1)),
+    # extents that do not divide the volume: the last blocks are cut at its edge
+    dict(Z=5, Y=5, X=7, window=(3, 3, 3), block=(2, 3, 4)),
+    dict(Z=4, Y=6, X=5, window=(1, 3, 5), block=(3, 4, 2)),
 ])
 @pytest.mark.parametrize("window_only", [False, True])
 def test_brute_force_masked_softmax(oracle_lib, cfg, window_only):
@@ -270,10 +280,13 @@ def test_sampled_forward_matches_full(oracle_lib):
 
 # ---- memory-order independence -------------------------------------------
 
-def test_packing_equivariance_bit_exact(oracle_lib):
+@pytest.mark.parametrize("dims,block", [((4, 8, 8), (2, 4, 4)), ((5, 7, 8), (2, 3, 3))],
+                         ids=["dividing", "cut_at_edge"])
+def test_packing_equivariance_bit_exact(oracle_lib, dims, block):
     """Property (iv): raster, Morton, block-contiguous and random packings of
     the same field give the same per-voxel outputs, bit for bit."""
-    s = shape(B=2, H=2, d=12, Z=4, Y=8, X=8, window=(3, 3, 3), block=(2, 4, 4))
+    Z, Y, X = dims
+    s = shape(B=2, H=2, d=12, Z=Z, Y=Y, X=X, window=(3, 3, 3), block=block)
     g = torch.Generator().manual_seed(11)
     N = s.Z * s.Y * s.X
     grid = {n: torch.randn(s.B, N, s.H, s.d, generator=g, dtype=torch.float64) for n in "qkv"}
@@ -297,13 +310,32 @@ def test_packing_equivariance_bit_exact(oracle_lib):
             np.testing.assert_array_equal(raster_lse, ref[1])
 
 
+def test_block_larger_than_volume_equals_the_volume_wide_block(oracle_lib):
+    """A block extent beyond the volume holds the same tokens as the extent of
+    the volume itself, so summaries, outputs and gradients agree bit for bit."""
+    base = dict(B=2, H=2, d=12, Z=4, Y=6, X=5, window=(3, 3, 3))
+    s_cut, s_fit = shape(block=(2, 3, 8), **base), shape(block=(2, 3, 5), **base)
+    packed, coords, _ = rand_inputs(s_fit, seed=21)
+    args = (coords, packed["q"], packed["k"], packed["v"])
+    for got, want in zip(oracle.block_summaries(s_cut, coords, packed["k"], packed["v"]),
+                         oracle.block_summaries(s_fit, coords, packed["k"], packed["v"])):
+        np.testing.assert_array_equal(got, want)
+    for got, want in zip(oracle.forward(s_cut, *args), oracle.forward(s_fit, *args)):
+        np.testing.assert_array_equal(got, want)
+    for got, want in zip(oracle.backward(s_cut, *args, packed["dout"]),
+                         oracle.backward(s_fit, *args, packed["dout"])):
+        np.testing.assert_array_equal(got, want)
+
+
 # ---- backward -------------------------------------------------------------
 
 @pytest.mark.parametrize("window_only", [False, True])
-def test_backward_finite_differences(oracle_lib, window_only):
+@pytest.mark.parametrize("block", [(2, 2, 3), (3, 3, 4)], ids=["dividing", "cut_at_edge"])
+def test_backward_finite_differences(oracle_lib, window_only, block):
     """Central differences of sum(dout * out) against the analytic gradients,
-    including the paths through the rotation and through the block means."""
-    s = shape(B=1, H=2, d=12, Z=4, Y=4, X=6, window=(3, 3, 3), block=(2, 2, 3))
+    including the paths through the rotation and through the block means (with
+    blocks cut at the volume's edge in the second case)."""
+    s = shape(B=1, H=2, d=12, Z=4, Y=4, X=6, window=(3, 3, 3), block=block)
     packed, coords, _ = rand_inputs(s, seed=12)
     dq, dk, dv = oracle.backward(s, coords, packed["q"], packed["k"], packed["v"],
                                  packed["dout"], window_only=window_only)
