@@ -211,6 +211,22 @@ def whole_job_rate(tokens_per_rank, world, ms):
     return tokens_per_rank * world / (ms * 1e-3)
 
 
+def run_config(wl, packing, world):
+    """The workload a line is quoted on; both arms print the same one."""
+    B, N, H, d = wl.B, wl.N, wl.H, wl.d
+    return {
+        "workload": f"{wl.name}: {N} tokens x batch {B}, {H} heads, head_dim {d}, "
+                    f"window {'x'.join(map(str, wl.window))}, blocks "
+                    f"{'x'.join(map(str, wl.block))} ({wl.n_blocks} summaries), {packing} packing",
+        "step": "index build + block summaries fused with key/value staging + attention (out, lse)",
+        "global_batch": B * world,
+        "seq_len": N,
+        "parallelism": f"replicas x{world} (independent batches, no collective)",
+        "l2": "inputs larger than L2: q, k, v = "
+              f"{3 * B * N * H * d * 2 / 1e6:.0f} MB per step, no flush",
+    }
+
+
 def run_ours(args):
     import torch
 
@@ -409,17 +425,7 @@ def run_ours(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded N(0,1)/sqrt(96) q, k, v; random packing)",
-        "config": {
-            "workload": f"{wl.name}: {wl.N} tokens x batch {B}, {H} heads, head_dim {d}, "
-                        f"window {'x'.join(map(str, wl.window))}, blocks "
-                        f"{'x'.join(map(str, wl.block))} ({nb} summaries), {args.packing} packing",
-            "step": "index build + block summaries fused with key/value staging + attention (out, lse)",
-            "global_batch": B * world,
-            "seq_len": N,
-            "parallelism": f"replicas x{world} (independent batches, no collective)",
-            "l2": "inputs larger than L2: q, k, v = "
-                  f"{3 * B * N * H * d * 2 / 1e6:.0f} MB per step, no flush",
-        },
+        "config": run_config(wl, args.packing, world),
         "gpu_launches": KERNELS_PER_STEP * args.steps,
         "roofline": {
             "bound": "tensor",
@@ -520,10 +526,11 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(times) / len(times),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (same workload and seed as the CUDA arm)",
-        "config": {"workload": f"{wl.name}, {args.packing} packing; each step a sample of "
-                               f"{n} query tokens x {wl.H} heads (summaries precomputed)"},
+        "config": run_config(wl, args.packing, world),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.max_threads(),
-                         "kind": "oracle", "sample": f"{n} tokens x {wl.H} heads per step"},
+                         "kind": "oracle",
+                         "sample": f"each step {n} random query tokens x {wl.H} heads of "
+                                   f"{wl.name} (block summaries precomputed)"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)

@@ -72,3 +72,28 @@ def test_reference_arm_only_on_rank_zero(monkeypatch):
     with redirect_stdout(buf):
         bench.run_reference(args)
     assert buf.getvalue() == ""
+
+
+def test_reference_arm_line_on_rank_zero(monkeypatch):
+    """Rank 0 of the oracle arm prints one JSON line with the CUDA arm's metric,
+    unit and config, the cpu_baseline it measured and a zero-copy e2e."""
+    import bench
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    monkeypatch.setenv("RANK", "0")
+    args = type("A", (), dict(workload="tiny_8x8x8", packing="raster", steps=1, warmup=3,
+                              cpu_sample=64))()
+    buf = io.StringIO()
+    with redirect_stdout(buf):
+        bench.run_reference(args)
+    lines = [ln for ln in buf.getvalue().splitlines() if ln.strip()]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference"
+    assert line["metric"] == bench.METRIC and line["unit"] == bench.UNIT
+    assert line["higher_is_better"] is True and line["value"] > 0
+    assert (line["steps"], line["warmup"], line["n_gpus"]) == (1, 3, 1)
+    assert line["config"] == bench.run_config(bench.workload("tiny_8x8x8"), "raster", 1)
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1
+    assert line["e2e"] == {"value": line["value"], "unit": bench.UNIT,
+                           "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
