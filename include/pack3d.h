@@ -234,7 +234,7 @@ PACK3D_API int pack3d_backward(const pack3d_params* p, const pack3d_index* idx, 
                     pack3d_stream_t stream);
 
 /* Size of the device scratch array behind pack3d_backward_noalloc. */
-#define PACK3D_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+#define PACK3D_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
 
 /* The backward of pack3d_backward for callers that cannot allocate device
  * memory: code that is handed its input and output buffers by a host
@@ -245,13 +245,13 @@ PACK3D_API int pack3d_backward(const pack3d_params* p, const pack3d_index* idx, 
  * workspace.
  *
  * The workspace lives in a static device array of
- * PACK3D_NOALLOC_SCRATCH_BYTES (16 MiB) inside this library; every GPU on
+ * PACK3D_NOALLOC_SCRATCH_BYTES (32 MiB) inside this library; every GPU on
  * which the library is used holds that array until the process exits.  The
  * first call on a device looks up the array's device address with that device
  * current (cudaGetSymbolAddress); make that first call before any stream
  * capture.  Shapes whose workspace (pack3d_backward_workspace_bytes) exceeds
  * the array are rejected with PACK3D_ERR_UNSUPPORTED before anything is
- * launched (the 65k-token, 8-head training shape needs 7 MiB).  Nothing is
+ * launched (the 65k-token, 8-head training shape needs 20.5 MiB).  Nothing is
  * allocated or freed.  Every call on every stream shares the one array: calls
  * whose executions overlap on the GPU race and give wrong results, so issue
  * them on one stream or serialise them.  Each call writes every scratch byte it

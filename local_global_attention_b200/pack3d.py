@@ -316,7 +316,7 @@ def pack3d_backward(params: Params, index: IndexBuffers, q, k, v, out, lse, dout
     return dq, dk, dv
 
 
-NOALLOC_SCRATCH_BYTES = 16 << 20
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 def pack3d_backward_noalloc(params: Params, index: IndexBuffers, q, k, v, out, lse, dout,

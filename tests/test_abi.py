@@ -117,3 +117,14 @@ def test_forward_workspace_size_and_checks(lib):
                                   ws, ctypes.c_size_t(nbytes), fake, fake, None) == P.ERR_ARG
         assert lib.pack3d_window_forward(ctypes.byref(p), ctypes.byref(idx), fake, fake, fake, ws,
                                          ctypes.c_size_t(nbytes), fake, fake, None) == P.ERR_ARG
+
+
+def test_noalloc_scratch_holds_the_training_shape(lib):
+    """The allocation-free backward's static array (its size stated in the
+    header) holds the 65k-token training shape's workspace."""
+    from local_global_attention_b200 import configs as C
+    hdr = open(HEADER).read()
+    m = re.search(r"#define PACK3D_NOALLOC_SCRATCH_BYTES \(\(size_t\)(\d+) << 20\)", hdr)
+    assert m and (int(m.group(1)) << 20) == P.NOALLOC_SCRATCH_BYTES
+    need = lib.pack3d_backward_workspace_bytes(ctypes.byref(P.make_params(C.TRAIN65K)))
+    assert 0 < need <= P.NOALLOC_SCRATCH_BYTES
