@@ -6,9 +6,12 @@ never does, and this package never touches the CUDA library.  Every numeric
 step lives in the C file, which states the definition it follows.
 
 Functions take a *shape* object with attributes ``B, H, d, Z, Y, X, window,
-block, rope_base`` (and optionally ``scale``) and torch tensors or numpy arrays
-in packed order; bf16 inputs are passed as their exact bit patterns, fp32 and
-fp64 as is.  Outputs are fp64 numpy arrays.
+block, rope_base`` (and optionally ``scale``, ``rope_mode`` and ``n_tokens``)
+and torch tensors or numpy arrays in packed order; bf16 inputs are passed as
+their exact bit patterns, fp32 and fp64 as is.  Outputs are fp64 numpy arrays.
+``n_tokens`` > 0 describes a partly occupied volume: every batch item holds
+that many tokens at distinct voxels (coords [B, n_tokens, 3]); 0 or absent
+means one token per voxel.
 """
 from __future__ import annotations
 
@@ -30,7 +33,8 @@ ERR = {0: "ok", -1: "bad argument", -2: "bad coordinates", -3: "out of memory"}
 class Params(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
                 ("B", "H", "d", "Z", "Y", "X", "wz", "wy", "wx", "bz", "by", "bx")] + [
-        ("base", ctypes.c_double), ("scale", ctypes.c_double), ("rope_mode", ctypes.c_int32)]
+        ("base", ctypes.c_double), ("scale", ctypes.c_double), ("rope_mode", ctypes.c_int32),
+        ("n_tokens", ctypes.c_int32)]
 
 # rope_mode: 0 = axial RoPE on grid coordinates (PACK3D); 1 = one-dimensional
 # RoPE on the packed position (the packed-sequence comparison mode)
@@ -78,7 +82,12 @@ def params(shape) -> Params:
     w, b = tuple(shape.window), tuple(shape.block)
     return Params(shape.B, shape.H, shape.d, shape.Z, shape.Y, shape.X, w[0], w[1], w[2],
                   b[0], b[1], b[2], float(shape.rope_base), float(getattr(shape, "scale", 0.0) or 0.0),
-                  int(getattr(shape, "rope_mode", 0) or 0))
+                  int(getattr(shape, "rope_mode", 0) or 0), int(getattr(shape, "n_tokens", 0) or 0))
+
+
+def n_tokens(shape) -> int:
+    """Tokens per batch item: n_tokens when the volume is partly occupied, else Z*Y*X."""
+    return int(getattr(shape, "n_tokens", 0) or 0) or shape.Z * shape.Y * shape.X
 
 
 def _as_input(x):
@@ -154,7 +163,7 @@ def rope(shape, coords, x, transpose=False):
     """R(c_i) x_i (or R(c_i)^T x_i) for every row, fp64 [B, N, H, d]."""
     c = _coords(coords)
     a, dt = _as_input(x)
-    out = np.empty((shape.B, shape.Z * shape.Y * shape.X, shape.H, shape.d), np.float64)
+    out = np.empty((shape.B, n_tokens(shape), shape.H, shape.d), np.float64)
     _check(lib().oracle_rope(ctypes.byref(params(shape)), _ptr(c), _ptr(a), dt,
                              int(bool(transpose)), _ptr(out)))
     return out
@@ -185,7 +194,7 @@ def forward(shape, coords, q, k, v, sel=None, window_only=False, summaries=None)
     qa, dt = _as_input(q)
     ka, _ = _as_input(k)
     va, _ = _as_input(v)
-    N = shape.Z * shape.Y * shape.X
+    N = n_tokens(shape)
     full = sel is None
     if full:
         sel = np.arange(shape.B * shape.H * N, dtype=np.int64)
@@ -213,7 +222,7 @@ def backward(shape, coords, q, k, v, dout, window_only=False):
     ka, _ = _as_input(k)
     va, _ = _as_input(v)
     da, _ = _as_input(dout)
-    shp = (shape.B, shape.Z * shape.Y * shape.X, shape.H, shape.d)
+    shp = (shape.B, n_tokens(shape), shape.H, shape.d)
     dq, dk, dv = (np.zeros(shp, np.float64) for _ in range(3))
     _check(lib().oracle_backward(ctypes.byref(params(shape)), _ptr(c), _ptr(qa), _ptr(ka),
                                  _ptr(va), _ptr(da), dt, int(bool(window_only)), _ptr(dq),
@@ -223,5 +232,5 @@ def backward(shape, coords, q, k, v, dout, window_only=False):
 
 def flat_index(shape, b, h, i):
     """Flat query selector ``(b*H + h)*N + i`` used by :func:`forward`."""
-    N = shape.Z * shape.Y * shape.X
+    N = n_tokens(shape)
     return (np.asarray(b, np.int64) * shape.H + np.asarray(h, np.int64)) * N + np.asarray(i, np.int64)

@@ -46,6 +46,12 @@
  * Layouts: q, k, v, dout, dq, dk, dv are [B][N][H][d] in packed order; coords
  * is int16 [B][N][3] as (z, y, x); summaries are [B][H][nb][d] in block raster
  * order; lse is [B][H][N].
+ *
+ * Occupancy: by default (n_tokens = 0) the tokens fill the volume, N = Z*Y*X,
+ * one token per voxel.  With n_tokens > 0 every batch item holds N = n_tokens
+ * tokens at distinct voxels and the other voxels are empty: windows and blocks
+ * then hold only the tokens present, a block's summary averages over its
+ * present tokens, and a block holding none has no summary (it is in no S(i)).
  */
 #include <math.h>
 #include <stdint.h>
@@ -62,6 +68,7 @@ typedef struct {
   double base;
   double scale;      /* tau; <= 0 means 1/sqrt(d) */
   int32_t rope_mode; /* 0: axial on grid coordinates; 1: 1-D on the packed position */
+  int32_t n_tokens;  /* 0: dense volume (N = Z*Y*X); > 0: N tokens at distinct voxels */
 } orc_params;
 
 enum { ORC_OK = 0, ORC_ERR_ARG = -1, ORC_ERR_COORDS = -2, ORC_ERR_MEM = -3 };
@@ -86,6 +93,7 @@ static int check_params(const orc_params* p) {
   if (p->bz < 1 || p->by < 1 || p->bx < 1) return ORC_ERR_ARG;
   if (!(p->base > 0.0)) return ORC_ERR_ARG;
   if (p->rope_mode != 0 && p->rope_mode != 1) return ORC_ERR_ARG;
+  if (p->n_tokens < 0 || (int64_t)p->n_tokens > (int64_t)p->Z * p->Y * p->X) return ORC_ERR_ARG;
   return ORC_OK;
 }
 
@@ -94,6 +102,9 @@ static double tau_of(const orc_params* p) {
 }
 
 static size_t nvox(const orc_params* p) { return (size_t)p->Z * p->Y * p->X; }
+
+/* Tokens per batch item. */
+static size_t ntok(const orc_params* p) { return p->n_tokens > 0 ? (size_t)p->n_tokens : nvox(p); }
 
 static size_t vox_id(const orc_params* p, int z, int y, int x) {
   return ((size_t)z * p->Y + y) * p->X + x;
@@ -107,12 +118,15 @@ static int nblocks(const orc_params* p) {
   return nb_axis(p->Z, p->bz) * nb_axis(p->Y, p->by) * nb_axis(p->X, p->bx);
 }
 
-/* Number of tokens block (Bz, By, Bx) holds: its box clipped to the volume. */
-static double block_count(const orc_params* p, int Bz, int By, int Bx) {
-  int lz = (Bz + 1) * p->bz < p->Z ? p->bz : p->Z - Bz * p->bz;
-  int ly = (By + 1) * p->by < p->Y ? p->by : p->Y - By * p->by;
-  int lx = (Bx + 1) * p->bx < p->X ? p->bx : p->X - Bx * p->bx;
-  return (double)lz * ly * lx;
+/* Tokens held by every block of one batch item (vb: its volume, -1 where a
+ * voxel is empty): cnt[B] for B in block raster order. */
+static void block_members(const orc_params* p, const int32_t* vb, int32_t* cnt) {
+  int nby = nb_axis(p->Y, p->by), nbx = nb_axis(p->X, p->bx), nb = nblocks(p);
+  for (int B = 0; B < nb; ++B) cnt[B] = 0;
+  for (int z = 0; z < p->Z; ++z)
+    for (int y = 0; y < p->Y; ++y)
+      for (int x = 0; x < p->X; ++x)
+        if (vb[vox_id(p, z, y, x)] >= 0) ++cnt[((z / p->bz) * nby + y / p->by) * nbx + x / p->bx];
 }
 
 /* Axial mode: cos and sin of c * theta_j for every axis, coordinate value and
@@ -121,7 +135,7 @@ static double block_count(const orc_params* p, int Bz, int By, int Bx) {
  * and pair j < d/2: tab[(p * (d/2) + j) * 2 + {0,1}]. */
 static double* rope_table(const orc_params* p) {
   if (p->rope_mode == 1) {
-    size_t N = nvox(p);
+    size_t N = ntok(p);
     int half = p->d / 2;
     double* tab = (double*)malloc(N * half * 2 * sizeof(double));
     if (!tab) return NULL;
@@ -179,12 +193,12 @@ static void rope_apply(const orc_params* p, const double* tab, const double* in,
 
 static void load_row(const void* base, int dtype, const orc_params* p, int b, size_t i, int h,
                      double* row) {
-  size_t o = (((size_t)b * nvox(p) + i) * p->H + h) * p->d;
+  size_t o = (((size_t)b * ntok(p) + i) * p->H + h) * p->d;
   for (int c = 0; c < p->d; ++c) row[c] = widen(base, dtype, o + c);
 }
 
 static void coord_of(const int16_t* coords, const orc_params* p, int b, size_t i, int c[3]) {
-  const int16_t* t = coords + ((size_t)b * nvox(p) + i) * 3;
+  const int16_t* t = coords + ((size_t)b * ntok(p) + i) * 3;
   c[0] = t[0];
   c[1] = t[1];
   c[2] = t[2];
@@ -192,15 +206,16 @@ static void coord_of(const int16_t* coords, const orc_params* p, int b, size_t i
 
 /* ---- coordinate volume ------------------------------------------------ */
 
-/* vol[b][voxel] = packed index of the token at that voxel.  Every voxel must
- * be held by exactly one token. */
+/* vol[b][voxel] = packed index of the token at that voxel, -1 where empty.
+ * No voxel may hold two tokens (with n_tokens = 0 there are Z*Y*X tokens, so
+ * every voxel holds exactly one). */
 int oracle_volume(const orc_params* p, const int16_t* coords, int32_t* vol) {
   if (check_params(p)) return ORC_ERR_ARG;
-  size_t N = nvox(p);
+  size_t N = nvox(p), NT = ntok(p);
   for (int b = 0; b < p->B; ++b) {
     int32_t* vb = vol + (size_t)b * N;
     for (size_t v = 0; v < N; ++v) vb[v] = -1;
-    for (size_t i = 0; i < N; ++i) {
+    for (size_t i = 0; i < NT; ++i) {
       int c[3];
       coord_of(coords, p, b, i, c);
       if (c[0] < 0 || c[0] >= p->Z || c[1] < 0 || c[1] >= p->Y || c[2] < 0 || c[2] >= p->X)
@@ -225,6 +240,7 @@ int oracle_volume(const orc_params* p, const int16_t* coords, int32_t* vol) {
 int oracle_build_index(const orc_params* p, const int16_t* coords, int tz, int ty, int tx,
                        int32_t* vol, int32_t* perm, int32_t* tile_off, int64_t* nbr_off,
                        int32_t* nbr) {
+  if (ntok(p) != nvox(p)) return ORC_ERR_ARG; /* the index is built for dense volumes */
   int rc = oracle_volume(p, coords, vol);
   if (rc) return rc;
   if (tz < 1 || ty < 1 || tx < 1) return ORC_ERR_ARG;
@@ -279,7 +295,7 @@ int oracle_rope(const orc_params* p, const int16_t* coords, const void* x, int d
   if (check_params(p)) return ORC_ERR_ARG;
   double* tab = rope_table(p);
   if (!tab) return ORC_ERR_MEM;
-  size_t N = nvox(p);
+  size_t N = ntok(p);
   double* row = (double*)malloc(sizeof(double) * p->d);
   for (int b = 0; b < p->B; ++b)
     for (size_t i = 0; i < N; ++i) {
@@ -308,12 +324,14 @@ static void summaries_bh(const orc_params* p, const double* tab, const int32_t* 
     int Bz = B / (nby * nbx), By = (B / nbx) % nby, Bx = B % nbx;
     double* kd = ks + (size_t)B * d;
     double* vd = vs + (size_t)B * d;
-    double cnt = block_count(p, Bz, By, Bx);
+    double cnt = 0.0;
     for (int c = 0; c < d; ++c) kd[c] = vd[c] = 0.0;
     for (int z = Bz * p->bz; z < (Bz + 1) * p->bz && z < p->Z; ++z)
       for (int y = By * p->by; y < (By + 1) * p->by && y < p->Y; ++y)
         for (int x = Bx * p->bx; x < (Bx + 1) * p->bx && x < p->X; ++x) {
+          if (vb[vox_id(p, z, y, x)] < 0) continue;
           size_t j = (size_t)vb[vox_id(p, z, y, x)];
+          cnt += 1.0;
           int cj[3];
           coord_of(coords, p, b, j, cj);
           load_row(k, dtype, p, b, j, h, row);
@@ -322,10 +340,11 @@ static void summaries_bh(const orc_params* p, const double* tab, const int32_t* 
           load_row(v, dtype, p, b, j, h, row);
           for (int c = 0; c < d; ++c) vd[c] += row[c];
         }
-    for (int c = 0; c < d; ++c) {
-      kd[c] /= cnt;
-      vd[c] /= cnt;
-    }
+    if (cnt > 0.0) /* an empty block keeps zero means and gets no summary term */
+      for (int c = 0; c < d; ++c) {
+        kd[c] /= cnt;
+        vd[c] /= cnt;
+      }
   }
   free(row);
   free(rot);
@@ -382,9 +401,9 @@ typedef struct {
 
 /* Logits of one query (grid-order list), returns how many. */
 static int query_logits(const orc_params* p, const double* tab, const int32_t* vb,
-                        const int16_t* coords, const void* q, const void* k, int dtype,
-                        const double* ks, int b, int h, size_t i, int window_only,
-                        orc_scratch* s) {
+                        const int32_t* bcnt, const int16_t* coords, const void* q,
+                        const void* k, int dtype, const double* ks, int b, int h, size_t i,
+                        int window_only, orc_scratch* s) {
   int d = p->d;
   double tau = tau_of(p);
   int c[3];
@@ -398,7 +417,7 @@ static int query_logits(const orc_params* p, const double* tab, const int32_t* v
     for (int y = c[1] - ry; y <= c[1] + ry; ++y) {
       if (y < 0 || y >= p->Y) continue;
       for (int x = c[2] - rx; x <= c[2] + rx; ++x) {
-        if (x < 0 || x >= p->X) continue;
+        if (x < 0 || x >= p->X || vb[vox_id(p, z, y, x)] < 0) continue;
         size_t j = (size_t)vb[vox_id(p, z, y, x)];
         int cj[3] = {z, y, x};
         load_row(k, dtype, p, b, j, h, s->row);
@@ -415,7 +434,7 @@ static int query_logits(const orc_params* p, const double* tab, const int32_t* v
     int nby = nb_axis(p->Y, p->by), nbx = nb_axis(p->X, p->bx), nb = nblocks(p);
     for (int B = 0; B < nb; ++B) {
       int Bc[3] = {B / (nby * nbx), (B / nbx) % nby, B % nbx};
-      if (block_meets_window(p, Bc, c)) continue;
+      if (bcnt[B] == 0 || block_meets_window(p, Bc, c)) continue;
       const double* kb = ks + (size_t)B * d;
       double acc = 0.0;
       for (int e = 0; e < d; ++e) acc += s->qrot[e] * kb[e];
@@ -466,8 +485,15 @@ int oracle_forward(const orc_params* p, const int16_t* coords, const void* q, co
     free(tab);
     return rc;
   }
-  size_t per = (size_t)nblocks(p) * p->d;
-  int d = p->d;
+  size_t per = (size_t)nblocks(p) * p->d, NT = ntok(p);
+  int d = p->d, nb = nblocks(p);
+  int32_t* bcnt = (int32_t*)malloc(sizeof(int32_t) * (size_t)nb * p->B);
+  if (!bcnt) {
+    free(vol);
+    free(tab);
+    return ORC_ERR_MEM;
+  }
+  for (int b = 0; b < p->B; ++b) block_members(p, vol + (size_t)b * N, bcnt + (size_t)b * nb);
 #pragma omp parallel
   {
     orc_scratch s;
@@ -476,12 +502,12 @@ int oracle_forward(const orc_params* p, const int16_t* coords, const void* q, co
 #pragma omp for schedule(dynamic, 64)
     for (int64_t n = 0; n < nsel; ++n) {
       int64_t f = sel[n];
-      size_t i = (size_t)(f % (int64_t)N);
-      int bh = (int)(f / (int64_t)N), b = bh / p->H, h = bh % p->H;
+      size_t i = (size_t)(f % (int64_t)NT);
+      int bh = (int)(f / (int64_t)NT), b = bh / p->H, h = bh % p->H;
       const double* ks = window_only ? NULL : ksum + bh * per;
       const double* vs = window_only ? NULL : vsum + bh * per;
-      int nt = query_logits(p, tab, vol + (size_t)b * N, coords, q, k, dtype, ks, b, h, i,
-                            window_only, &s);
+      int nt = query_logits(p, tab, vol + (size_t)b * N, bcnt + (size_t)b * nb, coords, q, k,
+                            dtype, ks, b, h, i, window_only, &s);
       double m = -INFINITY;
       for (int t = 0; t < nt; ++t)
         if (s.logit[t] > m) m = s.logit[t];
@@ -505,6 +531,7 @@ int oracle_forward(const orc_params* p, const int16_t* coords, const void* q, co
     free(row);
     scratch_free(&s);
   }
+  free(bcnt);
   free(vol);
   free(tab);
   return ORC_OK;
@@ -534,17 +561,20 @@ int oracle_backward(const orc_params* p, const int16_t* coords, const void* q, c
   }
   double tau = tau_of(p);
   int nby = nb_axis(p->Y, p->by), nbx = nb_axis(p->X, p->bx);
+  size_t NT = ntok(p);
   int BH = p->B * p->H;
 #pragma omp parallel for schedule(dynamic, 1)
   for (int bh = 0; bh < BH; ++bh) {
     int b = bh / p->H, h = bh % p->H;
     const int32_t* vb = vol + (size_t)b * N;
+    int32_t* bcnt = (int32_t*)malloc(sizeof(int32_t) * (size_t)nb);
+    block_members(p, vb, bcnt);
     double* ks = (double*)calloc((size_t)nb * d, sizeof(double));
     double* vs = (double*)calloc((size_t)nb * d, sizeof(double));
     double* dks = (double*)calloc((size_t)nb * d, sizeof(double));
     double* dvs = (double*)calloc((size_t)nb * d, sizeof(double));
-    double* dkrot = (double*)calloc(N * d, sizeof(double)); /* d/dk~ in packed order */
-    double* dvacc = (double*)calloc(N * d, sizeof(double));
+    double* dkrot = (double*)calloc(NT * d, sizeof(double)); /* d/dk~ in packed order */
+    double* dvacc = (double*)calloc(NT * d, sizeof(double));
     double* dO = (double*)malloc(sizeof(double) * d);
     double* vrow = (double*)malloc(sizeof(double) * d);
     double* dqr = (double*)malloc(sizeof(double) * d);
@@ -557,8 +587,10 @@ int oracle_backward(const orc_params* p, const int16_t* coords, const void* q, c
     for (int z = 0; z < p->Z; ++z)
       for (int y = 0; y < p->Y; ++y)
         for (int x = 0; x < p->X; ++x) {
+          if (vb[vox_id(p, z, y, x)] < 0) continue;
           size_t i = (size_t)vb[vox_id(p, z, y, x)];
-          int nt = query_logits(p, tab, vb, coords, q, k, dtype, ks, b, h, i, window_only, &s);
+          int nt = query_logits(p, tab, vb, bcnt, coords, q, k, dtype, ks, b, h, i, window_only,
+                                &s);
           double m = -INFINITY;
           for (int t = 0; t < nt; ++t)
             if (s.logit[t] > m) m = s.logit[t];
@@ -605,16 +637,17 @@ int oracle_backward(const orc_params* p, const int16_t* coords, const void* q, c
             }
           }
           int ci[3] = {z, y, x};
-          rope_apply(p, tab, dqr, ci, i, 1, dq + (((size_t)b * N + i) * p->H + h) * d);
+          rope_apply(p, tab, dqr, ci, i, 1, dq + (((size_t)b * NT + i) * p->H + h) * d);
         }
     /* Spread the summary gradients over the block members, rotate back. */
     for (int z = 0; z < p->Z; ++z)
       for (int y = 0; y < p->Y; ++y)
         for (int x = 0; x < p->X; ++x) {
+          if (vb[vox_id(p, z, y, x)] < 0) continue;
           size_t j = (size_t)vb[vox_id(p, z, y, x)];
           if (!window_only) {
             size_t B = ((size_t)(z / p->bz) * nby + (size_t)(y / p->by)) * nbx + (x / p->bx);
-            double cnt = block_count(p, z / p->bz, y / p->by, x / p->bx);
+            double cnt = (double)bcnt[B];
             for (int e = 0; e < d; ++e) {
               dkrot[j * d + e] += dks[B * d + e] / cnt;
               dvacc[j * d + e] += dvs[B * d + e] / cnt;
@@ -622,9 +655,10 @@ int oracle_backward(const orc_params* p, const int16_t* coords, const void* q, c
           }
           int cj[3] = {z, y, x};
           for (int e = 0; e < d; ++e) tmp[e] = dkrot[j * d + e];
-          rope_apply(p, tab, tmp, cj, j, 1, dk + (((size_t)b * N + j) * p->H + h) * d);
-          for (int e = 0; e < d; ++e) dv[(((size_t)b * N + j) * p->H + h) * d + e] = dvacc[j * d + e];
+          rope_apply(p, tab, tmp, cj, j, 1, dk + (((size_t)b * NT + j) * p->H + h) * d);
+          for (int e = 0; e < d; ++e) dv[(((size_t)b * NT + j) * p->H + h) * d + e] = dvacc[j * d + e];
         }
+    free(bcnt);
     free(P);
     free(dP);
     scratch_free(&s);

@@ -23,9 +23,10 @@ from local_global_attention_b200 import inputs as I
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 
 
-def shape(B=1, H=1, d=12, Z=4, Y=5, X=6, window=(3, 3, 3), block=(2, 5, 3), base=100.0):
+def shape(B=1, H=1, d=12, Z=4, Y=5, X=6, window=(3, 3, 3), block=(2, 5, 3), base=100.0,
+          n_tokens=0):
     return SimpleNamespace(B=B, H=H, d=d, Z=Z, Y=Y, X=X, window=window, block=block,
-                           rope_base=base, scale=0.0)
+                           rope_base=base, scale=0.0, n_tokens=n_tokens)
 
 
 def rand_inputs(s, seed=0, packing="random"):
@@ -209,9 +210,10 @@ def test_summary_logit_is_mean_of_member_logits(oracle_lib, dims, block):
 def brute_force(s, packed, coords, b, window_only=False):
     """Masked dense softmax over [keys | block summaries] with the geometry
     decided by enumeration: a key is local when every axis offset is within the
-    radius; a block is excluded when any of its voxels is local to the query."""
-    N = s.Z * s.Y * s.X
+    radius; a block is excluded when any voxel of its box (cut at the volume's
+    edge) is local to the query; a block holding no token has no summary."""
     c = coords[b].astype(np.int64)
+    N = c.shape[0]
     r = (np.asarray(s.window) - 1) // 2
     cf = c.astype(np.float64)[:, None, :]
     qr = rotate_complex(packed["q"][b].numpy(), cf, s.rope_base)
@@ -223,6 +225,11 @@ def brute_force(s, packed, coords, b, window_only=False):
     cells = c // blk
     keys = sorted({tuple(x) for x in cells})
     members = [np.nonzero(np.all(cells == np.asarray(kk), axis=1))[0] for kk in keys]
+    boxes = [np.stack(np.meshgrid(*[np.arange(kk[a] * blk[a], min((kk[a] + 1) * blk[a], n))
+                                    for a, n in enumerate((s.Z, s.Y, s.X))], indexing="ij"),
+                      -1).reshape(-1, 3) for kk in keys]
+    seen = np.stack([np.all(np.abs(c[:, None, :] - bx[None]) <= r, axis=-1).any(axis=1)
+                     for bx in boxes], axis=1)  # [Nq, nb]
     tau = 1.0 / math.sqrt(s.d)
     outs, lses = np.zeros((N, s.H, s.d)), np.zeros((s.H, N))
     for h in range(s.H):
@@ -232,7 +239,6 @@ def brute_force(s, packed, coords, b, window_only=False):
         if not window_only:
             kbar = np.stack([kr[m, h].mean(0) for m in members])
             vbar = np.stack([v[m, h].mean(0) for m in members])
-            seen = np.stack([local[:, m].any(axis=1) for m in members], axis=1)  # [Nq, nb]
             cols.append(np.where(seen, -np.inf, tau * qr[:, h] @ kbar.T))
             vals.append(vbar)
         L = np.concatenate(cols, axis=1)
@@ -516,3 +522,105 @@ def test_packed_mode_depends_on_the_packing(oracle_lib):
         res[mode] = np.abs(outs[0] - outs[1]).max()
     assert res[oracle.ROPE_AXIAL] == 0.0
     assert res[oracle.ROPE_PACKED] > 1e-3
+
+
+# ---- partly occupied volumes ----------------------------------------------
+
+def partial_inputs(s, seed):
+    """s.n_tokens distinct voxels per batch item (seeded), in a random packed
+    order, with N(0, 1) q, k, v and dout per token."""
+    g = torch.Generator().manual_seed(seed)
+    V = s.Z * s.Y * s.X
+    coords = np.stack([I.coords_of_order(torch.randperm(V, generator=g)[:s.n_tokens].numpy(),
+                                         s.Z, s.Y, s.X) for _ in range(s.B)])
+    packed = {n: torch.randn(s.B, s.n_tokens, s.H, s.d, generator=g, dtype=torch.float64)
+              for n in ("q", "k", "v", "dout")}
+    return packed, coords
+
+
+PARTIAL = [
+    dict(Z=4, Y=5, X=6, window=(3, 3, 3), block=(2, 3, 4), n_tokens=70),
+    dict(Z=5, Y=4, X=6, window=(3, 1, 5), block=(2, 2, 3), n_tokens=24),
+]
+
+
+@pytest.mark.parametrize("cfg", PARTIAL, ids=["70_of_120", "24_of_120"])
+@pytest.mark.parametrize("window_only", [False, True])
+def test_partly_occupied_brute_force(oracle_lib, cfg, window_only):
+    """Windows and blocks hold only the tokens present; a block's summary
+    averages over them, a block holding none has no summary, exclusion follows
+    the block's box; checked against the enumeration of brute_force."""
+    s = shape(B=2, H=2, d=12, **cfg)
+    packed, coords = partial_inputs(s, seed=31)
+    out, lse = oracle.forward(s, coords, packed["q"], packed["k"], packed["v"],
+                              window_only=window_only)
+    assert out.shape == (s.B, s.n_tokens, s.H, s.d)
+    for b in range(s.B):
+        ro, rl = brute_force(s, packed, coords, b, window_only)
+        np.testing.assert_allclose(out[b], ro, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse[b], rl, rtol=0, atol=1e-12)
+
+
+def test_sparse_case_has_empty_blocks(oracle_lib):
+    """The sparse case above really leaves blocks without tokens (so the
+    no-summary rule is exercised)."""
+    s = shape(B=2, H=2, d=12, **PARTIAL[1])
+    _, coords = partial_inputs(s, seed=31)
+    nblk = np.prod([-(-n // e) for n, e in zip((s.Z, s.Y, s.X), s.block)])
+    for b in range(s.B):
+        held = {tuple(x) for x in coords[b].astype(np.int64) // np.asarray(s.block)}
+        assert len(held) < nblk
+
+
+def test_partly_occupied_packing_equivariance(oracle_lib):
+    """Reordering the tokens of a partly occupied volume permutes the outputs
+    and changes nothing else, bit for bit."""
+    s = shape(B=2, H=2, d=12, **PARTIAL[0])
+    packed, coords = partial_inputs(s, seed=32)
+    out, lse = oracle.forward(s, coords, packed["q"], packed["k"], packed["v"])
+    g = torch.Generator().manual_seed(5)
+    perm = [torch.randperm(s.n_tokens, generator=g).numpy() for _ in range(s.B)]
+    c2 = np.stack([coords[b][perm[b]] for b in range(s.B)])
+    pk2 = {n: torch.stack([packed[n][b][torch.from_numpy(perm[b])] for b in range(s.B)])
+           for n in "qkv"}
+    out2, lse2 = oracle.forward(s, c2, pk2["q"], pk2["k"], pk2["v"])
+    for b in range(s.B):
+        np.testing.assert_array_equal(out2[b], out[b][perm[b]])
+        np.testing.assert_array_equal(lse2[b], lse[b][:, perm[b]])
+
+
+def test_full_occupancy_equals_dense(oracle_lib):
+    """n_tokens = Z*Y*X describes the dense volume: same results, bit for bit."""
+    s0 = shape(B=2, H=2, d=12, Z=4, Y=5, X=6, block=(2, 5, 3))
+    s1 = shape(B=2, H=2, d=12, Z=4, Y=5, X=6, block=(2, 5, 3), n_tokens=120)
+    packed, coords, _ = rand_inputs(s0, seed=33)
+    args = (coords, packed["q"], packed["k"], packed["v"])
+    for got, want in zip(oracle.forward(s1, *args), oracle.forward(s0, *args)):
+        np.testing.assert_array_equal(got, want)
+    for got, want in zip(oracle.backward(s1, *args, packed["dout"]),
+                         oracle.backward(s0, *args, packed["dout"])):
+        np.testing.assert_array_equal(got, want)
+
+
+def test_partly_occupied_backward_finite_differences(oracle_lib):
+    """Central differences of sum(dout * out) against the analytic gradients on
+    a partly occupied volume with cut and empty blocks."""
+    s = shape(B=1, H=2, d=12, Z=4, Y=4, X=5, window=(3, 3, 3), block=(3, 2, 2), n_tokens=30)
+    packed, coords = partial_inputs(s, seed=34)
+    dq, dk, dv = oracle.backward(s, coords, packed["q"], packed["k"], packed["v"],
+                                 packed["dout"])
+    grads = {"q": dq, "k": dk, "v": dv}
+    rng = np.random.default_rng(2)
+    eps = 1e-6
+    dout = packed["dout"].numpy()
+    for name in "qkv":
+        for _ in range(12):
+            idx = tuple(int(rng.integers(0, n)) for n in packed[name].shape)
+            vals = {}
+            for sign in (+1, -1):
+                pk = {n: packed[n].clone() for n in "qkv"}
+                pk[name][idx] += sign * eps
+                out, _ = oracle.forward(s, coords, pk["q"], pk["k"], pk["v"])
+                vals[sign] = (out * dout).sum()
+            fd = (vals[1] - vals[-1]) / (2 * eps)
+            assert abs(fd - grads[name][idx]) <= 1e-6 * max(1.0, abs(fd)), (name, idx)
