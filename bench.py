@@ -40,7 +40,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "forward_tc_vol_32x32x64.md")
 TC_SOURCE = os.path.join(ROOT, "local_global_attention_b200", "csrc", "attn_tc.cu")
 FP32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # CUDA-core fp32 FMA peak, nominal
-KERNELS_PER_STEP = 11  # index build 9, summaries + staging 1, attention 1
+KERNELS_PER_STEP = 10  # index build 8 (plus two memsets), summaries + staging 1, attention 1
 
 
 def peaks():
