@@ -128,3 +128,28 @@ def test_noalloc_scratch_holds_the_training_shape(lib):
     assert m and (int(m.group(1)) << 20) == P.NOALLOC_SCRATCH_BYTES
     need = lib.pack3d_backward_workspace_bytes(ctypes.byref(P.make_params(C.TRAIN65K)))
     assert 0 < need <= P.NOALLOC_SCRATCH_BYTES
+
+
+def test_backward_workspace_layout(lib):
+    """Backward workspace = delta [B][H][N] + k/v summaries and their gradients
+    (4 x [B][H][nb][d] fp32, each 256-byte aligned) + the d = 96 summary
+    kernel's per-split partial sums (2 x splits x [B][H][nb][d]); the splits
+    fill one wave of two CTAs per SM (148 SMs) over B*H*ceil(nb/64) groups,
+    at most one per query tile and at most 32."""
+    from local_global_attention_b200 import configs as C
+
+    def a256(x):
+        return (x + 255) // 256 * 256
+
+    for wl in (C.TRAIN65K, C.VOL16K):
+        nb, nT = wl.n_blocks, -(-wl.Z // 4) * -(-wl.Y // 4) * -(-wl.X // 8)
+        groups = wl.B * wl.H * -(-nb // 64)
+        splits = max(1, min(296 // groups, nT, 32))
+        ns = 4 * wl.B * wl.H * nb * wl.d
+        want = a256(4 * wl.B * wl.H * wl.N) + 4 * a256(ns) + 2 * splits * ns
+        assert lib.pack3d_backward_workspace_bytes(ctypes.byref(P.make_params(wl))) == want
+    # other head dims use the simple summary kernel: no partial sums
+    wl = C.TINY
+    ns = 4 * wl.B * wl.H * wl.n_blocks * wl.d
+    assert lib.pack3d_backward_workspace_bytes(ctypes.byref(P.make_params(wl))) == \
+        a256(4 * wl.B * wl.H * wl.N) + 4 * a256(ns)
