@@ -1118,17 +1118,14 @@ int backward_typed(const Geo& g, const pack3d_index* idx, const void* q, const v
   if constexpr (D == 96) {
     const int nsplit = summary96_splits(g);
     const int nbc = (g.nb + S96_NB - 1) / S96_NB;
-    static bool attr_set = false;
-    if (!attr_set) {
-      cudaError_t e = cudaFuncSetAttribute(k_bwd_summary96<T>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)sizeof(Sum96Smem));
-      if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(k_bwd_summary96<T>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                 (int)cudaSharedmemCarveoutMaxShared);
-      if (e != cudaSuccess) return cuda_status(e);
-      attr_set = true;
-    }
+    // set on every call: the attributes belong to the current device
+    cudaError_t e = cudaFuncSetAttribute(k_bwd_summary96<T>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)sizeof(Sum96Smem));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k_bwd_summary96<T>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return cuda_status(e);
     dim3 sgrid(nbc * nsplit, g.B, g.H);
     k_bwd_summary96<T><<<sgrid, S96_THREADS, sizeof(Sum96Smem), s>>>(
         g, *idx, (const T*)q, (const T*)dout, lse, w.delta, w.ksum, w.vsum, nsplit, w.part);
@@ -1143,15 +1140,13 @@ int backward_typed(const Geo& g, const pack3d_index* idx, const void* q, const v
   // one halo row must fit in a staged chunk
   if (TX + 2 * g.rx > CAPK) return PACK3D_ERR_UNSUPPORTED;
   const size_t dyn = 2 * (size_t)CAPK * D * sizeof(float);
-  static bool local_attr_set = false;
-  if (!local_attr_set) {
+  {
     cudaError_t e = cudaFuncSetAttribute(k_bwd_dq<T, D, true>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(k_bwd_dkdv<T, D, true>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
     if (e != cudaSuccess) return cuda_status(e);
-    local_attr_set = true;
   }
   dim3 grid(g.nT, g.H, g.B);
   dim3 block(TILE * Split<D>::G);
