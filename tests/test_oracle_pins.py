@@ -624,3 +624,17 @@ def test_partly_occupied_backward_finite_differences(oracle_lib):
                 vals[sign] = (out * dout).sum()
             fd = (vals[1] - vals[-1]) / (2 * eps)
             assert abs(fd - grads[name][idx]) <= 1e-6 * max(1.0, abs(fd)), (name, idx)
+
+
+def test_batch_items_are_independent(oracle_lib):
+    """Batch items never interact: a two-item call equals two one-item calls,
+    bit for bit (so ragged batches are item-by-item calls)."""
+    s2 = shape(B=2, H=2, d=12, **PARTIAL[0])
+    packed, coords = partial_inputs(s2, seed=35)
+    out, lse = oracle.forward(s2, coords, packed["q"], packed["k"], packed["v"])
+    s1 = shape(B=1, H=2, d=12, **PARTIAL[0])
+    for b in range(2):
+        o1, l1 = oracle.forward(s1, coords[b:b + 1], packed["q"][b:b + 1], packed["k"][b:b + 1],
+                                packed["v"][b:b + 1])
+        np.testing.assert_array_equal(o1[0], out[b])
+        np.testing.assert_array_equal(l1[0], lse[b])
