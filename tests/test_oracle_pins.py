@@ -638,3 +638,41 @@ def test_batch_items_are_independent(oracle_lib):
                                 packed["v"][b:b + 1])
         np.testing.assert_array_equal(o1[0], out[b])
         np.testing.assert_array_equal(l1[0], lse[b])
+
+
+# ---- random geometries -------------------------------------------------------
+
+from hypothesis import HealthCheck, given, settings
+from hypothesis import strategies as st
+
+
+@st.composite
+def geometries(draw):
+    Z, Y, X = (draw(st.integers(1, 5)) for _ in range(3))
+    window = tuple(draw(st.sampled_from((1, 3, 5))) for _ in range(3))
+    block = tuple(draw(st.integers(1, 4)) for _ in range(3))
+    V = Z * Y * X
+    n = draw(st.integers(1, V))
+    return dict(B=draw(st.integers(1, 2)), H=draw(st.integers(1, 2)),
+                d=draw(st.sampled_from((6, 12))), Z=Z, Y=Y, X=X, window=window, block=block,
+                n_tokens=0 if n == V else n), draw(st.integers(0, 2**16)), draw(st.booleans())
+
+
+@settings(max_examples=40, deadline=None, derandomize=True,
+          suppress_health_check=[HealthCheck.too_slow, HealthCheck.function_scoped_fixture])
+@given(geometries())
+def test_random_geometries_against_brute_force(oracle_lib, case):
+    """Random small volumes, windows, block extents (dividing or not) and
+    occupancies, with and without summaries, against brute_force."""
+    cfg, seed, window_only = case
+    s = shape(**cfg)
+    if s.n_tokens:
+        packed, coords = partial_inputs(s, seed)
+    else:
+        packed, coords, _ = rand_inputs(s, seed=seed)
+    out, lse = oracle.forward(s, coords, packed["q"], packed["k"], packed["v"],
+                              window_only=window_only)
+    for b in range(s.B):
+        ro, rl = brute_force(s, packed, coords, b, window_only)
+        np.testing.assert_allclose(out[b], ro, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse[b], rl, rtol=0, atol=1e-12)
