@@ -16,6 +16,8 @@ from types import SimpleNamespace
 import numpy as np
 import pytest
 import torch
+from hypothesis import HealthCheck, given, settings
+from hypothesis import strategies as st
 
 import oracle
 from local_global_attention_b200 import inputs as I
@@ -641,10 +643,6 @@ def test_batch_items_are_independent(oracle_lib):
 
 
 # ---- random geometries -------------------------------------------------------
-
-from hypothesis import HealthCheck, given, settings
-from hypothesis import strategies as st
-
 
 @st.composite
 def geometries(draw):
