@@ -153,3 +153,21 @@ def test_backward_workspace_layout(lib):
     ns = 4 * wl.B * wl.H * wl.n_blocks * wl.d
     assert lib.pack3d_backward_workspace_bytes(ctypes.byref(P.make_params(wl))) == \
         a256(4 * wl.B * wl.H * wl.N) + 4 * a256(ns)
+
+
+def test_size_limits(lib):
+    """The header's limits: extents up to 32767 per axis and
+    B * N * H * head_dim below 2^31 (32-bit element offsets); beyond them the
+    shape is rejected before anything is sized or launched."""
+    ok = shape(B=1, H=1, d=96, Z=1, Y=1, X=32767, window=(1, 1, 1), block=(1, 1, 1))
+    assert lib.pack3d_index_bytes(ctypes.byref(P.make_params(ok))) > 0
+    for bad in (dict(X=32768), dict(Z=-1)):
+        s = shape(B=1, H=1, d=96, Z=1, Y=1, X=32767, window=(1, 1, 1), block=(1, 1, 1))
+        s.__dict__.update(bad)
+        assert lib.pack3d_index_bytes(ctypes.byref(P.make_params(s))) == 0, bad
+    # 3 x 8 heads x 2^20 tokens x 96 = 1.125 * 2^31 elements: too many
+    big = shape(B=3, H=8, d=96, Z=64, Y=128, X=128, window=(5, 7, 7), block=(4, 16, 16))
+    assert lib.pack3d_index_bytes(ctypes.byref(P.make_params(big))) == 0
+    # two items fit (0.75 * 2^31)
+    fits = shape(B=2, H=8, d=96, Z=64, Y=128, X=128, window=(5, 7, 7), block=(4, 16, 16))
+    assert lib.pack3d_index_bytes(ctypes.byref(P.make_params(fits))) > 0
