@@ -97,3 +97,33 @@ def test_reference_arm_line_on_rank_zero(monkeypatch):
     assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1
     assert line["e2e"] == {"value": line["value"], "unit": bench.UNIT,
                            "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_algorithmic_work_counts_terms_by_enumeration():
+    """The roofline's numerator: bench.algorithmic_work's local and summary
+    term counts (per-axis closed forms) against a direct enumeration over
+    every query voxel, its clipped window and every block box."""
+    import itertools
+
+    import numpy as np
+
+    import bench
+    from local_global_attention_b200 import inputs as I
+    wl = I.Workload(name="enum", B=1, H=1, d=12, Z=5, Y=7, X=9, window=(3, 5, 3),
+                    block=(5, 7, 3))
+    r = [(w - 1) // 2 for w in wl.window]
+    dims = (wl.Z, wl.Y, wl.X)
+    nbs = [n // b for n, b in zip(dims, wl.block)]
+    local = summ = 0
+    for c in itertools.product(*(range(n) for n in dims)):
+        lo = [max(c[a] - r[a], 0) for a in range(3)]
+        hi = [min(c[a] + r[a], dims[a] - 1) for a in range(3)]
+        local += int(np.prod([hi[a] - lo[a] + 1 for a in range(3)]))
+        for B in itertools.product(*(range(n) for n in nbs)):
+            meets = all(B[a] * wl.block[a] <= hi[a] and (B[a] + 1) * wl.block[a] - 1 >= lo[a]
+                        for a in range(3))
+            summ += 0 if meets else 1
+    w = bench.algorithmic_work(wl)
+    assert w["local_flop"] == 4 * wl.d * local
+    assert w["summary_flop"] == 4 * wl.d * summ
+    assert w["bwd_flop"] == 10 * wl.d * (local + summ)
