@@ -40,7 +40,6 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "forward_tc_vol_32x32x64.md")
 TC_SOURCE = os.path.join(ROOT, "local_global_attention_b200", "csrc", "attn_tc.cu")
 FP32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # CUDA-core fp32 FMA peak, nominal
-KERNELS_PER_STEP = 10  # index build 8 (plus two memsets), summaries + staging 1, attention 1
 
 
 def peaks():
@@ -91,21 +90,6 @@ def algorithmic_work(wl):
             "bwd_flop": BH * per_bh_bwd,
             "flop": BH * (per_bh_local + per_bh_sum), "hbm_bytes": hbm,
             "fwd_bytes": rows * esz * 4 + wl.B * wl.H * wl.N * 4}
-
-
-def profile_traffic():
-    """DRAM bytes per forward launch from the committed ncu summary, if it was
-    taken on the current kernel source; else None."""
-    try:
-        text = open(PROFILE_SUMMARY).read()
-    except OSError:
-        return None
-    m_sha = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
-    m_tr = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    if not (m_sha and m_tr):
-        return None
-    sha = hashlib.sha256(open(TC_SOURCE, "rb").read()).hexdigest()
-    return float(m_tr.group(1)) if sha == m_sha.group(1) else None
 
 
 class ClockSampler:
@@ -227,7 +211,180 @@ def run_config(wl, packing, world):
     }
 
 
+class Runner:
+    """One workload on this GPU: its inputs in HBM, index, workspace and the
+    calls of one step, made through the C ABI (ctypes) on one stream."""
+
+    def __init__(self, wl, inp, packed_rope=False):
+        import ctypes
+
+        import torch
+
+        from local_global_attention_b200 import pack3d as P
+        self.torch, self.ctypes, self.P = torch, ctypes, P
+        self.wl = wl
+        self.dev = {k: v.cuda() for k, v in inp.items() if k != "order"}
+        self.params = P.make_params(wl)
+        if packed_rope:
+            self.params.rope_mode = P.ROPE_PACKED
+        self.idx = P.IndexBuffers(self.params)
+        B, N, H, d = wl.B, wl.N, wl.H, wl.d
+        self.ksum = torch.empty(B, H, wl.n_blocks, d, dtype=torch.float32, device="cuda")
+        self.vsum = torch.empty_like(self.ksum)
+        self.out = torch.empty_like(self.dev["q"])
+        self.lse = torch.empty(B, H, N, dtype=torch.float32, device="cuda")
+        self.ws_bytes = P.pack3d_forward_workspace_bytes(self.params)
+        self.ws = torch.empty(max(self.ws_bytes, 1), dtype=torch.uint8, device="cuda")
+        self.stream = torch.cuda.current_stream()
+        self.lib = P.load()
+        self.sp = ctypes.c_void_p(self.stream.cuda_stream)
+        self.pp, self.ip = ctypes.byref(self.params), ctypes.byref(self.idx.struct)
+        self.phase_events = []
+
+    def ptr(self, t):
+        return self.ctypes.c_void_p(t.data_ptr())
+
+    def event(self):
+        e = self.torch.cuda.Event(enable_timing=True)
+        e.record(self.stream)
+        return e
+
+    def step(self, window=False, record=False, bufs=None, res=None):
+        """Index build; block summaries computed in the pass that stages the
+        rotated keys and the values in grid order (pack3d_stage_kv); the
+        attention (pack3d_forward_staged).  With record, CUDA events between
+        the three phases."""
+        c_size = self.ctypes.c_size_t
+        d_ = self.dev if bufs is None else bufs
+        o_, l_ = (self.out, self.lse) if res is None else res
+        ev = [self.event()] if record else None
+        rc = self.lib.pack3d_build_index(self.pp, self.ptr(d_["coords"]), self.ip, self.sp)
+        if record:
+            ev.append(self.event())
+        rc |= self.lib.pack3d_stage_kv(self.pp, self.ip, self.ptr(d_["k"]), self.ptr(d_["v"]),
+                                       None if window else self.ptr(self.ksum),
+                                       None if window else self.ptr(self.vsum),
+                                       self.ptr(self.ws), c_size(self.ws_bytes), self.sp)
+        if record:
+            ev.append(self.event())
+        rc |= self.lib.pack3d_forward_staged(self.pp, self.ip, self.ptr(d_["q"]),
+                                             self.ptr(self.ws), c_size(self.ws_bytes),
+                                             0 if window else 1, self.ptr(o_), self.ptr(l_),
+                                             self.sp)
+        if record:
+            ev.append(self.event())
+            self.phase_events.append(ev)
+        if rc:
+            raise RuntimeError(f"pack3d call failed: {rc}")
+
+    def phase_ms(self):
+        """Mean ms of (index build, staging + summaries, attention) over the
+        recorded steps."""
+        ev = self.phase_events
+        return [statistics.mean(e[i].elapsed_time(e[i + 1]) for e in ev) for i in range(3)]
+
+    def timed(self, steps, warmup, world, window=False, record=False):
+        """ms per step over `steps` timed steps (barrier + synchronize on both
+        sides, CUDA events on the launching stream, max over ranks) and the
+        number of library kernels launched in the timed region."""
+        torch = self.torch
+        self.phase_events = []
+        for _ in range(warmup):
+            self.step(window=window)
+        torch.cuda.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
+        n0 = self.P.pack3d_kernel_launches()
+        t0 = self.event()
+        for _ in range(steps):
+            self.step(window=window, record=record)
+        t1 = self.event()
+        n1 = self.P.pack3d_kernel_launches()
+        torch.cuda.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
+        st = self.P.pack3d_index_check(self.idx)
+        if st != self.P.OK:
+            raise RuntimeError(f"index status {self.P.strerror(st)}")
+        return max_over_ranks(t0.elapsed_time(t1) / steps, world), n1 - n0
+
+    def time_calls(self, fn, calls, warmup=3):
+        """Mean ms of fn() over `calls` back-to-back calls (CUDA events)."""
+        for _ in range(warmup):
+            fn()
+        self.torch.cuda.synchronize()
+        t0 = self.event()
+        for _ in range(calls):
+            fn()
+        t1 = self.event()
+        self.torch.cuda.synchronize()
+        return t0.elapsed_time(t1) / calls
+
+    def block_summaries(self):
+        rc = self.lib.pack3d_block_summaries(self.pp, self.ip, self.ptr(self.dev["k"]),
+                                             self.ptr(self.dev["v"]), self.ptr(self.ksum),
+                                             self.ptr(self.vsum), self.sp)
+        if rc:
+            raise RuntimeError(f"pack3d_block_summaries failed: {rc}")
+
+
+def profile_value(key):
+    """A figure from the committed ncu summary of the attention kernel, if it
+    was taken on the current kernel source; else None."""
+    try:
+        text = open(PROFILE_SUMMARY).read()
+    except OSError:
+        return None
+    m_sha = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
+    m = re.search(key + r":\s*([0-9.eE+]+)", text)
+    if not (m_sha and m):
+        return None
+    sha = hashlib.sha256(open(TC_SOURCE, "rb").read()).hexdigest()
+    return float(m.group(1)) if sha == m_sha.group(1) else None
+
+
+def micro1m_line(args, pk):
+    """The 1,048,576-token microscopy-shaped workload (smooth field, block
+    packing): PACK3D step and window-only step, with the attention kernel's
+    useful FLOP rate.  Its summary term (1,024 blocks) dwarfs the local one."""
+    import torch
+
+    from local_global_attention_b200 import configs as C
+    from local_global_attention_b200 import inputs as I
+    wl = C.MICRO1M
+    t_gen = time.perf_counter()
+    inp = I.make_inputs(wl, "block", grid=I.grid_tensors(wl, device="cuda"))
+    t_gen = time.perf_counter() - t_gen
+    r = Runner(wl, inp)
+    steps = max(3, min(args.steps, 20))
+    ms, launches = r.timed(steps, args.warmup, 1, record=True)
+    idx_ms, stage_ms, attn_ms = r.phase_ms()
+    wms, _ = r.timed(steps, args.warmup, 1, window=True, record=True)
+    w_attn = r.phase_ms()[2]
+    work = algorithmic_work(wl)
+    tf = work["flop"] / (attn_ms * 1e-3) / 1e12
+    res = {
+        "workload": f"{wl.name}: {wl.N} tokens x batch {wl.B}, {wl.H} heads, head_dim {wl.d}, "
+                    f"window {'x'.join(map(str, wl.window))}, blocks "
+                    f"{'x'.join(map(str, wl.block))} ({wl.n_blocks} summaries), block packing, "
+                    "smooth random field",
+        "ms_per_step": ms, "value": wl.B * wl.N / (ms * 1e-3), "unit": UNIT, "steps": steps,
+        "phases_ms": {"index": idx_ms, "stage_and_summaries": stage_ms, "attention": attn_ms},
+        "attention_tflops_useful": tf, "attention_frac_of_burst_peak": tf / pk["bf16_tflops"],
+        "local_flop": work["local_flop"], "summary_flop": work["summary_flop"],
+        "window_only": {"ms_per_step": wms, "attention_ms": w_attn,
+                        "pack3d_over_window": ms / wms},
+        "gpu_launches_per_step": launches / steps,
+        "input_generation_s": t_gen,
+    }
+    del r, inp
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args):
+    import ctypes
+
     import torch
 
     from local_global_attention_b200 import inputs as I
@@ -237,126 +394,70 @@ def run_ours(args):
     wl = workload(args.workload)
     wl_r = rank_workload(wl, rank)
     inp = I.make_inputs(wl_r, args.packing)
-    dev = {k: v.cuda() for k, v in inp.items() if k != "order"}
-    params = P.make_params(wl_r)
-    idx = P.IndexBuffers(params)
+    r = Runner(wl_r, inp)
     B, N, H, d = wl.B, wl.N, wl.H, wl.d
-    nb = wl.n_blocks
-    ksum = torch.empty(B, H, nb, d, dtype=torch.float32, device="cuda")
-    vsum = torch.empty_like(ksum)
-    out = torch.empty_like(dev["q"])
-    lse = torch.empty(B, H, N, dtype=torch.float32, device="cuda")
-    ws_bytes = P.pack3d_forward_workspace_bytes(params)
-    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device="cuda")
-    stream = torch.cuda.current_stream()
-    lib = P.load()
-    import ctypes
-    sp = ctypes.c_void_p(stream.cuda_stream)
-    pp_ax, ip_ax = ctypes.byref(params), ctypes.byref(idx.struct)
-    ptr = lambda t: ctypes.c_void_p(t.data_ptr())
-
-    fwd_events = []
-
-    # the packed-sequence comparison mode (1-D RoPE on the packed index): its own
-    # params and index (the rotation table differs), the same step
-    params_pk = P.make_params(wl_r)
-    params_pk.rope_mode = P.ROPE_PACKED
-    idx_pk = P.IndexBuffers(params_pk)
-    pp_pk, ip_pk = ctypes.byref(params_pk), ctypes.byref(idx_pk.struct)
-
-    def step(record=False, window=False, bufs=None, res=None, packed_rope=False):
-        # index build; block summaries computed in the pass that stages the
-        # rotated keys and the values in grid order (pack3d_stage_kv); the
-        # attention (pack3d_forward_staged), timed on its own
-        d_ = dev if bufs is None else bufs
-        o_, l_ = (out, lse) if res is None else res
-        pp, ip = (pp_pk, ip_pk) if packed_rope else (pp_ax, ip_ax)
-        rc = lib.pack3d_build_index(pp, ptr(d_["coords"]), ip, sp)
-        rc |= lib.pack3d_stage_kv(pp, ip, ptr(d_["k"]), ptr(d_["v"]),
-                                  None if window else ptr(ksum), None if window else ptr(vsum),
-                                  ptr(ws), ctypes.c_size_t(ws_bytes), sp)
-        if record:
-            e0 = torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-        rc |= lib.pack3d_forward_staged(pp, ip, ptr(d_["q"]), ptr(ws), ctypes.c_size_t(ws_bytes),
-                                        0 if window else 1, ptr(o_), ptr(l_), sp)
-        if record:
-            e1 = torch.cuda.Event(enable_timing=True)
-            e1.record(stream)
-            fwd_events.append((e0, e1))
-        if rc:
-            raise RuntimeError(f"pack3d call failed: {rc}")
-
-    def timed(window=False, record=False, packed_rope=False):
-        for _ in range(args.warmup):
-            step(window=window, packed_rope=packed_rope)
-        torch.cuda.synchronize()
-        barrier(world)
-        torch.cuda.synchronize()
-        t0 = torch.cuda.Event(enable_timing=True)
-        t1 = torch.cuda.Event(enable_timing=True)
-        t0.record(stream)
-        for _ in range(args.steps):
-            step(record=record, window=window, packed_rope=packed_rope)
-        t1.record(stream)
-        torch.cuda.synchronize()
-        barrier(world)
-        torch.cuda.synchronize()
-        return max_over_ranks(t0.elapsed_time(t1) / args.steps, world)
 
     with ClockSampler(local) as clk:
-        ms = timed(record=True)
-    st = P.pack3d_index_check(idx)
-    if st != P.OK:
-        raise RuntimeError(f"index status {P.strerror(st)}")
-    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in fwd_events)
-    window_ms = timed(window=True)
-    packed_ms = timed(packed_rope=True)
+        ms, launches = r.timed(args.steps, args.warmup, world, record=True)
+    idx_ms, stage_ms, fwd_ms = r.phase_ms()
+    pk, pk_src = peaks()
+    work = algorithmic_work(wl)
+    tokens = B * N * world
+    if args.only == "forward":
+        # the forward step alone, then three pack3d_block_summaries calls (a
+        # short run for profilers); one line, no extras
+        for _ in range(3):
+            r.block_summaries()
+        torch.cuda.synchronize()
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "value": whole_job_rate(B * N, world, ms),
+                              "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                              "ms_per_step": ms, "only": "forward"}), flush=True)
+        return
+
+    window_ms, _ = r.timed(args.steps, args.warmup, world, window=True)
+    # the packed-sequence comparison mode (1-D RoPE on the packed index): its own
+    # params and index (the rotation table differs), the same step
+    r_pk = Runner(wl_r, inp, packed_rope=True)
+    packed_ms, _ = r_pk.timed(args.steps, args.warmup, world)
+    del r_pk
+    # pack3d_block_summaries alone (HBM-bound: k and v read once)
+    sum_ms = r.time_calls(r.block_summaries, 20)
 
     # the backward (dq, dk, dv from the forward's out and lse) at the same shape,
-    # with dO ~ N(0, 1): CUDA cores, fp32 arithmetic
+    # with dO ~ N(0, 1)
     g_do = torch.Generator().manual_seed(wl_r.seed + 7)
-    dout = torch.randn(B, N, H, d, generator=g_do).to(dev["q"].dtype).cuda()
-    dq, dk, dv = (torch.empty_like(dev["q"]) for _ in range(3))
-    bws_bytes = P.pack3d_backward_workspace_bytes(params)
+    dout = torch.randn(B, N, H, d, generator=g_do).to(r.dev["q"].dtype).cuda()
+    dq, dk, dv = (torch.empty_like(r.dev["q"]) for _ in range(3))
+    bws_bytes = P.pack3d_backward_workspace_bytes(r.params)
     bws = torch.empty(max(bws_bytes, 1), dtype=torch.uint8, device="cuda")
-    step()  # the forward the backward reads
+    r.step()  # the forward the backward reads
+    ptr = r.ptr
 
     def backward():
-        rc = lib.pack3d_backward(pp_ax, ip_ax, ptr(dev["q"]), ptr(dev["k"]), ptr(dev["v"]),
-                                 ptr(out), ptr(lse), ptr(dout), ptr(dq), ptr(dk), ptr(dv),
-                                 ptr(bws), ctypes.c_size_t(bws_bytes), sp)
+        rc = r.lib.pack3d_backward(r.pp, r.ip, ptr(r.dev["q"]), ptr(r.dev["k"]), ptr(r.dev["v"]),
+                                   ptr(r.out), ptr(r.lse), ptr(dout), ptr(dq), ptr(dk), ptr(dv),
+                                   ptr(bws), ctypes.c_size_t(bws_bytes), r.sp)
         if rc:
             raise RuntimeError(f"pack3d_backward failed: {rc}")
 
     bw_steps = max(3, min(args.steps, 20))
-    for _ in range(3):
-        backward()
-    torch.cuda.synchronize()
-    b0 = torch.cuda.Event(enable_timing=True)
-    b1 = torch.cuda.Event(enable_timing=True)
-    b0.record(stream)
-    for _ in range(bw_steps):
-        backward()
-    b1.record(stream)
-    torch.cuda.synchronize()
-    bwd_ms = max_over_ranks(b0.elapsed_time(b1) / bw_steps, world)
-    if P.pack3d_index_check(idx) != P.OK:
+    bwd_ms = max_over_ranks(r.time_calls(backward, bw_steps), world)
+    if P.pack3d_index_check(r.idx) != P.OK:
         raise RuntimeError("index status after the backward")
-    if P.pack3d_index_check(idx_pk) != P.OK:
-        raise RuntimeError("index status of the packed-RoPE run")
 
     # End to end through the C ABI: every step copies its inputs from pinned
     # host memory and reads its outputs back.  Two device buffer sets and two
     # copy streams let step i's upload, step i-1's compute and step i-2's
     # download overlap (PCIe is full duplex); every byte of every step is still
     # copied inside the timed region.
+    stream = r.stream
     names = ("coords", "q", "k", "v")
     host = {k: inp[k].pin_memory() for k in names}
-    sets = [dev, {k: torch.empty_like(dev[k]) for k in names}]
-    results = [(out, lse), (torch.empty_like(out), torch.empty_like(lse))]
-    host_res = [(torch.empty(out.shape, dtype=out.dtype).pin_memory(),
-                 torch.empty(lse.shape, dtype=lse.dtype).pin_memory()) for _ in range(2)]
+    sets = [r.dev, {k: torch.empty_like(r.dev[k]) for k in names}]
+    results = [(r.out, r.lse), (torch.empty_like(r.out), torch.empty_like(r.lse))]
+    host_res = [(torch.empty(r.out.shape, dtype=r.out.dtype).pin_memory(),
+                 torch.empty(r.lse.shape, dtype=r.lse.dtype).pin_memory()) for _ in range(2)]
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
     computed = [None, None]  # compute of the last step on buffer set b done
     drained = [None, None]   # download of the last step on buffer set b done
@@ -373,7 +474,7 @@ def run_ours(args):
         stream.wait_event(ready)
         if drained[b] is not None:
             stream.wait_event(drained[b])
-        step(bufs=sets[b], res=results[b])
+        r.step(bufs=sets[b], res=results[b])
         ev = torch.cuda.Event()
         ev.record(stream)
         computed[b] = ev
@@ -402,16 +503,19 @@ def run_ours(args):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
     h2d = sum(host[k_].numel() * host[k_].element_size() for k_ in host)
     d2h = sum(t.numel() * t.element_size() for t in host_res[0])
+    del sets, results, host_res, host
+
+    micro = None
+    if args.micro1m and world == 1:
+        micro = micro1m_line(args, pk)
 
     if rank != 0:
         barrier(world)
         return
-    pk, pk_src = peaks()
-    work = algorithmic_work(wl)
-    tokens = B * N * world
-    achieved_tflops = work["flop"] / (fwd_ms * 1e-3) / 1e12
-    peak_tf = pk["bf16_tflops_sustained"]
-    traffic = profile_traffic()
+    achieved = work["flop"] / (fwd_ms * 1e-3) / 1e12
+    local_achieved = work["local_flop"] / (fwd_ms * 1e-3) / 1e12
+    peak_tf = pk["bf16_tflops"]
+    stage_bytes = work["fwd_bytes"] - wl.B * wl.H * wl.N * 4  # k, v read + grid copies written
     line = {
         "metric": METRIC,
         "value": whole_job_rate(B * N, world, ms),
@@ -426,19 +530,38 @@ def run_ours(args):
         "dtype": "bf16",
         "data": "synthetic (seeded N(0,1)/sqrt(96) q, k, v; random packing)",
         "config": run_config(wl, args.packing, world),
-        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "gpu_launches": launches,
+        "gpu_launches_note": "library kernel launches issued inside the timed region "
+                             "(pack3d_kernel_launches before and after)",
         "roofline": {
             "bound": "tensor",
             "kernel": "k_forward_tc (local window + summaries, tcgen05)",
-            "achieved": achieved_tflops,
+            "achieved": achieved,
             "peak": peak_tf,
             "unit": "TFLOP/s",
-            "frac": achieved_tflops / peak_tf,
-            "peak_source": f"{pk_src} bf16_tflops_sustained",
-            "traffic": traffic,
+            "frac": achieved / peak_tf,
+            "peak_source": f"{pk_src} bf16_tflops (burst: a ~1 ms kernel timed alone)",
+            "local_frac": local_achieved / peak_tf,
+            "local_note": "local-window FLOPs only (the summary terms left out)",
+            "tensor_pipe_active_pct_ncu": profile_value("tensor_pipe_active_pct"),
+            "traffic": profile_value("dram_bytes_per_launch"),
             "algorithmic_flop_per_launch": work["flop"],
             "forward_ms": fwd_ms,
             "forward_hbm_frac": (work["fwd_bytes"] / (fwd_ms * 1e-3) / 1e9) / pk["hbm_gbs"],
+        },
+        "memory_bound": {
+            "unit": "GB/s", "peak": pk["hbm_gbs"], "peak_source": f"{pk_src} hbm_gbs (copy)",
+            "stage_and_summaries": {
+                "kernel": "k_summaries_bulk<1>", "ms": stage_ms,
+                "algorithmic_bytes": stage_bytes,
+                "achieved": stage_bytes / (stage_ms * 1e-3) / 1e9,
+                "frac": stage_bytes / (stage_ms * 1e-3) / 1e9 / pk["hbm_gbs"]},
+            "block_summaries": {
+                "kernel": "k_summaries_bulk<0> (pack3d_block_summaries)", "ms": sum_ms,
+                "algorithmic_bytes": stage_bytes / 2,
+                "achieved": stage_bytes / 2 / (sum_ms * 1e-3) / 1e9,
+                "frac": stage_bytes / 2 / (sum_ms * 1e-3) / 1e9 / pk["hbm_gbs"]},
+            "index_build_ms": idx_ms,
         },
         "backward": {
             "ms_per_call": bwd_ms,
@@ -460,6 +583,8 @@ def run_ours(args):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "clocks": clk.summary(),
     }
+    if micro is not None:
+        line["micro1m"] = micro
     if not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(wl, inp, args.cpu_sample)
     barrier(world)
@@ -547,6 +672,11 @@ def main():
     ap.add_argument("--cpu-sample", type=int, default=32768,
                     help="query tokens the CPU oracle computes for the baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", default="all", choices=["all", "forward"],
+                    help="forward: time the forward step alone and print a short line "
+                         "(for profiler runs)")
+    ap.add_argument("--no-micro1m", dest="micro1m", action="store_false",
+                    help="skip the 1M-token workload section")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -32,7 +32,9 @@
  *     (a dense volume); each batch item may use its own packing.
  *
  * Memory: every buffer is allocated and owned by the caller; the library
- * never allocates or frees device memory and keeps no global state.  All
+ * never allocates or frees device memory.  Its only global state is a count of
+ * the kernels it has launched (pack3d_kernel_launches) and the static scratch
+ * array of pack3d_backward_noalloc.  All
  * pointers except the params and index structs are DEVICE pointers.  Layouts:
  *   q, k, v, out, dout, dq, dk, dv : [B][N][H][head_dim], packed order,
  *                                    bf16 (dtype PACK3D_BF16) or fp32
@@ -246,9 +248,10 @@ PACK3D_API int pack3d_backward(const pack3d_params* p, const pack3d_index* idx, 
  *
  * The workspace lives in a static device array of
  * PACK3D_NOALLOC_SCRATCH_BYTES (32 MiB) inside this library; every GPU on
- * which the library is used holds that array until the process exits.  The
- * first call on a device looks up the array's device address with that device
- * current (cudaGetSymbolAddress); make that first call before any stream
+ * which the library is used holds that array until the process exits.  Every
+ * call looks up the array's device address on the current device
+ * (cudaGetSymbolAddress); on the first call on a device that lookup also loads
+ * the library's device code there, so make that first call before any stream
  * capture.  Shapes whose workspace (pack3d_backward_workspace_bytes) exceeds
  * the array are rejected with PACK3D_ERR_UNSUPPORTED before anything is
  * launched (the 65k-token, 8-head training shape needs 20.5 MiB).  Nothing is
@@ -260,6 +263,13 @@ PACK3D_API int pack3d_backward_noalloc(const pack3d_params* p, const pack3d_inde
                                        const void* q, const void* k, const void* v,
                                        const void* out, const float* lse, const void* dout,
                                        void* dq, void* dk, void* dv, pack3d_stream_t stream);
+
+/* Number of kernels this library has launched in this process, over every
+ * call, device and stream (a host-side counter, incremented when a launch is
+ * issued; no CUDA call).  The difference of two readings counts the launches
+ * of the calls made in between, e.g. inside a timed region.  No counterpart in
+ * the paper: an instrumentation aid. */
+PACK3D_API uint64_t pack3d_kernel_launches(void);
 
 /* Human-readable text of a status code (static storage). */
 PACK3D_API const char* pack3d_strerror(int status);

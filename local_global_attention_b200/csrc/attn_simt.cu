@@ -1040,6 +1040,7 @@ int forward_launch(const Geo& g, const pack3d_index* idx, const void* q, const v
   else
     k_forward_simt<T, TO, D, false><<<grid, block, 0, s>>>(
         g, *idx, (const T*)q, (const T*)k, (const T*)v, ksum, vsum, (TO*)out, lse);
+  count_launches(1);
   return cuda_status(cudaGetLastError());
 }
 
@@ -1113,6 +1114,7 @@ int backward_typed(const Geo& g, const pack3d_index* idx, const void* q, const v
   else
     k_bwd_delta<T, T><<<(unsigned)((rows + 255) / 256), 256, 0, s>>>(
         g, idx->err, (const T*)out, (const T*)dout, w.delta);
+  count_launches(1);
   int rc = launch_block_summaries(g, idx, k, v, w.ksum, w.vsum, s);
   if (rc) return rc;
   if constexpr (D == 96) {
@@ -1132,13 +1134,13 @@ int backward_typed(const Geo& g, const pack3d_index* idx, const void* q, const v
     const int64_t per = (int64_t)g.B * g.H * g.nb * g.d;
     k_bwd_summary_reduce<<<(unsigned)((per + 255) / 256), 256, 0, s>>>(g, idx->err, nsplit,
                                                                        w.part, w.dks, w.dvs);
+    count_launches(2);
   } else {
     dim3 sgrid((g.nb + BC - 1) / BC, g.B, g.H);
     k_bwd_summary<T, D><<<sgrid, 256, 0, s>>>(g, *idx, (const T*)q, (const T*)dout, lse,
                                               w.delta, w.ksum, w.vsum, w.dks, w.dvs);
+    count_launches(1);
   }
-  // one halo row must fit in a staged chunk
-  if (TX + 2 * g.rx > CAPK) return PACK3D_ERR_UNSUPPORTED;
   const size_t dyn = 2 * (size_t)CAPK * D * sizeof(float);
   {
     cudaError_t e = cudaFuncSetAttribute(k_bwd_dq<T, D, true>,
@@ -1156,6 +1158,7 @@ int backward_typed(const Geo& g, const pack3d_index* idx, const void* q, const v
   k_bwd_dkdv<T, D, true><<<grid, block, dyn, s>>>(g, *idx, (const T*)q, (const T*)k,
                                                   (const T*)v, (const T*)dout, lse, w.delta,
                                                   w.dks, w.dvs, (T*)dk, (T*)dv);
+  count_launches(2);
   return cuda_status(cudaGetLastError());
 }
 
@@ -1180,6 +1183,12 @@ int launch_forward_simt(const Geo& g, const pack3d_index* idx, const void* q, co
   if (g.dtype == PACK3D_BF16)
     return forward_dispatch<__nv_bfloat16>(g, idx, q, k, v, ksum, vsum, out, lse, summaries, s);
   return forward_dispatch<float>(g, idx, q, k, v, ksum, vsum, out, lse, summaries, s);
+}
+
+int backward_supported(const Geo& g) {
+  // one halo row (the tile's 8 columns widened by the window radius on both
+  // sides, clipped to the volume) must fit in a staged chunk
+  return std::min(g.X, TX + 2 * g.rx) <= CAPK ? PACK3D_OK : PACK3D_ERR_UNSUPPORTED;
 }
 
 size_t backward_workspace_bytes(const Geo& g) {

@@ -838,6 +838,7 @@ int launch_stage_kv(const Geo& g, const pack3d_index* idx, const void* k, const 
     k_grid_kv<<<ggrid, 256, 0, s>>>(g, *idx, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
                                     reinterpret_cast<__nv_bfloat16*>(base + w.kg),
                                     reinterpret_cast<__nv_bfloat16*>(base + w.vg));
+    count_launches(1);
   } else if (rc) {
     return rc;
   }
@@ -847,6 +848,7 @@ int launch_stage_kv(const Geo& g, const pack3d_index* idx, const void* k, const 
     k_summaries_bf16<<<blocks, 256, 0, s>>>((const float4*)ksum, (const float4*)vsum,
                                             reinterpret_cast<uint2*>(base + w.ks),
                                             reinterpret_cast<uint2*>(base + w.vs), n4, idx->err);
+    count_launches(1);
   }
   return cuda_status(cudaGetLastError());
 }
@@ -875,6 +877,7 @@ int launch_attention_tc(const Geo& g, const pack3d_index* idx, const void* q, vo
                            (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess)
     return PACK3D_ERR_CUDA;
   kern<<<grid, NTHREADS, SMEM_REQUEST, s>>>(g, *idx, (const __nv_bfloat16*)q, maps, out, lse);
+  count_launches(1);
   return cuda_status(cudaGetLastError());
 }
 

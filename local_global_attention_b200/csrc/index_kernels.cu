@@ -181,6 +181,7 @@ int launch_build_index(const Geo& g, const int16_t* coords, const pack3d_index* 
       (g.rope_mode == PACK3D_ROPE_PACKED ? (int64_t)g.N : (int64_t)(g.Z + g.Y + g.X)) *
       g.rope_len;
   k_rope_table<<<(unsigned)((entries + 255) / 256), 256, 0, s>>>(g, rope_base, idx->rope);
+  count_launches(8);
   return cuda_status(cudaGetLastError());
 }
 

@@ -4,9 +4,17 @@
 #include <math.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "pack3d_internal.cuh"
 
 namespace p3d {
+
+namespace {
+std::atomic<uint64_t> g_kernel_launches{0};
+}
+
+void count_launches(int n) { g_kernel_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 
 int64_t halo_axis_total(int extent, int tile, int r) {
   int64_t s = 0;
@@ -270,9 +278,12 @@ int pack3d_backward(const pack3d_params* p, const pack3d_index* idx, const void*
     return PACK3D_ERR_ARG;
   if (((uintptr_t)workspace & 255) || workspace_bytes < backward_workspace_bytes(g))
     return PACK3D_ERR_ARG;
+  if ((rc = backward_supported(g))) return rc;
   return launch_backward(g, idx, q, k, v, out, lse, dout, dq, dk, dv, workspace,
                          (cudaStream_t)stream);
 }
+
+uint64_t pack3d_kernel_launches(void) { return g_kernel_launches.load(std::memory_order_relaxed); }
 
 const char* pack3d_strerror(int status) {
   switch (status) {

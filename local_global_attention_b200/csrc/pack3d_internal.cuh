@@ -129,11 +129,18 @@ int launch_stage_kv(const Geo& g, const pack3d_index* idx, const void* k, const 
                     cudaStream_t s);
 int launch_attention_tc(const Geo& g, const pack3d_index* idx, const void* q, void* ws,
                         void* out, float* lse, bool summaries, cudaStream_t s);
+// PACK3D_OK when the backward kernels are built for this shape, else
+// PACK3D_ERR_UNSUPPORTED (checked before anything is launched).
+int backward_supported(const Geo& g);
 size_t backward_workspace_bytes(const Geo& g);
 int launch_backward(const Geo& g, const pack3d_index* idx, const void* q, const void* k,
                     const void* v, const void* out, const float* lse, const void* dout, void* dq,
                     void* dk, void* dv, void* workspace, cudaStream_t s);
 
 inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? PACK3D_OK : PACK3D_ERR_CUDA; }
+
+// Adds n to the process-wide count of kernel launches this library has issued
+// (read by pack3d_kernel_launches); every launcher calls it for its kernels.
+void count_launches(int n);
 
 }  // namespace p3d

@@ -521,6 +521,7 @@ int launch_bulk(const Geo& g, const pack3d_index* idx, const void* k, const void
   kern<<<dim3(g.nb, g.B), BS_THREADS, smem, s>>>(g, idx->vol, idx->rope, idx->err,
                                                   (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
                                                   ksum, vsum, so);
+  count_launches(1);
   return cuda_status(cudaGetLastError());
 }
 
@@ -533,6 +534,7 @@ int launch_block_summaries(const Geo& g, const pack3d_index* idx, const void* k,
     k_block_summaries_bf16_d96<false><<<grid96, TG96 * LANES96, 0, s>>>(
         g, idx->vol, idx->rope, idx->err, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, ksum,
         vsum, StageOut{});
+    count_launches(1);
     return cuda_status(cudaGetLastError());
   }
   int threads = TG * (g.d / 4);
@@ -545,6 +547,7 @@ int launch_block_summaries(const Geo& g, const pack3d_index* idx, const void* k,
     k_block_summaries<float><<<grid, threads, smem, s>>>(g, idx->vol, idx->rope, idx->err,
                                                          (const float*)k, (const float*)v, ksum,
                                                          vsum);
+  count_launches(1);
   return cuda_status(cudaGetLastError());
 }
 
@@ -565,6 +568,7 @@ int launch_block_summaries_staged(const Geo& g, const pack3d_index* idx, const v
   k_block_summaries_bf16_d96<true><<<grid96, TG96 * LANES96, 0, s>>>(
       g, idx->vol, idx->rope, idx->err, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, ksum,
       vsum, so);
+  count_launches(1);
   return cuda_status(cudaGetLastError());
 }
 

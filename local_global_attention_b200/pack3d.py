@@ -23,7 +23,7 @@ EXPORTS = ("pack3d_index_bytes", "pack3d_index_init", "pack3d_build_index", "pac
            "pack3d_block_summaries", "pack3d_forward_workspace_bytes", "pack3d_forward",
            "pack3d_window_forward", "pack3d_stage_kv", "pack3d_forward_staged",
            "pack3d_backward_workspace_bytes", "pack3d_backward", "pack3d_backward_noalloc",
-           "pack3d_strerror")
+           "pack3d_kernel_launches", "pack3d_strerror")
 
 
 class Params(ctypes.Structure):
@@ -88,12 +88,19 @@ def load(build_if_missing: bool = True):
                                         vp, ctypes.c_size_t, vp]
         lib.pack3d_backward_noalloc.argtypes = [P(Params), P(Index), vp, vp, vp, vp, vp, vp, vp,
                                                 vp, vp, vp]
+        lib.pack3d_kernel_launches.argtypes = []
+        lib.pack3d_kernel_launches.restype = ctypes.c_uint64
         lib.pack3d_strerror.argtypes = [ctypes.c_int]
         lib.pack3d_strerror.restype = ctypes.c_char_p
         for name in EXPORTS:
             getattr(lib, name).restype = getattr(lib, name).restype or ctypes.c_int
         _lib = lib
     return _lib
+
+
+def pack3d_kernel_launches() -> int:
+    """Kernels the library has launched in this process so far."""
+    return int(load().pack3d_kernel_launches())
 
 
 def strerror(status: int) -> str:

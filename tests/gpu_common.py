@@ -59,6 +59,21 @@ def assert_close(got, want, dtype, what=""):
     return mx, mean
 
 
+def assert_grad_close(got, want, dtype, what=""):
+    """Gradient parity: the stated absolute bound (max-abs, mean-abs), and the
+    same bound relative to the gradient's own largest magnitude when that is
+    below 1, so that small gradients (bf16 dq and dk are O(1e-3) on the
+    1/sqrt(96)-scaled workloads) are checked as tightly as O(1) outputs are."""
+    mx, mean = assert_close(got, want, dtype, what)
+    ref = float(np.abs(np.asarray(want, np.float64)).max())
+    if 0.0 < ref < 1.0:
+        tmax, tmean = TOL[dtype]
+        assert mx <= tmax * ref and mean <= tmean * ref, (
+            f"{what}: max-abs {mx:.3g} (<= {tmax * ref:.3g}), mean-abs {mean:.3g} "
+            f"(<= {tmean * ref:.3g}) relative to max |{what}| = {ref:.3g}")
+    return mx, mean
+
+
 def sample_queries(wl, order, n, seed=0):
     """Packed indices of a query sample for one batch item: the 8 corners,
     points on faces and edges (one or two coordinates at the volume edge), and

@@ -171,3 +171,35 @@ def test_size_limits(lib):
     # two items fit (0.75 * 2^31)
     fits = shape(B=2, H=8, d=96, Z=64, Y=128, X=128, window=(5, 7, 7), block=(4, 16, 16))
     assert lib.pack3d_index_bytes(ctypes.byref(P.make_params(fits))) > 0
+
+
+def test_backward_rejects_unbuilt_halo_before_any_launch(lib):
+    """The backward stages one halo row (the tile's 8 columns widened by the
+    window radius on both sides and clipped to the volume) at a time, so rows
+    longer than its staging buffer report ERR_UNSUPPORTED.  The check runs on
+    the host before anything is launched: here, on a machine without a GPU, a
+    launch would have returned ERR_CUDA instead.  The allocation-free variant
+    rejects the same shape the same way."""
+    wide = shape(B=1, H=1, d=96, Z=4, Y=4, X=200, window=(1, 1, 161), block=(4, 4, 8))
+    p = P.make_params(wide)
+    idx = P.Index()
+    assert lib.pack3d_index_init(ctypes.byref(p), ctypes.c_void_p(1 << 20),
+                                 ctypes.c_size_t(1 << 40), ctypes.byref(idx)) == P.OK
+    need = lib.pack3d_backward_workspace_bytes(ctypes.byref(p))
+    fake = ctypes.c_void_p(1 << 30)
+    assert lib.pack3d_backward(ctypes.byref(p), ctypes.byref(idx), *([fake] * 9),
+                               ctypes.c_void_p(1 << 32), ctypes.c_size_t(need),
+                               None) == P.ERR_UNSUPPORTED
+    assert lib.pack3d_backward_noalloc(ctypes.byref(p), ctypes.byref(idx), *([fake] * 9),
+                                       None) == P.ERR_UNSUPPORTED
+
+
+def test_kernel_launch_counter_without_cuda(lib):
+    """The launch counter is host-side: readable without a GPU, and calls that
+    are rejected before launching leave it unchanged."""
+    n0 = P.pack3d_kernel_launches()
+    p = P.make_params(shape())
+    idx = P.Index()
+    assert lib.pack3d_forward(ctypes.byref(p), ctypes.byref(idx), None, None, None, None, None,
+                              None, ctypes.c_size_t(0), None, None, None) == P.ERR_ARG
+    assert P.pack3d_kernel_launches() == n0

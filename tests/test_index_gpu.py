@@ -24,7 +24,9 @@ def coords_of(wl, packing):
 
 @pytest.mark.parametrize("wl,packing", [(C.TINY, "raster"), (C.VOL16K, "morton"),
                                         (RAGGED, "random"), (RAGGED, "block"),
-                                        (C.VOL65K, "random"), (C.MICRO1M, "block")])
+                                        (C.VOL65K, "raster"), (C.VOL65K, "morton"),
+                                        (C.VOL65K, "block"), (C.VOL65K, "random"),
+                                        (C.MICRO1M, "block")])
 def test_index_bit_exact(oracle_lib, wl, packing):
     coords = coords_of(wl, packing)
     params = P.make_params(wl)
