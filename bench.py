@@ -106,10 +106,18 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "50"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+        # wait (up to 3 s) for the first sample, so that sampling already runs
+        # when the timed region starts
+        self.first = None
+        if self.proc is not None:
+            import select
+            r, _, _ = select.select([self.proc.stdout], [], [], 3.0)
+            if r:
+                self.first = self.proc.stdout.readline()
         return self
 
     def __exit__(self, *a):
@@ -121,6 +129,7 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
                 out, _ = self.proc.communicate()
+            # the sample taken before the timed region is left out
             self.lines = [ln for ln in out.splitlines() if ln.strip()]
 
     def summary(self):

@@ -1185,21 +1185,21 @@ int launch_forward_simt(const Geo& g, const pack3d_index* idx, const void* q, co
   return forward_dispatch<float>(g, idx, q, k, v, ksum, vsum, out, lse, summaries, s);
 }
 
-int backward_supported(const Geo& g) {
+int backward_simt_supported(const Geo& g) {
   // one halo row (the tile's 8 columns widened by the window radius on both
   // sides, clipped to the volume) must fit in a staged chunk
   return std::min(g.X, TX + 2 * g.rx) <= CAPK ? PACK3D_OK : PACK3D_ERR_UNSUPPORTED;
 }
 
-size_t backward_workspace_bytes(const Geo& g) {
+size_t backward_simt_workspace_bytes(const Geo& g) {
   size_t nd = sizeof(float) * (size_t)g.B * g.H * g.N;
   size_t ns = sizeof(float) * (size_t)g.B * g.H * g.nb * g.d;
   return align256(nd) + 4 * align256(ns) + 2 * (size_t)summary96_splits(g) * ns;
 }
 
-int launch_backward(const Geo& g, const pack3d_index* idx, const void* q, const void* k,
-                    const void* v, const void* out, const float* lse, const void* dout, void* dq,
-                    void* dk, void* dv, void* workspace, cudaStream_t s) {
+int launch_backward_simt(const Geo& g, const pack3d_index* idx, const void* q, const void* k,
+                         const void* v, const void* out, const float* lse, const void* dout,
+                         void* dq, void* dk, void* dv, void* workspace, cudaStream_t s) {
   if (g.dtype == PACK3D_BF16)
     return backward_dispatch<__nv_bfloat16>(g, idx, q, k, v, out, lse, dout, dq, dk, dv,
                                             workspace, s);

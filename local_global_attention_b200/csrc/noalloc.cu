@@ -1,7 +1,10 @@
 // Backward that uses a static device scratch array instead of a
 // caller-allocated workspace, for callers that cannot allocate device memory.
-// It runs the same kernels as pack3d_backward; only where the workspace comes
-// from differs.
+// It runs the CUDA-core backward kernels (fp32 arithmetic), whose workspace -
+// row statistics, the recomputed summaries and their gradients - fits a
+// modest static array; the tensor-core backward of pack3d_backward stages
+// grid-order copies of q, k, v and dO (hundreds of MB at the 65k shape),
+// which no static array of a stated modest size holds.
 #include "pack3d_internal.cuh"
 
 namespace {
@@ -32,12 +35,12 @@ extern "C" int pack3d_backward_noalloc(const pack3d_params* p, const pack3d_inde
   p3d::Geo g;
   int rc = p3d::make_geo(p, &g);
   if (rc) return rc;
-  if ((rc = p3d::backward_supported(g))) return rc;
-  if (p3d::backward_workspace_bytes(g) > PACK3D_NOALLOC_SCRATCH_BYTES)
+  if ((rc = p3d::backward_simt_supported(g))) return rc;
+  if (p3d::backward_workspace_bytes(g, true) > PACK3D_NOALLOC_SCRATCH_BYTES)
     return PACK3D_ERR_UNSUPPORTED;
   if (!idx || !q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv) return PACK3D_ERR_ARG;
   void* scratch = nullptr;
   if ((rc = scratch_for_current_device(&scratch))) return rc;
-  return pack3d_backward(p, idx, q, k, v, out, lse, dout, dq, dk, dv, scratch,
-                         PACK3D_NOALLOC_SCRATCH_BYTES, stream);
+  return p3d::backward_call(p, idx, q, k, v, out, lse, dout, dq, dk, dv, scratch,
+                            PACK3D_NOALLOC_SCRATCH_BYTES, true, (cudaStream_t)stream);
 }

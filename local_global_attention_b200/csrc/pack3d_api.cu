@@ -80,6 +80,11 @@ int make_geo(const pack3d_params* p, Geo* g) {
   return PACK3D_OK;
 }
 
+size_t backward_workspace_bytes(const Geo& g, bool simt) {
+  if (!simt && backward_tc_supported(g)) return backward_tc_workspace_bytes(g);
+  return backward_simt_workspace_bytes(g);
+}
+
 namespace {
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -124,6 +129,25 @@ int check_index(const Geo& g, const pack3d_index* ix) {
 }
 
 }  // namespace
+
+int backward_call(const pack3d_params* p, const pack3d_index* idx, const void* q, const void* k,
+                  const void* v, const void* out, const float* lse, const void* dout, void* dq,
+                  void* dk, void* dv, void* workspace, size_t ws_bytes, bool simt,
+                  cudaStream_t s) {
+  Geo g;
+  int rc = make_geo(p, &g);
+  if (rc) return rc;
+  if ((rc = check_index(g, idx))) return rc;
+  if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv || !workspace)
+    return PACK3D_ERR_ARG;
+  if (((uintptr_t)workspace & 255) || ws_bytes < backward_workspace_bytes(g, simt))
+    return PACK3D_ERR_ARG;
+  if (!simt && backward_tc_supported(g))
+    return launch_backward_tc(g, idx, q, k, v, out, lse, dout, dq, dk, dv, workspace, s);
+  if ((rc = backward_simt_supported(g))) return rc;
+  return launch_backward_simt(g, idx, q, k, v, out, lse, dout, dq, dk, dv, workspace, s);
+}
+
 }  // namespace p3d
 
 using namespace p3d;
@@ -270,17 +294,8 @@ int pack3d_backward(const pack3d_params* p, const pack3d_index* idx, const void*
                     const void* v, const void* out, const float* lse, const void* dout, void* dq,
                     void* dk, void* dv, void* workspace, size_t workspace_bytes,
                     pack3d_stream_t stream) {
-  Geo g;
-  int rc = make_geo(p, &g);
-  if (rc) return rc;
-  if ((rc = check_index(g, idx))) return rc;
-  if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv || !workspace)
-    return PACK3D_ERR_ARG;
-  if (((uintptr_t)workspace & 255) || workspace_bytes < backward_workspace_bytes(g))
-    return PACK3D_ERR_ARG;
-  if ((rc = backward_supported(g))) return rc;
-  return launch_backward(g, idx, q, k, v, out, lse, dout, dq, dk, dv, workspace,
-                         (cudaStream_t)stream);
+  return backward_call(p, idx, q, k, v, out, lse, dout, dq, dk, dv, workspace, workspace_bytes,
+                       false, (cudaStream_t)stream);
 }
 
 uint64_t pack3d_kernel_launches(void) { return g_kernel_launches.load(std::memory_order_relaxed); }

@@ -129,13 +129,30 @@ int launch_stage_kv(const Geo& g, const pack3d_index* idx, const void* k, const 
                     cudaStream_t s);
 int launch_attention_tc(const Geo& g, const pack3d_index* idx, const void* q, void* ws,
                         void* out, float* lse, bool summaries, cudaStream_t s);
-// PACK3D_OK when the backward kernels are built for this shape, else
-// PACK3D_ERR_UNSUPPORTED (checked before anything is launched).
-int backward_supported(const Geo& g);
-size_t backward_workspace_bytes(const Geo& g);
-int launch_backward(const Geo& g, const pack3d_index* idx, const void* q, const void* k,
-                    const void* v, const void* out, const float* lse, const void* dout, void* dq,
-                    void* dk, void* dv, void* workspace, cudaStream_t s);
+// Backward on the CUDA cores (fp32 arithmetic; every dtype and head dim):
+// PACK3D_OK when its kernels are built for this shape, else
+// PACK3D_ERR_UNSUPPORTED (checked before anything is launched); its
+// workspace; its launch.
+int backward_simt_supported(const Geo& g);
+size_t backward_simt_workspace_bytes(const Geo& g);
+int launch_backward_simt(const Geo& g, const pack3d_index* idx, const void* q, const void* k,
+                         const void* v, const void* out, const float* lse, const void* dout,
+                         void* dq, void* dk, void* dv, void* workspace, cudaStream_t s);
+// Backward on the tensor cores (bf16, head_dim 96): whether it applies, its
+// workspace (0 when it does not apply), its launch.
+bool backward_tc_supported(const Geo& g);
+size_t backward_tc_workspace_bytes(const Geo& g);
+int launch_backward_tc(const Geo& g, const pack3d_index* idx, const void* q, const void* k,
+                       const void* v, const void* out, const float* lse, const void* dout,
+                       void* dq, void* dk, void* dv, void* workspace, cudaStream_t s);
+// The backward pack3d_backward runs: the tensor-core one where it applies,
+// else the CUDA-core one (or, with simt, always the CUDA-core one).
+size_t backward_workspace_bytes(const Geo& g, bool simt = false);
+// Argument checks and launch of the backward with a workspace of ws_bytes.
+int backward_call(const pack3d_params* p, const pack3d_index* idx, const void* q, const void* k,
+                  const void* v, const void* out, const float* lse, const void* dout, void* dq,
+                  void* dk, void* dv, void* workspace, size_t ws_bytes, bool simt,
+                  cudaStream_t s);
 
 inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? PACK3D_OK : PACK3D_ERR_CUDA; }
 

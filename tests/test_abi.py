@@ -119,40 +119,59 @@ def test_forward_workspace_size_and_checks(lib):
                                          ctypes.c_size_t(nbytes), fake, fake, None) == P.ERR_ARG
 
 
+def simt_backward_bytes(wl):
+    """Workspace of the CUDA-core backward: delta [B][H][N] + k/v summaries and
+    their gradients (4 x [B][H][nb][d] fp32, each 256-byte aligned) + the
+    d = 96 summary kernel's per-split partial sums (2 x splits x
+    [B][H][nb][d]); the splits fill one wave of two CTAs per SM (148 SMs) over
+    B*H*ceil(nb/64) groups, at most one per query tile and at most 32."""
+    def a256(x):
+        return (x + 255) // 256 * 256
+    nb, nT = wl.n_blocks, -(-wl.Z // 4) * -(-wl.Y // 4) * -(-wl.X // 8)
+    ns = 4 * wl.B * wl.H * nb * wl.d
+    splits = 0
+    if wl.d == 96:
+        splits = max(1, min(296 // (wl.B * wl.H * -(-nb // 64)), nT, 32))
+    return a256(4 * wl.B * wl.H * wl.N) + 4 * a256(ns) + 2 * splits * ns
+
+
 def test_noalloc_scratch_holds_the_training_shape(lib):
-    """The allocation-free backward's static array (its size stated in the
-    header) holds the 65k-token training shape's workspace."""
+    """The allocation-free backward runs the CUDA-core kernels; the static
+    array (its size stated in the header) holds their workspace at the
+    65k-token training shape."""
     from local_global_attention_b200 import configs as C
     hdr = open(HEADER).read()
     m = re.search(r"#define PACK3D_NOALLOC_SCRATCH_BYTES \(\(size_t\)(\d+) << 20\)", hdr)
     assert m and (int(m.group(1)) << 20) == P.NOALLOC_SCRATCH_BYTES
-    need = lib.pack3d_backward_workspace_bytes(ctypes.byref(P.make_params(C.TRAIN65K)))
-    assert 0 < need <= P.NOALLOC_SCRATCH_BYTES
+    assert 0 < simt_backward_bytes(C.TRAIN65K) <= P.NOALLOC_SCRATCH_BYTES
 
 
 def test_backward_workspace_layout(lib):
-    """Backward workspace = delta [B][H][N] + k/v summaries and their gradients
-    (4 x [B][H][nb][d] fp32, each 256-byte aligned) + the d = 96 summary
-    kernel's per-split partial sums (2 x splits x [B][H][nb][d]); the splits
-    fill one wave of two CTAs per SM (148 SMs) over B*H*ceil(nb/64) groups,
-    at most one per query tile and at most 32."""
+    """bf16 at head_dim 96 runs the tensor-core backward, whose workspace holds
+    grid-order copies of rotated k, v, rotated q and dO (4 x [B][H][N][96]
+    bf16), per-voxel (lse, delta) pairs padded to 16 bytes, the fp32 summaries,
+    their bf16 copies, the summary gradients, and the summary role's per-split
+    partial sums (2 x splits x [B][H][nb][96] fp32; the splits fill one wave of
+    148 CTAs over B*H*ceil(nb/128) row tiles, at most 64); every section
+    256-byte aligned.  Other dtypes and head dims run the CUDA-core backward."""
     from local_global_attention_b200 import configs as C
 
     def a256(x):
         return (x + 255) // 256 * 256
 
     for wl in (C.TRAIN65K, C.VOL16K):
-        nb, nT = wl.n_blocks, -(-wl.Z // 4) * -(-wl.Y // 4) * -(-wl.X // 8)
-        groups = wl.B * wl.H * -(-nb // 64)
-        splits = max(1, min(296 // groups, nT, 32))
-        ns = 4 * wl.B * wl.H * nb * wl.d
-        want = a256(4 * wl.B * wl.H * wl.N) + 4 * a256(ns) + 2 * splits * ns
+        nb = wl.n_blocks
+        vox = wl.B * wl.H * wl.N
+        s32 = 4 * wl.B * wl.H * nb * wl.d
+        chunks = -(-wl.Z // 2) * -(-wl.Y // 2) * -(-wl.X // 16)
+        groups = wl.B * wl.H * -(-nb // 128)
+        splits = max(1, min(-(-148 // groups), chunks, 64))
+        want = (4 * a256(vox * 96 * 2) + a256(vox * 16) + 2 * a256(s32) + 2 * a256(s32 // 2) +
+                2 * a256(s32) + a256(splits * 2 * s32))
         assert lib.pack3d_backward_workspace_bytes(ctypes.byref(P.make_params(wl))) == want
-    # other head dims use the simple summary kernel: no partial sums
-    wl = C.TINY
-    ns = 4 * wl.B * wl.H * wl.n_blocks * wl.d
-    assert lib.pack3d_backward_workspace_bytes(ctypes.byref(P.make_params(wl))) == \
-        a256(4 * wl.B * wl.H * wl.N) + 4 * a256(ns)
+    for wl in (C.TINY, C.TRAIN65K.replace(dtype="fp32")):
+        assert lib.pack3d_backward_workspace_bytes(ctypes.byref(P.make_params(wl))) == \
+            simt_backward_bytes(wl)
 
 
 def test_size_limits(lib):
@@ -174,13 +193,14 @@ def test_size_limits(lib):
 
 
 def test_backward_rejects_unbuilt_halo_before_any_launch(lib):
-    """The backward stages one halo row (the tile's 8 columns widened by the
-    window radius on both sides and clipped to the volume) at a time, so rows
-    longer than its staging buffer report ERR_UNSUPPORTED.  The check runs on
+    """The CUDA-core backward stages one halo row (the tile's 8 columns widened
+    by the window radius on both sides and clipped to the volume) at a time, so
+    rows longer than its staging buffer report ERR_UNSUPPORTED.  The check runs on
     the host before anything is launched: here, on a machine without a GPU, a
     launch would have returned ERR_CUDA instead.  The allocation-free variant
     rejects the same shape the same way."""
-    wide = shape(B=1, H=1, d=96, Z=4, Y=4, X=200, window=(1, 1, 161), block=(4, 4, 8))
+    wide = shape(B=1, H=1, d=96, Z=4, Y=4, X=200, window=(1, 1, 161), block=(4, 4, 8),
+                 dtype="fp32")
     p = P.make_params(wide)
     idx = P.Index()
     assert lib.pack3d_index_init(ctypes.byref(p), ctypes.c_void_p(1 << 20),
@@ -191,6 +211,13 @@ def test_backward_rejects_unbuilt_halo_before_any_launch(lib):
                                ctypes.c_void_p(1 << 32), ctypes.c_size_t(need),
                                None) == P.ERR_UNSUPPORTED
     assert lib.pack3d_backward_noalloc(ctypes.byref(p), ctypes.byref(idx), *([fake] * 9),
+                                       None) == P.ERR_UNSUPPORTED
+    # bf16 at head_dim 96: pack3d_backward runs the tensor-core kernels, which
+    # stream halo chunks and have no such limit; the allocation-free backward
+    # runs the CUDA-core kernels and rejects the shape as well
+    pb = P.make_params(shape(B=1, H=1, d=96, Z=4, Y=4, X=200, window=(1, 1, 161),
+                             block=(4, 4, 8)))
+    assert lib.pack3d_backward_noalloc(ctypes.byref(pb), ctypes.byref(idx), *([fake] * 9),
                                        None) == P.ERR_UNSUPPORTED
 
 

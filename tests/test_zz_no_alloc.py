@@ -15,6 +15,8 @@ from local_global_attention_b200 import configs as C
 from local_global_attention_b200 import inputs as I
 from local_global_attention_b200 import pack3d as P
 
+from gpu_common import assert_grad_close
+
 pytestmark = pytest.mark.gpu
 
 CASES = [
@@ -41,17 +43,25 @@ def prepare(wl):
 
 def test_noalloc_backward_matches_workspace_backward():
     """The two cases alternate (A, B, A, B), so every call but the first finds
-    the scratch array filled by a call of another shape and dtype.  The
-    reductions run in a fixed order, so the results must equal the workspace
-    backward's bit for bit."""
+    the scratch array filled by a call of another shape and dtype.  Each call
+    must agree with the workspace backward within the stated tolerance (for
+    bf16 at head_dim 96 that one runs on the tensor cores, this one on the CUDA
+    cores), and the two calls of a case must agree bit for bit: the reductions
+    run in a fixed order, and no call reads scratch it has not written."""
     prepared = [prepare(wl) for wl in CASES]
+    first = {}
     for call in range(2):
         for wl, (params, idx, args, ref) in zip(CASES, prepared):
             got = P.pack3d_backward_noalloc(params, idx, *args)
             torch.cuda.synchronize()
             for name, g_, r_ in zip(("dq", "dk", "dv"), got, ref):
-                assert torch.equal(g_, r_), (wl.name, call, name,
-                                             float((g_.float() - r_.float()).abs().max()))
+                assert_grad_close(g_.cpu(), r_.double().cpu().numpy(), wl.dtype,
+                                  f"{wl.name} call {call} {name}")
+            if call == 0:
+                first[wl.name] = [t.clone() for t in got]
+            else:
+                for name, g_, f_ in zip(("dq", "dk", "dv"), got, first[wl.name]):
+                    assert torch.equal(g_, f_), (wl.name, name)
     for _, idx, _, _ in prepared:
         assert P.pack3d_index_check(idx) == P.OK
 
