@@ -39,7 +39,6 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "forward_tc_vol_32x32x64.md")
 TC_SOURCE = os.path.join(ROOT, "local_global_attention_b200", "csrc", "attn_tc.cu")
-FP32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # CUDA-core fp32 FMA peak, nominal
 
 
 def peaks():
@@ -352,6 +351,35 @@ def profile_value(key):
     return float(m.group(1)) if sha == m_sha.group(1) else None
 
 
+def backward_runner(r, wl):
+    """A closure that runs pack3d_backward once through the C ABI on the
+    runner's inputs and the forward's out and lse (computed here), with
+    dO ~ N(0, 1)."""
+    import ctypes
+
+    import torch
+
+    from local_global_attention_b200 import pack3d as P
+    B, N, H, d = wl.B, wl.N, wl.H, wl.d
+    g_do = torch.Generator().manual_seed(wl.seed + 7)
+    dout = torch.randn(B, N, H, d, generator=g_do).to(r.dev["q"].dtype).cuda()
+    dq, dk, dv = (torch.empty_like(r.dev["q"]) for _ in range(3))
+    nbytes = P.pack3d_backward_workspace_bytes(r.params)
+    ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device="cuda")
+    r.step()  # the forward the backward reads
+    ptr = r.ptr
+    keep = (dout, dq, dk, dv, ws)
+
+    def backward():
+        _ = keep
+        rc = r.lib.pack3d_backward(r.pp, r.ip, ptr(r.dev["q"]), ptr(r.dev["k"]), ptr(r.dev["v"]),
+                                   ptr(r.out), ptr(r.lse), ptr(dout), ptr(dq), ptr(dk), ptr(dv),
+                                   ptr(ws), ctypes.c_size_t(nbytes), r.sp)
+        if rc:
+            raise RuntimeError(f"pack3d_backward failed: {rc}")
+    return backward
+
+
 def micro1m_line(args, pk):
     """The 1,048,576-token microscopy-shaped workload (smooth field, block
     packing): PACK3D step and window-only step, with the attention kernel's
@@ -424,6 +452,16 @@ def run_ours(args):
                               "ms_per_step": ms, "only": "forward"}), flush=True)
         return
 
+    if args.only == "backward":
+        # the forward once, then the backward calls alone (a short run for
+        # profilers); one line, no extras
+        bwd = backward_runner(r, wl_r)
+        bwd_ms = r.time_calls(bwd, max(1, args.steps), warmup=args.warmup)
+        if rank == 0:
+            print(json.dumps({"metric": "backward ms per call", "value": bwd_ms, "unit": "ms",
+                              "only": "backward", "steps": args.steps}), flush=True)
+        return
+
     window_ms, _ = r.timed(args.steps, args.warmup, world, window=True)
     # the packed-sequence comparison mode (1-D RoPE on the packed index): its own
     # params and index (the rotation table differs), the same step
@@ -435,21 +473,7 @@ def run_ours(args):
 
     # the backward (dq, dk, dv from the forward's out and lse) at the same shape,
     # with dO ~ N(0, 1)
-    g_do = torch.Generator().manual_seed(wl_r.seed + 7)
-    dout = torch.randn(B, N, H, d, generator=g_do).to(r.dev["q"].dtype).cuda()
-    dq, dk, dv = (torch.empty_like(r.dev["q"]) for _ in range(3))
-    bws_bytes = P.pack3d_backward_workspace_bytes(r.params)
-    bws = torch.empty(max(bws_bytes, 1), dtype=torch.uint8, device="cuda")
-    r.step()  # the forward the backward reads
-    ptr = r.ptr
-
-    def backward():
-        rc = r.lib.pack3d_backward(r.pp, r.ip, ptr(r.dev["q"]), ptr(r.dev["k"]), ptr(r.dev["v"]),
-                                   ptr(r.out), ptr(r.lse), ptr(dout), ptr(dq), ptr(dk), ptr(dv),
-                                   ptr(bws), ctypes.c_size_t(bws_bytes), r.sp)
-        if rc:
-            raise RuntimeError(f"pack3d_backward failed: {rc}")
-
+    backward = backward_runner(r, wl_r)
     bw_steps = max(3, min(args.steps, 20))
     bwd_ms = max_over_ranks(r.time_calls(backward, bw_steps), world)
     if P.pack3d_index_check(r.idx) != P.OK:
@@ -575,14 +599,15 @@ def run_ours(args):
         "backward": {
             "ms_per_call": bwd_ms,
             "calls": bw_steps,
-            "kernels": "attn_simt.cu (CUDA cores, fp32 arithmetic)",
-            "roofline": {"bound": "alu", "unit": "TFLOP/s",
+            "kernels": "attn_bwd_tc.cu (tcgen05: staging, summary gradients, dq, dk/dv)",
+            "roofline": {"bound": "tensor", "unit": "TFLOP/s",
                          "achieved": work["bwd_flop"] / (bwd_ms * 1e-3) / 1e12,
-                         "peak": FP32_TFLOPS,
-                         "frac": work["bwd_flop"] / (bwd_ms * 1e-3) / 1e12 / FP32_TFLOPS,
-                         "peak_source": "148 SMs x 128 fp32 FMA lanes x 2 FLOP x 1.965 GHz "
-                                        "(nominal unit count and clock)",
-                         "algorithmic_flop_per_call": work["bwd_flop"]},
+                         "peak": peak_tf,
+                         "frac": work["bwd_flop"] / (bwd_ms * 1e-3) / 1e12 / peak_tf,
+                         "peak_source": f"{pk_src} bf16_tflops (burst)",
+                         "algorithmic_flop_per_call": work["bwd_flop"],
+                         "note": "whole call (staging included) against the useful FLOPs: "
+                                 "10 d per window key and per unmasked summary of each query"},
         },
         "window_only": {"ms_per_step": window_ms, "value": tokens / (window_ms * 1e-3),
                         "pack3d_over_window": ms / window_ms},
@@ -681,8 +706,8 @@ def main():
     ap.add_argument("--cpu-sample", type=int, default=32768,
                     help="query tokens the CPU oracle computes for the baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", default="all", choices=["all", "forward"],
-                    help="forward: time the forward step alone and print a short line "
+    ap.add_argument("--only", default="all", choices=["all", "forward", "backward"],
+                    help="forward / backward: time that alone and print a short line "
                          "(for profiler runs)")
     ap.add_argument("--no-micro1m", dest="micro1m", action="store_false",
                     help="skip the 1M-token workload section")

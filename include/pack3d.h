@@ -18,14 +18,12 @@
  *     on that axis); v is not rotated.
  *   - window (wz, wy, wx), all odd: the box of half-widths (w - 1) / 2
  *     centred on the query, clipped at the volume edge (never shifted).
- *   - blocks (bz, by, bx) tile the volume; this library is built for extents
- *     that divide Z, Y, X (others report PACK3D_ERR_UNSUPPORTED: the operator
- *     then cuts the last block along an axis at the volume's edge and averages
- *     over the tokens it holds); a block's summary is the mean of its tokens'
- *     rotated keys and the mean
- *     of their values; a query sees the summary of every block whose box does
- *     not intersect its window box, with logit scale * q~ . kbar and no
- *     count bias.
+ *   - blocks (bz, by, bx) tile the volume in raster order; where an extent
+ *     does not divide the volume, the last block along that axis is cut at the
+ *     volume's edge and holds only the tokens inside it; a block's summary is
+ *     the mean of its tokens' rotated keys and the mean of their values; a
+ *     query sees the summary of every block whose box does not intersect its
+ *     window box, with logit scale * q~ . kbar and no count bias.
  *   - scale defaults to 1 / sqrt(head_dim); lse is the natural log of the
  *     softmax normaliser, summaries included.
  *   - coordinates must be a bijection onto the Z x Y x X grid per batch item
@@ -41,7 +39,8 @@
  *                                    (out is fp32 when out_fp32 is set);
  *   coords                        : int16 [B][N][3] as (z, y, x);
  *   ksum, vsum                    : fp32 [B][H][nb][head_dim], blocks in
- *                                    raster order (nb = Z/bz * Y/by * X/bx);
+ *                                    raster order (nb = ceil(Z/bz) *
+ *                                    ceil(Y/by) * ceil(X/bx));
  *   lse                           : fp32 [B][H][N].
  * N = Z * Y * X.  Every call is asynchronous on the given stream (a
  * cudaStream_t; 0 is the legacy default stream) and returns a status code
@@ -82,9 +81,8 @@ enum {
 
 /* Operator shape and conventions.  head_dim must be a multiple of 12 and at
  * most 96 (12, 24, 48, 96 are built), windows odd and positive, block extents
- * positive (extents that do not divide the volume report
- * PACK3D_ERR_UNSUPPORTED), 1 <= Z, Y, X <= 32767 and
- * B * N * H * head_dim < 2^31. */
+ * positive (any size: blocks that do not divide the volume are cut at its
+ * edge), 1 <= Z, Y, X <= 32767 and B * N * H * head_dim < 2^31. */
 typedef struct {
   int32_t B, H, head_dim;
   int32_t Z, Y, X;

@@ -613,7 +613,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (active) {
           const int kj = ix.vol[((int64_t)b * g.Z + rz) * g.Y * g.X + (int64_t)ry * g.X + rx];
           const int Bk = ((rz / g.bz) * g.nby + ry / g.by) * g.nbx + rx / g.bx;
-          const float inv = 1.f / (float)(g.bz * g.by * g.bx);
+          const BlockExt be = block_ext(g, rz / g.bz, ry / g.by, rx / g.bx);
+          const float inv = 1.f / (float)(be.ez * be.ey * be.ex);
           const float4* srow = reinterpret_cast<const float4*>(
               (hf == 0 ? args.dks : args.dvs) + (((int64_t)b * g.H + h) * g.nb + Bk) * D);
           const float sc = hf == 0 ? g.tau : 1.f;

@@ -1000,7 +1000,8 @@ __global__ void __launch_bounds__(TILE * Split<D>::G) k_bwd_dkdv(
   if (SUMMARY && active) {
     int B = ((cz / g.bz) * g.nby + cy / g.by) * g.nbx + cx / g.bx;
     const int64_t srow = (((int64_t)b * g.H + h) * g.nb + B) * D;
-    const float inv = 1.f / (float)(g.bz * g.by * g.bx);
+    const BlockExt be = block_ext(g, cz / g.bz, cy / g.by, cx / g.bx);
+    const float inv = 1.f / (float)(be.ez * be.ey * be.ex);
 #pragma unroll
     for (int u = 0; u < CPT; ++u) {
       int c = lane * CPT + u;

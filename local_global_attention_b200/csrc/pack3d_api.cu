@@ -44,8 +44,6 @@ int make_geo(const pack3d_params* p, Geo* g) {
   if ((int64_t)p->B * N * p->H * p->head_dim >= (int64_t)1 << 31) return PACK3D_ERR_ARG;
   if (p->head_dim != 12 && p->head_dim != 24 && p->head_dim != 48 && p->head_dim != 96)
     return PACK3D_ERR_UNSUPPORTED;
-  // blocks cut at the volume's edge are a valid operator the kernels do not build
-  if (p->Z % p->bz || p->Y % p->by || p->X % p->bx) return PACK3D_ERR_UNSUPPORTED;
   g->B = p->B;
   g->H = p->H;
   g->d = p->head_dim;
@@ -61,9 +59,10 @@ int make_geo(const pack3d_params* p, Geo* g) {
   g->bz = p->bz;
   g->by = p->by;
   g->bx = p->bx;
-  g->nbz = p->Z / p->bz;
-  g->nby = p->Y / p->by;
-  g->nbx = p->X / p->bx;
+  // blocks that do not divide the volume are cut at its edge: counts round up
+  g->nbz = (p->Z + p->bz - 1) / p->bz;
+  g->nby = (p->Y + p->by - 1) / p->by;
+  g->nbx = (p->X + p->bx - 1) / p->bx;
   g->nb = g->nbz * g->nby * g->nbx;
   g->nTz = (p->Z + TZ - 1) / TZ;
   g->nTy = (p->Y + TY - 1) / TY;

@@ -54,6 +54,15 @@ __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
   return __float2bfloat16_rn(x);
 }
 
+// Extents of block (Bz, By, Bx) cut at the volume's edge (a block that
+// does not fit holds only its voxels inside the volume).
+struct BlockExt {
+  int ez, ey, ex;
+};
+__device__ __forceinline__ BlockExt block_ext(const Geo& g, int Bz, int By, int Bx) {
+  return {min(g.bz, g.Z - Bz * g.bz), min(g.by, g.Y - By * g.by), min(g.bx, g.X - Bx * g.bx)};
+}
+
 // Rotation table entry (cos, sin) of pair j for a token: axial mode, the row of
 // coordinate c on axis a (rows: Z values, then Y, then X); packed mode, the row
 // of the token's packed index pos.

@@ -60,12 +60,13 @@ __global__ void __launch_bounds__(256) k_block_summaries(Geo g, const int32_t* _
   const int c2 = c1 + g.rope_len;            // channels of x2 (and +1)
   float kx1a = 0.f, kx1b = 0.f, kx2a = 0.f, kx2b = 0.f;
   float vx1a = 0.f, vx1b = 0.f, vx2a = 0.f, vx2b = 0.f;
-  const int cnt = g.bz * g.by * g.bx;
+  const BlockExt be = block_ext(g, Bz, By, Bx);  // cut at the volume's edge
+  const int cnt = be.ez * be.ey * be.ex;
   const int32_t* vb = vol + (int64_t)b * g.N;
   if (grp < TG) {
 #pragma unroll 4
     for (int e = grp; e < cnt; e += TG) {
-      int x = e % g.bx, y = (e / g.bx) % g.by, z = e / (g.bx * g.by);
+      int x = e % be.ex, y = (e / be.ex) % be.ey, z = e / (be.ex * be.ey);
       int cz = Bz * g.bz + z, cy = By * g.by + y, cx = Bx * g.bx + x;
       int tok = vb[(cz * g.Y + cy) * g.X + cx];
       int64_t row = (((int64_t)b * g.N + tok) * g.H + h) * g.d;
@@ -154,10 +155,13 @@ __global__ void __launch_bounds__(TG96 * LANES96) k_block_summaries_bf16_d96(
     const int rows = g.bz + g.by + g.bx;
     for (int e = threadIdx.x; e < rows * 16; e += blockDim.x) {
       const int r = e / 16, jj = e % 16;
-      const int grow = r < g.bz ? Bz * g.bz + r
-                                : (r < g.bz + g.by ? g.Z + By * g.by + r - g.bz
-                                                   : g.Z + g.Y + Bx * g.bx + r - g.bz - g.by);
-      tab_s[r * TABS96 + jj] = gtab[grow * 16 + jj];
+      // coordinate of table row r on its axis (rows past the volume's edge, in a
+      // cut block, are not needed)
+      const int c = r < g.bz ? Bz * g.bz + r
+                             : (r < g.bz + g.by ? By * g.by + r - g.bz : Bx * g.bx + r - g.bz - g.by);
+      const int ext = r < g.bz ? g.Z : (r < g.bz + g.by ? g.Y : g.X);
+      const int off = r < g.bz ? 0 : (r < g.bz + g.by ? g.Z : g.Z + g.Y);
+      if (c < ext) tab_s[r * TABS96 + jj] = gtab[(off + c) * 16 + jj];
     }
     __syncthreads();
     tab = a == 0 ? tab_s : (a == 1 ? tab_s + g.bz * TABS96 : tab_s + (g.bz + g.by) * TABS96);
@@ -171,12 +175,13 @@ __global__ void __launch_bounds__(TG96 * LANES96) k_block_summaries_bf16_d96(
   float kx1[8], kx2[8], vx1[8], vx2[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) kx1[i] = kx2[i] = vx1[i] = vx2[i] = 0.f;
-  const int cnt = g.bz * g.by * g.bx;
+  const BlockExt be = block_ext(g, Bz, By, Bx);  // cut at the volume's edge
+  const int cnt = be.ez * be.ey * be.ex;
   const int32_t* vb = vol + (int64_t)b * g.N;
   auto voxel = [&](int e, int& cz, int& cy, int& cx) {
-    cx = Bx * g.bx + e % g.bx;
-    cy = By * g.by + (e / g.bx) % g.by;
-    cz = Bz * g.bz + e / (g.bx * g.by);
+    cx = Bx * g.bx + e % be.ex;
+    cy = By * g.by + (e / be.ex) % be.ey;
+    cz = Bz * g.bz + e / (be.ex * be.ey);
   };
   // One token's rows (already loaded): rotate, accumulate, and with STAGE
   // write the grid-order copies.
@@ -327,7 +332,8 @@ __global__ void __launch_bounds__(BS_THREADS, 2) k_summaries_bulk(
   const int tid = threadIdx.x;
   const int blk = blockIdx.x, b = blockIdx.y;
   const int Bz = blk / (g.nby * g.nbx), By = (blk / g.nbx) % g.nby, Bx = blk % g.nbx;
-  const int cnt = g.bz * g.by * g.bx;
+  const BlockExt be = block_ext(g, Bz, By, Bx);  // cut at the volume's edge
+  const int cnt = be.ez * be.ey * be.ex;
   const int n_stage_rounds = (cnt + BS_TPS - 1) / BS_TPS;
   const uint32_t row_bytes = (uint32_t)g.H * 96 * 2;
   volatile int32_t* abort_flag = &sm.abort;
@@ -344,16 +350,19 @@ __global__ void __launch_bounds__(BS_THREADS, 2) k_summaries_bulk(
   const int tab_rows = g.rope_mode == PACK3D_ROPE_PACKED ? 0 : g.bz + g.by + g.bx;
   for (int e = tid; e < tab_rows * 16; e += BS_THREADS) {
     const int r = e / 16, jj = e % 16;
-    const int grow = r < g.bz ? Bz * g.bz + r
-                              : (r < g.bz + g.by ? g.Z + By * g.by + r - g.bz
-                                                 : g.Z + g.Y + Bx * g.bx + r - g.bz - g.by);
-    sm.tab[r * TABS96 + jj] = gtab[grow * 16 + jj];
+    // coordinate of table row r on its axis (rows past the volume's edge, in a
+    // cut block, are not needed)
+    const int c = r < g.bz ? Bz * g.bz + r
+                           : (r < g.bz + g.by ? By * g.by + r - g.bz : Bx * g.bx + r - g.bz - g.by);
+    const int ext = r < g.bz ? g.Z : (r < g.bz + g.by ? g.Y : g.X);
+    const int off = r < g.bz ? 0 : (r < g.bz + g.by ? g.Z : g.Z + g.Y);
+    if (c < ext) sm.tab[r * TABS96 + jj] = gtab[(off + c) * 16 + jj];
   }
   __syncthreads();
   auto voxel = [&](int e, int& cz, int& cy, int& cx) {
-    cx = Bx * g.bx + e % g.bx;
-    cy = By * g.by + (e / g.bx) % g.by;
-    cz = Bz * g.bz + e / (g.bx * g.by);
+    cx = Bx * g.bx + e % be.ex;
+    cy = By * g.by + (e / be.ex) % be.ey;
+    cz = Bz * g.bz + e / (be.ex * be.ey);
   };
   // consumer item and partial sums (8 channels of k and their partners, same of v)
   const int grp = tid / BS_ITEMS, c = tid % BS_ITEMS;

@@ -214,7 +214,8 @@ def pack3d_block_summaries(params: Params, index: IndexBuffers, k, v, ksum=None,
                            stream=None):
     _need_cuda(k, v)
     B, N, H, d = _dims(params)
-    nb = (params.Z // params.bz) * (params.Y // params.by) * (params.X // params.bx)
+    # blocks that do not divide the volume are cut at its edge: counts round up
+    nb = (-(-params.Z // params.bz)) * (-(-params.Y // params.by)) * (-(-params.X // params.bx))
     if ksum is None:
         ksum = torch.empty(B, H, nb, d, dtype=torch.float32, device=k.device)
     if vsum is None:

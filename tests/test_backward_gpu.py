@@ -78,3 +78,35 @@ PACKED_CASES = [
 def test_backward_packed_rope_mode(oracle_lib, wl):
     """The comparison mode (1-D RoPE on the packed index) through the backward."""
     test_backward_full(oracle_lib, wl)
+
+
+# blocks cut at the volume's edge: a cut block's summary gradient is spread
+# over the voxels it holds
+CUT_CASES = [
+    I.Workload(name="cut_bf16_6x10x20", B=2, H=2, d=96, Z=6, Y=10, X=20, window=(3, 5, 7),
+               block=(4, 3, 8), dtype="bf16", value_scale=1.0 / np.sqrt(96), seed=48),
+    I.Workload(name="cut_fp32_5x7x19", B=1, H=2, d=96, Z=5, Y=7, X=19, window=(3, 3, 5),
+               block=(2, 4, 6), dtype="fp32", seed=49),
+    I.Workload(name="cut_d12_fp32_5x6x7", B=1, H=2, d=12, Z=5, Y=6, X=7, window=(3, 3, 3),
+               block=(2, 4, 3), dtype="fp32", seed=50),
+]
+
+
+@pytest.mark.parametrize("wl", CUT_CASES, ids=lambda w: w.name)
+def test_backward_cut_blocks(oracle_lib, wl):
+    test_backward_full(oracle_lib, wl)
+
+
+def test_backward_cut_blocks_noalloc(oracle_lib):
+    """The allocation-free backward (CUDA-core kernels) on cut blocks, bf16."""
+    wl = CUT_CASES[0]
+    inp = I.make_inputs(wl, "random", with_dout=True)
+    res = gpu_run(wl, inp)
+    from local_global_attention_b200 import pack3d as P
+    d = {k: v.cuda() for k, v in inp.items() if k != "order"}
+    got = P.pack3d_backward_noalloc(res["params"], res["index"], d["q"], d["k"], d["v"],
+                                    res["out"].cuda(), res["lse"].cuda(), d["dout"])
+    torch.cuda.synchronize()
+    want = oracle.backward(wl, inp["coords"], inp["q"], inp["k"], inp["v"], inp["dout"])
+    for name, g_, w_ in zip(("dq", "dk", "dv"), got, want):
+        assert_grad_close(g_.cpu(), w_, wl.dtype, name)

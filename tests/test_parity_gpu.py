@@ -210,3 +210,43 @@ def test_packed_rope_mode_65k(oracle_lib, grid65k):
         outs.append(I.unpack_rows(res["out"], inp["order"]).float())
     # (axial RoPE gives bit-identical outputs here, see the equivariance test)
     assert (outs[0] - outs[1]).abs().max().item() > 1e-4
+
+
+# ---- blocks cut at the volume's edge -----------------------------------------
+# Where a block extent does not divide the volume, the last block along that
+# axis holds only the voxels inside the volume; its summary averages over them.
+
+CUT_SMALL = [
+    I.Workload(name="cut_bf16_d96_6x10x20", B=2, H=2, d=96, Z=6, Y=10, X=20, window=(3, 5, 7),
+               block=(4, 3, 8), dtype="bf16", value_scale=1.0, seed=61),
+    I.Workload(name="cut_fp32_d96_5x7x19", B=1, H=2, d=96, Z=5, Y=7, X=19, window=(3, 3, 5),
+               block=(2, 4, 6), dtype="fp32", seed=62),
+    I.Workload(name="cut_bf16_d48_7x5x9", B=1, H=3, d=48, Z=7, Y=5, X=9, window=(3, 3, 3),
+               block=(3, 2, 4), dtype="bf16", seed=63),
+    # a block wider than the volume along x and z (one cut block per axis)
+    I.Workload(name="cut_wide_bf16_d96_3x8x12", B=1, H=2, d=96, Z=3, Y=8, X=12,
+               window=(1, 3, 3), block=(4, 3, 16), dtype="bf16", seed=64),
+    # more heads than the bulk gather takes (the per-thread gather kernel)
+    I.Workload(name="cut_heads10_bf16_d96_5x6x10", B=1, H=10, d=96, Z=5, Y=6, X=10,
+               window=(3, 3, 5), block=(2, 4, 4), dtype="bf16", seed=65),
+]
+
+
+@pytest.mark.parametrize("wl", CUT_SMALL, ids=lambda w: w.name)
+def test_cut_blocks_forward_and_summaries(oracle_lib, wl):
+    inp = I.make_inputs(wl, "random")
+    res = gpu_run(wl, inp)
+    out, lse = full_oracle(wl, inp, False)
+    assert_close(res["out"], out, wl.dtype, "out")
+    assert_close(res["lse"], lse, wl.dtype, "lse")
+    ks, vs = oracle.block_summaries(wl, inp["coords"], inp["k"], inp["v"])
+    assert res["ksum"].shape[2] == wl.n_blocks
+    np.testing.assert_allclose(res["ksum"].double().numpy(), ks, rtol=0, atol=2e-5)
+    np.testing.assert_allclose(res["vsum"].double().numpy(), vs, rtol=0, atol=2e-5)
+
+
+@pytest.mark.parametrize("wl", [CUT_SMALL[0], CUT_SMALL[3], CUT_SMALL[4]], ids=lambda w: w.name)
+def test_cut_blocks_staged_halves(oracle_lib, wl):
+    """The fused staging pass computes the cut blocks' summaries bit for bit as
+    pack3d_block_summaries does."""
+    test_staged_halves(oracle_lib, wl)
