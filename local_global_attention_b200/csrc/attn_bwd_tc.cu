@@ -59,7 +59,7 @@ using namespace tc;
 using namespace tca;
 
 constexpr int D = 96;
-constexpr int NSTAGE = 4;
+constexpr int NSTAGE = 6;
 constexpr int SEGC = KCH * 64;    // one 32-channel segment of a 64-row chunk (4 KB)
 constexpr int SEGR = 128 * 64;    // one 32-channel segment of the 128-row tile (8 KB)
 constexpr uint32_t CHUNK_BYTES = 6 * SEGC;
@@ -540,25 +540,27 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tmem_ld32(tS, sv);
         tmem_ld32(tdP, dv);
         tmem_wait_ld();
+        const float2 c2p = make_float2(c2, c2);
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          float pe[2], de[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int n = 2 * i + e;
-            float L = Lrow, dl = Drow;
-            if (COL_STATS) {
-              const float2 cs = *reinterpret_cast<const float2*>(&sm.st[s][32 * hf + n]);
-              L = cs.x;
-              dl = cs.y;
-            }
-            const bool keep = !use_bits || ((bits >> n) & 1u);
-            const float p = keep ? ex2(fmaf(__uint_as_float(sv[n]), c2, -L)) : 0.f;
-            pe[e] = p;
-            de[e] = p * (__uint_as_float(dv[n]) - dl);
+          float2 L = make_float2(Lrow, Lrow), dl = make_float2(Drow, Drow);
+          if (COL_STATS) {
+            const float4 s0 = sm.st[s][32 * hf + 2 * i], s1 = sm.st[s][32 * hf + 2 * i + 1];
+            L = make_float2(s0.x, s1.x);
+            dl = make_float2(s0.y, s1.y);
           }
-          pw[i] = pack_bf16x2(pe[0], pe[1]);
-          dw[i] = pack_bf16x2(de[0], de[1]);
+          float2 a = f2_fma(make_float2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])),
+                            c2p, make_float2(-L.x, -L.y));
+          if (use_bits) {
+            if (!((bits >> (2 * i)) & 1u)) a.x = -INFINITY;
+            if (!((bits >> (2 * i + 1)) & 1u)) a.y = -INFINITY;
+          }
+          const float2 p = make_float2(ex2(a.x), ex2(a.y));
+          const float2 ds = f2_mul(
+              p, f2_add(make_float2(__uint_as_float(dv[2 * i]), __uint_as_float(dv[2 * i + 1])),
+                        make_float2(-dl.x, -dl.y)));
+          pw[i] = pack_bf16x2(p.x, p.y);
+          dw[i] = pack_bf16x2(ds.x, ds.y);
         }
       }
       // P over this half's S columns, dS over its dP columns (each half writes
