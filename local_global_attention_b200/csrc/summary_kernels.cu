@@ -371,22 +371,33 @@ __global__ void __launch_bounds__(BS_THREADS, 2) k_summaries_bulk(
   for (int i = 0; i < 8; ++i) kx1[i] = kx2[i] = vx1[i] = vx2[i] = 0.f;
   if (tid >= BS_CONSUMERS) {
     // ---- producer warp: lane i copies token i of each stage ----
+    // The voxel -> token lookups run ahead of the copies: lane 8 q + i holds
+    // token i of round 4 n + q for the batch n of four rounds being issued
+    // (cur) and for the next batch (nxt), so no round waits on a lookup.
+    static_assert(BS_TPS == 8, "four rounds of token lookups per warp");
     const int lane = tid - BS_CONSUMERS;
     const int32_t* vb = vol + (int64_t)b * g.N;
+    auto lookup = [&](int rr) -> int32_t {
+      const int e = rr * BS_TPS + (lane & 7);
+      if (rr >= n_stage_rounds || e >= cnt) return 0;
+      int cz, cy, cx;
+      voxel(e, cz, cy, cx);
+      return vb[(cz * g.Y + cy) * g.X + cx];
+    };
+    int32_t cur = lookup(lane >> 3), nxt = lookup(4 + (lane >> 3));
     for (int r = 0; r < n_stage_rounds; ++r) {
       const int s = r % BS_STAGES;
+      if (r > 0 && (r & 3) == 0) {
+        cur = nxt;
+        nxt = lookup(r + 4 + (lane >> 3));
+      }
       bool ok = true;
       if (lane == 0 && r >= BS_STAGES)
         ok = mbar_wait_or_abort(&sm.empty[s], ((r / BS_STAGES) - 1) & 1, BS_WAIT, abort_flag);
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       const int ntok = min(BS_TPS, cnt - r * BS_TPS);
-      int64_t tok = 0;
-      if (lane < ntok) {
-        int cz, cy, cx;
-        voxel(r * BS_TPS + lane, cz, cy, cx);
-        tok = vb[(cz * g.Y + cy) * g.X + cx];
-        sm.tok[s][lane] = (int32_t)tok;  // published by the arrive below
-      }
+      const int64_t tok = __shfl_sync(0xffffffffu, cur, 8 * (r & 3) + (lane & 7));
+      if (lane < ntok) sm.tok[s][lane] = (int32_t)tok;  // published by the arrive below
       __syncwarp();
       if (lane == 0) mbar_arrive_expect_tx(&sm.full[s], (uint32_t)ntok * 2 * row_bytes);
       __syncwarp();
