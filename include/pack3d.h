@@ -26,8 +26,12 @@
  *     window box, with logit scale * q~ . kbar and no count bias.
  *   - scale defaults to 1 / sqrt(head_dim); lse is the natural log of the
  *     softmax normaliser, summaries included.
- *   - coordinates must be a bijection onto the Z x Y x X grid per batch item
- *     (a dense volume); each batch item may use its own packing.
+ *   - occupancy: by default (n_tokens = 0) the coordinates are a bijection
+ *     onto the Z x Y x X grid per batch item (a dense volume).  With
+ *     n_tokens > 0 every batch item holds n_tokens tokens at distinct voxels
+ *     and the other voxels are empty: windows and blocks hold only the tokens
+ *     present, a block's summary averages over its tokens, and a block
+ *     holding none has no summary.  Each batch item may use its own packing.
  *
  * Memory: every buffer is allocated and owned by the caller; the library
  * never allocates or frees device memory.  Its only global state is a count of
@@ -40,9 +44,10 @@
  *   coords                        : int16 [B][N][3] as (z, y, x);
  *   ksum, vsum                    : fp32 [B][H][nb][head_dim], blocks in
  *                                    raster order (nb = ceil(Z/bz) *
- *                                    ceil(Y/by) * ceil(X/bx));
+ *                                    ceil(Y/by) * ceil(X/bx)); 0 for an
+ *                                    empty block;
  *   lse                           : fp32 [B][H][N].
- * N = Z * Y * X.  Every call is asynchronous on the given stream (a
+ * N = n_tokens if n_tokens > 0, else Z * Y * X.  Every call is asynchronous on the given stream (a
  * cudaStream_t; 0 is the legacy default stream) and returns a status code
  * (0 on success, a negative PACK3D_ERR_* otherwise); no call synchronises
  * except pack3d_index_check.  Errors found on the host (bad arguments) are
@@ -98,13 +103,20 @@ typedef struct {
                         one-dimensional RoPE on the token's packed index (pairs
                         j, j + head_dim/2, theta_j = rope_base^(-2j/head_dim));
                         windows, blocks and summaries stay geometric */
+  int32_t n_tokens;  /* 0: a dense volume, N = Z * Y * X tokens per batch item;
+                        1 .. Z*Y*X: a partly occupied volume of N = n_tokens
+                        tokens per batch item at distinct voxels (the forward
+                        and backward run it on the tensor-core path, bf16 at
+                        head_dim 96; other dtypes and head dims report
+                        PACK3D_ERR_UNSUPPORTED for it) */
 } pack3d_params;
 
 /* Geometry index of one packing, built by pack3d_build_index into one
  * caller-allocated device buffer (see pack3d_index_init).  Query tiles are
  * tile[0] x tile[1] x tile[2] boxes (z, y, x) in raster order, cut by the
  * volume edge where the extents do not divide.
- *   vol      int32 [B][Z*Y*X]   packed index of the token at each voxel
+ *   vol      int32 [B][Z*Y*X]   packed index of the token at each voxel, -1 for
+ *                               an empty voxel
  *   perm     int32 [B][N]       tile-ordered permutation: tile by tile, raster
  *                               order inside a tile, the packed index of each
  *                               token (a counting sort by tile)
@@ -112,15 +124,19 @@ typedef struct {
  *   nbr_off  int32 [T+1]        start of tile t's halo list (same for every
  *                               batch item)
  *   nbr      int32 [B][n_halo]  halo lists: for each tile, the packed indices
- *                               of the tokens in the tile box widened by the
+ *                               of the voxels in the tile box widened by the
  *                               window radius and clipped to the volume, in
- *                               raster order
+ *                               raster order (-1 for an empty voxel)
  *   rope     float [(Z+Y+X)][head_dim/6][2]  cos and sin of c * theta_j per
  *                               axis (z rows, then y, then x), computed in fp64
  *   err      int32 [2]          [0]: 0 or a bit set of 1 = coordinate out of
  *                               range, 2 = voxel held twice, 4 = a kernel
  *                               gave up a bounded device-side wait; [1]:
  *                               smallest offending flat token index b * N + i
+ *   bcount   int32 [B][nb]      tokens held by each block
+ *   bocc     uint32 [B][ceil(nb/32)]  bit B % 32 of word B / 32: block B holds
+ *                               at least one token (built for partly occupied
+ *                               volumes only)
  */
 typedef struct {
   int32_t* vol;
@@ -130,6 +146,8 @@ typedef struct {
   int32_t* nbr;
   float* rope;
   int32_t* err;
+  int32_t* bcount;
+  uint32_t* bocc;
   int32_t tile[3];
   int32_t n_tiles;
   int64_t n_halo;

@@ -310,7 +310,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       }
       if (PENALTY && j < n_local) {
-        penalty_rows(sm.cp[s], g, tb, z, y, x, lane);
+        penalty_rows(sm.cp[s], g, tb, z, y, x, lane, ix.vol + (int64_t)b * g.V);
         fence_proxy_async_smem();
       }
       __syncwarp();
@@ -403,8 +403,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       ry = tb.y0 + lyi;
       rx = tb.x0 + lxi;
       vox = (((int64_t)bh * g.Z + rz) * g.Y + ry) * g.X + rx;
+      // an empty voxel of a partly occupied volume is no row
+      if (active && !occupied(g, ix.vol, b, rz, ry, rx)) active = false;
     } else {
-      active = B0 + r < g.nb;
+      // an empty block has no summary
+      active = B0 + r < g.nb && (!g.partial || ix.bcount[(int64_t)b * g.nb + B0 + r] > 0);
     }
     {
       // A1 row into this lane: channels 0-63 from half 0, 64-95 and the
@@ -504,6 +507,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         } else {
           use_bits = true;
           bits = 0u;
+          // partly occupied volume: the half's 32 query voxels that hold a token
+          // (lane n looks up column n)
+          uint32_t occ = 0xffffffffu;
+          if (g.partial) {
+            const int oz = qz, oy = y + (lane >> 4), ox = x + (lane & 15);
+            const bool in = oz < g.Z && oy < g.Y && ox < g.X && occupied(g, ix.vol, b, oz, oy, ox);
+            occ = __ballot_sync(0xffffffffu, in);
+          }
           if (active && qz < g.Z) {
             const bool zin = qz >= mzlo && qz <= mzhi;
             const uint32_t xs = bit_range(0, min(BXK, g.X - x) - 1);  // in the volume
@@ -516,6 +527,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               const bool meets_zy = zin && qy >= mylo && qy <= myhi;
               bits |= (xs & (meets_zy ? ~xm : 0xffffu)) << (16 * dy);
             }
+            bits &= occ;
           }
           skip = __ballot_sync(0xffffffffu, bits != 0u) == 0u;
         }
@@ -526,6 +538,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         bits = active ? summary_bits(bc, Bs, g.nb, g.nbx, g.nby, bzlo, bzhi, bylo, byhi, bxlo,
                                      bxhi)
                       : 0u;
+        // empty blocks have no summary (Bs is a multiple of 32)
+        if (g.partial && Bs < g.nb) bits &= ix.bocc[(int64_t)b * ((g.nb + 31) / 32) + Bs / 32];
         use_bits = true;
         skip = __ballot_sync(0xffffffffu, bits != 0u) == 0u;
       }
@@ -615,8 +629,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (active) {
           const int kj = ix.vol[((int64_t)b * g.Z + rz) * g.Y * g.X + (int64_t)ry * g.X + rx];
           const int Bk = ((rz / g.bz) * g.nby + ry / g.by) * g.nbx + rx / g.bx;
+          // the tokens the key's block holds (cut at the volume's edge; in a
+          // partly occupied volume, the tokens present)
           const BlockExt be = block_ext(g, rz / g.bz, ry / g.by, rx / g.bx);
-          const float inv = 1.f / (float)(be.ez * be.ey * be.ex);
+          const int held = g.partial ? ix.bcount[(int64_t)b * g.nb + Bk] : be.ez * be.ey * be.ex;
+          const float inv = 1.f / (float)held;
           const float4* srow = reinterpret_cast<const float4*>(
               (hf == 0 ? args.dks : args.dvs) + (((int64_t)b * g.H + h) * g.nb + Bk) * D);
           const float sc = hf == 0 ? g.tau : 1.f;
@@ -688,17 +705,25 @@ __global__ void __launch_bounds__(256)
   __syncthreads();
   const int H = g.H;
   auto grid_row = [&](int hh) { return ((((int64_t)b * H + hh) * g.Z + z) * g.Y + y) * g.X + xb; };
+  // an empty voxel (token -1, partly occupied volumes) gets zero rows and
+  // statistics (0, 0)
   for (int it = threadIdx.x; it < H * nx * 6; it += blockDim.x) {
     const int w = it % 6, rem = it / 6;
     const int x = rem % nx, hh = rem / nx;
     const Item96 item = item96(g, w);
-    const int64_t row = (((int64_t)b * g.N + tok[x]) * H + hh) * D;
-    const uint4* src = reinterpret_cast<const uint4*>(q + row);
-    const uint4* dsrc = reinterpret_cast<const uint4*>(dout + row);
-    uint4 lo = __ldg(src + item.c1), hi = __ldg(src + item.c2);
-    const uint4 dlo = __ldg(dsrc + item.c1), dhi = __ldg(dsrc + item.c2);
-    const int c = item.a == 0 ? z : (item.a == 1 ? y : xb + x);
-    rot_chunk(lo, hi, rope_row96(ix.rope, g, item.a, c, tok[x]), item.j0);
+    const int tk = tok[x];
+    uint4 lo = make_uint4(0, 0, 0, 0), hi = lo, dlo = lo, dhi = lo;
+    if (tk >= 0) {
+      const int64_t row = (((int64_t)b * g.N + tk) * H + hh) * D;
+      const uint4* src = reinterpret_cast<const uint4*>(q + row);
+      const uint4* dsrc = reinterpret_cast<const uint4*>(dout + row);
+      lo = __ldg(src + item.c1);
+      hi = __ldg(src + item.c2);
+      dlo = __ldg(dsrc + item.c1);
+      dhi = __ldg(dsrc + item.c2);
+      const int c = item.a == 0 ? z : (item.a == 1 ? y : xb + x);
+      rot_chunk(lo, hi, rope_row96(ix.rope, g, item.a, c, tk), item.j0);
+    }
     uint4* qd = reinterpret_cast<uint4*>(qg + (grid_row(hh) + x) * D);
     uint4* dd = reinterpret_cast<uint4*>(dog + (grid_row(hh) + x) * D);
     qd[item.c1] = lo;
@@ -708,6 +733,10 @@ __global__ void __launch_bounds__(256)
   }
   for (int it = threadIdx.x; it < H * nx; it += blockDim.x) {
     const int x = it % nx, hh = it / nx;
+    if (tok[x] < 0) {
+      stat[grid_row(hh) + x] = make_float4(0.f, 0.f, 0.f, 0.f);
+      continue;
+    }
     const int64_t row = (((int64_t)b * g.N + tok[x]) * H + hh) * D;
     const uint4* dsrc = reinterpret_cast<const uint4*>(dout + row);
     float acc = 0.f;
@@ -760,7 +789,7 @@ int dsum_splits(const Geo& g) {
 
 BwdWs bwd_layout(const Geo& g) {
   auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
-  const size_t vox = (size_t)g.B * g.H * g.N;
+  const size_t vox = (size_t)g.B * g.H * g.V;  // grid order: one row per voxel
   const size_t vol = vox * D * 2;
   const size_t sum32 = (size_t)g.B * g.H * g.nb * D * 4;
   const size_t sum16 = sum32 / 2;

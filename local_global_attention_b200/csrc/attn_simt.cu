@@ -1187,8 +1187,10 @@ int launch_forward_simt(const Geo& g, const pack3d_index* idx, const void* q, co
 }
 
 int backward_simt_supported(const Geo& g) {
-  // one halo row (the tile's 8 columns widened by the window radius on both
-  // sides, clipped to the volume) must fit in a staged chunk
+  // dense volumes only; one halo row (the tile's 8 columns widened by the
+  // window radius on both sides, clipped to the volume) must fit in a staged
+  // chunk
+  if (g.partial) return PACK3D_ERR_UNSUPPORTED;
   return std::min(g.X, TX + 2 * g.rx) <= CAPK ? PACK3D_OK : PACK3D_ERR_UNSUPPORTED;
 }
 

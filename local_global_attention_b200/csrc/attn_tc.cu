@@ -117,6 +117,7 @@ __global__ void __launch_bounds__(256)
   const int z = zy / g.Y, y = zy % g.Y;
   const int nx = min(GRID_XS, g.X - xb);
   const int64_t vox0 = ((int64_t)b * g.Z * g.Y + zy) * g.X + xb;
+  // an empty voxel (token -1, partly occupied volumes) gets zero rows
   for (int i = threadIdx.x; i < nx; i += blockDim.x) tok[i] = ix.vol[vox0 + i];
   __syncthreads();
   const int H = g.H;
@@ -128,11 +129,15 @@ __global__ void __launch_bounds__(256)
     const int w = it % 6, rem = it / 6;
     const int x = rem % nx, h = rem / nx;
     const Item96 item = item96(g, w);
-    const uint4* src =
-        reinterpret_cast<const uint4*>(k + (((int64_t)b * g.N + tok[x]) * H + h) * D);
-    uint4 lo = __ldg(src + item.c1), hi = __ldg(src + item.c2);
-    const int c = item.a == 0 ? z : (item.a == 1 ? y : xb + x);
-    rot_chunk(lo, hi, rope_row96(ix.rope, g, item.a, c, tok[x]), item.j0);
+    const int tk = tok[x];
+    uint4 lo = make_uint4(0, 0, 0, 0), hi = lo;
+    if (tk >= 0) {
+      const uint4* src = reinterpret_cast<const uint4*>(k + (((int64_t)b * g.N + tk) * H + h) * D);
+      lo = __ldg(src + item.c1);
+      hi = __ldg(src + item.c2);
+      const int c = item.a == 0 ? z : (item.a == 1 ? y : xb + x);
+      rot_chunk(lo, hi, rope_row96(ix.rope, g, item.a, c, tk), item.j0);
+    }
     uint4* dst = reinterpret_cast<uint4*>(kg + (grid_row(h) + x) * D);
     dst[item.c1] = lo;
     dst[item.c2] = hi;
@@ -140,10 +145,10 @@ __global__ void __launch_bounds__(256)
   for (int it = threadIdx.x; it < H * nx * 12; it += blockDim.x) {
     const int c = it % 12, rem = it / 12;
     const int x = rem % nx, h = rem / nx;
-    const uint4* src =
-        reinterpret_cast<const uint4*>(v + (((int64_t)b * g.N + tok[x]) * H + h) * D) + c;
     uint4* dst = reinterpret_cast<uint4*>(vg + (grid_row(h) + x) * D) + c;
-    *dst = __ldg(src);
+    *dst = tok[x] >= 0 ? __ldg(reinterpret_cast<const uint4*>(
+                             v + (((int64_t)b * g.N + tok[x]) * H + h) * D) + c)
+                       : make_uint4(0, 0, 0, 0);
   }
 }
 
@@ -313,7 +318,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       if (j < n_local) {
         // penalty rows of the chunk's keys (dz, dy, dx): key r = (dz * 2 + dy) * 16 + dx
         penalty_rows(sm.kp[s], g, tb, tb.hz0 + BZK * zc, tb.hy0 + BYK * yc, tb.hx0 + BXK * xc,
-                     lane);
+                     lane, ix.vol + (int64_t)b * g.V);
         fence_proxy_async_smem();
         if (++xc == nxc) {
           xc = 0;
@@ -396,10 +401,14 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     // so the warp skips about a third of the chunks.
     const int lzi = (warp >> 1) * 2 + (lane >> 4), lyi = (warp & 1) * 2 + ((lane >> 3) & 1),
               lxi = lane & 7;
-    const bool active = lzi < tb.lz && lyi < tb.ly && lxi < tb.lx;
+    bool active = lzi < tb.lz && lyi < tb.ly && lxi < tb.lx;
     const int cz = tb.z0 + lzi, cy = tb.y0 + lyi, cx = tb.x0 + lxi;
     int qi = 0;
     if (active) qi = ix.vol[(((int64_t)b * g.Z + cz) * g.Y + cy) * g.X + cx];
+    if (qi < 0) {  // an empty voxel of a partly occupied volume: no query
+      active = false;
+      qi = 0;
+    }
     {
       // this thread's query row: gathered, rotated, stored once
       uint4 r[12];
@@ -508,6 +517,12 @@ __global__ void __launch_bounds__(NTHREADS, 2)
         bits0 = summary_bits(bc, B0, g.nb, g.nbx, g.nby, bzlo, bzhi, bylo, byhi, bxlo, bxhi);
         bc.advance_to(B0 + 32, g.nbx, g.nby);
         bits1 = summary_bits(bc, B0 + 32, g.nb, g.nbx, g.nby, bzlo, bzhi, bylo, byhi, bxlo, bxhi);
+        if (g.partial) {
+          // empty blocks have no summary (B0 is a multiple of 64)
+          const uint32_t* occ = ix.bocc + (int64_t)b * ((g.nb + 31) / 32) + B0 / 32;
+          bits0 &= occ[0];
+          if (B0 + 32 < g.nb) bits1 &= occ[1];
+        }
         if (!active) bits0 = bits1 = 0u;
       }
       const bool skip = __ballot_sync(0xffffffffu, (bits0 | bits1) != 0u) == 0u;

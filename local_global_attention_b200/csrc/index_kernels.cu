@@ -14,9 +14,9 @@ namespace {
 constexpr int ERR_RANGE = 1, ERR_DUP = 2;
 
 // Scatter packed index -> voxel, detect out-of-range and duplicated voxels,
-// count tokens per query tile (histogram of the counting sort).
+// count tokens per query tile (histogram of the counting sort) and per block.
 __global__ void k_scatter_coords(Geo g, const int16_t* __restrict__ coords, int32_t* vol,
-                                 int32_t* cnt, int32_t* err) {
+                                 int32_t* cnt, int32_t* bcount, int32_t* err) {
   int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   if (t >= (int64_t)g.B * g.N) return;
   int b = (int)(t / g.N);
@@ -28,7 +28,7 @@ __global__ void k_scatter_coords(Geo g, const int16_t* __restrict__ coords, int3
     return;
   }
   int v = (z * g.Y + y) * g.X + x;
-  int old = atomicCAS(&vol[(int64_t)b * g.N + v], -1, i);
+  int old = atomicCAS(&vol[(int64_t)b * g.V + v], -1, i);
   if (old != -1) {
     atomicOr(&err[0], ERR_DUP);
     atomicMin(&err[1], (int32_t)t);
@@ -36,6 +36,8 @@ __global__ void k_scatter_coords(Geo g, const int16_t* __restrict__ coords, int3
   }
   int tile = ((z / TZ) * g.nTy + (y / TY)) * g.nTx + (x / TX);
   atomicAdd(&cnt[(int64_t)b * g.nT + tile], 1);
+  int blk = ((z / g.bz) * g.nby + (y / g.by)) * g.nbx + (x / g.bx);
+  atomicAdd(&bcount[(int64_t)b * g.nb + blk], 1);
 }
 
 // Exclusive scan of n ints per row (one CTA per row), writes n + 1 values.
@@ -98,6 +100,49 @@ __global__ void k_tile_scatter(Geo g, const int16_t* __restrict__ coords,
   if (slot < g.N) perm[(int64_t)b * g.N + slot] = i;
 }
 
+// Counting-sort scatter of a partly occupied volume: one warp per tile walks
+// its voxels in raster order and gives each token present the next slot (a
+// ballot prefix count), so perm holds the tile's tokens in raster order.
+__global__ void k_tile_perm(Geo g, const int32_t* __restrict__ vol,
+                            const int32_t* __restrict__ tile_off, int32_t* perm,
+                            const int32_t* __restrict__ err) {
+  if (err[0]) return;
+  const int t = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32, b = blockIdx.y;
+  const int lane = threadIdx.x % 32;
+  if (t >= g.nT) return;
+  int z0, y0, x0, lz, ly, lx;
+  tile_box(g, t, z0, y0, x0, lz, ly, lx);
+  const int n = lz * ly * lx;
+  const int base = tile_off[(int64_t)b * (g.nT + 1) + t];
+  const int32_t* vb = vol + (int64_t)b * g.V;
+  int run = 0;
+  for (int e0 = 0; e0 < n; e0 += 32) {
+    const int e = e0 + lane;
+    int tok = -1;
+    if (e < n) {
+      const int x = x0 + e % lx, y = y0 + (e / lx) % ly, z = z0 + e / (lx * ly);
+      tok = vb[(z * g.Y + y) * g.X + x];
+    }
+    const uint32_t present = __ballot_sync(0xffffffffu, tok >= 0);
+    const int pos = run + __popc(present & ((1u << lane) - 1u));
+    if (tok >= 0 && base + pos < g.N) perm[(int64_t)b * g.N + base + pos] = tok;
+    run += __popc(present);
+  }
+}
+
+// Occupancy mask of the blocks: bit B % 32 of word B / 32 set when block B
+// holds a token.
+__global__ void k_block_occ(Geo g, const int32_t* __restrict__ bcount, uint32_t* bocc) {
+  const int nw = (g.nb + 31) / 32;
+  const int64_t w = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (w >= (int64_t)g.B * nw) return;
+  const int b = (int)(w / nw), w0 = (int)(w % nw) * 32;
+  uint32_t bits = 0;
+  for (int i = 0; i < 32 && w0 + i < g.nb; ++i)
+    if (bcount[(int64_t)b * g.nb + w0 + i] > 0) bits |= 1u << i;
+  bocc[w] = bits;
+}
+
 __device__ __forceinline__ void halo_box(const Geo& g, int t, int& hz0, int& hy0, int& hx0,
                                          int& hz, int& hy, int& hx) {
   int z0, y0, x0, lz, ly, lx;
@@ -127,7 +172,7 @@ __global__ void k_halo_lists(Geo g, const int32_t* __restrict__ vol,
   int hz0, hy0, hx0, hz, hy, hx;
   halo_box(g, t, hz0, hy0, hx0, hz, hy, hx);
   int n = hz * hy * hx;
-  const int32_t* vb = vol + (int64_t)b * g.N;
+  const int32_t* vb = vol + (int64_t)b * g.V;
   int32_t* dst = nbr + (int64_t)b * g.n_halo + nbr_off[t];
   for (int e = threadIdx.x; e < n; e += blockDim.x) {
     int x = e % hx, y = (e / hx) % hy, z = e / (hx * hy);
@@ -163,16 +208,26 @@ int launch_build_index(const Geo& g, const int16_t* coords, const pack3d_index* 
                        float rope_base, cudaStream_t s) {
   int64_t tokens = (int64_t)g.B * g.N;
   int32_t* cnt = idx->nbr;  // the halo lists are written last; their space holds the histogram
-  if (cudaMemsetAsync(idx->vol, 0xff, sizeof(int32_t) * tokens, s) != cudaSuccess)
+  if (cudaMemsetAsync(idx->vol, 0xff, sizeof(int32_t) * (size_t)g.B * g.V, s) != cudaSuccess)
     return PACK3D_ERR_CUDA;
   if (cudaMemsetAsync(cnt, 0, sizeof(int32_t) * (size_t)g.B * g.nT, s) != cudaSuccess)
+    return PACK3D_ERR_CUDA;
+  if (cudaMemsetAsync(idx->bcount, 0, sizeof(int32_t) * (size_t)g.B * g.nb, s) != cudaSuccess)
     return PACK3D_ERR_CUDA;
   k_init_err<<<1, 1, 0, s>>>(idx->err);
   int nthr = 256;
   unsigned nblk = (unsigned)((tokens + nthr - 1) / nthr);
-  k_scatter_coords<<<nblk, nthr, 0, s>>>(g, coords, idx->vol, cnt, idx->err);
+  k_scatter_coords<<<nblk, nthr, 0, s>>>(g, coords, idx->vol, cnt, idx->bcount, idx->err);
   k_exclusive_scan<1024><<<g.B, 1024, 0, s>>>(cnt, idx->tile_off, g.nT, g.nT, g.nT + 1);
-  k_tile_scatter<<<nblk, nthr, 0, s>>>(g, coords, idx->tile_off, idx->perm, idx->err);
+  if (g.partial) {
+    k_tile_perm<<<dim3((g.nT + 3) / 4, g.B), 128, 0, s>>>(g, idx->vol, idx->tile_off, idx->perm,
+                                                          idx->err);
+    const int64_t words = (int64_t)g.B * ((g.nb + 31) / 32);
+    k_block_occ<<<(unsigned)((words + 255) / 256), 256, 0, s>>>(g, idx->bcount, idx->bocc);
+    count_launches(1);
+  } else {
+    k_tile_scatter<<<nblk, nthr, 0, s>>>(g, coords, idx->tile_off, idx->perm, idx->err);
+  }
   // Halo sizes reuse the histogram space (tile_off already holds the scan).
   k_halo_sizes<<<(g.nT + 255) / 256, 256, 0, s>>>(g, cnt);
   k_exclusive_scan<1024><<<1, 1024, 0, s>>>(cnt, idx->nbr_off, g.nT, 0, 0);

@@ -40,8 +40,10 @@ int make_geo(const pack3d_params* p, Geo* g) {
   if (p->dtype != PACK3D_BF16 && p->dtype != PACK3D_FP32) return PACK3D_ERR_ARG;
   if (p->rope_mode != PACK3D_ROPE_AXIAL && p->rope_mode != PACK3D_ROPE_PACKED)
     return PACK3D_ERR_ARG;
-  int64_t N = (int64_t)p->Z * p->Y * p->X;
-  if ((int64_t)p->B * N * p->H * p->head_dim >= (int64_t)1 << 31) return PACK3D_ERR_ARG;
+  const int64_t V = (int64_t)p->Z * p->Y * p->X;
+  if (p->n_tokens < 0 || p->n_tokens > V) return PACK3D_ERR_ARG;
+  const int64_t N = p->n_tokens > 0 ? p->n_tokens : V;
+  if ((int64_t)p->B * V * p->H * p->head_dim >= (int64_t)1 << 31) return PACK3D_ERR_ARG;
   if (p->head_dim != 12 && p->head_dim != 24 && p->head_dim != 48 && p->head_dim != 96)
     return PACK3D_ERR_UNSUPPORTED;
   g->B = p->B;
@@ -53,6 +55,8 @@ int make_geo(const pack3d_params* p, Geo* g) {
   g->Y = p->Y;
   g->X = p->X;
   g->N = (int)N;
+  g->V = (int)V;
+  g->partial = N < V ? 1 : 0;
   g->rz = (p->wz - 1) / 2;
   g->ry = (p->wy - 1) / 2;
   g->rx = (p->wx - 1) / 2;
@@ -89,14 +93,14 @@ namespace {
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct IndexLayout {
-  size_t vol, perm, tile_off, nbr_off, nbr, rope, err, total;
+  size_t vol, perm, tile_off, nbr_off, nbr, rope, err, bcount, bocc, total;
 };
 
 IndexLayout index_layout(const Geo& g) {
   IndexLayout L;
   size_t o = 0;
   L.vol = o;
-  o += align256(sizeof(int32_t) * (size_t)g.B * g.N);
+  o += align256(sizeof(int32_t) * (size_t)g.B * g.V);
   L.perm = o;
   o += align256(sizeof(int32_t) * (size_t)g.B * g.N);
   L.tile_off = o;
@@ -113,13 +117,17 @@ IndexLayout index_layout(const Geo& g) {
   o += align256(sizeof(float) * 2 * rope_rows * g.rope_len);
   L.err = o;
   o += 256;
+  L.bcount = o;
+  o += align256(sizeof(int32_t) * (size_t)g.B * g.nb);
+  L.bocc = o;
+  o += align256(sizeof(uint32_t) * (size_t)g.B * ((g.nb + 31) / 32));
   L.total = o;
   return L;
 }
 
 int check_index(const Geo& g, const pack3d_index* ix) {
   if (!ix || !ix->vol || !ix->perm || !ix->tile_off || !ix->nbr_off || !ix->nbr || !ix->rope ||
-      !ix->err)
+      !ix->err || !ix->bcount || !ix->bocc)
     return PACK3D_ERR_ARG;
   if (ix->tile[0] != TZ || ix->tile[1] != TY || ix->tile[2] != TX || ix->n_tiles != g.nT ||
       ix->n_halo != g.n_halo)
@@ -174,6 +182,8 @@ int pack3d_index_init(const pack3d_params* p, void* buffer, size_t bytes, pack3d
   out->nbr = (int32_t*)(base + L.nbr);
   out->rope = (float*)(base + L.rope);
   out->err = (int32_t*)(base + L.err);
+  out->bcount = (int32_t*)(base + L.bcount);
+  out->bocc = (uint32_t*)(base + L.bocc);
   out->tile[0] = TZ;
   out->tile[1] = TY;
   out->tile[2] = TX;
@@ -235,6 +245,8 @@ static int forward_common(const pack3d_params* p, const pack3d_index* idx, const
       return rc;
     return launch_attention_tc(g, idx, q, ws, out, lse, summaries, s);
   }
+  // partly occupied volumes run on the tensor-core path only
+  if (g.partial) return PACK3D_ERR_UNSUPPORTED;
   return launch_forward_simt(g, idx, q, k, v, ksum, vsum, out, lse, summaries, s);
 }
 

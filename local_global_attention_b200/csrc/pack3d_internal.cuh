@@ -15,7 +15,10 @@ constexpr int TZ = 4, TY = 4, TX = 8, TILE = TZ * TY * TX;
 // Geometry derived once on the host from pack3d_params and passed by value.
 struct Geo {
   int B, H, d, da, half;      // half = da / 2 rotation pairs per axis
-  int Z, Y, X, N;
+  int Z, Y, X;
+  int N;                      // tokens per batch item
+  int V;                      // voxels per batch item (Z * Y * X)
+  int partial;                // N < V: a partly occupied volume
   int rz, ry, rx;             // window radii
   int bz, by, bx;             // block extents
   int nbz, nby, nbx, nb;      // block counts
@@ -52,6 +55,13 @@ __device__ __forceinline__ float from_f32<float>(float x) { return x; }
 template <>
 __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
   return __float2bfloat16_rn(x);
+}
+
+// Whether voxel (z, y, x) of batch item b holds a token: always in a dense
+// volume; else the coordinate volume has its token or -1.
+__device__ __forceinline__ bool occupied(const Geo& g, const int32_t* vol, int b, int z, int y,
+                                         int x) {
+  return !g.partial || vol[(((int64_t)b * g.Z + z) * g.Y + y) * g.X + x] >= 0;
 }
 
 // Extents of block (Bz, By, Bx) cut at the volume's edge (a block that

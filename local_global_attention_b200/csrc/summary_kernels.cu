@@ -40,6 +40,7 @@ template <typename T>
 __global__ void __launch_bounds__(256) k_block_summaries(Geo g, const int32_t* __restrict__ vol,
                                                          const float* __restrict__ rope,
                                                          const int32_t* __restrict__ err,
+                                                         const int32_t* __restrict__ bcount,
                                                          const T* __restrict__ k,
                                                          const T* __restrict__ v, float* ksum,
                                                          float* vsum) {
@@ -62,13 +63,14 @@ __global__ void __launch_bounds__(256) k_block_summaries(Geo g, const int32_t* _
   float vx1a = 0.f, vx1b = 0.f, vx2a = 0.f, vx2b = 0.f;
   const BlockExt be = block_ext(g, Bz, By, Bx);  // cut at the volume's edge
   const int cnt = be.ez * be.ey * be.ex;
-  const int32_t* vb = vol + (int64_t)b * g.N;
+  const int32_t* vb = vol + (int64_t)b * g.V;
   if (grp < TG) {
 #pragma unroll 4
     for (int e = grp; e < cnt; e += TG) {
       int x = e % be.ex, y = (e / be.ex) % be.ey, z = e / (be.ex * be.ey);
       int cz = Bz * g.bz + z, cy = By * g.by + y, cx = Bx * g.bx + x;
       int tok = vb[(cz * g.Y + cy) * g.X + cx];
+      if (tok < 0) continue;  // an empty voxel (partly occupied volume)
       int64_t row = (((int64_t)b * g.N + tok) * g.H + h) * g.d;
       float2 k1 = Pair2<T>::f(*reinterpret_cast<const P2*>(k + row + c1));
       float2 k2 = Pair2<T>::f(*reinterpret_cast<const P2*>(k + row + c2));
@@ -97,7 +99,9 @@ __global__ void __launch_bounds__(256) k_block_summaries(Geo g, const int32_t* _
     rv[c2 + 1] = vx2b;
   }
   __syncthreads();
-  const float inv = 1.0f / (float)cnt;
+  // mean over the tokens the block holds (0 for an empty block)
+  const int held = g.partial ? bcount[(int64_t)b * g.nb + blk] : cnt;
+  const float inv = held > 0 ? 1.0f / (float)held : 0.f;
   int64_t base = (((int64_t)b * g.H + h) * g.nb + blk) * g.d;
   for (int c = threadIdx.x; c < 2 * g.d; c += blockDim.x) {
     int which = c / g.d, ch = c % g.d;
@@ -131,8 +135,9 @@ constexpr int TABS96 = 18;  // staged row stride in float2 (16 + padding against
 template <bool STAGE>
 __global__ void __launch_bounds__(TG96 * LANES96) k_block_summaries_bf16_d96(
     Geo g, const int32_t* __restrict__ vol, const float* __restrict__ rope,
-    const int32_t* __restrict__ err, const __nv_bfloat16* __restrict__ k,
-    const __nv_bfloat16* __restrict__ v, float* ksum, float* vsum, StageOut so) {
+    const int32_t* __restrict__ err, const int32_t* __restrict__ bcount,
+    const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v, float* ksum,
+    float* vsum, StageOut so) {
   if (err[0]) return;
   __shared__ float red[TG96][HG96][2][96];
   __shared__ float2 tab_s[TAB96 * TABS96];
@@ -177,7 +182,7 @@ __global__ void __launch_bounds__(TG96 * LANES96) k_block_summaries_bf16_d96(
   for (int i = 0; i < 8; ++i) kx1[i] = kx2[i] = vx1[i] = vx2[i] = 0.f;
   const BlockExt be = block_ext(g, Bz, By, Bx);  // cut at the volume's edge
   const int cnt = be.ez * be.ey * be.ex;
-  const int32_t* vb = vol + (int64_t)b * g.N;
+  const int32_t* vb = vol + (int64_t)b * g.V;
   auto voxel = [&](int e, int& cz, int& cy, int& cx) {
     cx = Bx * g.bx + e % be.ex;
     cy = By * g.by + (e / be.ex) % be.ey;
@@ -188,7 +193,8 @@ __global__ void __launch_bounds__(TG96 * LANES96) k_block_summaries_bf16_d96(
   auto consume = [&](const uint4& ka, const uint4& kb, const uint4& va, const uint4& vb2, int cz,
                      int cy, int cx, int tok_of_consume) {
     const int ca = a == 0 ? cz : (a == 1 ? cy : cx);
-    const float2* t = packed ? rope_row96(rope, g, 0, 0, tok_of_consume) + j0
+    // (an empty voxel's rows are zeros: any table row rotates them to zeros)
+    const float2* t = packed ? rope_row96(rope, g, 0, 0, max(tok_of_consume, 0)) + j0
                              : tab + (ca - base) * stride + j0;
     const uint32_t* kaw = reinterpret_cast<const uint32_t*>(&ka);
     const uint32_t* kbw = reinterpret_cast<const uint32_t*>(&kb);
@@ -246,12 +252,19 @@ __global__ void __launch_bounds__(TG96 * LANES96) k_block_summaries_bf16_d96(
     const int nta = lookup(e + 2 * TG96, naz, nay, nax);
     const int ntb = lookup(e + 3 * TG96, nbz, nby, nbx);
     if (live) {
-      const uint4* kra = reinterpret_cast<const uint4*>(k + (((int64_t)b * g.N + ta) * g.H + h) * 96);
-      const uint4* vra = reinterpret_cast<const uint4*>(v + (((int64_t)b * g.N + ta) * g.H + h) * 96);
-      const uint4 ka = __ldg(kra + c1), kb = __ldg(kra + c2), va = __ldg(vra + c1),
-                  vb2 = __ldg(vra + c2);
+      // an empty voxel (token -1) contributes zero rows: nothing to the sums,
+      // zeros to the grid-order copies
+      uint4 ka = make_uint4(0, 0, 0, 0), kb = ka, va = ka, vb2 = ka;
+      if (ta >= 0) {
+        const uint4* kra = reinterpret_cast<const uint4*>(k + (((int64_t)b * g.N + ta) * g.H + h) * 96);
+        const uint4* vra = reinterpret_cast<const uint4*>(v + (((int64_t)b * g.N + ta) * g.H + h) * 96);
+        ka = __ldg(kra + c1);
+        kb = __ldg(kra + c2);
+        va = __ldg(vra + c1);
+        vb2 = __ldg(vra + c2);
+      }
       uint4 kbA = make_uint4(0, 0, 0, 0), kbB = kbA, vbA = kbA, vbB = kbA;
-      if (has_b) {
+      if (has_b && tb2 >= 0) {
         const uint4* krb =
             reinterpret_cast<const uint4*>(k + (((int64_t)b * g.N + tb2) * g.H + h) * 96);
         const uint4* vrb =
@@ -284,7 +297,8 @@ __global__ void __launch_bounds__(TG96 * LANES96) k_block_summaries_bf16_d96(
     float acc = 0.f;
     for (int q = 0; q < TG96; ++q) acc += red[q][oh][which][ch];
     const int64_t idx = (((int64_t)b * g.H + hout) * g.nb + blk) * 96 + ch;
-    const float mean = acc / (float)cnt;
+    const int held = g.partial ? bcount[(int64_t)b * g.nb + blk] : cnt;
+    const float mean = held > 0 ? acc / (float)held : 0.f;
     (which ? vsum : ksum)[idx] = mean;
     if (STAGE) (which ? so.vsb : so.ksb)[idx] = __float2bfloat16_rn(mean);
   }
@@ -322,8 +336,9 @@ static_assert(sizeof(float) * BS_TPS * BS_ITEMS * 32 <= sizeof(uint8_t) * BS_STA
 template <bool STAGE>
 __global__ void __launch_bounds__(BS_THREADS, 2) k_summaries_bulk(
     Geo g, const int32_t* __restrict__ vol, const float* __restrict__ rope,
-    int32_t* __restrict__ err, const __nv_bfloat16* __restrict__ k,
-    const __nv_bfloat16* __restrict__ v, float* ksum, float* vsum, StageOut so) {
+    int32_t* __restrict__ err, const int32_t* __restrict__ bcount,
+    const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v, float* ksum,
+    float* vsum, StageOut so) {
   using namespace tc;
   if (err[0]) return;
   extern __shared__ uint8_t bs_raw[];
@@ -376,7 +391,7 @@ __global__ void __launch_bounds__(BS_THREADS, 2) k_summaries_bulk(
     // (cur) and for the next batch (nxt), so no round waits on a lookup.
     static_assert(BS_TPS == 8, "four rounds of token lookups per warp");
     const int lane = tid - BS_CONSUMERS;
-    const int32_t* vb = vol + (int64_t)b * g.N;
+    const int32_t* vb = vol + (int64_t)b * g.V;
     auto lookup = [&](int rr) -> int32_t {
       const int e = rr * BS_TPS + (lane & 7);
       if (rr >= n_stage_rounds || e >= cnt) return 0;
@@ -398,10 +413,12 @@ __global__ void __launch_bounds__(BS_THREADS, 2) k_summaries_bulk(
       const int ntok = min(BS_TPS, cnt - r * BS_TPS);
       const int64_t tok = __shfl_sync(0xffffffffu, cur, 8 * (r & 3) + (lane & 7));
       if (lane < ntok) sm.tok[s][lane] = (int32_t)tok;  // published by the arrive below
+      // empty voxels (token -1, partly occupied volumes) are not copied
+      const int nload = __popc(__ballot_sync(0xffffffffu, lane < ntok && tok >= 0));
       __syncwarp();
-      if (lane == 0) mbar_arrive_expect_tx(&sm.full[s], (uint32_t)ntok * 2 * row_bytes);
+      if (lane == 0) mbar_arrive_expect_tx(&sm.full[s], (uint32_t)nload * 2 * row_bytes);
       __syncwarp();
-      if (lane < ntok) {
+      if (lane < ntok && tok >= 0) {
         bulk_load(sm.ring[s][lane][0], k + (((int64_t)b * g.N + tok) * g.H) * 96, row_bytes,
                   &sm.full[s]);
         bulk_load(sm.ring[s][lane][1], v + (((int64_t)b * g.N + tok) * g.H) * 96, row_bytes,
@@ -433,9 +450,14 @@ __global__ void __launch_bounds__(BS_THREADS, 2) k_summaries_bulk(
         voxel(e, cz, cy, cx);
         const uint4* kr = reinterpret_cast<const uint4*>(sm.ring[s][grp][0] + h * 192);
         const uint4* vr = reinterpret_cast<const uint4*>(sm.ring[s][grp][1] + h * 192);
-        const uint4 ka = kr[c1], kb = kr[c2], va = vr[c1], vb2 = vr[c2];
+        // an empty voxel (token -1, not copied) contributes zero rows: nothing
+        // to the sums, zeros to the grid-order copies
+        const int tk = sm.tok[s][grp];
+        const uint4 z4 = make_uint4(0, 0, 0, 0);
+        const uint4 ka = tk >= 0 ? kr[c1] : z4, kb = tk >= 0 ? kr[c2] : z4;
+        const uint4 va = tk >= 0 ? vr[c1] : z4, vb2 = tk >= 0 ? vr[c2] : z4;
         const int ca = a == 0 ? cz : (a == 1 ? cy : cx);
-        const float2* t = packed ? rope_row96(rope, g, 0, 0, sm.tok[s][grp]) + j0
+        const float2* t = packed ? rope_row96(rope, g, 0, 0, max(tk, 0)) + j0
                                  : tab + (ca - base) * TABS96 + j0;
         const uint32_t* kaw = reinterpret_cast<const uint32_t*>(&ka);
         const uint32_t* kbw = reinterpret_cast<const uint32_t*>(&kb);
@@ -501,7 +523,9 @@ __global__ void __launch_bounds__(BS_THREADS, 2) k_summaries_bulk(
   __syncthreads();
   // sums over the groups in order, means, outputs
   const float* red = reinterpret_cast<const float*>(&sm.ring[0][0][0][0]);
-  const float inv_cnt = 1.f / (float)cnt;
+  // mean over the tokens the block holds (0 for an empty block)
+  const int held = g.partial ? bcount[(int64_t)b * g.nb + blk] : cnt;
+  const float inv_cnt = held > 0 ? 1.f / (float)held : 0.f;
   for (int o = tid; o < g.H * 2 * 96; o += BS_THREADS) {
     const int h = o / 192, which = (o / 96) % 2, ch = o % 96;
     // channel ch of head h: 16-byte chunk ch / 8 is chunk c1 (slots 0-7) or c2
@@ -538,7 +562,7 @@ int launch_bulk(const Geo& g, const pack3d_index* idx, const void* k, const void
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return PACK3D_ERR_CUDA;
-  kern<<<dim3(g.nb, g.B), BS_THREADS, smem, s>>>(g, idx->vol, idx->rope, idx->err,
+  kern<<<dim3(g.nb, g.B), BS_THREADS, smem, s>>>(g, idx->vol, idx->rope, idx->err, idx->bcount,
                                                   (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
                                                   ksum, vsum, so);
   count_launches(1);
@@ -552,8 +576,8 @@ int launch_block_summaries(const Geo& g, const pack3d_index* idx, const void* k,
     if (bulk_supported(g)) return launch_bulk<false>(g, idx, k, v, ksum, vsum, StageOut{}, s);
     dim3 grid96(g.nb, g.B, (g.H + HG96 - 1) / HG96);
     k_block_summaries_bf16_d96<false><<<grid96, TG96 * LANES96, 0, s>>>(
-        g, idx->vol, idx->rope, idx->err, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, ksum,
-        vsum, StageOut{});
+        g, idx->vol, idx->rope, idx->err, idx->bcount, (const __nv_bfloat16*)k,
+        (const __nv_bfloat16*)v, ksum, vsum, StageOut{});
     count_launches(1);
     return cuda_status(cudaGetLastError());
   }
@@ -561,11 +585,12 @@ int launch_block_summaries(const Geo& g, const pack3d_index* idx, const void* k,
   size_t smem = sizeof(float) * TG * 2 * g.d;
   if (g.dtype == PACK3D_BF16)
     k_block_summaries<__nv_bfloat16><<<grid, threads, smem, s>>>(
-        g, idx->vol, idx->rope, idx->err, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
-        ksum, vsum);
+        g, idx->vol, idx->rope, idx->err, idx->bcount, (const __nv_bfloat16*)k,
+        (const __nv_bfloat16*)v, ksum, vsum);
   else
     k_block_summaries<float><<<grid, threads, smem, s>>>(g, idx->vol, idx->rope, idx->err,
-                                                         (const float*)k, (const float*)v, ksum,
+                                                         idx->bcount, (const float*)k,
+                                                         (const float*)v, ksum,
                                                          vsum);
   count_launches(1);
   return cuda_status(cudaGetLastError());
@@ -586,8 +611,8 @@ int launch_block_summaries_staged(const Geo& g, const pack3d_index* idx, const v
   StageOut so{(__nv_bfloat16*)kg, (__nv_bfloat16*)vg, (__nv_bfloat16*)ksb, (__nv_bfloat16*)vsb};
   if (bulk_supported(g)) return launch_bulk<true>(g, idx, k, v, ksum, vsum, so, s);
   k_block_summaries_bf16_d96<true><<<grid96, TG96 * LANES96, 0, s>>>(
-      g, idx->vol, idx->rope, idx->err, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v, ksum,
-      vsum, so);
+      g, idx->vol, idx->rope, idx->err, idx->bcount, (const __nv_bfloat16*)k,
+      (const __nv_bfloat16*)v, ksum, vsum, so);
   count_launches(1);
   return cuda_status(cudaGetLastError());
 }

@@ -73,14 +73,18 @@ __device__ __forceinline__ void onehot_words(int lz, int ly, int lx, uint32_t (&
 
 // Penalty rows of one chunk (64 rows of 32 bytes, 32-byte swizzle) against the
 // tile `tb`: the chunk's box starts at (cz0, cy0, cx0); every lane of the warp
-// writes two rows.  Rows outside the volume are masked in every channel.
+// writes two rows.  Rows outside the volume, and (partly occupied volumes,
+// volb = the batch item's coordinate volume) rows at empty voxels, are masked
+// in every channel.
 __device__ __forceinline__ void penalty_rows(uint8_t* dst, const Geo& g, const TileBox& tb,
-                                             int cz0, int cy0, int cx0, int lane) {
+                                             int cz0, int cy0, int cx0, int lane,
+                                             const int32_t* volb) {
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
     const int r = lane + 32 * half;
     const int kz = cz0 + (r >> 5), ky = cy0 + ((r >> 4) & 1), kx = cx0 + (r & 15);
-    const bool inside = kz < g.Z && ky < g.Y && kx < g.X;
+    bool inside = kz < g.Z && ky < g.Y && kx < g.X;
+    if (inside && g.partial) inside = volb[((int64_t)kz * g.Y + ky) * g.X + kx] >= 0;
     uint32_t w[8];
 #pragma unroll
     for (int a = 0; a < 4; a += 2) {

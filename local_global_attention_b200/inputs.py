@@ -126,6 +126,7 @@ class Workload:
     value_scale: float = 1.0     # multiplies the N(0,1) draws ("normal" only)
     rope_base: float = 100.0
     rope_mode: int = 0           # 0: axial RoPE on grid coordinates; 1: 1-D RoPE on the packed position
+    n_tokens: int = 0            # 0: dense; > 0: that many tokens per item at distinct voxels
     packings: tuple = ("raster",)
     seed: int = 0
     backward: bool = False
@@ -133,8 +134,13 @@ class Workload:
     extra: dict = field(default_factory=dict)
 
     @property
-    def N(self) -> int:
+    def V(self) -> int:
         return self.Z * self.Y * self.X
+
+    @property
+    def N(self) -> int:
+        """Tokens per batch item."""
+        return self.n_tokens or self.V
 
     @property
     def n_blocks(self) -> int:
@@ -149,7 +155,8 @@ class Workload:
 
 
 def grid_tensors(wl: Workload, with_dout: bool = False, device="cpu"):
-    """q, k, v (and dO) in grid raster order, fp32, shape [B, N, H, d].
+    """q, k, v (and dO) in grid raster order, fp32, shape [B, V, H, d] (one
+    row per voxel; a partly occupied workload takes the rows of its tokens).
 
     Drawn from one generator seeded with ``wl.seed``, in the order q, k, v, dO."""
     g = torch.Generator().manual_seed(wl.seed)
@@ -157,14 +164,14 @@ def grid_tensors(wl: Workload, with_dout: bool = False, device="cpu"):
     out = {}
     for nm in names:
         if wl.values == "normal" or nm == "dout":
-            t = torch.randn(wl.B, wl.N, wl.H, wl.d, generator=g, dtype=torch.float32)
+            t = torch.randn(wl.B, wl.V, wl.H, wl.d, generator=g, dtype=torch.float32)
             if nm != "dout":
                 t = t * wl.value_scale
         elif wl.values == "smooth":
-            t = torch.empty(wl.B, wl.N, wl.H, wl.d, dtype=torch.float32)
+            t = torch.empty(wl.B, wl.V, wl.H, wl.d, dtype=torch.float32)
             for b in range(wl.B):
                 t[b] = smooth_field(g, wl.Z, wl.Y, wl.X, wl.H * wl.d, device=device).view(
-                    wl.N, wl.H, wl.d)
+                    wl.V, wl.H, wl.d)
         else:
             raise ValueError(wl.values)
         out[nm] = t
@@ -188,6 +195,16 @@ def make_inputs(wl: Workload, packing: str, with_dout: bool = False, grid=None, 
     dt = torch_dtype(wl.dtype)
     orders = np.stack([packing_order(packing, wl.Z, wl.Y, wl.X, wl.block, wl.seed, b)
                        for b in range(wl.B)])
+    if wl.n_tokens:
+        # a partly occupied volume: a seeded set of n_tokens voxels per item,
+        # packed in the packing's order restricted to the set
+        kept = []
+        for b in range(wl.B):
+            gen = torch.Generator().manual_seed(7_000_003 * (wl.seed + 1) + b)
+            held = np.zeros(wl.V, bool)
+            held[torch.randperm(wl.V, generator=gen)[:wl.n_tokens].numpy()] = True
+            kept.append(orders[b][held[orders[b]]])
+        orders = np.stack(kept)
     coords = np.stack([coords_of_order(orders[b], wl.Z, wl.Y, wl.X) for b in range(wl.B)])
     res = {"coords": torch.from_numpy(coords), "order": torch.from_numpy(orders)}
     idx = torch.from_numpy(orders)
@@ -198,7 +215,8 @@ def make_inputs(wl: Workload, packing: str, with_dout: bool = False, grid=None, 
 
 
 def unpack_rows(t: torch.Tensor, order: torch.Tensor) -> torch.Tensor:
-    """Inverse of the packing along dim 1: packed [B, N, ...] -> raster [B, N, ...]."""
+    """Inverse of the packing along dim 1: packed [B, N, ...] -> raster [B, N, ...]
+    (dense volumes)."""
     out = torch.empty_like(t)
     for b in range(t.shape[0]):
         out[b].index_copy_(0, order[b].to(t.device), t[b])

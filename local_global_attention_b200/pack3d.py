@@ -30,13 +30,14 @@ class Params(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
                 ("B", "H", "head_dim", "Z", "Y", "X", "wz", "wy", "wx", "bz", "by", "bx")] + [
         ("rope_base", ctypes.c_float), ("scale", ctypes.c_float), ("dtype", ctypes.c_int32),
-        ("out_fp32", ctypes.c_int32), ("rope_mode", ctypes.c_int32)]
+        ("out_fp32", ctypes.c_int32), ("rope_mode", ctypes.c_int32), ("n_tokens", ctypes.c_int32)]
 
 
 class Index(ctypes.Structure):
     _fields_ = [("vol", ctypes.c_void_p), ("perm", ctypes.c_void_p),
                 ("tile_off", ctypes.c_void_p), ("nbr_off", ctypes.c_void_p),
                 ("nbr", ctypes.c_void_p), ("rope", ctypes.c_void_p), ("err", ctypes.c_void_p),
+                ("bcount", ctypes.c_void_p), ("bocc", ctypes.c_void_p),
                 ("tile", ctypes.c_int32 * 3), ("n_tiles", ctypes.c_int32),
                 ("n_halo", ctypes.c_int64)]
 
@@ -114,14 +115,15 @@ def _check(status: int, what: str):
 
 def make_params(shape, dtype=None, scale: float = 0.0, out_fp32: bool = False) -> Params:
     """Params from any object with ``B, H, d, Z, Y, X, window, block, rope_base``
-    (and ``dtype`` "bf16"/"fp32" unless given, ``rope_mode`` 0 unless set).
-    ``out_fp32`` makes the forward output fp32 for bf16 inputs."""
+    (and ``dtype`` "bf16"/"fp32" unless given, ``rope_mode`` 0 and ``n_tokens``
+    0 (a dense volume) unless set).  ``out_fp32`` makes the forward output fp32
+    for bf16 inputs."""
     dt = dtype if dtype is not None else getattr(shape, "dtype", "bf16")
     code = {"bf16": BF16, "fp32": FP32, torch.bfloat16: BF16, torch.float32: FP32}[dt]
     w, b = tuple(shape.window), tuple(shape.block)
     return Params(shape.B, shape.H, shape.d, shape.Z, shape.Y, shape.X, w[0], w[1], w[2],
                   b[0], b[1], b[2], float(shape.rope_base), float(scale), code, int(bool(out_fp32)),
-                  int(getattr(shape, "rope_mode", 0) or 0))
+                  int(getattr(shape, "rope_mode", 0) or 0), int(getattr(shape, "n_tokens", 0) or 0))
 
 
 def out_dtype(params: Params, like: torch.Tensor) -> torch.dtype:
@@ -175,10 +177,13 @@ class IndexBuffers:
 
     def arrays(self):
         p, s = self.params, self.struct
-        N = p.Z * p.Y * p.X
+        V = p.Z * p.Y * p.X
+        N = p.n_tokens or V
         T = s.n_tiles
+        nb = (-(-p.Z // p.bz)) * (-(-p.Y // p.by)) * (-(-p.X // p.bx))
         return {
-            "vol": self._view("vol", p.B * N, torch.int32).view(p.B, N),
+            "vol": self._view("vol", p.B * V, torch.int32).view(p.B, V),
+            "bcount": self._view("bcount", p.B * nb, torch.int32).view(p.B, nb),
             "perm": self._view("perm", p.B * N, torch.int32).view(p.B, N),
             "tile_off": self._view("tile_off", p.B * (T + 1), torch.int32).view(p.B, T + 1),
             "nbr_off": self._view("nbr_off", T + 1, torch.int32),
@@ -207,7 +212,7 @@ def pack3d_index_check(index: IndexBuffers, stream=None) -> int:
 
 
 def _dims(params):
-    return params.B, params.Z * params.Y * params.X, params.H, params.head_dim
+    return params.B, params.n_tokens or params.Z * params.Y * params.X, params.H, params.head_dim
 
 
 def pack3d_block_summaries(params: Params, index: IndexBuffers, k, v, ksum=None, vsum=None,

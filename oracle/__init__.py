@@ -142,13 +142,15 @@ def volume(shape, coords):
 
 
 def build_index(shape, coords, tile=(4, 4, 8)):
-    """vol, perm, tile_off, nbr_off, nbr (halo lists) for query tiles ``tile``."""
+    """vol, perm, tile_off, nbr_off, nbr (halo lists) for query tiles ``tile``
+    (vol and nbr hold -1 at the empty voxels of a partly occupied volume, perm
+    only the tokens present)."""
     c = _coords(coords)
     p = params(shape)
-    N = shape.Z * shape.Y * shape.X
+    V = shape.Z * shape.Y * shape.X
     nT = -(-shape.Z // tile[0]) * -(-shape.Y // tile[1]) * -(-shape.X // tile[2])
-    vol = np.empty((shape.B, N), np.int32)
-    perm = np.empty((shape.B, N), np.int32)
+    vol = np.empty((shape.B, V), np.int32)
+    perm = np.empty((shape.B, n_tokens(shape)), np.int32)
     toff = np.empty((shape.B, nT + 1), np.int32)
     noff = np.empty((shape.B, nT + 1), np.int64)
     _check(lib().oracle_build_index(ctypes.byref(p), _ptr(c), tile[0], tile[1], tile[2],

@@ -234,23 +234,25 @@ int oracle_volume(const orc_params* p, const int16_t* coords, int32_t* vol) {
  * axis may be cut by the volume edge).  perm lists, tile by tile and in raster
  * order inside a tile, the packed index of each token; tile_off[b][t] is where
  * tile t starts.  The halo of tile t is the tile box widened by r per axis and
- * clipped to the volume; nbr lists the packed indices of the tokens in it, in
- * raster order, starting at nbr_off[b][t] within batch item b's list (the
- * lists of item b start at b * nbr_off[0][nT]). */
+ * clipped to the volume; nbr lists what the coordinate volume holds at each of
+ * its voxels (a packed index, or -1 for an empty voxel of a partly occupied
+ * volume), in raster order, starting at nbr_off[b][t] within batch item b's
+ * list (the lists of item b start at b * nbr_off[0][nT]).  In a partly
+ * occupied volume perm lists only the tokens present, so a tile's stretch of
+ * perm is as long as the tokens it holds. */
 int oracle_build_index(const orc_params* p, const int16_t* coords, int tz, int ty, int tx,
                        int32_t* vol, int32_t* perm, int32_t* tile_off, int64_t* nbr_off,
                        int32_t* nbr) {
-  if (ntok(p) != nvox(p)) return ORC_ERR_ARG; /* the index is built for dense volumes */
   int rc = oracle_volume(p, coords, vol);
   if (rc) return rc;
   if (tz < 1 || ty < 1 || tx < 1) return ORC_ERR_ARG;
   int nTz = (p->Z + tz - 1) / tz, nTy = (p->Y + ty - 1) / ty, nTx = (p->X + tx - 1) / tx;
   int nT = nTz * nTy * nTx;
   int rz = (p->wz - 1) / 2, ry = (p->wy - 1) / 2, rx = (p->wx - 1) / 2;
-  size_t N = nvox(p);
+  size_t V = nvox(p), N = ntok(p);
   int64_t per_item = 0; /* halo list length of one batch item (geometry only) */
   for (int b = 0; b < p->B; ++b) {
-    const int32_t* vb = vol + (size_t)b * N;
+    const int32_t* vb = vol + (size_t)b * V;
     int32_t* pb = perm + (size_t)b * N;
     int32_t* tob = tile_off + (size_t)b * (nT + 1);
     int64_t* nob = nbr_off + (size_t)b * (nT + 1);
@@ -268,7 +270,8 @@ int oracle_build_index(const orc_params* p, const int16_t* coords, int tz, int t
           tob[t] = fill;
           for (int z = z0; z < z1; ++z)
             for (int y = y0; y < y1; ++y)
-              for (int x = x0; x < x1; ++x) pb[fill++] = vb[vox_id(p, z, y, x)];
+              for (int x = x0; x < x1; ++x)
+                if (vb[vox_id(p, z, y, x)] >= 0) pb[fill++] = vb[vox_id(p, z, y, x)];
           int hz0 = z0 - rz < 0 ? 0 : z0 - rz, hz1 = z1 + rz < p->Z ? z1 + rz : p->Z;
           int hy0 = y0 - ry < 0 ? 0 : y0 - ry, hy1 = y1 + ry < p->Y ? y1 + ry : p->Y;
           int hx0 = x0 - rx < 0 ? 0 : x0 - rx, hx1 = x1 + rx < p->X ? x1 + rx : p->X;

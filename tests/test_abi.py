@@ -230,3 +230,22 @@ def test_kernel_launch_counter_without_cuda(lib):
     assert lib.pack3d_forward(ctypes.byref(p), ctypes.byref(idx), None, None, None, None, None,
                               None, ctypes.c_size_t(0), None, None, None) == P.ERR_ARG
     assert P.pack3d_kernel_launches() == n0
+
+
+def test_partly_occupied_params(lib):
+    """n_tokens: 0 is a dense volume; 1 .. Z*Y*X tokens at distinct voxels is a
+    partly occupied one (the index holds the same arrays, the coordinate volume
+    sized by voxels, the permutation by tokens); outside that range the params
+    are rejected."""
+    dense = P.make_params(shape(B=1, H=2, d=96, Z=4, Y=8, X=16, block=(2, 4, 4)))
+    part = P.make_params(shape(B=1, H=2, d=96, Z=4, Y=8, X=16, block=(2, 4, 4), n_tokens=100))
+    assert lib.pack3d_index_bytes(ctypes.byref(part)) > 0
+    # the permutation shrinks with the token count
+    assert lib.pack3d_index_bytes(ctypes.byref(part)) <= lib.pack3d_index_bytes(ctypes.byref(dense))
+    for bad in (-1, 4 * 8 * 16 + 1):
+        p = P.make_params(shape(B=1, H=2, d=96, Z=4, Y=8, X=16, block=(2, 4, 4), n_tokens=bad))
+        assert lib.pack3d_index_bytes(ctypes.byref(p)) == 0, bad
+    idx = P.Index()
+    assert lib.pack3d_index_init(ctypes.byref(part), ctypes.c_void_p(1 << 20),
+                                 ctypes.c_size_t(1 << 30), ctypes.byref(idx)) == P.OK
+    assert idx.bcount and idx.bocc and idx.bocc > idx.bcount

@@ -424,6 +424,41 @@ def test_index_against_sorting(oracle_lib, dims, window, tile):
             assert np.array_equal(got, halo)
 
 
+def test_index_partly_occupied_against_sorting(oracle_lib):
+    """A partly occupied volume: vol holds the token at each occupied voxel and
+    -1 elsewhere; perm = the tokens present sorted by (tile, raster inside the
+    tile) with numpy's lexsort, tile_off their counts per tile; the halo lists
+    hold, for every voxel of the widened tile box in raster order, its token
+    or -1 (the box is geometry, not occupancy)."""
+    tile = (2, 3, 4)
+    s = shape(B=2, H=1, d=12, Z=5, Y=6, X=7, window=(3, 3, 5), block=(1, 1, 1), n_tokens=97)
+    _, coords = partial_inputs(s, seed=16)
+    ix = oracle.build_index(s, coords, tile)
+    Z, Y, X = s.Z, s.Y, s.X
+    nTz, nTy, nTx = -(-Z // tile[0]), -(-Y // tile[1]), -(-X // tile[2])
+    r = (np.asarray(s.window) - 1) // 2
+    for b in range(s.B):
+        c = coords[b].astype(np.int64)
+        raster = (c[:, 0] * Y + c[:, 1]) * X + c[:, 2]
+        vol = np.full(Z * Y * X, -1)
+        vol[raster] = np.arange(s.n_tokens)
+        assert np.array_equal(ix["vol"][b], vol)
+        tid = ((c[:, 0] // tile[0]) * nTy + c[:, 1] // tile[1]) * nTx + c[:, 2] // tile[2]
+        want = np.lexsort((raster, tid))
+        assert np.array_equal(ix["perm"][b], want)
+        counts = np.bincount(tid, minlength=nTz * nTy * nTx)
+        assert np.array_equal(ix["tile_off"][b], np.concatenate([[0], np.cumsum(counts)]))
+        grid = np.stack(np.meshgrid(np.arange(Z), np.arange(Y), np.arange(X), indexing="ij"),
+                        -1).reshape(-1, 3)
+        for t in range(nTz * nTy * nTx):
+            Tz, Ty, Tx = t // (nTy * nTx), (t // nTx) % nTy, t % nTx
+            lo = np.array([Tz * tile[0], Ty * tile[1], Tx * tile[2]])
+            hi = np.minimum(lo + tile, (Z, Y, X)) - 1
+            near = np.all((grid >= lo - r) & (grid <= hi + r), axis=1)
+            got = ix["nbr"][b, ix["nbr_off"][b, t]:ix["nbr_off"][b, t + 1]]
+            assert np.array_equal(got, vol[np.nonzero(near)[0]])
+
+
 def test_bad_coordinates_rejected(oracle_lib):
     s = shape(B=1, H=1, d=12, Z=2, Y=2, X=2, block=(1, 1, 1))
     _, coords, _ = rand_inputs(s, seed=15)
