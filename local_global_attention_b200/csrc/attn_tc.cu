@@ -167,24 +167,6 @@ __global__ void k_summaries_bf16(const float4* __restrict__ ks, const float4* __
 
 // ---- softmax arithmetic ---------------------------------------------------------
 
-// P = 2^(S c2 + mneg) for the keys in `bits`, 0 elsewhere, packed in pairs into
-// p[0..15]; returns the sum.
-__device__ __forceinline__ float exp_pack(const uint32_t (&sv)[32], uint32_t bits, float c2,
-                                          float mneg, uint32_t* p) {
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const float a0 = ((bits >> (2 * i)) & 1u) ? fmaf(__uint_as_float(sv[2 * i]), c2, mneg)
-                                              : -INFINITY;
-    const float a1 = ((bits >> (2 * i + 1)) & 1u) ? fmaf(__uint_as_float(sv[2 * i + 1]), c2, mneg)
-                                                  : -INFINITY;
-    const float e0 = ex2(a0), e1 = ex2(a1);
-    acc[i & 3] += e0 + e1;
-    p[i] = pack_bf16x2(e0, e1);
-  }
-  return (acc[0] + acc[1]) + (acc[2] + acc[3]);
-}
-
 // P = 2^(S c2 + mneg) for all 32 keys (masked ones carry the penalty), packed
 // in pairs into p[0..15]; returns the sum.
 // The scaling and the running sums use the paired fp32 instructions
@@ -224,15 +206,27 @@ __device__ __forceinline__ float plain_max(const uint32_t (&sv)[32]) {
   return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
 }
 
-// Maximum of S over the keys in `bits` (-inf if none), with independent chains.
-__device__ __forceinline__ float masked_max(const uint32_t (&sv)[32], uint32_t bits) {
-  float m[4];
+// Keys outside `bits` get S = -inf, so the unmasked max and exponentials give
+// them no weight.
+__device__ __forceinline__ void apply_mask(uint32_t (&sv)[32], uint32_t bits) {
 #pragma unroll
-  for (int i = 0; i < 4; ++i) m[i] = -INFINITY;
-#pragma unroll
-  for (int i = 0; i < 32; ++i)
-    if ((bits >> i) & 1u) m[i & 3] = fmaxf(m[i & 3], __uint_as_float(sv[i]));
-  return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+  for (int i = 0; i < 32; ++i) sv[i] = ((bits >> i) & 1u) ? sv[i] : 0xff800000u;
+}
+
+// Summary mask of the 64 blocks [B0, B0 + 64) for one query: every valid block
+// except those whose box meets the query's window, i.e. the blocks
+// (bz, by, bx) with bz in [bzlo, bzhi], by in [bylo, byhi], bx in [bxlo, bxhi]
+// - one raster run of blocks per (bz, by).
+__device__ __forceinline__ uint64_t summary_mask64(const Geo& g, int B0, int bzlo, int bzhi,
+                                                   int bylo, int byhi, int bxlo, int bxhi) {
+  uint64_t m = bit_range64(0, min(64, g.nb - B0) - 1);
+  for (int bz = bzlo; bz <= bzhi; ++bz)
+    for (int by = bylo; by <= byhi; ++by) {
+      const int row = (bz * g.nby + by) * g.nbx - B0;
+      const int lo = max(row + bxlo, 0), hi = min(row + bxhi, 63);
+      m &= ~bit_range64(lo, hi);
+    }
+  return m;
 }
 
 struct Maps {
@@ -482,7 +476,10 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     const uint32_t tS = tbase + lane_base + COL_S;
     const float c2 = g.tau * LOG2E;  // logits -> log2 units
     float m_run = M_FLOOR, l_run = 0.f;
-    RowCursor bc = {0, 0, 0};  // block rows (nbx blocks each, nby rows per plane)
+    // the box of blocks this query's window touches
+    const int bzlo = max(cz - g.rz, 0) / g.bz, bzhi = min(cz + g.rz, g.Z - 1) / g.bz;
+    const int bylo = max(cy - g.ry, 0) / g.by, byhi = min(cy + g.ry, g.Y - 1) / g.by;
+    const int bxlo = max(cx - g.rx, 0) / g.bx, bxhi = min(cx + g.rx, g.X - 1) / g.bx;
     int xc = 0, yc = 0, zc = 0;
     bool ok = true;
     for (int j = 0; j < nch; ++j) {
@@ -509,14 +506,9 @@ __global__ void __launch_bounds__(NTHREADS, 2)
         }
       } else {
         const int B0 = (j - n_local) * KCH;
-        // the box of blocks this query's window touches
-        const int bzlo = max(cz - g.rz, 0) / g.bz, bzhi = min(cz + g.rz, g.Z - 1) / g.bz;
-        const int bylo = max(cy - g.ry, 0) / g.by, byhi = min(cy + g.ry, g.Y - 1) / g.by;
-        const int bxlo = max(cx - g.rx, 0) / g.bx, bxhi = min(cx + g.rx, g.X - 1) / g.bx;
-        bc.advance_to(B0, g.nbx, g.nby);
-        bits0 = summary_bits(bc, B0, g.nb, g.nbx, g.nby, bzlo, bzhi, bylo, byhi, bxlo, bxhi);
-        bc.advance_to(B0 + 32, g.nbx, g.nby);
-        bits1 = summary_bits(bc, B0 + 32, g.nb, g.nbx, g.nby, bzlo, bzhi, bylo, byhi, bxlo, bxhi);
+        const uint64_t m64 = summary_mask64(g, B0, bzlo, bzhi, bylo, byhi, bxlo, bxhi);
+        bits0 = (uint32_t)m64;
+        bits1 = (uint32_t)(m64 >> 32);
         if (g.partial) {
           // empty blocks have no summary (B0 is a multiple of 64)
           const uint32_t* occ = ix.bocc + (int64_t)b * ((g.nb + 31) / 32) + B0 / 32;
@@ -544,8 +536,11 @@ __global__ void __launch_bounds__(NTHREADS, 2)
         for (int i = 0; i < 32; ++i) p[i] = 0u;
       } else {
         const bool local = !SUMMARY || j < n_local;  // masked by the penalty channels
-        const float cmax = local ? fmaxf(plain_max(sa), plain_max(sb))
-                                 : fmaxf(masked_max(sa, bits0), masked_max(sb, bits1));
+        if (!local) {
+          apply_mask(sa, bits0);
+          apply_mask(sb, bits1);
+        }
+        const float cmax = fmaxf(plain_max(sa), plain_max(sb));
         const float cmax2 = cmax * c2;
         if (cmax2 > m_run + RESCALE_THRESHOLD) {
           corr = ex2(m_run - cmax2);
@@ -556,13 +551,8 @@ __global__ void __launch_bounds__(NTHREADS, 2)
         }
         const float mneg = -m_run;
         // keys 0-63 -> P columns 0-31
-        if (local) {
-          l_run += exp_pack_all(sa, c2, mneg, p);
-          l_run += exp_pack_all(sb, c2, mneg, p + 16);
-        } else {
-          l_run += exp_pack(sa, bits0, c2, mneg, p);
-          l_run += exp_pack(sb, bits1, c2, mneg, p + 16);
-        }
+        l_run += exp_pack_all(sa, c2, mneg, p);
+        l_run += exp_pack_all(sb, c2, mneg, p + 16);
       }
       // P and O are free once PV_{j-1} is done (the MMA issues PV_j only after
       // p_full below, so this phase is never two behind)
