@@ -109,6 +109,26 @@ typedef struct {
                         and backward run it on the tensor-core path, bf16 at
                         head_dim 96; other dtypes and head dims report
                         PACK3D_ERR_UNSUPPORTED for it) */
+  int32_t Z_total;   /* 0: the volume is the whole problem.  > 0: spatial sharding
+                        along z.  The call's volume holds planes
+                        [z_origin, z_origin + Z) of a volume of Z_total planes
+                        (one rank's z-slab with its halo planes): coordinates
+                        stay local (0 .. Z-1), RoPE angles and the block grid
+                        follow the global plane z + z_origin (nb counts the
+                        blocks of the whole volume), and only the local planes
+                        [own_lo, own_hi) are owned.  Outputs (out, lse) are
+                        written for tokens in owned planes only, and
+                        pack3d_block_summaries computes the blocks lying wholly
+                        in owned planes and writes zeros for the others, so
+                        that a sum over the ranks (an all-reduce) gives every
+                        block's summary.  A query's window must lie inside the
+                        call's volume: rz halo planes on each side of the owned
+                        planes where the whole volume continues.  Forward on the
+                        tensor-core path only (bf16, head_dim 96), dense
+                        volumes, axial RoPE; others report
+                        PACK3D_ERR_UNSUPPORTED. */
+  int32_t z_origin;  /* global plane of local plane 0 (sharding; 0 otherwise) */
+  int32_t own_lo, own_hi; /* owned local planes (sharding; both 0 otherwise) */
 } pack3d_params;
 
 /* Geometry index of one packing, built by pack3d_build_index into one

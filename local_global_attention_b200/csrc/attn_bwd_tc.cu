@@ -464,7 +464,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int bzlo = max(rz - g.rz, 0) / g.bz, bzhi = min(rz + g.rz, g.Z - 1) / g.bz;
     const int bylo = max(ry - g.ry, 0) / g.by, byhi = min(ry + g.ry, g.Y - 1) / g.by;
     const int bxlo = max(rx - g.rx, 0) / g.bx, bxhi = min(rx + g.rx, g.X - 1) / g.bx;
-    RowCursor bc = {0, 0, 0};
     // DSUM: the range of query coordinates whose window meets this row's block
     int mzlo = 0, mzhi = -1, mylo = 0, myhi = -1, mxlo = 0, mxhi = -1;
     if (ROLE == ROLE_DSUM) {
@@ -534,9 +533,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       } else {
         // DQ: summaries B .. B + 31 of this half
         const int Bs = (j - n_local) * KCH + 32 * hf;
-        bc.advance_to(Bs, g.nbx, g.nby);
-        bits = active ? summary_bits(bc, Bs, g.nb, g.nbx, g.nby, bzlo, bzhi, bylo, byhi, bxlo,
-                                     bxhi)
+        bits = active ? (uint32_t)(summary_mask64(g, (j - n_local) * KCH, bzlo, bzhi, bylo, byhi,
+                                                  bxlo, bxhi) >>
+                                   (32 * hf))
                       : 0u;
         // empty blocks have no summary (Bs is a multiple of 32)
         if (g.partial && Bs < g.nb) bits &= ix.bocc[(int64_t)b * ((g.nb + 31) / 32) + Bs / 32];

@@ -1190,7 +1190,7 @@ int backward_simt_supported(const Geo& g) {
   // dense volumes only; one halo row (the tile's 8 columns widened by the
   // window radius on both sides, clipped to the volume) must fit in a staged
   // chunk
-  if (g.partial) return PACK3D_ERR_UNSUPPORTED;
+  if (g.partial || g.sharded) return PACK3D_ERR_UNSUPPORTED;
   return std::min(g.X, TX + 2 * g.rx) <= CAPK ? PACK3D_OK : PACK3D_ERR_UNSUPPORTED;
 }
 

@@ -213,22 +213,6 @@ __device__ __forceinline__ void apply_mask(uint32_t (&sv)[32], uint32_t bits) {
   for (int i = 0; i < 32; ++i) sv[i] = ((bits >> i) & 1u) ? sv[i] : 0xff800000u;
 }
 
-// Summary mask of the 64 blocks [B0, B0 + 64) for one query: every valid block
-// except those whose box meets the query's window, i.e. the blocks
-// (bz, by, bx) with bz in [bzlo, bzhi], by in [bylo, byhi], bx in [bxlo, bxhi]
-// - one raster run of blocks per (bz, by).
-__device__ __forceinline__ uint64_t summary_mask64(const Geo& g, int B0, int bzlo, int bzhi,
-                                                   int bylo, int byhi, int bxlo, int bxhi) {
-  uint64_t m = bit_range64(0, min(64, g.nb - B0) - 1);
-  for (int bz = bzlo; bz <= bzhi; ++bz)
-    for (int by = bylo; by <= byhi; ++by) {
-      const int row = (bz * g.nby + by) * g.nbx - B0;
-      const int lo = max(row + bxlo, 0), hi = min(row + bxhi, 63);
-      m &= ~bit_range64(lo, hi);
-    }
-  return m;
-}
-
 struct Maps {
   CUtensorMap kg, vg;  // [B*H][Z][Y][X][96] bf16, box {32, 16, 2, 2, 1}
   CUtensorMap ks, vs;  // [B*H][nb][96] bf16, box {32, 64, 1}
@@ -395,7 +379,9 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     // so the warp skips about a third of the chunks.
     const int lzi = (warp >> 1) * 2 + (lane >> 4), lyi = (warp & 1) * 2 + ((lane >> 3) & 1),
               lxi = lane & 7;
-    bool active = lzi < tb.lz && lyi < tb.ly && lxi < tb.lx;
+    // (a z-slab writes its owned planes only)
+    bool active = lzi < tb.lz && lyi < tb.ly && lxi < tb.lx && tb.z0 + lzi >= g.own_lo &&
+                  tb.z0 + lzi < g.own_hi;
     const int cz = tb.z0 + lzi, cy = tb.y0 + lyi, cx = tb.x0 + lxi;
     int qi = 0;
     if (active) qi = ix.vol[(((int64_t)b * g.Z + cz) * g.Y + cy) * g.X + cx];
@@ -476,8 +462,9 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     const uint32_t tS = tbase + lane_base + COL_S;
     const float c2 = g.tau * LOG2E;  // logits -> log2 units
     float m_run = M_FLOOR, l_run = 0.f;
-    // the box of blocks this query's window touches
-    const int bzlo = max(cz - g.rz, 0) / g.bz, bzhi = min(cz + g.rz, g.Z - 1) / g.bz;
+    // the box of blocks this query's window touches (global planes: the
+    // block grid of a z-slab is the whole volume's)
+    const int bzlo = max(cz + g.zo - g.rz, 0) / g.bz, bzhi = min(cz + g.zo + g.rz, g.Zt - 1) / g.bz;
     const int bylo = max(cy - g.ry, 0) / g.by, byhi = min(cy + g.ry, g.Y - 1) / g.by;
     const int bxlo = max(cx - g.rx, 0) / g.bx, bxhi = min(cx + g.rx, g.X - 1) / g.bx;
     int xc = 0, yc = 0, zc = 0;

@@ -36,7 +36,7 @@ __global__ void k_scatter_coords(Geo g, const int16_t* __restrict__ coords, int3
   }
   int tile = ((z / TZ) * g.nTy + (y / TY)) * g.nTx + (x / TX);
   atomicAdd(&cnt[(int64_t)b * g.nT + tile], 1);
-  int blk = ((z / g.bz) * g.nby + (y / g.by)) * g.nbx + (x / g.bx);
+  int blk = (((z + g.zo) / g.bz) * g.nby + (y / g.by)) * g.nbx + (x / g.bx);
   atomicAdd(&bcount[(int64_t)b * g.nb + blk], 1);
 }
 
@@ -189,7 +189,8 @@ __global__ void k_rope_table(Geo g, float base, float* tab) {
   int64_t rows = packed ? g.N : g.Z + g.Y + g.X;
   if (e >= rows * g.rope_len) return;
   int row = (int)(e / g.rope_len), j = (int)(e % g.rope_len);
-  int c = packed ? row : (row < g.Z ? row : (row < g.Z + g.Y ? row - g.Z : row - g.Z - g.Y));
+  // axial rows: the z rows of a z-slab turn by the global plane z + z_origin
+  int c = packed ? row : (row < g.Z ? row + g.zo : (row < g.Z + g.Y ? row - g.Z : row - g.Z - g.Y));
   double theta = pow((double)base, -2.0 * (double)j / (double)(packed ? g.d : g.da));
   double sn, cs;
   sincos((double)c * theta, &sn, &cs);

@@ -57,14 +57,26 @@ int make_geo(const pack3d_params* p, Geo* g) {
   g->N = (int)N;
   g->V = (int)V;
   g->partial = N < V ? 1 : 0;
+  // spatial sharding along z: this call's volume is planes
+  // [z_origin, z_origin + Z) of a volume of Z_total planes
+  if (p->Z_total < 0) return PACK3D_ERR_ARG;
+  g->sharded = p->Z_total > 0 ? 1 : 0;
+  g->Zt = g->sharded ? p->Z_total : p->Z;
+  g->zo = g->sharded ? p->z_origin : 0;
+  g->own_lo = g->sharded ? p->own_lo : 0;
+  g->own_hi = g->sharded ? p->own_hi : p->Z;
+  if (g->sharded && (p->z_origin < 0 || p->z_origin + p->Z > p->Z_total || p->own_lo < 0 ||
+                     p->own_lo >= p->own_hi || p->own_hi > p->Z || p->Z_total > 32767))
+    return PACK3D_ERR_ARG;
   g->rz = (p->wz - 1) / 2;
   g->ry = (p->wy - 1) / 2;
   g->rx = (p->wx - 1) / 2;
   g->bz = p->bz;
   g->by = p->by;
   g->bx = p->bx;
-  // blocks that do not divide the volume are cut at its edge: counts round up
-  g->nbz = (p->Z + p->bz - 1) / p->bz;
+  // blocks that do not divide the volume are cut at its edge: counts round
+  // up; a z-slab uses the block grid of the whole volume
+  g->nbz = (g->Zt + p->bz - 1) / p->bz;
   g->nby = (p->Y + p->by - 1) / p->by;
   g->nbx = (p->X + p->bx - 1) / p->bx;
   g->nb = g->nbz * g->nby * g->nbx;
@@ -91,6 +103,12 @@ size_t backward_workspace_bytes(const Geo& g, bool simt) {
 namespace {
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// z-slabs (spatial sharding) are built for dense volumes with axial RoPE.
+int shard_supported(const Geo& g) {
+  return g.sharded && (g.partial || g.rope_mode != PACK3D_ROPE_AXIAL) ? PACK3D_ERR_UNSUPPORTED
+                                                                      : PACK3D_OK;
+}
 
 struct IndexLayout {
   size_t vol, perm, tile_off, nbr_off, nbr, rope, err, bcount, bocc, total;
@@ -147,6 +165,7 @@ int backward_call(const pack3d_params* p, const pack3d_index* idx, const void* q
   if ((rc = check_index(g, idx))) return rc;
   if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv || !workspace)
     return PACK3D_ERR_ARG;
+  if (g.sharded) return PACK3D_ERR_UNSUPPORTED;  // z-slabs: the forward only
   if (((uintptr_t)workspace & 255) || ws_bytes < backward_workspace_bytes(g, simt))
     return PACK3D_ERR_ARG;
   if (!simt && backward_tc_supported(g))
@@ -237,6 +256,7 @@ static int forward_common(const pack3d_params* p, const pack3d_index* idx, const
   if (rc) return rc;
   if ((rc = check_index(g, idx))) return rc;
   if (!q || !k || !v || !out || !lse || (summaries && (!ksum || !vsum))) return PACK3D_ERR_ARG;
+  if ((rc = shard_supported(g))) return rc;
   const size_t need = forward_tc_workspace_bytes(g);
   if (need) {
     if (!ws || ((uintptr_t)ws & 255) || ws_bytes < need) return PACK3D_ERR_ARG;
@@ -245,8 +265,8 @@ static int forward_common(const pack3d_params* p, const pack3d_index* idx, const
       return rc;
     return launch_attention_tc(g, idx, q, ws, out, lse, summaries, s);
   }
-  // partly occupied volumes run on the tensor-core path only
-  if (g.partial) return PACK3D_ERR_UNSUPPORTED;
+  // partly occupied volumes and z-slabs run on the tensor-core path only
+  if (g.partial || g.sharded) return PACK3D_ERR_UNSUPPORTED;
   return launch_forward_simt(g, idx, q, k, v, ksum, vsum, out, lse, summaries, s);
 }
 
@@ -259,6 +279,7 @@ int pack3d_stage_kv(const pack3d_params* p, const pack3d_index* idx, const void*
   if ((rc = check_index(g, idx))) return rc;
   const size_t need = forward_tc_workspace_bytes(g);
   if (!need) return PACK3D_ERR_UNSUPPORTED;
+  if ((rc = shard_supported(g))) return rc;
   if (!k || !v || (!ksum != !vsum) || !workspace || ((uintptr_t)workspace & 255) ||
       workspace_bytes < need)
     return PACK3D_ERR_ARG;
@@ -275,6 +296,7 @@ int pack3d_forward_staged(const pack3d_params* p, const pack3d_index* idx, const
   if ((rc = check_index(g, idx))) return rc;
   const size_t need = forward_tc_workspace_bytes(g);
   if (!need) return PACK3D_ERR_UNSUPPORTED;
+  if ((rc = shard_supported(g))) return rc;
   if (!q || !out || !lse || !workspace || ((uintptr_t)workspace & 255) || workspace_bytes < need)
     return PACK3D_ERR_ARG;
   return launch_attention_tc(g, idx, q, const_cast<void*>(workspace), out, lse,

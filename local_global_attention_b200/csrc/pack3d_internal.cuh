@@ -19,6 +19,9 @@ struct Geo {
   int N;                      // tokens per batch item
   int V;                      // voxels per batch item (Z * Y * X)
   int partial;                // N < V: a partly occupied volume
+  int sharded;                // a z-slab of a larger volume (Z_total > 0)
+  int Zt, zo;                 // global planes, global plane of local plane 0
+  int own_lo, own_hi;         // owned local planes (all planes when not sharded)
   int rz, ry, rx;             // window radii
   int bz, by, bx;             // block extents
   int nbz, nby, nbx, nb;      // block counts
@@ -65,12 +68,26 @@ __device__ __forceinline__ bool occupied(const Geo& g, const int32_t* vol, int b
 }
 
 // Extents of block (Bz, By, Bx) cut at the volume's edge (a block that
-// does not fit holds only its voxels inside the volume).
+// does not fit holds only its voxels inside the volume); the global volume's
+// edge when the call is a z-slab.
 struct BlockExt {
   int ez, ey, ex;
 };
 __device__ __forceinline__ BlockExt block_ext(const Geo& g, int Bz, int By, int Bx) {
-  return {min(g.bz, g.Z - Bz * g.bz), min(g.by, g.Y - By * g.by), min(g.bx, g.X - Bx * g.bx)};
+  return {min(g.bz, g.Zt - Bz * g.bz), min(g.by, g.Y - By * g.by), min(g.bx, g.X - Bx * g.bx)};
+}
+
+// The local planes [z0, z1) of block row Bz inside this call's volume (the
+// block cut at the volume's edge; a z-slab holds part of the block grid), and
+// whether the block's summary is this call's to give: always, except in a
+// z-slab, where only blocks lying wholly in the owned planes count (the
+// others get zero summaries, so that a sum over the ranks gives every block).
+// The staging passes walk the planes either way.
+__device__ __forceinline__ void block_planes(const Geo& g, int Bz, int& z0, int& z1, bool& own) {
+  const int gz0 = Bz * g.bz, gz1 = min(gz0 + g.bz, g.Zt);
+  z0 = max(gz0 - g.zo, 0);
+  z1 = max(min(gz1 - g.zo, g.Z), z0);
+  own = !g.sharded || (gz0 - g.zo >= g.own_lo && gz1 - g.zo <= g.own_hi);
 }
 
 // Rotation table entry (cos, sin) of pair j for a token: axial mode, the row of

@@ -62,13 +62,16 @@ __global__ void __launch_bounds__(256) k_block_summaries(Geo g, const int32_t* _
   float kx1a = 0.f, kx1b = 0.f, kx2a = 0.f, kx2b = 0.f;
   float vx1a = 0.f, vx1b = 0.f, vx2a = 0.f, vx2b = 0.f;
   const BlockExt be = block_ext(g, Bz, By, Bx);  // cut at the volume's edge
-  const int cnt = be.ez * be.ey * be.ex;
+  int bz0, bz1;  // local planes walked
+  bool own;      // the block's summary is this call's to give
+  block_planes(g, Bz, bz0, bz1, own);
+  const int cnt = (bz1 - bz0) * be.ey * be.ex;
   const int32_t* vb = vol + (int64_t)b * g.V;
   if (grp < TG) {
 #pragma unroll 4
     for (int e = grp; e < cnt; e += TG) {
       int x = e % be.ex, y = (e / be.ex) % be.ey, z = e / (be.ex * be.ey);
-      int cz = Bz * g.bz + z, cy = By * g.by + y, cx = Bx * g.bx + x;
+      int cz = bz0 + z, cy = By * g.by + y, cx = Bx * g.bx + x;
       int tok = vb[(cz * g.Y + cy) * g.X + cx];
       if (tok < 0) continue;  // an empty voxel (partly occupied volume)
       int64_t row = (((int64_t)b * g.N + tok) * g.H + h) * g.d;
@@ -99,9 +102,10 @@ __global__ void __launch_bounds__(256) k_block_summaries(Geo g, const int32_t* _
     rv[c2 + 1] = vx2b;
   }
   __syncthreads();
-  // mean over the tokens the block holds (0 for an empty block)
+  // mean over the tokens the block holds (0 for an empty block, and for a
+  // block a z-slab does not own)
   const int held = g.partial ? bcount[(int64_t)b * g.nb + blk] : cnt;
-  const float inv = held > 0 ? 1.0f / (float)held : 0.f;
+  const float inv = held > 0 && own ? 1.0f / (float)held : 0.f;
   int64_t base = (((int64_t)b * g.H + h) * g.nb + blk) * g.d;
   for (int c = threadIdx.x; c < 2 * g.d; c += blockDim.x) {
     int which = c / g.d, ch = c % g.d;
@@ -162,15 +166,16 @@ __global__ void __launch_bounds__(TG96 * LANES96) k_block_summaries_bf16_d96(
       const int r = e / 16, jj = e % 16;
       // coordinate of table row r on its axis (rows past the volume's edge, in a
       // cut block, are not needed)
-      const int c = r < g.bz ? Bz * g.bz + r
+      // (local planes of a z-slab: the block row starts at Bz bz - z_origin)
+      const int c = r < g.bz ? Bz * g.bz - g.zo + r
                              : (r < g.bz + g.by ? By * g.by + r - g.bz : Bx * g.bx + r - g.bz - g.by);
       const int ext = r < g.bz ? g.Z : (r < g.bz + g.by ? g.Y : g.X);
       const int off = r < g.bz ? 0 : (r < g.bz + g.by ? g.Z : g.Z + g.Y);
-      if (c < ext) tab_s[r * TABS96 + jj] = gtab[(off + c) * 16 + jj];
+      if (c >= 0 && c < ext) tab_s[r * TABS96 + jj] = gtab[(off + c) * 16 + jj];
     }
     __syncthreads();
     tab = a == 0 ? tab_s : (a == 1 ? tab_s + g.bz * TABS96 : tab_s + (g.bz + g.by) * TABS96);
-    base = a == 0 ? Bz * g.bz : (a == 1 ? By * g.by : Bx * g.bx);
+    base = a == 0 ? Bz * g.bz - g.zo : (a == 1 ? By * g.by : Bx * g.bx);
     stride = TABS96;
   } else {
     tab = a == 0 ? gtab : (a == 1 ? gtab + g.Z * 16 : gtab + (g.Z + g.Y) * 16);
@@ -181,12 +186,15 @@ __global__ void __launch_bounds__(TG96 * LANES96) k_block_summaries_bf16_d96(
 #pragma unroll
   for (int i = 0; i < 8; ++i) kx1[i] = kx2[i] = vx1[i] = vx2[i] = 0.f;
   const BlockExt be = block_ext(g, Bz, By, Bx);  // cut at the volume's edge
-  const int cnt = be.ez * be.ey * be.ex;
+  int bz0, bz1;  // local planes walked
+  bool own;      // the block's summary is this call's to give
+  block_planes(g, Bz, bz0, bz1, own);
+  const int cnt = (bz1 - bz0) * be.ey * be.ex;
   const int32_t* vb = vol + (int64_t)b * g.V;
   auto voxel = [&](int e, int& cz, int& cy, int& cx) {
     cx = Bx * g.bx + e % be.ex;
     cy = By * g.by + (e / be.ex) % be.ey;
-    cz = Bz * g.bz + e / (be.ex * be.ey);
+    cz = bz0 + e / (be.ex * be.ey);
   };
   // One token's rows (already loaded): rotate, accumulate, and with STAGE
   // write the grid-order copies.
@@ -298,7 +306,7 @@ __global__ void __launch_bounds__(TG96 * LANES96) k_block_summaries_bf16_d96(
     for (int q = 0; q < TG96; ++q) acc += red[q][oh][which][ch];
     const int64_t idx = (((int64_t)b * g.H + hout) * g.nb + blk) * 96 + ch;
     const int held = g.partial ? bcount[(int64_t)b * g.nb + blk] : cnt;
-    const float mean = held > 0 ? acc / (float)held : 0.f;
+    const float mean = held > 0 && own ? acc / (float)held : 0.f;
     (which ? vsum : ksum)[idx] = mean;
     if (STAGE) (which ? so.vsb : so.ksb)[idx] = __float2bfloat16_rn(mean);
   }
@@ -348,7 +356,10 @@ __global__ void __launch_bounds__(BS_THREADS, 2) k_summaries_bulk(
   const int blk = blockIdx.x, b = blockIdx.y;
   const int Bz = blk / (g.nby * g.nbx), By = (blk / g.nbx) % g.nby, Bx = blk % g.nbx;
   const BlockExt be = block_ext(g, Bz, By, Bx);  // cut at the volume's edge
-  const int cnt = be.ez * be.ey * be.ex;
+  int bz0, bz1;  // local planes walked
+  bool own;      // the block's summary is this call's to give
+  block_planes(g, Bz, bz0, bz1, own);
+  const int cnt = (bz1 - bz0) * be.ey * be.ex;
   const int n_stage_rounds = (cnt + BS_TPS - 1) / BS_TPS;
   const uint32_t row_bytes = (uint32_t)g.H * 96 * 2;
   volatile int32_t* abort_flag = &sm.abort;
@@ -367,17 +378,18 @@ __global__ void __launch_bounds__(BS_THREADS, 2) k_summaries_bulk(
     const int r = e / 16, jj = e % 16;
     // coordinate of table row r on its axis (rows past the volume's edge, in a
     // cut block, are not needed)
-    const int c = r < g.bz ? Bz * g.bz + r
+    // (local planes of a z-slab: the block row starts at Bz bz - z_origin)
+    const int c = r < g.bz ? Bz * g.bz - g.zo + r
                            : (r < g.bz + g.by ? By * g.by + r - g.bz : Bx * g.bx + r - g.bz - g.by);
     const int ext = r < g.bz ? g.Z : (r < g.bz + g.by ? g.Y : g.X);
     const int off = r < g.bz ? 0 : (r < g.bz + g.by ? g.Z : g.Z + g.Y);
-    if (c < ext) sm.tab[r * TABS96 + jj] = gtab[(off + c) * 16 + jj];
+    if (c >= 0 && c < ext) sm.tab[r * TABS96 + jj] = gtab[(off + c) * 16 + jj];
   }
   __syncthreads();
   auto voxel = [&](int e, int& cz, int& cy, int& cx) {
     cx = Bx * g.bx + e % be.ex;
     cy = By * g.by + (e / be.ex) % be.ey;
-    cz = Bz * g.bz + e / (be.ex * be.ey);
+    cz = bz0 + e / (be.ex * be.ey);
   };
   // consumer item and partial sums (8 channels of k and their partners, same of v)
   const int grp = tid / BS_ITEMS, c = tid % BS_ITEMS;
@@ -438,7 +450,7 @@ __global__ void __launch_bounds__(BS_THREADS, 2) k_summaries_bulk(
     const int a = item.a, c1 = item.c1, c2 = item.c2, j0 = item.j0;
     const bool packed = g.rope_mode == PACK3D_ROPE_PACKED;
     const float2* tab = a == 0 ? sm.tab : (a == 1 ? sm.tab + g.bz * TABS96 : sm.tab + (g.bz + g.by) * TABS96);
-    const int base = a == 0 ? Bz * g.bz : (a == 1 ? By * g.by : Bx * g.bx);
+    const int base = a == 0 ? Bz * g.bz - g.zo : (a == 1 ? By * g.by : Bx * g.bx);
     for (int r = 0; r < n_stage_rounds; ++r) {
       const int s = r % BS_STAGES;
       if (!__all_sync(0xffffffffu, mbar_wait_or_abort(&sm.full[s], (r / BS_STAGES) & 1, BS_WAIT,
@@ -523,9 +535,10 @@ __global__ void __launch_bounds__(BS_THREADS, 2) k_summaries_bulk(
   __syncthreads();
   // sums over the groups in order, means, outputs
   const float* red = reinterpret_cast<const float*>(&sm.ring[0][0][0][0]);
-  // mean over the tokens the block holds (0 for an empty block)
+  // mean over the tokens the block holds (0 for an empty block, and for a
+  // block a z-slab does not own)
   const int held = g.partial ? bcount[(int64_t)b * g.nb + blk] : cnt;
-  const float inv_cnt = held > 0 ? 1.f / (float)held : 0.f;
+  const float inv_cnt = held > 0 && own ? 1.f / (float)held : 0.f;
   for (int o = tid; o < g.H * 2 * 96; o += BS_THREADS) {
     const int h = o / 192, which = (o / 96) % 2, ch = o % 96;
     // channel ch of head h: 16-byte chunk ch / 8 is chunk c1 (slots 0-7) or c2

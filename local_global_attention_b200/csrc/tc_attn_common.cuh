@@ -122,50 +122,20 @@ __device__ __forceinline__ void rot_chunk(uint4& lo, uint4& hi, const float2* t,
   }
 }
 
-// Walks the rows of a raster-ordered box (rows of `len` items, `ny` rows per
-// plane) in step with 32-item segments, so no division is needed per segment.
-struct RowCursor {
-  int start;  // index of the first item of the current row
-  int z, y;   // the current row's plane and row within the plane
-  __device__ __forceinline__ void advance_to(int e, int len, int ny) {
-    while (start + len <= e) {
-      start += len;
-      if (++y == ny) {
-        y = 0;
-        ++z;
-      }
+// Summary mask of the 64 blocks [B0, B0 + 64) for one query: every valid block
+// except those whose box meets the query's window, i.e. the blocks
+// (bz, by, bx) with bz in [bzlo, bzhi], by in [bylo, byhi], bx in [bxlo, bxhi]
+// - one raster run of blocks per (bz, by).
+__device__ __forceinline__ uint64_t summary_mask64(const Geo& g, int B0, int bzlo, int bzhi,
+                                                   int bylo, int byhi, int bxlo, int bxhi) {
+  uint64_t m = bit_range64(0, min(64, g.nb - B0) - 1);
+  for (int bz = bzlo; bz <= bzhi; ++bz)
+    for (int by = bylo; by <= byhi; ++by) {
+      const int row = (bz * g.nby + by) * g.nbx - B0;
+      const int lo = max(row + bxlo, 0), hi = min(row + bxhi, 63);
+      m &= ~bit_range64(lo, hi);
     }
-  }
-};
-
-// Summary mask of the 32 blocks [B0, B0 + 32) (raster order over an
-// nbz x nby x nbx grid): set for blocks outside the box [blo, bhi] of blocks
-// the query's window touches.  `c` is at the block row holding B0.
-__device__ __forceinline__ uint32_t summary_bits(RowCursor c, int B0, int nb, int nbx, int nby,
-                                                 int bzlo, int bzhi, int bylo, int byhi, int bxlo,
-                                                 int bxhi) {
-  uint32_t bits = 0;
-  int pos = c.start - B0;
-  int z = c.z, y = c.y;
-  while (pos < 32) {
-    const int lo = max(pos, 0), hi = min(pos + nbx - 1, 31);
-    if (lo <= hi) {
-      uint32_t row = bit_range(lo, hi);
-      if (z >= bzlo && z <= bzhi && y >= bylo && y <= byhi) {
-        const int elo = max(pos + bxlo, 0), ehi = min(pos + bxhi, 31);
-        if (elo <= ehi) row &= ~bit_range(elo, ehi);
-      }
-      bits |= row;
-    }
-    pos += nbx;
-    if (++y == nby) {
-      y = 0;
-      ++z;
-    }
-  }
-  const int valid = nb - B0;
-  if (valid < 32) bits &= valid <= 0 ? 0u : (0xffffffffu >> (32 - valid));
-  return bits;
+  return m;
 }
 
 // ---- host: tensor maps ------------------------------------------------------------

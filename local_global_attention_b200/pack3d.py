@@ -30,7 +30,9 @@ class Params(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
                 ("B", "H", "head_dim", "Z", "Y", "X", "wz", "wy", "wx", "bz", "by", "bx")] + [
         ("rope_base", ctypes.c_float), ("scale", ctypes.c_float), ("dtype", ctypes.c_int32),
-        ("out_fp32", ctypes.c_int32), ("rope_mode", ctypes.c_int32), ("n_tokens", ctypes.c_int32)]
+        ("out_fp32", ctypes.c_int32), ("rope_mode", ctypes.c_int32), ("n_tokens", ctypes.c_int32),
+        ("Z_total", ctypes.c_int32), ("z_origin", ctypes.c_int32), ("own_lo", ctypes.c_int32),
+        ("own_hi", ctypes.c_int32)]
 
 
 class Index(ctypes.Structure):
@@ -115,15 +117,18 @@ def _check(status: int, what: str):
 
 def make_params(shape, dtype=None, scale: float = 0.0, out_fp32: bool = False) -> Params:
     """Params from any object with ``B, H, d, Z, Y, X, window, block, rope_base``
-    (and ``dtype`` "bf16"/"fp32" unless given, ``rope_mode`` 0 and ``n_tokens``
-    0 (a dense volume) unless set).  ``out_fp32`` makes the forward output fp32
-    for bf16 inputs."""
+    (and ``dtype`` "bf16"/"fp32" unless given, ``rope_mode`` 0, ``n_tokens`` 0
+    (a dense volume) and no z-slab (``Z_total``, ``z_origin``, ``own_lo``,
+    ``own_hi``) unless set).  ``out_fp32`` makes the forward output fp32 for
+    bf16 inputs."""
     dt = dtype if dtype is not None else getattr(shape, "dtype", "bf16")
     code = {"bf16": BF16, "fp32": FP32, torch.bfloat16: BF16, torch.float32: FP32}[dt]
     w, b = tuple(shape.window), tuple(shape.block)
     return Params(shape.B, shape.H, shape.d, shape.Z, shape.Y, shape.X, w[0], w[1], w[2],
                   b[0], b[1], b[2], float(shape.rope_base), float(scale), code, int(bool(out_fp32)),
-                  int(getattr(shape, "rope_mode", 0) or 0), int(getattr(shape, "n_tokens", 0) or 0))
+                  int(getattr(shape, "rope_mode", 0) or 0), int(getattr(shape, "n_tokens", 0) or 0),
+                  *(int(getattr(shape, f, 0) or 0) for f in ("Z_total", "z_origin", "own_lo",
+                                                             "own_hi")))
 
 
 def out_dtype(params: Params, like: torch.Tensor) -> torch.dtype:
@@ -180,7 +185,7 @@ class IndexBuffers:
         V = p.Z * p.Y * p.X
         N = p.n_tokens or V
         T = s.n_tiles
-        nb = (-(-p.Z // p.bz)) * (-(-p.Y // p.by)) * (-(-p.X // p.bx))
+        nb = (-(-(p.Z_total or p.Z) // p.bz)) * (-(-p.Y // p.by)) * (-(-p.X // p.bx))
         return {
             "vol": self._view("vol", p.B * V, torch.int32).view(p.B, V),
             "bcount": self._view("bcount", p.B * nb, torch.int32).view(p.B, nb),
@@ -219,8 +224,10 @@ def pack3d_block_summaries(params: Params, index: IndexBuffers, k, v, ksum=None,
                            stream=None):
     _need_cuda(k, v)
     B, N, H, d = _dims(params)
-    # blocks that do not divide the volume are cut at its edge: counts round up
-    nb = (-(-params.Z // params.bz)) * (-(-params.Y // params.by)) * (-(-params.X // params.bx))
+    # blocks that do not divide the volume are cut at its edge: counts round
+    # up; a z-slab uses the block grid of the whole volume
+    Zg = params.Z_total or params.Z
+    nb = (-(-Zg // params.bz)) * (-(-params.Y // params.by)) * (-(-params.X // params.bx))
     if ksum is None:
         ksum = torch.empty(B, H, nb, d, dtype=torch.float32, device=k.device)
     if vsum is None:
