@@ -153,7 +153,8 @@ typedef struct {
  *                               range, 2 = voxel held twice, 4 = a kernel
  *                               gave up a bounded device-side wait; [1]:
  *                               smallest offending flat token index b * N + i
- *   bcount   int32 [B][nb]      tokens held by each block
+ *   bcount   int32 [B][nb]      tokens held by each block (built for partly
+ *                               occupied volumes only)
  *   bocc     uint32 [B][ceil(nb/32)]  bit B % 32 of word B / 32: block B holds
  *                               at least one token (built for partly occupied
  *                               volumes only)

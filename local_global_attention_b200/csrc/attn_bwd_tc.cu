@@ -184,7 +184,9 @@ __device__ __forceinline__ void load_acc_row(uint32_t taddr, float (&v)[96]) {
   }
 }
 
-template <int ROLE>
+// PARTIAL: a partly occupied volume (empty voxels and blocks masked; compiled
+// out of the dense kernels).
+template <int ROLE, bool PARTIAL>
 __global__ void __launch_bounds__(NTHREADS, 1)
     k_bwd_tc(Geo g, pack3d_index ix, const __grid_constant__ BwdMaps maps, BwdArgs args) {
   if (ix.err[0]) return;
@@ -310,7 +312,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       }
       if (PENALTY && j < n_local) {
-        penalty_rows(sm.cp[s], g, tb, z, y, x, lane, ix.vol + (int64_t)b * g.V);
+        penalty_rows<PARTIAL>(sm.cp[s], g, tb, z, y, x, lane, ix.vol + (int64_t)b * g.V);
         fence_proxy_async_smem();
       }
       __syncwarp();
@@ -404,10 +406,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       rx = tb.x0 + lxi;
       vox = (((int64_t)bh * g.Z + rz) * g.Y + ry) * g.X + rx;
       // an empty voxel of a partly occupied volume is no row
-      if (active && !occupied(g, ix.vol, b, rz, ry, rx)) active = false;
+      if (PARTIAL && active && !occupied(g, ix.vol, b, rz, ry, rx)) active = false;
     } else {
       // an empty block has no summary
-      active = B0 + r < g.nb && (!g.partial || ix.bcount[(int64_t)b * g.nb + B0 + r] > 0);
+      active = B0 + r < g.nb && (!PARTIAL || ix.bcount[(int64_t)b * g.nb + B0 + r] > 0);
     }
     {
       // A1 row into this lane: channels 0-63 from half 0, 64-95 and the
@@ -509,7 +511,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           // partly occupied volume: the half's 32 query voxels that hold a token
           // (lane n looks up column n)
           uint32_t occ = 0xffffffffu;
-          if (g.partial) {
+          if (PARTIAL) {
             const int oz = qz, oy = y + (lane >> 4), ox = x + (lane & 15);
             const bool in = oz < g.Z && oy < g.Y && ox < g.X && occupied(g, ix.vol, b, oz, oy, ox);
             occ = __ballot_sync(0xffffffffu, in);
@@ -538,7 +540,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                                    (32 * hf))
                       : 0u;
         // empty blocks have no summary (Bs is a multiple of 32)
-        if (g.partial && Bs < g.nb) bits &= ix.bocc[(int64_t)b * ((g.nb + 31) / 32) + Bs / 32];
+        if (PARTIAL && Bs < g.nb) bits &= ix.bocc[(int64_t)b * ((g.nb + 31) / 32) + Bs / 32];
         use_bits = true;
         skip = __ballot_sync(0xffffffffu, bits != 0u) == 0u;
       }
@@ -631,7 +633,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           // the tokens the key's block holds (cut at the volume's edge; in a
           // partly occupied volume, the tokens present)
           const BlockExt be = block_ext(g, rz / g.bz, ry / g.by, rx / g.bx);
-          const int held = g.partial ? ix.bcount[(int64_t)b * g.nb + Bk] : be.ez * be.ey * be.ex;
+          const int held = PARTIAL ? ix.bcount[(int64_t)b * g.nb + Bk] : be.ez * be.ey * be.ex;
           const float inv = 1.f / (float)held;
           const float4* srow = reinterpret_cast<const float4*>(
               (hf == 0 ? args.dks : args.dvs) + (((int64_t)b * g.H + h) * g.nb + Bk) * D);
@@ -813,7 +815,7 @@ BwdWs bwd_layout(const Geo& g) {
 template <int ROLE>
 int launch_role(const Geo& g, const pack3d_index* idx, const BwdMaps& maps, const BwdArgs& args,
                 dim3 grid, cudaStream_t s) {
-  auto kern = k_bwd_tc<ROLE>;
+  auto kern = g.partial ? k_bwd_tc<ROLE, true> : k_bwd_tc<ROLE, false>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)SMEM_REQUEST) != cudaSuccess)
     return PACK3D_ERR_CUDA;

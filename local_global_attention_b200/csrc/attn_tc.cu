@@ -218,7 +218,9 @@ struct Maps {
   CUtensorMap ks, vs;  // [B*H][nb][96] bf16, box {32, 64, 1}
 };
 
-template <bool SUMMARY>
+// PARTIAL: a partly occupied volume (empty voxels masked; compiled out of the
+// dense kernel).
+template <bool SUMMARY, bool PARTIAL>
 __global__ void __launch_bounds__(NTHREADS, 2)
     k_forward_tc(Geo g, pack3d_index ix, const __nv_bfloat16* __restrict__ q,
                  const __grid_constant__ Maps maps, void* __restrict__ out_raw,
@@ -295,7 +297,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       }
       if (j < n_local) {
         // penalty rows of the chunk's keys (dz, dy, dx): key r = (dz * 2 + dy) * 16 + dx
-        penalty_rows(sm.kp[s], g, tb, tb.hz0 + BZK * zc, tb.hy0 + BYK * yc, tb.hx0 + BXK * xc,
+        penalty_rows<PARTIAL>(sm.kp[s], g, tb, tb.hz0 + BZK * zc, tb.hy0 + BYK * yc, tb.hx0 + BXK * xc,
                      lane, ix.vol + (int64_t)b * g.V);
         fence_proxy_async_smem();
         if (++xc == nxc) {
@@ -385,7 +387,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     const int cz = tb.z0 + lzi, cy = tb.y0 + lyi, cx = tb.x0 + lxi;
     int qi = 0;
     if (active) qi = ix.vol[(((int64_t)b * g.Z + cz) * g.Y + cy) * g.X + cx];
-    if (qi < 0) {  // an empty voxel of a partly occupied volume: no query
+    if (PARTIAL && qi < 0) {  // an empty voxel of a partly occupied volume: no query
       active = false;
       qi = 0;
     }
@@ -496,7 +498,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
         const uint64_t m64 = summary_mask64(g, B0, bzlo, bzhi, bylo, byhi, bxlo, bxhi);
         bits0 = (uint32_t)m64;
         bits1 = (uint32_t)(m64 >> 32);
-        if (g.partial) {
+        if (PARTIAL) {
           // empty blocks have no summary (B0 is a multiple of 64)
           const uint32_t* occ = ix.bocc + (int64_t)b * ((g.nb + 31) / 32) + B0 / 32;
           bits0 &= occ[0];
@@ -697,7 +699,8 @@ int launch_attention_tc(const Geo& g, const pack3d_index* idx, const void* q, vo
       !encode_bf16(&maps.vs, base + w.vs, 3, sdims, sbox))
     return PACK3D_ERR_CUDA;
   dim3 grid(g.nT, g.H, g.B);
-  auto kern = summaries ? k_forward_tc<true> : k_forward_tc<false>;
+  auto kern = summaries ? (g.partial ? k_forward_tc<true, true> : k_forward_tc<true, false>)
+                        : (g.partial ? k_forward_tc<false, true> : k_forward_tc<false, false>);
   // Two CTAs per SM: enough shared memory for both, and the largest carveout.
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)SMEM_REQUEST) != cudaSuccess ||

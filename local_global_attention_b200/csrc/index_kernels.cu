@@ -36,8 +36,10 @@ __global__ void k_scatter_coords(Geo g, const int16_t* __restrict__ coords, int3
   }
   int tile = ((z / TZ) * g.nTy + (y / TY)) * g.nTx + (x / TX);
   atomicAdd(&cnt[(int64_t)b * g.nT + tile], 1);
-  int blk = (((z + g.zo) / g.bz) * g.nby + (y / g.by)) * g.nbx + (x / g.bx);
-  atomicAdd(&bcount[(int64_t)b * g.nb + blk], 1);
+  if (g.partial) {  // block counts: only partly occupied volumes need them
+    int blk = (((z + g.zo) / g.bz) * g.nby + (y / g.by)) * g.nbx + (x / g.bx);
+    atomicAdd(&bcount[(int64_t)b * g.nb + blk], 1);
+  }
 }
 
 // Exclusive scan of n ints per row (one CTA per row), writes n + 1 values.
@@ -213,7 +215,8 @@ int launch_build_index(const Geo& g, const int16_t* coords, const pack3d_index* 
     return PACK3D_ERR_CUDA;
   if (cudaMemsetAsync(cnt, 0, sizeof(int32_t) * (size_t)g.B * g.nT, s) != cudaSuccess)
     return PACK3D_ERR_CUDA;
-  if (cudaMemsetAsync(idx->bcount, 0, sizeof(int32_t) * (size_t)g.B * g.nb, s) != cudaSuccess)
+  if (g.partial &&
+      cudaMemsetAsync(idx->bcount, 0, sizeof(int32_t) * (size_t)g.B * g.nb, s) != cudaSuccess)
     return PACK3D_ERR_CUDA;
   k_init_err<<<1, 1, 0, s>>>(idx->err);
   int nthr = 256;

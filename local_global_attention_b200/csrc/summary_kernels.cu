@@ -341,7 +341,9 @@ struct BulkSmem {
 static_assert(sizeof(float) * BS_TPS * BS_ITEMS * 32 <= sizeof(uint8_t) * BS_STAGES * BS_TPS * 2 * BS_ROW,
               "reduction buffer must fit the ring");
 
-template <bool STAGE>
+// PARTIAL: a partly occupied volume (empty voxels skipped; compiled out of the
+// dense kernels).
+template <bool STAGE, bool PARTIAL>
 __global__ void __launch_bounds__(BS_THREADS, 2) k_summaries_bulk(
     Geo g, const int32_t* __restrict__ vol, const float* __restrict__ rope,
     int32_t* __restrict__ err, const int32_t* __restrict__ bcount,
@@ -426,11 +428,11 @@ __global__ void __launch_bounds__(BS_THREADS, 2) k_summaries_bulk(
       const int64_t tok = __shfl_sync(0xffffffffu, cur, 8 * (r & 3) + (lane & 7));
       if (lane < ntok) sm.tok[s][lane] = (int32_t)tok;  // published by the arrive below
       // empty voxels (token -1, partly occupied volumes) are not copied
-      const int nload = __popc(__ballot_sync(0xffffffffu, lane < ntok && tok >= 0));
+      const int nload = PARTIAL ? __popc(__ballot_sync(0xffffffffu, lane < ntok && tok >= 0)) : ntok;
       __syncwarp();
       if (lane == 0) mbar_arrive_expect_tx(&sm.full[s], (uint32_t)nload * 2 * row_bytes);
       __syncwarp();
-      if (lane < ntok && tok >= 0) {
+      if (lane < ntok && (!PARTIAL || tok >= 0)) {
         bulk_load(sm.ring[s][lane][0], k + (((int64_t)b * g.N + tok) * g.H) * 96, row_bytes,
                   &sm.full[s]);
         bulk_load(sm.ring[s][lane][1], v + (((int64_t)b * g.N + tok) * g.H) * 96, row_bytes,
@@ -464,10 +466,11 @@ __global__ void __launch_bounds__(BS_THREADS, 2) k_summaries_bulk(
         const uint4* vr = reinterpret_cast<const uint4*>(sm.ring[s][grp][1] + h * 192);
         // an empty voxel (token -1, not copied) contributes zero rows: nothing
         // to the sums, zeros to the grid-order copies
-        const int tk = sm.tok[s][grp];
+        const int tk = PARTIAL || packed ? sm.tok[s][grp] : 0;
+        const bool held_tok = !PARTIAL || tk >= 0;
         const uint4 z4 = make_uint4(0, 0, 0, 0);
-        const uint4 ka = tk >= 0 ? kr[c1] : z4, kb = tk >= 0 ? kr[c2] : z4;
-        const uint4 va = tk >= 0 ? vr[c1] : z4, vb2 = tk >= 0 ? vr[c2] : z4;
+        const uint4 ka = held_tok ? kr[c1] : z4, kb = held_tok ? kr[c2] : z4;
+        const uint4 va = held_tok ? vr[c1] : z4, vb2 = held_tok ? vr[c2] : z4;
         const int ca = a == 0 ? cz : (a == 1 ? cy : cx);
         const float2* t = packed ? rope_row96(rope, g, 0, 0, max(tk, 0)) + j0
                                  : tab + (ca - base) * TABS96 + j0;
@@ -537,7 +540,7 @@ __global__ void __launch_bounds__(BS_THREADS, 2) k_summaries_bulk(
   const float* red = reinterpret_cast<const float*>(&sm.ring[0][0][0][0]);
   // mean over the tokens the block holds (0 for an empty block, and for a
   // block a z-slab does not own)
-  const int held = g.partial ? bcount[(int64_t)b * g.nb + blk] : cnt;
+  const int held = PARTIAL ? bcount[(int64_t)b * g.nb + blk] : cnt;
   const float inv_cnt = held > 0 && own ? 1.f / (float)held : 0.f;
   for (int o = tid; o < g.H * 2 * 96; o += BS_THREADS) {
     const int h = o / 192, which = (o / 96) % 2, ch = o % 96;
@@ -571,7 +574,7 @@ template <bool STAGE>
 int launch_bulk(const Geo& g, const pack3d_index* idx, const void* k, const void* v, float* ksum,
                 float* vsum, StageOut so, cudaStream_t s) {
   const size_t smem = sizeof(BulkSmem) + 128;
-  auto kern = k_summaries_bulk<STAGE>;
+  auto kern = g.partial ? k_summaries_bulk<STAGE, true> : k_summaries_bulk<STAGE, false>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return PACK3D_ERR_CUDA;

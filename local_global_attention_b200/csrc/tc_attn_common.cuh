@@ -75,7 +75,9 @@ __device__ __forceinline__ void onehot_words(int lz, int ly, int lx, uint32_t (&
 // tile `tb`: the chunk's box starts at (cz0, cy0, cx0); every lane of the warp
 // writes two rows.  Rows outside the volume, and (partly occupied volumes,
 // volb = the batch item's coordinate volume) rows at empty voxels, are masked
-// in every channel.
+// in every channel.  PARTIAL: the volume may be partly occupied (compiled out
+// of the dense kernels).
+template <bool PARTIAL>
 __device__ __forceinline__ void penalty_rows(uint8_t* dst, const Geo& g, const TileBox& tb,
                                              int cz0, int cy0, int cx0, int lane,
                                              const int32_t* volb) {
@@ -84,7 +86,7 @@ __device__ __forceinline__ void penalty_rows(uint8_t* dst, const Geo& g, const T
     const int r = lane + 32 * half;
     const int kz = cz0 + (r >> 5), ky = cy0 + ((r >> 4) & 1), kx = cx0 + (r & 15);
     bool inside = kz < g.Z && ky < g.Y && kx < g.X;
-    if (inside && g.partial) inside = volb[((int64_t)kz * g.Y + ky) * g.X + kx] >= 0;
+    if (PARTIAL && inside) inside = volb[((int64_t)kz * g.Y + ky) * g.X + kx] >= 0;
     uint32_t w[8];
 #pragma unroll
     for (int a = 0; a < 4; a += 2) {
