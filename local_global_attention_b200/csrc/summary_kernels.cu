@@ -335,6 +335,7 @@ struct BulkSmem {
   uint8_t ring[BS_STAGES][BS_TPS][2][BS_ROW];  // reused for the final reduction
   float2 tab[TAB96 * TABS96];
   int32_t tok[BS_STAGES][BS_TPS];  // packed index of each slot's token
+  int4 crd[BS_STAGES][BS_TPS];     // (z, y, x) of each slot's voxel
   uint64_t full[BS_STAGES], empty[BS_STAGES];
   int32_t abort;
 };
@@ -426,7 +427,14 @@ __global__ void __launch_bounds__(BS_THREADS, 2) k_summaries_bulk(
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       const int ntok = min(BS_TPS, cnt - r * BS_TPS);
       const int64_t tok = __shfl_sync(0xffffffffu, cur, 8 * (r & 3) + (lane & 7));
-      if (lane < ntok) sm.tok[s][lane] = (int32_t)tok;  // published by the arrive below
+      if (lane < ntok) {
+        // published by the arrive below: the slot's token and voxel, so the
+        // consumers need no division to find the voxel
+        sm.tok[s][lane] = (int32_t)tok;
+        int cz, cy, cx;
+        voxel(r * BS_TPS + lane, cz, cy, cx);
+        sm.crd[s][lane] = make_int4(cz, cy, cx, 0);
+      }
       // empty voxels (token -1, partly occupied volumes) are not copied
       const int nload = PARTIAL ? __popc(__ballot_sync(0xffffffffu, lane < ntok && tok >= 0)) : ntok;
       __syncwarp();
@@ -460,8 +468,8 @@ __global__ void __launch_bounds__(BS_THREADS, 2) k_summaries_bulk(
         break;
       const int e = r * BS_TPS + grp;
       if (live && e < cnt) {
-        int cz, cy, cx;
-        voxel(e, cz, cy, cx);
+        const int4 cc = sm.crd[s][grp];
+        const int cz = cc.x, cy = cc.y, cx = cc.z;
         const uint4* kr = reinterpret_cast<const uint4*>(sm.ring[s][grp][0] + h * 192);
         const uint4* vr = reinterpret_cast<const uint4*>(sm.ring[s][grp][1] + h * 192);
         // an empty voxel (token -1, not copied) contributes zero rows: nothing
