@@ -123,10 +123,13 @@ typedef struct {
                         that a sum over the ranks (an all-reduce) gives every
                         block's summary.  A query's window must lie inside the
                         call's volume: rz halo planes on each side of the owned
-                        planes where the whole volume continues.  Forward on the
+                        planes where the whole volume continues.  The
                         tensor-core path only (bf16, head_dim 96), dense
                         volumes, axial RoPE; others report
-                        PACK3D_ERR_UNSUPPORTED. */
+                        PACK3D_ERR_UNSUPPORTED.  The backward of a slab runs
+                        as the two calls of pack3d_backward_summary_grads
+                        with an all-reduce between them (pack3d_backward
+                        reports PACK3D_ERR_UNSUPPORTED for a slab). */
   int32_t z_origin;  /* global plane of local plane 0 (sharding; 0 otherwise) */
   int32_t own_lo, own_hi; /* owned local planes (sharding; both 0 otherwise) */
 } pack3d_params;
@@ -271,6 +274,48 @@ PACK3D_API int pack3d_backward(const pack3d_params* p, const pack3d_index* idx, 
                     const void* v, const void* out, const float* lse, const void* dout, void* dq,
                     void* dk, void* dv, void* workspace, size_t workspace_bytes,
                     pack3d_stream_t stream);
+
+/* The backward of pack3d_backward in two calls, for a volume cut into
+ * z-slabs (params with Z_total > 0).  The gradient of a block summary is a sum
+ * over every query of the volume whose window misses the block, so on a slab it
+ * is a partial sum: the caller adds the ranks' partial sums (an all-reduce)
+ * between the two calls.  The operator's definition is the one the abstract
+ * and the method section of the paper give (global branch = attention to the
+ * mean-pooled key and value of each block); the split is this library's.
+ *
+ * pack3d_backward_summary_grads stages q, k, v, out, lse and dout into the
+ * workspace and writes dks, dvs [B, H, nb, head_dim] fp32 (the blocks of the
+ * whole volume, nb = pack3d_params.nb order): the gradients of sum(dout * out)
+ * with respect to the block summaries, over the call's owned queries (all
+ * queries unless the call is a slab).  ksum, vsum [B, H, nb, head_dim] fp32:
+ * the summaries the forward used - for a slab the all-reduced summaries of the
+ * whole volume, required; otherwise NULL (both) to compute them from k and v
+ * here.  A slab's call needs q, k, v, out, lse and dout of its halo planes too
+ * (the neighbours' tokens: their queries reach the owned keys).
+ *
+ * pack3d_backward_from_summary_grads then writes dq, dk, dv for the call's
+ * owned tokens (other rows are left untouched), from the workspace left by
+ * the first call (same params, index and workspace, unmodified in between)
+ * and the summary gradients of the whole volume (for a slab, the sum over
+ * ranks).  The two calls with no exchange between them give exactly
+ * pack3d_backward's results.
+ *
+ * workspace: at least pack3d_backward_workspace_bytes(p) bytes, 256-byte
+ * aligned (PACK3D_ERR_ARG otherwise).  Built on the tensor-core path only (bf16,
+ * head_dim 96); other shapes and slabs of partly occupied volumes or of the
+ * packed RoPE mode report PACK3D_ERR_UNSUPPORTED.  Fixed-order reductions, no
+ * floating-point atomics. */
+PACK3D_API int pack3d_backward_summary_grads(const pack3d_params* p, const pack3d_index* idx,
+                                             const void* q, const void* k, const void* v,
+                                             const void* out, const float* lse, const void* dout,
+                                             const float* ksum, const float* vsum, float* dks,
+                                             float* dvs, void* workspace, size_t workspace_bytes,
+                                             pack3d_stream_t stream);
+PACK3D_API int pack3d_backward_from_summary_grads(const pack3d_params* p, const pack3d_index* idx,
+                                                  const float* dks, const float* dvs,
+                                                  void* workspace, size_t workspace_bytes,
+                                                  void* dq, void* dk, void* dv,
+                                                  pack3d_stream_t stream);
 
 /* Size of the device scratch array behind pack3d_backward_noalloc. */
 #define PACK3D_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)

@@ -220,8 +220,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int rt = blockIdx.x % nrt;
     split = blockIdx.x / nrt;
     B0 = rt * 128;
-    cz0 = cy0 = cx0 = 0;
-    const int nzc = (g.Z + BZK - 1) / BZK;
+    // the queries of the owned planes (all planes unless the call is a z-slab)
+    cz0 = g.own_lo;
+    cy0 = cx0 = 0;
+    const int nzc = (g.own_hi - g.own_lo + BZK - 1) / BZK;
     nyc = (g.Y + BYK - 1) / BYK;
     nxc = (g.X + BXK - 1) / BXK;
     const int total = nzc * nyc * nxc;
@@ -400,7 +402,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     int64_t vox = 0;  // grid index of the row (tile roles)
     if (TILE_ROWS) {
       lane_pos(r, lzi, lyi, lxi);
-      active = lzi < tb.lz && lyi < tb.ly && lxi < tb.lx;
+      active = lzi < tb.lz && lyi < tb.ly && lxi < tb.lx && tb.z0 + lzi >= g.own_lo &&
+               tb.z0 + lzi < g.own_hi;  // (a z-slab gives its owned planes only)
       rz = tb.z0 + lzi;
       ry = tb.y0 + lyi;
       rx = tb.x0 + lxi;
@@ -463,7 +466,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     WarpExtent we{};
     if (TILE_ROWS) we = warp_extent(active, rz, ry, rx);
     // DQ summary chunks: the box of blocks this query's window touches
-    const int bzlo = max(rz - g.rz, 0) / g.bz, bzhi = min(rz + g.rz, g.Z - 1) / g.bz;
+    // (global planes: the block grid of a z-slab is the whole volume's)
+    const int bzlo = max(rz + g.zo - g.rz, 0) / g.bz, bzhi = min(rz + g.zo + g.rz, g.Zt - 1) / g.bz;
     const int bylo = max(ry - g.ry, 0) / g.by, byhi = min(ry + g.ry, g.Y - 1) / g.by;
     const int bxlo = max(rx - g.rx, 0) / g.bx, bxhi = min(rx + g.rx, g.X - 1) / g.bx;
     // DSUM: the range of query coordinates whose window meets this row's block
@@ -471,8 +475,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (ROLE == ROLE_DSUM) {
       const int Br = B0 + r;
       const int bz = Br / (g.nby * g.nbx), by = (Br / g.nbx) % g.nby, bx = Br % g.nbx;
-      mzlo = bz * g.bz - g.rz;
-      mzhi = bz * g.bz + g.bz - 1 + g.rz;
+      mzlo = bz * g.bz - g.zo - g.rz;  // local planes of a z-slab
+      mzhi = bz * g.bz - g.zo + g.bz - 1 + g.rz;
       mylo = by * g.by - g.ry;
       myhi = by * g.by + g.by - 1 + g.ry;
       mxlo = bx * g.bx - g.rx;
@@ -516,7 +520,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const bool in = oz < g.Z && oy < g.Y && ox < g.X && occupied(g, ix.vol, b, oz, oy, ox);
             occ = __ballot_sync(0xffffffffu, in);
           }
-          if (active && qz < g.Z) {
+          if (active && qz < g.own_hi) {
             const bool zin = qz >= mzlo && qz <= mzhi;
             const uint32_t xs = bit_range(0, min(BXK, g.X - x) - 1);  // in the volume
             const int elo = max(mxlo - x, 0), ehi = min(mxhi - x, BXK - 1);
@@ -629,10 +633,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         load_acc_row(tbase + lane_base + (hf == 0 ? COL_ACC1 : COL_ACC2), v);
         if (active) {
           const int kj = ix.vol[((int64_t)b * g.Z + rz) * g.Y * g.X + (int64_t)ry * g.X + rx];
-          const int Bk = ((rz / g.bz) * g.nby + ry / g.by) * g.nbx + rx / g.bx;
+          const int Bk = (((rz + g.zo) / g.bz) * g.nby + ry / g.by) * g.nbx + rx / g.bx;
           // the tokens the key's block holds (cut at the volume's edge; in a
           // partly occupied volume, the tokens present)
-          const BlockExt be = block_ext(g, rz / g.bz, ry / g.by, rx / g.bx);
+          const BlockExt be = block_ext(g, (rz + g.zo) / g.bz, ry / g.by, rx / g.bx);
           const int held = PARTIAL ? ix.bcount[(int64_t)b * g.nb + Bk] : be.ez * be.ey * be.ex;
           const float inv = 1.f / (float)held;
           const float4* srow = reinterpret_cast<const float4*>(
@@ -781,7 +785,8 @@ struct BwdWs {
 // most one chunk each, at most 64.
 int dsum_splits(const Geo& g) {
   const int nrt = (g.nb + 127) / 128;
-  const int64_t chunks = (int64_t)((g.Z + 1) / 2) * ((g.Y + 1) / 2) * ((g.X + 15) / 16);
+  const int64_t chunks =
+      (int64_t)((g.own_hi - g.own_lo + 1) / 2) * ((g.Y + 1) / 2) * ((g.X + 15) / 16);
   const int64_t groups = (int64_t)g.B * g.H * nrt;
   int64_t s = (148 + groups - 1) / groups;
   s = std::min<int64_t>(s, std::min<int64_t>(chunks, 64));
@@ -832,9 +837,64 @@ size_t backward_tc_workspace_bytes(const Geo& g) {
   return backward_tc_supported(g) ? bwd_layout(g).total : 0;
 }
 
-int launch_backward_tc(const Geo& g, const pack3d_index* idx, const void* q, const void* k,
-                       const void* v, const void* out, const float* lse, const void* dout,
-                       void* dq, void* dk, void* dv, void* workspace, cudaStream_t s) {
+namespace {
+
+// The three roles' tensor maps over a staged workspace.
+struct RoleMaps {
+  BwdMaps q, k, s;  // dq, dk/dv, summary gradients
+};
+
+bool encode_role_maps(const Geo& g, uint8_t* base, const BwdWs& w, RoleMaps& m) {
+  const uint64_t BH = (uint64_t)g.B * g.H;
+  const uint64_t vdims[5] = {(uint64_t)D, (uint64_t)g.X, (uint64_t)g.Y, (uint64_t)g.Z, BH};
+  const uint32_t cbox[5] = {32, BXK, BYK, BZK, 1};
+  const uint32_t rbox[5] = {32, TX, 2, 2, 1};
+  const uint64_t sdims[3] = {(uint64_t)D, (uint64_t)g.nb, BH};
+  const uint32_t scbox[3] = {32, KCH, 1};
+  const uint32_t srbox[3] = {32, 128, 1};
+  const uint64_t tdims[5] = {4, (uint64_t)g.X, (uint64_t)g.Y, (uint64_t)g.Z, BH};
+  const uint32_t tbox[5] = {4, BXK, BYK, BZK, 1};
+  m = RoleMaps{};
+  bool ok = true;
+  // summary role: columns q~ / dO, stats; rows kbar (a1), vbar (A2)
+  ok &= encode_bf16(&m.s.c1, base + w.qg, 5, vdims, cbox);
+  ok &= encode_bf16(&m.s.c2, base + w.dog, 5, vdims, cbox);
+  ok &= encode_map(&m.s.st, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base + w.stat, 5, tdims, tbox,
+                   CU_TENSOR_MAP_SWIZZLE_NONE);
+  ok &= encode_bf16(&m.s.a2, base + w.vsb, 3, sdims, srbox);
+  m.s.c1s = m.s.c1;
+  m.s.c2s = m.s.c2;
+  // dk / dv role: columns q~ / dO, stats; rows k~ (a1), v (A2)
+  m.k = m.s;
+  ok &= encode_bf16(&m.k.a2, base + w.vg, 5, vdims, rbox);
+  // dq role: columns k~ / v then kbar / vbar; rows q~ (a1), dO (A2)
+  ok &= encode_bf16(&m.q.c1, base + w.kg, 5, vdims, cbox);
+  ok &= encode_bf16(&m.q.c2, base + w.vg, 5, vdims, cbox);
+  ok &= encode_bf16(&m.q.c1s, base + w.ksb, 3, sdims, scbox);
+  ok &= encode_bf16(&m.q.c2s, base + w.vsb, 3, sdims, scbox);
+  ok &= encode_bf16(&m.q.a2, base + w.dog, 5, vdims, rbox);
+  m.q.st = m.s.st;
+  return ok;
+}
+
+// fp32 summaries -> the bf16 copies the MMAs read.
+__global__ void k_bwd_summary_copies(const float* __restrict__ ks, const float* __restrict__ vs,
+                                     __nv_bfloat16* __restrict__ kb, __nv_bfloat16* __restrict__ vb,
+                                     int64_t n, const int32_t* __restrict__ err) {
+  if (err[0]) return;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    kb[i] = __float2bfloat16_rn(ks[i]);
+    vb[i] = __float2bfloat16_rn(vs[i]);
+  }
+}
+
+}  // namespace
+
+int backward_tc_summary_grads(const Geo& g, const pack3d_index* idx, const void* q, const void* k,
+                              const void* v, const void* out, const float* lse, const void* dout,
+                              const float* ksum, const float* vsum, float* dks, float* dvs,
+                              void* workspace, cudaStream_t s) {
   const BwdWs w = bwd_layout(g);
   uint8_t* base = static_cast<uint8_t*>(workspace);
   auto bf = [&](size_t off) { return reinterpret_cast<__nv_bfloat16*>(base + off); };
@@ -843,6 +903,15 @@ int launch_backward_tc(const Geo& g, const pack3d_index* idx, const void* q, con
   int rc = launch_block_summaries_staged(g, idx, k, v, f32(w.ksum), f32(w.vsum), base + w.kg,
                                          base + w.vg, base + w.ksb, base + w.vsb, s);
   if (rc) return rc;
+  if (ksum) {
+    // given summaries (the whole volume's, e.g. summed over z-slabs) replace
+    // the ones computed from this call's tokens
+    const int64_t n = (int64_t)g.B * g.H * g.nb * D;
+    k_bwd_summary_copies<<<(unsigned)std::min<int64_t>((n + 255) / 256, 148 * 8), 256, 0, s>>>(
+        ksum, vsum, bf(w.ksb), bf(w.vsb), n, idx->err);
+    count_launches(1);
+    if ((rc = cuda_status(cudaGetLastError()))) return rc;
+  }
   {
     dim3 grid((g.X + STAGE_XS - 1) / STAGE_XS, g.Z * g.Y, g.B);
     if (g.out_fp32)
@@ -857,77 +926,61 @@ int launch_backward_tc(const Geo& g, const pack3d_index* idx, const void* q, con
     count_launches(1);
     if ((rc = cuda_status(cudaGetLastError()))) return rc;
   }
-  const uint64_t BH = (uint64_t)g.B * g.H;
-  const uint64_t vdims[5] = {(uint64_t)D, (uint64_t)g.X, (uint64_t)g.Y, (uint64_t)g.Z, BH};
-  const uint32_t cbox[5] = {32, BXK, BYK, BZK, 1};
-  const uint32_t rbox[5] = {32, TX, 2, 2, 1};
-  const uint64_t sdims[3] = {(uint64_t)D, (uint64_t)g.nb, BH};
-  const uint32_t scbox[3] = {32, KCH, 1};
-  const uint32_t srbox[3] = {32, 128, 1};
-  const uint64_t tdims[5] = {4, (uint64_t)g.X, (uint64_t)g.Y, (uint64_t)g.Z, BH};
-  const uint32_t tbox[5] = {4, BXK, BYK, BZK, 1};
-  BwdMaps mq{}, mk{}, ms{};
-  bool okm = true;
-  // summary role: columns q~ / dO, stats; rows kbar (a1), vbar (A2)
-  okm &= encode_bf16(&ms.c1, base + w.qg, 5, vdims, cbox);
-  okm &= encode_bf16(&ms.c2, base + w.dog, 5, vdims, cbox);
-  okm &= encode_map(&ms.st, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base + w.stat, 5, tdims, tbox,
-                    CU_TENSOR_MAP_SWIZZLE_NONE);
-  okm &= encode_bf16(&ms.a2, base + w.vsb, 3, sdims, srbox);
-  ms.c1s = ms.c1;
-  ms.c2s = ms.c2;
-  // dk / dv role: columns q~ / dO, stats; rows k~ (a1), v (A2)
-  mk.c1 = ms.c1;
-  mk.c2 = ms.c2;
-  mk.st = ms.st;
-  mk.c1s = ms.c1;
-  mk.c2s = ms.c2;
-  okm &= encode_bf16(&mk.a2, base + w.vg, 5, vdims, rbox);
-  // dq role: columns k~ / v then kbar / vbar; rows q~ (a1), dO (A2)
-  okm &= encode_bf16(&mq.c1, base + w.kg, 5, vdims, cbox);
-  okm &= encode_bf16(&mq.c2, base + w.vg, 5, vdims, cbox);
-  okm &= encode_bf16(&mq.c1s, base + w.ksb, 3, sdims, scbox);
-  okm &= encode_bf16(&mq.c2s, base + w.vsb, 3, sdims, scbox);
-  okm &= encode_bf16(&mq.a2, base + w.dog, 5, vdims, rbox);
-  mq.st = ms.st;
-  if (!okm) return PACK3D_ERR_CUDA;
-
-  const float4* stat = reinterpret_cast<const float4*>(base + w.stat);
+  RoleMaps m;
+  if (!encode_role_maps(g, base, w, m)) return PACK3D_ERR_CUDA;
   // summary gradients, then their reduction in split order
   const int nsplit = dsum_splits(g);
-  {
-    BwdArgs a{};
-    a.a1 = bf(w.ksb);
-    a.stat = stat;
-    a.part = f32(w.part);
-    a.nsplit = nsplit;
-    const int nrt = (g.nb + 127) / 128;
-    if ((rc = launch_role<ROLE_DSUM>(g, idx, ms, a, dim3(nrt * nsplit, g.H, g.B), s))) return rc;
-    const int64_t n = (int64_t)g.B * g.H * g.nb * D;
-    k_bwd_sum_reduce<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(g, idx->err, nsplit,
-                                                                  f32(w.part), f32(w.dks),
-                                                                  f32(w.dvs));
-    count_launches(1);
-    if ((rc = cuda_status(cudaGetLastError()))) return rc;
-  }
+  BwdArgs a{};
+  a.a1 = bf(w.ksb);
+  a.stat = reinterpret_cast<const float4*>(base + w.stat);
+  a.part = f32(w.part);
+  a.nsplit = nsplit;
+  const int nrt = (g.nb + 127) / 128;
+  if ((rc = launch_role<ROLE_DSUM>(g, idx, m.s, a, dim3(nrt * nsplit, g.H, g.B), s))) return rc;
+  const int64_t n = (int64_t)g.B * g.H * g.nb * D;
+  k_bwd_sum_reduce<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(g, idx->err, nsplit, f32(w.part),
+                                                                dks, dvs);
+  count_launches(1);
+  return cuda_status(cudaGetLastError());
+}
+
+int backward_tc_from_summary_grads(const Geo& g, const pack3d_index* idx, const float* dks,
+                                   const float* dvs, void* dq, void* dk, void* dv,
+                                   void* workspace, cudaStream_t s) {
+  const BwdWs w = bwd_layout(g);
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  auto bf = [&](size_t off) { return reinterpret_cast<__nv_bfloat16*>(base + off); };
+  RoleMaps m;
+  if (!encode_role_maps(g, base, w, m)) return PACK3D_ERR_CUDA;
+  const float4* stat = reinterpret_cast<const float4*>(base + w.stat);
+  int rc;
   {
     BwdArgs a{};
     a.a1 = bf(w.qg);
     a.stat = stat;
     a.out1 = (__nv_bfloat16*)dq;
-    if ((rc = launch_role<ROLE_DQ>(g, idx, mq, a, dim3(g.nT, g.H, g.B), s))) return rc;
+    if ((rc = launch_role<ROLE_DQ>(g, idx, m.q, a, dim3(g.nT, g.H, g.B), s))) return rc;
   }
-  {
-    BwdArgs a{};
-    a.a1 = bf(w.kg);
-    a.stat = stat;
-    a.out1 = (__nv_bfloat16*)dk;
-    a.out2 = (__nv_bfloat16*)dv;
-    a.dks = f32(w.dks);
-    a.dvs = f32(w.dvs);
-    if ((rc = launch_role<ROLE_DKDV>(g, idx, mk, a, dim3(g.nT, g.H, g.B), s))) return rc;
-  }
-  return PACK3D_OK;
+  BwdArgs a{};
+  a.a1 = bf(w.kg);
+  a.stat = stat;
+  a.out1 = (__nv_bfloat16*)dk;
+  a.out2 = (__nv_bfloat16*)dv;
+  a.dks = dks;
+  a.dvs = dvs;
+  return launch_role<ROLE_DKDV>(g, idx, m.k, a, dim3(g.nT, g.H, g.B), s);
+}
+
+int launch_backward_tc(const Geo& g, const pack3d_index* idx, const void* q, const void* k,
+                       const void* v, const void* out, const float* lse, const void* dout,
+                       void* dq, void* dk, void* dv, void* workspace, cudaStream_t s) {
+  const BwdWs w = bwd_layout(g);
+  float* dks = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.dks);
+  float* dvs = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.dvs);
+  int rc = backward_tc_summary_grads(g, idx, q, k, v, out, lse, dout, nullptr, nullptr, dks, dvs,
+                                     workspace, s);
+  if (rc) return rc;
+  return backward_tc_from_summary_grads(g, idx, dks, dvs, dq, dk, dv, workspace, s);
 }
 
 }  // namespace p3d

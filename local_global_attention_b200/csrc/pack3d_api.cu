@@ -165,7 +165,8 @@ int backward_call(const pack3d_params* p, const pack3d_index* idx, const void* q
   if ((rc = check_index(g, idx))) return rc;
   if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv || !workspace)
     return PACK3D_ERR_ARG;
-  if (g.sharded) return PACK3D_ERR_UNSUPPORTED;  // z-slabs: the forward only
+  // z-slabs: the summary gradients need an exchange (the two-call form)
+  if (g.sharded) return PACK3D_ERR_UNSUPPORTED;
   if (((uintptr_t)workspace & 255) || ws_bytes < backward_workspace_bytes(g, simt))
     return PACK3D_ERR_ARG;
   if (!simt && backward_tc_supported(g))
@@ -329,6 +330,49 @@ int pack3d_backward(const pack3d_params* p, const pack3d_index* idx, const void*
                     pack3d_stream_t stream) {
   return backward_call(p, idx, q, k, v, out, lse, dout, dq, dk, dv, workspace, workspace_bytes,
                        false, (cudaStream_t)stream);
+}
+
+namespace {
+
+int backward_phase_check(const pack3d_params* p, const pack3d_index* idx, void* workspace,
+                         size_t workspace_bytes, Geo& g) {
+  int rc = make_geo(p, &g);
+  if (rc) return rc;
+  if ((rc = check_index(g, idx))) return rc;
+  if (!workspace || ((uintptr_t)workspace & 255)) return PACK3D_ERR_ARG;
+  if (!backward_tc_supported(g)) return PACK3D_ERR_UNSUPPORTED;
+  if ((rc = shard_supported(g))) return rc;
+  if (workspace_bytes < backward_tc_workspace_bytes(g)) return PACK3D_ERR_ARG;
+  return PACK3D_OK;
+}
+
+}  // namespace
+
+int pack3d_backward_summary_grads(const pack3d_params* p, const pack3d_index* idx, const void* q,
+                                  const void* k, const void* v, const void* out, const float* lse,
+                                  const void* dout, const float* ksum, const float* vsum,
+                                  float* dks, float* dvs, void* workspace, size_t workspace_bytes,
+                                  pack3d_stream_t stream) {
+  Geo g;
+  int rc = backward_phase_check(p, idx, workspace, workspace_bytes, g);
+  if (rc) return rc;
+  if (!q || !k || !v || !out || !lse || !dout || !dks || !dvs || (!ksum) != (!vsum) ||
+      (g.sharded && !ksum))
+    return PACK3D_ERR_ARG;
+  return backward_tc_summary_grads(g, idx, q, k, v, out, lse, dout, ksum, vsum, dks, dvs,
+                                   workspace, (cudaStream_t)stream);
+}
+
+int pack3d_backward_from_summary_grads(const pack3d_params* p, const pack3d_index* idx,
+                                       const float* dks, const float* dvs, void* workspace,
+                                       size_t workspace_bytes, void* dq, void* dk, void* dv,
+                                       pack3d_stream_t stream) {
+  Geo g;
+  int rc = backward_phase_check(p, idx, workspace, workspace_bytes, g);
+  if (rc) return rc;
+  if (!dks || !dvs || !dq || !dk || !dv) return PACK3D_ERR_ARG;
+  return backward_tc_from_summary_grads(g, idx, dks, dvs, dq, dk, dv, workspace,
+                                        (cudaStream_t)stream);
 }
 
 uint64_t pack3d_kernel_launches(void) { return g_kernel_launches.load(std::memory_order_relaxed); }

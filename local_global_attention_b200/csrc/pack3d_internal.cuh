@@ -181,6 +181,17 @@ size_t backward_tc_workspace_bytes(const Geo& g);
 int launch_backward_tc(const Geo& g, const pack3d_index* idx, const void* q, const void* k,
                        const void* v, const void* out, const float* lse, const void* dout,
                        void* dq, void* dk, void* dv, void* workspace, cudaStream_t s);
+// The two halves of the tensor-core backward: staging and the summary
+// gradients over the call's (owned) queries (ksum, vsum: given summaries of the
+// whole volume to use, or null for the ones computed from the call's tokens),
+// then dq and dk/dv from the same workspace and the given summary gradients.
+int backward_tc_summary_grads(const Geo& g, const pack3d_index* idx, const void* q, const void* k,
+                              const void* v, const void* out, const float* lse, const void* dout,
+                              const float* ksum, const float* vsum, float* dks, float* dvs,
+                              void* workspace, cudaStream_t s);
+int backward_tc_from_summary_grads(const Geo& g, const pack3d_index* idx, const float* dks,
+                                   const float* dvs, void* dq, void* dk, void* dv,
+                                   void* workspace, cudaStream_t s);
 // The backward pack3d_backward runs: the tensor-core one where it applies,
 // else the CUDA-core one (or, with simt, always the CUDA-core one).
 size_t backward_workspace_bytes(const Geo& g, bool simt = false);

@@ -22,7 +22,8 @@ OK, ERR_ARG, ERR_COORDS, ERR_CUDA, ERR_TIMEOUT, ERR_UNSUPPORTED = 0, -1, -2, -3,
 EXPORTS = ("pack3d_index_bytes", "pack3d_index_init", "pack3d_build_index", "pack3d_index_check",
            "pack3d_block_summaries", "pack3d_forward_workspace_bytes", "pack3d_forward",
            "pack3d_window_forward", "pack3d_stage_kv", "pack3d_forward_staged",
-           "pack3d_backward_workspace_bytes", "pack3d_backward", "pack3d_backward_noalloc",
+           "pack3d_backward_workspace_bytes", "pack3d_backward", "pack3d_backward_summary_grads",
+           "pack3d_backward_from_summary_grads", "pack3d_backward_noalloc",
            "pack3d_kernel_launches", "pack3d_strerror")
 
 
@@ -89,6 +90,11 @@ def load(build_if_missing: bool = True):
         lib.pack3d_backward_workspace_bytes.restype = ctypes.c_size_t
         lib.pack3d_backward.argtypes = [P(Params), P(Index), vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                         vp, ctypes.c_size_t, vp]
+        lib.pack3d_backward_summary_grads.argtypes = [P(Params), P(Index), vp, vp, vp, vp, vp,
+                                                      vp, vp, vp, vp, vp, vp, ctypes.c_size_t,
+                                                      vp]
+        lib.pack3d_backward_from_summary_grads.argtypes = [P(Params), P(Index), vp, vp, vp,
+                                                           ctypes.c_size_t, vp, vp, vp, vp]
         lib.pack3d_backward_noalloc.argtypes = [P(Params), P(Index), vp, vp, vp, vp, vp, vp, vp,
                                                 vp, vp, vp]
         lib.pack3d_kernel_launches.argtypes = []
@@ -220,14 +226,18 @@ def _dims(params):
     return params.B, params.n_tokens or params.Z * params.Y * params.X, params.H, params.head_dim
 
 
+def n_blocks(params: Params) -> int:
+    """Blocks of the volume (a z-slab: of the whole volume); blocks that do not
+    divide the volume are cut at its edge, so the counts round up."""
+    Zg = params.Z_total or params.Z
+    return (-(-Zg // params.bz)) * (-(-params.Y // params.by)) * (-(-params.X // params.bx))
+
+
 def pack3d_block_summaries(params: Params, index: IndexBuffers, k, v, ksum=None, vsum=None,
                            stream=None):
     _need_cuda(k, v)
     B, N, H, d = _dims(params)
-    # blocks that do not divide the volume are cut at its edge: counts round
-    # up; a z-slab uses the block grid of the whole volume
-    Zg = params.Z_total or params.Z
-    nb = (-(-Zg // params.bz)) * (-(-params.Y // params.by)) * (-(-params.X // params.bx))
+    nb = n_blocks(params)
     if ksum is None:
         ksum = torch.empty(B, H, nb, d, dtype=torch.float32, device=k.device)
     if vsum is None:
@@ -333,6 +343,43 @@ def pack3d_backward(params: Params, index: IndexBuffers, q, k, v, out, lse, dout
                                   _ptr(dk), _ptr(dv), _ptr(workspace),
                                   ctypes.c_size_t(workspace.numel() * workspace.element_size()),
                                   _stream(stream)), "pack3d_backward")
+    return dq, dk, dv
+
+
+def pack3d_backward_summary_grads(params: Params, index: IndexBuffers, q, k, v, out, lse, dout,
+                                  ksum=None, vsum=None, dks=None, dvs=None, workspace=None,
+                                  stream=None):
+    """First half of the two-call backward: stages the inputs into `workspace`
+    (allocated when None) and returns (dks, dvs, workspace), the summary
+    gradients [B, H, nb, d] fp32 over the call's owned queries."""
+    _need_cuda(q, k, v, out, lse, dout)
+    B, N, H, d = _dims(params)
+    nb = n_blocks(params)
+    dks = torch.empty(B, H, nb, d, dtype=torch.float32, device=q.device) if dks is None else dks
+    dvs = torch.empty(B, H, nb, d, dtype=torch.float32, device=q.device) if dvs is None else dvs
+    if workspace is None:
+        workspace = torch.empty(pack3d_backward_workspace_bytes(params), dtype=torch.uint8,
+                                device=q.device)
+    _need_cuda(dks, dvs, workspace)
+    if ksum is not None:
+        _need_cuda(ksum, vsum)
+    _check(load().pack3d_backward_summary_grads(
+        ctypes.byref(params), ctypes.byref(index.struct), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
+        _ptr(lse), _ptr(dout), _ptr(ksum), _ptr(vsum), _ptr(dks), _ptr(dvs), _ptr(workspace),
+        ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(stream)),
+        "pack3d_backward_summary_grads")
+    return dks, dvs, workspace
+
+
+def pack3d_backward_from_summary_grads(params: Params, index: IndexBuffers, dks, dvs, workspace,
+                                       dq, dk, dv, stream=None):
+    """Second half: dq, dk, dv of the owned tokens from the staged workspace and
+    the summary gradients of the whole volume."""
+    _need_cuda(dks, dvs, workspace, dq, dk, dv)
+    _check(load().pack3d_backward_from_summary_grads(
+        ctypes.byref(params), ctypes.byref(index.struct), _ptr(dks), _ptr(dvs), _ptr(workspace),
+        ctypes.c_size_t(workspace.numel() * workspace.element_size()), _ptr(dq), _ptr(dk),
+        _ptr(dv), _stream(stream)), "pack3d_backward_from_summary_grads")
     return dq, dk, dv
 
 

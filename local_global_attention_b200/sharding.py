@@ -20,6 +20,14 @@ planes, and outputs are written for the owned tokens only.  The window of an
 owned query lies inside the held planes, and the axial RoPE logits depend only
 on coordinate differences, so the owned outputs equal the unsharded ones.
 
+The backward (sharded_backward) needs one more exchange.  The gradient of a
+block summary sums over every query of the volume, so each rank computes the
+partial sum over its owned queries (pack3d_backward_summary_grads) and an
+all-reduce adds them; the rank then finishes dq, dk, dv of its owned tokens
+(pack3d_backward_from_summary_grads).  The keys of a slab also receive
+gradient from the queries in its halo planes, so the halo exchange carries q,
+k, v, out, lse and dout.
+
 Host-side orchestration only: the arithmetic runs in the library's kernels; this
 module selects, exchanges and reduces tensors with torch.distributed (NCCL on
 GPUs, gloo for the CPU tests).  Each slab must be at least rz planes thick, so
@@ -155,14 +163,8 @@ def sharded_forward(shape, slab: Slab, coords: torch.Tensor, q, k, v, group=None
     packed order."""
     from . import pack3d as P
     rz = (shape.window[0] - 1) // 2
-    held_c, held = [], {"q": [], "k": [], "v": []}
-    for b in range(coords.shape[0]):
-        c, t = exchange_halo(slab, coords[b], {"q": q[b], "k": k[b], "v": v[b]}, rz, group)
-        held_c.append(c)
-        for n in held:
-            held[n].append(t[n])
-    hc = torch.stack(held_c).contiguous()
-    hq, hk, hv = (torch.stack(held[n]).contiguous() for n in ("q", "k", "v"))
+    hc, held = _held_batch(slab, coords, {"q": q, "k": k, "v": v}, rz, group)
+    hq, hk, hv = held["q"], held["k"], held["v"]
     params = P.make_params(slab_shape(shape, slab))
     idx = P.pack3d_build_index(params, hc)
     ksum, vsum = P.pack3d_block_summaries(params, idx, hk, hv)
@@ -170,3 +172,42 @@ def sharded_forward(shape, slab: Slab, coords: torch.Tensor, q, k, v, group=None
     out, lse = P.pack3d_forward(params, idx, hq, hk, hv, ksum, vsum)
     n_own = coords.shape[1]
     return out[:, :n_own], lse[:, :, :n_own]
+
+
+def _held_batch(slab: Slab, coords: torch.Tensor, tensors: dict, rz: int, group):
+    """Halo exchange of every batch item; the held coordinates [B, n_held, 3]
+    and tensors {name: [B, n_held, ...]}."""
+    held_c, held = [], {n: [] for n in tensors}
+    for b in range(coords.shape[0]):
+        c, t = exchange_halo(slab, coords[b], {n: x[b] for n, x in tensors.items()}, rz, group)
+        held_c.append(c)
+        for n in held:
+            held[n].append(t[n])
+    return (torch.stack(held_c).contiguous(),
+            {n: torch.stack(x).contiguous() for n, x in held.items()})
+
+
+def sharded_backward(shape, slab: Slab, coords: torch.Tensor, q, k, v, out, lse, dout,
+                     group=None):
+    """Gradients of sum(dout * out) with respect to this rank's owned q, k, v.
+    coords [B, n_own, 3] (global z); q, k, v, out, dout [B, n_own, H, d] and lse
+    [B, H, n_own] as sharded_forward returned them.  Returns dq, dk, dv
+    [B, n_own, H, d].  The summaries of the whole volume are computed again
+    (one pass over the held keys and values and an all-reduce)."""
+    from . import pack3d as P
+    rz = (shape.window[0] - 1) // 2
+    hc, held = _held_batch(slab, coords, {"q": q, "k": k, "v": v, "out": out, "dout": dout,
+                                          "lse": lse.transpose(1, 2)}, rz, group)
+    params = P.make_params(slab_shape(shape, slab))
+    idx = P.pack3d_build_index(params, hc)
+    ksum, vsum = P.pack3d_block_summaries(params, idx, held["k"], held["v"])
+    allreduce_summaries(ksum, vsum, group)
+    hlse = held["lse"].transpose(1, 2).contiguous()
+    dks, dvs, ws = P.pack3d_backward_summary_grads(params, idx, held["q"], held["k"], held["v"],
+                                                   held["out"], hlse, held["dout"], ksum, vsum)
+    # the gradient of a summary sums over the queries of every rank
+    allreduce_summaries(dks, dvs, group)
+    dq, dk, dv = (torch.zeros_like(held[n]) for n in ("q", "k", "v"))
+    P.pack3d_backward_from_summary_grads(params, idx, dks, dvs, ws, dq, dk, dv)
+    n_own = coords.shape[1]
+    return dq[:, :n_own], dk[:, :n_own], dv[:, :n_own]

@@ -249,3 +249,63 @@ def test_partly_occupied_params(lib):
     assert lib.pack3d_index_init(ctypes.byref(part), ctypes.c_void_p(1 << 20),
                                  ctypes.c_size_t(1 << 30), ctypes.byref(idx)) == P.OK
     assert idx.bcount and idx.bocc and idx.bocc > idx.bcount
+
+
+def test_two_call_backward_checks_without_cuda(lib):
+    """The two-call backward: missing pointers, a short workspace and a slab
+    call without the whole volume's summaries are ERR_ARG; the CUDA-core shapes
+    and slabs of the packed-RoPE mode are ERR_UNSUPPORTED; all of it before any
+    launch (the counter does not move)."""
+    n0 = P.pack3d_kernel_launches()
+    fake = ctypes.c_void_p(1 << 30)
+    ws = ctypes.c_void_p(1 << 32)
+
+    def index_for(p):
+        idx = P.Index()
+        assert lib.pack3d_index_init(ctypes.byref(p), ctypes.c_void_p(1 << 20),
+                                     ctypes.c_size_t(1 << 40), ctypes.byref(idx)) == P.OK
+        return idx
+
+    def first(p, idx, ksum, nbytes):
+        return lib.pack3d_backward_summary_grads(ctypes.byref(p), ctypes.byref(idx),
+                                                 *([fake] * 6), ksum, ksum, fake, fake, ws,
+                                                 ctypes.c_size_t(nbytes), None)
+
+    def second(p, idx, nbytes, dq=fake):
+        return lib.pack3d_backward_from_summary_grads(ctypes.byref(p), ctypes.byref(idx), fake,
+                                                      fake, ws, ctypes.c_size_t(nbytes), dq,
+                                                      fake, fake, None)
+
+    dense = shape(B=1, H=2, d=96, Z=16, Y=8, X=16, block=(4, 4, 4), window=(5, 3, 7))
+    p = P.make_params(dense)
+    idx = index_for(p)
+    need = lib.pack3d_backward_workspace_bytes(ctypes.byref(p))
+    assert need > 0
+    assert first(p, idx, None, need - 1) == P.ERR_ARG
+    assert second(p, idx, need - 1) == P.ERR_ARG
+    assert second(p, idx, need, dq=None) == P.ERR_ARG
+    assert lib.pack3d_backward_summary_grads(ctypes.byref(p), ctypes.byref(idx), None,
+                                             *([fake] * 5), None, None, fake, fake, ws,
+                                             ctypes.c_size_t(need), None) == P.ERR_ARG
+    # given summaries: both or neither
+    assert lib.pack3d_backward_summary_grads(ctypes.byref(p), ctypes.byref(idx), *([fake] * 6),
+                                             fake, None, fake, fake, ws, ctypes.c_size_t(need),
+                                             None) == P.ERR_ARG
+    # CUDA-core shapes
+    p32 = P.make_params(SimpleNamespace(**{**dense.__dict__, "dtype": "fp32"}))
+    idx32 = index_for(p32)
+    assert first(p32, idx32, None, 1 << 40) == P.ERR_UNSUPPORTED
+    assert second(p32, idx32, 1 << 40) == P.ERR_UNSUPPORTED
+    # a z-slab (planes 0 .. 11 of 16, owning 0 .. 8) needs the given summaries
+    slab = SimpleNamespace(**{**dense.__dict__, "Z": 11, "Z_total": 16, "z_origin": 0,
+                              "own_lo": 0, "own_hi": 8})
+    ps = P.make_params(slab)
+    idxs = index_for(ps)
+    need_s = lib.pack3d_backward_workspace_bytes(ctypes.byref(ps))
+    assert first(ps, idxs, None, need_s) == P.ERR_ARG
+    assert lib.pack3d_backward(ctypes.byref(ps), ctypes.byref(idxs), *([fake] * 9), ws,
+                               ctypes.c_size_t(need_s), None) == P.ERR_UNSUPPORTED
+    psr = P.make_params(SimpleNamespace(**{**slab.__dict__, "rope_mode": 1}))
+    idxr = index_for(psr)
+    assert first(psr, idxr, fake, 1 << 40) == P.ERR_UNSUPPORTED
+    assert P.pack3d_kernel_launches() == n0

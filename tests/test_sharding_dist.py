@@ -1,5 +1,6 @@
 """Host logic of the z-slab sharding on CPU: the slab plan, the halo exchange
-and the summary all-reduce as two gloo ranks (torch.distributed, the same calls
+(single and batched, as the forward and the backward run it) and the summary
+all-reduce as two gloo ranks (torch.distributed, the same calls
 NCCL runs on GPUs)."""
 import json
 import os
@@ -67,7 +68,17 @@ def worker(rank, world, port, out_dir, Z, Y, X, bz, rz):
         ks[B] = torch.tensor([B + 1.0, -(B + 1.0)])
     vs = ks.clone() * 2
     S.allreduce_summaries(ks, vs)
+    # batched exchange as the backward runs it: two items, and a per-head
+    # row tensor laid out [B, H, n] (as lse is) exchanged through its transpose
+    cb = torch.stack([coords, coords.flip(0)])
+    lse = torch.stack([voxel_value(c.long(), ch).T for c in cb])  # [2, 3, n]
+    hb_c, hb = S._held_batch(slab, cb, {"lse_t": lse.transpose(1, 2)}, rz, None)
+    batch_ok = all(
+        torch.equal(hb["lse_t"][b].T,
+                    voxel_value(hb_c[b].long() + torch.tensor([slab.h_lo, 0, 0]), ch).T)
+        for b in range(2))
     res = {
+        "batch_ok": bool(batch_ok),
         "held": sorted(map(tuple, gc.tolist())),
         "values_ok": bool(torch.equal(held["val"], voxel_value(gc, ch))),
         "own_first": bool(torch.equal(held_c[:coords.shape[0]].long() + torch.tensor([slab.h_lo, 0, 0]),
@@ -91,6 +102,6 @@ def test_halo_exchange_and_summary_allreduce(tmp_path, world):
         h_lo, h_hi = res["slab"]
         want = sorted([z, y, x] for z in range(h_lo, h_hi) for y in range(Y) for x in range(X))
         assert res["held"] == want  # every voxel of the held planes, once
-        assert res["values_ok"] and res["own_first"]
+        assert res["values_ok"] and res["own_first"] and res["batch_ok"]
         assert res["ks"] == [[B + 1.0, -(B + 1.0)] for B in range(nb)]
         assert res["vs"] == [[2 * (B + 1.0), -2 * (B + 1.0)] for B in range(nb)]

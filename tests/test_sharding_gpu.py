@@ -1,7 +1,8 @@
-"""The z-slab sharded forward on one GPU: the ranks' library calls run one after
-another on the same device (each on its slab with its halo planes, summaries of
-its own blocks summed over the ranks), and the owned outputs, put together,
-match the unsharded forward and the oracle."""
+"""The z-slab sharded forward and backward on one GPU: the ranks' library calls
+run one after another on the same device (each on its slab with its halo
+planes; the all-reduces of the summaries and of the summary gradients are sums
+over the ranks), and the owned outputs and gradients, put together, match the
+unsharded calls and the oracle."""
 import numpy as np
 import pytest
 import torch
@@ -12,7 +13,7 @@ from local_global_attention_b200 import inputs as I
 from local_global_attention_b200 import pack3d as P
 from local_global_attention_b200 import sharding as S
 
-from gpu_common import assert_close, gpu_run, oracle_sample
+from gpu_common import assert_close, assert_grad_close, gpu_run, oracle_sample
 
 pytestmark = pytest.mark.gpu
 
@@ -91,10 +92,113 @@ def test_sharded_forward_65k_two_slabs(oracle_lib):
     assert_close(lse[b, h, i], l, wl.dtype, "lse")
 
 
+def emulated_sharded_backward(wl, inp, world, out, lse):
+    """The backward of every rank in turn: held tensors (halo planes included)
+    cut from the global ones, summary gradients over each rank's owned queries
+    summed over the ranks, then each rank's owned dq, dk, dv.  out, lse: the
+    global forward results the backward differentiates."""
+    rz = (wl.window[0] - 1) // 2
+    slabs = [s for s in S.plan_slabs(wl.Z, wl.block[0], rz, world) if s.owned]
+    dev = {k: v.cuda() for k, v in inp.items() if k != "order"}
+    dev["out"] = out.cuda()
+    dev["lse_t"] = lse.cuda().transpose(1, 2)
+    names = ("q", "k", "v", "out", "dout", "lse_t")
+    calls = []
+    ksum = vsum = None
+    for slab in slabs:
+        held_c, held = [], {n: [] for n in names}
+        for b in range(wl.B):
+            c, t = S.held_from_global(slab, dev["coords"][b], {n: dev[n][b] for n in names})
+            held_c.append(c)
+            for n in names:
+                held[n].append(t[n])
+        hc = torch.stack(held_c).contiguous()
+        h = {n: torch.stack(held[n]).contiguous() for n in names}
+        h["lse"] = h.pop("lse_t").transpose(1, 2).contiguous()
+        params = P.make_params(S.slab_shape(wl, slab))
+        idx = P.pack3d_build_index(params, hc)
+        assert P.pack3d_index_check(idx) == P.OK
+        ks, vs = P.pack3d_block_summaries(params, idx, h["k"], h["v"])
+        ksum = ks if ksum is None else ksum + ks
+        vsum = vs if vsum is None else vsum + vs
+        calls.append((slab, params, idx, h))
+    dks = dvs = None
+    staged = []
+    for slab, params, idx, h in calls:
+        a, c, ws = P.pack3d_backward_summary_grads(params, idx, h["q"], h["k"], h["v"], h["out"],
+                                                   h["lse"], h["dout"], ksum, vsum)
+        dks = a if dks is None else dks + a
+        dvs = c if dvs is None else dvs + c
+        staged.append(ws)
+    grads = {n: torch.zeros_like(dev[n]) for n in ("q", "k", "v")}
+    for (slab, params, idx, h), ws in zip(calls, staged):
+        g = [torch.zeros_like(h[n]) for n in ("q", "k", "v")]
+        P.pack3d_backward_from_summary_grads(params, idx, dks, dvs, ws, *g)
+        for b in range(wl.B):
+            own = ((dev["coords"][b, :, 0] >= slab.z_lo) & (dev["coords"][b, :, 0] < slab.z_hi))
+            pos = own.nonzero().squeeze(1)
+            for n, t in zip(("q", "k", "v"), g):
+                grads[n][b].index_copy_(0, pos, t[b, :pos.numel()])
+        assert P.pack3d_index_check(idx) == P.OK
+    torch.cuda.synchronize()
+    return grads["q"].cpu(), grads["k"].cpu(), grads["v"].cpu()
+
+
+@pytest.mark.parametrize("wl,world", SHARD_CASES, ids=lambda x: getattr(x, "name", str(x)))
+def test_sharded_backward_matches(oracle_lib, wl, world):
+    wl = wl.replace(value_scale=1.0 / np.sqrt(96))
+    inp = I.make_inputs(wl, "random", with_dout=True)
+    ref = gpu_run(wl, inp, with_backward=True)
+    got = emulated_sharded_backward(wl, inp, world, ref["out"], ref["lse"])
+    want = oracle.backward(wl, inp["coords"], inp["q"], inp["k"], inp["v"], inp["dout"])
+    for name, g, w in zip(("dq", "dk", "dv"), got, want):
+        assert_grad_close(g, ref[name].double().numpy(), wl.dtype, f"{name} vs unsharded")
+        assert_grad_close(g, w, wl.dtype, name)
+
+
+def test_two_call_backward_is_the_backward():
+    """Without a slab, the two calls with nothing between them are
+    pack3d_backward, bit for bit (given summaries or computed ones)."""
+    wl = SHARD_CASES[0][0].replace(value_scale=1.0 / np.sqrt(96), name="two_call")
+    inp = I.make_inputs(wl, "random", with_dout=True)
+    ref = gpu_run(wl, inp, with_backward=True)
+    d = {k: v.cuda() for k, v in inp.items() if k != "order"}
+    params, idx = ref["params"], ref["index"]
+    out, lse = ref["out"].cuda(), ref["lse"].cuda()
+    ksum, vsum = ref["ksum"].cuda(), ref["vsum"].cuda()
+    for given in (False, True):
+        dks, dvs, ws = P.pack3d_backward_summary_grads(
+            params, idx, d["q"], d["k"], d["v"], out, lse, d["dout"],
+            ksum if given else None, vsum if given else None)
+        g = [torch.empty_like(d[n]) for n in ("q", "k", "v")]
+        P.pack3d_backward_from_summary_grads(params, idx, dks, dvs, ws, *g)
+        torch.cuda.synchronize()
+        for name, t in zip(("dq", "dk", "dv"), g):
+            assert torch.equal(t.cpu(), ref[name]), (given, name)
+
+
+def test_sharded_backward_65k_two_slabs(oracle_lib):
+    """The 65k training shape cut into two z-slabs: every gradient against the
+    unsharded backward, and one (batch item, head) slice against the oracle."""
+    wl = C.TRAIN65K
+    inp = I.make_inputs(wl, "random", with_dout=True)
+    ref = gpu_run(wl, inp, with_backward=True)
+    got = emulated_sharded_backward(wl, inp, 2, ref["out"], ref["lse"])
+    for name, g in zip(("dq", "dk", "dv"), got):
+        assert_grad_close(g, ref[name].double().numpy(), wl.dtype, f"{name} vs unsharded")
+    one = wl.replace(B=1, H=1)
+    b, h = 1, 3
+    sl = {n: inp[n][b:b + 1, :, h:h + 1].contiguous() for n in ("q", "k", "v", "dout")}
+    want = oracle.backward(one, inp["coords"][b:b + 1], sl["q"], sl["k"], sl["v"], sl["dout"])
+    for name, g, w in zip(("dq", "dk", "dv"), got, want):
+        assert_grad_close(g[b:b + 1, :, h:h + 1], w, wl.dtype, f"{name}[b={b}, h={h}]")
+
+
 def test_slab_calls_reject_other_paths():
-    """z-slabs run the tensor-core forward of dense volumes with axial RoPE:
-    the backward, fp32, the packed-RoPE mode and partly occupied volumes report
-    ERR_UNSUPPORTED."""
+    """z-slabs run the tensor-core path of dense volumes with axial RoPE:
+    fp32 and the packed-RoPE mode report ERR_UNSUPPORTED, and so does the
+    one-call backward (a slab's summary gradients need the exchange between the
+    two calls)."""
     wl = SHARD_CASES[0][0]
     slab = S.plan_slabs(wl.Z, wl.block[0], 2, 2)[0]
     for variant in (dict(dtype="fp32"), dict(rope_mode=1)):
