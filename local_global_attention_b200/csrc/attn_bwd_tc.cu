@@ -79,6 +79,7 @@ struct Smem {
   uint8_t c2[NSTAGE][3 * SEGC];  // column operand 2
   uint8_t cp[NSTAGE][KCH * 32];  // penalty channels of the column rows (32-byte swizzle)
   float4 st[NSTAGE][KCH];        // per-column (L, delta, 0, 0)
+  PenaltyTable pt;               // the tile's penalty channels per axis (dense volumes)
   uint64_t a_full;               // A1 in tensor memory and A2 loaded
   uint64_t kv_full[NSTAGE], kv_empty[NSTAGE];
   uint64_t s_full[2];    // S and dP of the buffer's chunk computed
@@ -285,6 +286,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       }
     }
+    // dense volumes whose halo box fits the per-axis tables: penalty rows by
+    // table lookups
+    const bool table = PENALTY && !PARTIAL && tb.hz <= PEN_TAB && tb.hy <= PEN_TAB &&
+                       tb.hx <= PEN_TAB;
+    if (table) {
+      penalty_table(sm.pt, g, tb, lane);
+      __syncwarp();
+    }
     int issued = 0;
     for (int j = 0; j < nch; ++j) {
       const int s = j % NSTAGE, round = j / NSTAGE;
@@ -314,7 +323,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       }
       if (PENALTY && j < n_local) {
-        penalty_rows<PARTIAL>(sm.cp[s], g, tb, z, y, x, lane, ix.vol + (int64_t)b * g.V);
+        if (table)
+          penalty_rows_table(sm.cp[s], sm.pt, tb, z, y, x, lane);
+        else
+          penalty_rows<PARTIAL>(sm.cp[s], g, tb, z, y, x, lane, ix.vol + (int64_t)b * g.V);
         fence_proxy_async_smem();
       }
       __syncwarp();

@@ -85,6 +85,7 @@ struct Smem {
   uint8_t k[NSTAGE][3 * KSEG];
   uint8_t v[NSTAGE][3 * KSEG];
   uint8_t kp[NSTAGE][KCH * 32];  // penalty channels of each stage's key rows (32-byte swizzle)
+  PenaltyTable pt;               // the tile's penalty channels per axis (dense volumes)
   uint64_t q_full;               // Q is in tensor memory
   uint64_t kv_full[NSTAGE];
   uint64_t kv_empty[NSTAGE];
@@ -269,6 +270,10 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       tma_prefetch_map(&maps.vg);
     }
     const int bh = b * g.H + h;
+    if (!PARTIAL) {
+      penalty_table(sm.pt, g, tb, lane);
+      __syncwarp();
+    }
     int xc = 0, yc = 0, zc = 0;
     int issued = 0;
     for (int j = 0; j < nch; ++j) {
@@ -297,8 +302,11 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       }
       if (j < n_local) {
         // penalty rows of the chunk's keys (dz, dy, dx): key r = (dz * 2 + dy) * 16 + dx
-        penalty_rows<PARTIAL>(sm.kp[s], g, tb, tb.hz0 + BZK * zc, tb.hy0 + BYK * yc, tb.hx0 + BXK * xc,
-                     lane, ix.vol + (int64_t)b * g.V);
+        const int cz0 = tb.hz0 + BZK * zc, cy0 = tb.hy0 + BYK * yc, cx0 = tb.hx0 + BXK * xc;
+        if (PARTIAL)
+          penalty_rows<true>(sm.kp[s], g, tb, cz0, cy0, cx0, lane, ix.vol + (int64_t)b * g.V);
+        else
+          penalty_rows_table(sm.kp[s], sm.pt, tb, cz0, cy0, cx0, lane);
         fence_proxy_async_smem();
         if (++xc == nxc) {
           xc = 0;

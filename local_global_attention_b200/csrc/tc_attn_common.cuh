@@ -108,6 +108,55 @@ __device__ __forceinline__ void penalty_rows(uint8_t* dst, const Geo& g, const T
   }
 }
 
+// The penalty channels of one axis depend only on the key's coordinate on
+// that axis, so a tile's penalty rows are a product of three small tables over
+// its halo box: entry o describes key coordinate (halo origin + o) on that axis
+// - channels 0-3 (z: the tile's query planes), 4-7 (y), 8-15 (x).  A key
+// outside the volume on an axis has every channel of that axis set, which masks
+// it for every query.  Dense volumes only (an empty voxel does not factorise);
+// halo boxes up to PEN_TAB per axis.
+constexpr int PEN_TAB = 64;
+struct PenaltyTable {
+  uint2 z[PEN_TAB];
+  uint2 y[PEN_TAB];
+  uint4 x[PEN_TAB];
+};
+
+__device__ __forceinline__ uint32_t pen_pair(bool lo, bool hi) {
+  return (lo ? (uint32_t)BF16_PEN : 0u) | ((hi ? (uint32_t)BF16_PEN : 0u) << 16);
+}
+
+// Fill the table of tile `tb` (the 32 lanes of one warp).
+__device__ __forceinline__ void penalty_table(PenaltyTable& t, const Geo& g, const TileBox& tb,
+                                              int lane) {
+  for (int o = lane; o < PEN_TAB; o += 32) {
+    const int kz = tb.hz0 + o, ky = tb.hy0 + o, kx = tb.hx0 + o;
+    const bool zo = kz >= g.Z, yo = ky >= g.Y, xo = kx >= g.X;
+    auto zm = [&](int a) { return zo || abs(kz - (tb.z0 + a)) > g.rz; };
+    auto ym = [&](int a) { return yo || abs(ky - (tb.y0 + a)) > g.ry; };
+    auto xm = [&](int a) { return xo || abs(kx - (tb.x0 + a)) > g.rx; };
+    t.z[o] = make_uint2(pen_pair(zm(0), zm(1)), pen_pair(zm(2), zm(3)));
+    t.y[o] = make_uint2(pen_pair(ym(0), ym(1)), pen_pair(ym(2), ym(3)));
+    t.x[o] = make_uint4(pen_pair(xm(0), xm(1)), pen_pair(xm(2), xm(3)), pen_pair(xm(4), xm(5)),
+                        pen_pair(xm(6), xm(7)));
+  }
+}
+
+// penalty_rows of a dense volume from the tile's table: the same 64 rows.
+__device__ __forceinline__ void penalty_rows_table(uint8_t* dst, const PenaltyTable& t,
+                                                   const TileBox& tb, int cz0, int cy0, int cx0,
+                                                   int lane) {
+  const uint2 yw = t.y[cy0 - tb.hy0 + ((lane >> 4) & 1)];
+  const uint4 xw = t.x[cx0 - tb.hx0 + (lane & 15)];
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const int r = lane + 32 * half;
+    const uint2 zw = t.z[cz0 - tb.hz0 + half];
+    *reinterpret_cast<uint4*>(dst + sw32_off(r, 0)) = make_uint4(zw.x, zw.y, yw.x, yw.y);
+    *reinterpret_cast<uint4*>(dst + sw32_off(r, 1)) = xw;
+  }
+}
+
 // Rotate four words of pair members (lo) against their partners (hi): word u of
 // lo holds channels j0 + 2u, j0 + 2u + 1 of a segment, word u of hi the same
 // pairs' second members.  t = rotation-table row (16 (cos, sin) pairs) of the
