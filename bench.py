@@ -38,7 +38,10 @@ UNIT = "tokens/s"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "forward_tc_vol_32x32x64.md")
-TC_SOURCE = os.path.join(ROOT, "local_global_attention_b200", "csrc", "attn_tc.cu")
+# the attention kernel's source and the headers it includes
+TC_SOURCES = [os.path.join(ROOT, "local_global_attention_b200", "csrc", f)
+              for f in ("attn_tc.cu", "tc_attn_common.cuh", "tc_primitives.cuh",
+                        "pack3d_internal.cuh")]
 
 
 def peaks():
@@ -336,6 +339,14 @@ class Runner:
             raise RuntimeError(f"pack3d_block_summaries failed: {rc}")
 
 
+def kernel_sources_sha256():
+    """sha256 over the attention kernel's source files, in order."""
+    h = hashlib.sha256()
+    for f in TC_SOURCES:
+        h.update(open(f, "rb").read())
+    return h.hexdigest()
+
+
 def profile_value(key):
     """A figure from the committed ncu summary of the attention kernel, if it
     was taken on the current kernel source; else None."""
@@ -347,7 +358,7 @@ def profile_value(key):
     m = re.search(key + r":\s*([0-9.eE+]+)", text)
     if not (m_sha and m):
         return None
-    sha = hashlib.sha256(open(TC_SOURCE, "rb").read()).hexdigest()
+    sha = kernel_sources_sha256()
     return float(m.group(1)) if sha == m_sha.group(1) else None
 
 
