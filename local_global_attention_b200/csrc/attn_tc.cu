@@ -19,27 +19,35 @@
 //     16 (x) x 2 (y) x 2 (z) = 64 keys, then the block summaries (bf16 copies,
 //     64 per chunk), all streamed through one online softmax.  Roles:
 //
-//     * TMA (warp 5, one thread): per chunk six box loads (three 32-channel
+//     * TMA (warp 5): per chunk six box loads by one thread (three 32-channel
 //       segments of K and of V, 64-byte swizzle: exactly the K-major operand
 //       layout of the MMAs) into a 3-stage shared-memory ring; positions
-//       outside the volume are filled with zeros by the copy and masked;
-//     * MMA (warp 4, one thread): S_j = Q K_j^T (six tcgen05.mma, K = 16) into
-//       one of two TMEM S buffers, and O += P_j V_j (four tcgen05.mma, A = P
-//       from TMEM, B = V MN-major in shared memory), so S_{j+1} is computed
-//       while the softmax works on S_j;
+//       outside the volume are filled with zeros by the copy and masked.  The
+//       warp also writes the chunk's penalty rows (below), assembled from
+//       per-axis tables built once per tile;
+//     * MMA (warp 4, one thread): S_j = Q K_j^T (six tcgen05.mma, K = 16, plus
+//       one for the window penalty) into one of two TMEM S buffers, with both
+//       Q and K read from shared memory, and O += P_j V_j (four tcgen05.mma,
+//       A = P from TMEM, B = V MN-major in shared memory).  S_{j+2} is issued
+//       as soon as PV_j is done, so two S products run ahead of the softmax;
 //     * softmax (warps 0-3, one query row per thread, warp w = a 2 x 2 x 8 box):
-//       gather and rotate the query rows once; per chunk form the window mask
-//       from three per-query bit sets over the halo (z planes, y rows, x
-//       columns), read the chunk's 64 S values in one go, keep the online max
-//       and sum, write P (bf16) over S in TMEM.  A warp whose 32 queries see
-//       none of a chunk's keys (its plane or row pair outside their windows)
-//       only writes zeros.  Summary chunks use the mask "block box does not meet the
-//       window box"; there is no count bias.  The running max moves only when
-//       a row's maximum grows by more than 8 (log2 units), so O is rescaled in
-//       TMEM rarely; the result is the same softmax.
+//       gather and rotate the query rows once into the shared-memory Q tile;
+//       per chunk form the window mask from three per-query bit sets over the
+//       halo (z planes, y rows, x columns), read the chunk's 64 S values in one
+//       go, keep the online max and sum, write P (bf16) over the first half of
+//       the S buffer it read.  A warp whose 32 queries see none of a chunk's
+//       keys (its plane or row pair outside their windows) only writes zeros.
+//       Summary chunks use the mask "block box does not meet the window box";
+//       there is no count bias.  The running max moves only when a row's
+//       maximum grows by more than 8 (log2 units), so O is rescaled in TMEM
+//       rarely; the result is the same softmax.
+//
+// The window mask rides in the S product: 16 extra contraction channels hold
+// the query's one-hot tile position and the key's -2^14 penalties.
 //
 // The epilogue divides by the row sum and writes out (packed order) and the
-// natural-log LSE.  Two CTAs share an SM (256 TMEM columns each).  Every wait
+// natural-log LSE.  Two CTAs share an SM (256 TMEM columns and ~110 KB of
+// shared memory each).  Every wait
 // is bounded; a CTA that gives up sets the timeout bit of the index error word.
 #include <cuda.h>
 #include <math.h>
@@ -58,15 +66,16 @@ using namespace tc;
 using namespace tca;
 
 constexpr int D = 96;                      // head dim handled by this path
-constexpr int NSTAGE = 4;                  // K/V shared-memory ring depth
+constexpr int NSTAGE = 3;                  // K/V shared-memory ring depth
 constexpr int KSEG = KCH * 64;             // one 32-channel segment of a chunk
 constexpr uint32_t CHUNK_BYTES = 6 * KSEG; // K and V of one chunk
 constexpr uint32_t TMEM_COLS = 256;
-// Tensor memory (128 lanes = query rows, 256 columns of 32 bits):
-constexpr uint32_t COL_O = 0;              // O accumulator, fp32: columns [0, 96)
-constexpr uint32_t COL_P = 96;             // P, bf16 pairs: columns [96, 128)
-constexpr uint32_t COL_S = 128;            // S, fp32: columns [128, 192)
-constexpr uint32_t COL_Q = 192;            // rotated Q + penalty one-hot, bf16 pairs: [192, 248)
+// Tensor memory (128 lanes = query rows, 256 columns of 32 bits): the O
+// accumulator (fp32, columns [0, 96)) and two S buffers (fp32, [96, 160) and
+// [160, 224)); P (bf16 pairs) is written over the first 32 columns of its S.
+constexpr uint32_t COL_O = 0;
+constexpr uint32_t COL_S = 96;
+constexpr int QSEG = 128 * 64;             // one 32-channel segment of the Q tile
 constexpr int MMA_WARP = 4;
 constexpr int TMA_WARP = 5;
 constexpr int NTHREADS = 192;
@@ -82,18 +91,19 @@ constexpr int MAX_HALO = 64;               // halo extent per axis the 64-bit ma
 constexpr float M_FLOOR = -1000.0f;
 
 struct Smem {
+  uint8_t q[3 * QSEG];           // rotated Q rows (K-major, 64-byte swizzle), row = TMEM lane
+  uint8_t qp[128 * 32];          // the rows' penalty one-hot (32-byte swizzle)
   uint8_t k[NSTAGE][3 * KSEG];
   uint8_t v[NSTAGE][3 * KSEG];
   uint8_t kp[NSTAGE][KCH * 32];  // penalty channels of each stage's key rows (32-byte swizzle)
   PenaltyTable pt;               // the tile's penalty channels per axis (dense volumes)
-  uint64_t q_full;               // Q is in tensor memory
+  uint64_t q_full;               // Q is in shared memory
   uint64_t kv_full[NSTAGE];
   uint64_t kv_empty[NSTAGE];
-  uint64_t s_full;   // one phase per chunk: S_j computed
-  uint64_t s_free;   // one phase per chunk: S_j read by the softmax
-  uint64_t p_full;   // one phase per chunk: P_j written
-  uint64_t o_done;   // one phase per PV product (P and O may be touched)
-  uint64_t o_final;  // one phase: every PV product of the tile is done
+  uint64_t s_full[2];    // S of the buffer's chunk computed
+  uint64_t p_full[2];    // P of the buffer's chunk written
+  uint64_t buf_free[2];  // the PV product reading the buffer's P is done
+  uint64_t o_final;      // one phase: every PV product of the tile is done
   uint32_t tmem_base;
   int32_t abort;
 };
@@ -246,10 +256,11 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       mbar_init(&sm.kv_full[s], 2);  // TMA bytes + the penalty rows
       mbar_init(&sm.kv_empty[s], 1);
     }
-    mbar_init(&sm.s_full, 1);
-    mbar_init(&sm.s_free, 4);
-    mbar_init(&sm.p_full, 4);
-    mbar_init(&sm.o_done, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.s_full[i], 1);
+      mbar_init(&sm.p_full[i], 4);
+      mbar_init(&sm.buf_free[i], 1);
+    }
     mbar_init(&sm.o_final, 1);
     sm.abort = 0;
     fence_barrier_init();
@@ -337,47 +348,52 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       const uint64_t kd0 = sdesc_sw64(smem_u32(sm.k[0]), 16, 512);
       const uint64_t vd0 = sdesc_sw64(smem_u32(sm.v[0]), KSEG, 512);
       const uint64_t kpd0 = sdesc_sw32(smem_u32(sm.kp[0]), 16, 256);
+      const uint64_t qd0 = sdesc_sw64(smem_u32(sm.q), 16, 512);
+      const uint64_t qpd = sdesc_sw32(smem_u32(sm.qp), 16, 256);
       auto wait_all = [&](uint64_t* bar, uint32_t parity) {
         return __all_sync(0xffffffffu, mbar_wait_or_abort(bar, parity, WAIT_LIMIT, abort_flag));
       };
       bool ok = wait_all(&sm.q_full, 0);
-      // S_j = Q K_j^T: A = Q from tensor memory (8 columns per K = 16 step),
-      // B = the chunk's key rows (K-major, 64-byte swizzle)
+      // S_j = Q K_j^T into buffer j % 2: A = the Q tile, B = the chunk's key
+      // rows (both K-major, 64-byte swizzle, 16-channel steps)
       auto issue_s = [&](int j) -> bool {
         const int s = j % NSTAGE;
         if (!wait_all(&sm.kv_full[s], (j / NSTAGE) & 1)) return false;
         tc_fence_after();
+        const uint32_t dS = tbase + COL_S + 64 * (j & 1);
         const uint64_t kd = kd0 + (uint64_t)((s * 3 * KSEG) >> 4);
 #pragma unroll
         for (int st = 0; st < D / 16; ++st)
-          mma_ts_warp(tbase + COL_S, tbase + COL_Q + 8 * st,
+          mma_ss_warp(dS, qd0 + (uint64_t)(((st >> 1) * QSEG + (st & 1) * 32) >> 4),
                       kd + (uint64_t)(((st >> 1) * KSEG + (st & 1) * 32) >> 4), idesc_s, st > 0);
         if (j < n_local)  // + the window penalty (summary chunks are masked by the softmax)
-          mma_ts_warp(tbase + COL_S, tbase + COL_Q + 48, kpd0 + (uint64_t)((s * KCH * 32) >> 4),
-                      idesc_s, 1u);
-        mma_commit_warp(&sm.s_full);
+          mma_ss_warp(dS, qpd, kpd0 + (uint64_t)((s * KCH * 32) >> 4), idesc_s, 1u);
+        mma_commit_warp(&sm.s_full[j & 1]);
         return true;
       };
-      if (ok && nch > 0) {
-        tc_fence_after();
-        ok = issue_s(0);
-      }
+      if (ok) tc_fence_after();
+      for (int j = 0; j < min(2, nch) && ok; ++j) ok = issue_s(j);
       for (int j = 0; j < nch && ok; ++j) {
-        // S_{j+1} once the softmax has read S_j: it runs while P_j is formed
-        if (j + 1 < nch) {
-          if (!wait_all(&sm.s_free, j & 1)) break;
-          if (!(ok = issue_s(j + 1))) break;
-        }
-        if (!wait_all(&sm.p_full, j & 1)) break;
+        const int bi = j & 1;
+        if (!(ok = wait_all(&sm.p_full[bi], (j >> 1) & 1))) break;
         tc_fence_after();
+        // O += P_j V_j: A = P over the buffer's first 32 columns, B = V
+        // MN-major (key rows 16 u .. 16 u + 15 at byte offset 1024 u)
         const uint64_t vd = vd0 + (uint64_t)(((j % NSTAGE) * 3 * KSEG) >> 4);
+        const uint32_t pS = tbase + COL_S + 64 * bi;
 #pragma unroll
         for (int st = 0; st < KCH / 16; ++st)
-          mma_ts_warp(tbase + COL_O, tbase + COL_P + 8 * st, vd + (uint64_t)((st * 16 * 64) >> 4),
-                      idesc_o, (j > 0 || st > 0) ? 1u : 0u);
-        mma_commit_warp(&sm.o_done);
+          mma_ts_warp(tbase + COL_O, pS + 8 * st, vd + (uint64_t)((st * 16 * 64) >> 4), idesc_o,
+                      (j > 0 || st > 0) ? 1u : 0u);
+        mma_commit_warp(&sm.buf_free[bi]);
         mma_commit_warp(&sm.kv_empty[j % NSTAGE]);
         if (j == nch - 1) mma_commit_warp(&sm.o_final);
+        // S_{j+2} overwrites P_j: after PV_j is done
+        if (j + 2 < nch) {
+          if (!(ok = wait_all(&sm.buf_free[bi], (j >> 1) & 1))) break;
+          tc_fence_after();
+          if (!(ok = issue_s(j + 2))) break;
+        }
       }
     }
     __syncwarp();
@@ -427,34 +443,18 @@ __global__ void __launch_bounds__(NTHREADS, 2)
 #pragma unroll
         for (int i = 0; i < 12; ++i) r[i] = make_uint4(0, 0, 0, 0);
       }
-      // into this thread's tensor-memory lane: channel pairs in columns
-      // [COL_Q, COL_Q + 48), then the penalty channels
-      const uint32_t tq = tbase + ((uint32_t)(warp * 32) << 16) + COL_Q;
-      {
-        uint32_t w32[32], w16[16];
+      // into the Q tile, row tid (this thread's TMEM lane): 16-byte chunk i
+      // of the row is chunk i % 4 of segment i / 4; then the penalty one-hot
+      const uint32_t rr = (uint32_t)tid;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          w32[4 * i] = r[i].x;
-          w32[4 * i + 1] = r[i].y;
-          w32[4 * i + 2] = r[i].z;
-          w32[4 * i + 3] = r[i].w;
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          w16[4 * i] = r[8 + i].x;
-          w16[4 * i + 1] = r[8 + i].y;
-          w16[4 * i + 2] = r[8 + i].z;
-          w16[4 * i + 3] = r[8 + i].w;
-        }
-        tmem_st32(tq, w32);
-        tmem_st16(tq + 32, w16);
-      }
-      // penalty channels: one-hot of (z, y, x) within the tile
+      for (int i = 0; i < 12; ++i)
+        *reinterpret_cast<uint4*>(sm.q + (i >> 2) * QSEG + sw64_off(rr, i & 3)) = r[i];
       uint32_t w[8];
       onehot_words(lzi, lyi, lxi, w);
-      tmem_st8(tq + 48, w);
-      tmem_wait_st();
-      tc_fence_before();
+      *reinterpret_cast<uint4*>(sm.qp + sw32_off(rr, 0)) = make_uint4(w[0], w[1], w[2], w[3]);
+      *reinterpret_cast<uint4*>(sm.qp + sw32_off(rr, 1)) = make_uint4(w[4], w[5], w[6], w[7]);
+      // visible to the tensor core (async proxy) before the arrival
+      fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.q_full);
     }
@@ -468,8 +468,6 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     }
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     const uint32_t tO = tbase + lane_base + COL_O;
-    const uint32_t tP = tbase + lane_base + COL_P;
-    const uint32_t tS = tbase + lane_base + COL_S;
     const float c2 = g.tau * LOG2E;  // logits -> log2 units
     float m_run = M_FLOOR, l_run = 0.f;
     // the box of blocks this query's window touches (global planes: the
@@ -480,9 +478,11 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     int xc = 0, yc = 0, zc = 0;
     bool ok = true;
     for (int j = 0; j < nch; ++j) {
+      const int bi = j & 1;
+      const uint32_t tS = tbase + lane_base + COL_S + 64 * bi;
       // a warp leaves together: the TMEM accesses below are warp-collective
       ok = __all_sync(0xffffffffu,
-                      mbar_wait_or_abort(&sm.s_full, j & 1, WAIT_LIMIT, abort_flag));
+                      mbar_wait_or_abort(&sm.s_full[bi], (j >> 1) & 1, WAIT_LIMIT, abort_flag));
       if (!ok) break;
       tc_fence_after();
       uint32_t bits0, bits1;
@@ -521,10 +521,6 @@ __global__ void __launch_bounds__(NTHREADS, 2)
         tmem_ld32(tS + 32, sb);
         tmem_wait_ld();
       }
-      // S_j is in registers: the MMA may overwrite it with S_{j+1}
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.s_free);
       uint32_t p[32];
       float corr = 1.f;
       bool rescale_o = false;
@@ -551,16 +547,18 @@ __global__ void __launch_bounds__(NTHREADS, 2)
         l_run += exp_pack_all(sa, c2, mneg, p);
         l_run += exp_pack_all(sb, c2, mneg, p + 16);
       }
-      // P and O are free once PV_{j-1} is done (the MMA issues PV_j only after
-      // p_full below, so this phase is never two behind)
-      if (j > 0) {
-        ok = __all_sync(0xffffffffu,
-                        mbar_wait_or_abort(&sm.o_done, (j - 1) & 1, WAIT_LIMIT, abort_flag));
-        if (!ok) break;
-        tc_fence_after();
-      }
-      tmem_st32(tP, p);
+      // P over the first 32 columns of S_j (read above)
+      tmem_st32(tS, p);
       if (__any_sync(0xffffffffu, rescale_o)) {
+        // O may be rescaled once PV_{j-1} is done (the next product on that
+        // barrier, PV_{j+1}, needs this warp's later arrivals)
+        if (j > 0) {
+          ok = __all_sync(0xffffffffu, mbar_wait_or_abort(&sm.buf_free[(j - 1) & 1],
+                                                          ((j - 1) >> 1) & 1, WAIT_LIMIT,
+                                                          abort_flag));
+          if (!ok) break;
+          tc_fence_after();
+        }
         const float co = rescale_o ? corr : 1.f;
 #pragma unroll 1
         for (int part = 0; part < 6; ++part) {
@@ -575,7 +573,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.p_full);
+      if (lane == 0) mbar_arrive(&sm.p_full[bi]);
     }
     // ---- epilogue ----
     // o_final completes once, after the last PV product.  (Waiting on o_done
