@@ -92,6 +92,43 @@ def test_sharded_forward_65k_two_slabs(oracle_lib):
     assert_close(lse[b, h, i], l, wl.dtype, "lse")
 
 
+def test_sharded_window_only_forward(oracle_lib):
+    """The window-only forward on slabs needs no exchange but the halo: every
+    rank's owned outputs against the unsharded window-only forward and the
+    oracle."""
+    wl, world = SHARD_CASES[1]
+    inp = I.make_inputs(wl, "random")
+    rz = (wl.window[0] - 1) // 2
+    dev = {k: v.cuda() for k, v in inp.items() if k != "order"}
+    out = torch.zeros_like(dev["q"])
+    lse = torch.zeros(wl.B, wl.H, wl.N, device="cuda")
+    for slab in (s for s in S.plan_slabs(wl.Z, wl.block[0], rz, world) if s.owned):
+        held_c, held = [], {"q": [], "k": [], "v": []}
+        for b in range(wl.B):
+            c, t = S.held_from_global(slab, dev["coords"][b],
+                                      {n: dev[n][b] for n in ("q", "k", "v")})
+            held_c.append(c)
+            for n in held:
+                held[n].append(t[n])
+        params = P.make_params(S.slab_shape(wl, slab))
+        idx = P.pack3d_build_index(params, torch.stack(held_c).contiguous())
+        assert P.pack3d_index_check(idx) == P.OK
+        o, l = P.pack3d_window_forward(params, idx, *(torch.stack(held[n]).contiguous()
+                                                      for n in ("q", "k", "v")))
+        for b in range(wl.B):
+            own = (dev["coords"][b, :, 0] >= slab.z_lo) & (dev["coords"][b, :, 0] < slab.z_hi)
+            pos = own.nonzero().squeeze(1)
+            out[b].index_copy_(0, pos, o[b, :pos.numel()])
+            lse[b].index_copy_(1, pos, l[b, :, :pos.numel()])
+    torch.cuda.synchronize()
+    ref = gpu_run(wl, inp, window_only=True)
+    assert_close(out.cpu(), ref["out"].double().numpy(), wl.dtype, "out vs unsharded")
+    want_out, want_lse = oracle.forward(wl, inp["coords"], inp["q"], inp["k"], inp["v"],
+                                        window_only=True)
+    assert_close(out.cpu(), want_out, wl.dtype, "out")
+    assert_close(lse.cpu(), want_lse, wl.dtype, "lse")
+
+
 def emulated_sharded_backward(wl, inp, world, out, lse):
     """The backward of every rank in turn: held tensors (halo planes included)
     cut from the global ones, summary gradients over each rank's owned queries
@@ -175,6 +212,25 @@ def test_two_call_backward_is_the_backward():
         torch.cuda.synchronize()
         for name, t in zip(("dq", "dk", "dv"), g):
             assert torch.equal(t.cpu(), ref[name]), (given, name)
+
+
+@pytest.mark.parametrize("variant", ["partial", "packed_rope"])
+def test_two_call_backward_other_modes(variant):
+    """The two calls equal pack3d_backward bit for bit for a partly occupied
+    volume and in the packed-sequence RoPE mode (both unsharded)."""
+    base = SHARD_CASES[0][0].replace(value_scale=1.0 / np.sqrt(96), name="two_call_" + variant)
+    wl = base.replace(n_tokens=1500) if variant == "partial" else base.replace(rope_mode=1)
+    inp = I.make_inputs(wl, "random", with_dout=True)
+    ref = gpu_run(wl, inp, with_backward=True)
+    d = {k: v.cuda() for k, v in inp.items() if k != "order"}
+    dks, dvs, ws = P.pack3d_backward_summary_grads(
+        ref["params"], ref["index"], d["q"], d["k"], d["v"], ref["out"].cuda(),
+        ref["lse"].cuda(), d["dout"])
+    g = [torch.empty_like(d[n]) for n in ("q", "k", "v")]
+    P.pack3d_backward_from_summary_grads(ref["params"], ref["index"], dks, dvs, ws, *g)
+    torch.cuda.synchronize()
+    for name, t in zip(("dq", "dk", "dv"), g):
+        assert torch.equal(t.cpu(), ref[name]), name
 
 
 def test_sharded_backward_65k_two_slabs(oracle_lib):
