@@ -279,13 +279,14 @@ PACK3D_API int pack3d_backward(const pack3d_params* p, const pack3d_index* idx, 
  * z-slabs (params with Z_total > 0).  The gradient of a block summary is a sum
  * over every query of the volume whose window misses the block, so on a slab it
  * is a partial sum: the caller adds the ranks' partial sums (an all-reduce)
- * between the two calls.  The operator's definition is the one the abstract
- * and the method section of the paper give (global branch = attention to the
- * mean-pooled key and value of each block); the split is this library's.
+ * between the two calls.  The operator is the one the paper's abstract
+ * describes (each query also attends to the mean-pooled keys and values of the
+ * blocks its window misses); the split into two calls is this library's.
  *
  * pack3d_backward_summary_grads stages q, k, v, out, lse and dout into the
- * workspace and writes dks, dvs [B, H, nb, head_dim] fp32 (the blocks of the
- * whole volume, nb = pack3d_params.nb order): the gradients of sum(dout * out)
+ * workspace and writes dks, dvs [B, H, nb, head_dim] fp32 (nb blocks of the
+ * whole volume in block-raster order, as pack3d_block_summaries writes the
+ * summaries): the gradients of sum(dout * out)
  * with respect to the block summaries, over the call's owned queries (all
  * queries unless the call is a slab).  ksum, vsum [B, H, nb, head_dim] fp32:
  * the summaries the forward used - for a slab the all-reduced summaries of the
