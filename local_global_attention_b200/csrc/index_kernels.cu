@@ -13,10 +13,34 @@ namespace {
 
 constexpr int ERR_RANGE = 1, ERR_DUP = 2;
 
+// cos and sin of c * base^(-2j/da) (axial: c a coordinate value of an axis)
+// or of p * base^(-2j/d) (packed mode: p a packed position), evaluated in
+// double precision.
+__device__ __forceinline__ void rope_entry(const Geo& g, float base, float* tab, int64_t e) {
+  const bool packed = g.rope_mode == PACK3D_ROPE_PACKED;
+  int64_t rows = packed ? g.N : g.Z + g.Y + g.X;
+  if (e >= rows * g.rope_len) return;
+  int row = (int)(e / g.rope_len), j = (int)(e % g.rope_len);
+  // axial rows: the z rows of a z-slab turn by the global plane z + z_origin
+  int c = packed ? row : (row < g.Z ? row + g.zo : (row < g.Z + g.Y ? row - g.Z : row - g.Z - g.Y));
+  double theta = pow((double)base, -2.0 * (double)j / (double)(packed ? g.d : g.da));
+  double sn, cs;
+  sincos((double)c * theta, &sn, &cs);
+  tab[2 * e + 0] = (float)cs;
+  tab[2 * e + 1] = (float)sn;
+}
+
 // Scatter packed index -> voxel, detect out-of-range and duplicated voxels,
 // count tokens per query tile (histogram of the counting sort) and per block.
+// Blocks past the tokens' (blockIdx.x >= nblk) fill the rotation table, which
+// depends on the geometry only, alongside.
 __global__ void k_scatter_coords(Geo g, const int16_t* __restrict__ coords, int32_t* vol,
-                                 int32_t* cnt, int32_t* bcount, int32_t* err) {
+                                 int32_t* cnt, int32_t* bcount, int32_t* err, unsigned nblk,
+                                 float rope_base, float* rope) {
+  if (blockIdx.x >= nblk) {
+    rope_entry(g, rope_base, rope, (blockIdx.x - nblk) * (int64_t)blockDim.x + threadIdx.x);
+    return;
+  }
   int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   if (t >= (int64_t)g.B * g.N) return;
   int b = (int)(t / g.N);
@@ -157,12 +181,36 @@ __device__ __forceinline__ void halo_box(const Geo& g, int t, int& hz0, int& hy0
   hx = min(g.X, x0 + lx + g.rx) - hx0;
 }
 
-__global__ void k_halo_sizes(Geo g, int32_t* sizes) {
-  int t = blockIdx.x * blockDim.x + threadIdx.x;
-  if (t >= g.nT) return;
-  int hz0, hy0, hx0, hz, hy, hx;
-  halo_box(g, t, hz0, hy0, hx0, hz, hy, hx);
-  sizes[t] = hz * hy * hx;
+// Offsets of the tiles' halo lists (exclusive scan of the halo box sizes, a
+// pure function of the geometry), one CTA of NT threads.
+template <int NT>
+__global__ void k_halo_offsets(Geo g, int32_t* off) {
+  __shared__ int32_t part[NT];
+  const int n = g.nT;
+  const int per = (n + NT - 1) / NT;
+  const int lo = threadIdx.x * per, hi = min(n, lo + per);
+  auto size = [&](int t) {
+    int hz0, hy0, hx0, hz, hy, hx;
+    halo_box(g, t, hz0, hy0, hx0, hz, hy, hx);
+    return hz * hy * hx;
+  };
+  int32_t s = 0;
+  for (int i = lo; i < hi; ++i) s += size(i);
+  part[threadIdx.x] = s;
+  __syncthreads();
+  // Hillis-Steele inclusive scan of the per-thread sums.
+  for (int d = 1; d < NT; d <<= 1) {
+    int32_t add = threadIdx.x >= d ? part[threadIdx.x - d] : 0;
+    __syncthreads();
+    part[threadIdx.x] += add;
+    __syncthreads();
+  }
+  int32_t run = threadIdx.x == 0 ? 0 : part[threadIdx.x - 1];
+  for (int i = lo; i < hi; ++i) {
+    off[i] = run;
+    run += size(i);
+  }
+  if (threadIdx.x == NT - 1) off[n] = part[NT - 1];
 }
 
 // Halo lists, one CTA per (tile, batch item), raster order over the halo box.
@@ -180,24 +228,6 @@ __global__ void k_halo_lists(Geo g, const int32_t* __restrict__ vol,
     int x = e % hx, y = (e / hx) % hy, z = e / (hx * hy);
     dst[e] = vb[((hz0 + z) * g.Y + (hy0 + y)) * g.X + (hx0 + x)];
   }
-}
-
-// cos and sin of c * base^(-2j/da) (axial: c a coordinate value of an axis)
-// or of p * base^(-2j/d) (packed mode: p a packed position), evaluated in
-// double precision.
-__global__ void k_rope_table(Geo g, float base, float* tab) {
-  int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-  const bool packed = g.rope_mode == PACK3D_ROPE_PACKED;
-  int64_t rows = packed ? g.N : g.Z + g.Y + g.X;
-  if (e >= rows * g.rope_len) return;
-  int row = (int)(e / g.rope_len), j = (int)(e % g.rope_len);
-  // axial rows: the z rows of a z-slab turn by the global plane z + z_origin
-  int c = packed ? row : (row < g.Z ? row + g.zo : (row < g.Z + g.Y ? row - g.Z : row - g.Z - g.Y));
-  double theta = pow((double)base, -2.0 * (double)j / (double)(packed ? g.d : g.da));
-  double sn, cs;
-  sincos((double)c * theta, &sn, &cs);
-  tab[2 * e + 0] = (float)cs;
-  tab[2 * e + 1] = (float)sn;
 }
 
 __global__ void k_init_err(int32_t* err) {
@@ -221,7 +251,12 @@ int launch_build_index(const Geo& g, const int16_t* coords, const pack3d_index* 
   k_init_err<<<1, 1, 0, s>>>(idx->err);
   int nthr = 256;
   unsigned nblk = (unsigned)((tokens + nthr - 1) / nthr);
-  k_scatter_coords<<<nblk, nthr, 0, s>>>(g, coords, idx->vol, cnt, idx->bcount, idx->err);
+  const int64_t entries =
+      (g.rope_mode == PACK3D_ROPE_PACKED ? (int64_t)g.N : (int64_t)(g.Z + g.Y + g.X)) *
+      g.rope_len;
+  const unsigned rope_blk = (unsigned)((entries + nthr - 1) / nthr);
+  k_scatter_coords<<<nblk + rope_blk, nthr, 0, s>>>(g, coords, idx->vol, cnt, idx->bcount,
+                                                    idx->err, nblk, rope_base, idx->rope);
   k_exclusive_scan<1024><<<g.B, 1024, 0, s>>>(cnt, idx->tile_off, g.nT, g.nT, g.nT + 1);
   if (g.partial) {
     k_tile_perm<<<dim3((g.nT + 3) / 4, g.B), 128, 0, s>>>(g, idx->vol, idx->tile_off, idx->perm,
@@ -232,15 +267,9 @@ int launch_build_index(const Geo& g, const int16_t* coords, const pack3d_index* 
   } else {
     k_tile_scatter<<<nblk, nthr, 0, s>>>(g, coords, idx->tile_off, idx->perm, idx->err);
   }
-  // Halo sizes reuse the histogram space (tile_off already holds the scan).
-  k_halo_sizes<<<(g.nT + 255) / 256, 256, 0, s>>>(g, cnt);
-  k_exclusive_scan<1024><<<1, 1024, 0, s>>>(cnt, idx->nbr_off, g.nT, 0, 0);
+  k_halo_offsets<1024><<<1, 1024, 0, s>>>(g, idx->nbr_off);
   k_halo_lists<<<dim3(g.nT, g.B), 256, 0, s>>>(g, idx->vol, idx->nbr_off, idx->nbr, idx->err);
-  const int64_t entries =
-      (g.rope_mode == PACK3D_ROPE_PACKED ? (int64_t)g.N : (int64_t)(g.Z + g.Y + g.X)) *
-      g.rope_len;
-  k_rope_table<<<(unsigned)((entries + 255) / 256), 256, 0, s>>>(g, rope_base, idx->rope);
-  count_launches(8);
+  count_launches(6);
   return cuda_status(cudaGetLastError());
 }
 
