@@ -340,10 +340,15 @@ class Runner:
 
 
 def kernel_sources_sha256():
-    """sha256 over the attention kernel's source files, in order."""
+    """sha256 over the attention kernel's source files, in order, with line
+    comments and blank lines dropped (a comment edit leaves the kernel as it
+    was profiled)."""
     h = hashlib.sha256()
     for f in TC_SOURCES:
-        h.update(open(f, "rb").read())
+        for line in open(f, encoding="utf-8"):
+            code = line.split("//", 1)[0].rstrip()
+            if code:
+                h.update(code.encode() + b"\n")
     return h.hexdigest()
 
 

@@ -576,9 +576,9 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       if (lane == 0) mbar_arrive(&sm.p_full[bi]);
     }
     // ---- epilogue ----
-    // o_final completes once, after the last PV product.  (Waiting on o_done
-    // here could name a phase by a parity the barrier has already passed twice:
-    // a wait must never trail the barrier by two phases.)
+    // o_final completes once, after the last PV product.  (Waiting on a
+    // buffer's buf_free here could name a phase by a parity the barrier has
+    // already passed twice: a wait must never trail the barrier by two phases.)
     if (ok)
       ok = __all_sync(0xffffffffu, mbar_wait_or_abort(&sm.o_final, 0, WAIT_LIMIT, abort_flag));
     if (ok) {
