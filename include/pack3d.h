@@ -354,6 +354,17 @@ PACK3D_API int pack3d_backward_noalloc(const pack3d_params* p, const pack3d_inde
  * the paper: an instrumentation aid. */
 PACK3D_API uint64_t pack3d_kernel_launches(void);
 
+/* Diagnostic of the bounded device-side waits (no counterpart in the paper).
+ * Every wait in the library's kernels polls an mbarrier at most a fixed number
+ * of times; a CTA that runs out sets the timeout bit of the index error word
+ * (reported as PACK3D_ERR_TIMEOUT by pack3d_index_check), lets its own copies
+ * and tensor-core products land and returns.  This call launches one warp
+ * that waits, with at most `polls` polls (1 .. 2^24), on a barrier phase that
+ * nothing completes, then synchronises the stream and returns
+ * PACK3D_ERR_TIMEOUT - the status a timed-out wait produces; PACK3D_ERR_ARG
+ * for a poll count out of range. */
+PACK3D_API int pack3d_wait_selftest(uint32_t polls, pack3d_stream_t stream);
+
 /* Human-readable text of a status code (static storage). */
 PACK3D_API const char* pack3d_strerror(int status);
 

@@ -86,6 +86,7 @@ struct Smem {
   uint64_t p_full[2];    // P and dS of the buffer's chunk written
   uint64_t acc_done[2];  // the accumulations reading the buffer are done
   uint64_t acc_final;    // every accumulation of the CTA is done
+  uint64_t drain;         // a CTA that gave up: its issued MMAs are done
   uint32_t tmem_base;
   int32_t abort;
 };
@@ -254,6 +255,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(&sm.acc_done[i], 1);
     }
     mbar_init(&sm.acc_final, 1);
+    mbar_init(&sm.drain, 1);
     sm.abort = 0;
     fence_barrier_init();
   }
@@ -674,6 +676,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   __syncthreads();
   if (sm.abort && tid == 0) atomicOr(&ix.err[0], ERR_TIMEOUT_BIT);
   if (warp == MMA_WARP) {
+    // A CTA that gave up may still have products in flight (no role waited
+    // for the last one): they land before the columns are freed (bounded).
+    if (sm.abort) {
+      mma_commit_warp(&sm.drain);
+      if (lane == 0) mbar_wait(&sm.drain, 0, WAIT_LIMIT);
+      __syncwarp();
+    }
     tc_fence_after();
     tmem_dealloc(tbase, TMEM_COLS);
   }

@@ -104,6 +104,7 @@ struct Smem {
   uint64_t p_full[2];    // P of the buffer's chunk written
   uint64_t buf_free[2];  // the PV product reading the buffer's P is done
   uint64_t o_final;      // one phase: every PV product of the tile is done
+  uint64_t drain;         // a CTA that gave up: its issued MMAs are done
   uint32_t tmem_base;
   int32_t abort;
 };
@@ -262,6 +263,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
       mbar_init(&sm.buf_free[i], 1);
     }
     mbar_init(&sm.o_final, 1);
+    mbar_init(&sm.drain, 1);
     sm.abort = 0;
     fence_barrier_init();
   }
@@ -623,6 +625,13 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   __syncthreads();
   if (sm.abort && tid == 0) atomicOr(&ix.err[0], ERR_TIMEOUT_BIT);
   if (warp == MMA_WARP) {
+    // A CTA that gave up may still have products in flight (no role waited
+    // for the last one): they land before the columns are freed (bounded).
+    if (sm.abort) {
+      mma_commit_warp(&sm.drain);
+      if (lane == 0) mbar_wait(&sm.drain, 0, WAIT_LIMIT);
+      __syncwarp();
+    }
     tc_fence_after();
     tmem_dealloc(tbase, TMEM_COLS);
   }

@@ -24,7 +24,7 @@ EXPORTS = ("pack3d_index_bytes", "pack3d_index_init", "pack3d_build_index", "pac
            "pack3d_window_forward", "pack3d_stage_kv", "pack3d_forward_staged",
            "pack3d_backward_workspace_bytes", "pack3d_backward", "pack3d_backward_summary_grads",
            "pack3d_backward_from_summary_grads", "pack3d_backward_noalloc",
-           "pack3d_kernel_launches", "pack3d_strerror")
+           "pack3d_kernel_launches", "pack3d_wait_selftest", "pack3d_strerror")
 
 
 class Params(ctypes.Structure):
@@ -97,6 +97,7 @@ def load(build_if_missing: bool = True):
                                                            ctypes.c_size_t, vp, vp, vp, vp]
         lib.pack3d_backward_noalloc.argtypes = [P(Params), P(Index), vp, vp, vp, vp, vp, vp, vp,
                                                 vp, vp, vp]
+        lib.pack3d_wait_selftest.argtypes = [ctypes.c_uint32, vp]
         lib.pack3d_kernel_launches.argtypes = []
         lib.pack3d_kernel_launches.restype = ctypes.c_uint64
         lib.pack3d_strerror.argtypes = [ctypes.c_int]
@@ -110,6 +111,11 @@ def load(build_if_missing: bool = True):
 def pack3d_kernel_launches() -> int:
     """Kernels the library has launched in this process so far."""
     return int(load().pack3d_kernel_launches())
+
+
+def pack3d_wait_selftest(polls: int = 1000, stream=None) -> int:
+    """Status of a bounded device wait that runs out (ERR_TIMEOUT expected)."""
+    return int(load().pack3d_wait_selftest(ctypes.c_uint32(polls), _stream(stream)))
 
 
 def strerror(status: int) -> str:

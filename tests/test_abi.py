@@ -309,3 +309,11 @@ def test_two_call_backward_checks_without_cuda(lib):
     idxr = index_for(psr)
     assert first(psr, idxr, fake, 1 << 40) == P.ERR_UNSUPPORTED
     assert P.pack3d_kernel_launches() == n0
+
+
+def test_wait_selftest_argument_checks_without_cuda(lib):
+    """A poll count of 0 or above 2^24 is rejected before anything is launched."""
+    n0 = P.pack3d_kernel_launches()
+    assert lib.pack3d_wait_selftest(ctypes.c_uint32(0), None) == P.ERR_ARG
+    assert lib.pack3d_wait_selftest(ctypes.c_uint32((1 << 24) + 1), None) == P.ERR_ARG
+    assert P.pack3d_kernel_launches() == n0

@@ -2,7 +2,8 @@
 a one-voxel volume (its block always meets the window: no summary term, the
 output is v), one-voxel-thick planes and lines (a 1 x 1 x X line, a Z x 1 x 1
 column), a block as large as the whole volume (one summary, never seen), and a
-partly occupied volume holding a single token or one token per block."""
+partly occupied volume holding a single token or one token per block; and a
+bounded device wait that runs out (ERR_TIMEOUT, the context stays usable)."""
 import numpy as np
 import pytest
 
@@ -58,3 +59,15 @@ def test_one_voxel_output_is_v():
     inp = I.make_inputs(wl, "random")
     res = gpu_run(wl, inp)
     np.testing.assert_array_equal(res["out"].float().numpy(), inp["v"].float().numpy())
+
+
+def test_bounded_wait_times_out_and_the_context_stays_usable(oracle_lib):
+    """A device wait on a barrier phase that nothing completes gives up after
+    its poll limit and reports ERR_TIMEOUT; the next calls run normally."""
+    from local_global_attention_b200 import pack3d as P
+    assert P.pack3d_wait_selftest(1000) == P.ERR_TIMEOUT
+    wl = EDGE[2]
+    inp = I.make_inputs(wl, "random")
+    res = gpu_run(wl, inp)
+    out, lse = oracle.forward(wl, inp["coords"], inp["q"], inp["k"], inp["v"])
+    assert_close(res["out"], out, wl.dtype, "out after the timed-out wait")
