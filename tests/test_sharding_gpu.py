@@ -277,3 +277,32 @@ def test_slab_calls_reject_other_paths():
     with pytest.raises(P.Pack3dError) as e:
         P.pack3d_backward(params, idx, x, x, x, x, lse, x)
     assert e.value.status == P.ERR_UNSUPPORTED
+
+
+def test_sharded_entry_points_single_rank():
+    """sharding.sharded_forward and sharded_backward end to end in a one-rank
+    process group (gloo): the slab is the whole volume, so out, lse and the
+    gradients equal the unsharded calls bit for bit."""
+    import socket
+
+    import torch.distributed as dist
+    wl = SHARD_CASES[0][0].replace(value_scale=1.0 / np.sqrt(96), name="single_rank")
+    inp = I.make_inputs(wl, "random", with_dout=True)
+    ref = gpu_run(wl, inp, with_backward=True)
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1)
+    try:
+        slab = S.plan_slabs(wl.Z, wl.block[0], (wl.window[0] - 1) // 2, 1)[0]
+        d = {k: v.cuda() for k, v in inp.items() if k != "order"}
+        coords = d["coords"].to(torch.int16)
+        out, lse = S.sharded_forward(wl, slab, coords, d["q"], d["k"], d["v"])
+        dq, dk, dv = S.sharded_backward(wl, slab, coords, d["q"], d["k"], d["v"], out, lse,
+                                        d["dout"])
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()
+    assert torch.equal(out.cpu(), ref["out"]) and torch.equal(lse.cpu(), ref["lse"])
+    for name, g in zip(("dq", "dk", "dv"), (dq, dk, dv)):
+        assert torch.equal(g.cpu(), ref[name]), name
