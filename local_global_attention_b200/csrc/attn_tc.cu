@@ -181,32 +181,22 @@ __global__ void k_summaries_bf16(const float4* __restrict__ ks, const float4* __
 
 // P = 2^(S c2 + mneg) for all 32 keys (masked ones carry the penalty), packed
 // in pairs into p[0..15]; returns the sum.
-// The scaling and the running sums use the paired fp32 instructions
-// (fma/add.rn.f32x2: two values per instruction).
+// The scaling and the running sums use the paired fp32 arithmetic (two values
+// per instruction).
 __device__ __forceinline__ float exp_pack_all(const uint32_t (&sv)[32], float c2, float mneg,
                                               uint32_t* p) {
-  uint64_t acc[2] = {0ull, 0ull};
-  uint64_t cc, mm;
-  asm("mov.b64 %0, {%1, %1};" : "=l"(cc) : "f"(c2));
-  asm("mov.b64 %0, {%1, %1};" : "=l"(mm) : "f"(mneg));
+  float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  const float2 cc = make_float2(c2, c2), mm = make_float2(mneg, mneg);
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    uint64_t sp, a;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(sp) : "r"(sv[2 * i]), "r"(sv[2 * i + 1]));
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(a) : "l"(sp), "l"(cc), "l"(mm));
-    float a0, a1;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(a));
-    const float e0 = ex2(a0), e1 = ex2(a1);
-    uint64_t ep;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(ep) : "f"(e0), "f"(e1));
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(acc[i & 1]) : "l"(acc[i & 1]), "l"(ep));
-    p[i] = pack_bf16x2(e0, e1);
+    const float2 a = f2_fma(make_float2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])),
+                            cc, mm);
+    const float2 e = make_float2(ex2(a.x), ex2(a.y));
+    acc[i & 1] = f2_add(acc[i & 1], e);
+    p[i] = pack_bf16x2(e.x, e.y);
   }
-  uint64_t t;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(t) : "l"(acc[0]), "l"(acc[1]));
-  float t0, t1;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(t0), "=f"(t1) : "l"(t));
-  return t0 + t1;
+  const float2 t = f2_add(acc[0], acc[1]);
+  return t.x + t.y;
 }
 
 __device__ __forceinline__ float plain_max(const uint32_t (&sv)[32]) {
