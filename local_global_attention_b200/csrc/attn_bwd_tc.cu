@@ -592,13 +592,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           const float2 ds = f2_mul(
               p, f2_add(make_float2(__uint_as_float(dv[2 * i]), __uint_as_float(dv[2 * i + 1])),
                         make_float2(-dl.x, -dl.y)));
-          pw[i] = pack_bf16x2(p.x, p.y);
+          if (TWO_ACC) pw[i] = pack_bf16x2(p.x, p.y);
           dw[i] = pack_bf16x2(ds.x, ds.y);
         }
       }
-      // P over this half's S columns, dS over its dP columns (each half writes
-      // only columns it has read)
-      tmem_st16(tS, pw);
+      // P over this half's S columns (only the roles whose second product reads
+      // it), dS over its dP columns (each half writes only columns it has read)
+      if (TWO_ACC) tmem_st16(tS, pw);
       tmem_st16(tdP, dw);
       tmem_wait_st();
       tc_fence_before();
