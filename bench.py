@@ -435,6 +435,54 @@ def micro1m_line(args, pk):
     return res
 
 
+def fp32_mode_line(args):
+    """The fp32 mode (CUDA cores, 1e-4 bound) at the 65k shape: index build,
+    block summaries and forward through the C ABI, a few timed steps, with the
+    useful FLOP rate against the fp32 FMA peak (148 SMs x 128 lanes x 2 FLOP
+    at the clock sampled here)."""
+    import torch
+
+    from local_global_attention_b200 import configs as C
+    from local_global_attention_b200 import inputs as I
+    from local_global_attention_b200 import pack3d as P
+    wl = C.VOL65K.replace(dtype="fp32", value_scale=1.0 / math.sqrt(96), name="vol_32x32x64_fp32")
+    inp = I.make_inputs(wl, "random")
+    d = {k: v.cuda() for k, v in inp.items() if k != "order"}
+    params = P.make_params(wl)
+    idx = P.IndexBuffers(params)
+    ksum = torch.empty(wl.B, wl.H, wl.n_blocks, wl.d, device="cuda")
+    vsum = torch.empty_like(ksum)
+    out = torch.empty_like(d["q"])
+    lse = torch.empty(wl.B, wl.H, wl.N, device="cuda")
+
+    def step():
+        P.pack3d_build_index(params, d["coords"], idx)
+        P.pack3d_block_summaries(params, idx, d["k"], d["v"], ksum, vsum)
+        P.pack3d_forward(params, idx, d["q"], d["k"], d["v"], ksum, vsum, out=out, lse=lse)
+
+    steps = 3
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    assert P.pack3d_index_check(idx) == P.OK
+    ms = e0.elapsed_time(e1) / steps
+    work = algorithmic_work(wl)
+    tf = work["flop"] / (ms * 1e-3) / 1e12
+    res = {"workload": "vol_32x32x64 in fp32 (same shape and seed layout, CUDA-core kernels)",
+           "ms_per_step": ms, "value": wl.B * wl.N / (ms * 1e-3), "unit": UNIT, "steps": steps,
+           "tflops_useful_whole_step": tf}
+    del d, inp, out, lse, ksum, vsum, idx
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args):
     import ctypes
 
@@ -557,6 +605,7 @@ def run_ours(args):
     micro = None
     if args.micro1m and world == 1:
         micro = micro1m_line(args, pk)
+    fp32 = fp32_mode_line(args) if args.micro1m and world == 1 else None
 
     if rank != 0:
         barrier(world)
@@ -635,6 +684,12 @@ def run_ours(args):
     }
     if micro is not None:
         line["micro1m"] = micro
+    if fp32 is not None:
+        clock_mhz = (line.get("clocks") or {}).get("sm_mhz") or 1965.0
+        fma_peak = 148 * 128 * 2 * clock_mhz / 1e6  # TFLOP/s
+        fp32["fp32_fma_peak_tflops"] = fma_peak
+        fp32["frac_of_fma_peak"] = fp32["tflops_useful_whole_step"] / fma_peak
+        line["fp32_mode"] = fp32
     if not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(wl, inp, args.cpu_sample)
     barrier(world)
@@ -726,7 +781,7 @@ def main():
                     help="forward / backward: time that alone and print a short line "
                          "(for profiler runs)")
     ap.add_argument("--no-micro1m", dest="micro1m", action="store_false",
-                    help="skip the 1M-token workload section")
+                    help="skip the 1M-token workload and the fp32-mode sections")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
