@@ -13,7 +13,8 @@
 // Kernels of one call:
 //   staging: the rotated keys and the values in grid order with the block
 //     summaries (the forward's staging kernel), and k_bwd_stage_q: the rotated
-//     queries and dO in grid order, and per voxel (lse log2 e, delta).
+//     queries and dO in grid order, and per voxel (lse log2 e, delta) in fp32
+//     and as statistic channels (below).
 //   k_bwd_tc<DSUM>: rows = 128 block summaries, columns = every query of the
 //     volume in chunks, split over CTAs; partial dkbar, dvbar per split, added
 //     in split order by k_bwd_sum_reduce (deterministic).
@@ -32,13 +33,21 @@
 //   channel-contiguous B operands.  S and dP are double-buffered, so the next
 //   chunk's products run while the elementwise warps work on this one.
 //
+//   Where L and delta belong to the columns (dk/dv and the summary role) they
+//   ride in the products: 16 more contraction channels hold, per column,
+//   -L / (tau log2 e) and -delta, each split into three bf16 parts (their sum is
+//   the fp32 value), against ones in the rows' channels (A1's in tensor memory,
+//   A2's in shared memory).  S and dP then arrive as S - L / (tau log2 e) and
+//   dP - delta, so the elementwise warps read no per-column statistics.
+//
 //   role  A1 (TMEM)   A2 (smem)  C1         C2      L, delta    acc1     acc2
 //   DQ    q~ tile     dO tile    k~ / kbar  v / vbar per row    dq~      -
 //   DKDV  k~ tile     v tile     q~ chunk   dO      per column  dk~      dv
 //   DSUM  kbar rows   vbar rows  q~ chunk   dO      per column  dkbar    dvbar
 //
 // Tensor memory (512 columns, one CTA per SM): acc1 [0, 96), acc2 [96, 192),
-// buffers b = 0, 1 at 192 + 128 b (S: 64 columns, dP: 64 columns), A1 [448, 504).
+// buffers b = 0, 1 at 192 + 128 b (S: 64 columns, dP: 64 columns), A1 [448, 512)
+// (96 channels, 16 penalty channels, 16 statistic channels).
 // Warps 0-7 elementwise (warp w: TMEM lanes 32 (w % 4) .., columns of half
 // w / 4 of the chunk), warp 8 MMA issue, warp 9 TMA producer.  Every wait is
 // bounded; a CTA that gives up sets the timeout bit of the index error word.
@@ -63,7 +72,7 @@ constexpr int NSTAGE = 6;
 constexpr int SEGC = KCH * 64;    // one 32-channel segment of a 64-row chunk (4 KB)
 constexpr int SEGR = 128 * 64;    // one 32-channel segment of the 128-row tile (8 KB)
 constexpr uint32_t CHUNK_BYTES = 6 * SEGC;
-constexpr uint32_t STAT_BYTES = KCH * 16;  // (L, delta, 0, 0) per column
+constexpr uint32_t STAT_BYTES = KCH * 32;  // 16 bf16 statistic channels per column
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t COL_ACC1 = 0, COL_ACC2 = 96, COL_BUF = 192, BUF_COLS = 128, COL_A1 = 448;
 constexpr int NSOFT_WARPS = 8, MMA_WARP = 8, TMA_WARP = 9, NTHREADS = 320;
@@ -78,7 +87,8 @@ struct Smem {
   uint8_t c1[NSTAGE][3 * SEGC];  // column operand 1 of each stage
   uint8_t c2[NSTAGE][3 * SEGC];  // column operand 2
   uint8_t cp[NSTAGE][KCH * 32];  // penalty channels of the column rows (32-byte swizzle)
-  float4 st[NSTAGE][KCH];        // per-column (L, delta, 0, 0)
+  uint8_t cs[NSTAGE][KCH * 32];  // statistic channels of the column rows (32-byte swizzle)
+  uint8_t a2x[128 * 32];         // the rows' statistic channels of the dP product
   PenaltyTable pt;               // the tile's penalty channels per axis (dense volumes)
   uint64_t a_full;               // A1 in tensor memory and A2 loaded
   uint64_t kv_full[NSTAGE], kv_empty[NSTAGE];
@@ -91,6 +101,10 @@ struct Smem {
   int32_t abort;
 };
 constexpr size_t SMEM_REQUEST = sizeof(Smem) + 1024;
+static_assert(SMEM_REQUEST <= 232448, "shared memory of one CTA");
+static_assert(offsetof(Smem, cs) % 1024 == 0 && offsetof(Smem, a2x) % 256 == 0 &&
+                  offsetof(Smem, cp) % 1024 == 0,
+              "32-byte-swizzled operands start on their pattern's boundary");
 
 // Pointers of one backward kernel launch (which ones a role reads is in the
 // role table above).
@@ -108,7 +122,7 @@ struct BwdArgs {
 struct BwdMaps {
   CUtensorMap c1, c2;    // column chunks: grid-order volumes, box {32, 16, 2, 2, 1}
   CUtensorMap c1s, c2s;  // DQ summary columns: bf16 summaries, box {32, 64, 1}
-  CUtensorMap st;        // per-column statistics: [B*H][Z][Y][X][4] fp32, box {4, 16, 2, 2, 1}
+  CUtensorMap st;        // per-column statistic channels: [B*H][Z][Y][X][16] bf16, box {16, 16, 2, 2, 1}
   CUtensorMap a2;        // row operand 2: box {32, 8, 2, 2, 1} (tile) or {32, 128, 1} (summaries)
 };
 
@@ -313,7 +327,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tma_load_5d(sm.c1[s] + seg * SEGC, &maps.c1, seg * 32, x, y, z, bh, &sm.kv_full[s]);
             tma_load_5d(sm.c2[s] + seg * SEGC, &maps.c2, seg * 32, x, y, z, bh, &sm.kv_full[s]);
           }
-          if (COL_STATS) tma_load_5d(&sm.st[s][0], &maps.st, 0, x, y, z, bh, &sm.kv_full[s]);
+          if (COL_STATS) tma_load_5d(sm.cs[s], &maps.st, 0, x, y, z, bh, &sm.kv_full[s]);
         } else {
           mbar_arrive_expect_tx(&sm.kv_full[s], CHUNK_BYTES);
           const int Bs = (j - n_local) * KCH;
@@ -355,6 +369,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint64_t c2m = sdesc_sw64(smem_u32(sm.c2[0]), SEGC, 512);
     const uint64_t a2d = sdesc_sw64(smem_u32(sm.a2), 16, 512);
     const uint64_t cpd = sdesc_sw32(smem_u32(sm.cp[0]), 16, 256);
+    const uint64_t csd = sdesc_sw32(smem_u32(sm.cs[0]), 16, 256);
+    const uint64_t a2xd = sdesc_sw32(smem_u32(sm.a2x), 16, 256);
     auto wait_all = [&](uint64_t* bar, uint32_t parity) {
       return __all_sync(0xffffffffu, mbar_wait_or_abort(bar, parity, WAIT_LIMIT, abort_flag));
     };
@@ -376,12 +392,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         if (PENALTY && j < n_local)
           mma_ts_warp(tS, tbase + COL_A1 + 48, cpd + ((uint32_t)(s * KCH * 32) >> 4), idesc_s, 1u);
+        // S - L / (tau log2 e) and dP - delta: the column statistics ride in
+        // 16 more contraction channels (ones in the rows' channels)
+        if (COL_STATS)
+          mma_ts_warp(tS, tbase + COL_A1 + 56, csd + ((uint32_t)(s * KCH * 32) >> 4), idesc_s, 1u);
 #pragma unroll
         for (int st = 0; st < D / 16; ++st) {
           const uint32_t ao = (st >> 1) * SEGR + (st & 1) * 32;
           const uint32_t ko = so + (st >> 1) * SEGC + (st & 1) * 32;
           mma_ss_warp(tdP, a2d + (ao >> 4), c2k + (ko >> 4), idesc_s, st > 0);
         }
+        if (COL_STATS)
+          mma_ss_warp(tdP, a2xd, csd + ((uint32_t)(s * KCH * 32) >> 4), idesc_s, 1u);
         mma_commit_warp(&sm.s_full[bf]);
       }
       if (j >= 1) {
@@ -464,6 +486,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         tmem_st16(tq + 32, w16);
         tmem_st8(tq + 48, w8);
+        if (COL_STATS) {
+          // statistic channels: ones at 0-2 (the S product's -L / (tau log2 e)
+          // parts), and in shared memory ones at 3-5 for the dP product (-delta)
+          uint32_t ws[8] = {0x3f803f80u, 0x00003f80u, 0u, 0u, 0u, 0u, 0u, 0u};
+          tmem_st8(tq + 56, ws);
+          const uint32_t rr = (uint32_t)r;
+          *reinterpret_cast<uint4*>(sm.a2x + sw32_off(rr, 0)) =
+              make_uint4(0u, 0x3f800000u, 0x3f803f80u, 0u);
+          *reinterpret_cast<uint4*>(sm.a2x + sw32_off(rr, 1)) = make_uint4(0u, 0u, 0u, 0u);
+          fence_proxy_async_smem();
+        }
       }
       tmem_wait_st();
       tc_fence_before();
@@ -499,15 +532,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
     bool ok = true;
     for (int j = 0; j < nch; ++j) {
-      const int s = j % NSTAGE, bf = j & 1;
+      const int bf = j & 1;
       ok = __all_sync(0xffffffffu,
                       mbar_wait_or_abort(&sm.s_full[bf], (j >> 1) & 1, WAIT_LIMIT, abort_flag));
-      // the per-column statistics were written by the stage's copies: observe
-      // their completion directly (the stage is released only after this
-      // warp's p_full arrival below, so this phase is still the current one)
-      if (ok && COL_STATS)
-        ok = __all_sync(0xffffffffu, mbar_wait_or_abort(&sm.kv_full[s], (j / NSTAGE) & 1,
-                                                        WAIT_LIMIT, abort_flag));
       if (!ok) break;
       tc_fence_after();
       // which of this half's 32 columns count: all (the penalty channels mask
@@ -576,22 +603,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const float2 c2p = make_float2(c2, c2);
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          float2 L = make_float2(Lrow, Lrow), dl = make_float2(Drow, Drow);
-          if (COL_STATS) {
-            const float4 s0 = sm.st[s][32 * hf + 2 * i], s1 = sm.st[s][32 * hf + 2 * i + 1];
-            L = make_float2(s0.x, s1.x);
-            dl = make_float2(s0.y, s1.y);
-          }
-          float2 a = f2_fma(make_float2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])),
-                            c2p, make_float2(-L.x, -L.y));
+          const float2 sp = make_float2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1]));
+          const float2 dpp = make_float2(__uint_as_float(dv[2 * i]), __uint_as_float(dv[2 * i + 1]));
+          // column roles: the products already hold S - L / (tau log2 e) and dP - delta
+          float2 a = COL_STATS ? f2_mul(sp, c2p) : f2_fma(sp, c2p, make_float2(-Lrow, -Lrow));
           if (use_bits) {
             if (!((bits >> (2 * i)) & 1u)) a.x = -INFINITY;
             if (!((bits >> (2 * i + 1)) & 1u)) a.y = -INFINITY;
           }
           const float2 p = make_float2(ex2(a.x), ex2(a.y));
-          const float2 ds = f2_mul(
-              p, f2_add(make_float2(__uint_as_float(dv[2 * i]), __uint_as_float(dv[2 * i + 1])),
-                        make_float2(-dl.x, -dl.y)));
+          const float2 ds = f2_mul(p, COL_STATS ? dpp : f2_add(dpp, make_float2(-Drow, -Drow)));
           if (TWO_ACC) pw[i] = pack_bf16x2(p.x, p.y);
           dw[i] = pack_bf16x2(ds.x, ds.y);
         }
@@ -715,12 +736,23 @@ __global__ void k_bwd_sum_reduce(Geo g, const int32_t* __restrict__ err, int nsp
 // batch item), as the forward's staging of keys and values.
 constexpr int STAGE_XS = 64;
 
+// x as hi + mid + lo, each the bf16 rounding of what is left (bit patterns).
+__device__ __forceinline__ void split3_bf16(float x, uint32_t (&w)[3]) {
+#pragma unroll
+  for (int i = 0; i < 3; ++i) {
+    const __nv_bfloat16 h = __float2bfloat16_rn(x);
+    w[i] = (uint32_t)__bfloat16_as_ushort(h);
+    x -= __bfloat162float(h);
+  }
+}
+
 template <typename TO>
 __global__ void __launch_bounds__(256)
     k_bwd_stage_q(Geo g, pack3d_index ix, const __nv_bfloat16* __restrict__ q,
                   const __nv_bfloat16* __restrict__ dout, const TO* __restrict__ out,
                   const float* __restrict__ lse, __nv_bfloat16* __restrict__ qg,
-                  __nv_bfloat16* __restrict__ dog, float4* __restrict__ stat) {
+                  __nv_bfloat16* __restrict__ dog, float4* __restrict__ stat,
+                  uint4* __restrict__ schan) {
   if (ix.err[0]) return;
   __shared__ int32_t tok[STAGE_XS];
   const int xb = blockIdx.x * STAGE_XS, zy = blockIdx.y, b = blockIdx.z;
@@ -761,6 +793,8 @@ __global__ void __launch_bounds__(256)
     const int x = it % nx, hh = it / nx;
     if (tok[x] < 0) {
       stat[grid_row(hh) + x] = make_float4(0.f, 0.f, 0.f, 0.f);
+      schan[2 * (grid_row(hh) + x)] = make_uint4(0u, 0u, 0u, 0u);
+      schan[2 * (grid_row(hh) + x) + 1] = make_uint4(0u, 0u, 0u, 0u);
       continue;
     }
     const int64_t row = (((int64_t)b * g.N + tok[x]) * H + hh) * D;
@@ -795,11 +829,19 @@ __global__ void __launch_bounds__(256)
     }
     const float L = lse[((int64_t)b * H + hh) * g.N + tok[x]] * LOG2E;
     stat[grid_row(hh) + x] = make_float4(L, acc, 0.f, 0.f);
+    // the column roles' statistic channels: -L / (tau log2 e) and -delta, each
+    // as three bf16 parts whose sum is the fp32 value (to fp32 precision)
+    uint32_t wl[3], wd[3];
+    split3_bf16(-L / (g.tau * LOG2E), wl);
+    split3_bf16(-acc, wd);
+    schan[2 * (grid_row(hh) + x)] =
+        make_uint4(wl[0] | (wl[1] << 16), wl[2] | (wd[0] << 16), wd[1] | (wd[2] << 16), 0u);
+    schan[2 * (grid_row(hh) + x) + 1] = make_uint4(0u, 0u, 0u, 0u);
   }
 }
 
 struct BwdWs {
-  size_t kg, vg, qg, dog, stat, ksum, vsum, ksb, vsb, dks, dvs, part, total;
+  size_t kg, vg, qg, dog, stat, schan, ksum, vsum, ksb, vsb, dks, dvs, part, total;
 };
 
 // Splits of the summary role: as many CTAs as fill one wave (one per SM), at
@@ -827,6 +869,7 @@ BwdWs bwd_layout(const Geo& g) {
   w.qg = o;   o += al(vol);
   w.dog = o;  o += al(vol);
   w.stat = o; o += al(vox * 16);
+  w.schan = o; o += al(vox * 32);
   w.ksum = o; o += al(sum32);
   w.vsum = o; o += al(sum32);
   w.ksb = o;  o += al(sum16);
@@ -873,15 +916,15 @@ bool encode_role_maps(const Geo& g, uint8_t* base, const BwdWs& w, RoleMaps& m) 
   const uint64_t sdims[3] = {(uint64_t)D, (uint64_t)g.nb, BH};
   const uint32_t scbox[3] = {32, KCH, 1};
   const uint32_t srbox[3] = {32, 128, 1};
-  const uint64_t tdims[5] = {4, (uint64_t)g.X, (uint64_t)g.Y, (uint64_t)g.Z, BH};
-  const uint32_t tbox[5] = {4, BXK, BYK, BZK, 1};
+  const uint64_t tdims[5] = {16, (uint64_t)g.X, (uint64_t)g.Y, (uint64_t)g.Z, BH};
+  const uint32_t tbox[5] = {16, BXK, BYK, BZK, 1};
   m = RoleMaps{};
   bool ok = true;
   // summary role: columns q~ / dO, stats; rows kbar (a1), vbar (A2)
   ok &= encode_bf16(&m.s.c1, base + w.qg, 5, vdims, cbox);
   ok &= encode_bf16(&m.s.c2, base + w.dog, 5, vdims, cbox);
-  ok &= encode_map(&m.s.st, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base + w.stat, 5, tdims, tbox,
-                   CU_TENSOR_MAP_SWIZZLE_NONE);
+  ok &= encode_map(&m.s.st, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base + w.schan, 5, tdims, tbox,
+                   CU_TENSOR_MAP_SWIZZLE_32B);
   ok &= encode_bf16(&m.s.a2, base + w.vsb, 3, sdims, srbox);
   m.s.c1s = m.s.c1;
   m.s.c2s = m.s.c2;
@@ -938,12 +981,13 @@ int backward_tc_summary_grads(const Geo& g, const pack3d_index* idx, const void*
     if (g.out_fp32)
       k_bwd_stage_q<float><<<grid, 256, 0, s>>>(
           g, *idx, (const __nv_bfloat16*)q, (const __nv_bfloat16*)dout, (const float*)out, lse,
-          bf(w.qg), bf(w.dog), reinterpret_cast<float4*>(base + w.stat));
+          bf(w.qg), bf(w.dog), reinterpret_cast<float4*>(base + w.stat),
+          reinterpret_cast<uint4*>(base + w.schan));
     else
       k_bwd_stage_q<__nv_bfloat16><<<grid, 256, 0, s>>>(
           g, *idx, (const __nv_bfloat16*)q, (const __nv_bfloat16*)dout,
           (const __nv_bfloat16*)out, lse, bf(w.qg), bf(w.dog),
-          reinterpret_cast<float4*>(base + w.stat));
+          reinterpret_cast<float4*>(base + w.stat), reinterpret_cast<uint4*>(base + w.schan));
     count_launches(1);
     if ((rc = cuda_status(cudaGetLastError()))) return rc;
   }

@@ -149,7 +149,8 @@ def test_noalloc_scratch_holds_the_training_shape(lib):
 def test_backward_workspace_layout(lib):
     """bf16 at head_dim 96 runs the tensor-core backward, whose workspace holds
     grid-order copies of rotated k, v, rotated q and dO (4 x [B][H][N][96]
-    bf16), per-voxel (lse, delta) pairs padded to 16 bytes, the fp32 summaries,
+    bf16), per-voxel (lse, delta) pairs padded to 16 bytes, the same as 16 bf16
+    contraction channels per voxel (32 bytes), the fp32 summaries,
     their bf16 copies, the summary gradients, and the summary role's per-split
     partial sums (2 x splits x [B][H][nb][96] fp32; the splits fill one wave of
     148 CTAs over B*H*ceil(nb/128) row tiles, at most 64); every section
@@ -166,7 +167,8 @@ def test_backward_workspace_layout(lib):
         chunks = -(-wl.Z // 2) * -(-wl.Y // 2) * -(-wl.X // 16)
         groups = wl.B * wl.H * -(-nb // 128)
         splits = max(1, min(-(-148 // groups), chunks, 64))
-        want = (4 * a256(vox * 96 * 2) + a256(vox * 16) + 2 * a256(s32) + 2 * a256(s32 // 2) +
+        want = (4 * a256(vox * 96 * 2) + a256(vox * 16) + a256(vox * 32) + 2 * a256(s32) +
+                2 * a256(s32 // 2) +
                 2 * a256(s32) + a256(splits * 2 * s32))
         assert lib.pack3d_backward_workspace_bytes(ctypes.byref(P.make_params(wl))) == want
     for wl in (C.TINY, C.TRAIN65K.replace(dtype="fp32")):
