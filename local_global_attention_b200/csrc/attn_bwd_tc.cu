@@ -576,6 +576,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             bits &= occ;
           }
           skip = __ballot_sync(0xffffffffu, bits != 0u) == 0u;
+          // (most chunks mask nothing for any row of the warp)
+          use_bits = __any_sync(0xffffffffu, bits != 0xffffffffu);
         }
       } else {
         // DQ: summaries B .. B + 31 of this half
@@ -586,7 +588,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                       : 0u;
         // empty blocks have no summary (Bs is a multiple of 32)
         if (PARTIAL && Bs < g.nb) bits &= ix.bocc[(int64_t)b * ((g.nb + 31) / 32) + Bs / 32];
-        use_bits = true;
+        use_bits = __any_sync(0xffffffffu, bits != 0xffffffffu);
         skip = __ballot_sync(0xffffffffu, bits != 0u) == 0u;
       }
       const uint32_t tS = tbase + lane_base + COL_BUF + BUF_COLS * bf + 32 * hf;

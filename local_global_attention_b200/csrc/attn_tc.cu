@@ -521,7 +521,8 @@ __global__ void __launch_bounds__(NTHREADS, 2)
         for (int i = 0; i < 32; ++i) p[i] = 0u;
       } else {
         const bool local = !SUMMARY || j < n_local;  // masked by the penalty channels
-        if (!local) {
+        // (most summary chunks mask nothing for any row of the warp)
+        if (!local && __any_sync(0xffffffffu, (bits0 & bits1) != 0xffffffffu)) {
           apply_mask(sa, bits0);
           apply_mask(sb, bits1);
         }
