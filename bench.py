@@ -435,8 +435,9 @@ def micro1m_line(args, pk):
     return res
 
 
-def fp32_mode_line(args):
-    """The fp32 mode (CUDA cores, 1e-4 bound) at the 65k shape: index build,
+def cuda_core_line(args, dtype="fp32", d=96):
+    """A configuration the CUDA-core kernels run, at the 65k shape: the fp32
+    mode (1e-4 bound), or bf16 at a head dim other than 96.  Index build,
     block summaries and forward through the C ABI, a few timed steps, with the
     useful FLOP rate against the fp32 FMA peak (148 SMs x 128 lanes x 2 FLOP
     at the clock sampled here)."""
@@ -445,20 +446,21 @@ def fp32_mode_line(args):
     from local_global_attention_b200 import configs as C
     from local_global_attention_b200 import inputs as I
     from local_global_attention_b200 import pack3d as P
-    wl = C.VOL65K.replace(dtype="fp32", value_scale=1.0 / math.sqrt(96), name="vol_32x32x64_fp32")
+    name = f"vol_32x32x64_{dtype}" + ("" if d == 96 else f"_d{d}")
+    wl = C.VOL65K.replace(dtype=dtype, d=d, value_scale=1.0 / math.sqrt(d), name=name)
     inp = I.make_inputs(wl, "random")
-    d = {k: v.cuda() for k, v in inp.items() if k != "order"}
+    dev = {k: v.cuda() for k, v in inp.items() if k != "order"}
     params = P.make_params(wl)
     idx = P.IndexBuffers(params)
     ksum = torch.empty(wl.B, wl.H, wl.n_blocks, wl.d, device="cuda")
     vsum = torch.empty_like(ksum)
-    out = torch.empty_like(d["q"])
+    out = torch.empty_like(dev["q"])
     lse = torch.empty(wl.B, wl.H, wl.N, device="cuda")
 
     def step():
-        P.pack3d_build_index(params, d["coords"], idx)
-        P.pack3d_block_summaries(params, idx, d["k"], d["v"], ksum, vsum)
-        P.pack3d_forward(params, idx, d["q"], d["k"], d["v"], ksum, vsum, out=out, lse=lse)
+        P.pack3d_build_index(params, dev["coords"], idx)
+        P.pack3d_block_summaries(params, idx, dev["k"], dev["v"], ksum, vsum)
+        P.pack3d_forward(params, idx, dev["q"], dev["k"], dev["v"], ksum, vsum, out=out, lse=lse)
 
     steps = 3
     for _ in range(3):
@@ -475,10 +477,11 @@ def fp32_mode_line(args):
     ms = e0.elapsed_time(e1) / steps
     work = algorithmic_work(wl)
     tf = work["flop"] / (ms * 1e-3) / 1e12
-    res = {"workload": "vol_32x32x64 in fp32 (same shape and seed layout, CUDA-core kernels)",
+    res = {"workload": f"vol_32x32x64 in {dtype}, head_dim {d} (same shape and seed layout, "
+                       "CUDA-core kernels)",
            "ms_per_step": ms, "value": wl.B * wl.N / (ms * 1e-3), "unit": UNIT, "steps": steps,
            "tflops_useful_whole_step": tf}
-    del d, inp, out, lse, ksum, vsum, idx
+    del dev, inp, out, lse, ksum, vsum, idx
     torch.cuda.empty_cache()
     return res
 
@@ -605,7 +608,8 @@ def run_ours(args):
     micro = None
     if args.micro1m and world == 1:
         micro = micro1m_line(args, pk)
-    fp32 = fp32_mode_line(args) if args.micro1m and world == 1 else None
+    fp32 = cuda_core_line(args) if args.micro1m and world == 1 else None
+    d48 = cuda_core_line(args, "bf16", 48) if args.micro1m and world == 1 else None
 
     if rank != 0:
         barrier(world)
@@ -690,6 +694,9 @@ def run_ours(args):
         fp32["fp32_fma_peak_tflops"] = fma_peak
         fp32["frac_of_fma_peak"] = fp32["tflops_useful_whole_step"] / fma_peak
         line["fp32_mode"] = fp32
+        d48["fp32_fma_peak_tflops"] = fma_peak
+        d48["frac_of_fma_peak"] = d48["tflops_useful_whole_step"] / fma_peak
+        line["bf16_head_dim_48"] = d48
     if not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(wl, inp, args.cpu_sample)
     barrier(world)
@@ -781,7 +788,8 @@ def main():
                     help="forward / backward: time that alone and print a short line "
                          "(for profiler runs)")
     ap.add_argument("--no-micro1m", dest="micro1m", action="store_false",
-                    help="skip the 1M-token workload and the fp32-mode sections")
+                    help="skip the 1M-token workload and the CUDA-core sections (fp32 mode, "
+                         "bf16 at head dim 48)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
