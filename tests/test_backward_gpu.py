@@ -22,6 +22,11 @@ CASES = [
                block=(8, 8, 8), dtype="bf16", value_scale=1.0 / np.sqrt(96), seed=43),
     I.Workload(name="d12_fp32_4x6x8", B=1, H=2, d=12, Z=4, Y=6, X=8, window=(3, 3, 3),
                block=(2, 3, 4), dtype="fp32", seed=44),
+    # unscaled N(0,1) rows: logits of standard deviation ~1, a peaked softmax and
+    # lse up to ~6, so the statistic channels of the dk/dv and summary products
+    # carry larger values (gradients stay below 2, within the absolute bound)
+    I.Workload(name="sharp_bf16_6x8x16", B=1, H=2, d=96, Z=6, Y=8, X=16, window=(5, 5, 5),
+               block=(3, 4, 8), dtype="bf16", value_scale=1.0, seed=49),
     # a wide y/x window: a halo plane (18 rows of 22) is staged in three row
     # chunks, and halo rows clipped at the volume edge have odd lengths
     I.Workload(name="wide_window_fp32_5x20x26", B=1, H=2, d=96, Z=5, Y=20, X=26,
