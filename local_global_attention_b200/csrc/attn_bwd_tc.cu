@@ -734,9 +734,11 @@ __global__ void k_bwd_sum_reduce(Geo g, const int32_t* __restrict__ err, int nsp
 
 // Rotated queries and dO in grid order ([B][H][Z][Y][X][96] bf16) and per voxel
 // (lse log2 e, delta = sum_c dO_c out_c, 0, 0), read once through the
-// coordinate volume.  One CTA per (64-voxel piece of an x row, row z * Y + y,
-// batch item), as the forward's staging of keys and values.
-constexpr int STAGE_XS = 64;
+// coordinate volume.  One CTA per (64-voxel piece of an x row and group of up
+// to 8 heads, row z * Y + y, batch item), as the forward's staging of keys and
+// values.  delta is summed per 16-channel item of a row as its dO and out
+// pieces arrive, then over the six items in item order.
+constexpr int STAGE_XS = 64, STAGE_HG = 8;
 
 // x as hi + mid + lo, each the bf16 rounding of what is left (bit patterns).
 __device__ __forceinline__ void split3_bf16(float x, uint32_t (&w)[3]) {
@@ -757,33 +759,77 @@ __global__ void __launch_bounds__(256)
                   uint4* __restrict__ schan) {
   if (ix.err[0]) return;
   __shared__ int32_t tok[STAGE_XS];
-  const int xb = blockIdx.x * STAGE_XS, zy = blockIdx.y, b = blockIdx.z;
+  // delta partials: per (voxel, head of the group) the dot products of the six items
+  __shared__ float part[STAGE_XS][STAGE_HG][6];
+  const int nxb = (g.X + STAGE_XS - 1) / STAGE_XS;
+  const int xb = (blockIdx.x % nxb) * STAGE_XS, h0 = (blockIdx.x / nxb) * STAGE_HG;
+  const int zy = blockIdx.y, b = blockIdx.z;
+  const int nh = min(STAGE_HG, g.H - h0);  // this CTA's heads h0 ..
   const int z = zy / g.Y, y = zy % g.Y;
   const int nx = min(STAGE_XS, g.X - xb);
   const int64_t vox0 = ((int64_t)b * g.Z * g.Y + zy) * g.X + xb;
   for (int i = threadIdx.x; i < nx; i += blockDim.x) tok[i] = ix.vol[vox0 + i];
   __syncthreads();
   const int H = g.H;
-  auto grid_row = [&](int hh) { return ((((int64_t)b * H + hh) * g.Z + z) * g.Y + y) * g.X + xb; };
+  // (hh: a head of the group)
+  auto grid_row = [&](int hh) {
+    return ((((int64_t)b * H + h0 + hh) * g.Z + z) * g.Y + y) * g.X + xb;
+  };
   // an empty voxel (token -1, partly occupied volumes) gets zero rows and
   // statistics (0, 0)
-  for (int it = threadIdx.x; it < H * nx * 6; it += blockDim.x) {
+  for (int it = threadIdx.x; it < nh * nx * 6; it += blockDim.x) {
     const int w = it % 6, rem = it / 6;
     const int x = rem % nx, hh = rem / nx;
     const Item96 item = item96(g, w);
     const int tk = tok[x];
     uint4 lo = make_uint4(0, 0, 0, 0), hi = lo, dlo = lo, dhi = lo;
+    float dot = 0.f;
     if (tk >= 0) {
-      const int64_t row = (((int64_t)b * g.N + tk) * H + hh) * D;
+      const int64_t row = (((int64_t)b * g.N + tk) * H + h0 + hh) * D;
       const uint4* src = reinterpret_cast<const uint4*>(q + row);
       const uint4* dsrc = reinterpret_cast<const uint4*>(dout + row);
       lo = __ldg(src + item.c1);
       hi = __ldg(src + item.c2);
       dlo = __ldg(dsrc + item.c1);
       dhi = __ldg(dsrc + item.c2);
+      // dO . O over this item's 16 channels
+      float o[16];
+      if constexpr (sizeof(TO) == 4) {
+        const float4* os = reinterpret_cast<const float4*>(out + row);
+        const float4 a0 = __ldg(os + 2 * item.c1), a1 = __ldg(os + 2 * item.c1 + 1);
+        const float4 b0 = __ldg(os + 2 * item.c2), b1 = __ldg(os + 2 * item.c2 + 1);
+        o[0] = a0.x; o[1] = a0.y; o[2] = a0.z; o[3] = a0.w;
+        o[4] = a1.x; o[5] = a1.y; o[6] = a1.z; o[7] = a1.w;
+        o[8] = b0.x; o[9] = b0.y; o[10] = b0.z; o[11] = b0.w;
+        o[12] = b1.x; o[13] = b1.y; o[14] = b1.z; o[15] = b1.w;
+      } else {
+        const uint4* os = reinterpret_cast<const uint4*>(out + row);
+        const uint4 oa = __ldg(os + item.c1), ob = __ldg(os + item.c2);
+        const uint32_t* pa = reinterpret_cast<const uint32_t*>(&oa);
+        const uint32_t* pb = reinterpret_cast<const uint32_t*>(&ob);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float2 fa = unpack_bf16x2(pa[u]), fb = unpack_bf16x2(pb[u]);
+          o[2 * u] = fa.x;
+          o[2 * u + 1] = fa.y;
+          o[8 + 2 * u] = fb.x;
+          o[8 + 2 * u + 1] = fb.y;
+        }
+      }
+      const uint32_t* dl = reinterpret_cast<const uint32_t*>(&dlo);
+      const uint32_t* dh = reinterpret_cast<const uint32_t*>(&dhi);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float2 fa = unpack_bf16x2(dl[u]), fb = unpack_bf16x2(dh[u]);
+        dot += fa.x * o[2 * u];
+        dot += fa.y * o[2 * u + 1];
+        dot += fb.x * o[8 + 2 * u];
+        dot += fb.y * o[8 + 2 * u + 1];
+      }
       const int c = item.a == 0 ? z : (item.a == 1 ? y : xb + x);
       rot_chunk(lo, hi, rope_row96(ix.rope, g, item.a, c, tk), item.j0);
     }
+    part[x][hh][w] = dot;
     uint4* qd = reinterpret_cast<uint4*>(qg + (grid_row(hh) + x) * D);
     uint4* dd = reinterpret_cast<uint4*>(dog + (grid_row(hh) + x) * D);
     qd[item.c1] = lo;
@@ -791,7 +837,8 @@ __global__ void __launch_bounds__(256)
     dd[item.c1] = dlo;
     dd[item.c2] = dhi;
   }
-  for (int it = threadIdx.x; it < H * nx; it += blockDim.x) {
+  __syncthreads();
+  for (int it = threadIdx.x; it < nh * nx; it += blockDim.x) {
     const int x = it % nx, hh = it / nx;
     if (tok[x] < 0) {
       stat[grid_row(hh) + x] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -799,37 +846,11 @@ __global__ void __launch_bounds__(256)
       schan[2 * (grid_row(hh) + x) + 1] = make_uint4(0u, 0u, 0u, 0u);
       continue;
     }
-    const int64_t row = (((int64_t)b * g.N + tok[x]) * H + hh) * D;
-    const uint4* dsrc = reinterpret_cast<const uint4*>(dout + row);
+    // the items' partial dot products added in item order
     float acc = 0.f;
 #pragma unroll
-    for (int c = 0; c < 12; ++c) {
-      const uint4 dw = __ldg(dsrc + c);
-      const uint32_t* dp = reinterpret_cast<const uint32_t*>(&dw);
-      float o[8];
-      if constexpr (sizeof(TO) == 4) {
-        const float4* os = reinterpret_cast<const float4*>(out + row) + 2 * c;
-        const float4 a = __ldg(os), bq = __ldg(os + 1);
-        o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
-        o[4] = bq.x; o[5] = bq.y; o[6] = bq.z; o[7] = bq.w;
-      } else {
-        const uint4 ow = __ldg(reinterpret_cast<const uint4*>(out + row) + c);
-        const uint32_t* op = reinterpret_cast<const uint32_t*>(&ow);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float2 f = unpack_bf16x2(op[u]);
-          o[2 * u] = f.x;
-          o[2 * u + 1] = f.y;
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float2 dd = unpack_bf16x2(dp[u]);
-        acc += dd.x * o[2 * u];
-        acc += dd.y * o[2 * u + 1];
-      }
-    }
-    const float L = lse[((int64_t)b * H + hh) * g.N + tok[x]] * LOG2E;
+    for (int w = 0; w < 6; ++w) acc += part[x][hh][w];
+    const float L = lse[((int64_t)b * H + h0 + hh) * g.N + tok[x]] * LOG2E;
     stat[grid_row(hh) + x] = make_float4(L, acc, 0.f, 0.f);
     // the column roles' statistic channels: -L / (tau log2 e) and -delta, each
     // as three bf16 parts whose sum is the fp32 value (to fp32 precision)
@@ -979,7 +1000,8 @@ int backward_tc_summary_grads(const Geo& g, const pack3d_index* idx, const void*
     if ((rc = cuda_status(cudaGetLastError()))) return rc;
   }
   {
-    dim3 grid((g.X + STAGE_XS - 1) / STAGE_XS, g.Z * g.Y, g.B);
+    dim3 grid(((g.X + STAGE_XS - 1) / STAGE_XS) * ((g.H + STAGE_HG - 1) / STAGE_HG), g.Z * g.Y,
+              g.B);
     if (g.out_fp32)
       k_bwd_stage_q<float><<<grid, 256, 0, s>>>(
           g, *idx, (const __nv_bfloat16*)q, (const __nv_bfloat16*)dout, (const float*)out, lse,

@@ -27,6 +27,9 @@ CASES = [
     # carry larger values (gradients stay below 2, within the absolute bound)
     I.Workload(name="sharp_bf16_6x8x16", B=1, H=2, d=96, Z=6, Y=8, X=16, window=(5, 5, 5),
                block=(3, 4, 8), dtype="bf16", value_scale=1.0, seed=49),
+    # ten heads: the staging of q and dO takes them in groups of eight
+    I.Workload(name="heads10_bf16_4x8x24", B=1, H=10, d=96, Z=4, Y=8, X=24, window=(3, 3, 5),
+               block=(2, 4, 8), dtype="bf16", value_scale=1.0 / np.sqrt(96), seed=50),
     # a wide y/x window: a halo plane (18 rows of 22) is staged in three row
     # chunks, and halo rows clipped at the volume edge have odd lengths
     I.Workload(name="wide_window_fp32_5x20x26", B=1, H=2, d=96, Z=5, Y=20, X=26,

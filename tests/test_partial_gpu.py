@@ -82,7 +82,7 @@ def test_partial_forward(oracle_lib, wl, window_only):
         np.testing.assert_allclose(res["vsum"].double().numpy(), vs, rtol=0, atol=2e-5)
 
 
-@pytest.mark.parametrize("wl", [PARTIAL[0], PARTIAL[1], PARTIAL[3]], ids=lambda w: w.name)
+@pytest.mark.parametrize("wl", PARTIAL, ids=lambda w: w.name)
 def test_partial_backward(oracle_lib, wl):
     wl = wl.replace(value_scale=1.0 / np.sqrt(96))
     inp = I.make_inputs(wl, "random", with_dout=True)
